@@ -1,0 +1,331 @@
+// api.cu -- the extern "C" entry points declared in sfnn.h.
+//
+// Host-side work only: argument checks, the hotness order, allocation of the
+// handle's buffers, and the sequence of kernel launches of each call.  Every
+// step of the computation runs in the kernels of layout.cu, predict.cu and
+// ffn.cu.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "common.cuh"
+
+using namespace sfnn;
+
+namespace {
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || (cudaSetDevice(dev) == cudaSuccess);
+  }
+  ~DeviceGuard() {
+    if (ok && prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+void free_handle(sfnn_ctx *h) {
+  if (!h) return;
+  void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err};
+  for (void *p : bufs)
+    if (p) cudaFree(p);
+  delete h;
+}
+
+sfnn_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SFNN_OK;
+  if (e == cudaErrorMemoryAllocation) return SFNN_ERR_OOM;
+  return SFNN_ERR_CUDA;
+}
+
+#define SFNN_TRY(expr)                               \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return from_cuda(e_);     \
+  } while (0)
+
+sfnn_status check_desc(const sfnn_layer_desc *d) {
+  if (!d) return SFNN_ERR_INVALID_ARG;
+  if (d->wdtype != SFNN_F32 && d->wdtype != SFNN_F16) return SFNN_ERR_INVALID_ARG;
+  if (d->act != SFNN_RELU && d->act != SFNN_REGLU) return SFNN_ERR_INVALID_ARG;
+  if (d->d < 1 || d->n < 1 || d->r < 1) return SFNN_ERR_INVALID_ARG;
+  if (d->max_batch < 1) return SFNN_ERR_INVALID_ARG;
+  if (!d->w_up || !d->b || !d->w_down || !d->pa || !d->pb || !d->pc) return SFNN_ERR_INVALID_ARG;
+  if (d->act == SFNN_REGLU && !d->w_gate) return SFNN_ERR_INVALID_ARG;
+  const int vec = d->wdtype == SFNN_F16 ? 8 : 4;
+  if (d->d % vec || d->r % vec) return SFNN_ERR_INVALID_ARG;
+  if (d->max_batch > kMaxBatch) return SFNN_ERR_UNSUPPORTED;
+  if ((int64_t)d->r * d->max_batch > 32768) return SFNN_ERR_UNSUPPORTED;
+  if (d->n > (1 << 24) || d->d > (1 << 16)) return SFNN_ERR_UNSUPPORTED;
+  return SFNN_OK;
+}
+
+bool same_device(const sfnn_ctx *h) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == h->device;
+}
+
+void record_if(cudaEvent_t ev, cudaStream_t s) {
+  if (ev) cudaEventRecord(ev, s);
+}
+
+// The shared body of forward / forward_batch / one stack layer.
+sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int32_t *idx, const int32_t *count,
+                      int32_t *idx_out, int32_t *cnt_out, const float *resid, float *Y, void *xnext,
+                      cudaStream_t s) {
+  cudaEvent_t before = h->prof_before, after = h->prof_after;
+  h->prof_before = h->prof_after = nullptr;
+  record_if(before, s);
+  if (predict) {
+    SFNN_TRY(launch_hidden(h, X, b, s));
+    SFNN_TRY(launch_logits(h, b, s));
+  } else {
+    SFNN_TRY(launch_mask_from_idx(h, idx, count, s));
+  }
+  SFNN_TRY(launch_compact(h, b, idx_out, cnt_out, s));
+  SFNN_TRY(launch_up(h, X, b, s));
+  int splits = 1;
+  SFNN_TRY(launch_down(h, b, &splits, s));
+  SFNN_TRY(launch_reduce(h, b, splits, resid, Y, xnext, s));
+  record_if(after, s);
+  h->launches += predict ? 6 : 5;
+  return SFNN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sfnn_status_str(sfnn_status s) {
+  switch (s) {
+    case SFNN_OK: return "ok";
+    case SFNN_ERR_INVALID_ARG: return "invalid argument";
+    case SFNN_ERR_CUDA: return "CUDA error";
+    case SFNN_ERR_OOM: return "out of device memory";
+    case SFNN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SFNN_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+sfnn_status sfnn_hotness_order(const float *hotness, int32_t n, int32_t *perm) {
+  if (!hotness || !perm || n < 1) return SFNN_ERR_INVALID_ARG;
+  std::vector<int32_t> p(n);
+  std::iota(p.begin(), p.end(), 0);
+  auto key = [&](int32_t i) { return std::isnan(hotness[i]) ? -INFINITY : hotness[i]; };
+  std::stable_sort(p.begin(), p.end(), [&](int32_t a, int32_t b) { return key(a) > key(b); });
+  std::memcpy(perm, p.data(), sizeof(int32_t) * n);
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_handle *out) {
+  if (!out) return SFNN_ERR_INVALID_ARG;
+  *out = nullptr;
+  sfnn_status st = check_desc(desc);
+  if (st != SFNN_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  sfnn_ctx *h = new (std::nothrow) sfnn_ctx();
+  if (!h) return SFNN_ERR_OOM;
+  std::memset(static_cast<void *>(h), 0, sizeof(*h));
+  Layout &L = h->L;
+  L.d = desc->d;
+  L.n = desc->n;
+  L.r = desc->r;
+  L.act = desc->act;
+  L.dt = desc->wdtype;
+  L.nproj = desc->act == SFNN_REGLU ? 3 : 2;
+  L.esize = desc->wdtype == SFNN_F16 ? 2 : 4;
+  L.vec = 16 / L.esize;
+  L.nwords = (L.n + 31) / 32;
+  h->max_batch = desc->max_batch;
+  h->batch_path = SFNN_BATCH_AUTO;
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    delete h;
+    return SFNN_ERR_CUDA;
+  }
+
+  // storage order
+  std::vector<int32_t> perm(L.n), iperm(L.n);
+  if (desc->hotness) {
+    sfnn_hotness_order(desc->hotness, L.n, perm.data());
+  } else {
+    std::iota(perm.begin(), perm.end(), 0);
+  }
+  for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
+  for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
+  if (desc->hotness) {
+    for (int b = 1; b <= kMaxBatch; ++b) {
+      double u = 0.0;
+      for (int i = 0; i < L.n; ++i) {
+        double p = std::isnan(desc->hotness[i]) ? 0.0 : std::min(1.0, std::max(0.0, (double)desc->hotness[i]));
+        u += 1.0 - std::pow(1.0 - p, b);
+      }
+      h->expected_union[b] = u / L.n;
+    }
+  }
+
+  const size_t e = L.esize, n = L.n, d = L.d, r = L.r, mb = h->max_batch;
+  struct Req {
+    void **ptr;
+    size_t bytes;
+    bool weight;
+  } reqs[] = {
+      {&h->rows, n * L.nproj * d * e, true},
+      {&h->At, r * d * e, true},
+      {&h->Bt, n * r * e, true},
+      {&h->cvec, n * e, true},
+      {&h->bias, n * e, true},
+      {(void **)&h->perm, n * 4, true},
+      {(void **)&h->iperm, n * 4, true},
+      {(void **)&h->h, mb * r * 4, false},
+      {(void **)&h->mask, mb * L.nwords * 4, false},
+      {(void **)&h->ulist, n * 4, false},
+      {(void **)&h->utok, n * 4, false},
+      {(void **)&h->ucount, 4, false},
+      {(void **)&h->acoef, n * mb * 4, false},
+      {(void **)&h->part, (size_t)kMaxSplits * mb * d * 4, false},
+      {&h->xin, mb * d * e, false},
+      {(void **)&h->err, 4, false},
+  };
+  for (auto &q : reqs) {
+    if (cudaMalloc(q.ptr, q.bytes) != cudaSuccess) {
+      cudaGetLastError();
+      free_handle(h);
+      return SFNN_ERR_OOM;
+    }
+    (q.weight ? h->weight_bytes : h->scratch_bytes) += (int64_t)q.bytes;
+  }
+  cudaError_t ce = cudaMemcpy(h->perm, perm.data(), n * 4, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess) ce = cudaMemcpy(h->iperm, iperm.data(), n * 4, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->err, 0, 4, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->ucount, 0, 4, s);
+  if (ce == cudaSuccess) ce = configure_predict();
+  if (ce == cudaSuccess) ce = configure_ffn();
+  if (ce == cudaSuccess) ce = launch_layout(h, desc, s);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+  if (ce != cudaSuccess) {
+    free_handle(h);
+    return from_cuda(ce);
+  }
+  *out = h;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_destroy(sfnn_handle h) {
+  if (!h) return SFNN_OK;
+  DeviceGuard g(h->device);
+  cudaDeviceSynchronize();
+  free_handle(h);
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_predict(sfnn_handle h, const void *x, int32_t *idx, int32_t *count, sfnn_stream_t stream) {
+  if (!h || !x || !idx || !count) return SFNN_ERR_INVALID_ARG;
+  if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SFNN_TRY(launch_hidden(h, x, 1, s));
+  SFNN_TRY(launch_logits(h, 1, s));
+  SFNN_TRY(launch_compact(h, 1, idx, count, s));
+  h->launches += 3;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *idx, const int32_t *count, float *y,
+                         sfnn_stream_t stream) {
+  if (!h || !x || !y || (idx && !count)) return SFNN_ERR_INVALID_ARG;
+  if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
+  return run_layer(h, x, 1, idx == nullptr, idx, count, nullptr, nullptr, nullptr, y, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b, float *Y, int32_t *idx, int32_t *counts,
+                               sfnn_stream_t stream) {
+  if (!h || !X || !Y || b < 1 || b > h->max_batch) return SFNN_ERR_INVALID_ARG;
+  if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
+  return run_layer(h, X, b, true, nullptr, nullptr, idx, counts, nullptr, Y, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_layers, const float *X0, int32_t b, float *XL,
+                               int32_t *idx, int32_t *counts, sfnn_stream_t stream) {
+  if (!layers || num_layers < 1 || !X0 || !XL || b < 1) return SFNN_ERR_INVALID_ARG;
+  const sfnn_ctx *l0 = layers[0];
+  if (!l0) return SFNN_ERR_INVALID_ARG;
+  for (int l = 0; l < num_layers; ++l) {
+    const sfnn_ctx *hl = layers[l];
+    if (!hl || hl->L.d != l0->L.d || hl->L.dt != l0->L.dt || hl->device != l0->device || b > hl->max_batch)
+      return SFNN_ERR_INVALID_ARG;
+    if (idx && hl->L.n != l0->L.n) return SFNN_ERR_INVALID_ARG;
+  }
+  if (!same_device(l0)) return SFNN_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t bd = (int64_t)b * l0->L.d;
+  SFNN_TRY(launch_round(X0, layers[0]->xin, l0->L.dt, bd, s));
+  layers[0]->launches += 1;
+  for (int l = 0; l < num_layers; ++l) {
+    sfnn_ctx *hl = layers[l];
+    const int n = hl->L.n;
+    int32_t *idx_l = idx ? idx + (size_t)l * b * n : nullptr;
+    int32_t *cnt_l = counts ? counts + (size_t)l * b : nullptr;
+    void *xnext = l + 1 < num_layers ? layers[l + 1]->xin : nullptr;
+    sfnn_status st =
+        run_layer(hl, hl->xin, b, true, nullptr, nullptr, idx_l, cnt_l, l == 0 ? X0 : XL, XL, xnext, s);
+    if (st != SFNN_OK) return st;
+  }
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (path != SFNN_BATCH_AUTO && path != SFNN_BATCH_CUDA_CORE && path != SFNN_BATCH_TENSOR_CORE)
+    return SFNN_ERR_INVALID_ARG;
+  if (path == SFNN_BATCH_TENSOR_CORE) return SFNN_ERR_UNSUPPORTED;
+  h->batch_path = path;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before, sfnn_event_t after) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  h->prof_before = reinterpret_cast<cudaEvent_t>(before);
+  h->prof_after = reinterpret_cast<cudaEvent_t>(after);
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_query(sfnn_handle h, sfnn_info *info) {
+  if (!h || !info) return SFNN_ERR_INVALID_ARG;
+  const Layout &L = h->L;
+  info->d = L.d;
+  info->n = L.n;
+  info->r = L.r;
+  info->max_batch = h->max_batch;
+  info->act = L.act;
+  info->wdtype = L.dt;
+  info->num_sms = h->num_sms;
+  info->batch_path = h->batch_path;
+  info->weight_bytes = h->weight_bytes;
+  info->scratch_bytes = h->scratch_bytes;
+  info->predictor_bytes = ((int64_t)L.d * L.r + (int64_t)L.r * L.n + L.n) * L.esize;
+  info->row_bytes_per_neuron = ((int64_t)L.nproj * L.d + 1) * L.esize;
+  info->launches = h->launches;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_get_error(sfnn_handle h) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  DeviceGuard g(h->device);
+  int32_t v = 0;
+  if (cudaMemcpy(&v, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFNN_ERR_CUDA;
+  if (v != 0 && cudaMemset(h->err, 0, 4) != cudaSuccess) return SFNN_ERR_CUDA;
+  return static_cast<sfnn_status>(v);
+}
+
+}  // extern "C"

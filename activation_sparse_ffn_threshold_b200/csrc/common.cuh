@@ -1,0 +1,141 @@
+// common.cuh -- internal types shared by the sfnn CUDA sources (not part of the C ABI).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sfnn.h"
+
+namespace sfnn {
+
+constexpr int kMaxBatch = 32;
+constexpr int kMaxSplits = 64;  // K-splits of the down projection (partials per token)
+
+// Device-side error word values (a subset of sfnn_status).
+constexpr int kErrInvalidIdx = SFNN_ERR_INVALID_ARG;
+constexpr int kErrTimeout = SFNN_ERR_TIMEOUT;
+
+struct Layout {
+  int d, n, r, nproj, act, dt, esize, vec, nwords;
+};
+
+}  // namespace sfnn
+
+struct sfnn_ctx {
+  sfnn::Layout L;
+  int max_batch;
+  int device;
+  int num_sms;
+  int batch_path;
+  double expected_union[sfnn::kMaxBatch + 1];  // E|U|/n by batch size, from the hotness profile
+  // re-laid-out weights (internal neuron order p = 0..n-1, hottest first)
+  void *rows;      // [n][nproj][d]: ReLU (up, down); ReGLU (gate, up, down)
+  void *At;        // [r][d]
+  void *Bt;        // [n][r]
+  void *cvec;      // [n]
+  void *bias;      // [n]
+  int32_t *perm;   // [n] internal -> original
+  int32_t *iperm;  // [n] original -> internal
+  // scratch
+  float *h;          // [max_batch][r]
+  uint32_t *mask;    // [max_batch][nwords]
+  int32_t *ulist;    // [n] union list (internal positions, ascending)
+  uint32_t *utok;    // [n] tokens active on each union row (bit t)
+  int32_t *ucount;   // [1]
+  float *acoef;      // [n][max_batch] activation of each union row for each token
+  float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
+  void *xin;         // [max_batch][d] wdtype: layer input inside a stack
+  int32_t *err;      // [1] latched device-side error
+  int64_t weight_bytes, scratch_bytes;
+  int64_t launches;  // kernels this handle has launched (or captured into a graph)
+  // one-shot profiling events around the dominant kernel
+  cudaEvent_t prof_before, prof_after;
+};
+
+namespace sfnn {
+
+// ---------------------------------------------------------------- element helpers
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+  static constexpr int kVec = 4;  // elements per 16-byte vector
+};
+template <>
+struct Elem<__half> {
+  static constexpr int kVec = 8;
+};
+
+// Read-only 16-byte load from global memory, not kept in L1 (weights stream once).
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Read-only 16-byte load that may stay in L1 (activations reused by a CTA).
+__device__ __forceinline__ uint4 ld_keep(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+
+template <typename T>
+__device__ __forceinline__ void unpack(const uint4 &v, float *f);
+
+template <>
+__device__ __forceinline__ void unpack<float>(const uint4 &v, float *f) {
+  f[0] = __uint_as_float(v.x);
+  f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z);
+  f[3] = __uint_as_float(v.w);
+}
+
+template <>
+__device__ __forceinline__ void unpack<__half>(const uint4 &v, float *f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h2 = *reinterpret_cast<const __half2 *>(&w[i]);
+    float2 f2 = __half22float2(h2);
+    f[2 * i] = f2.x;
+    f[2 * i + 1] = f2.y;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __half from_f<__half>(float v) { return __float2half_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void latch_error(int32_t *err, int code) { atomicCAS(err, 0, code); }
+
+// ---------------------------------------------------------------- launchers (defined in the .cu files)
+cudaError_t configure_predict();  // one-time kernel attributes (shared-memory limits)
+cudaError_t configure_ffn();
+cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s);
+cudaError_t launch_hidden(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
+cudaError_t launch_logits(const sfnn_ctx *h, int b, cudaStream_t s);
+cudaError_t launch_mask_from_idx(const sfnn_ctx *h, const int32_t *idx, const int32_t *count, cudaStream_t s);
+cudaError_t launch_compact(const sfnn_ctx *h, int b, int32_t *idx_out, int32_t *cnt_out, cudaStream_t s);
+cudaError_t launch_up(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
+cudaError_t launch_down(const sfnn_ctx *h, int b, int *splits, cudaStream_t s);
+cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *resid, float *Y, void *xnext,
+                          cudaStream_t s);
+cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s);
+
+}  // namespace sfnn

@@ -1,0 +1,289 @@
+// predict.cu -- the low-rank neuron predictor and the stream compaction of its decisions.
+//
+// The predictor marks neuron i active when sigmoid(relu(x.A).B + c)_i > 0.5,
+// evaluated as z_i > 0 (sigmoid is increasing, sigmoid(0) = 1/2).  It stands
+// for the small per-layer MLP predictors that DejaVu and PowerInfer train to
+// decide which FFN neurons to compute (53ai.com "sparsity for LLM inference"
+// page, sections 如何推理加速 and 自适应稀疏预测器).  h is kept in fp32; z is
+// accumulated in fp32 from fp16 (or fp32) weights.
+//
+// Kernels:
+//   k_hidden   H[t][j] = relu(At[j] . X[t])         one warp per row of At
+//   k_logits   bit i of token t = (Bt[i] . H[t] + c_i > 0)   one CTA per 32 neurons
+//   k_mask_from_idx   a caller-given index list as a bit mask
+//   k_compact  masks -> ascending index lists (per token, in caller numbering)
+//              and the union of the tokens' sets with, per union row, the bit
+//              set of tokens active on it (warp ballot + block prefix sum).
+#include "common.cuh"
+
+namespace sfnn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+template <typename T, int TB>
+__global__ void __launch_bounds__(kThreads) k_hidden(const T *__restrict__ At, const T *__restrict__ X,
+                                                     float *__restrict__ H, int r, int d, int b) {
+  constexpr int V = Elem<T>::kVec;
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int nch = d / V;
+  for (int j = gwarp; j < r; j += nwarps) {
+    const T *row = At + (size_t)j * d;
+    for (int t0 = 0; t0 < b; t0 += TB) {
+      float acc[TB];
+#pragma unroll
+      for (int t = 0; t < TB; ++t) acc[t] = 0.f;
+      for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+        uint4 w[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (c0 + 32 * u < nch) w[u] = ld_stream(row + (size_t)(c0 + 32 * u) * V);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int c = c0 + 32 * u;
+          if (c < nch) {
+            float wf[V];
+            unpack<T>(w[u], wf);
+#pragma unroll
+            for (int t = 0; t < TB; ++t) {
+              if (t0 + t < b) {
+                float xf[V];
+                unpack<T>(ld_keep(X + (size_t)(t0 + t) * d + (size_t)c * V), xf);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[t] = fmaf(wf[v], xf[v], acc[t]);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < TB; ++t) {
+        if (t0 + t < b) {
+          const float s = warp_sum(acc[t]);
+          if (lane == 0) H[(size_t)(t0 + t) * r + j] = s > 0.f ? s : 0.f;  // NaN -> 0
+        }
+      }
+    }
+  }
+}
+
+// One CTA per mask word (32 neurons); warp w takes neurons 4w..4w+3 of the word.
+template <typename T, int TB>
+__global__ void __launch_bounds__(kThreads) k_logits(const T *__restrict__ Bt, const T *__restrict__ cvec,
+                                                     const float *__restrict__ H, uint32_t *__restrict__ mask,
+                                                     int n, int r, int b, int nwords) {
+  constexpr int V = Elem<T>::kVec;
+  extern __shared__ float hs[];  // [b][r]
+  __shared__ uint32_t bits_s[TB];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < b * r; i += blockDim.x) hs[i] = H[i];
+  const int nch = r / V;
+  for (int word = blockIdx.x; word < nwords; word += gridDim.x) {
+    for (int t0 = 0; t0 < b; t0 += TB) {
+      if (threadIdx.x < TB) bits_s[threadIdx.x] = 0u;
+      __syncthreads();
+      for (int q = 0; q < 4; ++q) {
+        const int i = warp * 4 + q;
+        const int p = word * 32 + i;
+        if (p >= n) break;  // warp-uniform
+        const T *row = Bt + (size_t)p * r;
+        float acc[TB];
+#pragma unroll
+        for (int t = 0; t < TB; ++t) acc[t] = 0.f;
+#pragma unroll 4
+        for (int c = lane; c < nch; c += 32) {
+          float wf[V];
+          unpack<T>(ld_stream(row + (size_t)c * V), wf);
+#pragma unroll
+          for (int t = 0; t < TB; ++t) {
+            if (t0 + t < b) {
+              const float *hp = hs + (size_t)(t0 + t) * r + (size_t)c * V;
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[t] = fmaf(wf[v], hp[v], acc[t]);
+            }
+          }
+        }
+        const float cz = to_f<T>(cvec[p]);
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+          if (t0 + t < b) {
+            const float z = warp_sum(acc[t]) + cz;
+            if (lane == 0 && z > 0.f) atomicOr(&bits_s[t], 1u << i);  // NaN -> inactive
+          }
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x < TB && t0 + threadIdx.x < b)
+        mask[(size_t)(t0 + threadIdx.x) * nwords + word] = bits_s[threadIdx.x];
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024) k_mask_from_idx(const int32_t *__restrict__ idx,
+                                                        const int32_t *__restrict__ count,
+                                                        const int32_t *__restrict__ iperm,
+                                                        uint32_t *__restrict__ mask, int n, int nwords,
+                                                        int32_t *err) {
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) mask[w] = 0u;
+  __syncthreads();
+  int k = *count;
+  k = k < 0 ? 0 : (k > n ? n : k);
+  for (int e = threadIdx.x; e < k; e += blockDim.x) {
+    const int v = idx[e];
+    if (v < 0 || v >= n) {
+      latch_error(err, kErrInvalidIdx);
+      continue;
+    }
+    const int p = iperm[v];
+    atomicOr(&mask[p >> 5], 1u << (p & 31));
+  }
+}
+
+// Exclusive prefix sum over the block; returns this thread's offset, *total the block sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
+  __shared__ int warp_tot[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int wt = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wt, o);
+      if (lane >= o) wt += y;
+    }
+    if (lane < nw) warp_tot[lane] = wt;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = warp == 0 ? 0 : warp_tot[warp - 1];
+  *total = warp_tot[nw - 1];
+  __syncthreads();
+  return before + incl - v;
+}
+
+// Blocks 0..b-1 (only when token outputs are wanted): token lists.  Last block: the union.
+__global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ mask, int nwords, int n, int b,
+                                                  const int32_t *__restrict__ perm, int32_t *__restrict__ ulist,
+                                                  uint32_t *__restrict__ utok, int32_t *__restrict__ ucount,
+                                                  int32_t *__restrict__ idx_out, int32_t *__restrict__ cnt_out) {
+  const bool is_union = blockIdx.x == gridDim.x - 1;
+  const int t = blockIdx.x;
+  const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * wpt;
+  auto word = [&](int w) -> uint32_t {
+    if (!is_union) return mask[(size_t)t * nwords + w];
+    uint32_t m = 0u;
+    for (int tt = 0; tt < b; ++tt) m |= mask[(size_t)tt * nwords + w];
+    return m;
+  };
+  int cnt = 0;
+  for (int k = 0; k < wpt; ++k) {
+    const int w = w0 + k;
+    if (w < nwords) cnt += __popc(word(w));
+  }
+  int total;
+  int pos = block_exclusive_scan(cnt, &total);
+  for (int k = 0; k < wpt; ++k) {
+    const int w = w0 + k;
+    if (w >= nwords) break;
+    uint32_t m = word(w);
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1u;
+      const int p = w * 32 + i;
+      if (is_union) {
+        uint32_t tb = 0u;
+        for (int tt = 0; tt < b; ++tt) tb |= ((mask[(size_t)tt * nwords + w] >> i) & 1u) << tt;
+        ulist[pos] = p;
+        utok[pos] = tb;
+      } else if (idx_out) {
+        idx_out[(size_t)t * n + pos] = perm[p];
+      }
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (is_union)
+      *ucount = total;
+    else if (cnt_out)
+      cnt_out[t] = total;
+  }
+}
+
+template <typename T>
+cudaError_t hidden_impl(const sfnn_ctx *h, const void *X, int b, cudaStream_t s) {
+  const Layout &L = h->L;
+  const int grid = (L.r + kWarps - 1) / kWarps;
+  const T *At = static_cast<const T *>(h->At);
+  const T *Xp = static_cast<const T *>(X);
+  if (b == 1)
+    k_hidden<T, 1><<<grid, kThreads, 0, s>>>(At, Xp, h->h, L.r, L.d, b);
+  else
+    k_hidden<T, 8><<<grid, kThreads, 0, s>>>(At, Xp, h->h, L.r, L.d, b);
+  return cudaGetLastError();
+}
+
+constexpr int kLogitsSmemMax = 32768 * sizeof(float);  // r * max_batch <= 32768 (checked at create)
+
+template <typename T, int TB>
+cudaError_t logits_tb(const sfnn_ctx *h, int b, cudaStream_t s) {
+  const Layout &L = h->L;
+  const size_t smem = (size_t)b * L.r * sizeof(float);
+  auto kern = k_logits<T, TB>;
+  kern<<<L.nwords, kThreads, smem, s>>>(static_cast<const T *>(h->Bt), static_cast<const T *>(h->cvec), h->h,
+                                        h->mask, L.n, L.r, b, L.nwords);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t logits_impl(const sfnn_ctx *h, int b, cudaStream_t s) {
+  if (b == 1) return logits_tb<T, 1>(h, b, s);
+  if (b <= 8) return logits_tb<T, 8>(h, b, s);
+  return logits_tb<T, 32>(h, b, s);
+}
+
+}  // namespace
+
+cudaError_t configure_predict() {
+  const void *ks[] = {(const void *)k_logits<float, 1>, (const void *)k_logits<float, 8>,
+                      (const void *)k_logits<float, 32>, (const void *)k_logits<__half, 1>,
+                      (const void *)k_logits<__half, 8>, (const void *)k_logits<__half, 32>};
+  for (const void *k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kLogitsSmemMax);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_hidden(const sfnn_ctx *h, const void *X, int b, cudaStream_t s) {
+  return h->L.dt == SFNN_F16 ? hidden_impl<__half>(h, X, b, s) : hidden_impl<float>(h, X, b, s);
+}
+
+cudaError_t launch_logits(const sfnn_ctx *h, int b, cudaStream_t s) {
+  return h->L.dt == SFNN_F16 ? logits_impl<__half>(h, b, s) : logits_impl<float>(h, b, s);
+}
+
+cudaError_t launch_mask_from_idx(const sfnn_ctx *h, const int32_t *idx, const int32_t *count, cudaStream_t s) {
+  k_mask_from_idx<<<1, 1024, 0, s>>>(idx, count, h->iperm, h->mask, h->L.n, h->L.nwords, h->err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const sfnn_ctx *h, int b, int32_t *idx_out, int32_t *cnt_out, cudaStream_t s) {
+  const int grid = (idx_out || cnt_out) ? b + 1 : 1;
+  k_compact<<<grid, 1024, 0, s>>>(h->mask, h->L.nwords, h->L.n, b, h->perm, h->ulist, h->utok, h->ucount, idx_out,
+                                  cnt_out);
+  return cudaGetLastError();
+}
+
+}  // namespace sfnn

@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark: activation-sparse FFN decode, tokens/s per layer on B200.
+
+One step is one pass of the workload's decode sequence (512 tokens of the
+OPT-6.7B-shaped ReLU layer, d=4096 n=16384 r=1024, fp16) through the hot path:
+predictor, threshold and compaction, gathered up projection, gathered down
+projection and the final sum, one token at a time (batch 1).  The 512 tokens
+are captured once into a CUDA graph; a step is one replay.  Consecutive tokens
+use different replicas of the layer's weights so that no token finds the
+previous visit's lines in L2 (the bytes touched between two visits of one
+replica exceed twice the L2 size), as in a model where the other layers stream
+through between two visits of a layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sfnn|reference]
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on the
+host cores instead, on the same workload and metric.  With N > 1 (torchrun)
+each rank runs an independent replica on its own GPU (no data exchange); the
+time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workload as W  # noqa: E402
+
+WORKLOAD = "opt6.7b_relu"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sfnn_forward_opt6.7b_relu.md")
+CSRC = os.path.join(ROOT, "activation_sparse_ffn_threshold_b200", "csrc")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sfnn", "reference"], default="sfnn")
+    ap.add_argument("--workload", default=WORKLOAD, choices=list(W.CONFIGS))
+    ap.add_argument("--replicas", type=int, default=0, help="weight replicas (0: from the L2 size)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed plumbing
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local_rank)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+        if gpus != self.world and self.world > 1:
+            log(f"note: --gpus {gpus} but WORLD_SIZE {self.world}; using WORLD_SIZE")
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        return self._reduce(v, "max")
+
+    def sum(self, v: float) -> float:
+        return self._reduce(v, "sum")
+
+    def _reduce(self, v, op):
+        if self.pg is None:
+            return v
+        import torch
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX if op == "max" else self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------- clocks
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception as e:  # pragma: no cover
+            log(f"clock sampling unavailable: {e}")
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        smax = max(r["smax"] for r in rows)
+        load = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in load:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None, None
+    sha = traffic = None
+    for line in text.splitlines():
+        if line.startswith("source_sha256_16:"):
+            sha = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_token:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    if sha != source_digest():
+        return None, "stale"
+    return traffic, "ncu"
+
+
+def expected_tokens_active(cfg):
+    return cfg.mean_p * cfg.n
+
+
+def cpu_baseline(cfg, lay, X, seconds: float):
+    """The oracle as it stands, on this host's cores, over a bounded sample of tokens."""
+    import oracle
+    nthreads = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.forward(lay, X[0], nthreads)
+    t_one = max(1e-4, time.perf_counter() - t0)
+    count = int(max(1, min(X.shape[0] - 1, seconds / t_one)))
+    t0 = time.perf_counter()
+    active = 0
+    for t in range(1, 1 + count):
+        active += int(oracle.forward(lay, X[t], nthreads).mask.sum())
+    dt = time.perf_counter() - t0
+    tok_s = count / dt
+    gbs = W.touched_bytes(cfg, active / count) * tok_s / 1e9
+    return {"value": tok_s, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{count} tokens of {cfg.name} (predictor + sparse FFN, batch 1), fp64 C oracle",
+            "effective_gbs": gbs}
+
+
+# ---------------------------------------------------------------- reference arm (the CPU oracle)
+def run_reference(args, dist):
+    if dist.rank != 0:
+        return 0
+    import oracle
+    cfg = W.CONFIGS[args.workload]
+    lay = W.make_layer(cfg, seed=args.seed)
+    X = W.make_tokens(cfg, 64, seed=args.seed)
+    nthreads = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.forward(lay, X[0], nthreads)
+    t_one = max(1e-4, time.perf_counter() - t0)
+    budget = 150.0  # seconds for warm-up + timed steps together
+    per_step = max(1, min(cfg.tokens, int(budget / max(1, args.steps + args.warmup) / t_one)))
+    k = 0
+    for _ in range(args.warmup):
+        for _ in range(per_step):
+            oracle.forward(lay, X[k % X.shape[0]], nthreads)
+            k += 1
+    t0 = time.perf_counter()
+    active = 0
+    for _ in range(args.steps):
+        for _ in range(per_step):
+            active += int(oracle.forward(lay, X[k % X.shape[0]], nthreads).mask.sum())
+            k += 1
+    dt = time.perf_counter() - t0
+    tokens = args.steps * per_step
+    tok_s = tokens / dt
+    line = {
+        "impl": "reference", "metric": "sparse-FFN decode tokens/s per layer", "value": tok_s,
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": 1, "tokens_per_step": per_step},
+        "effective_gbs": W.touched_bytes(cfg, active / tokens) * tok_s / 1e9,
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{per_step} token(s) of {cfg.name} per step, fp64 C oracle"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- the CUDA path
+def run_sfnn(args, dist):
+    import torch
+
+    import activation_sparse_ffn_threshold_b200 as sf
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.workload]
+    T = cfg.tokens
+    lay = W.make_layer(cfg, seed=args.seed)
+    Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank)
+    e = cfg.esize
+
+    # replicas: bytes touched between two visits of a replica >= 2 x L2
+    props = torch.cuda.get_device_properties(dev)
+    l2 = props.L2_cache_size
+    per_token = W.touched_bytes(cfg, expected_tokens_active(cfg))
+    R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_token))
+    handles = [sf.SparseFFN.from_layer(lay, device=dev) for _ in range(R)]
+    info = handles[0].info()
+    torch.cuda.synchronize()
+
+    X = torch.from_numpy(Xh).to(dev)
+    Y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+    # active-set sizes of the captured tokens (for the algorithmic byte count)
+    counts = []
+    for t in range(T):
+        _, c = handles[0].predict(X[t])
+        counts.append(c)
+    counts = torch.cat(counts).cpu().numpy().astype(np.int64)
+    bytes_tok = (info["predictor_bytes"] + counts * info["row_bytes_per_neuron"] + cfg.d * e + cfg.d * 4)
+    bytes_step = float(bytes_tok.sum())
+
+    # per-token event pairs captured with the graph
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(T)]
+    s = torch.cuda.Stream(device=dev)
+    for a, b in ev:  # materialise the events
+        a.record(s)
+        b.record(s)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for t in range(T):
+            handles[t % R].forward(X[t], Y[t])
+    torch.cuda.synchronize()
+    launches0 = sum(h.info()["launches"] for h in handles)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for t in range(T):
+            handles[t % R].set_profile_events(ev[t][0], ev[t][1])
+            handles[t % R].forward(X[t], Y[t])
+    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
+
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    gpu_uuid = str(props.uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            start.record(s)
+            for _ in range(args.steps):
+                g.replay()
+            stop.record(s)
+        torch.cuda.synchronize()
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    try:
+        tok_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    except Exception as exc:  # pragma: no cover
+        log(f"per-token events unavailable: {exc}")
+        tok_ms = None
+    clocks = clk.summary()
+    err = max(h.get_error() for h in handles)
+    if err:
+        raise SystemExit(f"device-side error latched: {err}")
+
+    t_max = dist.max(elapsed_ms)
+    tokens_total = dist.sum(args.steps * T)
+    value = tokens_total / (t_max / 1e3)
+    eff_gbs = bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9
+
+    peak, peak_kind = measured_peak()
+    roofline = None
+    if tok_ms is not None:
+        hot_ms = float(tok_ms.mean())
+        achieved = float(bytes_tok.mean()) / (hot_ms / 1e3) / 1e9
+        traffic, tsrc = profiled_traffic()
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "kernel": "one sfnn_forward hot path (all kernels of one token), per-token events in the graph",
+                    "algorithmic_bytes_per_launch": float(bytes_tok.mean()),
+                    "avg_launch_us": hot_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                    if peak_kind == "measured" else "fallback 6.65 TB/s",
+                    "traffic_source": tsrc}
+
+    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        xin = torch.from_numpy(Xh).pin_memory()
+        yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
+        xd = torch.empty(cfg.d, dtype=X.dtype, device=dev)
+        yd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
+        e2e_steps = max(1, min(args.steps, 20))
+        with torch.cuda.stream(s):
+            for t in range(T):  # warm-up
+                xd.copy_(xin[t], non_blocking=True)
+                handles[t % R].forward(xd, yd, stream=s)
+                yout[t].copy_(yd, non_blocking=True)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        with torch.cuda.stream(s):
+            a.record(s)
+            for _ in range(e2e_steps):
+                for t in range(T):
+                    xd.copy_(xin[t], non_blocking=True)
+                    handles[t % R].forward(xd, yd, stream=s)
+                    yout[t].copy_(yd, non_blocking=True)
+            b.record(s)
+        torch.cuda.synchronize()
+        e_max = dist.max(a.elapsed_time(b))
+        e2e = {"value": dist.sum(e2e_steps * T) / (e_max / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * cfg.d * e, "d2h_bytes_per_step": T * cfg.d * 4,
+               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        Xc = W.make_tokens(cfg, 64, seed=args.seed + 99)
+        cpu = cpu_baseline(cfg, lay, Xc, args.cpu_seconds)
+
+    line = {
+        "metric": "sparse-FFN decode tokens/s per layer", "value": value, "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": 1, "tokens_per_step": T,
+                   "replicas": R, "l2": f"inputs larger than L2: {R} weight replicas rotated per token, "
+                                        f"{bytes_step / T / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist.world} (no exchange)",
+                   "mean_active_neurons": float(counts.mean())},
+        "effective_gbs": eff_gbs,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    for h in handles:
+        h.close()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist(args.gpus)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, dist)
+        return run_sfnn(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

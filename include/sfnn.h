@@ -1,0 +1,216 @@
+/*
+ * sfnn.h -- activation-sparse FFN decode on NVIDIA B200 (sm_100a): the C ABI.
+ *
+ * The operation.  For one FFN layer with n neurons over model width d,
+ *
+ *     y = sum_{i in S(x)} act_i(x) * W_down[:, i]
+ *     ReLU : act_i(x) = relu(W_up[i] . x + b_i)
+ *     ReGLU: act_i(x) = relu(W_gate[i] . x + b_i) * (W_up[i] . x)
+ *     S(x) = { i : sigmoid(relu(x . A) . B + c)_i > 0.5 } = { i : (relu(x.A).B + c)_i > 0 }
+ *
+ * and the rows of W_up / W_gate and the columns of W_down that belong to
+ * neurons outside S(x) are neither read nor multiplied.  Sources: ReLU makes
+ * most FFN neurons inactive, an inactive neuron's down-projection row adds an
+ * exact zero and can be skipped, turning the step into a sparse-vector times
+ * dense-matrix product that saves both bytes and FLOPs (53ai.com "sparsity for
+ * LLM inference" page, section 激活稀疏, activation sparsity); a small per-layer
+ * MLP predicts which MLP neurons will be active and only those are computed
+ * (same page, sections 概述 and 自适应稀疏预测器, the PowerInfer overview and
+ * its adaptive sparse predictor; DejaVu's MLP predictor in section 如何推理加速);
+ * the predictor used here is a rank-r two-layer MLP, sigmoid(relu(x.A).B + c),
+ * thresholded at 0.5, evaluated as z > 0 because sigmoid is strictly
+ * increasing with sigmoid(0) = 1/2 (a tie z == 0 and a NaN are inactive).
+ * Neurons are stored in descending order of an offline activation frequency
+ * ("hot" neurons first), after PowerInfer's offline hot/cold profiling (same
+ * page, section 概述; hexiedandong.com PowerInfer news page, the power-law
+ * paragraph on figure (a)).
+ *
+ * Conventions for every entry point.
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *    owns every buffer it passes; a handle owns the layer's re-laid-out weights
+ *    and its scratch memory.
+ *  - Element type: x / X and all weights use the handle's wdtype (IEEE fp32
+ *    or fp16); outputs y / Y are fp32; index lists and counts are int32.
+ *  - Every call after sfnn_create is asynchronous on `stream` and never
+ *    synchronises the host, never aborts and never throws.  Argument errors
+ *    are returned at once and launch nothing.  Errors found on the device
+ *    (an out-of-range index passed in, a bounded wait that ran out) are
+ *    latched in the handle and returned by sfnn_get_error.
+ *  - A handle must not be used from two streams at the same time: its scratch
+ *    memory is shared by its calls.
+ *  - Index lists have set semantics: they hold each selected neuron once, in
+ *    the caller's original numbering, in the handle's internal (hotness) order,
+ *    which is deterministic.
+ *  - Deterministic results: the same inputs give bitwise the same outputs.
+ */
+#ifndef SFNN_H
+#define SFNN_H
+
+#include <stdint.h>
+
+/* Entry points are the only symbols the shared library exports. */
+#if defined(__GNUC__)
+#define SFNN_API __attribute__((visibility("default")))
+#else
+#define SFNN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (struct CUstream_st *); 0 is the legacy default stream. */
+typedef struct CUstream_st *sfnn_stream_t;
+/* Same type as cudaEvent_t (struct CUevent_st *). */
+typedef struct CUevent_st *sfnn_event_t;
+
+typedef struct sfnn_ctx *sfnn_handle;
+
+typedef enum {
+    SFNN_OK = 0,
+    SFNN_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, an inconsistent descriptor */
+    SFNN_ERR_CUDA = 2,        /* a CUDA runtime call or kernel launch failed */
+    SFNN_ERR_OOM = 3,         /* device memory allocation failed in sfnn_create */
+    SFNN_ERR_UNSUPPORTED = 4, /* valid but outside what this build handles (see sfnn_create) */
+    SFNN_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (latched) */
+} sfnn_status;
+
+typedef enum { SFNN_RELU = 0, SFNN_REGLU = 1 } sfnn_act;
+typedef enum { SFNN_F32 = 0, SFNN_F16 = 1 } sfnn_dtype;
+
+/* Which kernels the batched path (b > 1) uses for the gathered rows. */
+typedef enum {
+    SFNN_BATCH_AUTO = 0,        /* choose from the expected union density */
+    SFNN_BATCH_CUDA_CORE = 1,   /* multi-token gather on CUDA cores */
+    SFNN_BATCH_TENSOR_CORE = 2  /* gathered GEMM on tcgen05 tensor cores */
+} sfnn_batch_path;
+
+/*
+ * One FFN layer in PyTorch layouts (row-major):
+ *   w_up   [n x d]  up.weight                (device, wdtype)
+ *   w_gate [n x d]  gate.weight, ReGLU only; NULL for ReLU
+ *   b      [n]      bias of the ReLU'd projection (up for ReLU, gate for ReGLU)
+ *   w_down [d x n]  down.weight
+ *   pa     [d x r]  predictor A;  pb [r x n] predictor B;  pc [n] predictor bias c
+ *   hotness[n]      HOST, optional: offline activation frequency of each neuron;
+ *                   NULL keeps the original order.  NaN counts as lowest.
+ * The inputs are read during sfnn_create only; they may be freed once it returns.
+ */
+typedef struct {
+    int32_t d, n, r;
+    int32_t max_batch; /* largest b later passed to sfnn_forward_batch / sfnn_forward_stack, 1..32 */
+    int32_t act;       /* sfnn_act */
+    int32_t wdtype;    /* sfnn_dtype */
+    const void *w_up;
+    const void *w_gate;
+    const void *b;
+    const void *w_down;
+    const void *pa;
+    const void *pb;
+    const void *pc;
+    const float *hotness;
+} sfnn_layer_desc;
+
+/* Read-only facts about a handle (sizes in bytes). */
+typedef struct {
+    int32_t d, n, r, max_batch, act, wdtype;
+    int32_t num_sms;              /* SMs of the device the handle lives on */
+    int32_t batch_path;           /* sfnn_batch_path in force */
+    int64_t weight_bytes;         /* re-laid-out weights held by the handle */
+    int64_t scratch_bytes;        /* scratch memory held by the handle */
+    int64_t predictor_bytes;      /* bytes of A, B and c one token's predictor reads */
+    int64_t row_bytes_per_neuron; /* bytes of rows + bias one active neuron costs */
+    int64_t launches;             /* kernels launched (or captured) by this handle so far */
+} sfnn_info;
+
+/*
+ * Build a handle for one layer on the current device.  Re-lays the weights out
+ * for the decode path: neurons in descending hotness; each neuron's rows
+ * (gate, up, and its W_down column as a contiguous row) stored together;
+ * A transposed to [r x d]; B transposed to neuron-major [n x r].
+ * Requirements: d, n, r >= 1; d and r multiples of 8 (fp16) or 4 (fp32);
+ * 1 <= max_batch <= 32; r * max_batch <= 32768 (SFNN_ERR_UNSUPPORTED otherwise).
+ * Allocates device memory (SFNN_ERR_OOM) and synchronises `stream` before
+ * returning.  On error *out is set to NULL.
+ */
+SFNN_API sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_handle *out);
+
+/* Free a handle (synchronises its device).  NULL is accepted. */
+SFNN_API sfnn_status sfnn_destroy(sfnn_handle h);
+
+/*
+ * Predictor only: the set S(x) for one token.
+ *   x     [d] wdtype
+ *   idx   [n] int32 out: the |S| selected neurons first (caller numbering); capacity n
+ *   count [1] int32 out: |S|
+ */
+SFNN_API sfnn_status sfnn_predict(sfnn_handle h, const void *x, int32_t *idx, int32_t *count, sfnn_stream_t stream);
+
+/*
+ * One decode step for one token: y = sum_{i in S} act_i(x) W_down[:, i].
+ *   x     [d] wdtype
+ *   idx   NULL: S = S(x) from the predictor.  Otherwise [*count] int32 neuron
+ *         indices (caller numbering) that replace the predictor's set; order is
+ *         free, duplicates count once, out-of-range entries are skipped and
+ *         latch SFNN_ERR_INVALID_ARG.
+ *   count [1] int32 (device), read only when idx != NULL; clamped to [0, n]
+ *   y     [d] fp32 out
+ */
+SFNN_API sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *idx, const int32_t *count, float *y,
+                         sfnn_stream_t stream);
+
+/*
+ * b independent tokens at once (1 <= b <= max_batch): row t of Y equals
+ * sfnn_forward of X[t].  The union of the b predicted sets is read once and
+ * applied to the tokens active on each row.
+ *   X      [b x d] wdtype;  Y [b x d] fp32 out
+ *   idx    [b x n] int32 out or NULL: token t's set in row t (first counts[t] entries)
+ *   counts [b] int32 out or NULL: |S_t|
+ */
+SFNN_API sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b, float *Y, int32_t *idx, int32_t *counts,
+                               sfnn_stream_t stream);
+
+/*
+ * A stack of layers with a residual stream:  X_{l+1} = X_l + FFN_l(round(X_l)),
+ * where round() converts the fp32 residual to the layers' wdtype (nearest even).
+ * All layers share d, wdtype and max_batch >= b (and n when idx != NULL).
+ *   layers [num_layers] HOST array of handles
+ *   X0     [b x d] fp32 in;  XL [b x d] fp32 out (may alias X0)
+ *   idx    [num_layers x b x n] int32 out or NULL;  counts [num_layers x b] int32 out or NULL
+ */
+SFNN_API sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_layers, const float *X0, int32_t b,
+                               float *XL, int32_t *idx, int32_t *counts, sfnn_stream_t stream);
+
+/* Choose the batched path (sfnn_batch_path); SFNN_BATCH_AUTO by default. */
+SFNN_API sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path);
+
+/*
+ * Diagnostics: when `before`/`after` are non-NULL, the next sfnn_forward or
+ * sfnn_forward_batch call of this handle records `before` on its stream just
+ * before the first kernel of its hot path and `after` just after the last one;
+ * the pair is consumed by that call.  Events may be recorded while the stream
+ * is being captured into a CUDA graph.
+ */
+SFNN_API sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before, sfnn_event_t after);
+
+/* Fill *info (host struct). */
+SFNN_API sfnn_status sfnn_query(sfnn_handle h, sfnn_info *info);
+
+/* Return and clear the latched device-side error of h (synchronises h's device). */
+SFNN_API sfnn_status sfnn_get_error(sfnn_handle h);
+
+/* Static description of a status code; never NULL. */
+SFNN_API const char *sfnn_status_str(sfnn_status s);
+
+/*
+ * Host only: the storage order sfnn_create uses.  perm[k] = the neuron stored
+ * at position k: hotness descending, ties by ascending index, NaN last.
+ *   hotness [n] HOST in;  perm [n] HOST out.
+ */
+SFNN_API sfnn_status sfnn_hotness_order(const float *hotness, int32_t n, int32_t *perm);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFNN_H */
