@@ -27,6 +27,7 @@ F32, F16 = 0, 1
 BATCH_AUTO, BATCH_CUDA_CORE, BATCH_TENSOR_CORE = 0, 1, 2
 STATUS = {0: "SFNN_OK", 1: "SFNN_ERR_INVALID_ARG", 2: "SFNN_ERR_CUDA", 3: "SFNN_ERR_OOM",
           4: "SFNN_ERR_UNSUPPORTED", 5: "SFNN_ERR_TIMEOUT"}
+STATUS_CODES = {v: k for k, v in STATUS.items()}
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libsfnn.so")
@@ -78,6 +79,8 @@ def load_library():
         "sfnn_forward_batch": ([P, P, I, P, P, P, P], S),
         "sfnn_forward_stack": ([P, I, P, I, P, P, P, P], S),
         "sfnn_set_batch_path": ([P, I], S),
+        "sfnn_set_fused_decode": ([P, I], S),
+        "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
         "sfnn_query": ([P, ctypes.POINTER(Info)], S),
         "sfnn_get_error": ([P], S),
@@ -235,6 +238,12 @@ class SparseFFN:
 
     def set_batch_path(self, path: int):
         _check(self._lib.sfnn_set_batch_path(self._h, int(path)), "sfnn_set_batch_path")
+
+    def set_fused_decode(self, enable: bool):
+        _check(self._lib.sfnn_set_fused_decode(self._h, int(bool(enable))), "sfnn_set_fused_decode")
+
+    def debug_stall_next_barrier(self, stream=None):
+        _check(self._lib.sfnn_debug_stall_next_barrier(self._h, _stream(stream)), "sfnn_debug_stall_next_barrier")
 
     def set_profile_events(self, before, after):
         """torch.cuda.Event pair bracketing the next forward call's kernels (events must exist)."""

@@ -33,7 +33,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -72,8 +72,15 @@ bool same_device(const sfnn_ctx *h) {
   return cudaGetDevice(&dev) == cudaSuccess && dev == h->device;
 }
 
+// Inside stream capture a plain record only orders work; the external flag makes it a
+// real event-record node whose timestamps can be read after the graph runs.
 void record_if(cudaEvent_t ev, cudaStream_t s) {
-  if (ev) cudaEventRecord(ev, s);
+  if (!ev) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, s);
 }
 
 // The shared body of forward / forward_batch / one stack layer.
@@ -83,6 +90,17 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
   cudaEvent_t before = h->prof_before, after = h->prof_after;
   h->prof_before = h->prof_after = nullptr;
   record_if(before, s);
+  if (b == 1 && predict && !idx_out && !cnt_out && h->fused_ok && h->fused_on) {
+    Decode1Params P = h->d1;
+    P.x = X;
+    P.y = Y;
+    P.resid = resid;
+    P.xnext = xnext;
+    SFNN_TRY(launch_decode1(P, s, true));
+    record_if(after, s);
+    h->launches += 1;
+    return SFNN_OK;
+  }
   if (predict) {
     SFNN_TRY(launch_hidden(h, X, b, s));
     SFNN_TRY(launch_logits(h, b, s));
@@ -97,6 +115,50 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
   record_if(after, s);
   h->launches += predict ? 6 : 5;
   return SFNN_OK;
+}
+
+// The fused single-token kernel's plan: ring stages sized to the largest of a neuron's
+// record and one B^T row, as many stages as fit next to the fixed buffers, one CTA per SM.
+void plan_decode1(sfnn_ctx *h, int G) {
+  const Layout &L = h->L;
+  Decode1Params &P = h->d1;
+  P = Decode1Params{};
+  h->fused_ok = false;
+  P.At = h->At;
+  P.Bt = h->Bt;
+  P.cvec = h->cvec;
+  P.bias = h->bias;
+  P.rows = h->rows;
+  P.hbuf = h->h;
+  P.part = h->part;
+  P.bar = h->bar;
+  P.err = h->err;
+  P.d = L.d;
+  P.n = L.n;
+  P.r = L.r;
+  P.nproj = L.nproj;
+  P.act = L.act;
+  P.dt = L.dt;
+  P.G = G;
+  const int rec = L.nproj * L.d * L.esize, btrow = L.r * L.esize;
+  P.SB = (int)decode1_align((size_t)std::max(rec, btrow), 128);
+  P.NPC = P.SB / btrow;
+  P.tile_max = (L.n + G - 1) / G;
+  P.chunks_max = (P.tile_max + P.NPC - 1) / P.NPC;
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  const int budget = std::min(optin, kDecode1SmemMax);
+  P.S = 0;
+  const size_t fixed = decode1_layout(P).total;
+  if ((int64_t)budget <= (int64_t)fixed) return;
+  P.S = std::min(64, (int)((budget - fixed) / P.SB));
+  while (P.S >= 2 && decode1_layout(P).total > (size_t)budget) --P.S;
+  if (P.S < 2) return;
+  if (L.d / L.vec > 256 * 8) return;  // columns per thread beyond the kernel's register plan
+  // the grid barriers need every CTA resident at once
+  if (decode1_blocks_per_sm(P) < 1) return;
+  h->fused_ok = true;
+  h->fused_on = true;
 }
 
 }  // namespace
@@ -153,13 +215,18 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
     return SFNN_ERR_CUDA;
   }
 
-  // storage order
-  std::vector<int32_t> perm(L.n), iperm(L.n);
+  // Storage order: hotness ranks (descending activation frequency, or the original
+  // order without a profile) dealt round-robin to G contiguous tiles, one per CTA of
+  // the fused kernel, so every tile gets the same mix of hot and cold neurons and
+  // keeps its hottest neurons first.
+  const int G = std::min(h->num_sms, L.n);
+  std::vector<int32_t> by_rank(L.n), perm(L.n), iperm(L.n);
   if (desc->hotness) {
-    sfnn_hotness_order(desc->hotness, L.n, perm.data());
+    sfnn_hotness_order(desc->hotness, L.n, by_rank.data());
   } else {
-    std::iota(perm.begin(), perm.end(), 0);
+    std::iota(by_rank.begin(), by_rank.end(), 0);
   }
+  for (int k = 0; k < L.n; ++k) perm[decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
   for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
   for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
   if (desc->hotness) {
@@ -192,9 +259,10 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->utok, n * 4, false},
       {(void **)&h->ucount, 4, false},
       {(void **)&h->acoef, n * mb * 4, false},
-      {(void **)&h->part, (size_t)kMaxSplits * mb * d * 4, false},
+      {(void **)&h->part, (size_t)std::max<size_t>((size_t)kMaxSplits * mb, (size_t)G) * d * 4, false},
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
+      {(void **)&h->bar, 8, false},
   };
   for (auto &q : reqs) {
     if (cudaMalloc(q.ptr, q.bytes) != cudaSuccess) {
@@ -208,8 +276,11 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = cudaMemcpy(h->iperm, iperm.data(), n * 4, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->err, 0, 4, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->ucount, 0, 4, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, 8, s);
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
+  if (ce == cudaSuccess) ce = configure_decode1();
+  if (ce == cudaSuccess) plan_decode1(h, G);
   if (ce == cudaSuccess) ce = launch_layout(h, desc, s);
   if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
   if (ce != cudaSuccess) {
@@ -293,6 +364,24 @@ sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
   return SFNN_OK;
 }
 
+sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (enable && !h->fused_ok) return SFNN_ERR_UNSUPPORTED;
+  h->fused_on = enable != 0;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_debug_stall_next_barrier(sfnn_handle h, sfnn_stream_t stream) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (!h->fused_ok) return SFNN_ERR_UNSUPPORTED;
+  // an arrival count already past the last arriver's value: no CTA completes the barrier
+  const uint32_t stuck = 0x40000000u;
+  return from_cuda(cudaMemcpyAsync(h->bar, &stuck, 4, cudaMemcpyHostToDevice,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                       ? cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream))
+                       : cudaErrorUnknown);
+}
+
 sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before, sfnn_event_t after) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   h->prof_before = reinterpret_cast<cudaEvent_t>(before);
@@ -325,6 +414,8 @@ sfnn_status sfnn_get_error(sfnn_handle h) {
   int32_t v = 0;
   if (cudaMemcpy(&v, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFNN_ERR_CUDA;
   if (v != 0 && cudaMemset(h->err, 0, 4) != cudaSuccess) return SFNN_ERR_CUDA;
+  // a timed-out grid barrier leaves its counter behind: start it afresh
+  if (v == SFNN_ERR_TIMEOUT && cudaMemset(h->bar, 0, 8) != cudaSuccess) return SFNN_ERR_CUDA;
   return static_cast<sfnn_status>(v);
 }
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "decode1.cuh"
 #include "sfnn.h"
 
 namespace sfnn {
@@ -47,6 +48,10 @@ struct sfnn_ctx {
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
+  uint32_t *bar;     // [2] grid barrier state of the fused kernel
+  bool fused_ok;     // the fused single-token kernel fits this layer
+  bool fused_on;     // ... and is enabled (sfnn_set_fused_decode)
+  sfnn::Decode1Params d1;  // its launch plan (pointers to x/y filled per call)
   int64_t weight_bytes, scratch_bytes;
   int64_t launches;  // kernels this handle has launched (or captured into a graph)
   // one-shot profiling events around the dominant kernel

@@ -181,6 +181,24 @@ SFNN_API sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b,
 SFNN_API sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_layers, const float *X0, int32_t b,
                                float *XL, int32_t *idx, int32_t *counts, sfnn_stream_t stream);
 
+/*
+ * Enable (default) or disable the fused single-token kernel, which runs a whole
+ * decode step of one token in one launch: one persistent CTA per SM, bulk async
+ * copies of the predictor's B^T tile and of the active neurons' rows through a
+ * shared-memory ring, grid-wide barriers with bounded waits.  Disabled, one token
+ * runs through the same multi-kernel path as a batch.  SFNN_ERR_UNSUPPORTED when
+ * enabling it on a layer it does not fit (too large a record or too few SMs).
+ */
+SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
+
+/*
+ * Fault injection for tests (synchronises `stream`): the next fused decode launch
+ * of h finds its grid barrier unable to complete, waits out its bound (about one
+ * second), returns without a result and latches SFNN_ERR_TIMEOUT; sfnn_get_error
+ * reports it and restores the barrier, after which h works normally.
+ */
+SFNN_API sfnn_status sfnn_debug_stall_next_barrier(sfnn_handle h, sfnn_stream_t stream);
+
 /* Choose the batched path (sfnn_batch_path); SFNN_BATCH_AUTO by default. */
 SFNN_API sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path);
 

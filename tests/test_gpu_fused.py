@@ -1,0 +1,100 @@
+"""The fused single-token decode kernel (one launch per token).
+
+* it agrees with the multi-kernel path and with the oracle, on layers whose
+  tiles hold one or several B^T chunks and whose rows need one or several
+  columns per thread (fp32 and fp16, ReLU and ReGLU, ragged n);
+* consecutive launches on the same handle (programmatic dependent launch lets
+  the next one start early) stay correct and bitwise reproducible;
+* the residual stack runs through it;
+* a grid barrier that cannot complete runs out after its bound, latches
+  SFNN_ERR_TIMEOUT, leaves the context usable, and the handle recovers.
+"""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_ffn_threshold_b200 as sf
+import oracle
+import workload as W
+from parity_util import check_token, dev, mask_from_idx
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    ("tiny_relu_f32", 512, 2048, 64),
+    ("opt6.7b_relu", 1024, 3001, 128),
+    ("70b_reglu", 2048, 5003, 256),
+    ("opt30b_relu", 7168, 4099, 1024),
+    ("70b_reglu", 8192, 1500, 1024),
+]
+
+
+@pytest.mark.parametrize("base,d,n,r", SHAPES)
+def test_fused_matches_multikernel_and_oracle(base, d, n, r):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=11)
+    h = sf.SparseFFN.from_layer(lay)
+    X = W.make_tokens(cfg, 4, seed=12)
+    for t in range(4):
+        xd = dev(X[t])
+        h.set_fused_decode(True)
+        yf = h.forward(xd).cpu().numpy()
+        h.set_fused_decode(False)
+        ym = h.forward(xd).cpu().numpy()
+        h.set_fused_decode(True)
+        assert oracle.within_tolerance(yf, ym.astype(np.float64))[0]
+        idx, cnt = h.predict(xd)
+        check_token(lay, X[t], yf, mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n), f"{base} t={t}")
+    assert h.get_error() == 0
+
+
+def test_back_to_back_launches_same_handle():
+    cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=2048, n=6000, r=256)
+    lay = W.make_layer(cfg, seed=13)
+    h = sf.SparseFFN.from_layer(lay)
+    X = dev(W.make_tokens(cfg, 16, seed=14))
+    Y1 = torch.empty((16, cfg.d), dtype=torch.float32, device="cuda")
+    for t in range(16):
+        h.forward(X[t], Y1[t])
+    torch.cuda.synchronize()
+    Y2 = torch.stack([h.forward(X[t]) for t in range(16)])
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    Xh = X.cpu().numpy()
+    for t in (0, 7, 15):
+        idx, cnt = h.predict(X[t])
+        check_token(lay, Xh[t], Y1[t].cpu().numpy(), mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n))
+    assert h.get_error() == 0
+
+
+def test_stack_through_fused_kernel():
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
+    layers = [W.make_layer(cfg, seed=15, layer=l) for l in range(3)]
+    hs = [sf.SparseFFN.from_layer(l) for l in layers]
+    x0 = W.make_tokens(cfg, 1, seed=16)[0]
+    X0 = torch.from_numpy(x0.astype(np.float32)).cuda()
+    XL_fused = sf.forward_stack(hs, X0).cpu().numpy()
+    XL_sets, sidx, scnt = sf.forward_stack(hs, X0, return_sets=True)
+    masks = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), cfg.n) for l in range(3)]
+    xref, recs = oracle.forward_stack(layers, x0.astype(np.float64), masks_other=masks)
+    assert all(r["mismatches"].size == 0 for r in recs)
+    base = x0.astype(np.float64)
+    assert oracle.within_tolerance(XL_fused.astype(np.float64) - base, xref - base)[0]
+    assert oracle.within_tolerance(XL_sets.cpu().numpy().astype(np.float64) - base, xref - base)[0]
+
+
+def test_grid_barrier_timeout_is_reported_and_recovers():
+    cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=1024, n=3000, r=128)
+    lay = W.make_layer(cfg, seed=17)
+    h = sf.SparseFFN.from_layer(lay)
+    xd = dev(W.make_tokens(cfg, 1, seed=18)[0])
+    y_ok = h.forward(xd).cpu().numpy()
+    assert h.get_error() == 0
+    h.debug_stall_next_barrier()
+    h.forward(xd)
+    torch.cuda.synchronize()  # returns: the kernel gave up after its bound
+    assert h.get_error() == sf.STATUS_CODES["SFNN_ERR_TIMEOUT"]
+    assert h.get_error() == 0
+    y_again = h.forward(xd).cpu().numpy()
+    assert np.array_equal(y_again, y_ok)
+    assert h.get_error() == 0
