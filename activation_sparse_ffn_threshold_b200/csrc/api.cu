@@ -67,6 +67,9 @@ sfnn_status check_desc(const sfnn_layer_desc *d) {
   return SFNN_OK;
 }
 
+// Inputs are read with 16-byte vector loads and bulk async copies.
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 bool same_device(const sfnn_ctx *h) {
   int dev = -1;
   return cudaGetDevice(&dev) == cudaSuccess && dev == h->device;
@@ -117,8 +120,8 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
   return SFNN_OK;
 }
 
-// The fused single-token kernel's plan: ring stages sized to the largest of a neuron's
-// record and one B^T row, as many stages as fit next to the fixed buffers, one CTA per SM.
+// The fused single-token kernel's plan: one CTA per SM, each owning a contiguous tile of
+// neurons; h is held in registers (at most 4 chunks per lane), all CTAs must be resident.
 void plan_decode1(sfnn_ctx *h, int G) {
   const Layout &L = h->L;
   Decode1Params &P = h->d1;
@@ -140,22 +143,9 @@ void plan_decode1(sfnn_ctx *h, int G) {
   P.act = L.act;
   P.dt = L.dt;
   P.G = G;
-  const int rec = L.nproj * L.d * L.esize, btrow = L.r * L.esize;
-  P.SB = (int)decode1_align((size_t)std::max(rec, btrow), 128);
-  P.NPC = P.SB / btrow;
   P.tile_max = (L.n + G - 1) / G;
-  P.chunks_max = (P.tile_max + P.NPC - 1) / P.NPC;
-  int optin = 0;
-  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
-  const int budget = std::min(optin, kDecode1SmemMax);
-  P.S = 0;
-  const size_t fixed = decode1_layout(P).total;
-  if ((int64_t)budget <= (int64_t)fixed) return;
-  P.S = std::min(64, (int)((budget - fixed) / P.SB));
-  while (P.S >= 2 && decode1_layout(P).total > (size_t)budget) --P.S;
-  if (P.S < 2) return;
-  if (L.d / L.vec > 256 * 8) return;  // columns per thread beyond the kernel's register plan
-  // the grid barriers need every CTA resident at once
+  P.nseg = (L.d / L.vec + 255) / 256;
+  if (L.r / L.vec > 32 * 4) return;
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
   h->fused_on = true;
@@ -262,7 +252,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->part, (size_t)std::max<size_t>((size_t)kMaxSplits * mb, (size_t)G) * d * 4, false},
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
-      {(void **)&h->bar, 8, false},
+      {(void **)&h->bar, sizeof(uint64_t), false},
   };
   for (auto &q : reqs) {
     if (cudaMalloc(q.ptr, q.bytes) != cudaSuccess) {
@@ -276,7 +266,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = cudaMemcpy(h->iperm, iperm.data(), n * 4, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->err, 0, 4, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->ucount, 0, 4, s);
-  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, 8, s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, sizeof(uint64_t), s);
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();
@@ -300,7 +290,7 @@ sfnn_status sfnn_destroy(sfnn_handle h) {
 }
 
 sfnn_status sfnn_predict(sfnn_handle h, const void *x, int32_t *idx, int32_t *count, sfnn_stream_t stream) {
-  if (!h || !x || !idx || !count) return SFNN_ERR_INVALID_ARG;
+  if (!h || !x || !idx || !count || !aligned16(x)) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   SFNN_TRY(launch_hidden(h, x, 1, s));
@@ -312,7 +302,7 @@ sfnn_status sfnn_predict(sfnn_handle h, const void *x, int32_t *idx, int32_t *co
 
 sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *idx, const int32_t *count, float *y,
                          sfnn_stream_t stream) {
-  if (!h || !x || !y || (idx && !count)) return SFNN_ERR_INVALID_ARG;
+  if (!h || !x || !y || (idx && !count) || !aligned16(x)) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
   return run_layer(h, x, 1, idx == nullptr, idx, count, nullptr, nullptr, nullptr, y, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
@@ -320,7 +310,7 @@ sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *idx, const
 
 sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b, float *Y, int32_t *idx, int32_t *counts,
                                sfnn_stream_t stream) {
-  if (!h || !X || !Y || b < 1 || b > h->max_batch) return SFNN_ERR_INVALID_ARG;
+  if (!h || !X || !Y || b < 1 || b > h->max_batch || !aligned16(X)) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
   return run_layer(h, X, b, true, nullptr, nullptr, idx, counts, nullptr, Y, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
@@ -374,12 +364,12 @@ sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable) {
 sfnn_status sfnn_debug_stall_next_barrier(sfnn_handle h, sfnn_stream_t stream) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   if (!h->fused_ok) return SFNN_ERR_UNSUPPORTED;
-  // an arrival count already past the last arriver's value: no CTA completes the barrier
-  const uint32_t stuck = 0x40000000u;
-  return from_cuda(cudaMemcpyAsync(h->bar, &stuck, 4, cudaMemcpyHostToDevice,
-                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-                       ? cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream))
-                       : cudaErrorUnknown);
+  // one arrival too many: the counter is off by one from every barrier instance, so the
+  // next launch's CTAs wait for a count that its own arrivals never reach
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_barrier_bump(h->bar, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return from_cuda(e);
 }
 
 sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before, sfnn_event_t after) {
@@ -415,7 +405,7 @@ sfnn_status sfnn_get_error(sfnn_handle h) {
   if (cudaMemcpy(&v, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return SFNN_ERR_CUDA;
   if (v != 0 && cudaMemset(h->err, 0, 4) != cudaSuccess) return SFNN_ERR_CUDA;
   // a timed-out grid barrier leaves its counter behind: start it afresh
-  if (v == SFNN_ERR_TIMEOUT && cudaMemset(h->bar, 0, 8) != cudaSuccess) return SFNN_ERR_CUDA;
+  if (v == SFNN_ERR_TIMEOUT && cudaMemset(h->bar, 0, sizeof(uint64_t)) != cudaSuccess) return SFNN_ERR_CUDA;
   return static_cast<sfnn_status>(v);
 }
 

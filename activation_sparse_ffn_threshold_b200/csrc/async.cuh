@@ -48,19 +48,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Nanoseconds of the GPU's global timer.
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
+// Non-blocking test of the same condition.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false once `limit_ns` have passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0;; ++i) {
+// Bounds of waits are counted in SM clock cycles (clock64 is a cheap per-SM counter);
+// 2^31 cycles is about one second at the B200's clocks.
+constexpr uint64_t kWaitCycles = 1ull << 31;
+
+// Wait for the phase with the given parity to complete; false after `limit` cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
+  const uint64_t t0 = clock64();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && globaltimer_ns() - t0 > limit_ns) return false;
+    if ((uint64_t)(clock64() - t0) > limit) return false;
   }
 }
 
@@ -88,24 +98,31 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   return v;
 }
 
-// Sense-reversing grid barrier over `nblocks` co-resident CTAs, called by ONE thread per
-// CTA.  state[0] counts arrivals, state[1] is the generation.  Returns false if the wait
-// ran out after `limit_ns` (the caller latches an error).
-__device__ __forceinline__ bool grid_barrier(uint32_t *state, uint32_t nblocks, uint64_t limit_ns) {
-  const uint32_t gen = ld_acquire_gpu(state + 1);
-  __threadfence();
-  const uint32_t arrived = atomicAdd(state, 1u);
-  if (arrived == nblocks - 1) {
-    atomicExch(state, 0u);
-    __threadfence();
-    atomicAdd(state + 1, 1u);
-    return true;
-  }
-  const uint64_t t0 = globaltimer_ns();
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t atom_add_release_gpu_u64(uint64_t *p, uint64_t v) {
+  uint64_t old;
+  asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+// Grid barrier over `nblocks` co-resident CTAs, called by ONE thread per CTA, on a 64-bit
+// arrival counter that only grows: the ticket an arrival draws names its barrier instance
+// (ticket / nblocks), which completes when the counter reaches the next multiple of
+// nblocks.  One release-add and acquire polls; nothing is reset between instances or
+// launches.  Returns false if the wait ran out after `limit` cycles (the caller latches
+// an error; the counter must then be zeroed before the next launch).
+__device__ __forceinline__ bool grid_barrier(uint64_t *count, uint32_t nblocks, uint64_t limit) {
+  const uint64_t ticket = atom_add_release_gpu_u64(count, 1ull);
+  const uint64_t target = (ticket / nblocks + 1) * nblocks;
+  const uint64_t t0 = clock64();
   for (;;) {
-    if (ld_acquire_gpu(state + 1) != gen) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-    __nanosleep(32);
+    if (ld_acquire_gpu_u64(count) >= target) return true;
+    if ((uint64_t)(clock64() - t0) > limit) return false;
   }
 }
 

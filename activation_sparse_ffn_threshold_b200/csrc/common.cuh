@@ -48,7 +48,7 @@ struct sfnn_ctx {
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
-  uint32_t *bar;     // [2] grid barrier state of the fused kernel
+  uint64_t *bar;     // grid barrier arrival counter of the fused kernel
   bool fused_ok;     // the fused single-token kernel fits this layer
   bool fused_on;     // ... and is enabled (sfnn_set_fused_decode)
   sfnn::Decode1Params d1;  // its launch plan (pointers to x/y filled per call)

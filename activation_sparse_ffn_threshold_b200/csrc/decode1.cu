@@ -1,39 +1,37 @@
 // decode1.cu -- the fused single-token decode kernel (batch 1): one launch per token.
 //
 // Decode is bound by reading weights, not by arithmetic (53ai.com "sparsity for LLM
-// inference" page, its opening analysis of decode latency: the I/O of loading
-// parameters dominates token generation), so this kernel is organised around keeping
-// HBM busy from the first cycle to the last:
+// inference" page, its opening analysis: the I/O of loading parameters dominates token
+// generation), so the kernel is a sequence of streaming phases, each keeping many
+// 16-byte loads in flight per SM, inside one persistent launch:
 //
-//   grid: one persistent CTA per SM (G CTAs).  CTA c owns a contiguous tile of
-//   neurons; the storage order deals hotness ranks round-robin to the tiles, so every
-//   tile holds the same mix of hot and cold neurons (equal expected work), hottest
-//   first inside the tile.
+//   grid: one CTA of 16 warps per SM (G CTAs, all resident).  CTA c owns a contiguous
+//   tile of neurons; the storage order deals hotness ranks round-robin to the tiles,
+//   so every tile holds the same mix of hot and cold neurons (equal expected work),
+//   hottest first inside the tile.
 //
-//   warp 8 (producer, one thread) streams everything the CTA reads through a ring of
-//   S shared-memory stages with 1-D bulk async copies (TMA engine, cp.async.bulk,
-//   mbarrier completion): first the tile's rows of the predictor's B^T (no dependence
-//   on x, so they are in flight while the hidden layer is computed), then, as soon as
-//   the consumers have decided a chunk of neurons, the [gate|up|down] record of every
-//   active neuron of that chunk.  Inactive neurons' records are never requested.
+//   A   h_j = relu(A^T[j] . x): one warp per predictor row, every chunk of the row
+//       requested at once (the first row before waiting for the previous kernel);
+//       meanwhile one warp asks L2 to prefetch the CTA's tile of B^T.  h goes to
+//       global memory; grid barrier.
+//   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron with a 3-deep
+//       register pipeline over the warp's neurons; neuron i is active iff z_i > 0
+//       (sigmoid(z) > 0.5).  The tile's active positions are compacted in order.
+//   C1  up (and gate) dot products of the active rows, split in 4 KB segments spread
+//       over all warps (2-deep pipeline); segment sums added in a fixed order, then
+//       ReLU / ReGLU.  Rows of inactive neurons are never requested.
+//   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
+//       column accumulators, 4 rows in flight.
+//   D   the CTA's partial y goes to global memory; grid barrier; CTA c sums a column
+//       slice of all G partials in a fixed order (two-phase, deterministic) -> y
+//       (+ residual, + rounded next-layer input).
 //
-//   warps 0-7 (consumers):
-//     P1  h_j = relu(A^T[j] . x) for the CTA's share of the r predictor rows (one warp
-//         per row, 128-bit loads), written to global; grid barrier.
-//     P2  per B^T chunk: z_i = B^T[i] . h + c_i, one warp per neuron; neuron i is
-//         active iff z_i > 0 (sigmoid(z) > 0.5); decisions go to a shared bit set the
-//         producer reads.
-//     P3  per active record: the up (and gate) dot products split over all 256
-//         threads and summed in a fixed order, ReLU / ReGLU, then the axpy of the
-//         neuron's contiguous W_down row into per-thread column accumulators.
-//     P4  the CTA's partial y goes to global; grid barrier; CTA c sums a column slice
-//         of all G partials in a fixed order (two-phase, deterministic) -> y
-//         (+ residual, + rounded next-layer input).
-//
-// PDL: the kernel lets the next kernel in the stream launch at once and reads x, and
-// writes anything, only after griddepcontrol.wait; weights are read before it.
-// Every wait is bounded; on a timeout the kernel latches SFNN_ERR_TIMEOUT, lets its
-// copies in flight land, and returns.
+// The predictor's dot products keep the order of the multi-kernel predictor (lane l
+// takes 16-byte chunks l, l+32, ... into one accumulator, then a butterfly sum), so
+// both paths decide every neuron identically.  PDL: the kernel lets the next one
+// launch at once and reads x, and writes anything, only after griddepcontrol.wait.
+// The two grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT
+// and returns without a result.
 #include "async.cuh"
 #include "common.cuh"
 #include "decode1.cuh"
@@ -41,416 +39,358 @@
 namespace sfnn {
 namespace {
 
-constexpr int kCW = 8;                 // consumer warps
-constexpr int kConsumers = kCW * 32;   // consumer threads
-constexpr int kThreads1 = kConsumers + 32;
-constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
-enum : int { kItemBt = 0, kItemRow = 1, kItemEnd = 2 };
+constexpr int kT = kDecode1Threads;
+constexpr int kW = kT / 32;
+constexpr int kSegChunks = 256;  // 16-byte chunks of one C1 segment (8 per lane)
+constexpr int kSmemCap = 200 * 1024;
 
-struct Smem {
-  unsigned char *ring;
-  unsigned char *x;
-  float *h, *bias, *c, *red, *red2;
-  uint32_t *bits;
-  int *decided;
-  int4 *desc;
-  uint64_t *full, *empty, *xbar, *sync;
-  int *abort_flag;
-};
-
-__device__ Smem carve(unsigned char *base, const Decode1Params &P) {
-  Decode1Layout l = decode1_layout(P);
-  Smem s;
-  s.ring = base;
-  s.x = base + l.x;
-  s.h = reinterpret_cast<float *>(base + l.h);
-  s.bias = reinterpret_cast<float *>(base + l.bias);
-  s.c = reinterpret_cast<float *>(base + l.c);
-  s.red = reinterpret_cast<float *>(base + l.red);
-  s.red2 = reinterpret_cast<float *>(base + l.red2);
-  s.bits = reinterpret_cast<uint32_t *>(base + l.bits);
-  s.decided = reinterpret_cast<int *>(base + l.decided);
-  s.desc = reinterpret_cast<int4 *>(base + l.desc);
-  s.full = reinterpret_cast<uint64_t *>(base + l.bars);
-  s.empty = s.full + P.S;
-  s.xbar = s.empty + P.S;
-  s.sync = s.xbar + 1;
-  s.abort_flag = reinterpret_cast<int *>(s.sync + 1);
-  return s;
-}
-
-__device__ __forceinline__ bool aborted(const Smem &s) { return *reinterpret_cast<volatile int *>(s.abort_flag); }
-
-__device__ __forceinline__ void do_abort(const Smem &s, int32_t *err) {
-  *reinterpret_cast<volatile int *>(s.abort_flag) = 1;
-  latch_error(err, kErrTimeout);
-}
-
-// Bounded wait that also gives up as soon as another thread of the CTA aborted.
-__device__ __forceinline__ bool wait_bar(const Smem &s, uint64_t *bar, uint32_t parity) {
-  uint64_t t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63) {
-      if (aborted(s)) return false;
-      const uint64_t now = globaltimer_ns();
-      if (t0 == 0)
-        t0 = now;
-      else if (now - t0 > kWaitNs)
-        return false;
-    }
-  }
-}
-
-// All consumer warps meet (mbarrier with kCW arrivals, bounded).
-__device__ __forceinline__ bool consumers_sync(const Smem &s, uint32_t &phase, int32_t *err) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(s.sync);
-  const bool ok = wait_bar(s, s.sync, phase & 1u);
-  ++phase;
-  if (!ok) do_abort(s, err);
-  return ok;
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 template <typename T>
-__device__ __forceinline__ void load_vec_smem(const void *p, float *f) {
-  unpack<T>(*reinterpret_cast<const uint4 *>(p), f);
+__device__ __forceinline__ float dot_chunk(const uint4 &w, const float *h, float a) {
+  constexpr int V = Elem<T>::kVec;
+  float f[V];
+  unpack<T>(w, f);
+#pragma unroll
+  for (int v = 0; v < V; ++v) a = fmaf(f[v], h[v], a);
+  return a;
+}
+
+template <typename T>
+__device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  constexpr int V = Elem<T>::kVec;
+  float f[V], xf[V];
+  unpack<T>(w, f);
+  unpack<T>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 16), xf);
+#pragma unroll
+  for (int v = 0; v < V; ++v) a = fmaf(f[v], xf[v], a);
+  return a;
+}
+
+// Grid barrier by thread 0, bracketed by CTA barriers; false (and the error latched)
+// if it timed out.
+__device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = grid_barrier(P.bar, (uint32_t)P.G, kWaitCycles);
+    if (!ok) latch_error(P.err, kErrTimeout);
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
 template <typename T, int ACT, int MAXM>
-__global__ void __launch_bounds__(kThreads1, 1) k_decode1(const Decode1Params P) {
+__global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr int V = Elem<T>::kVec;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  const Smem s = carve(smem_raw, P);
+  constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Decode1Layout L = decode1_layout(P);
+  unsigned char *xs = smem + L.x;
+  float *bias_s = reinterpret_cast<float *>(smem + L.bias);
+  float *c_s = reinterpret_cast<float *>(smem + L.c);
+  int *act_s = reinterpret_cast<int *>(smem + L.act);
+  float *a_s = reinterpret_cast<float *>(smem + L.a);
+  float *dots = reinterpret_cast<float *>(smem + L.dots);
+  float *red2 = reinterpret_cast<float *>(smem + L.red2);
+  uint32_t *bits = reinterpret_cast<uint32_t *>(smem + L.bits);
+  int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
+  int *flag_s = cnt_s + 1;
+
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = P.G;
   const int t0 = decode1_tile_start(c, P.n, G);
   const int tn = decode1_tile_start(c + 1, P.n, G) - t0;
-  const int nchunks = (tn + P.NPC - 1) / P.NPC;
-  const int nproj = P.nproj, d = P.d, r = P.r;
+  const int d = P.d, r = P.r, nproj = P.nproj;
+  const int nch_d = d / V, nch_r = r / V;
+  const T *At = static_cast<const T *>(P.At);
+  const T *Bt = static_cast<const T *>(P.Bt);
   const T *rows = static_cast<const T *>(P.rows);
 
-  if (tid == 0) {
-    for (int i = 0; i < P.S; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kCW);
-    }
-    mbar_init(s.xbar, 1);
-    mbar_init(s.sync, kCW);
-    *s.abort_flag = 0;
-    fence_mbar_init();
-  }
-  for (int i = tid; i < (P.tile_max + 31) / 32; i += blockDim.x) s.bits[i] = 0u;
-  for (int i = tid; i < P.chunks_max; i += blockDim.x) s.decided[i] = 0;
-  __syncthreads();
   pdl_launch_dependents();
-
-  if (warp == kCW) {
-    // ------------------------------------------------------------ producer
-    if (lane != 0) return;
-    const T *Bt = static_cast<const T *>(P.Bt);
-    const uint32_t rec_bytes = (uint32_t)(nproj * d * sizeof(T));
-    int seq = 0, next_chunk = 0, dec = 0, cursor = 0;
-    int last_item_bytes[64];  // per slot: bytes of the last item issued there (for the abort drain)
-    for (int i = 0; i < P.S; ++i) last_item_bytes[i] = 0;
-    bool x_issued = false, ok = true;
-    uint64_t idle_since = 0;
-    while (ok) {
-      // the input vector, once the previous kernel's writes are visible
-      if (!x_issued && (next_chunk >= P.S || next_chunk >= nchunks)) {
-        pdl_wait();
-        mbar_arrive_expect_tx(s.xbar, (uint32_t)(d * sizeof(T)));
-        bulk_g2s(s.x, P.x, (uint32_t)(d * sizeof(T)), s.xbar);
-        x_issued = true;
-      }
-      while (dec < next_chunk && *reinterpret_cast<volatile int *>(&s.decided[dec]) == kCW) ++dec;
-      __threadfence_block();
-      const int decided_upto = min(tn, dec * P.NPC);
-      // next active neuron among the decided positions; every position below `cursor`
-      // is decided and scanned
-      int p = -1;
-      while (cursor < decided_upto) {
-        const uint32_t w = *reinterpret_cast<volatile uint32_t *>(&s.bits[cursor >> 5]) >> (cursor & 31);
-        if (w) {
-          const int q = cursor + __ffs(w) - 1;
-          if (q < decided_upto)
-            p = q;
-          else
-            cursor = decided_upto;
-          break;
-        }
-        cursor = min((cursor | 31) + 1, decided_upto);
-      }
-      int4 item;
-      uint32_t bytes = 0;
-      const void *src = nullptr;
-      if (p >= 0) {
-        item = make_int4(kItemRow, p, 1, 0);
-        bytes = rec_bytes;
-        src = rows + (size_t)(t0 + p) * nproj * d;
-        cursor = p + 1;
-      } else if (next_chunk < nchunks) {
-        const int p0 = next_chunk * P.NPC;
-        const int cnt = min(P.NPC, tn - p0);
-        item = make_int4(kItemBt, p0, cnt, next_chunk);
-        bytes = (uint32_t)(cnt * r * sizeof(T));
-        src = Bt + (size_t)(t0 + p0) * r;
-        ++next_chunk;
-      } else if (dec == nchunks && cursor >= decided_upto) {
-        item = make_int4(kItemEnd, 0, 0, 0);
-      } else {  // rows not decided yet: wait for the consumers
-        const uint64_t now = globaltimer_ns();
-        if (idle_since == 0) idle_since = now;
-        if (now - idle_since > kWaitNs || aborted(s)) {
-          ok = false;
-          break;
-        }
-        __nanosleep(32);
-        continue;
-      }
-      idle_since = 0;
-      const int slot = seq % P.S;
-      if (seq >= P.S && !wait_bar(s, &s.empty[slot], (uint32_t)((seq / P.S) - 1) & 1u)) {
-        ok = false;
-        break;
-      }
-      s.desc[slot] = item;
-      if (bytes) {
-        mbar_arrive_expect_tx(&s.full[slot], bytes);
-        bulk_g2s(s.ring + (size_t)slot * P.SB, src, bytes, &s.full[slot]);
-      } else {
-        mbar_arrive(&s.full[slot]);
-      }
-      last_item_bytes[slot] = (int)bytes;
-      ++seq;
-      if (item.x == kItemEnd) break;
+  if (warp == kW - 1) {  // the tile's B^T rows, into L2 while phase A runs
+    const size_t tile_bytes = (size_t)tn * r * sizeof(T);
+    const unsigned char *src = reinterpret_cast<const unsigned char *>(Bt + (size_t)t0 * r);
+    for (size_t o = (size_t)lane * 16384; o < tile_bytes; o += (size_t)32 * 16384)
+      prefetch_l2(src + o, (uint32_t)min((size_t)16384, tile_bytes - o));
+  }
+  {
+    const T *bp = static_cast<const T *>(P.bias);
+    const T *cp = static_cast<const T *>(P.cvec);
+    for (int i = tid; i < tn; i += kT) {
+      bias_s[i] = to_f<T>(bp[t0 + i]);
+      c_s[i] = to_f<T>(cp[t0 + i]);
     }
-    if (!x_issued) {  // keep the x barrier consistent even on the abort path
-      pdl_wait();
-      mbar_arrive_expect_tx(s.xbar, (uint32_t)(d * sizeof(T)));
-      bulk_g2s(s.x, P.x, (uint32_t)(d * sizeof(T)), s.xbar);
-    }
-    if (!ok) {
-      do_abort(s, P.err);
-      // let every copy in flight land before the CTA's shared memory is released
-      for (int k = seq - 1; k >= 0 && k >= seq - P.S; --k) {
-        const int slot = k % P.S;
-        if (last_item_bytes[slot]) mbar_wait(&s.full[slot], (uint32_t)(k / P.S) & 1u, kWaitNs);
-      }
-      mbar_wait(s.xbar, 0, kWaitNs);
-    }
-    return;
+    for (int i = tid; i < (P.tile_max + 31) / 32; i += kT) bits[i] = 0u;
   }
 
-  // -------------------------------------------------------------- consumers
-  uint32_t sync_phase = 0;
-  const T *At = static_cast<const T *>(P.At);
-  const T *biasp = static_cast<const T *>(P.bias);
-  const T *cp = static_cast<const T *>(P.cvec);
-  for (int i = tid; i < tn; i += kConsumers) {
-    s.bias[i] = to_f<T>(biasp[t0 + i]);
-    s.c[i] = to_f<T>(cp[t0 + i]);
+  // ---------------------------------------------------------------- A: hidden layer
+  const int j0 = c + G * warp;
+  uint4 w0[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int ch = lane + 32 * u;
+    if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
   }
-  // P1: predictor hidden layer, rows j = c + G*(warp + kCW*k).  The weight loads are
-  // issued before waiting for x.
-  const int nch_d = d / V;
-  bool ok = true, x_ready = false;
-  for (int j = c + G * warp; ok && j < r; j += G * kCW) {
+  pdl_wait();  // x (and every buffer this kernel writes) belongs to earlier kernels until here
+  for (int i = tid; i < nch_d; i += kT)
+    *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
+        __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+  __syncthreads();
+  for (int j = j0; j < r; j += G * kW) {
     const T *row = At + (size_t)j * d;
-    float acc = 0.f;
+    float acc = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
     for (int cb = 0; cb < nch_d; cb += 32 * 16) {
-      uint4 w[16];
+      if (j != j0 || cb != 0) {  // the first batch of the first row is already in w0
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int ch = cb + lane + 32 * u;
-        if (ch < nch_d) w[u] = ld_stream(row + (size_t)ch * V);
-      }
-      if (!x_ready) {
-        ok = wait_bar(s, s.xbar, 0);
-        x_ready = true;
-        if (!ok) {
-          do_abort(s, P.err);
-          break;
+        for (int u = 0; u < 16; ++u) {
+          const int ch = cb + lane + 32 * u;
+          if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
         }
       }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int ch = cb + lane + 32 * u;
-        if (ch < nch_d) {
-          float wf[V], xf[V];
-          unpack<T>(w[u], wf);
-          load_vec_smem<T>(s.x + (size_t)ch * 16, xf);
-#pragma unroll
-          for (int v = 0; v < V; ++v) acc = fmaf(wf[v], xf[v], acc);
-        }
+        if (ch < nch_d) acc = dot_chunk_smem<T>(w0[u], xs, ch, acc);
       }
     }
-    if (!ok) break;
     const float hs = warp_sum(acc);
     if (lane == 0) P.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
   }
-  if (ok && !x_ready) {
-    ok = wait_bar(s, s.xbar, 0);
-    if (!ok) do_abort(s, P.err);
-  }
-  __threadfence();
-  ok = ok && consumers_sync(s, sync_phase, P.err);
-  if (ok && tid == 0 && !grid_barrier(P.bar, (uint32_t)G, kWaitNs)) do_abort(s, P.err);
-  ok = ok && consumers_sync(s, sync_phase, P.err) && !aborted(s);
-  for (int i = tid; ok && i < r; i += kConsumers) s.h[i] = __ldcg(P.hbuf + i);
-  ok = ok && consumers_sync(s, sync_phase, P.err);
+  if (!cta_grid_sync(P, flag_s)) return;
 
-  // P2 + P3: the stage loop
+  // ---------------------------------------------------------------- B: logits + threshold
+  {
+    float hreg[MAXH][V];
+#pragma unroll
+    for (int m = 0; m < MAXH; ++m) {
+      const int ch = lane + 32 * m;
+#pragma unroll
+      for (int v = 0; v < V; v += 4) {
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ch < nch_r) q = __ldcg(reinterpret_cast<const float4 *>(P.hbuf + (size_t)ch * V + v));
+        hreg[m][v] = q.x;
+        hreg[m][v + 1] = q.y;
+        hreg[m][v + 2] = q.z;
+        hreg[m][v + 3] = q.w;
+      }
+    }
+    constexpr int D = 3;
+    uint4 wb[D][MAXH];
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+      const int p = warp + kW * s;
+#pragma unroll
+      for (int m = 0; m < MAXH; ++m) {
+        const int ch = lane + 32 * m;
+        if (p < tn && ch < nch_r) wb[s][m] = ld_stream(Bt + (size_t)(t0 + p) * r + (size_t)ch * V);
+      }
+    }
+    for (int pb = warp; pb < tn; pb += D * kW) {
+#pragma unroll
+      for (int s = 0; s < D; ++s) {
+        const int p = pb + kW * s;
+        if (p < tn) {
+          float a = 0.f;
+#pragma unroll
+          for (int m = 0; m < MAXH; ++m)
+            if (lane + 32 * m < nch_r) a = dot_chunk<T>(wb[s][m], hreg[m], a);
+          const int pn = p + D * kW;
+#pragma unroll
+          for (int m = 0; m < MAXH; ++m) {
+            const int ch = lane + 32 * m;
+            if (pn < tn && ch < nch_r) wb[s][m] = ld_stream(Bt + (size_t)(t0 + pn) * r + (size_t)ch * V);
+          }
+          const float z = warp_sum(a) + c_s[p];
+          if (lane == 0 && z > 0.f) atomicOr(&bits[p >> 5], 1u << (p & 31));  // NaN -> inactive
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // the tile's active positions, ascending
+    const int nwords = (tn + 31) / 32;
+    int base = 0;
+    for (int wi = 0; wi < nwords; wi += 32) {
+      const uint32_t word = wi + lane < nwords ? bits[wi + lane] : 0u;
+      const int k = __popc(word);
+      int incl = k;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - k;
+      uint32_t m = word;
+      while (m) {
+        act_s[pos++] = (wi + lane) * 32 + __ffs(m) - 1;
+        m &= m - 1u;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *cnt_s = base;
+  }
+  __syncthreads();
+  const int cnt = *cnt_s;
+
+  // ---------------------------------------------------------------- C1: up / gate dots
+  {
+    constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
+    constexpr int D = 2;
+    constexpr int SU = kSegChunks / 32;  // chunks per lane and segment
+    const int nseg = P.nseg;
+    const int per_row = NPG * nseg;
+    const int items = cnt * per_row;
+    uint4 wc[D][SU];
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+      const int it = warp + kW * s;
+      if (it < items) {
+        const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+        const T *row = rows + ((size_t)(t0 + act_s[k]) * nproj + pj) * d;
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int ch = sg * kSegChunks + lane + 32 * u;
+          if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * V);
+        }
+      }
+    }
+    for (int ib = warp; ib < items; ib += D * kW) {
+#pragma unroll
+      for (int s = 0; s < D; ++s) {
+        const int it = ib + kW * s;
+        if (it < items) {
+          const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+          float a = 0.f;
+#pragma unroll
+          for (int u = 0; u < SU; ++u) {
+            const int ch = sg * kSegChunks + lane + 32 * u;
+            if (ch < nch_d) a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
+          }
+          const int itn = it + D * kW;
+          if (itn < items) {
+            const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
+            const T *row = rows + ((size_t)(t0 + act_s[kn]) * nproj + pjn) * d;
+#pragma unroll
+            for (int u = 0; u < SU; ++u) {
+              const int ch = sgn * kSegChunks + lane + 32 * u;
+              if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * V);
+            }
+          }
+          a = warp_sum(a);
+          if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+        }
+      }
+    }
+    __syncthreads();
+    for (int k = tid; k < cnt; k += kT) {
+      float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
+      for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
+      if (ACT == SFNN_REGLU)
+        for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
+      const float pre = g + bias_s[act_s[k]];
+      const float relu = pre > 0.f ? pre : 0.f;
+      a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
+    }
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- C2: down projection
   float acc[MAXM][V];
 #pragma unroll
   for (int m = 0; m < MAXM; ++m)
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
-  const int nch_r = r / V;
-  int buf = 0;
-  for (int seq = 0; ok; ++seq) {
-    const int slot = seq % P.S;
-    if (!wait_bar(s, &s.full[slot], (uint32_t)(seq / P.S) & 1u)) {
-      do_abort(s, P.err);
-      ok = false;
-      break;
-    }
-    const int4 item = s.desc[slot];
-    if (item.x == kItemEnd) break;
-    const unsigned char *st = s.ring + (size_t)slot * P.SB;
-    if (item.x == kItemBt) {
-      for (int k = warp; k < item.z; k += kCW) {
-        const unsigned char *brow = st + (size_t)k * r * sizeof(T);
-        float a = 0.f;
-#pragma unroll 4
-        for (int ch = lane; ch < nch_r; ch += 32) {
-          float wf[V];
-          load_vec_smem<T>(brow + (size_t)ch * 16, wf);
-          const float *hp = s.h + (size_t)ch * V;
+  {
+    constexpr int D = 4;
+    uint4 wd[D][MAXM];
 #pragma unroll
-          for (int v = 0; v < V; ++v) a = fmaf(wf[v], hp[v], a);
-        }
-        const int p = item.y + k;
-        const float z = warp_sum(a) + s.c[p];
-        if (lane == 0 && z > 0.f) atomicOr(&s.bits[p >> 5], 1u << (p & 31));  // NaN -> inactive
-      }
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        atomicAdd(&s.decided[item.w], 1);
-        mbar_arrive(&s.empty[slot]);
-      }
-      continue;
-    }
-    // a row record: [gate | up | down]
-    const unsigned char *gate = st;
-    const unsigned char *up = st + (ACT == SFNN_REGLU ? (size_t)d * sizeof(T) : 0);
-    const unsigned char *down = st + (size_t)(nproj - 1) * d * sizeof(T);
-    float su = 0.f, sg = 0.f;
+    for (int s = 0; s < D; ++s) {
+      if (s < cnt) {
+        const T *row = rows + ((size_t)(t0 + act_s[s]) * nproj + (nproj - 1)) * d;
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const int ch = tid + kConsumers * m;
-      if (ch < nch_d) {
-        float xf[V], wu[V];
-        load_vec_smem<T>(s.x + (size_t)ch * 16, xf);
-        load_vec_smem<T>(up + (size_t)ch * 16, wu);
-#pragma unroll
-        for (int v = 0; v < V; ++v) su = fmaf(wu[v], xf[v], su);
-        if (ACT == SFNN_REGLU) {
-          float wg[V];
-          load_vec_smem<T>(gate + (size_t)ch * 16, wg);
-#pragma unroll
-          for (int v = 0; v < V; ++v) sg = fmaf(wg[v], xf[v], sg);
+        for (int m = 0; m < MAXM; ++m) {
+          const int ch = tid + kT * m;
+          if (ch < nch_d) wd[s][m] = ld_stream(row + (size_t)ch * V);
         }
       }
     }
-    su = warp_sum(su);
-    if (ACT == SFNN_REGLU) sg = warp_sum(sg);
-    if (lane == 0) {
-      s.red[(buf * kCW + warp) * 2 + 0] = su;
-      s.red[(buf * kCW + warp) * 2 + 1] = sg;
-    }
-    if (!consumers_sync(s, sync_phase, P.err)) {
-      ok = false;
-      break;
-    }
-    float tu = 0.f, tg = 0.f;
+    for (int kb = 0; kb < cnt; kb += D) {
 #pragma unroll
-    for (int w = 0; w < kCW; ++w) {
-      tu += s.red[(buf * kCW + w) * 2 + 0];
-      tg += s.red[(buf * kCW + w) * 2 + 1];
-    }
-    const float bval = s.bias[item.y];
-    float a;
-    if (ACT == SFNN_RELU) {
-      const float g = tu + bval;
-      a = g > 0.f ? g : 0.f;
-    } else {
-      const float g = tg + bval;
-      a = (g > 0.f ? g : 0.f) * tu;
-    }
+      for (int s = 0; s < D; ++s) {
+        const int k = kb + s;
+        if (k < cnt) {
+          const float a = a_s[k];
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const int ch = tid + kConsumers * m;
-      if (ch < nch_d) {
-        float wd[V];
-        load_vec_smem<T>(down + (size_t)ch * 16, wd);
+          for (int m = 0; m < MAXM; ++m) {
+            if (tid + kT * m < nch_d) {
+              float f[V];
+              unpack<T>(wd[s][m], f);
 #pragma unroll
-        for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, wd[v], acc[m][v]);
+              for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, f[v], acc[m][v]);
+            }
+          }
+          if (k + D < cnt) {
+            const T *row = rows + ((size_t)(t0 + act_s[k + D]) * nproj + (nproj - 1)) * d;
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) {
+              const int ch = tid + kT * m;
+              if (ch < nch_d) wd[s][m] = ld_stream(row + (size_t)ch * V);
+            }
+          }
+        }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s.empty[slot]);
-    buf ^= 1;
   }
 
-  // P4: the CTA's partial, then the fixed-order column sums of all partials
+  // ---------------------------------------------------------------- D: partials, final sum
 #pragma unroll
   for (int m = 0; m < MAXM; ++m) {
-    const int ch = tid + kConsumers * m;
+    const int ch = tid + kT * m;
     if (ch < nch_d) {
       float4 *dst = reinterpret_cast<float4 *>(P.part + (size_t)c * d + (size_t)ch * V);
 #pragma unroll
       for (int v = 0; v < V; v += 4) dst[v / 4] = make_float4(acc[m][v], acc[m][v + 1], acc[m][v + 2], acc[m][v + 3]);
     }
   }
-  __threadfence();
-  ok = ok && consumers_sync(s, sync_phase, P.err);
-  if (ok && tid == 0 && !grid_barrier(P.bar, (uint32_t)G, kWaitNs)) do_abort(s, P.err);
-  ok = ok && consumers_sync(s, sync_phase, P.err) && !aborted(s);
-  if (!ok) return;
+  if (!cta_grid_sync(P, flag_s)) return;
   const int CW = (d + G - 1) / G;
   const int col0 = c * CW;
   const int ncol = max(0, min(CW, d - col0));
-  for (int cb = 0; cb < ncol; cb += kConsumers) {
-    const int width = min(kConsumers, ncol - cb);
+  for (int cb = 0; cb < ncol; cb += kT) {
+    const int width = min(kT, ncol - cb);
     const int gi = tid / width, j = tid % width;
-    const int ngu = kConsumers / width;  // groups of partials summed in parallel
+    const int ngu = kT / width;  // groups of partials summed in parallel
     if (gi < ngu) {
       const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
       const float *src = P.part + col0 + cb + j;
       float sum = 0.f;
       for (int k = k0; k < k1; ++k) sum += __ldcg(src + (size_t)k * d);
-      s.red2[gi * width + j] = sum;
+      red2[gi * width + j] = sum;
     }
-    if (!consumers_sync(s, sync_phase, P.err)) return;
+    __syncthreads();
     if (tid < width) {
       float tot = 0.f;
-      for (int g = 0; g < ngu; ++g) tot += s.red2[g * width + tid];
+      for (int g = 0; g < ngu; ++g) tot += red2[g * width + tid];
       const int col = col0 + cb + tid;
       if (P.resid) tot = P.resid[col] + tot;
       P.y[col] = tot;
       if (P.xnext) static_cast<T *>(P.xnext)[col] = from_f<T>(tot);
     }
-    if (!consumers_sync(s, sync_phase, P.err)) return;
+    __syncthreads();
   }
 }
+
+__global__ void k_barrier_bump(uint64_t *count) { atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull); }
 
 template <typename T, int ACT, int MAXM>
 cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.G);
-  cfg.blockDim = dim3(kThreads1);
+  cfg.blockDim = dim3(kT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -462,48 +402,59 @@ cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, b
 }
 
 template <typename T, int ACT>
-cudaError_t launch_act(const Decode1Params &P, size_t smem, cudaStream_t stream, bool pdl) {
-  const int nch = P.d / Elem<T>::kVec;
-  if (nch <= kConsumers * 4) return launch_t<T, ACT, 4>(P, smem, stream, pdl);
-  return launch_t<T, ACT, 8>(P, smem, stream, pdl);
+const void *pick_kernel(int nch) {
+  if (nch <= kT) return (const void *)k_decode1<T, ACT, 1>;
+  if (nch <= 2 * kT) return (const void *)k_decode1<T, ACT, 2>;
+  return (const void *)k_decode1<T, ACT, 4>;
 }
 
-template <typename T, int ACT, int MAXM>
-cudaError_t config_t() {
-  return cudaFuncSetAttribute((const void *)k_decode1<T, ACT, MAXM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kDecode1SmemMax);
+template <typename T, int ACT>
+cudaError_t launch_act(const Decode1Params &P, size_t smem, cudaStream_t stream, bool pdl) {
+  const int nch = P.d / Elem<T>::kVec;
+  if (nch <= kT) return launch_t<T, ACT, 1>(P, smem, stream, pdl);
+  if (nch <= 2 * kT) return launch_t<T, ACT, 2>(P, smem, stream, pdl);
+  return launch_t<T, ACT, 4>(P, smem, stream, pdl);
+}
+
+template <typename T, int ACT>
+cudaError_t config_act() {
+  const void *ks[] = {(const void *)k_decode1<T, ACT, 1>, (const void *)k_decode1<T, ACT, 2>,
+                      (const void *)k_decode1<T, ACT, 4>};
+  for (const void *k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t configure_decode1() {
-  cudaError_t e = config_t<float, SFNN_RELU, 4>();
-  if (e == cudaSuccess) e = config_t<float, SFNN_RELU, 8>();
-  if (e == cudaSuccess) e = config_t<float, SFNN_REGLU, 4>();
-  if (e == cudaSuccess) e = config_t<float, SFNN_REGLU, 8>();
-  if (e == cudaSuccess) e = config_t<__half, SFNN_RELU, 4>();
-  if (e == cudaSuccess) e = config_t<__half, SFNN_RELU, 8>();
-  if (e == cudaSuccess) e = config_t<__half, SFNN_REGLU, 4>();
-  if (e == cudaSuccess) e = config_t<__half, SFNN_REGLU, 8>();
+  cudaError_t e = config_act<float, SFNN_RELU>();
+  if (e == cudaSuccess) e = config_act<float, SFNN_REGLU>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU>();
   return e;
 }
 
-int decode1_threads() { return kThreads1; }
-
 int decode1_blocks_per_sm(const Decode1Params &P) {
   const size_t smem = decode1_layout(P).total;
+  if (smem > (size_t)kSmemCap) return 0;
   const int nch = P.d / (P.dt == SFNN_F16 ? 8 : 4);
-  const bool m8 = nch > kConsumers * 4;
+  if (nch > 4 * kT) return 0;  // beyond the kernel's register plan
   const void *k;
   if (P.dt == SFNN_F16)
-    k = P.act == SFNN_REGLU ? (m8 ? (const void *)k_decode1<__half, SFNN_REGLU, 8> : (const void *)k_decode1<__half, SFNN_REGLU, 4>)
-                            : (m8 ? (const void *)k_decode1<__half, SFNN_RELU, 8> : (const void *)k_decode1<__half, SFNN_RELU, 4>);
+    k = P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU>(nch) : pick_kernel<__half, SFNN_RELU>(nch);
   else
-    k = P.act == SFNN_REGLU ? (m8 ? (const void *)k_decode1<float, SFNN_REGLU, 8> : (const void *)k_decode1<float, SFNN_REGLU, 4>)
-                            : (m8 ? (const void *)k_decode1<float, SFNN_RELU, 8> : (const void *)k_decode1<float, SFNN_RELU, 4>);
+    k = P.act == SFNN_REGLU ? pick_kernel<float, SFNN_REGLU>(nch) : pick_kernel<float, SFNN_RELU>(nch);
   int blocks = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, kThreads1, smem) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, kT, smem) != cudaSuccess) return 0;
   return blocks;
+}
+
+cudaError_t launch_barrier_bump(uint64_t *count, cudaStream_t stream) {
+  k_barrier_bump<<<1, 1, 0, stream>>>(count);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl) {

@@ -8,7 +8,7 @@
 
 namespace sfnn {
 
-constexpr int kDecode1SmemMax = 227 * 1024;  // opt-in dynamic shared memory per CTA on sm_100
+constexpr int kDecode1Threads = 512;  // 16 warps per CTA, one CTA per SM
 
 struct Decode1Params {
   const void *At, *Bt, *cvec, *bias, *rows;  // re-laid-out weights
@@ -18,44 +18,43 @@ struct Decode1Params {
   void *xnext;                               // [d] or null: round(y) in wdtype
   float *hbuf;                               // [r] predictor hidden layer (scratch)
   float *part;                               // [G][d] per-CTA partial sums (scratch)
-  uint32_t *bar;                             // [2] grid barrier state (scratch, zeroed at create)
+  uint64_t *bar;                             // grid barrier arrival counter (scratch, zeroed at create)
   int32_t *err;                              // latched device error
   int d, n, r, nproj, act, dt;
-  int G;           // CTAs (one per SM) = tiles of neurons
-  int S, SB, NPC;  // ring stages, bytes per stage, neurons of B^T per stage
-  int tile_max, chunks_max;
+  int G;         // CTAs (one per SM) = tiles of neurons
+  int tile_max;  // largest tile
+  int nseg;      // 4 KB segments of one projection row (C1 work items per row and projection)
 };
 
 struct Decode1Layout {
-  size_t x, h, bias, c, red, red2, bits, decided, desc, bars, total;
+  size_t x, bias, c, act, a, dots, red2, bits, bars, total;
 };
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) {
   const size_t esz = P.dt == SFNN_F16 ? 2 : 4;
+  const size_t tm = (size_t)P.tile_max;
   Decode1Layout L;
-  size_t o = (size_t)P.S * P.SB;
+  size_t o = 0;
   L.x = o;
   o = decode1_align(o + (size_t)P.d * esz, 16);
-  L.h = o;
-  o = decode1_align(o + (size_t)P.r * 4, 16);
   L.bias = o;
-  o = decode1_align(o + (size_t)P.tile_max * 4, 16);
+  o = decode1_align(o + tm * 4, 16);
   L.c = o;
-  o = decode1_align(o + (size_t)P.tile_max * 4, 16);
-  L.red = o;
-  o = decode1_align(o + 2 * 8 * 2 * 4, 16);
+  o = decode1_align(o + tm * 4, 16);
+  L.act = o;  // active positions of the tile, ascending
+  o = decode1_align(o + tm * 4, 16);
+  L.a = o;  // their activations
+  o = decode1_align(o + tm * 4, 16);
+  L.dots = o;  // segment partials of the up (and gate) dot products
+  o = decode1_align(o + tm * 2 * (size_t)P.nseg * 4, 16);
   L.red2 = o;
-  o = decode1_align(o + 256 * 4, 16);
+  o = decode1_align(o + (size_t)kDecode1Threads * 4, 16);
   L.bits = o;
-  o = decode1_align(o + (size_t)((P.tile_max + 31) / 32) * 4, 16);
-  L.decided = o;
-  o = decode1_align(o + (size_t)P.chunks_max * 4, 16);
-  L.desc = o;
-  o = decode1_align(o + (size_t)P.S * 16, 16);
-  L.bars = o;
-  o = decode1_align(o + (size_t)(2 * P.S + 2) * 8 + 8, 16);
+  o = decode1_align(o + ((tm + 31) / 32) * 4 + 16, 16);
+  L.bars = o;  // one mbarrier-free word: the active count
+  o = decode1_align(o + 16, 16);
   L.total = o;
   return L;
 }
@@ -67,8 +66,8 @@ __host__ __device__ inline int decode1_tile_start(int c, int n, int G) {
 }
 
 cudaError_t configure_decode1();
-int decode1_threads();
 int decode1_blocks_per_sm(const Decode1Params &P);  // co-resident CTAs per SM for this plan
 cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl);
+cudaError_t launch_barrier_bump(uint64_t *count, cudaStream_t stream);
 
 }  // namespace sfnn

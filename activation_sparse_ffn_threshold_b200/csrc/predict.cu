@@ -101,9 +101,19 @@ __global__ void __launch_bounds__(kThreads) k_logits(const T *__restrict__ Bt, c
 #pragma unroll
           for (int t = 0; t < TB; ++t) {
             if (t0 + t < b) {
-              const float *hp = hs + (size_t)(t0 + t) * r + (size_t)c * V;
+              // two 16-byte reads per chunk instead of V scalar ones (fewer bank conflicts)
+              const float4 *hp4 = reinterpret_cast<const float4 *>(hs + (size_t)(t0 + t) * r + (size_t)c * V);
+              float hv[V];
 #pragma unroll
-              for (int v = 0; v < V; ++v) acc[t] = fmaf(wf[v], hp[v], acc[t]);
+              for (int q = 0; q < V / 4; ++q) {
+                const float4 f = hp4[q];
+                hv[4 * q] = f.x;
+                hv[4 * q + 1] = f.y;
+                hv[4 * q + 2] = f.z;
+                hv[4 * q + 3] = f.w;
+              }
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[t] = fmaf(wf[v], hv[v], acc[t]);
             }
           }
         }

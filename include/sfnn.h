@@ -31,6 +31,8 @@
  *    and its scratch memory.
  *  - Element type: x / X and all weights use the handle's wdtype (IEEE fp32
  *    or fp16); outputs y / Y are fp32; index lists and counts are int32.
+ *    x / X must start on a 16-byte boundary (SFNN_ERR_INVALID_ARG otherwise):
+ *    they are read with 16-byte vector loads and bulk async copies.
  *  - Every call after sfnn_create is asynchronous on `stream` and never
  *    synchronises the host, never aborts and never throws.  Argument errors
  *    are returned at once and launch nothing.  Errors found on the device

@@ -194,3 +194,19 @@ def test_reduced_batch_rows_match_single(act):
             check_token(lay, X[t], Y[t], m, f"b={b} t={t}")
             ys = h.forward(dev(X[t])).cpu().numpy()
             assert oracle.within_tolerance(Y[t], ys.astype(np.float64))[0]
+
+
+def test_misaligned_input_is_rejected(small_layer):
+    cfg, lay = small_layer
+    h = sf.SparseFFN.from_layer(lay, max_batch=2)
+    buf = torch.zeros(cfg.d + 8, dtype=torch.float16, device="cuda")
+    x_bad = buf[1:1 + cfg.d]  # 2-byte offset
+    with pytest.raises(sf.SfnnError) as e:
+        h.forward(x_bad)
+    assert e.value.status == 1
+    with pytest.raises(sf.SfnnError):
+        h.predict(x_bad)
+    X = torch.zeros(2 * cfg.d + 8, dtype=torch.float16, device="cuda")[4:4 + 2 * cfg.d].view(2, cfg.d)
+    with pytest.raises(sf.SfnnError):
+        h.forward_batch(X)
+    assert h.get_error() == 0
