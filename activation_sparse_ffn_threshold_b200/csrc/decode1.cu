@@ -11,17 +11,19 @@
 //   hottest first inside the tile.
 //
 //   A   h_j = relu(A^T[j] . x): one warp per predictor row, every chunk of the row
-//       requested at once (the first row before waiting for the previous kernel);
-//       meanwhile one warp asks L2 to prefetch the CTA's tile of B^T.  h goes to
-//       global memory; grid barrier.
+//       requested at once (the first row before waiting for the previous kernel).
+//       h goes to global memory; grid barrier.
 //   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron with a 3-deep
 //       register pipeline over the warp's neurons; neuron i is active iff z_i > 0
-//       (sigmoid(z) > 0.5).  The tile's active positions are compacted in order.
-//   C1  up (and gate) dot products of the active rows, split in 4 KB segments spread
+//       (sigmoid(z) > 0.5).  The tile's active positions, compacted in order, and
+//       their count are published; grid barrier.  Every CTA then takes an equal slice
+//       of the concatenated active list (tile order, so the same set always gives the
+//       same slices): the row work is balanced whatever each tile drew.
+//   C1  up (and gate) dot products of the slice's rows, split in 4 KB segments spread
 //       over all warps (2-deep pipeline); segment sums added in a fixed order, then
 //       ReLU / ReGLU.  Rows of inactive neurons are never requested.
-//   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
-//       column accumulators, 4 rows in flight.
+//   C2  the slice's rows of W_down (neuron-major, contiguous) are added into
+//       per-thread column accumulators, 8 rows in flight.
 //   D   the CTA's partial y goes to global memory; grid barrier; CTA c sums a column
 //       slice of all G partials in a fixed order (two-phase, deterministic) -> y
 //       (+ residual, + rounded next-layer input).
@@ -30,7 +32,7 @@
 // takes 16-byte chunks l, l+32, ... into one accumulator, then a butterfly sum), so
 // both paths decide every neuron identically.  PDL: the kernel lets the next one
 // launch at once and reads x, and writes anything, only after griddepcontrol.wait.
-// The two grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT
+// The three grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT
 // and returns without a result.
 #include "async.cuh"
 #include "common.cuh"
@@ -72,10 +74,11 @@ __device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned c
 // Grid barrier by thread 0, bracketed by CTA barriers; false (and the error latched)
 // if it timed out.
 __device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag) {
-  __threadfence();
-  __syncthreads();
+  __syncthreads();  // the CTA's writes happen before thread 0's fence and release
   if (threadIdx.x == 0) {
+    __threadfence();
     const bool ok = grid_barrier(P.bar, (uint32_t)P.G, kWaitCycles);
+    __threadfence();
     if (!ok) latch_error(P.err, kErrTimeout);
     *flag = ok ? 1 : 0;
   }
@@ -96,6 +99,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   float *a_s = reinterpret_cast<float *>(smem + L.a);
   float *dots = reinterpret_cast<float *>(smem + L.dots);
   float *red2 = reinterpret_cast<float *>(smem + L.red2);
+  int *pref = reinterpret_cast<int *>(smem + L.pref);
   uint32_t *bits = reinterpret_cast<uint32_t *>(smem + L.bits);
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
@@ -111,19 +115,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const T *rows = static_cast<const T *>(P.rows);
 
   pdl_launch_dependents();
-  if (warp == kW - 1) {  // the tile's B^T rows, into L2 while phase A runs
-    const size_t tile_bytes = (size_t)tn * r * sizeof(T);
-    const unsigned char *src = reinterpret_cast<const unsigned char *>(Bt + (size_t)t0 * r);
-    for (size_t o = (size_t)lane * 16384; o < tile_bytes; o += (size_t)32 * 16384)
-      prefetch_l2(src + o, (uint32_t)min((size_t)16384, tile_bytes - o));
-  }
   {
-    const T *bp = static_cast<const T *>(P.bias);
     const T *cp = static_cast<const T *>(P.cvec);
-    for (int i = tid; i < tn; i += kT) {
-      bias_s[i] = to_f<T>(bp[t0 + i]);
-      c_s[i] = to_f<T>(cp[t0 + i]);
-    }
+    for (int i = tid; i < tn; i += kT) c_s[i] = to_f<T>(cp[t0 + i]);
     for (int i = tid; i < (P.tile_max + 31) / 32; i += kT) bits[i] = 0u;
   }
 
@@ -234,7 +228,50 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     if (lane == 0) *cnt_s = base;
   }
   __syncthreads();
-  const int cnt = *cnt_s;
+  {  // publish the tile's active positions (global numbering) and their count
+    const int tc = *cnt_s;
+    for (int k = tid; k < tc; k += kT) P.gact[(size_t)c * P.tile_max + k] = t0 + act_s[k];
+    if (tid == 0) P.gcnt[c] = tc;
+  }
+  if (!cta_grid_sync(P, flag_s)) return;
+  if (warp == 0) {  // exclusive prefix of the tiles' counts
+    int base = 0;
+    for (int i0 = 0; i0 < G; i0 += 32) {
+      const int v = i0 + lane < G ? __ldcg(P.gcnt + i0 + lane) : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i0 + lane < G) pref[i0 + lane] = base + incl - v;
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) pref[G] = base;
+  }
+  __syncthreads();
+  // this CTA's slice [lo, hi) of the concatenated active list
+  const int K = pref[G];
+  const int lo = (int)(((int64_t)c * K) / G), hi = (int)(((int64_t)(c + 1) * K) / G);
+  const int cnt = hi - lo;
+  {
+    const T *bp = static_cast<const T *>(P.bias);
+    for (int k = tid; k < cnt; k += kT) {
+      const int g = lo + k;
+      int a = 0, b = G - 1;  // the tile holding g: pref[a] <= g < pref[a + 1]
+      while (a < b) {
+        const int mid = (a + b + 1) >> 1;
+        if (pref[mid] <= g)
+          a = mid;
+        else
+          b = mid - 1;
+      }
+      const int pos = __ldcg(P.gact + (size_t)a * P.tile_max + (g - pref[a]));
+      act_s[k] = pos;
+      bias_s[k] = to_f<T>(bp[pos]);
+    }
+  }
+  __syncthreads();
 
   // ---------------------------------------------------------------- C1: up / gate dots
   {
@@ -250,7 +287,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       const int it = warp + kW * s;
       if (it < items) {
         const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
-        const T *row = rows + ((size_t)(t0 + act_s[k]) * nproj + pj) * d;
+        const T *row = rows + ((size_t)act_s[k] * nproj + pj) * d;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
           const int ch = sg * kSegChunks + lane + 32 * u;
@@ -273,7 +310,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
           const int itn = it + D * kW;
           if (itn < items) {
             const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
-            const T *row = rows + ((size_t)(t0 + act_s[kn]) * nproj + pjn) * d;
+            const T *row = rows + ((size_t)act_s[kn] * nproj + pjn) * d;
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
               const int ch = sgn * kSegChunks + lane + 32 * u;
@@ -291,7 +328,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
       if (ACT == SFNN_REGLU)
         for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
-      const float pre = g + bias_s[act_s[k]];
+      const float pre = g + bias_s[k];
       const float relu = pre > 0.f ? pre : 0.f;
       a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
     }
@@ -305,12 +342,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
   {
-    constexpr int D = 4;
+    constexpr int D = MAXM == 1 ? 8 : (MAXM == 2 ? 4 : 2);
     uint4 wd[D][MAXM];
 #pragma unroll
     for (int s = 0; s < D; ++s) {
       if (s < cnt) {
-        const T *row = rows + ((size_t)(t0 + act_s[s]) * nproj + (nproj - 1)) * d;
+        const T *row = rows + ((size_t)act_s[s] * nproj + (nproj - 1)) * d;
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
           const int ch = tid + kT * m;
@@ -334,7 +371,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
             }
           }
           if (k + D < cnt) {
-            const T *row = rows + ((size_t)(t0 + act_s[k + D]) * nproj + (nproj - 1)) * d;
+            const T *row = rows + ((size_t)act_s[k + D] * nproj + (nproj - 1)) * d;
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) {
               const int ch = tid + kT * m;

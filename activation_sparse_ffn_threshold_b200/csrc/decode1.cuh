@@ -19,6 +19,8 @@ struct Decode1Params {
   float *hbuf;                               // [r] predictor hidden layer (scratch)
   float *part;                               // [G][d] per-CTA partial sums (scratch)
   uint64_t *bar;                             // grid barrier arrival counter (scratch, zeroed at create)
+  int32_t *gact;                             // [G][tile_max] active positions of each tile (scratch)
+  int32_t *gcnt;                             // [G] their counts (scratch)
   int32_t *err;                              // latched device error
   int d, n, r, nproj, act, dt;
   int G;         // CTAs (one per SM) = tiles of neurons
@@ -27,7 +29,7 @@ struct Decode1Params {
 };
 
 struct Decode1Layout {
-  size_t x, bias, c, act, a, dots, red2, bits, bars, total;
+  size_t x, bias, c, act, a, dots, red2, pref, bits, bars, total;
 };
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -51,6 +53,8 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) 
   o = decode1_align(o + tm * 2 * (size_t)P.nseg * 4, 16);
   L.red2 = o;
   o = decode1_align(o + (size_t)kDecode1Threads * 4, 16);
+  L.pref = o;  // exclusive prefix of the tiles' active counts (G + 1)
+  o = decode1_align(o + ((size_t)P.G + 1) * 4, 16);
   L.bits = o;
   o = decode1_align(o + ((tm + 31) / 32) * 4 + 16, 16);
   L.bars = o;  // one mbarrier-free word: the active count
