@@ -19,7 +19,8 @@ import os
 import numpy as np
 import torch
 
-__all__ = ["SparseFFN", "SfnnError", "forward_stack", "hotness_order", "library_path", "load_library",
+__all__ = ["SparseFFN", "SfnnError", "forward_stack", "predict_noalloc", "hotness_order", "library_path",
+           "load_library",
            "RELU", "REGLU", "F32", "F16", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
 
 RELU, REGLU = 0, 1
@@ -86,6 +87,7 @@ def load_library():
         "sfnn_get_error": ([P], S),
         "sfnn_status_str": ([S], ctypes.c_char_p),
         "sfnn_hotness_order": ([ctypes.POINTER(ctypes.c_float), I, ctypes.POINTER(ctypes.c_int32)], S),
+        "sfnn_predict_noalloc": ([P, P, P, P, I, I, I, I, P, P, P], S),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -268,6 +270,29 @@ class SparseFFN:
             self.close()
         except Exception:
             pass
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024
+
+
+def predict_noalloc(x, A, B, c, idx=None, count=None, stream=None):
+    """The predicted set of one token without a handle or any allocation in the library.
+
+    For callers that cannot allocate device memory (see sfnn_predict_noalloc in
+    include/sfnn.h).  x [d], A [d, r], B [r, n], c [n]: CUDA tensors of one dtype;
+    returns (idx [n] int32, count [1] int32), idx[:count] ascending.
+    """
+    lib = load_library()
+    d, r = A.shape
+    n = B.shape[1]
+    for t in (x, A, B, c):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or not t.is_contiguous() or t.dtype != A.dtype:
+            raise TypeError("x, A, B, c must be contiguous CUDA tensors of one dtype")
+    idx = idx if idx is not None else torch.empty(n, dtype=torch.int32, device=A.device)
+    count = count if count is not None else torch.empty(1, dtype=torch.int32, device=A.device)
+    _check(lib.sfnn_predict_noalloc(_ptr(x), _ptr(A), _ptr(B), _ptr(c), d, r, n, _dtype_code(A.dtype), _ptr(idx),
+                                    _ptr(count), _stream(stream)), "sfnn_predict_noalloc")
+    return idx, count
 
 
 def forward_stack(layers, X0, XL=None, idx=None, counts=None, return_sets: bool = False, stream=None):

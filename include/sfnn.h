@@ -213,6 +213,30 @@ SFNN_API sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path);
  */
 SFNN_API sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before, sfnn_event_t after);
 
+/*
+ * The predictor for one token without any allocation.  The pages have no
+ * counterpart: this entry point exists for callers that cannot call cudaMalloc --
+ * code that runs while a CUDA graph is being captured, runtimes whose device memory
+ * belongs entirely to their own pool allocator, embedded users that forbid allocation
+ * after start-up -- and so cannot build a handle with sfnn_create.
+ *   x  [d], pa = A [d x r], pb = B [r x n], pc = c [n]: DEVICE, PyTorch layouts, wdtype
+ *   idx [n] int32 out: the selected neurons in ascending order (first *count entries)
+ *   count [1] int32 out
+ * The set is S(x) = { i : (relu(x.A).B + c)_i > 0 }, as sfnn_predict computes it.
+ * Scratch (the hidden layer and the decision mask) lives in one static device array
+ * of SFNN_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until exit;
+ * the call needs 4*r rounded up to 256, plus 4*ceil(n/32) bytes of it, and returns
+ * SFNN_ERR_UNSUPPORTED, launching nothing, when r and n need more.  It calls no
+ * allocation routine.  The first call on a device looks up that device's address of
+ * the array (cudaGetSymbolAddress); make it before any stream capture.  Every call
+ * shares the array: calls that overlap on the GPU (other streams, other host threads)
+ * race and must be serialised by the caller.  Asynchronous on `stream`.
+ */
+#define SFNN_NOALLOC_SCRATCH_BYTES (64 * 1024)
+SFNN_API sfnn_status sfnn_predict_noalloc(const void *x, const void *pa, const void *pb, const void *pc, int32_t d,
+                                          int32_t r, int32_t n, int32_t wdtype, int32_t *idx, int32_t *count,
+                                          sfnn_stream_t stream);
+
 /* Fill *info (host struct). */
 SFNN_API sfnn_status sfnn_query(sfnn_handle h, sfnn_info *info);
 
