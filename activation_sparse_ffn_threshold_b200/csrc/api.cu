@@ -33,8 +33,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar,
-                  h->gact, h->gcnt};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -136,8 +135,6 @@ void plan_decode1(sfnn_ctx *h, int G) {
   P.hbuf = h->h;
   P.part = h->part;
   P.bar = h->bar;
-  P.gact = h->gact;
-  P.gcnt = h->gcnt;
   P.err = h->err;
   P.d = L.d;
   P.n = L.n;
@@ -256,8 +253,6 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
       {(void **)&h->bar, sizeof(uint64_t), false},
-      {(void **)&h->gact, ((n + G - 1) / G) * (size_t)G * 4, false},
-      {(void **)&h->gcnt, (size_t)G * 4, false},
   };
   for (auto &q : reqs) {
     if (cudaMalloc(q.ptr, q.bytes) != cudaSuccess) {

@@ -1,7 +1,6 @@
-// async.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, 1-D bulk async copies
-// (the TMA engine's cp.async.bulk, no multicast), programmatic dependent launch, and a
-// grid-wide barrier.  Every wait here is bounded: after `limit` polls it reports failure
-// instead of spinning forever.
+// async.cuh -- thin inline-PTX wrappers for sm_100a: per-thread asynchronous copies into
+// shared memory (cp.async), bulk L2 prefetch (the TMA engine, no multicast), programmatic
+// dependent launch, and a bounded grid barrier.
 #pragma once
 
 #include <stdint.h>
@@ -12,75 +11,57 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-// Make initialised barriers visible to the async (TMA) proxy.
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking test of the same condition.
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounds of waits are counted in SM clock cycles (clock64 is a cheap per-SM counter);
 // 2^31 cycles is about one second at the B200's clocks.
 constexpr uint64_t kWaitCycles = 1ull << 31;
 
-// Wait for the phase with the given parity to complete; false after `limit` cycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
-  const uint64_t t0 = clock64();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((uint64_t)(clock64() - t0) > limit) return false;
+// 16-byte asynchronous copy global -> shared (bypassing L1), grouped per thread.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The same with a run-time count (0..15; other counts wait for all groups).
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  switch (n) {
+    case 15: cp_async_wait<15>(); break;
+    case 14: cp_async_wait<14>(); break;
+    case 13: cp_async_wait<13>(); break;
+    case 12: cp_async_wait<12>(); break;
+    case 11: cp_async_wait<11>(); break;
+    case 10: cp_async_wait<10>(); break;
+    case 9: cp_async_wait<9>(); break;
+    case 8: cp_async_wait<8>(); break;
+    case 7: cp_async_wait<7>(); break;
+    case 6: cp_async_wait<6>(); break;
+    case 5: cp_async_wait<5>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 1: cp_async_wait<1>(); break;
+    default: cp_async_wait<0>(); break;
   }
 }
 
-// global -> shared bulk copy completing on an mbarrier (16-byte aligned, size % 16 == 0).
-__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst_smem)),
-      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
+// Bulk prefetch of [p, p + bytes) into L2 (no completion to wait for); p and bytes must be
+// multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// Prefetch [p, p + bytes) in pieces of at most 16 KB, one piece per step of `lane0`
+// through `stride` (the callers' threads share the pieces).
+__device__ __forceinline__ void prefetch_l2_range(const void *p, size_t bytes, int lane0, int stride) {
+  constexpr size_t kPiece = 16384;
+  const unsigned char *b = static_cast<const unsigned char *>(p);
+  for (size_t off = (size_t)lane0 * kPiece; off < bytes; off += (size_t)stride * kPiece) {
+    const size_t len = bytes - off < kPiece ? bytes - off : kPiece;
+    prefetch_l2_bulk(b + off, (uint32_t)len);
+  }
 }
 
 // Programmatic dependent launch: let the next kernel in the stream start its prologue,
@@ -88,22 +69,11 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
   uint64_t v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-
 __device__ __forceinline__ uint64_t atom_add_release_gpu_u64(uint64_t *p, uint64_t v) {
   uint64_t old;
   asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
@@ -113,9 +83,9 @@ __device__ __forceinline__ uint64_t atom_add_release_gpu_u64(uint64_t *p, uint64
 // Grid barrier over `nblocks` co-resident CTAs, called by ONE thread per CTA, on a 64-bit
 // arrival counter that only grows: the ticket an arrival draws names its barrier instance
 // (ticket / nblocks), which completes when the counter reaches the next multiple of
-// nblocks.  One release-add and acquire polls; nothing is reset between instances or
-// launches.  Returns false if the wait ran out after `limit` cycles (the caller latches
-// an error; the counter must then be zeroed before the next launch).
+// nblocks.  One release-add, then acquire polls of one word; nothing is reset between
+// instances or launches.  Returns false if the wait ran out after `limit` cycles (the
+// caller latches an error; the counter must then be zeroed before the next launch).
 __device__ __forceinline__ bool grid_barrier(uint64_t *count, uint32_t nblocks, uint64_t limit) {
   const uint64_t ticket = atom_add_release_gpu_u64(count, 1ull);
   const uint64_t target = (ticket / nblocks + 1) * nblocks;

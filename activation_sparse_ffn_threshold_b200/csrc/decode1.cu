@@ -13,27 +13,30 @@
 //   A   h_j = relu(A^T[j] . x): one warp per predictor row, every chunk of the row
 //       requested at once (the first row before waiting for the previous kernel).
 //       h goes to global memory; grid barrier.
-//   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron with a 3-deep
-//       register pipeline over the warp's neurons; neuron i is active iff z_i > 0
-//       (sigmoid(z) > 0.5).  The tile's active positions, compacted in order, and
-//       their count are published; grid barrier.  Every CTA then takes an equal slice
-//       of the concatenated active list (tile order, so the same set always gives the
-//       same slices): the row work is balanced whatever each tile drew.
-//   C1  up (and gate) dot products of the slice's rows, split in 4 KB segments spread
-//       over all warps (2-deep pipeline); segment sums added in a fixed order, then
-//       ReLU / ReGLU.  Rows of inactive neurons are never requested.
-//   C2  the slice's rows of W_down (neuron-major, contiguous) are added into
-//       per-thread column accumulators, 8 rows in flight.
+//   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron; each warp's B^T rows
+//       stream through 4 shared-memory stages of its own (16-byte cp.async copies,
+//       the first ones requested during phase A); neuron i is active iff
+//       z_i > 0 (sigmoid(z) > 0.5).  The tile's active positions are compacted in order.
+//   C1  up (and gate) dot products of the tile's active rows, split in 4 KB segments
+//       spread over all warps (2-deep register pipeline); segment sums added in a
+//       fixed order, then ReLU / ReGLU.  Rows of inactive neurons are never requested.
+//   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
+//       column accumulators; each thread's chunks stream through up to 8 private
+//       shared-memory stages, the first ones requested before C1.
 //   D   the CTA's partial y goes to global memory; grid barrier; CTA c sums a column
 //       slice of all G partials in a fixed order (two-phase, deterministic) -> y
 //       (+ residual, + rounded next-layer input).
+//
+// Every CTA works on the active rows of its own tile: the rows are never exchanged, so
+// the kernel has two grid barriers, and the hotness deal keeps the tiles' expected
+// counts equal (the busiest tile of a token typically holds 1.5-1.7x the mean).
 //
 // The predictor's dot products keep the order of the multi-kernel predictor (lane l
 // takes 16-byte chunks l, l+32, ... into one accumulator, then a butterfly sum), so
 // both paths decide every neuron identically.  PDL: the kernel lets the next one
 // launch at once and reads x, and writes anything, only after griddepcontrol.wait.
-// The three grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT
-// and returns without a result.
+// Both grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT and
+// returns without a result.
 #include "async.cuh"
 #include "common.cuh"
 #include "decode1.cuh"
@@ -44,11 +47,7 @@ namespace {
 constexpr int kT = kDecode1Threads;
 constexpr int kW = kT / 32;
 constexpr int kSegChunks = 256;  // 16-byte chunks of one C1 segment (8 per lane)
-constexpr int kSmemCap = 200 * 1024;
-
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
+constexpr int kSmemCap = 227 * 1024;
 
 template <typename T>
 __device__ __forceinline__ float dot_chunk(const uint4 &w, const float *h, float a) {
@@ -90,19 +89,23 @@ template <typename T, int ACT, int MAXM>
 __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr int V = Elem<T>::kVec;
   constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
+  constexpr int DB = kDecode1BStages;
+  constexpr int DD = decode1_dstages(MAXM);
   extern __shared__ __align__(16) unsigned char smem[];
   const Decode1Layout L = decode1_layout(P);
   unsigned char *xs = smem + L.x;
-  float *bias_s = reinterpret_cast<float *>(smem + L.bias);
+  float *bias_s = reinterpret_cast<float *>(smem + L.bias);  // b of the active rows, in order
   float *c_s = reinterpret_cast<float *>(smem + L.c);
   int *act_s = reinterpret_cast<int *>(smem + L.act);
-  float *a_s = reinterpret_cast<float *>(smem + L.a);
+  float *a_s = reinterpret_cast<float *>(smem + L.a);  // b of the tile, then activations
   float *dots = reinterpret_cast<float *>(smem + L.dots);
   float *red2 = reinterpret_cast<float *>(smem + L.red2);
-  int *pref = reinterpret_cast<int *>(smem + L.pref);
   uint32_t *bits = reinterpret_cast<uint32_t *>(smem + L.bits);
+  int *wpref = reinterpret_cast<int *>(smem + L.wpref);
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
+  unsigned char *bstage = smem + L.bstage;
+  unsigned char *dstage = smem + L.dstage;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = P.G;
@@ -115,25 +118,51 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const T *rows = static_cast<const T *>(P.rows);
 
   pdl_launch_dependents();
-  {
-    const T *cp = static_cast<const T *>(P.cvec);
-    for (int i = tid; i < tn; i += kT) c_s[i] = to_f<T>(cp[t0 + i]);
-    for (int i = tid; i < (P.tile_max + 31) / 32; i += kT) bits[i] = 0u;
-  }
+  const int j0 = c + G * warp;  // this warp's first row of A^T
 
   // ---------------------------------------------------------------- A: hidden layer
-  const int j0 = c + G * warp;
+  // The first batch of the warp's first row is requested before anything else: phase A
+  // is the critical path into the first grid barrier.
   uint4 w0[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const int ch = lane + 32 * u;
     if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
   }
+  const T *cp = static_cast<const T *>(P.cvec);
+  const T *bp = static_cast<const T *>(P.bias);
+  T c_first = from_f<T>(0.f), b_first = from_f<T>(0.f);  // c and b at tile position tid
+  if (tid < tn) {
+    c_first = cp[t0 + tid];
+    b_first = bp[t0 + tid];
+  }
+  for (int i = tid; i < (P.tile_max + 31) / 32; i += kT) bits[i] = 0u;
+
+  // B^T rows of this warp's neurons stream through DB shared-memory stages private to the
+  // warp; each lane copies (cp.async) exactly the chunks it will read, so only its own
+  // wait is needed.  The first DB rows are requested during phase A, after x and the
+  // warp's row of A^T (the critical path into the first grid barrier), and land while
+  // phase A and the barrier run.
+  unsigned char *bst = bstage + (size_t)warp * DB * nch_r * 16;
+  auto stage_b = [&](int s, int p) {  // row p of the tile into stage s; always one group
+    if (p < tn) {
+#pragma unroll
+      for (int m = 0; m < MAXH; ++m) {
+        const int ch = lane + 32 * m;
+        if (ch < nch_r) cp_async16(bst + ((size_t)s * nch_r + ch) * 16, Bt + (size_t)(t0 + p) * r + (size_t)ch * V);
+      }
+    }
+    cp_async_commit();
+  };
   pdl_wait();  // x (and every buffer this kernel writes) belongs to earlier kernels until here
   for (int i = tid; i < nch_d; i += kT)
     *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
         __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
   __syncthreads();
+  if (j0 >= r) {
+#pragma unroll
+    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
+  }
   for (int j = j0; j < r; j += G * kW) {
     const T *row = At + (size_t)j * d;
     float acc = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
@@ -154,7 +183,23 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     const float hs = warp_sum(acc);
     if (lane == 0) P.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
   }
-  if (!cta_grid_sync(P, flag_s)) return;
+  if (j0 < r) {
+#pragma unroll
+    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
+  }
+  // c and b of the tile into shared memory
+  if (tid < tn) {
+    c_s[tid] = to_f<T>(c_first);
+    a_s[tid] = to_f<T>(b_first);
+  }
+  for (int i = tid + kT; i < tn; i += kT) {
+    c_s[i] = to_f<T>(cp[t0 + i]);
+    a_s[i] = to_f<T>(bp[t0 + i]);
+  }
+  if (!cta_grid_sync(P, flag_s)) {
+    cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+    return;
+  }
 
   // ---------------------------------------------------------------- B: logits + threshold
   {
@@ -172,106 +217,76 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         hreg[m][v + 3] = q.w;
       }
     }
-    constexpr int D = 3;
-    uint4 wb[D][MAXH];
+    for (int pb = warp; pb < tn; pb += DB * kW) {
 #pragma unroll
-    for (int s = 0; s < D; ++s) {
-      const int p = warp + kW * s;
-#pragma unroll
-      for (int m = 0; m < MAXH; ++m) {
-        const int ch = lane + 32 * m;
-        if (p < tn && ch < nch_r) wb[s][m] = ld_stream(Bt + (size_t)(t0 + p) * r + (size_t)ch * V);
-      }
-    }
-    for (int pb = warp; pb < tn; pb += D * kW) {
-#pragma unroll
-      for (int s = 0; s < D; ++s) {
+      for (int s = 0; s < DB; ++s) {
         const int p = pb + kW * s;
         if (p < tn) {
+          cp_async_wait<DB - 1>();  // this lane's copies of row p have landed
           float a = 0.f;
-#pragma unroll
-          for (int m = 0; m < MAXH; ++m)
-            if (lane + 32 * m < nch_r) a = dot_chunk<T>(wb[s][m], hreg[m], a);
-          const int pn = p + D * kW;
 #pragma unroll
           for (int m = 0; m < MAXH; ++m) {
             const int ch = lane + 32 * m;
-            if (pn < tn && ch < nch_r) wb[s][m] = ld_stream(Bt + (size_t)(t0 + pn) * r + (size_t)ch * V);
+            if (ch < nch_r)
+              a = dot_chunk<T>(*reinterpret_cast<const uint4 *>(bst + ((size_t)s * nch_r + ch) * 16), hreg[m], a);
           }
+          stage_b(s, p + DB * kW);
           const float z = warp_sum(a) + c_s[p];
           if (lane == 0 && z > 0.f) atomicOr(&bits[p >> 5], 1u << (p & 31));  // NaN -> inactive
         }
       }
     }
+    cp_async_wait<0>();
   }
   __syncthreads();
-  if (warp == 0) {  // the tile's active positions, ascending
-    const int nwords = (tn + 31) / 32;
+  // The tile's active positions, ascending: warp 0 scans the words' population counts,
+  // then every thread places its own positions.  The CTA takes its own tile's active
+  // rows: the hotness deal gives every tile the same expected count, and the rows stay
+  // where their decisions were made (no exchange).
+  const int nwords = (tn + 31) / 32;
+  if (warp == 0) {
     int base = 0;
     for (int wi = 0; wi < nwords; wi += 32) {
-      const uint32_t word = wi + lane < nwords ? bits[wi + lane] : 0u;
-      const int k = __popc(word);
+      const int k = wi + lane < nwords ? __popc(bits[wi + lane]) : 0;
       int incl = k;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      int pos = base + incl - k;
-      uint32_t m = word;
-      while (m) {
-        act_s[pos++] = (wi + lane) * 32 + __ffs(m) - 1;
-        m &= m - 1u;
-      }
+      if (wi + lane < nwords) wpref[wi + lane] = base + incl - k;
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) *cnt_s = base;
   }
   __syncthreads();
-  {  // publish the tile's active positions (global numbering) and their count
-    const int tc = *cnt_s;
-    for (int k = tid; k < tc; k += kT) P.gact[(size_t)c * P.tile_max + k] = t0 + act_s[k];
-    if (tid == 0) P.gcnt[c] = tc;
+  for (int p = tid; p < tn; p += kT) {
+    const uint32_t word = bits[p >> 5], bit = 1u << (p & 31);
+    if (word & bit) {
+      const int k = wpref[p >> 5] + __popc(word & (bit - 1u));
+      act_s[k] = t0 + p;
+      bias_s[k] = a_s[p];
+    }
   }
-  if (!cta_grid_sync(P, flag_s)) return;
-  if (warp == 0) {  // exclusive prefix of the tiles' counts
-    int base = 0;
-    for (int i0 = 0; i0 < G; i0 += 32) {
-      const int v = i0 + lane < G ? __ldcg(P.gcnt + i0 + lane) : 0;
-      int incl = v;
+  __syncthreads();
+  const int cnt = *cnt_s;
+
+  // C2's rows of W_down stream through DD shared-memory stages private to each thread;
+  // the first DD rows are requested now and land while C1 runs
+  auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
+  auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
+    if (k < cnt) {
+      const T *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * d;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      for (int m = 0; m < MAXM; ++m) {
+        const int ch = tid + kT * m;
+        if (ch < nch_d) cp_async16(dslot(s, m), row + (size_t)ch * V);
       }
-      if (i0 + lane < G) pref[i0 + lane] = base + incl - v;
-      base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) pref[G] = base;
-  }
-  __syncthreads();
-  // this CTA's slice [lo, hi) of the concatenated active list
-  const int K = pref[G];
-  const int lo = (int)(((int64_t)c * K) / G), hi = (int)(((int64_t)(c + 1) * K) / G);
-  const int cnt = hi - lo;
-  {
-    const T *bp = static_cast<const T *>(P.bias);
-    for (int k = tid; k < cnt; k += kT) {
-      const int g = lo + k;
-      int a = 0, b = G - 1;  // the tile holding g: pref[a] <= g < pref[a + 1]
-      while (a < b) {
-        const int mid = (a + b + 1) >> 1;
-        if (pref[mid] <= g)
-          a = mid;
-        else
-          b = mid - 1;
-      }
-      const int pos = __ldcg(P.gact + (size_t)a * P.tile_max + (g - pref[a]));
-      act_s[k] = pos;
-      bias_s[k] = to_f<T>(bp[pos]);
-    }
-  }
-  __syncthreads();
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < DD; ++s) stage_d(s, s);
 
   // ---------------------------------------------------------------- C1: up / gate dots
   {
@@ -341,47 +356,27 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   for (int m = 0; m < MAXM; ++m)
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
-  {
-    constexpr int D = MAXM == 1 ? 8 : (MAXM == 2 ? 4 : 2);
-    uint4 wd[D][MAXM];
+  for (int kb = 0; kb < cnt; kb += DD) {
 #pragma unroll
-    for (int s = 0; s < D; ++s) {
-      if (s < cnt) {
-        const T *row = rows + ((size_t)act_s[s] * nproj + (nproj - 1)) * d;
+    for (int s = 0; s < DD; ++s) {
+      const int k = kb + s;
+      if (k < cnt) {
+        cp_async_wait<DD - 1>();  // this thread's chunks of row k have landed
+        const float a = a_s[k];
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
-          const int ch = tid + kT * m;
-          if (ch < nch_d) wd[s][m] = ld_stream(row + (size_t)ch * V);
-        }
-      }
-    }
-    for (int kb = 0; kb < cnt; kb += D) {
+          if (tid + kT * m < nch_d) {
+            float f[V];
+            unpack<T>(*reinterpret_cast<const uint4 *>(dslot(s, m)), f);
 #pragma unroll
-      for (int s = 0; s < D; ++s) {
-        const int k = kb + s;
-        if (k < cnt) {
-          const float a = a_s[k];
-#pragma unroll
-          for (int m = 0; m < MAXM; ++m) {
-            if (tid + kT * m < nch_d) {
-              float f[V];
-              unpack<T>(wd[s][m], f);
-#pragma unroll
-              for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, f[v], acc[m][v]);
-            }
-          }
-          if (k + D < cnt) {
-            const T *row = rows + ((size_t)act_s[k + D] * nproj + (nproj - 1)) * d;
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m) {
-              const int ch = tid + kT * m;
-              if (ch < nch_d) wd[s][m] = ld_stream(row + (size_t)ch * V);
-            }
+            for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, f[v], acc[m][v]);
           }
         }
+        stage_d(s, k + DD);
       }
     }
   }
+  cp_async_wait<0>();
 
   // ---------------------------------------------------------------- D: partials, final sum
 #pragma unroll
@@ -404,8 +399,16 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     if (gi < ngu) {
       const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
       const float *src = P.part + col0 + cb + j;
-      float sum = 0.f;
-      for (int k = k0; k < k1; ++k) sum += __ldcg(src + (size_t)k * d);
+      float sum = 0.f;  // in ascending k; loads issued 8 at a time
+      int k = k0;
+      for (; k + 8 <= k1; k += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(k + u) * d);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum += v[u];
+      }
+      for (; k < k1; ++k) sum += __ldcg(src + (size_t)k * d);
       red2[gi * width + j] = sum;
     }
     __syncthreads();

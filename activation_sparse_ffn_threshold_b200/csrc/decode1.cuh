@@ -9,6 +9,14 @@
 namespace sfnn {
 
 constexpr int kDecode1Threads = 512;  // 16 warps per CTA, one CTA per SM
+constexpr int kDecode1BStages = 4;     // B^T rows staged per warp (thread-private shared staging)
+
+// W_down rows in flight per thread in the down phase, by 16-byte chunks per thread and row
+__host__ __device__ constexpr int decode1_dstages(int maxm) { return maxm == 1 ? 8 : (maxm == 2 ? 4 : 2); }
+// 16-byte chunks of a d-vector per thread (1, 2 or 4)
+__host__ __device__ inline int decode1_maxm(int nch_d) {
+  return nch_d <= kDecode1Threads ? 1 : (nch_d <= 2 * kDecode1Threads ? 2 : 4);
+}
 
 struct Decode1Params {
   const void *At, *Bt, *cvec, *bias, *rows;  // re-laid-out weights
@@ -19,8 +27,6 @@ struct Decode1Params {
   float *hbuf;                               // [r] predictor hidden layer (scratch)
   float *part;                               // [G][d] per-CTA partial sums (scratch)
   uint64_t *bar;                             // grid barrier arrival counter (scratch, zeroed at create)
-  int32_t *gact;                             // [G][tile_max] active positions of each tile (scratch)
-  int32_t *gcnt;                             // [G] their counts (scratch)
   int32_t *err;                              // latched device error
   int d, n, r, nproj, act, dt;
   int G;         // CTAs (one per SM) = tiles of neurons
@@ -29,10 +35,19 @@ struct Decode1Params {
 };
 
 struct Decode1Layout {
-  size_t x, bias, c, act, a, dots, red2, pref, bits, bars, total;
+  size_t x, bias, c, act, a, dots, red2, bits, wpref, bars, bstage, dstage, total;
 };
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Bytes of the staging region: B^T rows (phase B) and W_down chunks (C2) share it.
+__host__ __device__ inline size_t decode1_stage_bytes(const Decode1Params &P) {
+  const int vec = P.dt == SFNN_F16 ? 8 : 4;
+  const int maxm = decode1_maxm(P.d / vec);
+  const size_t bsz = (size_t)(kDecode1Threads / 32) * kDecode1BStages * (P.r / vec) * 16;
+  const size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
+  return bsz > dsz ? bsz : dsz;
+}
 
 __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) {
   const size_t esz = P.dt == SFNN_F16 ? 2 : 4;
@@ -53,12 +68,17 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) 
   o = decode1_align(o + tm * 2 * (size_t)P.nseg * 4, 16);
   L.red2 = o;
   o = decode1_align(o + (size_t)kDecode1Threads * 4, 16);
-  L.pref = o;  // exclusive prefix of the tiles' active counts (G + 1)
-  o = decode1_align(o + ((size_t)P.G + 1) * 4, 16);
   L.bits = o;
   o = decode1_align(o + ((tm + 31) / 32) * 4 + 16, 16);
-  L.bars = o;  // one mbarrier-free word: the active count
+  L.wpref = o;  // exclusive prefix of the bit words' population counts
+  o = decode1_align(o + ((tm + 31) / 32 + 1) * 4, 16);
+  L.bars = o;  // the active count and a flag
   o = decode1_align(o + 16, 16);
+  // The two staging areas share one region: B^T rows are staged only in phase B, the
+  // W_down chunks only after it (the CTA synchronises in between).
+  L.bstage = o;  // [warp][stage][chunk of the row]: B^T rows staged per warp
+  L.dstage = o;  // [stage][chunk m][thread]: W_down chunks staged per thread
+  o = decode1_align(o + decode1_stage_bytes(P), 16);
   L.total = o;
   return L;
 }
