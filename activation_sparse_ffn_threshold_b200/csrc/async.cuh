@@ -1,6 +1,5 @@
 // async.cuh -- thin inline-PTX wrappers for sm_100a: per-thread asynchronous copies into
-// shared memory (cp.async), bulk L2 prefetch (the TMA engine, no multicast), programmatic
-// dependent launch, and a bounded grid barrier.
+// shared memory (cp.async), programmatic dependent launch, and a bounded grid barrier.
 #pragma once
 
 #include <stdint.h>
@@ -24,44 +23,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// The same with a run-time count (0..15; other counts wait for all groups).
-__device__ __forceinline__ void cp_async_wait_n(int n) {
-  switch (n) {
-    case 15: cp_async_wait<15>(); break;
-    case 14: cp_async_wait<14>(); break;
-    case 13: cp_async_wait<13>(); break;
-    case 12: cp_async_wait<12>(); break;
-    case 11: cp_async_wait<11>(); break;
-    case 10: cp_async_wait<10>(); break;
-    case 9: cp_async_wait<9>(); break;
-    case 8: cp_async_wait<8>(); break;
-    case 7: cp_async_wait<7>(); break;
-    case 6: cp_async_wait<6>(); break;
-    case 5: cp_async_wait<5>(); break;
-    case 4: cp_async_wait<4>(); break;
-    case 3: cp_async_wait<3>(); break;
-    case 2: cp_async_wait<2>(); break;
-    case 1: cp_async_wait<1>(); break;
-    default: cp_async_wait<0>(); break;
-  }
-}
-
-// Bulk prefetch of [p, p + bytes) into L2 (no completion to wait for); p and bytes must be
-// multiples of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-// Prefetch [p, p + bytes) in pieces of at most 16 KB, one piece per step of `lane0`
-// through `stride` (the callers' threads share the pieces).
-__device__ __forceinline__ void prefetch_l2_range(const void *p, size_t bytes, int lane0, int stride) {
-  constexpr size_t kPiece = 16384;
-  const unsigned char *b = static_cast<const unsigned char *>(p);
-  for (size_t off = (size_t)lane0 * kPiece; off < bytes; off += (size_t)stride * kPiece) {
-    const size_t len = bytes - off < kPiece ? bytes - off : kPiece;
-    prefetch_l2_bulk(b + off, (uint32_t)len);
-  }
 }
 
 // Programmatic dependent launch: let the next kernel in the stream start its prologue,

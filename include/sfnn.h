@@ -185,11 +185,11 @@ SFNN_API sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_l
 
 /*
  * Enable (default) or disable the fused single-token kernel, which runs a whole
- * decode step of one token in one launch: one persistent CTA per SM, bulk async
- * copies of the predictor's B^T tile and of the active neurons' rows through a
- * shared-memory ring, grid-wide barriers with bounded waits.  Disabled, one token
- * runs through the same multi-kernel path as a batch.  SFNN_ERR_UNSUPPORTED when
- * enabling it on a layer it does not fit (too large a record or too few SMs).
+ * decode step of one token in one launch: one persistent CTA per SM owning a tile of
+ * neurons, the predictor's rows and the active neurons' rows streamed through
+ * shared memory, two grid-wide barriers with bounded waits.  Disabled, one token runs
+ * through the same multi-kernel path as a batch.  SFNN_ERR_UNSUPPORTED when enabling
+ * it on a layer it does not fit (shared memory or SM count).
  */
 SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
 
