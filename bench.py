@@ -40,7 +40,7 @@ import workload as W  # noqa: E402
 
 WORKLOAD = "opt6.7b_relu"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sfnn_forward_opt6.7b_relu.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "k_decode1_opt6.7b_relu.md")
 CSRC = os.path.join(ROOT, "activation_sparse_ffn_threshold_b200", "csrc")
 
 
