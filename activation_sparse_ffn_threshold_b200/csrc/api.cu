@@ -33,7 +33,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -111,9 +111,13 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
     SFNN_TRY(launch_mask_from_idx(h, idx, count, s));
   }
   SFNN_TRY(launch_compact(h, b, idx_out, cnt_out, s));
-  SFNN_TRY(launch_up(h, X, b, s));
   int splits = 1;
-  SFNN_TRY(launch_down(h, b, &splits, s));
+  if (h->batch_path == SFNN_BATCH_TENSOR_CORE && tc_batch_supported(h)) {
+    SFNN_TRY(launch_tc_batch(h, X, b, &splits, s));
+  } else {
+    SFNN_TRY(launch_up(h, X, b, s));
+    SFNN_TRY(launch_down(h, b, &splits, s));
+  }
   SFNN_TRY(launch_reduce(h, b, splits, resid, Y, xnext, s));
   record_if(after, s);
   h->launches += predict ? 6 : 5;
@@ -253,8 +257,10 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
       {(void **)&h->bar, sizeof(uint64_t), false},
+      {(void **)&h->hact, L.dt == SFNN_F16 && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
   };
   for (auto &q : reqs) {
+    if (q.bytes == 0) continue;  // not needed by this layer
     if (cudaMalloc(q.ptr, q.bytes) != cudaSuccess) {
       cudaGetLastError();
       free_handle(h);
@@ -270,6 +276,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();
+  if (ce == cudaSuccess && h->hact) ce = configure_tc_batch();
   if (ce == cudaSuccess) plan_decode1(h, G);
   if (ce == cudaSuccess) ce = launch_layout(h, desc, s);
   if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
@@ -349,7 +356,7 @@ sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   if (path != SFNN_BATCH_AUTO && path != SFNN_BATCH_CUDA_CORE && path != SFNN_BATCH_TENSOR_CORE)
     return SFNN_ERR_INVALID_ARG;
-  if (path == SFNN_BATCH_TENSOR_CORE) return SFNN_ERR_UNSUPPORTED;
+  if (path == SFNN_BATCH_TENSOR_CORE && !tc_batch_supported(h)) return SFNN_ERR_UNSUPPORTED;
   h->batch_path = path;
   return SFNN_OK;
 }

@@ -45,6 +45,7 @@ struct sfnn_ctx {
   uint32_t *utok;    // [n] tokens active on each union row (bit t)
   int32_t *ucount;   // [1]
   float *acoef;      // [n][max_batch] activation of each union row for each token
+  __half *hact;      // [32][n rounded up to 128] fp16 activations (tensor-core batch path) or null
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
@@ -142,5 +143,11 @@ cudaError_t launch_down(const sfnn_ctx *h, int b, int *splits, cudaStream_t s);
 cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *resid, float *Y, void *xnext,
                           cudaStream_t s);
 cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s);
+
+// Tensor-core (tcgen05) batch path: fp16 weights, d a multiple of 128.
+bool tc_batch_supported(const sfnn_ctx *h);
+int tc_hstride(int n);
+cudaError_t configure_tc_batch();
+cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits_out, cudaStream_t s);
 
 }  // namespace sfnn

@@ -1,0 +1,423 @@
+// tc_batch.cu -- the batched union FFN on the tensor cores (tcgen05, fp16 weights).
+//
+// With several tokens, the rows of the union of their sets are read once and serve every
+// token (53ai.com "sparsity for LLM inference" page, section 工程效果: the union grows with
+// the batch, so each row read is shared by more tokens).  At batch b the up (and gate)
+// projection of a union row is b dot products and its down row feeds b outputs, so the
+// work is a gathered GEMM whose arithmetic grows with b while its bytes stay the rows' ---
+// at b = 32 CUDA cores fall behind HBM, tcgen05 does not.
+//
+//   k_tc_up    D[union row][token] = W_up[U] . X^T (and W_gate[U] . X^T): one CTA per 128
+//              union rows; A = the gathered rows (K-major), B = the batch's x rows
+//              (K-major), accumulators in TMEM.  Epilogue: + b, ReLU / ReGLU, zero for
+//              the tokens whose set does not hold the row -> H[token][union] (fp16).
+//   k_tc_down  Y^T[cols][token] = W_down[U]^T . H^T over a split of the union: A = the
+//              gathered down rows, 128 output columns each (MN-major: a row is contiguous
+//              along d), B = H (K-major) -> part[split][token][cols]; k_reduce adds the
+//              splits in a fixed order.
+//
+// Operand tiles are 64 fp16 wide along K (one 128-byte swizzle row) and staged in shared
+// memory with 16-byte cp.async copies (the rows are gathered by index), 128-byte
+// swizzled, in the canonical layouts the MMA descriptors name.  Thread 0 issues the MMAs
+// of a stage and commits them to the stage's mbarrier, which frees the stage for the copy
+// of a later one.  Every wait is bounded: on a timeout the kernel latches
+// SFNN_ERR_TIMEOUT, frees its tensor memory and returns.
+#include "async.cuh"
+#include "common.cuh"
+
+namespace sfnn {
+namespace {
+
+constexpr int kTT = 128;  // threads per CTA (4 warps: warp w reads TMEM lanes 32w..32w+31)
+constexpr int kTM = 128;  // MMA M
+constexpr int kTK = 64;   // K of a stage: 64 fp16 = one 128-byte swizzle row
+constexpr int kTmemCols = 64;
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void mb_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mb_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+// Wait for the phase with this parity; false after kWaitCycles.
+__device__ __forceinline__ bool mb_wait(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = clock64();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((uint64_t)(clock64() - t0) > kWaitCycles) return false;
+  }
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Make this thread's generic-proxy writes to shared memory visible to the MMA's reads.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] . B[smem], one thread.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  const uint32_t mask0 = 0, mask1 = 0, mask2 = 0, mask3 = 0;  // no output lane disabled
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(mask0), "r"(mask1), "r"(mask2),
+      "r"(mask3)
+      : "memory");
+}
+// The mbarrier gets one arrival once every MMA this thread issued before has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// 16 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (the tile's 8-row atoms are
+// 1024-byte aligned).  K-major: lbo unused (16), sbo = stride of 8-row groups.
+// MN-major: lbo = stride of 64-element MN atoms, sbo = stride of 8-deep K groups.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: fp16 A and B, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+// Byte offset of 16-byte chunk c (0..7) of row `row` in a K-major 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int c) {
+  return (uint32_t)row * 128u + (uint32_t)((c ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void cp16(unsigned char *base, uint32_t off, const void *src) {
+  cp_async16(base + off, src);
+}
+
+// ---------------------------------------------------------------- k_tc_up
+// smem per stage: NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B).
+template <int ACT>
+__global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
+                                               const __half *__restrict__ X, const int32_t *__restrict__ ulist,
+                                               const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
+                                               __half *__restrict__ H, int hstride, int d, int b, int N, int nproj,
+                                               int stages, int32_t *err) {
+  constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t mbar[8];
+  __shared__ uint32_t tmem_base;
+  __shared__ int fail;
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int U = *ucount;
+  const int u0 = blockIdx.x * kTM;
+  if (u0 >= U) return;
+  const uint32_t stage_bytes = NP * 16384u + (uint32_t)N * 128u;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) mb_init(&mbar[s], 1);
+    mb_init_fence();
+    fail = 0;
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
+  const int c8 = tid & 7;
+  const __half *src[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int u = u0 + (tid >> 3) + 16 * i;
+    u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
+    src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
+  }
+  const int nk = d / kTK;
+  auto load = [&](int s, int kc) {
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        cp16(st + j * 16384, kmajor_off(row, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
+      }
+    unsigned char *xt = st + NP * 16384;
+    for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
+      const int t = q >> 3, c = q & 7;
+      const int tt = t < b ? t : b - 1;
+      cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+    }
+  };
+
+  const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
+  for (int s = 0; s < stages - 1; ++s) {
+    if (s < nk) load(s, s);
+    cp_async_commit();
+  }
+  bool ok = true;
+  for (int it = 0; it < nk && ok; ++it) {
+    const int s = it % stages;
+    // groups committed so far: stages - 1 + it; this stage's is the (it)-th
+    switch (stages) {
+      case 2: cp_async_wait<0>(); break;
+      case 3: cp_async_wait<1>(); break;
+      default: cp_async_wait<2>(); break;
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + (size_t)s * stage_bytes);
+      const uint32_t xt = st + NP * 16384;
+#pragma unroll
+      for (int k = 0; k < kTK / 16; ++k) {
+        const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
+                   (it > 0 || k > 0) ? 1u : 0u);
+      }
+      umma_commit(&mbar[s]);
+    }
+    // refill the stage the previous iteration's MMAs read, once they are done
+    const int nx = it + stages - 1;
+    if (nx < nk) {
+      if (it >= 1) {
+        const int ps = (it - 1) % stages;
+        if (!mb_wait(&mbar[ps], (uint32_t)(((it - 1) / stages) & 1))) {
+          fail = 1;
+        }
+      }
+      load(nx % stages, nx);
+    }
+    cp_async_commit();
+    __syncthreads();
+    ok = fail == 0;
+  }
+  cp_async_wait<0>();
+  if (ok && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) fail = 1;
+  tc_fence_after();
+  __syncthreads();
+  if (fail) {
+    if (tid == 0) latch_error(err, kErrTimeout);
+  } else {
+    const int row = warp * 32 + lane;
+    const int u = u0 + row;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float g[32], up[32];
+    for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + c0, g + c0);
+    if (ACT == SFNN_REGLU)
+      for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + N + c0, up + c0);
+    if (u < U) {
+      const int p = ulist[u];
+      const uint32_t tm = utok[u];
+      const float bv = __half2float(bias[p]);
+      for (int t = 0; t < N; ++t) {
+        float a = 0.f;
+        if (t < b && ((tm >> t) & 1u)) {
+          const float pre = g[t] + bv;
+          a = pre > 0.f ? pre : 0.f;
+          if (ACT == SFNN_REGLU) a *= up[t];
+        }
+        H[(size_t)t * hstride + u] = __float2half_rn(a);
+      }
+    } else if (u < hstride) {  // the union's padding up to the down GEMM's K chunks: zeros
+      for (int t = 0; t < N; ++t) H[(size_t)t * hstride + u] = __float2half_rn(0.f);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- k_tc_down
+// smem per stage: the A tile (64 union rows x 128 columns, MN-major, 16 KB) + the H tile
+// (N tokens x 64 union entries, K-major).
+__global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows, const __half *__restrict__ H,
+                                                 int hstride, const int32_t *__restrict__ ulist,
+                                                 const int32_t *__restrict__ ucount, float *__restrict__ part, int d,
+                                                 int b, int N, int nproj, int splits, int stages, int32_t *err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t mbar[8];
+  __shared__ uint32_t tmem_base;
+  __shared__ int fail;
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mt = blockIdx.x, ks = blockIdx.y;
+  const int U = *ucount;
+  const int nkc = (U + kTK - 1) / kTK;
+  const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
+  const int col0 = mt * kTM;
+  const uint32_t stage_bytes = 16384u + (uint32_t)N * 128u;
+
+  if (c0 == c1) {  // an empty split still provides its (zero) partial
+    for (int q = tid; q < b * kTM; q += kTT) part[((size_t)ks * b + q / kTM) * d + col0 + q % kTM] = 0.f;
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) mb_init(&mbar[s], 1);
+    mb_init_fence();
+    fail = 0;
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  // A: chunk q = tid + 128 i -> union row k = q / 16 of the stage, 16-byte column chunk
+  // c = q % 16; MN atom m' = c / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
+  auto load = [&](int s, int kc) {
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = tid + kTT * i;
+      const int k = q >> 4, c = q & 15;
+      int u = kc * kTK + k;
+      u = u < U ? u : U - 1;  // past the union: a repeated row times H's zero padding
+      const int k0 = k & 7, k1 = k >> 3, mp = c >> 3, cc = c & 7;
+      const uint32_t off = (uint32_t)(mp * 1024 + k1 * 2048 + k0 * 128 + ((cc ^ k0) << 4));
+      cp16(st, off, rows + ((size_t)ulist[u] * nproj + (nproj - 1)) * d + col0 + c * 8);
+    }
+    unsigned char *ht = st + 16384;
+    for (int q = tid; q < N * 8; q += kTT) {
+      const int t = q >> 3, c = q & 7;
+      cp16(ht, kmajor_off(t, c), H + (size_t)t * hstride + (size_t)kc * kTK + c * 8);
+    }
+  };
+
+  const uint32_t idesc = idesc_f16(kTM, N, 1, 0);
+  const int nk = c1 - c0;
+  for (int s = 0; s < stages - 1; ++s) {
+    if (s < nk) load(s, c0 + s);
+    cp_async_commit();
+  }
+  bool ok = true;
+  for (int it = 0; it < nk && ok; ++it) {
+    const int s = it % stages;
+    switch (stages) {
+      case 2: cp_async_wait<0>(); break;
+      case 3: cp_async_wait<1>(); break;
+      default: cp_async_wait<2>(); break;
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + (size_t)s * stage_bytes);
+      const uint32_t ht = st + 16384;
+#pragma unroll
+      for (int k = 0; k < kTK / 16; ++k)
+        umma_f16(tmem, sdesc_sw128(st + k * 4096, 1024, 2048), sdesc_sw128(ht + k * 32, 16, 1024), idesc,
+                 (it > 0 || k > 0) ? 1u : 0u);
+      umma_commit(&mbar[s]);
+    }
+    const int nx = it + stages - 1;
+    if (nx < nk) {
+      if (it >= 1) {
+        const int ps = (it - 1) % stages;
+        if (!mb_wait(&mbar[ps], (uint32_t)(((it - 1) / stages) & 1))) fail = 1;
+      }
+      load(nx % stages, c0 + nx);
+    }
+    cp_async_commit();
+    __syncthreads();
+    ok = fail == 0;
+  }
+  cp_async_wait<0>();
+  if (ok && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) fail = 1;
+  tc_fence_after();
+  __syncthreads();
+  if (fail) {
+    if (tid == 0) latch_error(err, kErrTimeout);
+  } else {
+    const int m = warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float v[32];
+    for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
+    for (int t = 0; t < b; ++t) part[((size_t)ks * b + t) * d + col0 + m] = v[t];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+constexpr int kUpStages = 3, kDownStages = 4;
+
+size_t up_smem(int act, int N) { return (size_t)kUpStages * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024; }
+size_t down_smem(int N) { return (size_t)kDownStages * (16384 + N * 128) + 1024; }
+
+}  // namespace
+
+bool tc_batch_supported(const sfnn_ctx *h) {
+  return h->L.dt == SFNN_F16 && h->L.d % kTM == 0 && h->hact != nullptr;
+}
+
+int tc_hstride(int n) { return (n + kTM - 1) / kTM * kTM; }
+
+cudaError_t configure_tc_batch() {
+  cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)up_smem(SFNN_RELU, 32));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)up_smem(SFNN_REGLU, 32));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32));
+  return e;
+}
+
+// Up / gate of the union rows for all b tokens -> h->hact; then the down projection into
+// `splits` partials of h->part.
+cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits_out, cudaStream_t s) {
+  const Layout &L = h->L;
+  const int N = b <= 16 ? 16 : 32;
+  const int hs = tc_hstride(L.n);
+  const __half *rows = static_cast<const __half *>(h->rows);
+  const int up_grid = (L.n + kTM - 1) / kTM;
+  if (L.act == SFNN_REGLU)
+    k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+  else
+    k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int mtiles = L.d / kTM;
+  // about two CTAs per SM over the output tiles and the splits of the union
+  int splits = (2 * h->num_sms + mtiles - 1) / mtiles;
+  splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
+  k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part, L.d, b, N,
+                                                            L.nproj, splits, kDownStages, h->err);
+  *splits_out = splits;
+  return cudaGetLastError();
+}
+
+}  // namespace sfnn

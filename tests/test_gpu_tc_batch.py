@@ -1,0 +1,77 @@
+"""The tensor-core (tcgen05) path of the batched union FFN.
+
+* every token of a batch agrees with the oracle (sets exact outside the arbitration
+  band, y within the tolerance), for ReLU and ReGLU, d a multiple of 128 up to 8192,
+  ragged n (the union's last tile and the down GEMM's last K chunk are partial), and
+  batch sizes on both sides of the MMA's N = 16 / 32 (2, 5, 16, 17, 32);
+* it agrees with the CUDA-core path within the tolerance and is bitwise reproducible;
+* the full-size batch configurations (OPT-30B-shaped b = 8, 70B-shaped b = 32) match
+  the oracle on every token;
+* layers it cannot serve (fp32 weights, d not a multiple of 128) refuse the path.
+"""
+import numpy as np
+import pytest
+
+import activation_sparse_ffn_threshold_b200 as sf
+import oracle
+import workload as W
+from parity_util import check_token, dev, mask_from_idx
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    ("opt6.7b_relu", 1024, 3001, 128),
+    ("70b_reglu", 2048, 5003, 256),
+    ("opt30b_relu", 7168, 4099, 1024),
+    ("70b_reglu", 8192, 1500, 1024),
+]
+
+
+def run_batch(h, X, path):
+    h.set_batch_path(path)
+    Y, idx, cnt = h.forward_batch(dev(X), return_sets=True)
+    return Y.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+@pytest.mark.parametrize("base,d,n,r", SHAPES)
+def test_tc_batch_matches_oracle_and_cuda_cores(base, d, n, r):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=41)
+    h = sf.SparseFFN.from_layer(lay, max_batch=32)
+    for b in (2, 5, 16, 17, 32):
+        X = W.make_tokens(cfg, b, seed=42, stream_key=b)
+        Yt, idx, cnt = run_batch(h, X, sf.BATCH_TENSOR_CORE)
+        Yc, idx_c, cnt_c = run_batch(h, X, sf.BATCH_CUDA_CORE)
+        assert np.array_equal(cnt, cnt_c) and np.array_equal(idx, idx_c)  # one predictor for both paths
+        for t in range(b):
+            check_token(lay, X[t], Yt[t], mask_from_idx(idx[t], cnt[t], n), f"{base} d={d} b={b} t={t}")
+            assert oracle.within_tolerance(Yt[t], Yc[t].astype(np.float64))[0]
+        Yt2, _, _ = run_batch(h, X, sf.BATCH_TENSOR_CORE)
+        assert np.array_equal(Yt, Yt2)
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("name,b", [("opt30b_relu", 8), ("70b_reglu", 32)])
+def test_tc_batch_full_size(name, b):
+    cfg = W.CONFIGS[name]
+    lay = W.make_layer(cfg, seed=0)
+    h = sf.SparseFFN.from_layer(lay, max_batch=b)
+    X = W.make_tokens(cfg, b, seed=43)
+    Y, idx, cnt = run_batch(h, X, sf.BATCH_TENSOR_CORE)
+    for t in range(b):
+        check_token(lay, X[t], Y[t], mask_from_idx(idx[t], cnt[t], cfg.n), f"{name} b={b} t={t}")
+    assert h.get_error() == 0
+
+
+def test_tc_batch_refused_where_it_cannot_run():
+    cfg32 = W.small_config(W.CONFIGS["tiny_relu_f32"], d=512, n=2048, r=64)
+    h = sf.SparseFFN.from_layer(W.make_layer(cfg32, seed=44), max_batch=4)
+    with pytest.raises(sf.SfnnError) as e:
+        h.set_batch_path(sf.BATCH_TENSOR_CORE)
+    assert e.value.status == 4
+    cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=1032, n=1000, r=64)  # d % 128 != 0
+    h = sf.SparseFFN.from_layer(W.make_layer(cfg, seed=45), max_batch=4)
+    with pytest.raises(sf.SfnnError) as e:
+        h.set_batch_path(sf.BATCH_TENSOR_CORE)
+    assert e.value.status == 4
+    h.set_batch_path(sf.BATCH_CUDA_CORE)
