@@ -33,7 +33,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -104,7 +104,12 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
     h->launches += 1;
     return SFNN_OK;
   }
-  if (predict) {
+  const bool tc = tc_batch_supported(h) && (h->batch_path == SFNN_BATCH_TENSOR_CORE ||
+                                            (h->batch_path == SFNN_BATCH_AUTO && b >= 2));
+  if (predict && tc && tc_predict_supported(h)) {
+    SFNN_TRY(launch_tc_predict(h, X, b, s));
+    h->launches += 1;  // three kernels instead of two
+  } else if (predict) {
     SFNN_TRY(launch_hidden(h, X, b, s));
     SFNN_TRY(launch_logits(h, b, s));
   } else {
@@ -112,7 +117,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
   }
   SFNN_TRY(launch_compact(h, b, idx_out, cnt_out, s));
   int splits = 1;
-  if (h->batch_path == SFNN_BATCH_TENSOR_CORE && tc_batch_supported(h)) {
+  if (tc) {
     SFNN_TRY(launch_tc_batch(h, X, b, &splits, s));
   } else {
     SFNN_TRY(launch_up(h, X, b, s));
@@ -258,6 +263,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->err, 4, false},
       {(void **)&h->bar, sizeof(uint64_t), false},
       {(void **)&h->hact, L.dt == SFNN_F16 && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
+      {(void **)&h->hpair, L.dt == SFNN_F16 && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
   };
   for (auto &q : reqs) {
     if (q.bytes == 0) continue;  // not needed by this layer

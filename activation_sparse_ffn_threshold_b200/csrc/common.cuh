@@ -46,6 +46,7 @@ struct sfnn_ctx {
   int32_t *ucount;   // [1]
   float *acoef;      // [n][max_batch] activation of each union row for each token
   __half *hact;      // [32][n rounded up to 128] fp16 activations (tensor-core batch path) or null
+  __half *hpair;     // [2][32][r] the batch's hidden layer as fp16 hi and lo parts (same path)
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
@@ -146,6 +147,8 @@ cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaS
 
 // Tensor-core (tcgen05) batch path: fp16 weights, d a multiple of 128.
 bool tc_batch_supported(const sfnn_ctx *h);
+bool tc_predict_supported(const sfnn_ctx *h);  // and r a multiple of 64
+cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
 int tc_hstride(int n);
 cudaError_t configure_tc_batch();
 cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits_out, cudaStream_t s);

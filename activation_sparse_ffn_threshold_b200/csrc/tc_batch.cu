@@ -15,6 +15,8 @@
 //              gathered down rows, 128 output columns each (MN-major: a row is contiguous
 //              along d), B = H (K-major) -> part[split][token][cols]; k_reduce adds the
 //              splits in a fixed order.
+//   k_tc_hidden, k_tc_hsum, k_tc_logits  the predictor of the batch (dense GEMMs over
+//              A^T and B^T), ending in the token-major decision masks k_compact reads.
 //
 // Operand tiles are 64 fp16 wide along K (one 128-byte swizzle row) and staged in shared
 // memory with 16-byte cp.async copies (the rows are gathered by index), 128-byte
@@ -22,6 +24,8 @@
 // of a stage and commits them to the stage's mbarrier, which frees the stage for the copy
 // of a later one.  Every wait is bounded: on a timeout the kernel latches
 // SFNN_ERR_TIMEOUT, frees its tensor memory and returns.
+#include <algorithm>
+
 #include "async.cuh"
 #include "common.cuh"
 
@@ -117,6 +121,71 @@ __device__ __forceinline__ void cp16(unsigned char *base, uint32_t off, const vo
   cp_async16(base + off, src);
 }
 
+// ---------------------------------------------------------------- shared pipeline
+// All threads: init the stage mbarriers, allocate tensor memory (warp 0), publish.
+__device__ __forceinline__ uint32_t tc_begin(uint64_t *mbar, int stages, uint32_t *tmem_slot, int *fail) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) mb_init(&mbar[s], 1);
+    mb_init_fence();
+    *fail = 0;
+  }
+  if ((threadIdx.x >> 5) == 0) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tmem_slot;
+}
+// All threads: release tensor memory once every read of it is done.
+__device__ __forceinline__ void tc_end(uint32_t tmem) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, kTmemCols);
+}
+// The K loop: `load(s, it)` copies iteration it's operands into stage s (cp.async, all
+// threads); `issue(stage_smem_addr, it)` issues its MMAs (thread 0), which are committed
+// to the stage's mbarrier; the stage is refilled once they are done.  Returns false if a
+// wait ran out (then `fail` is set).  On return every MMA has completed (or failed) and
+// the accumulators may be read after tc_fence_after.
+template <class Load, class Issue>
+__device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_bytes, int stages, int nk,
+                                            uint64_t *mbar, int *fail, Load load, Issue issue) {
+  const int tid = threadIdx.x;
+  for (int s = 0; s < stages - 1; ++s) {
+    if (s < nk) load(s, s);
+    cp_async_commit();
+  }
+  bool ok = true;
+  for (int it = 0; it < nk && ok; ++it) {
+    const int s = it % stages;
+    // committed groups: stages - 1 + it; iteration it's is the (it + 1)-th oldest
+    switch (stages) {
+      case 2: cp_async_wait<0>(); break;
+      case 3: cp_async_wait<1>(); break;
+      default: cp_async_wait<2>(); break;
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      issue(smem_u32(smem + (size_t)s * stage_bytes), it);
+      umma_commit(&mbar[s]);
+    }
+    const int nx = it + stages - 1;  // refill the stage iteration it - 1 read, once its MMAs are done
+    if (nx < nk) {
+      if (it >= 1 && !mb_wait(&mbar[(it - 1) % stages], (uint32_t)(((it - 1) / stages) & 1))) *fail = 1;
+      load(nx % stages, nx);
+    }
+    cp_async_commit();
+    __syncthreads();
+    ok = *fail == 0;
+  }
+  cp_async_wait<0>();
+  if (ok && nk > 0 && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) *fail = 1;
+  tc_fence_after();
+  __syncthreads();
+  return *fail == 0;
+}
+
 // ---------------------------------------------------------------- k_tc_up
 // smem per stage: NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B).
 template <int ACT>
@@ -128,7 +197,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
-  __shared__ uint32_t tmem_base;
+  __shared__ uint32_t tmem_slot;
   __shared__ int fail;
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -136,17 +205,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   const int u0 = blockIdx.x * kTM;
   if (u0 >= U) return;
   const uint32_t stage_bytes = NP * 16384u + (uint32_t)N * 128u;
-
-  if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mb_init(&mbar[s], 1);
-    mb_init_fence();
-    fail = 0;
-  }
-  if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
+  const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
 
   // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
   const int c8 = tid & 7;
@@ -157,16 +216,13 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
     u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
     src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
   }
-  const int nk = d / kTK;
   auto load = [&](int s, int kc) {
     unsigned char *st = smem + (size_t)s * stage_bytes;
 #pragma unroll
     for (int j = 0; j < NP; ++j)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int row = (tid >> 3) + 16 * i;
-        cp16(st + j * 16384, kmajor_off(row, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
-      }
+      for (int i = 0; i < 8; ++i)
+        cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
     unsigned char *xt = st + NP * 16384;
     for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
       const int t = q >> 3, c = q & 7;
@@ -174,57 +230,19 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
     }
   };
-
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
-  for (int s = 0; s < stages - 1; ++s) {
-    if (s < nk) load(s, s);
-    cp_async_commit();
-  }
-  bool ok = true;
-  for (int it = 0; it < nk && ok; ++it) {
-    const int s = it % stages;
-    // groups committed so far: stages - 1 + it; this stage's is the (it)-th
-    switch (stages) {
-      case 2: cp_async_wait<0>(); break;
-      case 3: cp_async_wait<1>(); break;
-      default: cp_async_wait<2>(); break;
-    }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t st = smem_u32(smem + (size_t)s * stage_bytes);
-      const uint32_t xt = st + NP * 16384;
+  auto issue = [&](uint32_t st, int it) {
+    const uint32_t xt = st + NP * 16384;
 #pragma unroll
-      for (int k = 0; k < kTK / 16; ++k) {
-        const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
+    for (int k = 0; k < kTK / 16; ++k) {
+      const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
-                   (it > 0 || k > 0) ? 1u : 0u);
-      }
-      umma_commit(&mbar[s]);
+      for (int j = 0; j < NP; ++j)
+        umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
+                 (it > 0 || k > 0) ? 1u : 0u);
     }
-    // refill the stage the previous iteration's MMAs read, once they are done
-    const int nx = it + stages - 1;
-    if (nx < nk) {
-      if (it >= 1) {
-        const int ps = (it - 1) % stages;
-        if (!mb_wait(&mbar[ps], (uint32_t)(((it - 1) / stages) & 1))) {
-          fail = 1;
-        }
-      }
-      load(nx % stages, nx);
-    }
-    cp_async_commit();
-    __syncthreads();
-    ok = fail == 0;
-  }
-  cp_async_wait<0>();
-  if (ok && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) fail = 1;
-  tc_fence_after();
-  __syncthreads();
-  if (fail) {
+  };
+  if (!tc_mainloop(smem, stage_bytes, stages, d / kTK, mbar, &fail, load, issue)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int row = warp * 32 + lane;
@@ -251,9 +269,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       for (int t = 0; t < N; ++t) H[(size_t)t * hstride + u] = __float2half_rn(0.f);
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  tc_end(tmem);
 }
 
 // ---------------------------------------------------------------- k_tc_down
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
                                                  int b, int N, int nproj, int splits, int stages, int32_t *err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
-  __shared__ uint32_t tmem_base;
+  __shared__ uint32_t tmem_slot;
   __shared__ int fail;
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -280,20 +296,12 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
     for (int q = tid; q < b * kTM; q += kTT) part[((size_t)ks * b + q / kTM) * d + col0 + q % kTM] = 0.f;
     return;
   }
-  if (tid == 0) {
-    for (int s = 0; s < stages; ++s) mb_init(&mbar[s], 1);
-    mb_init_fence();
-    fail = 0;
-  }
-  if (warp == 0) tmem_alloc(&tmem_base, kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
+  const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
 
   // A: chunk q = tid + 128 i -> union row k = q / 16 of the stage, 16-byte column chunk
   // c = q % 16; MN atom m' = c / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
-  auto load = [&](int s, int kc) {
+  auto load = [&](int s, int it) {
+    const int kc = c0 + it;
     unsigned char *st = smem + (size_t)s * stage_bytes;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -311,50 +319,15 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
       cp16(ht, kmajor_off(t, c), H + (size_t)t * hstride + (size_t)kc * kTK + c * 8);
     }
   };
-
   const uint32_t idesc = idesc_f16(kTM, N, 1, 0);
-  const int nk = c1 - c0;
-  for (int s = 0; s < stages - 1; ++s) {
-    if (s < nk) load(s, c0 + s);
-    cp_async_commit();
-  }
-  bool ok = true;
-  for (int it = 0; it < nk && ok; ++it) {
-    const int s = it % stages;
-    switch (stages) {
-      case 2: cp_async_wait<0>(); break;
-      case 3: cp_async_wait<1>(); break;
-      default: cp_async_wait<2>(); break;
-    }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t st = smem_u32(smem + (size_t)s * stage_bytes);
-      const uint32_t ht = st + 16384;
+  auto issue = [&](uint32_t st, int it) {
+    const uint32_t ht = st + 16384;
 #pragma unroll
-      for (int k = 0; k < kTK / 16; ++k)
-        umma_f16(tmem, sdesc_sw128(st + k * 4096, 1024, 2048), sdesc_sw128(ht + k * 32, 16, 1024), idesc,
-                 (it > 0 || k > 0) ? 1u : 0u);
-      umma_commit(&mbar[s]);
-    }
-    const int nx = it + stages - 1;
-    if (nx < nk) {
-      if (it >= 1) {
-        const int ps = (it - 1) % stages;
-        if (!mb_wait(&mbar[ps], (uint32_t)(((it - 1) / stages) & 1))) fail = 1;
-      }
-      load(nx % stages, c0 + nx);
-    }
-    cp_async_commit();
-    __syncthreads();
-    ok = fail == 0;
-  }
-  cp_async_wait<0>();
-  if (ok && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) fail = 1;
-  tc_fence_after();
-  __syncthreads();
-  if (fail) {
+    for (int k = 0; k < kTK / 16; ++k)
+      umma_f16(tmem, sdesc_sw128(st + k * 4096, 1024, 2048), sdesc_sw128(ht + k * 32, 16, 1024), idesc,
+               (it > 0 || k > 0) ? 1u : 0u);
+  };
+  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int m = warp * 32 + lane;
@@ -363,21 +336,162 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
     for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
     for (int t = 0; t < b; ++t) part[((size_t)ks * b + t) * d + col0 + m] = v[t];
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  tc_end(tmem);
 }
 
-constexpr int kUpStages = 3, kDownStages = 4;
+// ---------------------------------------------------------------- predictor
+// k_tc_hidden: partial hidden layer hp[ks][t][j] = A^T[j] . x_t over the ks-th split of d
+// (A^T rows contiguous, 128 per CTA).  k_tc_hsum: h = relu(sum over ks in order), split
+// into fp16 hi + lo (h - hi), the B operand pair of the logits.  k_tc_logits: z[i][t] =
+// B^T[i] . (hi_t + lo_t) + c_i for 128 neurons per CTA (two MMAs per step into one fp32
+// accumulator, so h keeps about 22 bits), active iff z > 0 -> one mask word per warp and
+// token by ballot (token-major masks, as k_compact reads them).
+__global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At, const __half *__restrict__ X,
+                                                   float *__restrict__ hp, int d, int r, int b, int N, int splits,
+                                                   int stages, int32_t *err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t mbar[8];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int fail;
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j0 = blockIdx.x * kTM, ks = blockIdx.y;
+  const int nkc = d / kTK;
+  const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
+  const uint32_t stage_bytes = 16384u + (uint32_t)N * 128u;
+  if (c0 == c1) {
+    for (int q = tid; q < b * kTM; q += kTT) {
+      const int t = q / kTM, j = j0 + q % kTM;
+      if (j < r) hp[((size_t)ks * b + t) * r + j] = 0.f;
+    }
+    return;
+  }
+  const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
+  const int c8 = tid & 7;
+  auto load = [&](int s, int it) {
+    const int kc = c0 + it;
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = (tid >> 3) + 16 * i;
+      const int j = j0 + row < r ? j0 + row : r - 1;
+      cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
+    }
+    unsigned char *xt = st + 16384;
+    for (int q = tid; q < N * 8; q += kTT) {
+      const int t = q >> 3, c = q & 7;
+      const int tt = t < b ? t : b - 1;
+      cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+    }
+  };
+  const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
+  auto issue = [&](uint32_t st, int it) {
+#pragma unroll
+    for (int k = 0; k < kTK / 16; ++k)
+      umma_f16(tmem, sdesc_sw128(st + k * 32, 16, 1024), sdesc_sw128(st + 16384 + k * 32, 16, 1024), idesc,
+               (it > 0 || k > 0) ? 1u : 0u);
+  };
+  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue)) {
+    if (tid == 0) latch_error(err, kErrTimeout);
+  } else {
+    const int j = j0 + warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float v[32];
+    for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
+    if (j < r)
+      for (int t = 0; t < b; ++t) hp[((size_t)ks * b + t) * r + j] = v[t];
+  }
+  tc_end(tmem);
+}
+
+__global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N, int r, __half *__restrict__ hhi,
+                          __half *__restrict__ hlo) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;  // t * r + j over N tokens
+  if (i >= N * r) return;
+  const int t = i / r;
+  float h = 0.f;
+  if (t < b) {
+    const int j = i - t * r;
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += hp[((size_t)k * b + t) * r + j];
+    h = s > 0.f ? s : 0.f;  // NaN -> 0
+  }
+  const __half hi = __float2half_rn(h);
+  hhi[i] = hi;
+  hlo[i] = __float2half_rn(h - __half2float(hi));
+}
+
+__global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt, const __half *__restrict__ cvec,
+                                                   const __half *__restrict__ hhi, const __half *__restrict__ hlo,
+                                                   uint32_t *__restrict__ mask, int n, int r, int nwords, int b, int N,
+                                                   int stages, int32_t *err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t mbar[8];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int fail;
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = blockIdx.x * kTM;
+  const uint32_t stage_bytes = 16384u + 2u * (uint32_t)N * 128u;
+  const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
+  const int c8 = tid & 7;
+  auto load = [&](int s, int kc) {
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = (tid >> 3) + 16 * i;
+      const int nn = i0 + row < n ? i0 + row : n - 1;
+      cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
+    }
+    unsigned char *ht = st + 16384;
+    for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
+      const int half = q / (N * 8), qq = q - half * N * 8;
+      const int t = qq >> 3, c = qq & 7;
+      cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
+    }
+  };
+  const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
+  auto issue = [&](uint32_t st, int it) {
+    const uint32_t ht = st + 16384;
+#pragma unroll
+    for (int k = 0; k < kTK / 16; ++k) {
+      const uint64_t ad = sdesc_sw128(st + k * 32, 16, 1024);
+      umma_f16(tmem, ad, sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
+      umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
+    }
+  };
+  if (!tc_mainloop(smem, stage_bytes, stages, r / kTK, mbar, &fail, load, issue)) {
+    if (tid == 0) latch_error(err, kErrTimeout);
+  } else {
+    const int i = i0 + warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float v[32];
+    for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
+    const float cv = i < n ? __half2float(cvec[i]) : 0.f;
+    const int word = (i0 + warp * 32) >> 5;
+    for (int t = 0; t < b; ++t) {
+      const bool on = i < n && v[t] + cv > 0.f;  // NaN -> inactive
+      const uint32_t bits = __ballot_sync(0xffffffffu, on);
+      if (lane == 0 && word < nwords) mask[(size_t)t * nwords + word] = bits;
+    }
+  }
+  tc_end(tmem);
+}
+
+constexpr int kUpStages = 3, kDownStages = 4, kPredStages = 4;
 
 size_t up_smem(int act, int N) { return (size_t)kUpStages * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024; }
 size_t down_smem(int N) { return (size_t)kDownStages * (16384 + N * 128) + 1024; }
+size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
+size_t logits_smem(int N) { return (size_t)kPredStages * (16384 + 2 * N * 128) + 1024; }
 
 }  // namespace
 
 bool tc_batch_supported(const sfnn_ctx *h) {
   return h->L.dt == SFNN_F16 && h->L.d % kTM == 0 && h->hact != nullptr;
 }
+
+bool tc_predict_supported(const sfnn_ctx *h) { return tc_batch_supported(h) && h->L.r % kTK == 0; }
 
 int tc_hstride(int n) { return (n + kTM - 1) / kTM * kTM; }
 
@@ -389,7 +503,39 @@ cudaError_t configure_tc_batch() {
                              (int)up_smem(SFNN_REGLU, 32));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)logits_smem(32));
   return e;
+}
+
+// The predictor of b tokens on the tensor cores -> h->mask (token-major bit words).
+cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStream_t s) {
+  const Layout &L = h->L;
+  const int N = b <= 16 ? 16 : 32;
+  const int rtiles = (L.r + kTM - 1) / kTM;
+  // split d so that the hidden layer runs on about one CTA per SM; the partials fit in
+  // the down projection's partial-sum buffer
+  const size_t cap = (size_t)std::max<size_t>((size_t)kMaxSplits * h->max_batch, (size_t)std::min(h->num_sms, L.n)) * L.d;
+  int splits = (h->num_sms + rtiles - 1) / rtiles;
+  splits = std::min(splits, L.d / kTK);
+  splits = std::min<int>(splits, (int)(cap / ((size_t)b * L.r)));
+  splits = splits < 1 ? 1 : splits;
+  k_tc_hidden<<<dim3(rtiles, splits), kTT, hidden_smem(N), s>>>(
+      static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r, b, N, splits,
+      kPredStages, h->err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  __half *hhi = h->hpair, *hlo = h->hpair + (size_t)32 * L.r;
+  k_tc_hsum<<<(N * L.r + 255) / 256, 256, 0, s>>>(h->part, splits, b, N, L.r, hhi, hlo);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_tc_logits<<<(L.n + kTM - 1) / kTM, kTT, logits_smem(N), s>>>(static_cast<const __half *>(h->Bt),
+                                                                  static_cast<const __half *>(h->cvec), hhi, hlo,
+                                                                  h->mask, L.n, L.r, L.nwords, b, N, kPredStages,
+                                                                  h->err);
+  return cudaGetLastError();
 }
 
 // Up / gate of the union rows for all b tokens -> h->hact; then the down projection into

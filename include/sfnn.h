@@ -80,11 +80,21 @@ typedef enum {
 typedef enum { SFNN_RELU = 0, SFNN_REGLU = 1 } sfnn_act;
 typedef enum { SFNN_F32 = 0, SFNN_F16 = 1 } sfnn_dtype;
 
-/* Which kernels the batched path (b > 1) uses for the gathered rows. */
+/*
+ * Which kernels the batched path (b > 1, and explicit sets) uses.  The tensor-core
+ * path runs the batch's predictor (hidden layer and logits as dense GEMMs; h enters
+ * the logits as an fp16 hi + lo pair, about 22 significant bits) and the union's
+ * up/gate and down projections (gathered GEMMs) on tcgen05 tensor cores, with fp32
+ * accumulation and the activations rounded to fp16 between the two projections; it
+ * needs fp16 weights, d a multiple of 128 and max_batch >= 2 (the predictor part also
+ * r a multiple of 64, else the CUDA-core predictor runs).  AUTO takes it for every
+ * batch of 2 or more tokens where it is available (measured faster at every batch
+ * size), and the CUDA-core path otherwise.
+ */
 typedef enum {
-    SFNN_BATCH_AUTO = 0,        /* choose from the expected union density */
+    SFNN_BATCH_AUTO = 0,
     SFNN_BATCH_CUDA_CORE = 1,   /* multi-token gather on CUDA cores */
-    SFNN_BATCH_TENSOR_CORE = 2  /* gathered GEMM on tcgen05 tensor cores */
+    SFNN_BATCH_TENSOR_CORE = 2  /* dense and gathered GEMMs on tcgen05 tensor cores */
 } sfnn_batch_path;
 
 /*
@@ -201,7 +211,8 @@ SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
  */
 SFNN_API sfnn_status sfnn_debug_stall_next_barrier(sfnn_handle h, sfnn_stream_t stream);
 
-/* Choose the batched path (sfnn_batch_path); SFNN_BATCH_AUTO by default. */
+/* Choose the batched path (sfnn_batch_path); SFNN_BATCH_AUTO by default.
+ * SFNN_ERR_UNSUPPORTED for SFNN_BATCH_TENSOR_CORE on a layer that path cannot serve. */
 SFNN_API sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path);
 
 /*

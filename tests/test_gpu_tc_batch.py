@@ -4,7 +4,10 @@
   band, y within the tolerance), for ReLU and ReGLU, d a multiple of 128 up to 8192,
   ragged n (the union's last tile and the down GEMM's last K chunk are partial), and
   batch sizes on both sides of the MMA's N = 16 / 32 (2, 5, 16, 17, 32);
-* it agrees with the CUDA-core path within the tolerance and is bitwise reproducible;
+* the batch's predictor runs on the tensor cores too (hidden layer split over d, logits
+  with h as an fp16 hi + lo pair): its sets pass the same arbitration;
+* it agrees with the CUDA-core path within the tolerance wherever both predict the same
+  set, and is bitwise reproducible;
 * the full-size batch configurations (OPT-30B-shaped b = 8, 70B-shaped b = 32) match
   the oracle on every token;
 * layers it cannot serve (fp32 weights, d not a multiple of 128) refuse the path.
@@ -42,10 +45,14 @@ def test_tc_batch_matches_oracle_and_cuda_cores(base, d, n, r):
         X = W.make_tokens(cfg, b, seed=42, stream_key=b)
         Yt, idx, cnt = run_batch(h, X, sf.BATCH_TENSOR_CORE)
         Yc, idx_c, cnt_c = run_batch(h, X, sf.BATCH_CUDA_CORE)
-        assert np.array_equal(cnt, cnt_c) and np.array_equal(idx, idx_c)  # one predictor for both paths
         for t in range(b):
-            check_token(lay, X[t], Yt[t], mask_from_idx(idx[t], cnt[t], n), f"{base} d={d} b={b} t={t}")
-            assert oracle.within_tolerance(Yt[t], Yc[t].astype(np.float64))[0]
+            mt = mask_from_idx(idx[t], cnt[t], n)
+            mc = mask_from_idx(idx_c[t], cnt_c[t], n)
+            check_token(lay, X[t], Yt[t], mt, f"{base} d={d} b={b} t={t}")
+            # the two predictors sum in different orders: they may part only where the
+            # oracle's logit is within the arbitration band, and agree on y where they agree
+            if np.array_equal(mt, mc):
+                assert oracle.within_tolerance(Yt[t], Yc[t].astype(np.float64))[0]
         Yt2, _, _ = run_batch(h, X, sf.BATCH_TENSOR_CORE)
         assert np.array_equal(Yt, Yt2)
     assert h.get_error() == 0
