@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="CPU budget of the reference arm (warm-up and timed steps together)")
     return ap.parse_args(argv)
 
 
@@ -245,7 +247,7 @@ def run_reference(args, dist):
     t0 = time.perf_counter()
     oracle.forward(lay, X[0], nthreads)
     t_one = max(1e-4, time.perf_counter() - t0)
-    budget = 150.0  # seconds for warm-up + timed steps together
+    budget = args.ref_seconds  # seconds for warm-up + timed steps together
     per_step = max(1, min(cfg.tokens, int(budget / max(1, args.steps + args.warmup) / t_one)))
     k = 0
     for _ in range(args.warmup):
