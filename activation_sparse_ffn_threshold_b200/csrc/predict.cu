@@ -182,7 +182,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
   return before + incl - v;
 }
 
-// Blocks 0..b-1 (only when token outputs are wanted): token lists.  Last block: the union.
+// Blocks 0..b-1 (only when token outputs are wanted): token lists.  Last block: the union,
+// with each union row's token mask; a thread reads the b tokens' words of its bit word
+// once (registers) and takes both the union bits and the masks from them.
 __global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ mask, int nwords, int n, int b,
                                                   const int32_t *__restrict__ perm, int32_t *__restrict__ ulist,
                                                   uint32_t *__restrict__ utok, int32_t *__restrict__ ucount,
@@ -191,10 +193,15 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ m
   const int t = blockIdx.x;
   const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
   const int w0 = threadIdx.x * wpt;
+  uint32_t mw[kMaxBatch];  // the tokens' words of the current bit word (union block)
   auto word = [&](int w) -> uint32_t {
     if (!is_union) return mask[(size_t)t * nwords + w];
     uint32_t m = 0u;
-    for (int tt = 0; tt < b; ++tt) m |= mask[(size_t)tt * nwords + w];
+#pragma unroll
+    for (int tt = 0; tt < kMaxBatch; ++tt) {
+      mw[tt] = tt < b ? mask[(size_t)tt * nwords + w] : 0u;
+      m |= mw[tt];
+    }
     return m;
   };
   int cnt = 0;
@@ -214,7 +221,8 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ m
       const int p = w * 32 + i;
       if (is_union) {
         uint32_t tb = 0u;
-        for (int tt = 0; tt < b; ++tt) tb |= ((mask[(size_t)tt * nwords + w] >> i) & 1u) << tt;
+#pragma unroll
+        for (int tt = 0; tt < kMaxBatch; ++tt) tb |= ((mw[tt] >> i) & 1u) << tt;
         ulist[pos] = p;
         utok[pos] = tb;
       } else if (idx_out) {

@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
   tc_end(tmem);
 }
 
-constexpr int kUpStages = 3, kDownStages = 4, kPredStages = 4;
+constexpr int kUpStages = 3, kDownStages = 3, kPredStages = 4;
 
 size_t up_smem(int act, int N) { return (size_t)kUpStages * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024; }
 size_t down_smem(int N) { return (size_t)kDownStages * (16384 + N * 128) + 1024; }
@@ -557,8 +557,9 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int mtiles = L.d / kTM;
-  // about two CTAs per SM over the output tiles and the splits of the union
-  int splits = (2 * h->num_sms + mtiles - 1) / mtiles;
+  // one wave: three CTAs fit on an SM (3 stages of 20 KB); the output tiles times the
+  // splits of the union fill them without a tail
+  int splits = (3 * h->num_sms) / mtiles;
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
   k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part, L.d, b, N,
                                                             L.nproj, splits, kDownStages, h->err);
