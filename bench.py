@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=1,
+                    help="tokens per forward call: 1 is the single-token decode (the headline); b > 1 "
+                         "times the batched union path on b tokens at a time")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="CPU budget of the reference arm (warm-up and timed steps together)")
     return ap.parse_args(argv)
@@ -434,6 +437,149 @@ def run_sfnn(args, dist):
         h.close()
     return 0
 
+# ---------------------------------------------------------------- the batched path
+def run_batch(args, dist):
+    """b tokens per forward_batch call: predictor of the batch, union of its sets, the
+    union's rows once for all b tokens.  A step is BATCHES_PER_STEP such calls over
+    rotating weight replicas, captured in one CUDA graph."""
+    import torch
+
+    import activation_sparse_ffn_threshold_b200 as sf
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    BATCHES_PER_STEP = 16
+    dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.workload]
+    b = args.batch
+    lay = W.make_layer(cfg, seed=args.seed)
+    Xh = W.make_tokens(cfg, BATCHES_PER_STEP * b, seed=args.seed + dist.rank, stream_key=b).reshape(
+        BATCHES_PER_STEP, b, cfg.d)
+    e = cfg.esize
+    props = torch.cuda.get_device_properties(dev)
+    l2 = props.L2_cache_size
+    per_batch = W.touched_bytes(cfg, W.expected_union_density(lay.p, b) * cfg.n, b)
+    R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b) for _ in range(R)]
+    info = handles[0].info()
+    path = "tcgen05" if cfg.dtype == "f16" and cfg.d % 128 == 0 else "cuda-core"
+    torch.cuda.synchronize()
+
+    X = torch.from_numpy(Xh).to(dev)
+    Y = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32, device=dev)
+    unions = []
+    for i in range(BATCHES_PER_STEP):  # union sizes, for the algorithmic byte count
+        _, idx, cnt = handles[0].forward_batch(X[i], return_sets=True)
+        m = torch.zeros(cfg.n, dtype=torch.bool, device=dev)
+        for t in range(b):
+            m[idx[t, :int(cnt[t])].long()] = True
+        unions.append(int(m.sum()))
+    unions = np.array(unions, dtype=np.int64)
+    bytes_batch = info["predictor_bytes"] + unions * info["row_bytes_per_neuron"] + b * cfg.d * (e + 4)
+    bytes_step = float(bytes_batch.sum())
+
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(BATCHES_PER_STEP):
+            handles[i % R].forward_batch(X[i], Y[i])
+    torch.cuda.synchronize()
+    launches0 = sum(h.info()["launches"] for h in handles)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(BATCHES_PER_STEP):
+            handles[i % R].forward_batch(X[i], Y[i])
+    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    gpu_uuid = str(props.uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            start.record(s)
+            for _ in range(args.steps):
+                g.replay()
+            stop.record(s)
+        torch.cuda.synchronize()
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    clocks = clk.summary()
+    err = max(h.get_error() for h in handles)
+    if err:
+        raise SystemExit(f"device-side error latched: {err}")
+    t_max = dist.max(elapsed_ms)
+    tokens_total = dist.sum(args.steps * BATCHES_PER_STEP * b)
+    value = tokens_total / (t_max / 1e3)
+    batch_us = elapsed_ms * 1e3 / (args.steps * BATCHES_PER_STEP)
+    achieved = float(bytes_batch.mean()) / (batch_us / 1e6) / 1e9
+    peak, peak_kind = measured_peak()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None,
+                "kernel": f"one batch of {b} tokens ({launches_per_step // BATCHES_PER_STEP} kernels, {path} path); "
+                          "duration = CUDA-event time of the timed region / batches",
+                "algorithmic_bytes_per_launch": float(bytes_batch.mean()), "avg_launch_us": batch_us,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s", "traffic_source": None}
+
+    e2e = None
+    if not args.no_e2e:
+        xin = torch.from_numpy(Xh).pin_memory()
+        yout = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32).pin_memory()
+        xd = torch.empty((b, cfg.d), dtype=X.dtype, device=dev)
+        yd = torch.empty((b, cfg.d), dtype=torch.float32, device=dev)
+        e2e_steps = max(1, min(args.steps, 20))
+
+        def one_step():
+            for i in range(BATCHES_PER_STEP):
+                xd.copy_(xin[i], non_blocking=True)
+                handles[i % R].forward_batch(xd, yd, stream=s)
+                yout[i].copy_(yd, non_blocking=True)
+        with torch.cuda.stream(s):
+            one_step()
+        torch.cuda.synchronize()
+        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        with torch.cuda.stream(s):
+            a.record(s)
+            for _ in range(e2e_steps):
+                one_step()
+            c.record(s)
+        torch.cuda.synchronize()
+        e_max = dist.max(a.elapsed_time(c))
+        e2e = {"value": dist.sum(e2e_steps * BATCHES_PER_STEP * b) / (e_max / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * e,
+               "d2h_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * 4,
+               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+
+    line = {
+        "metric": "sparse-FFN batched decode tokens/s per layer", "value": value, "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16" if e == 2 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": b, "batches_per_step": BATCHES_PER_STEP,
+                   "path": path, "replicas": R,
+                   "l2": f"inputs larger than L2: {R} weight replicas rotated per batch, "
+                         f"{bytes_step / BATCHES_PER_STEP / 1e6:.1f} MB touched per batch, L2 {l2 / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist.world} (no exchange)",
+                   "mean_union_rows": float(unions.mean())},
+        "effective_gbs": bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9,
+        "roofline": roofline,
+        "cpu_baseline": None,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    for h in handles:
+        h.close()
+    return 0
+
 
 def main(argv=None):
     args = parse_args(argv)
@@ -441,6 +587,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, dist)
+        if args.batch > 1:
+            return run_batch(args, dist)
         return run_sfnn(args, dist)
     finally:
         dist.close()
