@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   float *red2 = reinterpret_cast<float *>(smem + L.red2);
   uint32_t *bits = reinterpret_cast<uint32_t *>(smem + L.bits);
   int *wpref = reinterpret_cast<int *>(smem + L.wpref);
+  float *h_s = reinterpret_cast<float *>(smem + L.h);
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
   unsigned char *bstage = smem + L.bstage;
@@ -203,6 +204,10 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 
   // ---------------------------------------------------------------- B: logits + threshold
   {
+    // h once per CTA from L2 (every warp needs all of it), then into registers
+    for (int i = tid; i < r / 4; i += kT)
+      reinterpret_cast<float4 *>(h_s)[i] = __ldcg(reinterpret_cast<const float4 *>(P.hbuf) + i);
+    __syncthreads();
     float hreg[MAXH][V];
 #pragma unroll
     for (int m = 0; m < MAXH; ++m) {
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 #pragma unroll
       for (int v = 0; v < V; v += 4) {
         float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (ch < nch_r) q = __ldcg(reinterpret_cast<const float4 *>(P.hbuf + (size_t)ch * V + v));
+        if (ch < nch_r) q = *reinterpret_cast<const float4 *>(h_s + (size_t)ch * V + v);
         hreg[m][v] = q.x;
         hreg[m][v + 1] = q.y;
         hreg[m][v + 2] = q.z;

@@ -35,7 +35,7 @@ struct Decode1Params {
 };
 
 struct Decode1Layout {
-  size_t x, bias, c, act, a, dots, red2, bits, wpref, bars, bstage, dstage, total;
+  size_t x, h, bias, c, act, a, dots, red2, bits, wpref, bars, bstage, dstage, total;
 };
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -56,6 +56,8 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) 
   size_t o = 0;
   L.x = o;
   o = decode1_align(o + (size_t)P.d * esz, 16);
+  L.h = o;  // the hidden layer, read once per CTA
+  o = decode1_align(o + (size_t)P.r * 4, 16);
   L.bias = o;
   o = decode1_align(o + tm * 4, 16);
   L.c = o;
