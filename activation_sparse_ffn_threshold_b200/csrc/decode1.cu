@@ -22,7 +22,7 @@
 //       fixed order, then ReLU / ReGLU.  Rows of inactive neurons are never requested.
 //   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
 //       column accumulators; each thread's chunks stream through up to 8 private
-//       shared-memory stages, the first ones requested before C1.
+//       shared-memory stages, the first ones requested at C1's start.
 //   D   the CTA's partial y goes to global memory; grid barrier; CTA c sums a column
 //       slice of all G partials in a fixed order (two-phase, deterministic) -> y
 //       (+ residual, + rounded next-layer input).
@@ -71,13 +71,14 @@ __device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned c
 }
 
 // Grid barrier by thread 0, bracketed by CTA barriers; false (and the error latched)
-// if it timed out.
+// if it timed out.  No separate fences: the CTA's writes happen before thread 0's
+// release add through the CTA barrier, and another CTA's reads after its thread 0's
+// acquire load through its CTA barrier; causality order composes the CTA-scope and
+// GPU-scope synchronisations.
 __device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag) {
-  __syncthreads();  // the CTA's writes happen before thread 0's fence and release
+  __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     const bool ok = grid_barrier(P.bar, (uint32_t)P.G, kWaitCycles);
-    __threadfence();
     if (!ok) latch_error(P.err, kErrTimeout);
     *flag = ok ? 1 : 0;
   }
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int cnt = *cnt_s;
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread;
-  // the first DD rows are requested now and land while C1 runs
+  // the first DD rows are requested right after C1's first loads and land while C1 runs
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
     if (k < cnt) {
@@ -290,8 +291,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     }
     cp_async_commit();
   };
-#pragma unroll
-  for (int s = 0; s < DD; ++s) stage_d(s, s);
 
   // ---------------------------------------------------------------- C1: up / gate dots
   {
@@ -315,6 +314,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         }
       }
     }
+#pragma unroll
+    for (int s = 0; s < DD; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
       for (int s = 0; s < D; ++s) {
