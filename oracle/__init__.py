@@ -64,6 +64,10 @@ def _load():
         lib.oracle_ffn_masked.restype = None
         lib.oracle_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, I]
         lib.oracle_forward.restype = I
+        lib.oracle_quantize.argtypes = [I, I, I, P, L, L, P, P]
+        lib.oracle_quantize.restype = None
+        lib.oracle_ffn_masked_q.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, I]
+        lib.oracle_ffn_masked_q.restype = None
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = I
         _lib = lib
@@ -159,6 +163,72 @@ def forward(layer, x, nthreads: int = 1) -> Step:
     h, z, mask = predictor(x, layer.A, layer.B, layer.c, nthreads)
     a, y = ffn_masked(x, layer.w_up, layer.w_gate, layer.b, layer.w_down, mask, layer.cfg.act, nthreads)
     return Step(h, z, mask, a, y)
+
+
+# ---------------------------------------------------------------- int8 rows
+@dataclass
+class QRows:
+    """A layer's FFN rows as int8 codes and fp32 scales, one scale per neuron and
+    projection; q_down is neuron-major (neuron i's down row = column i of w_down)."""
+    q_up: np.ndarray
+    s_up: np.ndarray
+    q_gate: np.ndarray | None
+    s_gate: np.ndarray | None
+    q_down: np.ndarray
+    s_down: np.ndarray
+
+
+def quantize(w, units_along_rows: bool = True):
+    """Per-unit symmetric int8 codes of a 2-D array (units = rows, or columns when
+    ``units_along_rows`` is False): fp32 scale = absmax / 127, codes rounded to nearest
+    even in fp32 and clamped to [-127, 127].  Returns (q [units, len] int8, s [units])."""
+    w = _c(w)
+    assert w.ndim == 2
+    rows, cols = w.shape
+    units, length = (rows, cols) if units_along_rows else (cols, rows)
+    ustride, estride = (cols, 1) if units_along_rows else (1, cols)
+    q = np.empty((units, length), np.int8)
+    sc = np.empty(units, np.float32)
+    _load().oracle_quantize(units, length, _dt(w), _p(w), ustride, estride, _p(q), _p(sc))
+    return q, sc
+
+
+def quantize_layer(layer) -> QRows:
+    q_up, s_up = quantize(layer.w_up)
+    q_gate = s_gate = None
+    if layer.w_gate is not None:
+        q_gate, s_gate = quantize(layer.w_gate)
+    q_down, s_down = quantize(layer.w_down, units_along_rows=False)
+    return QRows(q_up, s_up, q_gate, s_gate, q_down, s_down)
+
+
+def ffn_masked_q(x, qr: QRows, b, mask, act, nthreads: int = 1):
+    """The FFN over the neurons with mask != 0, weights = codes * scales.  Returns (a, y)."""
+    x, b = _c(x), _c(b)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    n, d = qr.q_up.shape
+    assert qr.q_down.shape == (n, d) and mask.shape == (n,)
+    a = np.empty(n, np.float64)
+    y = np.empty(d, np.float64)
+    gate_q = qr.q_gate if qr.q_gate is not None else qr.q_up
+    gate_s = qr.s_gate if qr.s_gate is not None else qr.s_up
+    _load().oracle_ffn_masked_q(d, n, _act_code(act), _dt(x), _p(x), _p(np.ascontiguousarray(qr.q_up)),
+                                _p(np.ascontiguousarray(qr.s_up)), _p(np.ascontiguousarray(gate_q)),
+                                _p(np.ascontiguousarray(gate_s)), _p(b), _p(np.ascontiguousarray(qr.q_down)),
+                                _p(np.ascontiguousarray(qr.s_down)), _p(mask), _p(a), _p(y), nthreads)
+    return a, y
+
+
+def forward_q(layer, qr: QRows, x, nthreads: int = 1) -> Step:
+    """One decode step with int8 rows: the predictor as in ``forward``, then the FFN on
+    the dequantized rows."""
+    h, z, mask = predictor(x, layer.A, layer.B, layer.c, nthreads)
+    a, y = ffn_masked_q(x, qr, layer.b, mask, layer.cfg.act, nthreads)
+    return Step(h, z, mask, a, y)
+
+
+def forward_q_with_mask(layer, qr: QRows, x, mask, nthreads: int = 1) -> np.ndarray:
+    return ffn_masked_q(x, qr, layer.b, mask, layer.cfg.act, nthreads)[1]
 
 
 def forward_batch(layer, X, nthreads: int = 1) -> list[Step]:

@@ -174,6 +174,84 @@ int32_t oracle_forward(int32_t d, int32_t n, int32_t r, int32_t act, int32_t dt,
     return count;
 }
 
+/*
+ * Weight-only int8 rows (a NEXT step of the method: PowerInfer runs its weights in INT4
+ * on the smaller PC, 53ai.com page, section on evaluation; only the rows' storage
+ * changes, the arithmetic stays that of the FFN above).
+ *
+ * Quantisation of `units` units of `len` elements each (element k of unit i at
+ * w[i*unit_stride + k*elem_stride]): in IEEE fp32, scale_i = max_k |w_ik| / 127 and
+ * q_ik = round-to-nearest-even(w_ik / scale_i), clamped to [-127, 127]; an all-zero
+ * unit has scale 0 and codes 0.  The decision is taken in fp32 so that any fp32
+ * implementation of the same rule gives the same codes.  q is unit-major.
+ */
+void oracle_quantize(int32_t units, int32_t len, int32_t dt, const void *w, int64_t unit_stride,
+                     int64_t elem_stride, int8_t *q, float *scale) {
+    init_table();
+    for (int32_t i = 0; i < units; ++i) {
+        float amax = 0.0f;
+        for (int32_t k = 0; k < len; ++k) {
+            const float v = fabsf((float)ld(w, dt, (size_t)(i * unit_stride + k * elem_stride)));
+            if (v > amax) amax = v;
+        }
+        const float s = amax / 127.0f;
+        scale[i] = s;
+        for (int32_t k = 0; k < len; ++k) {
+            int32_t c = 0;
+            if (s > 0.0f) {
+                const float v = (float)ld(w, dt, (size_t)(i * unit_stride + k * elem_stride));
+                c = (int32_t)rintf(v / s);
+                c = c > 127 ? 127 : (c < -127 ? -127 : c);
+            }
+            q[(size_t)i * len + k] = (int8_t)c;
+        }
+    }
+}
+
+/* The FFN of oracle_ffn_masked with int8 rows: every weight is q * scale (exact in
+ * double).  q_up/q_gate [n][d] with scales [n]; q_down [n][d] neuron-major (neuron i's
+ * down row, i.e. column i of w_down) with scales [n].  x and b in dt. */
+void oracle_ffn_masked_q(int32_t d, int32_t n, int32_t act, int32_t dt, const void *x, const int8_t *q_up,
+                         const float *s_up, const int8_t *q_gate, const float *s_gate, const void *bias,
+                         const int8_t *q_down, const float *s_down, const uint8_t *mask, double *a, double *y,
+                         int32_t nthreads) {
+    init_table();
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int32_t i = 0; i < n; ++i) {
+        if (!mask[i]) {
+            a[i] = 0.0;
+            continue;
+        }
+        double up = 0.0;
+        for (int32_t k = 0; k < d; ++k) up += ((double)q_up[(size_t)i * d + k] * (double)s_up[i]) * ld(x, dt, k);
+        if (act == OR_RELU) {
+            const double pre = up + ld(bias, dt, i);
+            a[i] = pre > 0.0 ? pre : 0.0;
+        } else {
+            double gate = 0.0;
+            for (int32_t k = 0; k < d; ++k)
+                gate += ((double)q_gate[(size_t)i * d + k] * (double)s_gate[i]) * ld(x, dt, k);
+            gate += ld(bias, dt, i);
+            a[i] = (gate > 0.0 ? gate : 0.0) * up;
+        }
+    }
+    int32_t *list = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+    int32_t k = 0;
+    for (int32_t i = 0; i < n; ++i)
+        if (mask[i]) list[k++] = i;
+#pragma omp parallel for schedule(static)
+    for (int32_t j = 0; j < d; ++j) {
+        double s = 0.0;
+        for (int32_t t = 0; t < k; ++t) {
+            const int32_t i = list[t];
+            s += a[i] * ((double)q_down[(size_t)i * d + j] * (double)s_down[i]);
+        }
+        y[j] = s;
+    }
+    free(list);
+}
+
 int32_t oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -1,7 +1,8 @@
 """Planted mistakes in the oracle must be caught by its pins.
 
 Each mutant is a copy of oracle/oracle.c with one plausible error (a dropped
-term or clamp, a wrong comparison, a transposed operand, a wrong decode); it is
+term or clamp, a wrong comparison, a transposed operand, a wrong decode, a wrong
+quantization rule or scale); it is
 compiled on the CPU into a temporary library, swapped in for the real one, and
 the pin tests of test_oracle_pins.py are run against it.  Every mutant must
 fail at least one pin.  Nothing here touches a GPU.
@@ -30,10 +31,25 @@ MUTANTS = {
     "down_transposed": ("ld(w_down, dt, (size_t)j * n + list[t])", "ld(w_down, dt, (size_t)list[t] * d + j)"),
     "half_exponent_off": ("expo - 25", "expo - 24"),
     "half_sign_dropped": ("return sign ? -v : v;", "return v;"),
-    "inactive_not_skipped": ("if (!mask[i]) {", "if (0 && !mask[i]) {"),
+    "inactive_not_skipped": ("if (!mask[i]) {\n            a[i] = 0.0;\n            continue;\n        }\n        double up = 0.0;\n"
+                             "        for (int32_t k = 0; k < d; ++k) up += ld(w_up,",
+                             "if (0 && !mask[i]) {\n            a[i] = 0.0;\n            continue;\n        }\n"
+                             "        double up = 0.0;\n        for (int32_t k = 0; k < d; ++k) up += ld(w_up,"),
     "down_coefficient_by_position": ("s += a[list[t]] *", "s += a[t] *"),
     "reglu_gate_bias_dropped": ("g += ld(bias, dt, i);", "g += 0.0;"),
     "preact_bias_dropped": ("g[i] = s + ld(bias, dt, i);", "g[i] = s;"),
+    # int8 rows
+    "quant_scale_by_128": ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;"),
+    "quant_round_half_away": ("c = (int32_t)rintf(v / s);", "c = (int32_t)roundf(v / s);"),
+    "quant_truncates": ("c = (int32_t)rintf(v / s);", "c = (int32_t)(v / s);"),
+    "q_down_scale_of_up": ("* (double)s_down[i]);", "* (double)s_up[i]);"),
+    "q_relu_bias_dropped": ("const double pre = up + ld(bias, dt, i);", "const double pre = up;"),
+    "q_gate_clamp_dropped": ("a[i] = (gate > 0.0 ? gate : 0.0) * up;", "a[i] = gate * up;"),
+    "q_inactive_not_skipped": ("if (!mask[i]) {\n            a[i] = 0.0;\n            continue;\n        }\n        double up = 0.0;\n"
+                               "        for (int32_t k = 0; k < d; ++k) up += ((double)q_up",
+                               "if (0 && !mask[i]) {\n            a[i] = 0.0;\n            continue;\n        }\n"
+                               "        double up = 0.0;\n        for (int32_t k = 0; k < d; ++k) up += ((double)q_up"),
+    "q_gate_scale_dropped": ("((double)q_gate[(size_t)i * d + k] * (double)s_gate[i])", "((double)q_gate[(size_t)i * d + k])"),
 }
 
 
@@ -56,6 +72,8 @@ def _pin_calls(pins):
             calls.append(lambda dt=dt, act=act: pins.test_exact_set_equals_dense(act, dt))
     for act in ("relu", "reglu"):
         calls.append(lambda act=act: pins.test_all_ones_mask_equals_dense(act))
+        calls.append(lambda act=act: pins.test_forward_q_equals_forward_on_an_exact_grid(act))
+    calls += [pins.test_quantizer_hand_values, pins.test_quantizer_invariants]
     return calls
 
 

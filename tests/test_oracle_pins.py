@@ -11,7 +11,10 @@
 * the predictor's threshold against its definition sigmoid(z) > 0.5 evaluated
   with an exponential, h and z against an independent numpy evaluation;
 * the exact fp16 decoding against numpy for all 65536 bit patterns;
-* closed forms: one active neuron, the empty set, a tie and a NaN logit.
+* closed forms: one active neuron, the empty set, a tie and a NaN logit;
+* int8 rows: the quantizer's codes and scales worked by hand (ties to even, zero
+  rows), its error bound, and the int8-row step equal to the fp16 step on weights
+  that lie exactly on an int8 grid.
 """
 import json
 import os
@@ -264,3 +267,67 @@ def test_tolerance_rule():
     assert ok and not bad
     assert oracle.within_tolerance(np.zeros(3), np.zeros(3))[0]
     assert not oracle.within_tolerance(np.array([0, 1e-30, 0]), np.zeros(3))[0]
+
+
+# ---------------------------------------------------------------- int8 rows
+def test_quantizer_hand_values():
+    """Scale = absmax / 127 and codes rounded to nearest even, worked by hand: absmax
+    127 gives scale 1 (codes = rounded values, 2.5 -> 2), absmax 254 gives scale 2
+    (1.5 -> 2, -2.5 -> -2, 0.5 -> 0), an all-zero row gives scale 0 and codes 0."""
+    w = np.array([[127, -3.25, 2.5, 0.75, -127], [254, 3, -5, 1, 0], [0, 0, 0, 0, 0]], np.float16)
+    q, s = oracle.quantize(w)
+    assert q.tolist() == [[127, -3, 2, 1, -127], [127, 2, -2, 0, 0], [0, 0, 0, 0, 0]]
+    assert s.tolist() == [1.0, 2.0, 0.0]
+    qc, sc = oracle.quantize(np.ascontiguousarray(w.T), units_along_rows=False)
+    assert np.array_equal(qc, q) and np.array_equal(sc, s)
+
+
+def test_quantizer_invariants():
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((40, 96)) * rng.uniform(0.01, 3.0, (40, 1))).astype(np.float16)
+    w[5] = 0
+    q, s = oracle.quantize(w)
+    wf = w.astype(np.float64)
+    assert np.all(np.abs(q.astype(int)) <= 127)
+    nz = np.abs(wf).max(axis=1) > 0
+    assert np.all(np.abs(q[nz]).max(axis=1) == 127)
+    assert np.all(s[~nz] == 0) and np.all(q[~nz] == 0)
+    # |w - q s| <= s / 2, up to the fp32 rounding of w / s
+    err = np.abs(wf - q.astype(np.float64) * s[:, None].astype(np.float64))
+    assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 1e-5))
+    # the scale is the fp32 quotient absmax / 127
+    amax = np.abs(w.astype(np.float32)).max(axis=1)
+    assert np.array_equal(s, (amax / np.float32(127)).astype(np.float32))
+
+
+@pytest.mark.parametrize("act", ["relu", "reglu"])
+def test_forward_q_equals_forward_on_an_exact_grid(act):
+    """Weights that are int8 codes times 2^-7 (up, gate) or 2^-6 (down), exact in fp16,
+    each unit reaching +-127: quantization gives back those codes and scales, and the
+    int8-row step equals the fp16 step exactly."""
+    rng = np.random.default_rng(8)
+    d, n, r = 48, 40, 16
+
+    def grid(units, length):
+        q = rng.integers(-127, 128, (units, length))
+        q[np.arange(units), rng.integers(0, length, units)] = 127
+        return q
+
+    q_up, q_gate, q_down_t = grid(n, d), grid(n, d), grid(n, d)
+    w_up = (q_up / 128.0).astype(np.float16)
+    w_gate = (q_gate / 128.0).astype(np.float16) if act == "reglu" else None
+    w_down = np.ascontiguousarray((q_down_t / 64.0).astype(np.float16).T)  # another scale than up's
+    b = (rng.standard_normal(n) * 0.1).astype(np.float16)
+    A = (rng.standard_normal((d, r)) * 0.3).astype(np.float16)
+    B = (rng.standard_normal((r, n)) * 0.3).astype(np.float16)
+    c = (rng.standard_normal(n) * 0.1).astype(np.float16)
+    lay = _L(act, w_up, w_gate, b, w_down, A, B, c)
+    qr = oracle.quantize_layer(lay)
+    assert np.array_equal(qr.q_up, q_up) and np.all(qr.s_up == np.float32(2.0 ** -7))
+    assert np.array_equal(qr.q_down, q_down_t) and np.all(qr.s_down == np.float32(2.0 ** -6))
+    for t in range(3):
+        x = rng.standard_normal(d).astype(np.float16)
+        ref = oracle.forward(lay, x)
+        got = oracle.forward_q(lay, qr, x)
+        assert np.array_equal(got.mask, ref.mask) and ref.mask.sum() > 0
+        assert np.array_equal(got.a, ref.a) and np.array_equal(got.y, ref.y)
