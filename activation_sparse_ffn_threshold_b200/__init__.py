@@ -21,10 +21,10 @@ import torch
 
 __all__ = ["SparseFFN", "SfnnError", "forward_stack", "predict_noalloc", "hotness_order", "library_path",
            "load_library",
-           "RELU", "REGLU", "F32", "F16", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
+           "RELU", "REGLU", "F32", "F16", "I8", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
 
 RELU, REGLU = 0, 1
-F32, F16 = 0, 1
+F32, F16, I8 = 0, 1, 2
 BATCH_AUTO, BATCH_CUDA_CORE, BATCH_TENSOR_CORE = 0, 1, 2
 STATUS = {0: "SFNN_OK", 1: "SFNN_ERR_INVALID_ARG", 2: "SFNN_ERR_CUDA", 3: "SFNN_ERR_OOM",
           4: "SFNN_ERR_UNSUPPORTED", 5: "SFNN_ERR_TIMEOUT"}
@@ -50,7 +50,8 @@ class LayerDesc(ctypes.Structure):
                 ("max_batch", ctypes.c_int32), ("act", ctypes.c_int32), ("wdtype", ctypes.c_int32),
                 ("w_up", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("b", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p), ("pa", ctypes.c_void_p), ("pb", ctypes.c_void_p),
-                ("pc", ctypes.c_void_p), ("hotness", ctypes.POINTER(ctypes.c_float))]
+                ("pc", ctypes.c_void_p), ("hotness", ctypes.POINTER(ctypes.c_float)),
+                ("rows_dtype", ctypes.c_int32)]
 
 
 class Info(ctypes.Structure):
@@ -156,7 +157,9 @@ class SparseFFN:
     """
 
     def __init__(self, w_up, w_down, b, A, B, c, act: str = "relu", w_gate=None, hotness=None,
-                 max_batch: int = 1, device=None, stream=None):
+                 max_batch: int = 1, device=None, stream=None, rows: str | None = None):
+        """``rows="int8"`` stores the FFN rows as int8 codes with per-row fp32 scales
+        (fp16 layers; single-token fused path only, see sfnn_layer_desc.rows_dtype)."""
         lib = load_library()
         device = torch.device(device or "cuda")
         dtype = w_up.dtype if isinstance(w_up, torch.Tensor) else torch.from_numpy(np.asarray(w_up[:1])).dtype
@@ -180,18 +183,20 @@ class SparseFFN:
                          w_up_t.data_ptr(), w_gate_t.data_ptr() if w_gate_t is not None else None,
                          b_t.data_ptr(), w_down_t.data_ptr(), A_t.data_ptr(), B_t.data_ptr(), c_t.data_ptr(),
                          self._hot.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if self._hot is not None
-                         else None)
+                         else None, I8 if rows == "int8" else 0)
+        self.rows = rows
         self._h = ctypes.c_void_p()
         with torch.cuda.device(device):
             _check(lib.sfnn_create(ctypes.byref(desc), _stream(stream), ctypes.byref(self._h)), "sfnn_create")
         self._lib = lib
 
     @classmethod
-    def from_layer(cls, layer, max_batch: int = 1, use_hotness: bool = True, device=None, stream=None):
+    def from_layer(cls, layer, max_batch: int = 1, use_hotness: bool = True, device=None, stream=None,
+                   rows: str | None = None):
         """Build from a record with w_up, w_gate, b, w_down, A, B, c, p and cfg.act (numpy arrays)."""
         return cls(layer.w_up, layer.w_down, layer.b, layer.A, layer.B, layer.c, act=layer.cfg.act,
                    w_gate=layer.w_gate, hotness=layer.p if use_hotness else None, max_batch=max_batch,
-                   device=device, stream=stream)
+                   device=device, stream=stream, rows=rows)
 
     # ------------------------------------------------------------------ helpers
     def _check_x(self, x, rows=None):

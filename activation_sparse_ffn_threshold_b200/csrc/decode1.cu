@@ -59,6 +59,18 @@ __device__ __forceinline__ float dot_chunk(const uint4 &w, const float *h, float
   return a;
 }
 
+// 16 int8 codes of a row (one 16-byte chunk) against x[16 ch .. 16 ch + 15] (fp16 in
+// shared memory); the row's scale is applied to the finished sum.
+__device__ __forceinline__ float dot_chunk_i8(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  float xf[16];
+  unpack<__half>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 32), xf);
+  unpack<__half>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 32 + 16), xf + 8);
+  const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaf((float)(int8_t)(q[i >> 2] >> (8 * (i & 3))), xf[i], a);
+  return a;
+}
+
 template <typename T>
 __device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned char *xs, int ch, float a) {
   constexpr int V = Elem<T>::kVec;
@@ -86,9 +98,11 @@ __device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag)
   return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
-template <typename T, int ACT, int MAXM>
+template <typename T, int ACT, int MAXM, typename R>
 __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr int V = Elem<T>::kVec;
+  constexpr bool I8 = sizeof(R) == 1;  // int8 rows: codes with per-row scales
+  constexpr int VR = 16 / sizeof(R);   // row elements per 16-byte chunk
   constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
   constexpr int DB = kDecode1BStages;
   constexpr int DD = decode1_dstages(MAXM);
@@ -117,7 +131,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int nch_d = d / V, nch_r = r / V;
   const T *At = static_cast<const T *>(P.At);
   const T *Bt = static_cast<const T *>(P.Bt);
-  const T *rows = static_cast<const T *>(P.rows);
+  const R *rows = static_cast<const R *>(P.rows);
 
   pdl_launch_dependents();
   const int j0 = c + G * warp;  // this warp's first row of A^T
@@ -282,11 +296,16 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
     if (k < cnt) {
-      const T *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * d;
+      const R *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * d;
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
-        const int ch = tid + kT * m;
-        if (ch < nch_d) cp_async16(dslot(s, m), row + (size_t)ch * V);
+        const int ch = tid + kT * m;  // V columns (int8 rows: their V codes, 8 bytes)
+        if (ch < nch_d) {
+          if (I8)
+            cp_async8(dslot(s, m), row + (size_t)ch * V);
+          else
+            cp_async16(dslot(s, m), row + (size_t)ch * V);
+        }
       }
     }
     cp_async_commit();
@@ -300,17 +319,18 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     const int nseg = P.nseg;
     const int per_row = NPG * nseg;
     const int items = cnt * per_row;
+    const int nch_r8 = d / VR;  // 16-byte chunks of a row
     uint4 wc[D][SU];
 #pragma unroll
     for (int s = 0; s < D; ++s) {
       const int it = warp + kW * s;
       if (it < items) {
         const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
-        const T *row = rows + ((size_t)act_s[k] * nproj + pj) * d;
+        const R *row = rows + ((size_t)act_s[k] * nproj + pj) * d;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
           const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * V);
+          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
         }
       }
     }
@@ -326,16 +346,21 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 #pragma unroll
           for (int u = 0; u < SU; ++u) {
             const int ch = sg * kSegChunks + lane + 32 * u;
-            if (ch < nch_d) a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
+            if (ch < nch_r8) {
+              if (I8)
+                a = dot_chunk_i8(wc[s][u], xs, ch, a);
+              else
+                a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
+            }
           }
           const int itn = it + D * kW;
           if (itn < items) {
             const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
-            const T *row = rows + ((size_t)act_s[kn] * nproj + pjn) * d;
+            const R *row = rows + ((size_t)act_s[kn] * nproj + pjn) * d;
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
               const int ch = sgn * kSegChunks + lane + 32 * u;
-              if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * V);
+              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
             }
           }
           a = warp_sum(a);
@@ -349,9 +374,17 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
       if (ACT == SFNN_REGLU)
         for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
+      float sd = 1.f;
+      if (I8) {  // the codes' sums times their rows' scales; the down row's folded into a
+        const float *sc = P.rscale + (size_t)act_s[k] * nproj;
+        g *= sc[0];
+        if (ACT == SFNN_REGLU) u *= sc[1];
+        sd = sc[nproj - 1];
+      }
       const float pre = g + bias_s[k];
       const float relu = pre > 0.f ? pre : 0.f;
       a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
+      if (I8) a_s[k] *= sd;
     }
     __syncthreads();
   }
@@ -373,7 +406,13 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         for (int m = 0; m < MAXM; ++m) {
           if (tid + kT * m < nch_d) {
             float f[V];
-            unpack<T>(*reinterpret_cast<const uint4 *>(dslot(s, m)), f);
+            if (I8) {
+              const uint2 q = *reinterpret_cast<const uint2 *>(dslot(s, m));
+#pragma unroll
+              for (int v = 0; v < V; ++v) f[v] = (float)(int8_t)((v < 4 ? q.x : q.y) >> (8 * (v & 3)));
+            } else {
+              unpack<T>(*reinterpret_cast<const uint4 *>(dslot(s, m)), f);
+            }
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, f[v], acc[m][v]);
           }
@@ -432,7 +471,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 
 __global__ void k_barrier_bump(uint64_t *count) { atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull); }
 
-template <typename T, int ACT, int MAXM>
+template <typename T, int ACT, int MAXM, typename R>
 cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.G);
@@ -444,28 +483,28 @@ cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, b
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_decode1<T, ACT, MAXM>, P);
+  return cudaLaunchKernelEx(&cfg, k_decode1<T, ACT, MAXM, R>, P);
 }
 
-template <typename T, int ACT>
+template <typename T, int ACT, typename R>
 const void *pick_kernel(int nch) {
-  if (nch <= kT) return (const void *)k_decode1<T, ACT, 1>;
-  if (nch <= 2 * kT) return (const void *)k_decode1<T, ACT, 2>;
-  return (const void *)k_decode1<T, ACT, 4>;
+  if (nch <= kT) return (const void *)k_decode1<T, ACT, 1, R>;
+  if (nch <= 2 * kT) return (const void *)k_decode1<T, ACT, 2, R>;
+  return (const void *)k_decode1<T, ACT, 4, R>;
 }
 
-template <typename T, int ACT>
+template <typename T, int ACT, typename R>
 cudaError_t launch_act(const Decode1Params &P, size_t smem, cudaStream_t stream, bool pdl) {
   const int nch = P.d / Elem<T>::kVec;
-  if (nch <= kT) return launch_t<T, ACT, 1>(P, smem, stream, pdl);
-  if (nch <= 2 * kT) return launch_t<T, ACT, 2>(P, smem, stream, pdl);
-  return launch_t<T, ACT, 4>(P, smem, stream, pdl);
+  if (nch <= kT) return launch_t<T, ACT, 1, R>(P, smem, stream, pdl);
+  if (nch <= 2 * kT) return launch_t<T, ACT, 2, R>(P, smem, stream, pdl);
+  return launch_t<T, ACT, 4, R>(P, smem, stream, pdl);
 }
 
-template <typename T, int ACT>
+template <typename T, int ACT, typename R>
 cudaError_t config_act() {
-  const void *ks[] = {(const void *)k_decode1<T, ACT, 1>, (const void *)k_decode1<T, ACT, 2>,
-                      (const void *)k_decode1<T, ACT, 4>};
+  const void *ks[] = {(const void *)k_decode1<T, ACT, 1, R>, (const void *)k_decode1<T, ACT, 2, R>,
+                      (const void *)k_decode1<T, ACT, 4, R>};
   for (const void *k : ks) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
     if (e != cudaSuccess) return e;
@@ -473,13 +512,26 @@ cudaError_t config_act() {
   return cudaSuccess;
 }
 
+// The kernel for this plan: element types (fp32, fp16, or fp16 with int8 rows) and activation.
+const void *plan_kernel(const Decode1Params &P, int nch) {
+  if (P.dt != SFNN_F16)
+    return P.act == SFNN_REGLU ? pick_kernel<float, SFNN_REGLU, float>(nch) : pick_kernel<float, SFNN_RELU, float>(nch);
+  if (P.ri8)
+    return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, int8_t>(nch)
+                               : pick_kernel<__half, SFNN_RELU, int8_t>(nch);
+  return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, __half>(nch)
+                             : pick_kernel<__half, SFNN_RELU, __half>(nch);
+}
+
 }  // namespace
 
 cudaError_t configure_decode1() {
-  cudaError_t e = config_act<float, SFNN_RELU>();
-  if (e == cudaSuccess) e = config_act<float, SFNN_REGLU>();
-  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU>();
-  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU>();
+  cudaError_t e = config_act<float, SFNN_RELU, float>();
+  if (e == cudaSuccess) e = config_act<float, SFNN_REGLU, float>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, __half>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, __half>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, int8_t>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, int8_t>();
   return e;
 }
 
@@ -488,11 +540,7 @@ int decode1_blocks_per_sm(const Decode1Params &P) {
   if (smem > (size_t)kSmemCap) return 0;
   const int nch = P.d / (P.dt == SFNN_F16 ? 8 : 4);
   if (nch > 4 * kT) return 0;  // beyond the kernel's register plan
-  const void *k;
-  if (P.dt == SFNN_F16)
-    k = P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU>(nch) : pick_kernel<__half, SFNN_RELU>(nch);
-  else
-    k = P.act == SFNN_REGLU ? pick_kernel<float, SFNN_REGLU>(nch) : pick_kernel<float, SFNN_RELU>(nch);
+  const void *k = plan_kernel(P, nch);
   int blocks = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, kT, smem) != cudaSuccess) return 0;
   return blocks;
@@ -505,11 +553,14 @@ cudaError_t launch_barrier_bump(uint64_t *count, cudaStream_t stream) {
 
 cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl) {
   const size_t smem = decode1_layout(P).total;
-  if (P.dt == SFNN_F16)
-    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU>(P, smem, stream, pdl)
-                               : launch_act<__half, SFNN_RELU>(P, smem, stream, pdl);
-  return P.act == SFNN_REGLU ? launch_act<float, SFNN_REGLU>(P, smem, stream, pdl)
-                             : launch_act<float, SFNN_RELU>(P, smem, stream, pdl);
+  if (P.dt != SFNN_F16)
+    return P.act == SFNN_REGLU ? launch_act<float, SFNN_REGLU, float>(P, smem, stream, pdl)
+                               : launch_act<float, SFNN_RELU, float>(P, smem, stream, pdl);
+  if (P.ri8)
+    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, int8_t>(P, smem, stream, pdl)
+                               : launch_act<__half, SFNN_RELU, int8_t>(P, smem, stream, pdl);
+  return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, __half>(P, smem, stream, pdl)
+                             : launch_act<__half, SFNN_RELU, __half>(P, smem, stream, pdl);
 }
 
 }  // namespace sfnn

@@ -32,6 +32,8 @@ struct Decode1Params {
   int G;         // CTAs (one per SM) = tiles of neurons
   int tile_max;  // largest tile
   int nseg;      // 4 KB segments of one projection row (C1 work items per row and projection)
+  int ri8;       // rows are int8 codes; rscale [n][nproj] their fp32 scales
+  const float *rscale;
 };
 
 struct Decode1Layout {

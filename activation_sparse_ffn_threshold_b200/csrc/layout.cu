@@ -82,11 +82,63 @@ cudaError_t layout_impl(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s
   return cudaGetLastError();
 }
 
+// Int8 rows: one CTA per (neuron, projection) row of d fp16 values; in fp32, scale =
+// max|w| / 127 and code = w / scale rounded to nearest even, clamped to +-127 (an
+// all-zero row: scale 0, codes 0).
+__global__ void __launch_bounds__(256) k_quantize_rows(const __half *__restrict__ src, int d,
+                                                       int8_t *__restrict__ q, float *__restrict__ scale) {
+  __shared__ float red[8];
+  const size_t u = blockIdx.x;
+  const __half *w = src + u * d;
+  float m = 0.f;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) m = fmaxf(m, fabsf(__half2float(w[k])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float sc = red[0] / 127.0f;
+  if (threadIdx.x == 0) scale[u] = sc;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    int c = 0;
+    if (sc > 0.f) {
+      c = __float2int_rn(__half2float(w[k]) / sc);
+      c = c > 127 ? 127 : (c < -127 ? -127 : c);
+    }
+    q[u * d + k] = (int8_t)c;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s) {
-  if (h->L.esize == 2) return layout_impl<uint16_t>(h, desc, s);
-  return layout_impl<uint32_t>(h, desc, s);
+  if (!h->L.rows_i8) {
+    if (h->L.esize == 2) return layout_impl<uint16_t>(h, desc, s);
+    return layout_impl<uint32_t>(h, desc, s);
+  }
+  // fp16 rows in a temporary buffer, then their int8 codes and scales
+  const Layout &L = h->L;
+  void *codes = h->rows, *tmp = nullptr;
+  const size_t units = (size_t)L.n * L.nproj;
+  cudaError_t e = cudaMalloc(&tmp, units * L.d * 2);
+  if (e != cudaSuccess) return e;
+  h->rows = tmp;
+  e = layout_impl<uint16_t>(h, desc, s);
+  h->rows = codes;
+  if (e == cudaSuccess) {
+    k_quantize_rows<<<(unsigned)units, 256, 0, s>>>(static_cast<const __half *>(tmp), L.d,
+                                                   static_cast<int8_t *>(codes), h->rscale);
+    e = cudaGetLastError();
+  }
+  const cudaError_t e2 = cudaStreamSynchronize(s);
+  cudaFree(tmp);
+  return e != cudaSuccess ? e : e2;
 }
 
 }  // namespace sfnn

@@ -78,7 +78,7 @@ typedef enum {
 } sfnn_status;
 
 typedef enum { SFNN_RELU = 0, SFNN_REGLU = 1 } sfnn_act;
-typedef enum { SFNN_F32 = 0, SFNN_F16 = 1 } sfnn_dtype;
+typedef enum { SFNN_F32 = 0, SFNN_F16 = 1, SFNN_I8 = 2 } sfnn_dtype;
 
 /*
  * Which kernels the batched path (b > 1, and explicit sets) uses.  The tensor-core
@@ -121,6 +121,19 @@ typedef struct {
     const void *pb;
     const void *pc;
     const float *hotness;
+    /*
+     * Storage of the FFN rows (w_up, w_gate, w_down), given in wdtype as usual:
+     * SFNN_I8 stores them as int8 codes with one fp32 scale per neuron and projection
+     * (weight-only quantization; the predictor, b, x and all arithmetic keep their
+     * types).  The rule, in IEEE fp32: scale = max|w| / 127 over the neuron's row (its
+     * column of w_down), code = w / scale rounded to nearest even, clamped to +-127; an
+     * all-zero row has scale 0.  Needs wdtype = SFNN_F16; such a layer runs the fused
+     * single-token path only (sfnn_forward without explicit sets, sfnn_forward_stack
+     * with b = 1) and sfnn_predict; other calls return SFNN_ERR_UNSUPPORTED.  Any other
+     * value (0 included) stores the rows in wdtype.  No counterpart on the pages beyond
+     * their weight-quantized deployments.
+     */
+    int32_t rows_dtype;
 } sfnn_layer_desc;
 
 /* Read-only facts about a handle (sizes in bytes). */
