@@ -60,6 +60,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--rows", choices=["native", "int8"], default="native",
+                    help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 "
+                         "codes with per-row scales")
+    ap.add_argument("--stack", action="store_true",
+                    help="time the residual stack of the workload's layers (default workload: the "
+                         "4-layer LLaMA-7B-shaped ReGLU stack), one token at a time")
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call: 1 is the single-token decode (the headline); b > 1 "
                          "times the batched union path on b tokens at a time")
@@ -303,8 +309,11 @@ def run_sfnn(args, dist):
     props = torch.cuda.get_device_properties(dev)
     l2 = props.L2_cache_size
     per_token = W.touched_bytes(cfg, expected_tokens_active(cfg))
+    if args.rows == "int8":  # rows of one byte per weight and a scale per row
+        per_token -= expected_tokens_active(cfg) * cfg.nproj * (cfg.d * (e - 1) - 4)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_token))
-    handles = [sf.SparseFFN.from_layer(lay, device=dev) for _ in range(R)]
+    rows = "int8" if args.rows == "int8" else None
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for _ in range(R)]
     info = handles[0].info()
     torch.cuda.synchronize()
 
@@ -368,7 +377,7 @@ def run_sfnn(args, dist):
     launch_us = elapsed_ms * 1e3 / (args.steps * T)
     alg_bytes = float(bytes_tok.mean())
     achieved = alg_bytes / (launch_us / 1e6) / 1e9
-    traffic, tsrc = profiled_traffic()
+    traffic, tsrc = profiled_traffic() if rows is None else (None, None)  # the profile is of fp16 rows
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": "k_decode1 (fused single-token decode), the only kernel the timed region launches; "
@@ -418,7 +427,8 @@ def run_sfnn(args, dist):
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": cfg.description, "batch": 1, "tokens_per_step": T,
+        "config": {"workload": cfg.description + (", int8 rows (per-row fp32 scales)" if rows else ""),
+                   "batch": 1, "tokens_per_step": T,
                    "replicas": R, "l2": f"inputs larger than L2: {R} weight replicas rotated per token, "
                                         f"{bytes_step / T / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{dist.world} (no exchange)",
@@ -581,12 +591,143 @@ def run_batch(args, dist):
     return 0
 
 
+# ---------------------------------------------------------------- the residual stack
+def run_stack(args, dist):
+    """x_{l+1} = x_l + FFN_l(x_l) through the workload's layers, one token per
+    forward_stack call; a step is the workload's tokens, captured in one CUDA graph."""
+    import torch
+
+    import activation_sparse_ffn_threshold_b200 as sf
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[args.workload]
+    T, NL = cfg.tokens, cfg.layers
+    layers = W.make_stack(cfg, seed=args.seed)
+    Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank).astype(np.float32)
+    handles = [sf.SparseFFN.from_layer(lay, device=dev) for lay in layers]
+    info = handles[0].info()
+    e = cfg.esize
+    props = torch.cuda.get_device_properties(dev)
+    l2 = props.L2_cache_size
+    X = torch.from_numpy(Xh).to(dev)
+    Y = torch.empty_like(X)
+    active = np.zeros(NL)
+    for t in range(T):  # per-layer set sizes (the same decisions as the fused path), for the byte count
+        _, _, cnt = sf.forward_stack(handles, X[t], return_sets=True)
+        active += cnt.cpu().numpy().reshape(NL)
+    active /= T
+    bytes_layer_tok = info["predictor_bytes"] + active * info["row_bytes_per_neuron"] + cfg.d * (e + 4)
+    bytes_step = float(bytes_layer_tok.sum()) * T
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for t in range(T):
+            sf.forward_stack(handles, X[t], Y[t], stream=s)
+    torch.cuda.synchronize()
+    launches0 = sum(h.info()["launches"] for h in handles)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for t in range(T):
+            sf.forward_stack(handles, X[t], Y[t], stream=s)
+    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    gpu_uuid = str(props.uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            start.record(s)
+            for _ in range(args.steps):
+                g.replay()
+            stop.record(s)
+        torch.cuda.synchronize()
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    clocks = clk.summary()
+    err = max(h.get_error() for h in handles)
+    if err:
+        raise SystemExit(f"device-side error latched: {err}")
+    t_max = dist.max(elapsed_ms)
+    value = dist.sum(args.steps * T * NL) / (t_max / 1e3)
+    layer_us = elapsed_ms * 1e3 / (args.steps * T * NL)
+    achieved = float(bytes_layer_tok.mean()) / (layer_us / 1e6) / 1e9
+    peak, peak_kind = measured_peak()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None,
+                "kernel": f"k_decode1, one launch per layer and token ({launches_per_step // T} launches per token "
+                          "with the input rounding); duration = CUDA-event time of the region / layer-tokens",
+                "algorithmic_bytes_per_launch": float(bytes_layer_tok.mean()), "avg_launch_us": layer_us,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s", "traffic_source": None}
+    e2e = None
+    if not args.no_e2e:
+        xin = torch.from_numpy(Xh).pin_memory()
+        yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
+        xd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
+        yd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
+        e2e_steps = max(1, min(args.steps, 10))
+
+        def one_step():
+            for t in range(T):
+                xd.copy_(xin[t], non_blocking=True)
+                sf.forward_stack(handles, xd, yd, stream=s)
+                yout[t].copy_(yd, non_blocking=True)
+        with torch.cuda.stream(s):
+            one_step()
+        torch.cuda.synchronize()
+        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        with torch.cuda.stream(s):
+            a.record(s)
+            for _ in range(e2e_steps):
+                one_step()
+            c.record(s)
+        torch.cuda.synchronize()
+        e_max = dist.max(a.elapsed_time(c))
+        e2e = {"value": dist.sum(e2e_steps * T * NL) / (e_max / 1e3), "unit": "layer-tokens/s",
+               "h2d_bytes_per_step": T * cfg.d * 4, "d2h_bytes_per_step": T * cfg.d * 4,
+               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+    line = {
+        "metric": f"sparse-FFN decode layer-tokens/s ({NL}-layer residual stack)", "value": value,
+        "unit": "layer-tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": 1, "layers": NL, "tokens_per_step": T,
+                   "l2": f"inputs larger than L2: {NL} distinct layers per token, "
+                         f"{float(bytes_layer_tok.sum()) / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist.world} (no exchange)",
+                   "mean_active_neurons_per_layer": [float(v) for v in active]},
+        "effective_gbs": bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9,
+        "roofline": roofline,
+        "cpu_baseline": None,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    for h in handles:
+        h.close()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     dist = Dist(args.gpus)
     try:
         if args.impl == "reference":
             return run_reference(args, dist)
+        if args.stack:
+            if args.workload == WORKLOAD:
+                args.workload = "llama7b_reglu_stack"
+            return run_stack(args, dist)
         if args.batch > 1:
             return run_batch(args, dist)
         return run_sfnn(args, dist)
