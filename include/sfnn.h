@@ -154,7 +154,8 @@ typedef struct {
  * (gate, up, and its W_down column as a contiguous row) stored together;
  * A transposed to [r x d]; B transposed to neuron-major [n x r].
  * Requirements: d, n, r >= 1; d and r multiples of 8 (fp16) or 4 (fp32);
- * 1 <= max_batch <= 32; r * max_batch <= 32768 (SFNN_ERR_UNSUPPORTED otherwise).
+ * 1 <= max_batch <= 32; r * max_batch <= 32768; int8 rows: fp16 weights, d a
+ * multiple of 16 and a layer the fused kernel fits (SFNN_ERR_UNSUPPORTED otherwise).
  * Allocates device memory (SFNN_ERR_OOM) and synchronises `stream` before
  * returning.  On error *out is set to NULL.
  */
@@ -186,8 +187,12 @@ SFNN_API sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *i
 
 /*
  * b independent tokens at once (1 <= b <= max_batch): row t of Y equals
- * sfnn_forward of X[t].  The union of the b predicted sets is read once and
- * applied to the tokens active on each row.
+ * sfnn_forward of X[t] (within rounding: the tensor-core path rounds the
+ * activations to fp16).  The union of the b predicted sets is read once and
+ * applied to the tokens active on each row: as a batch's sets accumulate, the
+ * benefit of sparsity shrinks (53ai.com page, section 工程效果), so the rows are
+ * shared by every token that needs them.  The kernels follow sfnn_set_batch_path.
+ * A layer with int8 rows returns SFNN_ERR_UNSUPPORTED.
  *   X      [b x d] wdtype;  Y [b x d] fp32 out
  *   idx    [b x n] int32 out or NULL: token t's set in row t (first counts[t] entries)
  *   counts [b] int32 out or NULL: |S_t|
@@ -198,6 +203,9 @@ SFNN_API sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b,
 /*
  * A stack of layers with a residual stream:  X_{l+1} = X_l + FFN_l(round(X_l)),
  * where round() converts the fp32 residual to the layers' wdtype (nearest even).
+ * The pages name no normalisation between the layers; none is applied.  With
+ * b = 1 every layer runs the fused single-token kernel (unless disabled); with
+ * idx/counts requested or b > 1, the batched path.
  * All layers share d, wdtype and max_batch >= b (and n when idx != NULL).
  *   layers [num_layers] HOST array of handles
  *   X0     [b x d] fp32 in;  XL [b x d] fp32 out (may alias X0)
