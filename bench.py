@@ -387,35 +387,38 @@ def run_sfnn(args, dist):
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "traffic_source": tsrc}
 
-    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+    # end to end through the public API, eager: per step, the step's inputs from pinned
+    # host memory in one copy, one forward call per token, the step's outputs back in one
     e2e = None
     if not args.no_e2e:
         xin = torch.from_numpy(Xh).pin_memory()
         yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
-        xd = torch.empty(cfg.d, dtype=X.dtype, device=dev)
-        yd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
+        xd = torch.empty((T, cfg.d), dtype=X.dtype, device=dev)
+        yd = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
         e2e_steps = max(1, min(args.steps, 20))
+
+        def one_step():
+            xd.copy_(xin, non_blocking=True)
+            for t in range(T):
+                handles[t % R].forward(xd[t], yd[t], stream=s)
+            yout.copy_(yd, non_blocking=True)
         with torch.cuda.stream(s):
-            for t in range(T):  # warm-up
-                xd.copy_(xin[t], non_blocking=True)
-                handles[t % R].forward(xd, yd, stream=s)
-                yout[t].copy_(yd, non_blocking=True)
+            one_step()  # warm-up
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         dist.barrier()
         with torch.cuda.stream(s):
             a.record(s)
             for _ in range(e2e_steps):
-                for t in range(T):
-                    xd.copy_(xin[t], non_blocking=True)
-                    handles[t % R].forward(xd, yd, stream=s)
-                    yout[t].copy_(yd, non_blocking=True)
+                one_step()
             b.record(s)
         torch.cuda.synchronize()
         e_max = dist.max(a.elapsed_time(b))
         e2e = {"value": dist.sum(e2e_steps * T) / (e_max / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": T * cfg.d * e, "d2h_bytes_per_step": T * cfg.d * 4,
-               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+               "steps": e2e_steps,
+               "timing": "CUDA events around the eager loop (per step: one host-to-device copy of the step's "
+                         "inputs, one forward call per token, one device-to-host copy of the outputs), max over ranks"}
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -539,15 +542,15 @@ def run_batch(args, dist):
     if not args.no_e2e:
         xin = torch.from_numpy(Xh).pin_memory()
         yout = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32).pin_memory()
-        xd = torch.empty((b, cfg.d), dtype=X.dtype, device=dev)
-        yd = torch.empty((b, cfg.d), dtype=torch.float32, device=dev)
+        xd = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=X.dtype, device=dev)
+        yd = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32, device=dev)
         e2e_steps = max(1, min(args.steps, 20))
 
-        def one_step():
+        def one_step():  # the step's inputs in one copy, one call per batch, the outputs in one copy
+            xd.copy_(xin, non_blocking=True)
             for i in range(BATCHES_PER_STEP):
-                xd.copy_(xin[i], non_blocking=True)
-                handles[i % R].forward_batch(xd, yd, stream=s)
-                yout[i].copy_(yd, non_blocking=True)
+                handles[i % R].forward_batch(xd[i], yd[i], stream=s)
+            yout.copy_(yd, non_blocking=True)
         with torch.cuda.stream(s):
             one_step()
         torch.cuda.synchronize()
@@ -563,7 +566,9 @@ def run_batch(args, dist):
         e2e = {"value": dist.sum(e2e_steps * BATCHES_PER_STEP * b) / (e_max / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * e,
                "d2h_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * 4,
-               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+               "steps": e2e_steps, "timing": "CUDA events around the eager loop (per step: one host-to-device copy "
+                                            "of the step's inputs, the API calls, one device-to-host copy of the "
+                                            "outputs), max over ranks"}
 
     line = {
         "metric": "sparse-FFN batched decode tokens/s per layer", "value": value, "unit": "tokens/s",
@@ -669,15 +674,15 @@ def run_stack(args, dist):
     if not args.no_e2e:
         xin = torch.from_numpy(Xh).pin_memory()
         yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
-        xd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
-        yd = torch.empty(cfg.d, dtype=torch.float32, device=dev)
+        xd = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+        yd = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
         e2e_steps = max(1, min(args.steps, 10))
 
-        def one_step():
+        def one_step():  # the step's inputs in one copy, one stack call per token, the outputs in one copy
+            xd.copy_(xin, non_blocking=True)
             for t in range(T):
-                xd.copy_(xin[t], non_blocking=True)
-                sf.forward_stack(handles, xd, yd, stream=s)
-                yout[t].copy_(yd, non_blocking=True)
+                sf.forward_stack(handles, xd[t], yd[t], stream=s)
+            yout.copy_(yd, non_blocking=True)
         with torch.cuda.stream(s):
             one_step()
         torch.cuda.synchronize()
@@ -692,7 +697,9 @@ def run_stack(args, dist):
         e_max = dist.max(a.elapsed_time(c))
         e2e = {"value": dist.sum(e2e_steps * T * NL) / (e_max / 1e3), "unit": "layer-tokens/s",
                "h2d_bytes_per_step": T * cfg.d * 4, "d2h_bytes_per_step": T * cfg.d * 4,
-               "steps": e2e_steps, "timing": "CUDA events around the eager loop, max over ranks"}
+               "steps": e2e_steps, "timing": "CUDA events around the eager loop (per step: one host-to-device copy "
+                                            "of the step's inputs, the API calls, one device-to-host copy of the "
+                                            "outputs), max over ranks"}
     line = {
         "metric": f"sparse-FFN decode layer-tokens/s ({NL}-layer residual stack)", "value": value,
         "unit": "layer-tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
