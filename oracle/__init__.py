@@ -17,6 +17,8 @@ Definitions (see ``oracle.c`` for the passages they follow):
               ReGLU act_i = relu(W_gate[i].x + b_i) * (W_up[i].x)
   stack       x_{l+1} = x_l + y_l  (double), next layer's input = x_{l+1}
               rounded to the storage dtype (round to nearest even).
+  look-ahead  the same stack, but layer l+1's set is predicted from layer l's
+              input (its predictor applied one layer early); layer 0's from its own.
 """
 from __future__ import annotations
 
@@ -275,6 +277,38 @@ def forward_stack(layers, x0, masks_other=None, nthreads: int = 1):
             mask, mismatches = arbitrate(z, mask, masks_other[li])
         a, y = ffn_masked(xin, layer.w_up, layer.w_gate, layer.b, layer.w_down, mask, layer.cfg.act, nthreads)
         records.append(dict(x_in=xin, z=z, mask=mask, y=y, mismatches=mismatches))
+        resid = resid + y
+    return resid, records
+
+
+def forward_stack_lookahead(layers, x0, masks_other=None, nthreads: int = 1, qrows=None):
+    """Residual stack whose sets are predicted one layer ahead.
+
+    Follows the asynchronous predictor of DejaVu (53ai.com "sparsity for LLM inference"
+    page, section "如何推理加速"): the next layer's sparsity is predicted one step in
+    advance, so that the prediction can run beside the current layer.  Reading: layer l+1's
+    predictor (its own A, B, c) takes layer l's input u_l = round(x_l); layer 0, which
+    has no earlier input, predicts from u_0.  Everything else is ``forward_stack``:
+    x_{l+1} = x_l + y_l in double, u_{l+1} = round(x_{l+1}), y_l computed on u_l.
+    ``masks_other`` and the records are as in ``forward_stack``; each record adds
+    ``x_pred``, the input its set was predicted from.  ``qrows`` (one ``QRows`` per
+    layer) runs every layer's FFN on int8 rows (``ffn_masked_q``).
+    """
+    dt = layers[0].w_up.dtype
+    resid = np.asarray(x0, dtype=np.float64).copy()
+    records = []
+    for li, layer in enumerate(layers):
+        xin = resid.astype(dt)  # round to nearest even
+        xpred = xin if li == 0 else records[li - 1]["x_in"]
+        h, z, mask = predictor(xpred, layer.A, layer.B, layer.c, nthreads)
+        mismatches = np.empty(0, np.int64)
+        if masks_other is not None:
+            mask, mismatches = arbitrate(z, mask, masks_other[li])
+        if qrows is not None:
+            a, y = ffn_masked_q(xin, qrows[li], layer.b, mask, layer.cfg.act, nthreads)
+        else:
+            a, y = ffn_masked(xin, layer.w_up, layer.w_gate, layer.b, layer.w_down, mask, layer.cfg.act, nthreads)
+        records.append(dict(x_in=xin, x_pred=xpred, z=z, mask=mask, y=y, mismatches=mismatches))
         resid = resid + y
     return resid, records
 

@@ -73,7 +73,7 @@ def _pin_calls(pins):
     for act in ("relu", "reglu"):
         calls.append(lambda act=act: pins.test_all_ones_mask_equals_dense(act))
         calls.append(lambda act=act: pins.test_forward_q_equals_forward_on_an_exact_grid(act))
-    calls += [pins.test_quantizer_hand_values, pins.test_quantizer_invariants]
+    calls += [pins.test_quantizer_hand_values, pins.test_quantizer_invariants, pins.test_lookahead_hand_example]
     return calls
 
 
@@ -122,6 +122,41 @@ def test_mutant_is_caught(name):
                     failures += 1
         finally:
             oracle._lib = saved
+    assert failures > 0, f"no pin caught mutant {name}"
+
+
+# The look-ahead stack is bookkeeping in oracle/__init__.py: its mutants are copies of
+# that module with one mistake, loaded beside the real one (same compiled library).
+PY_SRC = os.path.join(os.path.dirname(HERE), "oracle", "__init__.py")
+PY_MUTANTS = {
+    "lookahead_from_current_input": ('xpred = xin if li == 0 else records[li - 1]["x_in"]', "xpred = xin"),
+    "lookahead_residual_dropped": ("""        records.append(dict(x_in=xin, x_pred=xpred, z=z, mask=mask, y=y, mismatches=mismatches))
+        resid = resid + y""", """        records.append(dict(x_in=xin, x_pred=xpred, z=z, mask=mask, y=y, mismatches=mismatches))
+        resid = y"""),
+    "lookahead_input_not_rounded": ("""        xin = resid.astype(dt)  # round to nearest even
+        xpred = xin if""", """        xin = resid.copy()
+        xpred = xin if"""),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_python_mutant_is_caught(name):
+    src = open(PY_SRC).read()
+    old, new = PY_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    spec = importlib.util.spec_from_loader("_oracle_mutant", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__file__ = PY_SRC
+    exec(compile(src.replace(old, new), PY_SRC, "exec"), mod.__dict__)
+    mod._lib = oracle._load()
+    pins = _pins_module()
+    pins.oracle = mod
+    failures = 0
+    for call in (pins.test_lookahead_hand_example, lambda: pins.test_lookahead_special_cases_equal_the_stack("relu")):
+        try:
+            call()
+        except AssertionError:
+            failures += 1
     assert failures > 0, f"no pin caught mutant {name}"
 
 

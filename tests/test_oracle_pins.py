@@ -12,6 +12,9 @@
   with an exponential, h and z against an independent numpy evaluation;
 * the exact fp16 decoding against numpy for all 65536 bit patterns;
 * closed forms: one active neuron, the empty set, a tie and a NaN logit;
+* the look-ahead stack (layer l+1's set predicted from layer l's input): a
+  two-layer example worked by hand where predicting one layer early changes the
+  set and the output, and the special cases where it must equal the plain stack;
 * int8 rows: the quantizer's codes and scales worked by hand (ties to even, zero
   rows), its error bound, and the int8-row step equal to the fp16 step on weights
   that lie exactly on an int8 grid.
@@ -111,6 +114,59 @@ def test_golden_stack_two_layers():
     assert [r["x_in"].astype(np.float64).tolist() for r in recs] == e["layer_inputs"]
     assert [np.flatnonzero(r["mask"]).tolist() for r in recs] == e["sets"]
     assert xL.tolist() == e["x_out"]
+
+
+# ------------------------------------------------------------------ look-ahead stack
+def _lookahead_hand_layers():
+    """Two ReLU layers, d = n = r = 2, every value exact in fp16.
+
+    Layer 0: A = B = I, c = 0, W_up = I, b = 0, W_down = [[-2, 0], [2, 0]].
+    Layer 1: A = B = I, c = 0, W_up = -I, b = 0, W_down = I.
+    With x0 = (1, -1): h = relu(x0) = (1, 0), so layer 0's set is {0} and
+    y_0 = 1 * W_down[:, 0] = (-2, 2), x_1 = (-1, 1).
+    Plain stack: layer 1 predicts from x_1: h = (0, 1), set {1}; its activation is
+    relu(-x_1[1]) = 0, so x_2 = x_1 = (-1, 1).
+    Look-ahead: layer 1 predicts from x0: h = (1, 0), set {0}; its activation is
+    relu(-x_1[0]) = 1, so y_1 = (1, 0) and x_2 = (0, 1).
+    """
+    f = lambda v: np.asarray(v, dtype=np.float16)
+    eye = np.eye(2)
+    z2 = np.zeros(2)
+    l0 = _L("relu", f(eye), None, f(z2), f([[-2, 0], [2, 0]]), f(eye), f(eye), f(z2))
+    l1 = _L("relu", f(-eye), None, f(z2), f(eye), f(eye), f(eye), f(z2))
+    return [l0, l1]
+
+
+def test_lookahead_hand_example():
+    layers = _lookahead_hand_layers()
+    x0 = np.array([1.0, -1.0])
+    xl, recs = oracle.forward_stack_lookahead(layers, x0)
+    assert [np.flatnonzero(r["mask"]).tolist() for r in recs] == [[0], [0]]
+    assert [r["y"].tolist() for r in recs] == [[-2.0, 2.0], [1.0, 0.0]]
+    assert xl.tolist() == [0.0, 1.0]
+    xs, recs_s = oracle.forward_stack(layers, x0)
+    assert [np.flatnonzero(r["mask"]).tolist() for r in recs_s] == [[0], [1]]
+    assert xs.tolist() == [-1.0, 1.0]
+
+
+@pytest.mark.parametrize("act", ["relu", "reglu"])
+def test_lookahead_special_cases_equal_the_stack(act):
+    rng = np.random.default_rng(31)
+    layers = [_rand_layer(rng, 24, 40, 8, act, np.float16) for _ in range(3)]
+    x0 = rng.standard_normal(24)
+    # one layer: nothing to look ahead of
+    a, ra = oracle.forward_stack_lookahead(layers[:1], x0)
+    b, rb = oracle.forward_stack(layers[:1], x0)
+    assert np.array_equal(a, b) and np.array_equal(ra[0]["mask"], rb[0]["mask"])
+    # layers that add nothing keep every input equal to u_0, so predicting from the
+    # previous input is predicting from the current one
+    for L in layers[:2]:
+        L.w_down = np.zeros_like(L.w_down)
+    a, ra = oracle.forward_stack_lookahead(layers, x0)
+    b, rb = oracle.forward_stack(layers, x0)
+    assert np.array_equal(a, b)
+    assert all(np.array_equal(p["mask"], q["mask"]) for p, q in zip(ra, rb))
+    assert np.any(a != x0)  # the last layer does add something
 
 
 # ------------------------------------------------------------------ dense identity
