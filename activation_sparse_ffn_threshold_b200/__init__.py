@@ -80,6 +80,7 @@ def load_library():
         "sfnn_forward": ([P, P, P, P, P, P], S),
         "sfnn_forward_batch": ([P, P, I, P, P, P, P], S),
         "sfnn_forward_stack": ([P, I, P, I, P, P, P, P], S),
+        "sfnn_forward_stack_lookahead": ([P, I, P, I, P, P, P, P], S),
         "sfnn_set_batch_path": ([P, I], S),
         "sfnn_set_fused_decode": ([P, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
@@ -300,8 +301,12 @@ def predict_noalloc(x, A, B, c, idx=None, count=None, stream=None):
     return idx, count
 
 
-def forward_stack(layers, X0, XL=None, idx=None, counts=None, return_sets: bool = False, stream=None):
-    """Residual stack X_{l+1} = X_l + FFN_l(round(X_l)); X0 [b, d] (or [d]) fp32 CUDA tensor."""
+def forward_stack(layers, X0, XL=None, idx=None, counts=None, return_sets: bool = False, lookahead: bool = False,
+                  stream=None):
+    """Residual stack X_{l+1} = X_l + FFN_l(round(X_l)); X0 [b, d] (or [d]) fp32 CUDA tensor.
+
+    ``lookahead``: layer l+1's set is predicted from layer l's input, one layer early
+    (sfnn_forward_stack_lookahead)."""
     lib = load_library()
     if X0.dtype != torch.float32 or X0.device.type != "cuda" or not X0.is_contiguous():
         raise TypeError("X0 must be a contiguous fp32 CUDA tensor")
@@ -313,6 +318,7 @@ def forward_stack(layers, X0, XL=None, idx=None, counts=None, return_sets: bool 
         counts = counts if counts is not None else torch.empty((len(layers), b), dtype=torch.int32,
                                                                device=X0.device)
     arr = (ctypes.c_void_p * len(layers))(*[l.handle.value for l in layers])
-    _check(lib.sfnn_forward_stack(arr, len(layers), _ptr(X0), b, _ptr(XL), _ptr(idx), _ptr(counts),
-                                  _stream(stream)), "sfnn_forward_stack")
+    name = "sfnn_forward_stack_lookahead" if lookahead else "sfnn_forward_stack"
+    _check(getattr(lib, name)(arr, len(layers), _ptr(X0), b, _ptr(XL), _ptr(idx), _ptr(counts), _stream(stream)),
+           name)
     return (XL, idx, counts) if return_sets else XL

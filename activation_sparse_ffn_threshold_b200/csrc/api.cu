@@ -33,7 +33,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -87,12 +87,22 @@ void record_if(cudaEvent_t ev, cudaStream_t s) {
     cudaEventRecord(ev, s);
 }
 
-// The shared body of forward / forward_batch / one stack layer.
-sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int32_t *idx, const int32_t *count,
+// Where a layer's active sets come from.
+enum SetSource {
+  kSetPredict,  // its own predictor on X
+  kSetGiven,    // a caller's index list
+  kSetReady,    // h->mask already holds them (predicted one layer ahead)
+};
+
+// The shared body of forward / forward_batch / one stack layer.  `ahead`, if given, is
+// the next layer of a look-ahead stack: its predictor runs on this layer's X after this
+// layer's sets are consumed and before the reduce overwrites the next input.
+sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const int32_t *idx, const int32_t *count,
                       int32_t *idx_out, int32_t *cnt_out, const float *resid, float *Y, void *xnext,
-                      cudaStream_t s) {
+                      sfnn_ctx *ahead, cudaStream_t s) {
   cudaEvent_t before = h->prof_before, after = h->prof_after;
-  const bool fused = b == 1 && predict && !idx_out && !cnt_out && h->fused_ok && h->fused_on;
+  const bool predict = src == kSetPredict;
+  const bool fused = b == 1 && predict && !ahead && !idx_out && !cnt_out && h->fused_ok && h->fused_on;
   if (h->L.rows_i8 && !fused) return SFNN_ERR_UNSUPPORTED;  // int8 rows: the fused path only
   h->prof_before = h->prof_after = nullptr;
   record_if(before, s);
@@ -115,7 +125,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
   } else if (predict) {
     SFNN_TRY(launch_hidden(h, X, b, s));
     SFNN_TRY(launch_logits(h, b, s));
-  } else {
+  } else if (src == kSetGiven) {
     SFNN_TRY(launch_mask_from_idx(h, idx, count, s));
   }
   SFNN_TRY(launch_compact(h, b, idx_out, cnt_out, s));
@@ -126,9 +136,14 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, bool predict, const int
     SFNN_TRY(launch_up(h, X, b, s));
     SFNN_TRY(launch_down(h, b, &splits, s));
   }
+  if (ahead) {  // h->mask is consumed (compacted): the next layer may overwrite its own
+    SFNN_TRY(launch_hidden(ahead, X, b, s));
+    SFNN_TRY(launch_logits(ahead, b, s));
+    ahead->launches += 2;
+  }
   SFNN_TRY(launch_reduce(h, b, splits, resid, Y, xnext, s));
   record_if(after, s);
-  h->launches += predict ? 6 : 5;
+  h->launches += 4 + (predict ? 2 : (src == kSetGiven ? 1 : 0));
   return SFNN_OK;
 }
 
@@ -163,6 +178,53 @@ void plan_decode1(sfnn_ctx *h, int G) {
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
   h->fused_on = true;
+}
+
+// Arguments shared by the two stack calls.
+sfnn_status check_stack(const sfnn_handle *layers, int num_layers, const float *X0, const float *XL, int b,
+                        const int32_t *idx) {
+  if (!layers || num_layers < 1 || !X0 || !XL || b < 1) return SFNN_ERR_INVALID_ARG;
+  const sfnn_ctx *l0 = layers[0];
+  if (!l0) return SFNN_ERR_INVALID_ARG;
+  for (int l = 0; l < num_layers; ++l) {
+    const sfnn_ctx *hl = layers[l];
+    if (!hl || hl->L.d != l0->L.d || hl->L.dt != l0->L.dt || hl->device != l0->device || b > hl->max_batch)
+      return SFNN_ERR_INVALID_ARG;
+    if (idx && hl->L.n != l0->L.n) return SFNN_ERR_INVALID_ARG;
+  }
+  if (!same_device(l0)) return SFNN_ERR_INVALID_ARG;
+  return SFNN_OK;
+}
+
+// The look-ahead kernel's view of the next layer (null: none).
+AheadParams ahead_params(const sfnn_ctx *nx) {
+  AheadParams Q{};
+  if (!nx) return Q;
+  Q.At = nx->At;
+  Q.Bt = nx->Bt;
+  Q.cvec = nx->cvec;
+  Q.bias = nx->bias;
+  Q.hbuf = nx->h;
+  Q.r = nx->L.r;
+  Q.n = nx->L.n;
+  Q.tile_max = nx->d1.tile_max;
+  Q.list_out = nx->alist;
+  Q.cnt_out = nx->acnt;
+  return Q;
+}
+
+// Every launch of a fused look-ahead stack fits: every layer runs its fused kernel, all
+// with the same tiles (a tile's list is written and read by the same CTA), and each
+// (layer, next layer) pair's shared-memory plan fits one CTA per SM.
+bool ahead_fused_ok(const sfnn_handle *layers, int num_layers) {
+  for (int l = 0; l < num_layers; ++l) {
+    const sfnn_ctx *hl = layers[l];
+    if (!hl->fused_ok || !hl->fused_on || hl->d1.G != layers[0]->d1.G) return false;
+    if (decode_ahead_layout(hl->d1, ahead_params(l + 1 < num_layers ? layers[l + 1] : nullptr)).total >
+        (size_t)kDecodeSmemCap)
+      return false;
+  }
+  return decode_ahead_layout(layers[0]->d1, ahead_params(layers[0])).total <= (size_t)kDecodeSmemCap;
 }
 
 }  // namespace
@@ -269,6 +331,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
       {(void **)&h->bar, sizeof(uint64_t), false},
+      {(void **)&h->alist, n * sizeof(int2), false},
+      {(void **)&h->acnt, (size_t)G * 4, false},
       {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_i8 && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
       {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_i8 && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
   };
@@ -286,9 +350,12 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->err, 0, 4, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->ucount, 0, 4, s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, sizeof(uint64_t), s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->alist, 0, n * sizeof(int2), s);
+  if (ce == cudaSuccess) ce = cudaMemsetAsync(h->acnt, 0, (size_t)G * 4, s);
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();
+  if (ce == cudaSuccess) ce = configure_decode_ahead();
   if (ce == cudaSuccess && h->hact) ce = configure_tc_batch();
   if (ce == cudaSuccess) plan_decode1(h, G);
   if (ce == cudaSuccess) ce = launch_layout(h, desc, s);
@@ -328,30 +395,23 @@ sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *idx, const
                          sfnn_stream_t stream) {
   if (!h || !x || !y || (idx && !count) || !aligned16(x)) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
-  return run_layer(h, x, 1, idx == nullptr, idx, count, nullptr, nullptr, nullptr, y, nullptr,
-                   reinterpret_cast<cudaStream_t>(stream));
+  return run_layer(h, x, 1, idx ? kSetGiven : kSetPredict, idx, count, nullptr, nullptr, nullptr, y, nullptr,
+                   nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b, float *Y, int32_t *idx, int32_t *counts,
                                sfnn_stream_t stream) {
   if (!h || !X || !Y || b < 1 || b > h->max_batch || !aligned16(X)) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
-  return run_layer(h, X, b, true, nullptr, nullptr, idx, counts, nullptr, Y, nullptr,
+  return run_layer(h, X, b, kSetPredict, nullptr, nullptr, idx, counts, nullptr, Y, nullptr, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_layers, const float *X0, int32_t b, float *XL,
                                int32_t *idx, int32_t *counts, sfnn_stream_t stream) {
-  if (!layers || num_layers < 1 || !X0 || !XL || b < 1) return SFNN_ERR_INVALID_ARG;
+  const sfnn_status chk = check_stack(layers, num_layers, X0, XL, b, idx);
+  if (chk != SFNN_OK) return chk;
   const sfnn_ctx *l0 = layers[0];
-  if (!l0) return SFNN_ERR_INVALID_ARG;
-  for (int l = 0; l < num_layers; ++l) {
-    const sfnn_ctx *hl = layers[l];
-    if (!hl || hl->L.d != l0->L.d || hl->L.dt != l0->L.dt || hl->device != l0->device || b > hl->max_batch)
-      return SFNN_ERR_INVALID_ARG;
-    if (idx && hl->L.n != l0->L.n) return SFNN_ERR_INVALID_ARG;
-  }
-  if (!same_device(l0)) return SFNN_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t bd = (int64_t)b * l0->L.d;
   SFNN_TRY(launch_round(X0, layers[0]->xin, l0->L.dt, bd, s));
@@ -363,7 +423,51 @@ sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_layers, co
     int32_t *cnt_l = counts ? counts + (size_t)l * b : nullptr;
     void *xnext = l + 1 < num_layers ? layers[l + 1]->xin : nullptr;
     sfnn_status st =
-        run_layer(hl, hl->xin, b, true, nullptr, nullptr, idx_l, cnt_l, l == 0 ? X0 : XL, XL, xnext, s);
+        run_layer(hl, hl->xin, b, kSetPredict, nullptr, nullptr, idx_l, cnt_l, l == 0 ? X0 : XL, XL, xnext, nullptr, s);
+    if (st != SFNN_OK) return st;
+  }
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_layers, const float *X0, int32_t b,
+                                         float *XL, int32_t *idx, int32_t *counts, sfnn_stream_t stream) {
+  sfnn_status st = check_stack(layers, num_layers, X0, XL, b, idx);
+  if (st != SFNN_OK) return st;
+  sfnn_ctx *l0 = layers[0];
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  SFNN_TRY(launch_round(X0, l0->xin, l0->L.dt, (int64_t)b * l0->L.d, s));
+  l0->launches += 1;
+  if (b == 1 && !idx && !counts && ahead_fused_ok(layers, num_layers)) {
+    // launch 0: layer 0's predictor on u_0; launch l + 1: layer l's rows and layer l+1's predictor
+    for (int l = -1; l < num_layers; ++l) {
+      sfnn_ctx *cur = l >= 0 ? layers[l] : l0;
+      sfnn_ctx *nxt = l + 1 < num_layers ? layers[l + 1] : nullptr;
+      Decode1Params P = cur->d1;
+      P.x = cur->xin;
+      P.y = l >= 0 ? XL : nullptr;
+      P.resid = l == 0 ? X0 : XL;
+      P.xnext = nxt && l >= 0 ? nxt->xin : nullptr;
+      AheadParams Q = ahead_params(nxt);
+      Q.list_in = l >= 0 ? cur->alist : nullptr;
+      Q.cnt_in = l >= 0 ? cur->acnt : nullptr;
+      SFNN_TRY(launch_decode_ahead(P, Q, s, true));
+      cur->launches += 1;
+    }
+    return SFNN_OK;
+  }
+  for (int l = 0; l < num_layers; ++l) {
+    sfnn_ctx *hl = layers[l];
+    const int n = hl->L.n;
+    if (l == 0) {  // layer 0 has no earlier input: its own
+      SFNN_TRY(launch_hidden(hl, hl->xin, b, s));
+      SFNN_TRY(launch_logits(hl, b, s));
+      hl->launches += 2;
+    }
+    int32_t *idx_l = idx ? idx + (size_t)l * b * n : nullptr;
+    int32_t *cnt_l = counts ? counts + (size_t)l * b : nullptr;
+    sfnn_ctx *nxt = l + 1 < num_layers ? layers[l + 1] : nullptr;
+    st = run_layer(hl, hl->xin, b, kSetReady, nullptr, nullptr, idx_l, cnt_l, l == 0 ? X0 : XL, XL,
+                   nxt ? nxt->xin : nullptr, nxt, s);
     if (st != SFNN_OK) return st;
   }
   return SFNN_OK;

@@ -53,6 +53,8 @@ struct sfnn_ctx {
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
   uint64_t *bar;     // grid barrier arrival counter of the fused kernel
+  int2 *alist;       // [n] look-ahead stack: this layer's predicted active lists per tile
+  int32_t *acnt;     // [G]   (storage position, bias) pairs and counts, from the launch before
   bool fused_ok;     // the fused single-token kernel fits this layer
   bool fused_on;     // ... and is enabled (sfnn_set_fused_decode)
   sfnn::Decode1Params d1;  // its launch plan (pointers to x/y filled per call)

@@ -10,6 +10,7 @@ namespace sfnn {
 
 constexpr int kDecode1Threads = 512;  // 16 warps per CTA, one CTA per SM
 constexpr int kDecode1BStages = 4;     // B^T rows staged per warp (thread-private shared staging)
+constexpr int kDecodeSmemCap = 227 * 1024;  // opt-in dynamic shared memory of one CTA
 
 // W_down rows in flight per thread in the down phase, by 16-byte chunks per thread and row
 __host__ __device__ constexpr int decode1_dstages(int maxm) { return maxm == 1 ? 8 : (maxm == 2 ? 4 : 2); }
@@ -93,7 +94,31 @@ __host__ __device__ inline int decode1_tile_start(int c, int n, int G) {
   return c * q + (c < rr ? c : rr);
 }
 
+// The look-ahead stack kernel (decode_ahead.cu): layer l's FFN on the set predicted by
+// the previous launch, beside layer l+1's predictor on the same input.
+struct AheadParams {
+  const void *At, *Bt, *cvec, *bias;  // the next layer's predictor and gated bias (At null: none)
+  float *hbuf;                        // [r] its hidden layer (scratch)
+  int r, n, tile_max;                 // its sizes; it has the same G tiles as this layer
+  const int2 *list_in;                // this layer's active lists: tile c's from position
+  const int32_t *cnt_in;              //   start(c), (storage position, bias) pairs; [G] counts
+                                      //   (list_in null: no FFN in this launch)
+  int2 *list_out;                     // the next layer's lists, written for the next launch
+  int32_t *cnt_out;
+};
+
+// The shared-memory plan of one look-ahead launch: the single-layer plan sized for this
+// layer's d and C1 segments, the next layer's r, and the larger of the two tiles.
+__host__ __device__ inline Decode1Layout decode_ahead_layout(const Decode1Params &P, const AheadParams &Q) {
+  Decode1Params M = P;
+  M.r = Q.At ? Q.r : (P.dt == SFNN_F16 ? 8 : 4);
+  M.tile_max = P.tile_max > Q.tile_max ? P.tile_max : Q.tile_max;
+  return decode1_layout(M);
+}
+
 cudaError_t configure_decode1();
+cudaError_t configure_decode_ahead();
+cudaError_t launch_decode_ahead(const Decode1Params &P, const AheadParams &Q, cudaStream_t stream, bool pdl);
 int decode1_blocks_per_sm(const Decode1Params &P);  // co-resident CTAs per SM for this plan
 cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl);
 cudaError_t launch_barrier_bump(uint64_t *count, cudaStream_t stream);

@@ -1,0 +1,473 @@
+// decode_ahead.cu -- the fused decode kernel of a residual stack whose active sets are
+// predicted one layer ahead.
+//
+// DejaVu's predictor runs asynchronously: the next layer's sparsity is predicted one
+// step in advance, so the prediction does not sit in front of the layer that uses it
+// (53ai.com "sparsity for LLM inference" page, section "如何推理加速").  Here layer
+// l+1's predictor takes layer l's input u_l, which lets one launch per layer carry both
+// halves (one CTA of 16 warps per SM, as the single-layer kernel):
+//
+//   P1  u_l and the CTA's active list of layer l (written by the previous launch) into
+//       shared memory; h' = relu(A'^T u_l) for the CTA's rows of layer l+1's A' (one warp
+//       per row, its first batch requested before the previous kernel ends); C1 / C2 on
+//       layer l's active rows of the tile, exactly as in the single-layer kernel; the
+//       CTA's partial y to global memory; the first B'^T rows of layer l+1's tile
+//       requested into the staging region C2 has left.
+//   grid barrier (the launch's only one)
+//   P2  the fixed-order column reduce of the partials -> y_l (+ residual), u_{l+1};
+//       z' = B'^T h' + c' on layer l+1's tile -> its active list, kept in global memory
+//       for the next launch.
+//
+// Against the single-layer kernel, each layer drops one grid barrier and the hidden
+// layer's phase from its critical chain, and the column reduce overlaps the logits.
+// CTA c owns tile c of every layer, so a tile's list is written and read by the same CTA
+// in consecutive launches.  The stack's first launch runs P1/P2's predictor half only
+// (layer 0 on u_0); its last launch has no next predictor.  Dot products keep the
+// single-layer kernel's orders, so a layer's y on a given set is the same to the bit.
+#include "async.cuh"
+#include "common.cuh"
+#include "decode1.cuh"
+#include "decode_dev.cuh"
+
+namespace sfnn {
+namespace {
+
+template <typename T, int ACT, int MAXM, typename R>
+__global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, const AheadParams Q) {
+  constexpr int V = Elem<T>::kVec;
+  constexpr bool I8 = sizeof(R) == 1;  // int8 rows: codes with per-row scales
+  constexpr int VR = 16 / sizeof(R);   // row elements per 16-byte chunk
+  constexpr int MAXH = 4;              // chunks of h' per lane (r <= 128 * V)
+  constexpr int DB = kDecode1BStages;
+  constexpr int DD = decode1_dstages(MAXM);
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Decode1Layout L = decode_ahead_layout(P, Q);
+  unsigned char *xs = smem + L.x;
+  float *bias_s = reinterpret_cast<float *>(smem + L.bias);  // b of this layer's active rows
+  float *c_s = reinterpret_cast<float *>(smem + L.c);        // c' of the next layer's tile
+  int *act_s = reinterpret_cast<int *>(smem + L.act);
+  float *a_s = reinterpret_cast<float *>(smem + L.a);  // activations, then b' of the next tile
+  float *dots = reinterpret_cast<float *>(smem + L.dots);
+  float *red2 = reinterpret_cast<float *>(smem + L.red2);
+  uint32_t *bits = reinterpret_cast<uint32_t *>(smem + L.bits);
+  int *wpref = reinterpret_cast<int *>(smem + L.wpref);
+  float *h_s = reinterpret_cast<float *>(smem + L.h);
+  int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
+  int *flag_s = cnt_s + 1;
+  int *ncnt_s = cnt_s + 2;
+  unsigned char *bstage = smem + L.bstage;
+  unsigned char *dstage = smem + L.dstage;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, G = P.G;
+  const bool cur = Q.list_in != nullptr, next = Q.At != nullptr;
+  const int t0 = decode1_tile_start(c, P.n, G);  // this layer's tile
+  const int tn = decode1_tile_start(c + 1, P.n, G) - t0;
+  const int u0 = decode1_tile_start(c, Q.n, G);  // the next layer's tile
+  const int un = next ? decode1_tile_start(c + 1, Q.n, G) - u0 : 0;
+  const int d = P.d, r = Q.r, nproj = P.nproj;
+  const int nch_d = d / V, nch_r = next ? r / V : 0;
+  const T *At = static_cast<const T *>(Q.At);
+  const T *Bt = static_cast<const T *>(Q.Bt);
+  const R *rows = static_cast<const R *>(P.rows);
+
+  pdl_launch_dependents();
+  const int j0 = c + G * warp;  // this warp's first row of A'^T
+
+  // Weights only until griddepcontrol.wait: the first batch of the warp's row of A'^T,
+  // and c', b' at tile position tid.
+  uint4 w0[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int ch = lane + 32 * u;
+    if (next && j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
+  }
+  const T *cp = static_cast<const T *>(Q.cvec);
+  const T *bp = static_cast<const T *>(Q.bias);
+  T c_first = from_f<T>(0.f), b_first = from_f<T>(0.f);
+  if (tid < un) {
+    c_first = cp[u0 + tid];
+    b_first = bp[u0 + tid];
+  }
+  for (int i = tid; i < (Q.tile_max + 31) / 32; i += kT) bits[i] = 0u;
+
+  pdl_wait();  // u_l, this layer's lists and every buffer written here belong to earlier kernels until here
+  for (int i = tid; i < nch_d; i += kT)
+    *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
+        __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+  if (cur) {
+    for (int i = tid; i < tn; i += kT) {  // the whole tile's slots: the count arrives with them
+      const int2 e = __ldcg(Q.list_in + t0 + i);
+      act_s[i] = e.x;
+      bias_s[i] = __int_as_float(e.y);
+    }
+    if (tid == 0) *cnt_s = __ldcg(Q.cnt_in + c);
+  }
+  __syncthreads();
+  const int cnt = cur ? min(max(*cnt_s, 0), tn) : 0;
+
+  // ---------------------------------------------------------------- A': next hidden layer
+  if (next) {
+    for (int j = j0; j < r; j += G * kW) {
+      const T *row = At + (size_t)j * d;
+      float acc = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
+      for (int cb = 0; cb < nch_d; cb += 32 * 16) {
+        if (j != j0 || cb != 0) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int ch = cb + lane + 32 * u;
+            if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int ch = cb + lane + 32 * u;
+          if (ch < nch_d) acc = dot_chunk_smem<T>(w0[u], xs, ch, acc);
+        }
+      }
+      const float hs = warp_sum(acc);
+      if (lane == 0) Q.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
+    }
+  }
+
+  // C2's rows of W_down stream through DD shared-memory stages private to each thread
+  auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
+  auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
+    if (k < cnt) {
+      const R *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * d;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const int ch = tid + kT * m;
+        if (ch < nch_d) {
+          if (I8)
+            cp_async8(dslot(s, m), row + (size_t)ch * V);
+          else
+            cp_async16(dslot(s, m), row + (size_t)ch * V);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+  float acc[MAXM][V];
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m)
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
+  if (cur) {
+    // -------------------------------------------------------------- C1: up / gate dots
+    constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;
+    constexpr int D = 2;
+    constexpr int SU = kSegChunks / 32;
+    const int nseg = P.nseg;
+    const int per_row = NPG * nseg;
+    const int items = cnt * per_row;
+    const int nch_r8 = d / VR;
+    uint4 wc[D][SU];
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+      const int it = warp + kW * s;
+      if (it < items) {
+        const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+        const R *row = rows + ((size_t)act_s[k] * nproj + pj) * d;
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int ch = sg * kSegChunks + lane + 32 * u;
+          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < DD; ++s) stage_d(s, s);
+    for (int ib = warp; ib < items; ib += D * kW) {
+#pragma unroll
+      for (int s = 0; s < D; ++s) {
+        const int it = ib + kW * s;
+        if (it < items) {
+          const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+          float a = 0.f;
+#pragma unroll
+          for (int u = 0; u < SU; ++u) {
+            const int ch = sg * kSegChunks + lane + 32 * u;
+            if (ch < nch_r8) {
+              if (I8)
+                a = dot_chunk_i8(wc[s][u], xs, ch, a);
+              else
+                a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
+            }
+          }
+          const int itn = it + D * kW;
+          if (itn < items) {
+            const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
+            const R *row = rows + ((size_t)act_s[kn] * nproj + pjn) * d;
+#pragma unroll
+            for (int u = 0; u < SU; ++u) {
+              const int ch = sgn * kSegChunks + lane + 32 * u;
+              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
+            }
+          }
+          a = warp_sum(a);
+          if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+        }
+      }
+    }
+    __syncthreads();
+    for (int k = tid; k < cnt; k += kT) {
+      float g = 0.f, u = 0.f;
+      for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
+      if (ACT == SFNN_REGLU)
+        for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
+      float sd = 1.f;
+      if (I8) {
+        const float *sc = P.rscale + (size_t)act_s[k] * nproj;
+        g *= sc[0];
+        if (ACT == SFNN_REGLU) u *= sc[1];
+        sd = sc[nproj - 1];
+      }
+      const float pre = g + bias_s[k];
+      const float relu = pre > 0.f ? pre : 0.f;
+      a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
+      if (I8) a_s[k] *= sd;
+    }
+    __syncthreads();
+
+    // -------------------------------------------------------------- C2: down projection
+    for (int kb = 0; kb < cnt; kb += DD) {
+#pragma unroll
+      for (int s = 0; s < DD; ++s) {
+        const int k = kb + s;
+        if (k < cnt) {
+          cp_async_wait<DD - 1>();
+          const float a = a_s[k];
+#pragma unroll
+          for (int m = 0; m < MAXM; ++m) {
+            if (tid + kT * m < nch_d) {
+              float f[V];
+              if (I8) {
+                const uint2 q = *reinterpret_cast<const uint2 *>(dslot(s, m));
+#pragma unroll
+                for (int v = 0; v < V; ++v) f[v] = (float)(int8_t)((v < 4 ? q.x : q.y) >> (8 * (v & 3)));
+              } else {
+                unpack<T>(*reinterpret_cast<const uint4 *>(dslot(s, m)), f);
+              }
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[m][v] = fmaf(a, f[v], acc[m][v]);
+            }
+          }
+          stage_d(s, k + DD);
+        }
+      }
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();  // C2's stages and activations are consumed: the region takes B'^T rows
+
+  // The next layer's B'^T rows stream through DB stages private to each warp, as in the
+  // single-layer kernel; the first DB rows land during the partial write and the barrier.
+  unsigned char *bst = bstage + (size_t)warp * DB * nch_r * 16;
+  auto stage_b = [&](int s, int p) {  // row p of the next tile into stage s; always one group
+    if (p < un) {
+#pragma unroll
+      for (int m = 0; m < MAXH; ++m) {
+        const int ch = lane + 32 * m;
+        if (ch < nch_r) cp_async16(bst + ((size_t)s * nch_r + ch) * 16, Bt + (size_t)(u0 + p) * r + (size_t)ch * V);
+      }
+    }
+    cp_async_commit();
+  };
+  if (next) {
+#pragma unroll
+    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
+    if (tid < un) {
+      c_s[tid] = to_f<T>(c_first);
+      a_s[tid] = to_f<T>(b_first);
+    }
+    for (int i = tid + kT; i < un; i += kT) {
+      c_s[i] = to_f<T>(cp[u0 + i]);
+      a_s[i] = to_f<T>(bp[u0 + i]);
+    }
+  }
+  if (cur) {
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const int ch = tid + kT * m;
+      if (ch < nch_d) {
+        float4 *dst = reinterpret_cast<float4 *>(P.part + (size_t)c * d + (size_t)ch * V);
+#pragma unroll
+        for (int v = 0; v < V; v += 4) dst[v / 4] = make_float4(acc[m][v], acc[m][v + 1], acc[m][v + 2], acc[m][v + 3]);
+      }
+    }
+  }
+  if (!cta_grid_sync(P, flag_s)) {
+    cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+    return;
+  }
+
+  // ---------------------------------------------------------------- P2
+  if (next)  // h' once per CTA from L2; its loads overlap the reduce's
+    for (int i = tid; i < r / 4; i += kT)
+      reinterpret_cast<float4 *>(h_s)[i] = __ldcg(reinterpret_cast<const float4 *>(Q.hbuf) + i);
+  if (cur) {  // y_l: CTA c sums a column slice of all G partials in a fixed order
+    const int CW = (d + G - 1) / G;
+    const int col0 = c * CW;
+    const int ncol = max(0, min(CW, d - col0));
+    for (int cb = 0; cb < ncol; cb += kT) {
+      const int width = min(kT, ncol - cb);
+      const int gi = tid / width, j = tid % width;
+      const int ngu = kT / width;
+      if (gi < ngu) {
+        const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
+        const float *src = P.part + col0 + cb + j;
+        float sum = 0.f;
+        int k = k0;
+        for (; k + 8 <= k1; k += 8) {
+          float v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(k + u) * d);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) sum += v[u];
+        }
+        for (; k < k1; ++k) sum += __ldcg(src + (size_t)k * d);
+        red2[gi * width + j] = sum;
+      }
+      __syncthreads();
+      if (tid < width) {
+        float tot = 0.f;
+        for (int g = 0; g < ngu; ++g) tot += red2[g * width + tid];
+        const int col = col0 + cb + tid;
+        if (P.resid) tot = P.resid[col] + tot;
+        P.y[col] = tot;
+        if (P.xnext) static_cast<T *>(P.xnext)[col] = from_f<T>(tot);
+      }
+      __syncthreads();
+    }
+  }
+  if (!next) return;
+  __syncthreads();
+
+  // ---------------------------------------------------------------- B': next logits
+  {
+    float hreg[MAXH][V];
+#pragma unroll
+    for (int m = 0; m < MAXH; ++m) {
+      const int ch = lane + 32 * m;
+#pragma unroll
+      for (int v = 0; v < V; v += 4) {
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ch < nch_r) q = *reinterpret_cast<const float4 *>(h_s + (size_t)ch * V + v);
+        hreg[m][v] = q.x;
+        hreg[m][v + 1] = q.y;
+        hreg[m][v + 2] = q.z;
+        hreg[m][v + 3] = q.w;
+      }
+    }
+    for (int pb = warp; pb < un; pb += DB * kW) {
+#pragma unroll
+      for (int s = 0; s < DB; ++s) {
+        const int p = pb + kW * s;
+        if (p < un) {
+          cp_async_wait<DB - 1>();
+          float a = 0.f;
+#pragma unroll
+          for (int m = 0; m < MAXH; ++m) {
+            const int ch = lane + 32 * m;
+            if (ch < nch_r)
+              a = dot_chunk<T>(*reinterpret_cast<const uint4 *>(bst + ((size_t)s * nch_r + ch) * 16), hreg[m], a);
+          }
+          stage_b(s, p + DB * kW);
+          const float z = warp_sum(a) + c_s[p];
+          if (lane == 0 && z > 0.f) atomicOr(&bits[p >> 5], 1u << (p & 31));  // NaN -> inactive
+        }
+      }
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();
+  // The next tile's active positions, ascending, with their biases -> the next launch
+  const int nwords = (un + 31) / 32;
+  if (warp == 0) {
+    int base = 0;
+    for (int wi = 0; wi < nwords; wi += 32) {
+      const int k = wi + lane < nwords ? __popc(bits[wi + lane]) : 0;
+      int incl = k;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (wi + lane < nwords) wpref[wi + lane] = base + incl - k;
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *ncnt_s = base;
+  }
+  __syncthreads();
+  for (int p = tid; p < un; p += kT) {
+    const uint32_t word = bits[p >> 5], bit = 1u << (p & 31);
+    if (word & bit) {
+      const int k = wpref[p >> 5] + __popc(word & (bit - 1u));
+      Q.list_out[u0 + k] = make_int2(u0 + p, __float_as_int(a_s[p]));
+    }
+  }
+  if (tid == 0) Q.cnt_out[c] = *ncnt_s;
+}
+
+template <typename T, int ACT, int MAXM, typename R>
+cudaError_t launch_t(const Decode1Params &P, const AheadParams &Q, size_t smem, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.G);
+  cfg.blockDim = dim3(kT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_decode_ahead<T, ACT, MAXM, R>, P, Q);
+}
+
+template <typename T, int ACT, typename R>
+cudaError_t launch_act(const Decode1Params &P, const AheadParams &Q, size_t smem, cudaStream_t stream, bool pdl) {
+  const int nch = P.d / Elem<T>::kVec;
+  if (nch <= kT) return launch_t<T, ACT, 1, R>(P, Q, smem, stream, pdl);
+  if (nch <= 2 * kT) return launch_t<T, ACT, 2, R>(P, Q, smem, stream, pdl);
+  return launch_t<T, ACT, 4, R>(P, Q, smem, stream, pdl);
+}
+
+template <typename T, int ACT, typename R>
+cudaError_t config_act() {
+  const void *ks[] = {(const void *)k_decode_ahead<T, ACT, 1, R>, (const void *)k_decode_ahead<T, ACT, 2, R>,
+                      (const void *)k_decode_ahead<T, ACT, 4, R>};
+  for (const void *k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCap);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t configure_decode_ahead() {
+  cudaError_t e = config_act<float, SFNN_RELU, float>();
+  if (e == cudaSuccess) e = config_act<float, SFNN_REGLU, float>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, __half>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, __half>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, int8_t>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, int8_t>();
+  return e;
+}
+
+cudaError_t launch_decode_ahead(const Decode1Params &P, const AheadParams &Q, cudaStream_t stream, bool pdl) {
+  const size_t smem = decode_ahead_layout(P, Q).total;
+  if (smem > (size_t)kSmemCap || P.d / (P.dt == SFNN_F16 ? 8 : 4) > 4 * kT) return cudaErrorInvalidValue;
+  if (P.dt != SFNN_F16)
+    return P.act == SFNN_REGLU ? launch_act<float, SFNN_REGLU, float>(P, Q, smem, stream, pdl)
+                               : launch_act<float, SFNN_RELU, float>(P, Q, smem, stream, pdl);
+  if (P.ri8)
+    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, int8_t>(P, Q, smem, stream, pdl)
+                               : launch_act<__half, SFNN_RELU, int8_t>(P, Q, smem, stream, pdl);
+  return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, __half>(P, Q, smem, stream, pdl)
+                             : launch_act<__half, SFNN_RELU, __half>(P, Q, smem, stream, pdl);
+}
+
+}  // namespace sfnn

@@ -1,0 +1,67 @@
+// decode_dev.cuh -- device helpers shared by the fused decode kernels (decode1.cu,
+// decode_ahead.cu): 16-byte chunk dot products and the bounded grid barrier.
+#pragma once
+
+#include "async.cuh"
+#include "common.cuh"
+#include "decode1.cuh"
+
+namespace sfnn {
+namespace {
+
+constexpr int kT = kDecode1Threads;
+constexpr int kW = kT / 32;
+constexpr int kSegChunks = 256;  // 16-byte chunks of one C1 segment (8 per lane)
+constexpr int kSmemCap = kDecodeSmemCap;
+
+template <typename T>
+__device__ __forceinline__ float dot_chunk(const uint4 &w, const float *h, float a) {
+  constexpr int V = Elem<T>::kVec;
+  float f[V];
+  unpack<T>(w, f);
+#pragma unroll
+  for (int v = 0; v < V; ++v) a = fmaf(f[v], h[v], a);
+  return a;
+}
+
+// 16 int8 codes of a row (one 16-byte chunk) against x[16 ch .. 16 ch + 15] (fp16 in
+// shared memory); the row's scale is applied to the finished sum.
+__device__ __forceinline__ float dot_chunk_i8(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  float xf[16];
+  unpack<__half>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 32), xf);
+  unpack<__half>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 32 + 16), xf + 8);
+  const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaf((float)(int8_t)(q[i >> 2] >> (8 * (i & 3))), xf[i], a);
+  return a;
+}
+
+template <typename T>
+__device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  constexpr int V = Elem<T>::kVec;
+  float f[V], xf[V];
+  unpack<T>(w, f);
+  unpack<T>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 16), xf);
+#pragma unroll
+  for (int v = 0; v < V; ++v) a = fmaf(f[v], xf[v], a);
+  return a;
+}
+
+// Grid barrier by thread 0, bracketed by CTA barriers; false (and the error latched)
+// if it timed out.  No separate fences: the CTA's writes happen before thread 0's
+// release add through the CTA barrier, and another CTA's reads after its thread 0's
+// acquire load through its CTA barrier; causality order composes the CTA-scope and
+// GPU-scope synchronisations.
+__device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = grid_barrier(P.bar, (uint32_t)P.G, kWaitCycles);
+    if (!ok) latch_error(P.err, kErrTimeout);
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int *>(flag) != 0;
+}
+
+}  // namespace
+}  // namespace sfnn

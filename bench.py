@@ -66,6 +66,9 @@ def parse_args(argv=None):
     ap.add_argument("--stack", action="store_true",
                     help="time the residual stack of the workload's layers (default workload: the "
                          "4-layer LLaMA-7B-shaped ReGLU stack), one token at a time")
+    ap.add_argument("--lookahead", action="store_true",
+                    help="with --stack: predict each layer's set from the previous layer's input, "
+                         "one layer ahead (one fused launch per layer and token, plus one)")
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call: 1 is the single-token decode (the headline); b > 1 "
                          "times the batched union path on b tokens at a time")
@@ -195,7 +198,7 @@ def measured_peak():
 
 
 # the sources k_decode1 is built from: a profile of it stays valid while they are unchanged
-DECODE1_SOURCES = ("async.cuh", "common.cuh", "decode1.cu", "decode1.cuh")
+DECODE1_SOURCES = ("async.cuh", "common.cuh", "decode1.cu", "decode1.cuh", "decode_dev.cuh")
 
 
 def source_digest() -> str:
@@ -611,7 +614,9 @@ def run_stack(args, dist):
     T, NL = cfg.tokens, cfg.layers
     layers = W.make_stack(cfg, seed=args.seed)
     Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank).astype(np.float32)
-    handles = [sf.SparseFFN.from_layer(lay, device=dev) for lay in layers]
+    rows = "int8" if args.rows == "int8" else None
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for lay in layers]
+    la = bool(args.lookahead)
     info = handles[0].info()
     e = cfg.esize
     props = torch.cuda.get_device_properties(dev)
@@ -619,9 +624,15 @@ def run_stack(args, dist):
     X = torch.from_numpy(Xh).to(dev)
     Y = torch.empty_like(X)
     active = np.zeros(NL)
-    for t in range(T):  # per-layer set sizes (the same decisions as the fused path), for the byte count
-        _, _, cnt = sf.forward_stack(handles, X[t], return_sets=True)
+    # per-layer set sizes (the same decisions as the fused path), for the byte count; int8
+    # rows run the fused path only, so their sets come from fp16 handles of the same layers
+    count_handles = handles if rows is None else [sf.SparseFFN.from_layer(lay, device=dev) for lay in layers]
+    for t in range(T):
+        _, _, cnt = sf.forward_stack(count_handles, X[t], return_sets=True, lookahead=la)
         active += cnt.cpu().numpy().reshape(NL)
+    if rows is not None:
+        for h in count_handles:
+            h.close()
     active /= T
     bytes_layer_tok = info["predictor_bytes"] + active * info["row_bytes_per_neuron"] + cfg.d * (e + 4)
     bytes_step = float(bytes_layer_tok.sum()) * T
@@ -629,13 +640,13 @@ def run_stack(args, dist):
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for t in range(T):
-            sf.forward_stack(handles, X[t], Y[t], stream=s)
+            sf.forward_stack(handles, X[t], Y[t], stream=s, lookahead=la)
     torch.cuda.synchronize()
     launches0 = sum(h.info()["launches"] for h in handles)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         for t in range(T):
-            sf.forward_stack(handles, X[t], Y[t], stream=s)
+            sf.forward_stack(handles, X[t], Y[t], stream=s, lookahead=la)
     launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
     for _ in range(args.warmup):
         g.replay()
@@ -665,8 +676,10 @@ def run_stack(args, dist):
     peak, peak_kind = measured_peak()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": None,
-                "kernel": f"k_decode1, one launch per layer and token ({launches_per_step // T} launches per token "
-                          "with the input rounding); duration = CUDA-event time of the region / layer-tokens",
+                "kernel": (f"k_decode_ahead (look-ahead stack), {launches_per_step // T} launches per token: the "
+                           "input rounding, layer 0's predictor, one per layer" if la else
+                           f"k_decode1, one launch per layer and token ({launches_per_step // T} launches per token "
+                           "with the input rounding)") + "; duration = CUDA-event time of the region / layer-tokens",
                 "algorithmic_bytes_per_launch": float(bytes_layer_tok.mean()), "avg_launch_us": layer_us,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s", "traffic_source": None}
@@ -681,7 +694,7 @@ def run_stack(args, dist):
         def one_step():  # the step's inputs in one copy, one stack call per token, the outputs in one copy
             xd.copy_(xin, non_blocking=True)
             for t in range(T):
-                sf.forward_stack(handles, xd[t], yd[t], stream=s)
+                sf.forward_stack(handles, xd[t], yd[t], stream=s, lookahead=la)
             yout.copy_(yd, non_blocking=True)
         with torch.cuda.stream(s):
             one_step()
@@ -701,11 +714,13 @@ def run_stack(args, dist):
                                             "of the step's inputs, the API calls, one device-to-host copy of the "
                                             "outputs), max over ranks"}
     line = {
-        "metric": f"sparse-FFN decode layer-tokens/s ({NL}-layer residual stack)", "value": value,
+        "metric": f"sparse-FFN decode layer-tokens/s ({NL}-layer residual stack"
+                  f"{', sets predicted one layer ahead' if la else ''})", "value": value,
         "unit": "layer-tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": cfg.description, "batch": 1, "layers": NL, "tokens_per_step": T,
+                   "predictor": "one layer ahead" if la else "own layer", "rows": args.rows,
                    "l2": f"inputs larger than L2: {NL} distinct layers per token, "
                          f"{float(bytes_layer_tok.sum()) / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{dist.world} (no exchange)",

@@ -215,6 +215,23 @@ SFNN_API sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_l
                                float *XL, int32_t *idx, int32_t *counts, sfnn_stream_t stream);
 
 /*
+ * The same residual stack with every layer's active set predicted one layer ahead:
+ * layer l+1's predictor (its own A, B, c) takes layer l's input round(X_l), so it can
+ * run beside layer l instead of in front of layer l+1 -- DejaVu's asynchronous
+ * predictor, which forecasts the next layer's sparsity one step early (53ai.com
+ * "sparsity for LLM inference" page, section "如何推理加速").  Layer 0 predicts from
+ * round(X_0).  The sets, and so XL, may differ from sfnn_forward_stack's.
+ * With b = 1 and no idx/counts, and every layer on the fused kernel with the same
+ * number of tiles (SMs), the stack runs as num_layers + 1 launches of one look-ahead
+ * kernel: launch l does layer l's rows on the set launch l-1 predicted and layer l+1's
+ * predictor, with one bounded grid barrier.  Otherwise the batched path, with each
+ * layer's prediction issued before the previous layer's reduce.
+ * Arguments, sharing rules and idx/counts layout as sfnn_forward_stack.
+ */
+SFNN_API sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_layers, const float *X0,
+                                         int32_t b, float *XL, int32_t *idx, int32_t *counts, sfnn_stream_t stream);
+
+/*
  * Enable (default) or disable the fused single-token kernel, which runs a whole
  * decode step of one token in one launch: one persistent CTA per SM owning a tile of
  * neurons, the predictor's rows and the active neurons' rows streamed through

@@ -68,6 +68,7 @@ def test_null_and_invalid_arguments_return_status():
     assert lib.sfnn_predict(None, 1, 1, 1, None) == 1
     assert lib.sfnn_forward_batch(None, 1, 1, 1, None, None, None) == 1
     assert lib.sfnn_forward_stack(None, 1, 1, 1, 1, None, None, None) == 1
+    assert lib.sfnn_forward_stack_lookahead(None, 1, 1, 1, 1, None, None, None) == 1
     assert lib.sfnn_destroy(None) == 0
     assert lib.sfnn_get_error(None) == 1
     assert lib.sfnn_set_batch_path(None, 0) == 1

@@ -1,0 +1,138 @@
+"""The look-ahead residual stack: layer l+1's set predicted from layer l's input.
+
+* the fused look-ahead kernel (one launch per layer plus one) and the multi-kernel
+  look-ahead path both match the oracle's look-ahead stack, with every layer's set
+  arbitrated against the oracle's, for ReLU and ReGLU, at a reduced size and at the
+  full LLaMA-7B-shaped 4-layer ReGLU stack;
+* the sets really are predicted one layer early: they differ from the plain stack's;
+* one layer (nothing to look ahead of) gives the plain stack's result to the bit;
+* a stack of one handle used for every layer, int8 rows, sets that are empty
+  (y = 0, so XL = X0 exactly), and a grid barrier that times out (reported, then the
+  stack recovers and reproduces its result).
+"""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_ffn_threshold_b200 as sf
+import oracle
+import workload as W
+from parity_util import NTHREADS, mask_from_idx
+
+pytestmark = pytest.mark.gpu
+
+
+def _x0(cfg, seed):
+    return W.make_tokens(cfg, 1, seed=seed)[0].astype(np.float32)
+
+
+def _run(hs, x0):
+    """(XL of the fused path, XL of the multi-kernel path, that path's per-layer masks)."""
+    X0 = torch.from_numpy(x0).cuda()
+    XL_fused = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
+    XL_sets, sidx, scnt = sf.forward_stack(hs, X0, return_sets=True, lookahead=True)
+    n = hs[0].n
+    masks = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), n) for l in range(len(hs))]
+    return XL_fused, XL_sets.cpu().numpy(), masks
+
+
+def _check(layers, hs, x0, qrows=None):
+    XL_fused, XL_sets, masks = _run(hs, x0)
+    xref, recs = oracle.forward_stack_lookahead(layers, x0.astype(np.float64), masks_other=masks,
+                                                nthreads=NTHREADS, qrows=qrows)
+    for l, rec in enumerate(recs):
+        assert rec["mismatches"].size == 0, f"layer {l}: sets differ outside the arbitration band"
+    base = x0.astype(np.float64)
+    for what, XL in (("fused", XL_fused), ("multi-kernel", XL_sets)):
+        ok, ratio = oracle.within_tolerance(XL.astype(np.float64) - base, xref - base)
+        assert ok, f"{what}: max|dx|/max|dx_ref| = {ratio:.3e}"
+    for h in hs:
+        assert h.get_error() == 0
+    return XL_fused, masks, recs
+
+
+@pytest.mark.parametrize("base", ["llama7b_reglu_stack", "opt6.7b_relu"])
+def test_lookahead_stack_matches_oracle(base):
+    cfg = W.small_config(W.CONFIGS[base], d=1024, n=2500, r=128)
+    layers = [W.make_layer(cfg, seed=51, layer=l) for l in range(4)]
+    hs = [sf.SparseFFN.from_layer(l) for l in layers]
+    x0 = _x0(cfg, 52)
+    _, masks, _ = _check(layers, hs, x0)
+    # predicted one layer early: some layer's set differs from the plain stack's
+    _, sidx, scnt = sf.forward_stack(hs, torch.from_numpy(x0).cuda(), return_sets=True)
+    plain = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), cfg.n) for l in range(4)]
+    assert np.array_equal(masks[0], plain[0])  # layer 0 predicts from its own input either way
+    assert any(not np.array_equal(masks[l], plain[l]) for l in range(1, 4))
+
+
+def test_lookahead_full_size_llama7b_reglu_stack():
+    cfg = W.CONFIGS["llama7b_reglu_stack"]
+    layers = W.make_stack(cfg, seed=0)
+    hs = [sf.SparseFFN.from_layer(l) for l in layers]
+    _check(layers, hs, _x0(cfg, 53))
+
+
+def test_lookahead_one_layer_is_the_plain_stack():
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=2048, n=3001, r=256)
+    h = sf.SparseFFN.from_layer(W.make_layer(cfg, seed=54))
+    X0 = torch.from_numpy(_x0(cfg, 55)).cuda()
+    a = sf.forward_stack([h], X0, lookahead=True)
+    b = sf.forward_stack([h], X0)
+    assert torch.equal(a, b)  # same set, same kernels' summation orders
+    assert h.get_error() == 0
+
+
+def test_lookahead_one_handle_for_every_layer():
+    cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=1024, n=2000, r=128)
+    lay = W.make_layer(cfg, seed=56)
+    h = sf.SparseFFN.from_layer(lay)
+    _check([lay] * 3, [h] * 3, _x0(cfg, 57))
+
+
+def test_lookahead_int8_rows():
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
+    layers = [W.make_layer(cfg, seed=58, layer=l) for l in range(3)]
+    hs = [sf.SparseFFN.from_layer(l, rows="int8") for l in layers]
+    x0 = _x0(cfg, 59)
+    X0 = torch.from_numpy(x0).cuda()
+    XL = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
+    # int8 rows run the fused kernel only: take the sets from fp16 handles of the same
+    # layers (same predictor, same kernels' decisions) for the arbitration
+    hf = [sf.SparseFFN.from_layer(l) for l in layers]
+    _, _, masks = _run(hf, x0)
+    qrows = [oracle.quantize_layer(l) for l in layers]
+    xref, recs = oracle.forward_stack_lookahead(layers, x0.astype(np.float64), masks_other=masks,
+                                                nthreads=NTHREADS, qrows=qrows)
+    assert all(r["mismatches"].size == 0 for r in recs)
+    base = x0.astype(np.float64)
+    assert oracle.within_tolerance(XL.astype(np.float64) - base, xref - base)[0]
+    assert all(h.get_error() == 0 for h in hs)
+
+
+def test_lookahead_empty_sets_leave_the_input():
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=1500, r=128)
+    layers = [W.make_layer(cfg, seed=60, layer=l) for l in range(3)]
+    for l in layers:
+        l.c = np.full_like(l.c, -1e4)  # every logit far below the threshold
+    hs = [sf.SparseFFN.from_layer(l) for l in layers]
+    x0 = _x0(cfg, 61)
+    XL_fused, XL_sets, masks = _run(hs, x0)
+    assert all(m.sum() == 0 for m in masks)
+    assert np.array_equal(XL_fused, x0) and np.array_equal(XL_sets, x0)
+
+
+def test_lookahead_barrier_timeout_is_reported_and_recovers():
+    cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=1024, n=3000, r=128)
+    layers = [W.make_layer(cfg, seed=62, layer=l) for l in range(2)]
+    hs = [sf.SparseFFN.from_layer(l) for l in layers]
+    X0 = torch.from_numpy(_x0(cfg, 63)).cuda()
+    ok = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
+    assert all(h.get_error() == 0 for h in hs)
+    hs[0].debug_stall_next_barrier()
+    sf.forward_stack(hs, X0, lookahead=True)
+    torch.cuda.synchronize()  # returns: the launches on layer 0's counter gave up after their bound
+    assert hs[0].get_error() == sf.STATUS_CODES["SFNN_ERR_TIMEOUT"]
+    assert hs[1].get_error() == 0
+    again = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
+    assert np.array_equal(again, ok)
+    assert all(h.get_error() == 0 for h in hs)
