@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "launch.cuh"
 
 using namespace sfnn;
 
@@ -64,7 +65,7 @@ sfnn_status check_desc(const sfnn_layer_desc *d) {
   if (d->d % vec || d->r % vec) return SFNN_ERR_INVALID_ARG;
   if (d->max_batch > kMaxBatch) return SFNN_ERR_UNSUPPORTED;
   if ((int64_t)d->r * d->max_batch > 32768) return SFNN_ERR_UNSUPPORTED;
-  if (d->n > (1 << 24) || d->d > (1 << 16)) return SFNN_ERR_UNSUPPORTED;
+  if (d->n > kMaxNeurons || d->d > (1 << 16)) return SFNN_ERR_UNSUPPORTED;
   return SFNN_OK;
 }
 
@@ -128,7 +129,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
   } else if (src == kSetGiven) {
     SFNN_TRY(launch_mask_from_idx(h, idx, count, s));
   }
-  SFNN_TRY(launch_compact(h, b, idx_out, cnt_out, s));
+  SFNN_TRY(launch_compact(h, b, true, idx_out, cnt_out, s));
   int splits = 1;
   if (tc) {
     SFNN_TRY(launch_tc_batch(h, X, b, &splits, s));
@@ -143,7 +144,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
   }
   SFNN_TRY(launch_reduce(h, b, splits, resid, Y, xnext, s));
   record_if(after, s);
-  h->launches += 4 + (predict ? 2 : (src == kSetGiven ? 1 : 0));
+  h->launches += 4 + (predict ? 2 : (src == kSetGiven ? 1 : 0)) + ((idx_out || cnt_out) ? 1 : 0);
   return SFNN_OK;
 }
 
@@ -214,9 +215,11 @@ AheadParams ahead_params(const sfnn_ctx *nx) {
 }
 
 // Every launch of a fused look-ahead stack fits: every layer runs its fused kernel, all
-// with the same tiles (a tile's list is written and read by the same CTA), and each
-// (layer, next layer) pair's shared-memory plan fits one CTA per SM.
+// with the same tiles (tile c's next list is written by CTA c), the row shares' counts
+// and prefix fit the kernel's scratch (2G + 5 words), and each (layer, next layer)
+// pair's shared-memory plan fits one CTA per SM.
 bool ahead_fused_ok(const sfnn_handle *layers, int num_layers) {
+  if (2 * layers[0]->d1.G + 5 > kDecode1Threads) return false;
   for (int l = 0; l < num_layers; ++l) {
     const sfnn_ctx *hl = layers[l];
     if (!hl->fused_ok || !hl->fused_on || hl->d1.G != layers[0]->d1.G) return false;
@@ -386,7 +389,7 @@ sfnn_status sfnn_predict(sfnn_handle h, const void *x, int32_t *idx, int32_t *co
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   SFNN_TRY(launch_hidden(h, x, 1, s));
   SFNN_TRY(launch_logits(h, 1, s));
-  SFNN_TRY(launch_compact(h, 1, idx, count, s));
+  SFNN_TRY(launch_compact(h, 1, false, idx, count, s));
   h->launches += 3;
   return SFNN_OK;
 }

@@ -7,10 +7,10 @@
 // l+1's predictor takes layer l's input u_l, which lets one launch per layer carry both
 // halves (one CTA of 16 warps per SM, as the single-layer kernel):
 //
-//   P1  u_l and the CTA's active list of layer l (written by the previous launch) into
+//   P1  u_l, and the active lists of layer l (written by the previous launch), into
 //       shared memory; h' = relu(A'^T u_l) for the CTA's rows of layer l+1's A' (one warp
 //       per row, its first batch requested before the previous kernel ends); C1 / C2 on
-//       layer l's active rows of the tile, exactly as in the single-layer kernel; the
+//       the CTA's share of layer l's active rows, as in the single-layer kernel; the
 //       CTA's partial y to global memory; the first B'^T rows of layer l+1's tile
 //       requested into the staging region C2 has left.
 //   grid barrier (the launch's only one)
@@ -20,10 +20,13 @@
 //
 // Against the single-layer kernel, each layer drops one grid barrier and the hidden
 // layer's phase from its critical chain, and the column reduce overlaps the logits.
-// CTA c owns tile c of every layer, so a tile's list is written and read by the same CTA
-// in consecutive launches.  The stack's first launch runs P1/P2's predictor half only
-// (layer 0 on u_0); its last launch has no next predictor.  Dot products keep the
-// single-layer kernel's orders, so a layer's y on a given set is the same to the bit.
+// Because all of a layer's lists are in global memory before its launch starts, the
+// active rows need not stay with the tile that predicted them: every CTA takes an equal
+// share (its own tile's rows up to the share, then rows the fuller tiles leave over),
+// which removes the busiest tile's surplus from the critical path at the cost of one
+// dependent load.  The stack's first launch runs the predictor half only (layer 0 on
+// u_0); its last launch has no next predictor.  The predictor's dot products keep the
+// single-layer kernel's orders, so both decide every neuron identically.
 #include "async.cuh"
 #include "common.cuh"
 #include "decode1.cuh"
@@ -95,16 +98,82 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   for (int i = tid; i < nch_d; i += kT)
     *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
         __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+  // The active rows are shared out evenly: CTA c takes T_c = floor((c+1)K/G) - floor(cK/G)
+  // of the layer's K rows, first o_c = min(cnt_c, T_c) of its own tile's, then f_c = T_c - o_c
+  // of the rows the tiles with more than their share leave over (e_t = cnt_t - o_t each,
+  // taken in tile order).  The assignment depends on the counts only: deterministic.
+  int *cnt_all = reinterpret_cast<int *>(red2);  // [G] counts, [G + 1] prefix of e, o_c f_c F_c K
+  int *epre = cnt_all + G;
+  int *own = epre + G + 1;
   if (cur) {
-    for (int i = tid; i < tn; i += kT) {  // the whole tile's slots: the count arrives with them
+    for (int i = tid; i < tn; i += kT) {  // the own tile's slots arrive with the counts
       const int2 e = __ldcg(Q.list_in + t0 + i);
       act_s[i] = e.x;
       bias_s[i] = __int_as_float(e.y);
     }
-    if (tid == 0) *cnt_s = __ldcg(Q.cnt_in + c);
+    for (int t = tid; t < G; t += kT) {
+      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
+      cnt_all[t] = min(max(__ldcg(Q.cnt_in + t), 0), sz);
+    }
   }
   __syncthreads();
-  const int cnt = cur ? min(max(*cnt_s, 0), tn) : 0;
+  if (cur && warp == 0) {
+    int K = 0;
+    for (int t = lane; t < G; t += 32) K += cnt_all[t];
+    K = __reduce_add_sync(0xffffffffu, K);
+    int baseE = 0, baseF = 0;
+    for (int wi = 0; wi < G; wi += 32) {
+      const int t = wi + lane;
+      int e = 0, f = 0, o = 0;
+      if (t < G) {
+        const int share = (int)(((int64_t)(t + 1) * K) / G - ((int64_t)t * K) / G);
+        o = min(cnt_all[t], share);
+        e = cnt_all[t] - o;
+        f = share - o;
+      }
+      int ie = e, jf = f;  // inclusive scans of e and f over the tiles
+#pragma unroll
+      for (int s = 1; s < 32; s <<= 1) {
+        const int ye = __shfl_up_sync(0xffffffffu, ie, s), yf = __shfl_up_sync(0xffffffffu, jf, s);
+        if (lane >= s) {
+          ie += ye;
+          jf += yf;
+        }
+      }
+      if (t < G) epre[t] = baseE + ie - e;
+      if (t == c) {
+        own[0] = o;
+        own[1] = f;
+        own[2] = baseF + jf - f;
+      }
+      baseE += __shfl_sync(0xffffffffu, ie, 31);
+      baseF += __shfl_sync(0xffffffffu, jf, 31);
+    }
+    if (lane == 0) {
+      epre[G] = baseE;
+      own[3] = K;
+    }
+  }
+  __syncthreads();
+  const int o_c = cur ? own[0] : 0, f_c = cur ? own[1] : 0, F_c = cur ? own[2] : 0, K = cur ? own[3] : 0;
+  // this CTA's excess row j is the layer's excess row g = F_c + j: tile t with
+  // epre[t] <= g < epre[t + 1], slot o_t + g - epre[t] of that tile
+  auto excess_entry = [&](int j) {
+    const int g = F_c + j;
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (epre[mid] <= g)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    const int share = (int)(((int64_t)(lo + 1) * K) / G - ((int64_t)lo * K) / G);
+    const int k = min(cnt_all[lo], share) + g - epre[lo];
+    return __ldcg(Q.list_in + decode1_tile_start(lo, P.n, G) + k);
+  };
+  int2 ex0 = make_int2(0, 0);
+  if (tid < f_c) ex0 = excess_entry(tid);  // lands while A' runs
 
   // ---------------------------------------------------------------- A': next hidden layer
   if (next) {
@@ -129,6 +198,18 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       if (lane == 0) Q.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
     }
   }
+
+  if (tid < f_c) {
+    act_s[o_c + tid] = ex0.x;
+    bias_s[o_c + tid] = __int_as_float(ex0.y);
+  }
+  for (int j = tid + kT; j < f_c; j += kT) {
+    const int2 e = excess_entry(j);
+    act_s[o_c + j] = e.x;
+    bias_s[o_c + j] = __int_as_float(e.y);
+  }
+  __syncthreads();
+  const int cnt = o_c + f_c;
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };

@@ -15,6 +15,7 @@
 //   k_reduce  y = sum over ks of part[ks] in ascending ks (+ residual).
 // Every sum runs in a fixed order, so results are bitwise reproducible.
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace sfnn {
 namespace {

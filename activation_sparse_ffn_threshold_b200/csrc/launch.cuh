@@ -1,0 +1,35 @@
+// launch.cuh -- host-side launchers of the kernels (defined in the .cu files) and the
+// size limits the host checks when a layer is created.
+#pragma once
+
+#include "common.cuh"
+
+namespace sfnn {
+
+constexpr int kMaxNeurons = 1 << 20;                  // n: the union's per-word offsets live in shared memory
+constexpr int kUnionSmemMax = (kMaxNeurons / 32) * 4;  // bytes of those offsets at the largest n
+
+cudaError_t configure_predict();  // one-time kernel attributes (shared-memory limits)
+cudaError_t configure_ffn();
+cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s);
+cudaError_t launch_hidden(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
+cudaError_t launch_logits(const sfnn_ctx *h, int b, cudaStream_t s);
+cudaError_t launch_mask_from_idx(const sfnn_ctx *h, const int32_t *idx, const int32_t *count, cudaStream_t s);
+// want_union: the batch's union list (k_union); idx_out/cnt_out: per-token lists (k_compact)
+cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *idx_out, int32_t *cnt_out,
+                           cudaStream_t s);
+cudaError_t launch_up(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
+cudaError_t launch_down(const sfnn_ctx *h, int b, int *splits, cudaStream_t s);
+cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *resid, float *Y, void *xnext,
+                          cudaStream_t s);
+cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s);
+
+// Tensor-core (tcgen05) batch path: fp16 weights, d a multiple of 128.
+bool tc_batch_supported(const sfnn_ctx *h);
+bool tc_predict_supported(const sfnn_ctx *h);  // and r a multiple of 64
+cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
+int tc_hstride(int n);
+cudaError_t configure_tc_batch();
+cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits_out, cudaStream_t s);
+
+}  // namespace sfnn

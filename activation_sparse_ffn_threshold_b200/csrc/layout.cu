@@ -9,6 +9,7 @@
 // touched, the row/column-structured sparsity the same page (section 激活稀疏)
 // calls hardware friendly.  These kernels only move bits; they run once.
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace sfnn {
 namespace {

@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace {
 

@@ -11,10 +11,12 @@
 //   k_hidden   H[t][j] = relu(At[j] . X[t])         one warp per row of At
 //   k_logits   bit i of token t = (Bt[i] . H[t] + c_i > 0)   one CTA per 32 neurons
 //   k_mask_from_idx   a caller-given index list as a bit mask
+//   k_union    masks -> the union of a batch's sets with each row's token mask
 //   k_compact  masks -> ascending index lists (per token, in caller numbering)
 //              and the union of the tokens' sets with, per union row, the bit
 //              set of tokens active on it (warp ballot + block prefix sum).
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace sfnn {
 namespace {
@@ -182,61 +184,87 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
   return before + incl - v;
 }
 
-// Blocks 0..b-1 (only when token outputs are wanted): token lists.  Last block: the union,
-// with each union row's token mask; a thread reads the b tokens' words of its bit word
-// once (registers) and takes both the union bits and the masks from them.
-__global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ mask, int nwords, int n, int b,
-                                                  const int32_t *__restrict__ perm, int32_t *__restrict__ ulist,
-                                                  uint32_t *__restrict__ utok, int32_t *__restrict__ ucount,
-                                                  int32_t *__restrict__ idx_out, int32_t *__restrict__ cnt_out) {
-  const bool is_union = blockIdx.x == gridDim.x - 1;
+// The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
+// token t's set holds the row).  One CTA: warp w takes bit words w, w + 32, ...; lane t
+// reads token t's word, the union word is their OR, and 32 ballots transpose the 32 x 32
+// bit block into the rows' token masks.  Pass 1 counts each word's union bits, a block
+// scan turns the counts into first positions, pass 2 writes the rows.
+__global__ void __launch_bounds__(1024) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
+                                                int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
+                                                int32_t *__restrict__ ucount) {
+  extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
+  auto union_word = [&](int w, uint32_t *mw) {
+    *mw = lane < b ? __ldcg(mask + (size_t)lane * nwords + w) : 0u;
+    const uint32_t u = __reduce_or_sync(0xffffffffu, *mw);
+    return w == nwords - 1 ? u & tail : u;
+  };
+  for (int w = warp; w < nwords; w += nw) {
+    uint32_t mw;
+    const uint32_t u = union_word(w, &mw);
+    if (lane == 0) woff[w] = __popc(u);
+  }
+  __syncthreads();
+  const int per = (nwords + blockDim.x - 1) / blockDim.x;  // words per thread in the scan
+  const int w0 = threadIdx.x * per;
+  int sum = 0;
+  for (int k = 0; k < per; ++k)
+    if (w0 + k < nwords) sum += woff[w0 + k];
+  int total;
+  int run = block_exclusive_scan(sum, &total);
+  for (int k = 0; k < per; ++k)
+    if (w0 + k < nwords) {
+      const int v = woff[w0 + k];
+      woff[w0 + k] = run;
+      run += v;
+    }
+  __syncthreads();
+  for (int w = warp; w < nwords; w += nw) {
+    uint32_t mw;
+    const uint32_t u = union_word(w, &mw);
+    if (u == 0u) continue;  // warp-uniform
+    uint32_t tb = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t col = __ballot_sync(0xffffffffu, (mw >> i) & 1u);
+      if (lane == i) tb = col;
+    }
+    if ((u >> lane) & 1u) {
+      const int pos = woff[w] + __popc(u & ((1u << lane) - 1u));
+      ulist[pos] = w * 32 + lane;
+      utok[pos] = tb;
+    }
+  }
+  if (threadIdx.x == 0) *ucount = total;
+}
+
+// Block t: token t's set as indices in the caller's numbering, ascending in storage order.
+__global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ mask, int nwords, int n,
+                                                  const int32_t *__restrict__ perm, int32_t *__restrict__ idx_out,
+                                                  int32_t *__restrict__ cnt_out) {
   const int t = blockIdx.x;
   const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
   const int w0 = threadIdx.x * wpt;
-  uint32_t mw[kMaxBatch];  // the tokens' words of the current bit word (union block)
-  auto word = [&](int w) -> uint32_t {
-    if (!is_union) return mask[(size_t)t * nwords + w];
-    uint32_t m = 0u;
-#pragma unroll
-    for (int tt = 0; tt < kMaxBatch; ++tt) {
-      mw[tt] = tt < b ? mask[(size_t)tt * nwords + w] : 0u;
-      m |= mw[tt];
-    }
-    return m;
-  };
   int cnt = 0;
   for (int k = 0; k < wpt; ++k) {
     const int w = w0 + k;
-    if (w < nwords) cnt += __popc(word(w));
+    if (w < nwords) cnt += __popc(mask[(size_t)t * nwords + w]);
   }
   int total;
   int pos = block_exclusive_scan(cnt, &total);
   for (int k = 0; k < wpt; ++k) {
     const int w = w0 + k;
     if (w >= nwords) break;
-    uint32_t m = word(w);
+    uint32_t m = mask[(size_t)t * nwords + w];
     while (m) {
       const int i = __ffs(m) - 1;
       m &= m - 1u;
-      const int p = w * 32 + i;
-      if (is_union) {
-        uint32_t tb = 0u;
-#pragma unroll
-        for (int tt = 0; tt < kMaxBatch; ++tt) tb |= ((mw[tt] >> i) & 1u) << tt;
-        ulist[pos] = p;
-        utok[pos] = tb;
-      } else if (idx_out) {
-        idx_out[(size_t)t * n + pos] = perm[p];
-      }
+      if (idx_out) idx_out[(size_t)t * n + pos] = perm[w * 32 + i];
       ++pos;
     }
   }
-  if (threadIdx.x == 0) {
-    if (is_union)
-      *ucount = total;
-    else if (cnt_out)
-      cnt_out[t] = total;
-  }
+  if (threadIdx.x == 0 && cnt_out) cnt_out[t] = total;
 }
 
 template <typename T>
@@ -274,6 +302,8 @@ cudaError_t logits_impl(const sfnn_ctx *h, int b, cudaStream_t s) {
 }  // namespace
 
 cudaError_t configure_predict() {
+  cudaError_t e0 = cudaFuncSetAttribute(k_union, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnionSmemMax);
+  if (e0 != cudaSuccess) return e0;
   const void *ks[] = {(const void *)k_logits<float, 1>, (const void *)k_logits<float, 8>,
                       (const void *)k_logits<float, 32>, (const void *)k_logits<__half, 1>,
                       (const void *)k_logits<__half, 8>, (const void *)k_logits<__half, 32>};
@@ -297,11 +327,19 @@ cudaError_t launch_mask_from_idx(const sfnn_ctx *h, const int32_t *idx, const in
   return cudaGetLastError();
 }
 
-cudaError_t launch_compact(const sfnn_ctx *h, int b, int32_t *idx_out, int32_t *cnt_out, cudaStream_t s) {
-  const int grid = (idx_out || cnt_out) ? b + 1 : 1;
-  k_compact<<<grid, 1024, 0, s>>>(h->mask, h->L.nwords, h->L.n, b, h->perm, h->ulist, h->utok, h->ucount, idx_out,
-                                  cnt_out);
-  return cudaGetLastError();
+cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *idx_out, int32_t *cnt_out,
+                           cudaStream_t s) {
+  const Layout &L = h->L;
+  cudaError_t e = cudaSuccess;
+  if (want_union) {
+    k_union<<<1, 1024, (size_t)L.nwords * sizeof(int), s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && (idx_out || cnt_out)) {
+    k_compact<<<b, 1024, 0, s>>>(h->mask, L.nwords, L.n, h->perm, idx_out, cnt_out);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace sfnn

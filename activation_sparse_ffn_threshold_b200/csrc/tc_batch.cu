@@ -28,6 +28,7 @@
 
 #include "async.cuh"
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace sfnn {
 namespace {

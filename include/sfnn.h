@@ -109,7 +109,7 @@ typedef enum {
  * The inputs are read during sfnn_create only; they may be freed once it returns.
  */
 typedef struct {
-    int32_t d, n, r;
+    int32_t d, n, r;   /* d <= 65536, n <= 2^20 (else SFNN_ERR_UNSUPPORTED) */
     int32_t max_batch; /* largest b later passed to sfnn_forward_batch / sfnn_forward_stack, 1..32 */
     int32_t act;       /* sfnn_act */
     int32_t wdtype;    /* sfnn_dtype */

@@ -5,7 +5,7 @@
   arbitrated against the oracle's, for ReLU and ReGLU, at a reduced size and at the
   full LLaMA-7B-shaped 4-layer ReGLU stack;
 * the sets really are predicted one layer early: they differ from the plain stack's;
-* one layer (nothing to look ahead of) gives the plain stack's result to the bit;
+* one layer (nothing to look ahead of) gives the plain stack's result;
 * a stack of one handle used for every layer, int8 rows, sets that are empty
   (y = 0, so XL = X0 exactly), and a grid barrier that times out (reported, then the
   stack recovers and reproduces its result).
@@ -74,11 +74,21 @@ def test_lookahead_full_size_llama7b_reglu_stack():
 
 def test_lookahead_one_layer_is_the_plain_stack():
     cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=2048, n=3001, r=256)
-    h = sf.SparseFFN.from_layer(W.make_layer(cfg, seed=54))
-    X0 = torch.from_numpy(_x0(cfg, 55)).cuda()
-    a = sf.forward_stack([h], X0, lookahead=True)
-    b = sf.forward_stack([h], X0)
-    assert torch.equal(a, b)  # same set, same kernels' summation orders
+    lay = W.make_layer(cfg, seed=54)
+    h = sf.SparseFFN.from_layer(lay)
+    x0 = _x0(cfg, 55)
+    X0 = torch.from_numpy(x0).cuda()
+    a = sf.forward_stack([h], X0, lookahead=True).cpu().numpy()
+    b = sf.forward_stack([h], X0).cpu().numpy()
+    # the same set (the predictors' orders are the same); the rows are shared out to the
+    # CTAs differently, so y agrees within the tolerance, and with the oracle's
+    _, _, masks = _run([h], x0)
+    xref, recs = oracle.forward_stack([lay], x0.astype(np.float64), masks_other=masks)
+    assert recs[0]["mismatches"].size == 0
+    base = x0.astype(np.float64)
+    for XL in (a, b):
+        assert oracle.within_tolerance(XL.astype(np.float64) - base, xref - base)[0]
+    assert oracle.within_tolerance(a.astype(np.float64) - base, b.astype(np.float64) - base)[0]
     assert h.get_error() == 0
 
 
@@ -90,14 +100,15 @@ def test_lookahead_one_handle_for_every_layer():
 
 
 def test_lookahead_int8_rows():
+    # Two layers: with look-ahead both sets are predicted from u_0, so they do not depend
+    # on the rows' storage, and the sets of fp16 handles of the same layers (int8 rows run
+    # the fused kernel only, which returns no sets) serve for the arbitration.
     cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
-    layers = [W.make_layer(cfg, seed=58, layer=l) for l in range(3)]
+    layers = [W.make_layer(cfg, seed=58, layer=l) for l in range(2)]
     hs = [sf.SparseFFN.from_layer(l, rows="int8") for l in layers]
     x0 = _x0(cfg, 59)
     X0 = torch.from_numpy(x0).cuda()
     XL = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
-    # int8 rows run the fused kernel only: take the sets from fp16 handles of the same
-    # layers (same predictor, same kernels' decisions) for the arbitration
     hf = [sf.SparseFFN.from_layer(l) for l in layers]
     _, _, masks = _run(hf, x0)
     qrows = [oracle.quantize_layer(l) for l in layers]
