@@ -185,55 +185,74 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
 }
 
 // The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
-// token t's set holds the row).  One CTA: warp w takes bit words w, w + 32, ...; lane t
-// reads token t's word, the union word is their OR, and 32 ballots transpose the 32 x 32
-// bit block into the rows' token masks.  Pass 1 counts each word's union bits, a block
-// scan turns the counts into first positions, pass 2 writes the rows.
+// token t's set holds the row).  One CTA; warp w takes a contiguous run of bit words, 16
+// at a time with all 16 loads in flight: lane t reads token t's words, a word's union is
+// their OR, and 32 ballots transpose its 32 x 32 bit block into the rows' token masks.
+// Pass 1 counts each word's union bits, a block scan turns the counts into first
+// positions, pass 2 writes the rows.
+constexpr int kUnionBatch = 16;
+
 __global__ void __launch_bounds__(1024) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
                                                 int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
                                                 int32_t *__restrict__ ucount) {
   extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
-  auto union_word = [&](int w, uint32_t *mw) {
-    *mw = lane < b ? __ldcg(mask + (size_t)lane * nwords + w) : 0u;
-    const uint32_t u = __reduce_or_sync(0xffffffffu, *mw);
+  const int chunk = (nwords + nw - 1) / nw;
+  const int wbeg = min(nwords, warp * chunk), wend = min(nwords, wbeg + chunk);
+  // this lane's token words of bit words w0 .. w0 + kUnionBatch - 1 (zero past the run)
+  auto load = [&](int w0, uint32_t *mw) {
+#pragma unroll
+    for (int j = 0; j < kUnionBatch; ++j)
+      mw[j] = lane < b && w0 + j < wend ? __ldcg(mask + (size_t)lane * nwords + w0 + j) : 0u;
+  };
+  auto union_of = [&](int w, uint32_t mw) {
+    const uint32_t u = __reduce_or_sync(0xffffffffu, mw);
     return w == nwords - 1 ? u & tail : u;
   };
-  for (int w = warp; w < nwords; w += nw) {
-    uint32_t mw;
-    const uint32_t u = union_word(w, &mw);
-    if (lane == 0) woff[w] = __popc(u);
+  for (int w0 = wbeg; w0 < wend; w0 += kUnionBatch) {
+    uint32_t mw[kUnionBatch];
+    load(w0, mw);
+#pragma unroll
+    for (int j = 0; j < kUnionBatch; ++j) {
+      const uint32_t u = union_of(w0 + j, mw[j]);
+      if (lane == 0 && w0 + j < wend) woff[w0 + j] = __popc(u);
+    }
   }
   __syncthreads();
   const int per = (nwords + blockDim.x - 1) / blockDim.x;  // words per thread in the scan
-  const int w0 = threadIdx.x * per;
+  const int s0 = threadIdx.x * per;
   int sum = 0;
   for (int k = 0; k < per; ++k)
-    if (w0 + k < nwords) sum += woff[w0 + k];
+    if (s0 + k < nwords) sum += woff[s0 + k];
   int total;
   int run = block_exclusive_scan(sum, &total);
   for (int k = 0; k < per; ++k)
-    if (w0 + k < nwords) {
-      const int v = woff[w0 + k];
-      woff[w0 + k] = run;
+    if (s0 + k < nwords) {
+      const int v = woff[s0 + k];
+      woff[s0 + k] = run;
       run += v;
     }
   __syncthreads();
-  for (int w = warp; w < nwords; w += nw) {
-    uint32_t mw;
-    const uint32_t u = union_word(w, &mw);
-    if (u == 0u) continue;  // warp-uniform
-    uint32_t tb = 0u;
+  for (int w0 = wbeg; w0 < wend; w0 += kUnionBatch) {
+    uint32_t mw[kUnionBatch];
+    load(w0, mw);
+#pragma unroll 1
+    for (int j = 0; j < kUnionBatch; ++j) {
+      const int w = w0 + j;
+      const uint32_t u = w < wend ? union_of(w, mw[j]) : 0u;
+      if (u == 0u) continue;  // warp-uniform
+      uint32_t tb = 0u;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const uint32_t col = __ballot_sync(0xffffffffu, (mw >> i) & 1u);
-      if (lane == i) tb = col;
-    }
-    if ((u >> lane) & 1u) {
-      const int pos = woff[w] + __popc(u & ((1u << lane) - 1u));
-      ulist[pos] = w * 32 + lane;
-      utok[pos] = tb;
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t col = __ballot_sync(0xffffffffu, (mw[j] >> i) & 1u);
+        if (lane == i) tb = col;
+      }
+      if ((u >> lane) & 1u) {
+        const int pos = woff[w] + __popc(u & ((1u << lane) - 1u));
+        ulist[pos] = w * 32 + lane;
+        utok[pos] = tb;
+      }
     }
   }
   if (threadIdx.x == 0) *ucount = total;
