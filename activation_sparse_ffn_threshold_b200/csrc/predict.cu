@@ -184,40 +184,57 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
   return before + incl - v;
 }
 
-// The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
-// token t's set holds the row).  One CTA; warp w takes a contiguous run of bit words, 16
-// at a time with all 16 loads in flight: lane t reads token t's words, a word's union is
-// their OR, and 32 ballots transpose its 32 x 32 bit block into the rows' token masks.
-// Pass 1 counts each word's union bits, a block scan turns the counts into first
-// positions, pass 2 writes the rows.
-constexpr int kUnionBatch = 16;
-
-__global__ void __launch_bounds__(1024) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
-                                                int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
-                                                int32_t *__restrict__ ucount) {
-  extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
-  const int chunk = (nwords + nw - 1) / nw;
-  const int wbeg = min(nwords, warp * chunk), wend = min(nwords, wbeg + chunk);
-  // this lane's token words of bit words w0 .. w0 + kUnionBatch - 1 (zero past the run)
-  auto load = [&](int w0, uint32_t *mw) {
+// 32 x 32 bit transpose in registers: afterwards bit t of a[i] is what bit i of a[t] was.
+// Recursive block swap: exchange the off-diagonal 16 x 16 blocks, then 8 x 8 inside each
+// half, down to single bits (5 rounds of 16 masked swaps), done on bit-reversed words so
+// that bit 0 is the first column.
+__device__ __forceinline__ void transpose32(uint32_t *a) {
 #pragma unroll
-    for (int j = 0; j < kUnionBatch; ++j)
-      mw[j] = lane < b && w0 + j < wend ? __ldcg(mask + (size_t)lane * nwords + w0 + j) : 0u;
-  };
-  auto union_of = [&](int w, uint32_t mw) {
-    const uint32_t u = __reduce_or_sync(0xffffffffu, mw);
+  for (int k = 0; k < 32; ++k) a[k] = __brev(a[k]);
+  uint32_t m = 0x0000ffffu;
+#pragma unroll
+  for (int j = 16; j != 0; j >>= 1) {
+#pragma unroll
+    for (int k = 0; k < 32; k = (k + j + 1) & ~j) {
+      const uint32_t t = (a[k] ^ (a[k + j] >> j)) & m;
+      a[k] ^= t;
+      a[k + j] ^= t << j;
+    }
+    m ^= m << (j >> 1);
+  }
+#pragma unroll
+  for (int k = 0; k < 32; ++k) a[k] = __brev(a[k]);
+}
+
+// The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
+// token t's set holds the row).  One CTA of kUnionThreads.  A warp takes 32 consecutive
+// bit words at a time, lane l word w = w0 + l: its b tokens' words arrive by coalesced
+// loads (the warp reads 32 consecutive words of one token at a time), the union word is
+// their OR, and a 32 x 32 bit transpose turns them into the token masks of the word's 32
+// rows.  Pass 1 counts each word's union bits, a block scan turns the counts into first
+// positions; pass 2 stages the warp's masks in shared memory and writes the rows word by
+// word, lane i taking bit i, so that the stores of a word are contiguous.
+constexpr int kUnionThreads = 512;
+constexpr int kUnionStage = 32 * 33;  // words of one warp's staged masks (rows padded to 33)
+
+__global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
+                                                         int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
+                                                         int32_t *__restrict__ ucount) {
+  extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  uint32_t *stage = reinterpret_cast<uint32_t *>(woff + ((nwords + 3) & ~3)) + warp * kUnionStage;
+  const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
+  auto load = [&](int w, uint32_t *mw) {  // token words of bit word w (w < nwords) -> their union
+#pragma unroll
+    for (int t = 0; t < kMaxBatch; ++t) mw[t] = t < b ? __ldcg(mask + (size_t)t * nwords + w) : 0u;
+    uint32_t u = 0u;
+#pragma unroll
+    for (int t = 0; t < kMaxBatch; ++t) u |= mw[t];
     return w == nwords - 1 ? u & tail : u;
   };
-  for (int w0 = wbeg; w0 < wend; w0 += kUnionBatch) {
-    uint32_t mw[kUnionBatch];
-    load(w0, mw);
-#pragma unroll
-    for (int j = 0; j < kUnionBatch; ++j) {
-      const uint32_t u = union_of(w0 + j, mw[j]);
-      if (lane == 0 && w0 + j < wend) woff[w0 + j] = __popc(u);
-    }
+  for (int w = threadIdx.x; w < nwords; w += blockDim.x) {
+    uint32_t mw[kMaxBatch];
+    woff[w] = __popc(load(w, mw));
   }
   __syncthreads();
   const int per = (nwords + blockDim.x - 1) / blockDim.x;  // words per thread in the scan
@@ -234,26 +251,27 @@ __global__ void __launch_bounds__(1024) k_union(const uint32_t *__restrict__ mas
       run += v;
     }
   __syncthreads();
-  for (int w0 = wbeg; w0 < wend; w0 += kUnionBatch) {
-    uint32_t mw[kUnionBatch];
-    load(w0, mw);
-#pragma unroll 1
-    for (int j = 0; j < kUnionBatch; ++j) {
-      const int w = w0 + j;
-      const uint32_t u = w < wend ? union_of(w, mw[j]) : 0u;
-      if (u == 0u) continue;  // warp-uniform
-      uint32_t tb = 0u;
+  for (int w0 = warp * 32; w0 < nwords; w0 += nwarps * 32) {  // warp-uniform
+    const int w = w0 + lane;
+    uint32_t mw[kMaxBatch];
+    const uint32_t u = w < nwords ? load(w, mw) : 0u;
+    const int base = w < nwords ? woff[w] : 0;
+    if (u != 0u) {
+      transpose32(mw);  // mw[i]: the tokens whose sets hold row 32 w + i
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const uint32_t col = __ballot_sync(0xffffffffu, (mw[j] >> i) & 1u);
-        if (lane == i) tb = col;
-      }
-      if ((u >> lane) & 1u) {
-        const int pos = woff[w] + __popc(u & ((1u << lane) - 1u));
-        ulist[pos] = w * 32 + lane;
-        utok[pos] = tb;
+      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = mw[i];
+    }
+    __syncwarp();
+    for (int l = 0; l < 32; ++l) {
+      const uint32_t ul = __shfl_sync(0xffffffffu, u, l);
+      const int bl = __shfl_sync(0xffffffffu, base, l);
+      if ((ul >> lane) & 1u) {
+        const int pos = bl + __popc(ul & ((1u << lane) - 1u));
+        ulist[pos] = (w0 + l) * 32 + lane;
+        utok[pos] = stage[l * 33 + lane];
       }
     }
+    __syncwarp();
   }
   if (threadIdx.x == 0) *ucount = total;
 }
@@ -321,7 +339,8 @@ cudaError_t logits_impl(const sfnn_ctx *h, int b, cudaStream_t s) {
 }  // namespace
 
 cudaError_t configure_predict() {
-  cudaError_t e0 = cudaFuncSetAttribute(k_union, cudaFuncAttributeMaxDynamicSharedMemorySize, kUnionSmemMax);
+  cudaError_t e0 = cudaFuncSetAttribute(k_union, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kUnionSmemMax + (kUnionThreads / 32) * kUnionStage * 4);
   if (e0 != cudaSuccess) return e0;
   const void *ks[] = {(const void *)k_logits<float, 1>, (const void *)k_logits<float, 8>,
                       (const void *)k_logits<float, 32>, (const void *)k_logits<__half, 1>,
@@ -351,7 +370,8 @@ cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *i
   const Layout &L = h->L;
   cudaError_t e = cudaSuccess;
   if (want_union) {
-    k_union<<<1, 1024, (size_t)L.nwords * sizeof(int), s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
+    const size_t smem = ((size_t)(L.nwords + 3) / 4 * 4 + (size_t)(kUnionThreads / 32) * kUnionStage) * 4;
+    k_union<<<1, kUnionThreads, smem, s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && (idx_out || cnt_out)) {
