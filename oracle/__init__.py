@@ -66,7 +66,7 @@ def _load():
         lib.oracle_ffn_masked.restype = None
         lib.oracle_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, I]
         lib.oracle_forward.restype = I
-        lib.oracle_quantize.argtypes = [I, I, I, P, L, L, P, P]
+        lib.oracle_quantize.argtypes = [I, I, I, P, L, L, I, P, P]
         lib.oracle_quantize.restype = None
         lib.oracle_ffn_masked_q.argtypes = [I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, I]
         lib.oracle_ffn_masked_q.restype = None
@@ -180,10 +180,14 @@ class QRows:
     s_down: np.ndarray
 
 
-def quantize(w, units_along_rows: bool = True):
-    """Per-unit symmetric int8 codes of a 2-D array (units = rows, or columns when
-    ``units_along_rows`` is False): fp32 scale = absmax / 127, codes rounded to nearest
-    even in fp32 and clamped to [-127, 127].  Returns (q [units, len] int8, s [units])."""
+QMAX = {8: 127, 4: 7}
+
+
+def quantize(w, units_along_rows: bool = True, bits: int = 8):
+    """Per-unit symmetric codes of a 2-D array (units = rows, or columns when
+    ``units_along_rows`` is False), 8 or 4 bits: fp32 scale = absmax / qmax (127 or 7),
+    codes rounded to nearest even in fp32 and clamped to [-qmax, qmax].
+    Returns (q [units, len] int8, one code per byte; s [units])."""
     w = _c(w)
     assert w.ndim == 2
     rows, cols = w.shape
@@ -191,16 +195,16 @@ def quantize(w, units_along_rows: bool = True):
     ustride, estride = (cols, 1) if units_along_rows else (1, cols)
     q = np.empty((units, length), np.int8)
     sc = np.empty(units, np.float32)
-    _load().oracle_quantize(units, length, _dt(w), _p(w), ustride, estride, _p(q), _p(sc))
+    _load().oracle_quantize(units, length, _dt(w), _p(w), ustride, estride, QMAX[bits], _p(q), _p(sc))
     return q, sc
 
 
-def quantize_layer(layer) -> QRows:
-    q_up, s_up = quantize(layer.w_up)
+def quantize_layer(layer, bits: int = 8) -> QRows:
+    q_up, s_up = quantize(layer.w_up, bits=bits)
     q_gate = s_gate = None
     if layer.w_gate is not None:
-        q_gate, s_gate = quantize(layer.w_gate)
-    q_down, s_down = quantize(layer.w_down, units_along_rows=False)
+        q_gate, s_gate = quantize(layer.w_gate, bits=bits)
+    q_down, s_down = quantize(layer.w_down, units_along_rows=False, bits=bits)
     return QRows(q_up, s_up, q_gate, s_gate, q_down, s_down)
 
 

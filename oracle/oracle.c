@@ -175,18 +175,20 @@ int32_t oracle_forward(int32_t d, int32_t n, int32_t r, int32_t act, int32_t dt,
 }
 
 /*
- * Weight-only int8 rows (a NEXT step of the method: PowerInfer runs its weights in INT4
- * on the smaller PC, 53ai.com page, section on evaluation; only the rows' storage
- * changes, the arithmetic stays that of the FFN above).
+ * Weight-only int8 and int4 rows (a NEXT step of the method: PowerInfer runs its weights
+ * in INT4 on the smaller PC, 53ai.com page, section on evaluation; only the rows'
+ * storage changes, the arithmetic stays that of the FFN above).
  *
  * Quantisation of `units` units of `len` elements each (element k of unit i at
- * w[i*unit_stride + k*elem_stride]): in IEEE fp32, scale_i = max_k |w_ik| / 127 and
- * q_ik = round-to-nearest-even(w_ik / scale_i), clamped to [-127, 127]; an all-zero
+ * w[i*unit_stride + k*elem_stride]) to symmetric codes in [-qmax, qmax] (qmax = 127 for
+ * int8, 7 for int4): in IEEE fp32, scale_i = max_k |w_ik| / qmax and
+ * q_ik = round-to-nearest-even(w_ik / scale_i), clamped to [-qmax, qmax]; an all-zero
  * unit has scale 0 and codes 0.  The decision is taken in fp32 so that any fp32
- * implementation of the same rule gives the same codes.  q is unit-major.
+ * implementation of the same rule gives the same codes.  q is unit-major, one code per
+ * byte whatever qmax.
  */
 void oracle_quantize(int32_t units, int32_t len, int32_t dt, const void *w, int64_t unit_stride,
-                     int64_t elem_stride, int8_t *q, float *scale) {
+                     int64_t elem_stride, int32_t qmax, int8_t *q, float *scale) {
     init_table();
     for (int32_t i = 0; i < units; ++i) {
         float amax = 0.0f;
@@ -194,21 +196,21 @@ void oracle_quantize(int32_t units, int32_t len, int32_t dt, const void *w, int6
             const float v = fabsf((float)ld(w, dt, (size_t)(i * unit_stride + k * elem_stride)));
             if (v > amax) amax = v;
         }
-        const float s = amax / 127.0f;
+        const float s = amax / (float)qmax;
         scale[i] = s;
         for (int32_t k = 0; k < len; ++k) {
             int32_t c = 0;
             if (s > 0.0f) {
                 const float v = (float)ld(w, dt, (size_t)(i * unit_stride + k * elem_stride));
                 c = (int32_t)rintf(v / s);
-                c = c > 127 ? 127 : (c < -127 ? -127 : c);
+                c = c > qmax ? qmax : (c < -qmax ? -qmax : c);
             }
             q[(size_t)i * len + k] = (int8_t)c;
         }
     }
 }
 
-/* The FFN of oracle_ffn_masked with int8 rows: every weight is q * scale (exact in
+/* The FFN of oracle_ffn_masked with quantised rows: every weight is q * scale (exact in
  * double).  q_up/q_gate [n][d] with scales [n]; q_down [n][d] neuron-major (neuron i's
  * down row, i.e. column i of w_down) with scales [n].  x and b in dt. */
 void oracle_ffn_masked_q(int32_t d, int32_t n, int32_t act, int32_t dt, const void *x, const int8_t *q_up,

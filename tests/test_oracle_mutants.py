@@ -39,7 +39,7 @@ MUTANTS = {
     "reglu_gate_bias_dropped": ("g += ld(bias, dt, i);", "g += 0.0;"),
     "preact_bias_dropped": ("g[i] = s + ld(bias, dt, i);", "g[i] = s;"),
     # int8 rows
-    "quant_scale_by_128": ("const float s = amax / 127.0f;", "const float s = amax / 128.0f;"),
+    "quant_scale_by_qmax_plus_1": ("const float s = amax / (float)qmax;", "const float s = amax / (float)(qmax + 1);"),
     "quant_round_half_away": ("c = (int32_t)rintf(v / s);", "c = (int32_t)roundf(v / s);"),
     "quant_truncates": ("c = (int32_t)rintf(v / s);", "c = (int32_t)(v / s);"),
     "q_down_scale_of_up": ("* (double)s_down[i]);", "* (double)s_up[i]);"),
@@ -72,8 +72,11 @@ def _pin_calls(pins):
             calls.append(lambda dt=dt, act=act: pins.test_exact_set_equals_dense(act, dt))
     for act in ("relu", "reglu"):
         calls.append(lambda act=act: pins.test_all_ones_mask_equals_dense(act))
-        calls.append(lambda act=act: pins.test_forward_q_equals_forward_on_an_exact_grid(act))
-    calls += [pins.test_quantizer_hand_values, pins.test_quantizer_invariants, pins.test_lookahead_hand_example]
+        for bits in (8, 4):
+            calls.append(lambda act=act, bits=bits: pins.test_forward_q_equals_forward_on_an_exact_grid(act, bits))
+    calls += [pins.test_quantizer_hand_values, pins.test_quantizer_hand_values_int4, pins.test_lookahead_hand_example]
+    for bits in (8, 4):
+        calls.append(lambda bits=bits: pins.test_quantizer_invariants(bits))
     return calls
 
 
@@ -95,7 +98,7 @@ def _bind(path):
         real = oracle._load()
         lib = ctypes.CDLL(path)
         for fn in ("oracle_decode", "oracle_predictor", "oracle_preact", "oracle_ffn_masked",
-                   "oracle_forward", "oracle_max_threads"):
+                   "oracle_forward", "oracle_max_threads", "oracle_quantize", "oracle_ffn_masked_q"):
             getattr(lib, fn).argtypes = getattr(real, fn).argtypes
             getattr(lib, fn).restype = getattr(real, fn).restype
         return lib
@@ -125,14 +128,16 @@ def test_mutant_is_caught(name):
     assert failures > 0, f"no pin caught mutant {name}"
 
 
-# The look-ahead stack is bookkeeping in oracle/__init__.py: its mutants are copies of
-# that module with one mistake, loaded beside the real one (same compiled library).
+# The look-ahead stack and the code widths are bookkeeping in oracle/__init__.py: their
+# mutants are copies of that module with one mistake, loaded beside the real one (same
+# compiled library).
 PY_SRC = os.path.join(os.path.dirname(HERE), "oracle", "__init__.py")
 PY_MUTANTS = {
     "lookahead_from_current_input": ('xpred = xin if li == 0 else records[li - 1]["x_in"]', "xpred = xin"),
     "lookahead_residual_dropped": ("""        records.append(dict(x_in=xin, x_pred=xpred, z=z, mask=mask, y=y, mismatches=mismatches))
         resid = resid + y""", """        records.append(dict(x_in=xin, x_pred=xpred, z=z, mask=mask, y=y, mismatches=mismatches))
         resid = y"""),
+    "int4_qmax_8": ("QMAX = {8: 127, 4: 7}", "QMAX = {8: 127, 4: 8}"),
     "lookahead_input_not_rounded": ("""        xin = resid.astype(dt)  # round to nearest even
         xpred = xin if""", """        xin = resid.copy()
         xpred = xin if"""),
@@ -152,7 +157,8 @@ def test_python_mutant_is_caught(name):
     pins = _pins_module()
     pins.oracle = mod
     failures = 0
-    for call in (pins.test_lookahead_hand_example, lambda: pins.test_lookahead_special_cases_equal_the_stack("relu")):
+    for call in (pins.test_lookahead_hand_example, lambda: pins.test_lookahead_special_cases_equal_the_stack("relu"),
+                 pins.test_quantizer_hand_values_int4):
         try:
             call()
         except AssertionError:

@@ -15,9 +15,9 @@
 * the look-ahead stack (layer l+1's set predicted from layer l's input): a
   two-layer example worked by hand where predicting one layer early changes the
   set and the output, and the special cases where it must equal the plain stack;
-* int8 rows: the quantizer's codes and scales worked by hand (ties to even, zero
-  rows), its error bound, and the int8-row step equal to the fp16 step on weights
-  that lie exactly on an int8 grid.
+* int8 and int4 rows: the quantizer's codes and scales worked by hand (ties to even,
+  zero rows), its error bound, and the quantized-row step equal to the fp16 step on
+  weights that lie exactly on an int8 or int4 grid.
 """
 import json
 import os
@@ -338,49 +338,63 @@ def test_quantizer_hand_values():
     assert np.array_equal(qc, q) and np.array_equal(sc, s)
 
 
-def test_quantizer_invariants():
+def test_quantizer_hand_values_int4():
+    """qmax 7: absmax 7 gives scale 1 (-3.25 -> -3, 2.5 -> 2, 0.75 -> 1), absmax 14 gives
+    scale 2 (1.5 -> 2, -2.5 -> -2, 0.5 -> 0), an all-zero row scale 0 and codes 0."""
+    w = np.array([[7, -3.25, 2.5, 0.75, -7], [14, 3, -5, 1, 0], [0, 0, 0, 0, 0]], np.float16)
+    q, s = oracle.quantize(w, bits=4)
+    assert q.tolist() == [[7, -3, 2, 1, -7], [7, 2, -2, 0, 0], [0, 0, 0, 0, 0]]
+    assert s.tolist() == [1.0, 2.0, 0.0]
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_quantizer_invariants(bits):
+    qmax = 127 if bits == 8 else 7
     rng = np.random.default_rng(7)
     w = (rng.standard_normal((40, 96)) * rng.uniform(0.01, 3.0, (40, 1))).astype(np.float16)
     w[5] = 0
-    q, s = oracle.quantize(w)
+    q, s = oracle.quantize(w, bits=bits)
     wf = w.astype(np.float64)
-    assert np.all(np.abs(q.astype(int)) <= 127)
+    assert np.all(np.abs(q.astype(int)) <= qmax)
     nz = np.abs(wf).max(axis=1) > 0
-    assert np.all(np.abs(q[nz]).max(axis=1) == 127)
+    assert np.all(np.abs(q[nz]).max(axis=1) == qmax)
     assert np.all(s[~nz] == 0) and np.all(q[~nz] == 0)
     # |w - q s| <= s / 2, up to the fp32 rounding of w / s
     err = np.abs(wf - q.astype(np.float64) * s[:, None].astype(np.float64))
     assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 1e-5))
-    # the scale is the fp32 quotient absmax / 127
+    # the scale is the fp32 quotient absmax / qmax
     amax = np.abs(w.astype(np.float32)).max(axis=1)
-    assert np.array_equal(s, (amax / np.float32(127)).astype(np.float32))
+    assert np.array_equal(s, (amax / np.float32(qmax)).astype(np.float32))
 
 
+@pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("act", ["relu", "reglu"])
-def test_forward_q_equals_forward_on_an_exact_grid(act):
-    """Weights that are int8 codes times 2^-7 (up, gate) or 2^-6 (down), exact in fp16,
-    each unit reaching +-127: quantization gives back those codes and scales, and the
-    int8-row step equals the fp16 step exactly."""
+def test_forward_q_equals_forward_on_an_exact_grid(act, bits):
+    """Weights that are codes times 2^-7 (int8) or 2^-3 (int4) for up and gate and twice
+    that for down, exact in fp16, each unit reaching +-qmax: quantization gives back those
+    codes and scales, and the quantized-row step equals the fp16 step exactly."""
+    qmax = 127 if bits == 8 else 7
+    unit = 2.0 ** -7 if bits == 8 else 2.0 ** -3
     rng = np.random.default_rng(8)
     d, n, r = 48, 40, 16
 
     def grid(units, length):
-        q = rng.integers(-127, 128, (units, length))
-        q[np.arange(units), rng.integers(0, length, units)] = 127
+        q = rng.integers(-qmax, qmax + 1, (units, length))
+        q[np.arange(units), rng.integers(0, length, units)] = qmax
         return q
 
     q_up, q_gate, q_down_t = grid(n, d), grid(n, d), grid(n, d)
-    w_up = (q_up / 128.0).astype(np.float16)
-    w_gate = (q_gate / 128.0).astype(np.float16) if act == "reglu" else None
-    w_down = np.ascontiguousarray((q_down_t / 64.0).astype(np.float16).T)  # another scale than up's
+    w_up = (q_up * unit).astype(np.float16)
+    w_gate = (q_gate * unit).astype(np.float16) if act == "reglu" else None
+    w_down = np.ascontiguousarray((q_down_t * 2 * unit).astype(np.float16).T)  # another scale than up's
     b = (rng.standard_normal(n) * 0.1).astype(np.float16)
     A = (rng.standard_normal((d, r)) * 0.3).astype(np.float16)
     B = (rng.standard_normal((r, n)) * 0.3).astype(np.float16)
     c = (rng.standard_normal(n) * 0.1).astype(np.float16)
     lay = _L(act, w_up, w_gate, b, w_down, A, B, c)
-    qr = oracle.quantize_layer(lay)
-    assert np.array_equal(qr.q_up, q_up) and np.all(qr.s_up == np.float32(2.0 ** -7))
-    assert np.array_equal(qr.q_down, q_down_t) and np.all(qr.s_down == np.float32(2.0 ** -6))
+    qr = oracle.quantize_layer(lay, bits=bits)
+    assert np.array_equal(qr.q_up, q_up) and np.all(qr.s_up == np.float32(unit))
+    assert np.array_equal(qr.q_down, q_down_t) and np.all(qr.s_down == np.float32(2 * unit))
     for t in range(3):
         x = rng.standard_normal(d).astype(np.float16)
         ref = oracle.forward(lay, x)
