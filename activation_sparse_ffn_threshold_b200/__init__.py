@@ -21,10 +21,10 @@ import torch
 
 __all__ = ["SparseFFN", "SfnnError", "forward_stack", "predict_noalloc", "hotness_order", "library_path",
            "load_library",
-           "RELU", "REGLU", "F32", "F16", "I8", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
+           "RELU", "REGLU", "F32", "F16", "I8", "I4", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
 
 RELU, REGLU = 0, 1
-F32, F16, I8 = 0, 1, 2
+F32, F16, I8, I4 = 0, 1, 2, 3
 BATCH_AUTO, BATCH_CUDA_CORE, BATCH_TENSOR_CORE = 0, 1, 2
 STATUS = {0: "SFNN_OK", 1: "SFNN_ERR_INVALID_ARG", 2: "SFNN_ERR_CUDA", 3: "SFNN_ERR_OOM",
           4: "SFNN_ERR_UNSUPPORTED", 5: "SFNN_ERR_TIMEOUT"}
@@ -159,8 +159,11 @@ class SparseFFN:
 
     def __init__(self, w_up, w_down, b, A, B, c, act: str = "relu", w_gate=None, hotness=None,
                  max_batch: int = 1, device=None, stream=None, rows: str | None = None):
-        """``rows="int8"`` stores the FFN rows as int8 codes with per-row fp32 scales
-        (fp16 layers; single-token fused path only, see sfnn_layer_desc.rows_dtype)."""
+        """``rows="int8"`` / ``"int4"`` stores the FFN rows as int8 / int4 codes with
+        per-row fp32 scales (fp16 layers; single-token fused path only, see
+        sfnn_layer_desc.rows_dtype)."""
+        if rows not in (None, "int8", "int4"):
+            raise ValueError("rows must be None, 'int8' or 'int4'")
         lib = load_library()
         device = torch.device(device or "cuda")
         dtype = w_up.dtype if isinstance(w_up, torch.Tensor) else torch.from_numpy(np.asarray(w_up[:1])).dtype
@@ -184,7 +187,7 @@ class SparseFFN:
                          w_up_t.data_ptr(), w_gate_t.data_ptr() if w_gate_t is not None else None,
                          b_t.data_ptr(), w_down_t.data_ptr(), A_t.data_ptr(), B_t.data_ptr(), c_t.data_ptr(),
                          self._hot.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if self._hot is not None
-                         else None, I8 if rows == "int8" else 0)
+                         else None, {"int8": I8, "int4": I4}.get(rows, 0))
         self.rows = rows
         self._h = ctypes.c_void_p()
         with torch.cuda.device(device):

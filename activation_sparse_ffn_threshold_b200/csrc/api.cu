@@ -59,6 +59,7 @@ sfnn_status check_desc(const sfnn_layer_desc *d) {
   if (d->d < 1 || d->n < 1 || d->r < 1) return SFNN_ERR_INVALID_ARG;
   if (d->max_batch < 1) return SFNN_ERR_INVALID_ARG;
   if (d->rows_dtype == SFNN_I8 && (d->wdtype != SFNN_F16 || d->d % 16)) return SFNN_ERR_UNSUPPORTED;
+  if (d->rows_dtype == SFNN_I4 && (d->wdtype != SFNN_F16 || d->d % 32)) return SFNN_ERR_UNSUPPORTED;
   if (!d->w_up || !d->b || !d->w_down || !d->pa || !d->pb || !d->pc) return SFNN_ERR_INVALID_ARG;
   if (d->act == SFNN_REGLU && !d->w_gate) return SFNN_ERR_INVALID_ARG;
   const int vec = d->wdtype == SFNN_F16 ? 8 : 4;
@@ -104,7 +105,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
   cudaEvent_t before = h->prof_before, after = h->prof_after;
   const bool predict = src == kSetPredict;
   const bool fused = b == 1 && predict && !ahead && !idx_out && !cnt_out && h->fused_ok && h->fused_on;
-  if (h->L.rows_i8 && !fused) return SFNN_ERR_UNSUPPORTED;  // int8 rows: the fused path only
+  if (h->L.rows_q && !fused) return SFNN_ERR_UNSUPPORTED;  // quantized rows: the fused path only
   h->prof_before = h->prof_after = nullptr;
   record_if(before, s);
   if (fused) {
@@ -172,9 +173,9 @@ void plan_decode1(sfnn_ctx *h, int G) {
   P.dt = L.dt;
   P.G = G;
   P.tile_max = (L.n + G - 1) / G;
-  P.ri8 = L.rows_i8;
+  P.rq = L.rows_q;
   P.rscale = h->rscale;
-  P.nseg = (L.d / (L.rows_i8 ? 16 : L.vec) + 255) / 256;  // 4 KB C1 segments of a row
+  P.nseg = (L.d / (L.rows_q ? 128 / L.rows_q : L.vec) + 255) / 256;  // 4 KB C1 segments of a row
   if (L.r / L.vec > 32 * 4) return;
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
@@ -276,7 +277,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   L.esize = desc->wdtype == SFNN_F16 ? 2 : 4;
   L.vec = 16 / L.esize;
   L.nwords = (L.n + 31) / 32;
-  L.rows_i8 = desc->rows_dtype == SFNN_I8;
+  L.rows_q = desc->rows_dtype == SFNN_I8 ? 8 : (desc->rows_dtype == SFNN_I4 ? 4 : 0);
   h->max_batch = desc->max_batch;
   h->batch_path = SFNN_BATCH_AUTO;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
@@ -316,8 +317,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
     size_t bytes;
     bool weight;
   } reqs[] = {
-      {&h->rows, n * L.nproj * d * (L.rows_i8 ? 1 : e), true},
-      {(void **)&h->rscale, L.rows_i8 ? n * L.nproj * 4 : 0, true},
+      {&h->rows, L.rows_q ? n * L.nproj * d * L.rows_q / 8 : n * L.nproj * d * e, true},
+      {(void **)&h->rscale, L.rows_q ? n * L.nproj * 4 : 0, true},
       {&h->At, r * d * e, true},
       {&h->Bt, n * r * e, true},
       {&h->cvec, n * e, true},
@@ -336,8 +337,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->bar, sizeof(uint64_t), false},
       {(void **)&h->alist, n * sizeof(int2), false},
       {(void **)&h->acnt, (size_t)G * 4, false},
-      {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_i8 && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
-      {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_i8 && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
+      {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
+      {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
   };
   for (auto &q : reqs) {
     if (q.bytes == 0) continue;  // not needed by this layer
@@ -367,7 +368,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
     free_handle(h);
     return from_cuda(ce);
   }
-  if (L.rows_i8 && !h->fused_ok) {  // int8 rows run the fused kernel only
+  if (L.rows_q && !h->fused_ok) {  // quantized rows run the fused kernel only
     free_handle(h);
     return SFNN_ERR_UNSUPPORTED;
   }
@@ -488,7 +489,7 @@ sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
 sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   if (enable && !h->fused_ok) return SFNN_ERR_UNSUPPORTED;
-  if (!enable && h->L.rows_i8) return SFNN_ERR_UNSUPPORTED;  // int8 rows run the fused path only
+  if (!enable && h->L.rows_q) return SFNN_ERR_UNSUPPORTED;  // quantized rows run the fused path only
   h->fused_on = enable != 0;
   return SFNN_OK;
 }
@@ -525,7 +526,7 @@ sfnn_status sfnn_query(sfnn_handle h, sfnn_info *info) {
   info->weight_bytes = h->weight_bytes;
   info->scratch_bytes = h->scratch_bytes;
   info->predictor_bytes = ((int64_t)L.d * L.r + (int64_t)L.r * L.n + L.n) * L.esize;
-  info->row_bytes_per_neuron = L.rows_i8 ? (int64_t)L.nproj * L.d + (int64_t)L.nproj * 4 + L.esize
+  info->row_bytes_per_neuron = L.rows_q ? (int64_t)L.nproj * L.d * L.rows_q / 8 + (int64_t)L.nproj * 4 + L.esize
                                          : ((int64_t)L.nproj * L.d + 1) * L.esize;
   info->launches = h->launches;
   return SFNN_OK;

@@ -19,7 +19,7 @@ constexpr int kErrTimeout = SFNN_ERR_TIMEOUT;
 
 struct Layout {
   int d, n, r, nproj, act, dt, esize, vec, nwords;
-  int rows_i8;  // rows stored as int8 codes with per-row fp32 scales
+  int rows_q;  // rows stored as 8- or 4-bit codes with per-row fp32 scales (0: in dt)
 };
 
 }  // namespace sfnn
@@ -46,7 +46,7 @@ struct sfnn_ctx {
   uint32_t *utok;    // [n] tokens active on each union row (bit t)
   int32_t *ucount;   // [1]
   float *acoef;      // [n][max_batch] activation of each union row for each token
-  float *rscale;     // [n][nproj] scales of int8 rows (storage order), or null
+  float *rscale;     // [n][nproj] scales of quantized rows (storage order), or null
   __half *hact;      // [32][n rounded up to 128] fp16 activations (tensor-core batch path) or null
   __half *hpair;     // [2][32][r] the batch's hidden layer as fp16 hi and lo parts (same path)
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection

@@ -48,8 +48,9 @@ namespace {
 template <typename T, int ACT, int MAXM, typename R>
 __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr int V = Elem<T>::kVec;
-  constexpr bool I8 = sizeof(R) == 1;  // int8 rows: codes with per-row scales
-  constexpr int VR = 16 / sizeof(R);   // row elements per 16-byte chunk
+  constexpr int RB = RowFmt<R>::kBits;  // bits of a stored row element
+  constexpr bool QR = RB <= 8;           // rows are codes with per-row scales
+  constexpr int VR = 128 / RB;           // row elements per 16-byte chunk
   constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
   constexpr int DB = kDecode1BStages;
   constexpr int DD = decode1_dstages(MAXM);
@@ -78,7 +79,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int nch_d = d / V, nch_r = r / V;
   const T *At = static_cast<const T *>(P.At);
   const T *Bt = static_cast<const T *>(P.Bt);
-  const R *rows = static_cast<const R *>(P.rows);
+  const unsigned char *rows = static_cast<const unsigned char *>(P.rows);
+  const size_t rowB = (size_t)P.d * RB / 8;  // bytes of one stored row
 
   pdl_launch_dependents();
   const int j0 = c + G * warp;  // this warp's first row of A^T
@@ -243,15 +245,18 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
     if (k < cnt) {
-      const R *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * d;
+      const unsigned char *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * rowB;
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
-        const int ch = tid + kT * m;  // V columns (int8 rows: their V codes, 8 bytes)
+        const int ch = tid + kT * m;  // V columns (code rows: their V codes, 8 or 4 bytes)
         if (ch < nch_d) {
-          if (I8)
-            cp_async8(dslot(s, m), row + (size_t)ch * V);
+          const unsigned char *src = row + (size_t)ch * V * RB / 8;
+          if (RB == 4)
+            cp_async4(dslot(s, m), src);
+          else if (RB == 8)
+            cp_async8(dslot(s, m), src);
           else
-            cp_async16(dslot(s, m), row + (size_t)ch * V);
+            cp_async16(dslot(s, m), src);
         }
       }
     }
@@ -273,11 +278,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       const int it = warp + kW * s;
       if (it < items) {
         const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
-        const R *row = rows + ((size_t)act_s[k] * nproj + pj) * d;
+        const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
           const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
+          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
         }
       }
     }
@@ -294,7 +299,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
           for (int u = 0; u < SU; ++u) {
             const int ch = sg * kSegChunks + lane + 32 * u;
             if (ch < nch_r8) {
-              if (I8)
+              if (RB == 4)
+                a = dot_chunk_i4(wc[s][u], xs, ch, a);
+              else if (RB == 8)
                 a = dot_chunk_i8(wc[s][u], xs, ch, a);
               else
                 a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
@@ -303,11 +310,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
           const int itn = it + D * kW;
           if (itn < items) {
             const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
-            const R *row = rows + ((size_t)act_s[kn] * nproj + pjn) * d;
+            const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
               const int ch = sgn * kSegChunks + lane + 32 * u;
-              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * VR);
+              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
             }
           }
           a = warp_sum(a);
@@ -322,7 +329,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       if (ACT == SFNN_REGLU)
         for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
       float sd = 1.f;
-      if (I8) {  // the codes' sums times their rows' scales; the down row's folded into a
+      if (QR) {  // the codes' sums times their rows' scales; the down row's folded into a
         const float *sc = P.rscale + (size_t)act_s[k] * nproj;
         g *= sc[0];
         if (ACT == SFNN_REGLU) u *= sc[1];
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       const float pre = g + bias_s[k];
       const float relu = pre > 0.f ? pre : 0.f;
       a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
-      if (I8) a_s[k] *= sd;
+      if (QR) a_s[k] *= sd;
     }
     __syncthreads();
   }
@@ -353,7 +360,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         for (int m = 0; m < MAXM; ++m) {
           if (tid + kT * m < nch_d) {
             float f[V];
-            if (I8) {
+            if (RB == 4) {
+              const uint32_t q = *reinterpret_cast<const uint32_t *>(dslot(s, m));
+#pragma unroll
+              for (int v = 0; v < V; ++v) f[v] = (float)((int32_t)(q << (28 - 4 * v)) >> 28);
+            } else if (RB == 8) {
               const uint2 q = *reinterpret_cast<const uint2 *>(dslot(s, m));
 #pragma unroll
               for (int v = 0; v < V; ++v) f[v] = (float)(int8_t)((v < 4 ? q.x : q.y) >> (8 * (v & 3)));
@@ -459,13 +470,14 @@ cudaError_t config_act() {
   return cudaSuccess;
 }
 
-// The kernel for this plan: element types (fp32, fp16, or fp16 with int8 rows) and activation.
+// The kernel for this plan: element types (fp32, fp16, or fp16 with int8 / int4 rows) and activation.
 const void *plan_kernel(const Decode1Params &P, int nch) {
   if (P.dt != SFNN_F16)
     return P.act == SFNN_REGLU ? pick_kernel<float, SFNN_REGLU, float>(nch) : pick_kernel<float, SFNN_RELU, float>(nch);
-  if (P.ri8)
-    return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, int8_t>(nch)
-                               : pick_kernel<__half, SFNN_RELU, int8_t>(nch);
+  if (P.rq == 8)
+    return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, Q8>(nch) : pick_kernel<__half, SFNN_RELU, Q8>(nch);
+  if (P.rq == 4)
+    return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, Q4>(nch) : pick_kernel<__half, SFNN_RELU, Q4>(nch);
   return P.act == SFNN_REGLU ? pick_kernel<__half, SFNN_REGLU, __half>(nch)
                              : pick_kernel<__half, SFNN_RELU, __half>(nch);
 }
@@ -477,8 +489,10 @@ cudaError_t configure_decode1() {
   if (e == cudaSuccess) e = config_act<float, SFNN_REGLU, float>();
   if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, __half>();
   if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, __half>();
-  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, int8_t>();
-  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, int8_t>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, Q8>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, Q8>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_RELU, Q4>();
+  if (e == cudaSuccess) e = config_act<__half, SFNN_REGLU, Q4>();
   return e;
 }
 
@@ -503,9 +517,12 @@ cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl
   if (P.dt != SFNN_F16)
     return P.act == SFNN_REGLU ? launch_act<float, SFNN_REGLU, float>(P, smem, stream, pdl)
                                : launch_act<float, SFNN_RELU, float>(P, smem, stream, pdl);
-  if (P.ri8)
-    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, int8_t>(P, smem, stream, pdl)
-                               : launch_act<__half, SFNN_RELU, int8_t>(P, smem, stream, pdl);
+  if (P.rq == 8)
+    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, Q8>(P, smem, stream, pdl)
+                               : launch_act<__half, SFNN_RELU, Q8>(P, smem, stream, pdl);
+  if (P.rq == 4)
+    return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, Q4>(P, smem, stream, pdl)
+                               : launch_act<__half, SFNN_RELU, Q4>(P, smem, stream, pdl);
   return P.act == SFNN_REGLU ? launch_act<__half, SFNN_REGLU, __half>(P, smem, stream, pdl)
                              : launch_act<__half, SFNN_RELU, __half>(P, smem, stream, pdl);
 }

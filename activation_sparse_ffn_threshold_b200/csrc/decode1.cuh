@@ -33,7 +33,7 @@ struct Decode1Params {
   int G;         // CTAs (one per SM) = tiles of neurons
   int tile_max;  // largest tile
   int nseg;      // 4 KB segments of one projection row (C1 work items per row and projection)
-  int ri8;       // rows are int8 codes; rscale [n][nproj] their fp32 scales
+  int rq;        // rows are 8- or 4-bit codes (0: dt); rscale [n][nproj] their fp32 scales
   const float *rscale;
 };
 

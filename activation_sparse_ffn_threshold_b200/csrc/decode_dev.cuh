@@ -7,6 +7,25 @@
 #include "decode1.cuh"
 
 namespace sfnn {
+
+// Storage of the FFN rows a decode kernel reads: the layer's element type, or codes with
+// per-row scales (Q8: int8, one per byte; Q4: int4, two per byte, element 2k in the low
+// nibble of byte k).
+struct Q8 {};
+struct Q4 {};
+template <typename R>
+struct RowFmt {
+  static constexpr int kBits = 8 * (int)sizeof(R);
+};
+template <>
+struct RowFmt<Q8> {
+  static constexpr int kBits = 8;
+};
+template <>
+struct RowFmt<Q4> {
+  static constexpr int kBits = 4;
+};
+
 namespace {
 
 constexpr int kT = kDecode1Threads;
@@ -33,6 +52,21 @@ __device__ __forceinline__ float dot_chunk_i8(const uint4 &w, const unsigned cha
   const uint32_t q[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int i = 0; i < 16; ++i) a = fmaf((float)(int8_t)(q[i >> 2] >> (8 * (i & 3))), xf[i], a);
+  return a;
+}
+
+// 32 int4 codes of a row (one 16-byte chunk) against x[32 ch .. 32 ch + 31] (fp16 in
+// shared memory), 8 codes per 32-bit word, low nibble first; the row's scale is applied
+// to the finished sum.
+__device__ __forceinline__ float dot_chunk_i4(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    float xf[8];
+    unpack<__half>(*reinterpret_cast<const uint4 *>(xs + (size_t)ch * 64 + h * 16), xf);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a = fmaf((float)((int32_t)(q[h] << (28 - 4 * j)) >> 28), xf[j], a);
+  }
   return a;
 }
 

@@ -83,11 +83,14 @@ cudaError_t layout_impl(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s
   return cudaGetLastError();
 }
 
-// Int8 rows: one CTA per (neuron, projection) row of d fp16 values; in fp32, scale =
-// max|w| / 127 and code = w / scale rounded to nearest even, clamped to +-127 (an
-// all-zero row: scale 0, codes 0).
+// Quantized rows: one CTA per (neuron, projection) row of d fp16 values; in fp32, scale =
+// max|w| / qmax and code = w / scale rounded to nearest even, clamped to +-qmax, with
+// qmax = 127 (int8, one code per byte) or 7 (int4, two per byte, element 2k in the low
+// nibble of byte k); an all-zero row: scale 0, codes 0.
+template <int BITS>
 __global__ void __launch_bounds__(256) k_quantize_rows(const __half *__restrict__ src, int d,
-                                                       int8_t *__restrict__ q, float *__restrict__ scale) {
+                                                       uint8_t *__restrict__ q, float *__restrict__ scale) {
+  constexpr int QMAX = BITS == 8 ? 127 : 7;
   __shared__ float red[8];
   const size_t u = blockIdx.x;
   const __half *w = src + u * d;
@@ -104,26 +107,32 @@ __global__ void __launch_bounds__(256) k_quantize_rows(const __half *__restrict_
     if (threadIdx.x == 0) red[0] = v;
   }
   __syncthreads();
-  const float sc = red[0] / 127.0f;
+  const float sc = red[0] / (float)QMAX;
   if (threadIdx.x == 0) scale[u] = sc;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+  auto code = [&](int k) {
     int c = 0;
     if (sc > 0.f) {
       c = __float2int_rn(__half2float(w[k]) / sc);
-      c = c > 127 ? 127 : (c < -127 ? -127 : c);
+      c = c > QMAX ? QMAX : (c < -QMAX ? -QMAX : c);
     }
-    q[u * d + k] = (int8_t)c;
+    return c;
+  };
+  if (BITS == 8) {
+    for (int k = threadIdx.x; k < d; k += blockDim.x) q[u * d + k] = (uint8_t)(int8_t)code(k);
+  } else {  // two codes per byte, element 2k in the low nibble
+    for (int k = threadIdx.x; k < d / 2; k += blockDim.x)
+      q[u * (d / 2) + k] = (uint8_t)((code(2 * k) & 0xf) | ((code(2 * k + 1) & 0xf) << 4));
   }
 }
 
 }  // namespace
 
 cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s) {
-  if (!h->L.rows_i8) {
+  if (!h->L.rows_q) {
     if (h->L.esize == 2) return layout_impl<uint16_t>(h, desc, s);
     return layout_impl<uint32_t>(h, desc, s);
   }
-  // fp16 rows in a temporary buffer, then their int8 codes and scales
+  // fp16 rows in a temporary buffer, then their codes and scales
   const Layout &L = h->L;
   void *codes = h->rows, *tmp = nullptr;
   const size_t units = (size_t)L.n * L.nproj;
@@ -133,8 +142,12 @@ cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t
   e = layout_impl<uint16_t>(h, desc, s);
   h->rows = codes;
   if (e == cudaSuccess) {
-    k_quantize_rows<<<(unsigned)units, 256, 0, s>>>(static_cast<const __half *>(tmp), L.d,
-                                                   static_cast<int8_t *>(codes), h->rscale);
+    if (L.rows_q == 8)
+      k_quantize_rows<8><<<(unsigned)units, 256, 0, s>>>(static_cast<const __half *>(tmp), L.d,
+                                                        static_cast<uint8_t *>(codes), h->rscale);
+    else
+      k_quantize_rows<4><<<(unsigned)units, 256, 0, s>>>(static_cast<const __half *>(tmp), L.d,
+                                                        static_cast<uint8_t *>(codes), h->rscale);
     e = cudaGetLastError();
   }
   const cudaError_t e2 = cudaStreamSynchronize(s);

@@ -60,8 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--rows", choices=["native", "int8"], default="native",
-                    help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 "
+    ap.add_argument("--rows", choices=["native", "int8", "int4"], default="native",
+                    help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 / int4 "
                          "codes with per-row scales")
     ap.add_argument("--stack", action="store_true",
                     help="time the residual stack of the workload's layers (default workload: the "
@@ -312,10 +312,11 @@ def run_sfnn(args, dist):
     props = torch.cuda.get_device_properties(dev)
     l2 = props.L2_cache_size
     per_token = W.touched_bytes(cfg, expected_tokens_active(cfg))
-    if args.rows == "int8":  # rows of one byte per weight and a scale per row
-        per_token -= expected_tokens_active(cfg) * cfg.nproj * (cfg.d * (e - 1) - 4)
+    rows = None if args.rows == "native" else args.rows
+    if rows:  # rows of one byte (int8) or half a byte (int4) per weight and a scale per row
+        qbytes = 1.0 if rows == "int8" else 0.5
+        per_token -= expected_tokens_active(cfg) * cfg.nproj * (cfg.d * (e - qbytes) - 4)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_token))
-    rows = "int8" if args.rows == "int8" else None
     handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for _ in range(R)]
     info = handles[0].info()
     torch.cuda.synchronize()
@@ -433,7 +434,7 @@ def run_sfnn(args, dist):
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": cfg.description + (", int8 rows (per-row fp32 scales)" if rows else ""),
+        "config": {"workload": cfg.description + (f", {rows} rows (per-row fp32 scales)" if rows else ""),
                    "batch": 1, "tokens_per_step": T,
                    "replicas": R, "l2": f"inputs larger than L2: {R} weight replicas rotated per token, "
                                         f"{bytes_step / T / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
@@ -614,7 +615,7 @@ def run_stack(args, dist):
     T, NL = cfg.tokens, cfg.layers
     layers = W.make_stack(cfg, seed=args.seed)
     Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank).astype(np.float32)
-    rows = "int8" if args.rows == "int8" else None
+    rows = None if args.rows == "native" else args.rows
     handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for lay in layers]
     la = bool(args.lookahead)
     info = handles[0].info()
@@ -624,7 +625,7 @@ def run_stack(args, dist):
     X = torch.from_numpy(Xh).to(dev)
     Y = torch.empty_like(X)
     active = np.zeros(NL)
-    # per-layer set sizes (the same decisions as the fused path), for the byte count; int8
+    # per-layer set sizes (the same decisions as the fused path), for the byte count; quantized
     # rows run the fused path only, so their sets come from fp16 handles of the same layers
     count_handles = handles if rows is None else [sf.SparseFFN.from_layer(lay, device=dev) for lay in layers]
     for t in range(T):

@@ -78,7 +78,7 @@ typedef enum {
 } sfnn_status;
 
 typedef enum { SFNN_RELU = 0, SFNN_REGLU = 1 } sfnn_act;
-typedef enum { SFNN_F32 = 0, SFNN_F16 = 1, SFNN_I8 = 2 } sfnn_dtype;
+typedef enum { SFNN_F32 = 0, SFNN_F16 = 1, SFNN_I8 = 2, SFNN_I4 = 3 } sfnn_dtype;
 
 /*
  * Which kernels the batched path (b > 1, and explicit sets) uses.  The tensor-core
@@ -123,15 +123,18 @@ typedef struct {
     const float *hotness;
     /*
      * Storage of the FFN rows (w_up, w_gate, w_down), given in wdtype as usual:
-     * SFNN_I8 stores them as int8 codes with one fp32 scale per neuron and projection
-     * (weight-only quantization; the predictor, b, x and all arithmetic keep their
-     * types).  The rule, in IEEE fp32: scale = max|w| / 127 over the neuron's row (its
-     * column of w_down), code = w / scale rounded to nearest even, clamped to +-127; an
-     * all-zero row has scale 0.  Needs wdtype = SFNN_F16; such a layer runs the fused
-     * single-token path only (sfnn_forward without explicit sets, sfnn_forward_stack
-     * with b = 1) and sfnn_predict; other calls return SFNN_ERR_UNSUPPORTED.  Any other
-     * value (0 included) stores the rows in wdtype.  No counterpart on the pages beyond
-     * their weight-quantized deployments.
+     * SFNN_I8 / SFNN_I4 store them as int8 / int4 codes with one fp32 scale per neuron
+     * and projection (weight-only quantization; the predictor, b, x and all arithmetic
+     * keep their types).  The rule, in IEEE fp32, with qmax = 127 (int8) or 7 (int4):
+     * scale = max|w| / qmax over the neuron's row (its column of w_down), code = w / scale
+     * rounded to nearest even, clamped to +-qmax; an all-zero row has scale 0.  int4
+     * codes are packed two per byte, element 2k in the low nibble of byte k.  Needs
+     * wdtype = SFNN_F16 and d a multiple of 16 (int8) or 32 (int4); such a layer runs
+     * the fused single-token path only (sfnn_forward without explicit sets,
+     * sfnn_forward_stack[_lookahead] with b = 1) and sfnn_predict; other calls return
+     * SFNN_ERR_UNSUPPORTED.  Any other value (0 included) stores the rows in wdtype.
+     * The pages deploy weight-quantized models (PowerInfer in INT4 on the smaller PC,
+     * 53ai.com "sparsity for LLM inference" page, evaluation) without fixing a scheme.
      */
     int32_t rows_dtype;
 } sfnn_layer_desc;

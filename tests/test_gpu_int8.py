@@ -1,11 +1,13 @@
-"""Weight-only int8 rows (the FFN's up, gate and down rows as int8 codes with one fp32
-scale per neuron and projection; the predictor, biases, x and all arithmetic unchanged).
+"""Weight-only int8 and int4 rows (the FFN's up, gate and down rows as codes with one
+fp32 scale per neuron and projection; the predictor, biases, x and all arithmetic
+unchanged).
 
-* the library's quantization follows the oracle's rule (fp32 scale = absmax / 127,
-  codes rounded to nearest even): every token agrees with the oracle's int8 step (sets
-  exact outside the arbitration band, y within the tolerance) for ReLU and ReGLU, d up
-  to 8192, ragged n, and the full OPT-6.7B- and 70B-shaped layers;
-* results are bitwise reproducible; the rows cost half the bytes of fp16 rows;
+* the library's quantization follows the oracle's rule (fp32 scale = absmax / qmax,
+  qmax 127 or 7, codes rounded to nearest even): every token agrees with the oracle's
+  quantized step (sets exact outside the arbitration band, y within the tolerance) for
+  ReLU and ReGLU, d up to 8192, ragged n, and the full OPT-6.7B- and 70B-shaped layers;
+* results are bitwise reproducible; the rows cost a half (int8) or a quarter (int4) of
+  the bytes of fp16 rows;
 * only the fused single-token path serves such a layer: batches, explicit sets and
   the multi-kernel path are refused with SFNN_ERR_UNSUPPORTED, the predictor works.
 """
@@ -29,8 +31,11 @@ def check_token_q(lay, qr, x, y_gpu, mask_gpu, what=""):
     assert ok, f"{what}: max|dy|/max|y_ref| = {ratio:.3e} > {REL_TOL}"
 
 
-def run_tokens(cfg, lay, h, count, seed):
-    qr = oracle.quantize_layer(lay)
+BITS = {"int8": 8, "int4": 4}
+
+
+def run_tokens(cfg, lay, h, count, seed, rows):
+    qr = oracle.quantize_layer(lay, bits=BITS[rows])
     X = W.make_tokens(cfg, count, seed=seed)
     for t in range(count):
         xd = dev(X[t])
@@ -41,35 +46,39 @@ def run_tokens(cfg, lay, h, count, seed):
         assert np.array_equal(h.forward(xd).cpu().numpy(), y)
 
 
+@pytest.mark.parametrize("rows", ["int8", "int4"])
 @pytest.mark.parametrize("base,d,n,r", [
     ("opt6.7b_relu", 1024, 3001, 128),
     ("70b_reglu", 2048, 5003, 256),
     ("opt30b_relu", 7168, 4099, 1024),
     ("70b_reglu", 8192, 1500, 1024),
 ])
-def test_int8_rows_match_oracle(base, d, n, r):
+def test_quantized_rows_match_oracle(base, d, n, r, rows):
     cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
     lay = W.make_layer(cfg, seed=51)
-    h = sf.SparseFFN.from_layer(lay, rows="int8")
-    run_tokens(cfg, lay, h, 4, seed=52)
+    h = sf.SparseFFN.from_layer(lay, rows=rows)
+    run_tokens(cfg, lay, h, 4, seed=52, rows=rows)
     assert h.get_error() == 0
 
 
+@pytest.mark.parametrize("rows", ["int8", "int4"])
 @pytest.mark.parametrize("name", ["opt6.7b_relu", "70b_reglu"])
-def test_int8_rows_full_size(name):
+def test_quantized_rows_full_size(name, rows):
     cfg = W.CONFIGS[name]
     lay = W.make_layer(cfg, seed=0)
-    h = sf.SparseFFN.from_layer(lay, rows="int8")
-    run_tokens(cfg, lay, h, 2, seed=53)
+    h = sf.SparseFFN.from_layer(lay, rows=rows)
+    run_tokens(cfg, lay, h, 2, seed=53, rows=rows)
     h16 = sf.SparseFFN.from_layer(lay)
-    i8, i16 = h.info(), h16.info()
-    assert i8["row_bytes_per_neuron"] < 0.51 * i16["row_bytes_per_neuron"]
+    iq, i16 = h.info(), h16.info()
+    share = 0.51 if rows == "int8" else 0.26
+    assert iq["row_bytes_per_neuron"] < share * i16["row_bytes_per_neuron"]
 
 
-def test_int8_rows_refuse_other_paths():
+@pytest.mark.parametrize("rows", ["int8", "int4"])
+def test_quantized_rows_refuse_other_paths(rows):
     cfg = W.small_config(W.CONFIGS["opt6.7b_relu"], d=1024, n=3001, r=128)
     lay = W.make_layer(cfg, seed=54)
-    h = sf.SparseFFN.from_layer(lay, rows="int8", max_batch=4)
+    h = sf.SparseFFN.from_layer(lay, rows=rows, max_batch=4)
     X = W.make_tokens(cfg, 2, seed=55)
     with pytest.raises(sf.SfnnError) as e:
         h.forward_batch(dev(X))
