@@ -6,6 +6,7 @@
   full LLaMA-7B-shaped 4-layer ReGLU stack;
 * the sets really are predicted one layer early: they differ from the plain stack's;
 * one layer (nothing to look ahead of) gives the plain stack's result;
+* batches of tokens through the multi-kernel path, on tensor and CUDA cores;
 * a stack of one handle used for every layer, int8 rows, sets that are empty
   (y = 0, so XL = X0 exactly), and a grid barrier that times out (reported, then the
   stack recovers and reproduces its result).
@@ -63,6 +64,29 @@ def test_lookahead_stack_matches_oracle(base):
     plain = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), cfg.n) for l in range(4)]
     assert np.array_equal(masks[0], plain[0])  # layer 0 predicts from its own input either way
     assert any(not np.array_equal(masks[l], plain[l]) for l in range(1, 4))
+
+
+@pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
+def test_lookahead_batch_of_tokens(path):
+    # b > 1 runs the multi-kernel path (tensor cores for the rows under AUTO at d = 1024,
+    # or CUDA cores); every token is its own look-ahead stack
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
+    layers = [W.make_layer(cfg, seed=64, layer=l) for l in range(3)]
+    hs = [sf.SparseFFN.from_layer(l, max_batch=4) for l in layers]
+    for h in hs:
+        h.set_batch_path(sf.BATCH_TENSOR_CORE if path == "tensor_core" else sf.BATCH_CUDA_CORE)
+    X0 = W.make_tokens(cfg, 3, seed=65).astype(np.float32)
+    XL, sidx, scnt = sf.forward_stack(hs, torch.from_numpy(X0).cuda(), return_sets=True, lookahead=True)
+    XL = XL.cpu().numpy()
+    for t in range(3):
+        masks = [mask_from_idx(sidx[l, t].cpu().numpy(), scnt[l, t].item(), cfg.n) for l in range(3)]
+        xref, recs = oracle.forward_stack_lookahead(layers, X0[t].astype(np.float64), masks_other=masks,
+                                                    nthreads=NTHREADS)
+        assert all(r["mismatches"].size == 0 for r in recs)
+        base = X0[t].astype(np.float64)
+        ok, ratio = oracle.within_tolerance(XL[t].astype(np.float64) - base, xref - base)
+        assert ok, f"token {t}: {ratio:.3e}"
+    assert all(h.get_error() == 0 for h in hs)
 
 
 def test_lookahead_full_size_llama7b_reglu_stack():
