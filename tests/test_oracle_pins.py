@@ -169,6 +169,20 @@ def test_lookahead_special_cases_equal_the_stack(act):
     assert np.any(a != x0)  # the last layer does add something
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+def test_lookahead_with_quantized_rows_is_the_quantized_step(bits):
+    """One layer of the look-ahead stack on quantized rows is the single quantized step:
+    x_1 = x_0 + y of forward_q on round(x_0)."""
+    rng = np.random.default_rng(33)
+    lay = _rand_layer(rng, 32, 48, 8, "reglu", np.float16)
+    qr = oracle.quantize_layer(lay, bits=bits)
+    x0 = rng.standard_normal(32)
+    xl, recs = oracle.forward_stack_lookahead([lay], x0, qrows=[qr])
+    step = oracle.forward_q(lay, qr, x0.astype(np.float16))
+    assert np.array_equal(recs[0]["mask"], step.mask)
+    assert np.array_equal(xl, x0 + step.y)
+
+
 # ------------------------------------------------------------------ dense identity
 def _rand_layer(rng, d, n, r, act, dtype):
     s = 1.0 / np.sqrt(d)
