@@ -21,11 +21,12 @@ import torch
 
 __all__ = ["SparseFFN", "SfnnError", "forward_stack", "predict_noalloc", "hotness_order", "library_path",
            "load_library",
-           "RELU", "REGLU", "F32", "F16", "I8", "I4", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE"]
+           "RELU", "REGLU", "F32", "F16", "I8", "I4", "BATCH_AUTO", "BATCH_CUDA_CORE", "BATCH_TENSOR_CORE",
+           "BATCH_FUSED"]
 
 RELU, REGLU = 0, 1
 F32, F16, I8, I4 = 0, 1, 2, 3
-BATCH_AUTO, BATCH_CUDA_CORE, BATCH_TENSOR_CORE = 0, 1, 2
+BATCH_AUTO, BATCH_CUDA_CORE, BATCH_TENSOR_CORE, BATCH_FUSED = 0, 1, 2, 3
 STATUS = {0: "SFNN_OK", 1: "SFNN_ERR_INVALID_ARG", 2: "SFNN_ERR_CUDA", 3: "SFNN_ERR_OOM",
           4: "SFNN_ERR_UNSUPPORTED", 5: "SFNN_ERR_TIMEOUT"}
 STATUS_CODES = {v: k for k, v in STATUS.items()}
@@ -83,6 +84,7 @@ def load_library():
         "sfnn_forward_stack_lookahead": ([P, I, P, I, P, P, P, P], S),
         "sfnn_set_batch_path": ([P, I], S),
         "sfnn_set_fused_decode": ([P, I], S),
+        "sfnn_set_hot_prefix": ([P, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
         "sfnn_query": ([P, ctypes.POINTER(Info)], S),
@@ -253,6 +255,10 @@ class SparseFFN:
     def set_fused_decode(self, enable: bool):
         _check(self._lib.sfnn_set_fused_decode(self._h, int(bool(enable))), "sfnn_set_fused_decode")
 
+    def set_hot_prefix(self, enable: bool):
+        """Read the hot prefix densely on the fused few-token path (default on)."""
+        _check(self._lib.sfnn_set_hot_prefix(self._h, int(bool(enable))), "sfnn_set_hot_prefix")
+
     def debug_stall_next_barrier(self, stream=None):
         _check(self._lib.sfnn_debug_stall_next_barrier(self._h, _stream(stream)), "sfnn_debug_stall_next_barrier")
 
@@ -292,15 +298,27 @@ def predict_noalloc(x, A, B, c, idx=None, count=None, stream=None):
     returns (idx [n] int32, count [1] int32), idx[:count] ascending.
     """
     lib = load_library()
-    d, r = A.shape
-    n = B.shape[1]
     for t in (x, A, B, c):
         if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or not t.is_contiguous() or t.dtype != A.dtype:
             raise TypeError("x, A, B, c must be contiguous CUDA tensors of one dtype")
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A must be [d, r] and B [r, n]")
+    d, r = A.shape
+    n = B.shape[1]
+    if x.numel() != d or B.shape[0] != r or c.numel() != n:
+        raise ValueError(f"inconsistent shapes: x {tuple(x.shape)}, A {tuple(A.shape)}, B {tuple(B.shape)}, "
+                         f"c {tuple(c.shape)}")
     idx = idx if idx is not None else torch.empty(n, dtype=torch.int32, device=A.device)
     count = count if count is not None else torch.empty(1, dtype=torch.int32, device=A.device)
-    _check(lib.sfnn_predict_noalloc(_ptr(x), _ptr(A), _ptr(B), _ptr(c), d, r, n, _dtype_code(A.dtype), _ptr(idx),
-                                    _ptr(count), _stream(stream)), "sfnn_predict_noalloc")
+    for name, t, need in (("idx", idx, n), ("count", count, 1)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != torch.int32 \
+                or not t.is_contiguous() or t.numel() < need:
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of at least {need} elements")
+    if any(t.device != A.device for t in (x, B, c, idx, count)):
+        raise ValueError("all tensors must be on one device")
+    with torch.cuda.device(A.device):  # the library runs on, and takes its scratch of, the current device
+        _check(lib.sfnn_predict_noalloc(_ptr(x), _ptr(A), _ptr(B), _ptr(c), d, r, n, _dtype_code(A.dtype),
+                                        _ptr(idx), _ptr(count), _stream(stream)), "sfnn_predict_noalloc")
     return idx, count
 
 

@@ -34,7 +34,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt, h->scnt};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -104,23 +104,48 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
                       sfnn_ctx *ahead, cudaStream_t s) {
   cudaEvent_t before = h->prof_before, after = h->prof_after;
   const bool predict = src == kSetPredict;
-  const bool fused = b == 1 && predict && !ahead && !idx_out && !cnt_out && h->fused_ok && h->fused_on;
+  const bool fused = b == 1 && predict && !ahead && h->fused_ok && h->fused_on;
   if (h->L.rows_q && !fused) return SFNN_ERR_UNSUPPORTED;  // quantized rows: the fused path only
   h->prof_before = h->prof_after = nullptr;
   record_if(before, s);
   if (fused) {
+    const bool sets = idx_out || cnt_out;  // the kernel reports the set it used
     Decode1Params P = h->d1;
     P.x = X;
     P.y = Y;
     P.resid = resid;
     P.xnext = xnext;
+    P.set_pos = sets ? h->ulist : nullptr;
+    P.set_cnt = sets ? h->scnt : nullptr;
     SFNN_TRY(launch_decode1(P, s, true));
     record_if(after, s);
-    h->launches += 1;
+    if (sets) SFNN_TRY(launch_tile_sets(h->ulist, 1, h->scnt, h->perm, h->L.n, P.G, idx_out, cnt_out, s));
+    h->launches += sets ? 2 : 1;
+    return SFNN_OK;
+  }
+  // a few tokens: the multi-token fused kernel on CUDA cores (AUTO and FUSED), when it fits
+  const bool multi = b >= 2 && b <= h->multi_max && predict && !ahead && h->fused_on &&
+                     (h->batch_path == SFNN_BATCH_AUTO || h->batch_path == SFNN_BATCH_FUSED);
+  if (multi) {
+    const bool sets = idx_out || cnt_out;
+    Decode1Params P = h->d1;
+    P.x = X;
+    P.y = Y;
+    P.resid = resid;
+    P.xnext = xnext;
+    P.set_pos = sets ? reinterpret_cast<int32_t *>(h->acoef) : nullptr;
+    P.set_cnt = sets ? h->scnt : nullptr;
+    P.hot = h->hot_on ? h->hot_rows[b] : 0;
+    SFNN_TRY(launch_decode_multi(P, b, s, true));
+    record_if(after, s);
+    if (sets)
+      SFNN_TRY(launch_tile_sets(P.set_pos, 1, h->scnt, h->perm, h->L.n, P.G, idx_out, cnt_out, s, b));
+    h->launches += sets ? 2 : 1;
     return SFNN_OK;
   }
   const bool tc = tc_batch_supported(h) && (h->batch_path == SFNN_BATCH_TENSOR_CORE ||
-                                            (h->batch_path == SFNN_BATCH_AUTO && b >= 2));
+                                            ((h->batch_path == SFNN_BATCH_AUTO || h->batch_path == SFNN_BATCH_FUSED) &&
+                                             b >= 2));
   if (predict && tc && tc_predict_supported(h)) {
     SFNN_TRY(launch_tc_predict(h, X, b, s));
     h->launches += 1;  // three kernels instead of two
@@ -180,6 +205,15 @@ void plan_decode1(sfnn_ctx *h, int G) {
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
   h->fused_on = true;
+  // the multi-token kernel: the largest batch (up to 4) whose plan fits, with its prefix
+  for (int nb = std::min(h->max_batch, kMultiMaxTokens); nb >= 2; --nb) {
+    Decode1Params Q = P;
+    Q.hot = h->hot_rows[nb];
+    if (decode_multi_blocks_per_sm(Q, nb) >= 1) {
+      h->multi_max = nb;
+      break;
+    }
+  }
 }
 
 // Arguments shared by the two stack calls.
@@ -300,6 +334,21 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   for (int k = 0; k < L.n; ++k) perm[decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
   for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
   for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
+  // The multi-token kernel's hot prefix for b tokens: the hottest ranks whose neuron is in
+  // a b-token union with probability 1 - (1 - p)^b >= 0.99 (at most 64 rows per tile).
+  h->hot_on = true;
+  for (int b = 0; b <= kMultiMaxTokens; ++b) {
+    h->hot_rows[b] = 0;
+    if (!desc->hotness || b < 2) continue;
+    int k = 0;
+    while (k < L.n && k < 64 * G) {
+      const float q = desc->hotness[by_rank[k]];
+      const double p = std::isnan(q) ? 0.0 : std::min(1.0, std::max(0.0, (double)q));
+      if (1.0 - std::pow(1.0 - p, b) < 0.99) break;
+      ++k;
+    }
+    h->hot_rows[b] = k;
+  }
   if (desc->hotness) {
     for (int b = 1; b <= kMaxBatch; ++b) {
       double u = 0.0;
@@ -331,12 +380,15 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->utok, n * 4, false},
       {(void **)&h->ucount, 4, false},
       {(void **)&h->acoef, n * mb * 4, false},
-      {(void **)&h->part, (size_t)std::max<size_t>((size_t)kMaxSplits * mb, (size_t)G) * d * 4, false},
+      {(void **)&h->part,
+       (size_t)std::max<size_t>((size_t)kMaxSplits * mb, (size_t)G * std::min<size_t>(mb, kMultiMaxTokens)) * d * 4,
+       false},
       {&h->xin, mb * d * e, false},
       {(void **)&h->err, 4, false},
       {(void **)&h->bar, sizeof(uint64_t), false},
       {(void **)&h->alist, n * sizeof(int2), false},
       {(void **)&h->acnt, (size_t)G * 4, false},
+      {(void **)&h->scnt, (size_t)G * 4 * mb, false},
       {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
       {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
   };
@@ -360,6 +412,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();
   if (ce == cudaSuccess) ce = configure_decode_ahead();
+  if (ce == cudaSuccess) ce = configure_decode_multi();
   if (ce == cudaSuccess && h->hact) ce = configure_tc_batch();
   if (ce == cudaSuccess) plan_decode1(h, G);
   if (ce == cudaSuccess) ce = launch_layout(h, desc, s);
@@ -441,7 +494,12 @@ sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   SFNN_TRY(launch_round(X0, l0->xin, l0->L.dt, (int64_t)b * l0->L.d, s));
   l0->launches += 1;
-  if (b == 1 && !idx && !counts && ahead_fused_ok(layers, num_layers)) {
+  // With sets requested, a layer's lists must survive its launch until they are gathered:
+  // the next launch writes the next layer's lists, which are the same memory when one
+  // handle serves two consecutive layers.
+  bool lists_kept = true;
+  for (int l = 0; l + 1 < num_layers; ++l) lists_kept = lists_kept && layers[l] != layers[l + 1];
+  if (b == 1 && (lists_kept || (!idx && !counts)) && ahead_fused_ok(layers, num_layers)) {
     // launch 0: layer 0's predictor on u_0; launch l + 1: layer l's rows and layer l+1's predictor
     for (int l = -1; l < num_layers; ++l) {
       sfnn_ctx *cur = l >= 0 ? layers[l] : l0;
@@ -456,6 +514,12 @@ sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_
       Q.cnt_in = l >= 0 ? cur->acnt : nullptr;
       SFNN_TRY(launch_decode_ahead(P, Q, s, true));
       cur->launches += 1;
+      if (l >= 0 && (idx || counts)) {  // layer l's set: the lists this launch consumed
+        SFNN_TRY(launch_tile_sets(reinterpret_cast<const int32_t *>(cur->alist), 2, cur->acnt, cur->perm, cur->L.n,
+                                  cur->d1.G, idx ? idx + (size_t)l * cur->L.n : nullptr, counts ? counts + l : nullptr,
+                                  s));
+        cur->launches += 1;
+      }
     }
     return SFNN_OK;
   }
@@ -479,10 +543,18 @@ sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_
 
 sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
   if (!h) return SFNN_ERR_INVALID_ARG;
-  if (path != SFNN_BATCH_AUTO && path != SFNN_BATCH_CUDA_CORE && path != SFNN_BATCH_TENSOR_CORE)
+  if (path != SFNN_BATCH_AUTO && path != SFNN_BATCH_CUDA_CORE && path != SFNN_BATCH_TENSOR_CORE &&
+      path != SFNN_BATCH_FUSED)
     return SFNN_ERR_INVALID_ARG;
   if (path == SFNN_BATCH_TENSOR_CORE && !tc_batch_supported(h)) return SFNN_ERR_UNSUPPORTED;
+  if (path == SFNN_BATCH_FUSED && h->multi_max < 2) return SFNN_ERR_UNSUPPORTED;
   h->batch_path = path;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_hot_prefix(sfnn_handle h, int32_t enable) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  h->hot_on = enable != 0;
   return SFNN_OK;
 }
 

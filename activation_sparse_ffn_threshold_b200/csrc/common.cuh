@@ -55,6 +55,11 @@ struct sfnn_ctx {
   uint64_t *bar;     // grid barrier arrival counter of the fused kernel
   int2 *alist;       // [n] look-ahead stack: this layer's predicted active lists per tile
   int32_t *acnt;     // [G]   (storage position, bias) pairs and counts, from the launch before
+  int32_t *scnt;     // [max_batch][G] per-tile counts of the sets a fused launch used (lists: ulist
+                     //   for one token, acoef's words for several)
+  int multi_max;     // largest batch the multi-token fused kernel serves (0: none)
+  int hot_rows[sfnn::kMultiMaxTokens + 1];  // its hot prefix by batch size: ranks in the union w.p. >= 0.99
+  bool hot_on;       // the hot prefix is read densely (sfnn_set_hot_prefix)
   bool fused_ok;     // the fused single-token kernel fits this layer
   bool fused_on;     // ... and is enabled (sfnn_set_fused_decode)
   sfnn::Decode1Params d1;  // its launch plan (pointers to x/y filled per call)

@@ -239,6 +239,10 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   }
   __syncthreads();
   const int cnt = *cnt_s;
+  if (P.set_pos) {  // the tile's decisions, exactly as the rows below are read
+    for (int k = tid; k < cnt; k += kT) P.set_pos[t0 + k] = act_s[k];
+    if (tid == 0) P.set_cnt[c] = cnt;
+  }
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread;
   // the first DD rows are requested right after C1's first loads and land while C1 runs

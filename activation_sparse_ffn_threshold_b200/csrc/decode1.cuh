@@ -35,6 +35,10 @@ struct Decode1Params {
   int nseg;      // 4 KB segments of one projection row (C1 work items per row and projection)
   int rq;        // rows are 8- or 4-bit codes (0: dt); rscale [n][nproj] their fp32 scales
   const float *rscale;
+  int hot;           // multi-token kernel: ranks of the hot prefix whose gate/up rows are read before
+                     //   the sets are known (0: none); rank k is position k / G of tile k % G
+  int32_t *set_pos;  // null, or [n]: tile c's active storage positions at [start(c), start(c) + cnt)
+  int32_t *set_cnt;  //   and [G] their counts -- the set this launch used, for callers that ask
 };
 
 struct Decode1Layout {
@@ -115,6 +119,69 @@ __host__ __device__ inline Decode1Layout decode_ahead_layout(const Decode1Params
   M.tile_max = P.tile_max > Q.tile_max ? P.tile_max : Q.tile_max;
   return decode1_layout(M);
 }
+
+// The multi-token fused kernel (decode_multi.cu): NB = 2..4 tokens per launch on the
+// single-token kernel's tile plan.  Its shared memory: the NB inputs, their hidden
+// layers, the tile's per-token decisions and the union's activations, and a staging
+// region for half rows of B^T (phase B, per warp) or W_down chunks (per thread).
+constexpr int kMultiMaxTokens = 4;
+constexpr int kMultiBStages = 6;  // B^T half rows staged per warp
+
+struct MultiLayout {
+  size_t x, h, bias, c, act, tok, a, zpart, dots, pdots, red2, tbits, ubits, wpref, bars, stage, total;
+};
+
+// Rows of tile c in the hot prefix of `hot` ranks (ranks are dealt round-robin to G tiles).
+__host__ __device__ inline int decode1_hot_rows(int hot, int c, int G) { return hot > c ? (hot - c + G - 1) / G : 0; }
+
+__host__ __device__ inline MultiLayout decode_multi_layout(const Decode1Params &P, int nb) {
+  const size_t tm = (size_t)P.tile_max;
+  const size_t words = (tm + 31) / 32;
+  const int vec = 8;  // fp16 only
+  MultiLayout L;
+  size_t o = 0;
+  L.x = o;
+  o = decode1_align(o + (size_t)nb * P.d * 2, 16);
+  L.h = o;
+  o = decode1_align(o + (size_t)nb * P.r * 4, 16);
+  L.bias = o;
+  o = decode1_align(o + tm * 4, 16);
+  L.c = o;
+  o = decode1_align(o + tm * 4, 16);
+  L.act = o;  // the tile's union positions, ascending
+  o = decode1_align(o + tm * 4, 16);
+  L.tok = o;  // and the tokens active on each (bit t)
+  o = decode1_align(o + tm * 4, 16);
+  L.a = o;  // the tile's b, then the union rows' activations [k][t]
+  o = decode1_align(o + tm * nb * 4, 16);
+  L.zpart = o;  // the two halves of each logit [half][p][t]
+  o = decode1_align(o + 2 * tm * nb * 4, 16);
+  L.dots = o;  // C1 segment sums [k][proj][seg][t]
+  o = decode1_align(o + tm * 2 * (size_t)P.nseg * nb * 4, 16);
+  L.pdots = o;  // the same for the tile's hot prefix, by tile position
+  o = decode1_align(o + (size_t)decode1_hot_rows(P.hot, 0, P.G) * 2 * (size_t)P.nseg * nb * 4, 16);
+  L.red2 = o;
+  o = decode1_align(o + (size_t)kDecode1Threads * 4, 16);
+  L.tbits = o;  // [t][word]
+  o = decode1_align(o + (size_t)nb * words * 4 + 16, 16);
+  L.ubits = o;
+  o = decode1_align(o + words * 4 + 16, 16);
+  L.wpref = o;
+  o = decode1_align(o + (words + 1) * 4, 16);
+  L.bars = o;  // the union count, a flag, the split barrier's target
+  o = decode1_align(o + 16, 16);
+  L.stage = o;
+  const int maxm = decode1_maxm(P.d / vec);
+  const size_t bsz = (size_t)(kDecode1Threads / 32) * kMultiBStages * 64 * 16;  // 2 chunks per lane and stage
+  const size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
+  o = decode1_align(o + (bsz > dsz ? bsz : dsz), 16);
+  L.total = o;
+  return L;
+}
+
+cudaError_t configure_decode_multi();
+cudaError_t launch_decode_multi(const Decode1Params &P, int nb, cudaStream_t stream, bool pdl);
+int decode_multi_blocks_per_sm(const Decode1Params &P, int nb);
 
 cudaError_t configure_decode1();
 cudaError_t configure_decode_ahead();

@@ -97,5 +97,34 @@ __device__ __forceinline__ bool cta_grid_sync(const Decode1Params &P, int *flag)
   return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
+// The same barrier in two halves, so that a CTA can work between them: every thread
+// calls cta_grid_arrive after the CTA's writes that other CTAs read (thread 0 draws the
+// ticket), and cta_grid_wait before reading theirs; `slot` keeps the target in shared
+// memory.  cta_grid_wait returns false (and the error is latched) if it timed out.
+__device__ __forceinline__ void cta_grid_arrive(const Decode1Params &P, unsigned long long *slot) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t ticket = atom_add_release_gpu_u64(P.bar, 1ull);
+    *slot = (ticket / (uint32_t)P.G + 1) * (uint32_t)P.G;
+  }
+}
+__device__ __forceinline__ bool cta_grid_wait(const Decode1Params &P, const unsigned long long *slot, int *flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t target = *slot;
+    const uint64_t t0 = clock64();
+    bool ok = true;
+    while (ld_acquire_gpu_u64(P.bar) < target)
+      if ((uint64_t)(clock64() - t0) > kWaitCycles) {
+        ok = false;
+        break;
+      }
+    if (!ok) latch_error(P.err, kErrTimeout);
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int *>(flag) != 0;
+}
+
 }  // namespace
 }  // namespace sfnn

@@ -22,6 +22,13 @@ cudaError_t launch_up(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
 cudaError_t launch_down(const sfnn_ctx *h, int b, int *splits, cudaStream_t s);
 cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *resid, float *Y, void *xnext,
                           cudaStream_t s);
+// The per-tile lists of a fused launch -> one index list in caller numbering (tile order)
+// and its length, for each of `ntok` tokens.  Token t's tile c holds cnt[t * G + c]
+// storage positions, every `stride`-th int32 of `list` from position t * n + start(c)
+// on (stride 1: plain positions; 2: the look-ahead kernel's (position, bias) pairs).
+// Token t's list goes to idx_out + t * n, its length to cnt_out[t]; either may be null.
+cudaError_t launch_tile_sets(const int32_t *list, int stride, const int32_t *cnt, const int32_t *perm, int n, int G,
+                             int32_t *idx_out, int32_t *cnt_out, cudaStream_t s, int ntok = 1);
 cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s);
 
 // Tensor-core (tcgen05) batch path: fp16 weights, d a multiple of 128.

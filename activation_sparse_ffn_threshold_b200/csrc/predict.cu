@@ -304,6 +304,35 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ m
   if (threadIdx.x == 0 && cnt_out) cnt_out[t] = total;
 }
 
+// Block c: tile c's part of a fused launch's set.  Its entries follow those of tiles
+// 0..c-1 (counts clamped to each tile's size), so the list is in storage order.
+__global__ void __launch_bounds__(256) k_tile_sets(const int32_t *__restrict__ list, int stride,
+                                                   const int32_t *__restrict__ cnt, const int32_t *__restrict__ perm,
+                                                   int n, int G, int32_t *__restrict__ idx_out,
+                                                   int32_t *__restrict__ cnt_out) {
+  const int c = blockIdx.x, tok = blockIdx.y;
+  list += (size_t)tok * n * stride;
+  cnt += (size_t)tok * G;
+  if (idx_out) idx_out += (size_t)tok * n;
+  if (cnt_out) cnt_out += tok;
+  auto tile_count = [&](int t) {
+    const int sz = decode1_tile_start(t + 1, n, G) - decode1_tile_start(t, n, G);
+    return min(max(cnt[t], 0), sz);
+  };
+  int before = 0;
+  for (int t = threadIdx.x; t < c; t += blockDim.x) before += tile_count(t);
+  int total;
+  block_exclusive_scan(before, &total);  // total = the entries of tiles 0..c-1
+  const int own = tile_count(c);
+  const int start = decode1_tile_start(c, n, G);
+  if (idx_out)
+    for (int k = threadIdx.x; k < own; k += blockDim.x) {
+      const int pos = list[(size_t)(start + k) * stride];
+      idx_out[total + k] = (unsigned)pos < (unsigned)n ? perm[pos] : -1;
+    }
+  if (cnt_out && c == G - 1 && threadIdx.x == 0) *cnt_out = total + own;
+}
+
 template <typename T>
 cudaError_t hidden_impl(const sfnn_ctx *h, const void *X, int b, cudaStream_t s) {
   const Layout &L = h->L;
@@ -379,6 +408,13 @@ cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *i
     e = cudaGetLastError();
   }
   return e;
+}
+
+cudaError_t launch_tile_sets(const int32_t *list, int stride, const int32_t *cnt, const int32_t *perm, int n, int G,
+                             int32_t *idx_out, int32_t *cnt_out, cudaStream_t s, int ntok) {
+  if (!idx_out && !cnt_out) return cudaSuccess;
+  k_tile_sets<<<dim3(G, ntok), 256, 0, s>>>(list, stride, cnt, perm, n, G, idx_out, cnt_out);
+  return cudaGetLastError();
 }
 
 }  // namespace sfnn

@@ -1,15 +1,22 @@
 #!/usr/bin/env python
 """Benchmark: activation-sparse FFN decode, tokens/s per layer on B200.
 
-One step is one pass of the workload's decode sequence (512 tokens of the
-OPT-6.7B-shaped ReLU layer, d=4096 n=16384 r=1024, fp16) through the hot path:
-predictor, threshold and compaction, gathered up projection, gathered down
-projection and the final sum, one token at a time (batch 1).  The 512 tokens
-are captured once into a CUDA graph; a step is one replay.  Consecutive tokens
-use different replicas of the layer's weights so that no token finds the
-previous visit's lines in L2 (the bytes touched between two visits of one
-replica exceed twice the L2 size), as in a model where the other layers stream
-through between two visits of a layer.
+The headline step is one pass of the workload's decode sequence through the hot path
+at batch 1: predictor, threshold and compaction, gathered up/gate projection,
+gathered down projection and the final sum, one token at a time.  The default
+workload is the largest single-GPU one, the 70B-shaped ReGLU layer (d=8192
+n=28672 r=1024, fp16, 43% of the neurons carry 80% of the activations; 128
+tokens per step).  The tokens are captured once into a CUDA graph; a step is one
+replay.  Consecutive tokens use different replicas of the layer's weights so that
+no token finds the previous visit's lines in L2 (the bytes touched between two
+visits of one replica exceed twice the L2 size), as in a model where the other
+layers stream through between two visits of a layer.
+
+The same run then measures every other workload the same way (``per_config`` in
+the JSON line): the tiny fp32 and OPT-6.7B-shaped layers at batch 1, the 4-layer
+LLaMA-7B-shaped residual stack (own-layer and one-layer-ahead predictor), the
+OPT-30B-shaped layer at batch 1, 2, 4, 8 and the 70B-shaped layer at batch
+2 ... 32 (16 batches per step over rotating replicas).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sfnn|reference]
 
@@ -38,9 +45,8 @@ import numpy as np  # noqa: E402
 
 import workload as W  # noqa: E402
 
-WORKLOAD = "opt6.7b_relu"
+WORKLOAD = "70b_reglu"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "k_decode1_opt6.7b_relu.md")
 CSRC = os.path.join(ROOT, "activation_sparse_ffn_threshold_b200", "csrc")
 
 
@@ -59,6 +65,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--rows", choices=["native", "int8", "int4"], default="native",
                     help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 / int4 "
@@ -209,10 +216,11 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
+def profiled_traffic(workload: str):
+    """DRAM bytes per k_decode1 launch from the committed ncu summary of this workload,
+    if it was taken on the current sources."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(os.path.join(ROOT, "profiles", f"k_decode1_{workload}.md")).read()
     except OSError:
         return None, None
     sha = traffic = None
@@ -294,107 +302,161 @@ def run_reference(args, dist):
 
 
 # ---------------------------------------------------------------- the CUDA path
-def run_sfnn(args, dist):
+def _device(dist):
     import torch
-
-    import activation_sparse_ffn_threshold_b200 as sf
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
     dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
     torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[args.workload]
-    T = cfg.tokens
-    lay = W.make_layer(cfg, seed=args.seed)
-    Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank)
-    e = cfg.esize
+    return dev
 
-    # replicas: bytes touched between two visits of a replica >= 2 x L2
-    props = torch.cuda.get_device_properties(dev)
-    l2 = props.L2_cache_size
-    per_token = W.touched_bytes(cfg, expected_tokens_active(cfg))
-    rows = None if args.rows == "native" else args.rows
-    if rows:  # rows of one byte (int8) or half a byte (int4) per weight and a scale per row
-        qbytes = 1.0 if rows == "int8" else 0.5
-        per_token -= expected_tokens_active(cfg) * cfg.nproj * (cfg.d * (e - qbytes) - 4)
-    R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_token))
-    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for _ in range(R)]
-    info = handles[0].info()
-    torch.cuda.synchronize()
 
-    X = torch.from_numpy(Xh).to(dev)
-    Y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
-    # active-set sizes of the captured tokens (for the algorithmic byte count)
-    counts = []
-    for t in range(T):
-        _, c = handles[0].predict(X[t])
-        counts.append(c)
-    counts = torch.cat(counts).cpu().numpy().astype(np.int64)
-    bytes_tok = (info["predictor_bytes"] + counts * info["row_bytes_per_neuron"] + cfg.d * e + cfg.d * 4)
-    bytes_step = float(bytes_tok.sum())
+def _gpu_id(dev) -> str:
+    import torch
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    return uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
 
-    # event pairs around every 8th token, captured with the graph (the other tokens keep
-    # the overlap of consecutive launches)
-    s = torch.cuda.Stream(device=dev)
-    s.wait_stream(torch.cuda.current_stream())
+
+def _launches(handles) -> int:
+    return sum(h.info()["launches"] for h in handles)
+
+
+def capture(s, fn, handles):
+    """Run ``fn`` once eagerly on stream ``s``, then capture it into a CUDA graph.
+    Returns (graph, kernels one replay launches)."""
+    import torch
     with torch.cuda.stream(s):
-        for t in range(T):
-            handles[t % R].forward(X[t], Y[t])
+        fn()
     torch.cuda.synchronize()
-    launches0 = sum(h.info()["launches"] for h in handles)
+    l0 = _launches(handles)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        for t in range(T):
-            handles[t % R].forward(X[t], Y[t])
-    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
-    # one fused launch per token, nothing else: the region's time / launches is the
-    # kernel's average launch duration
-    assert launches_per_step == T, launches_per_step
+        fn()
+    return g, _launches(handles) - l0
 
-    for _ in range(args.warmup):
+
+def time_graph(g, s, steps, warmup, dist, gpu_id):
+    """Warm-up replays, then ``steps`` replays between CUDA events on ``s``, bracketed by
+    a barrier and a device synchronisation; SM clocks sampled meanwhile.  Returns
+    (this rank's ms, max over ranks of ms, clocks)."""
+    import torch
+    for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
-    gpu_uuid = str(props.uuid)
-    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id) as clk:
         dist.barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(s):
             start.record(s)
-            for _ in range(args.steps):
+            for _ in range(steps):
                 g.replay()
             stop.record(s)
         torch.cuda.synchronize()
         dist.barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    clocks = clk.summary()
+    ms = start.elapsed_time(stop)
+    return ms, dist.max(ms), clk.summary()
+
+
+def time_eager(fn, s, steps, dist):
+    """The same, for an eager loop of API calls (end to end): (max over ranks of ms)."""
+    import torch
+    with torch.cuda.stream(s):
+        fn()  # warm-up
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with torch.cuda.stream(s):
+        a.record(s)
+        for _ in range(steps):
+            fn()
+        b.record(s)
+    torch.cuda.synchronize()
+    return dist.max(a.elapsed_time(b))
+
+
+def roofline(alg_bytes, unit_us, kernel, traffic=None, traffic_source=None):
+    peak, kind = measured_peak()
+    achieved = alg_bytes / (unit_us / 1e6) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel, "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_us": unit_us,
+            "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if kind == "measured" else "fallback 6.65 TB/s",
+            "traffic_source": traffic_source}
+
+
+def _check_errors(handles):
     err = max(h.get_error() for h in handles)
     if err:
         raise SystemExit(f"device-side error latched: {err}")
 
-    t_max = dist.max(elapsed_ms)
-    tokens_total = dist.sum(args.steps * T)
-    value = tokens_total / (t_max / 1e3)
-    eff_gbs = bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9
 
-    peak, peak_kind = measured_peak()
-    launch_us = elapsed_ms * 1e3 / (args.steps * T)
-    alg_bytes = float(bytes_tok.mean())
-    achieved = alg_bytes / (launch_us / 1e6) / 1e9
-    traffic, tsrc = profiled_traffic() if rows is None else (None, None)  # the profile is of fp16 rows
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": "k_decode1 (fused single-token decode), the only kernel the timed region launches; "
-                          "average launch duration = CUDA-event time of the region / its launches",
-                "algorithmic_bytes_per_launch": alg_bytes,
-                "avg_launch_us": launch_us, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
-                if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "traffic_source": tsrc}
+def _free(*objs):
+    import gc
 
-    # end to end through the public API, eager: per step, the step's inputs from pinned
-    # host memory in one copy, one forward call per token, the step's outputs back in one
-    e2e = None
-    if not args.no_e2e:
+    import torch
+    for o in objs:
+        for h in (o if isinstance(o, (list, tuple)) else [o]):
+            if hasattr(h, "close"):
+                h.close()
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def measure_single(cfg, args, dist, dev, rows=None, headline=False):
+    """Batch-1 decode: the workload's tokens, one forward call each, over rotating weight
+    replicas, captured in one CUDA graph; one step = one replay."""
+    import torch
+
+    import activation_sparse_ffn_threshold_b200 as sf
+    T = cfg.tokens
+    lay = W.make_layer(cfg, seed=args.seed)
+    Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank)
+    e = cfg.esize
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_token = W.touched_bytes(cfg, expected_tokens_active(cfg))
+    if rows:  # rows of one byte (int8) or half a byte (int4) per weight and a scale per row
+        qbytes = 1.0 if rows == "int8" else 0.5
+        per_token -= expected_tokens_active(cfg) * cfg.nproj * (cfg.d * (e - qbytes) - 4)
+    # replicas: bytes touched between two visits of a replica >= 2 x L2 (at most one per
+    # token: a layer too small for that, the tiny fp32 one, stays L2-resident anyway)
+    R = args.replicas or min(T, max(2, 1 + math.ceil(2 * l2 / per_token)))
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for _ in range(R)]
+    info = handles[0].info()
+    torch.cuda.synchronize()
+    X = torch.from_numpy(Xh).to(dev)
+    Y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+    # the sets the fused kernel uses for the captured tokens (for the algorithmic byte count)
+    counts = np.empty(T, np.int64)
+    for t in range(T):
+        _, _, c = handles[0].forward_batch(X[t:t + 1], return_sets=True)
+        counts[t] = int(c.item())
+    bytes_tok = info["predictor_bytes"] + counts * info["row_bytes_per_neuron"] + cfg.d * e + cfg.d * 4
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        for t in range(T):
+            handles[t % R].forward(X[t], Y[t], stream=s)
+    g, launches = capture(s, step, handles)
+    # one fused launch per token, nothing else: the region's time / launches is the
+    # kernel's average launch duration
+    assert launches == T, launches
+    ms, t_max, clocks = time_graph(g, s, args.steps, args.warmup, dist, _gpu_id(dev))
+    _check_errors(handles)
+    unit_us = ms * 1e3 / (args.steps * T)
+    out = {"value": dist.sum(args.steps * T) / (t_max / 1e3), "unit": "tokens/s", "ms_per_step": t_max / args.steps,
+           "avg_us": unit_us, "avg_of": "one token (one k_decode1 launch)", "replicas": R,
+           "mean_active_neurons": float(counts.mean()), "gpu_launches": int(launches * args.steps),
+           "clocks": clocks, "bytes_per_step": float(bytes_tok.sum())}
+    traffic, tsrc = (profiled_traffic(cfg.name) if rows is None else (None, None))
+    out["roofline"] = roofline(float(bytes_tok.mean()), unit_us,
+                               "k_decode1 (fused single-token decode), the only kernel the timed region launches; "
+                               "average launch duration = CUDA-event time of the region / its launches",
+                               traffic, tsrc)
+    out["effective_gbs"] = float(bytes_tok.sum()) * args.steps / (ms / 1e3) / 1e9
+    if headline and not args.no_e2e:
+        # end to end through the public API, eager: per step, the step's inputs from pinned
+        # host memory in one copy, one forward call per token, the step's outputs back in one
         xin = torch.from_numpy(Xh).pin_memory()
         yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
         xd = torch.empty((T, cfg.d), dtype=X.dtype, device=dev)
@@ -406,285 +468,122 @@ def run_sfnn(args, dist):
             for t in range(T):
                 handles[t % R].forward(xd[t], yd[t], stream=s)
             yout.copy_(yd, non_blocking=True)
-        with torch.cuda.stream(s):
-            one_step()  # warm-up
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        dist.barrier()
-        with torch.cuda.stream(s):
-            a.record(s)
-            for _ in range(e2e_steps):
-                one_step()
-            b.record(s)
-        torch.cuda.synchronize()
-        e_max = dist.max(a.elapsed_time(b))
-        e2e = {"value": dist.sum(e2e_steps * T) / (e_max / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": T * cfg.d * e, "d2h_bytes_per_step": T * cfg.d * 4,
-               "steps": e2e_steps,
-               "timing": "CUDA events around the eager loop (per step: one host-to-device copy of the step's "
-                         "inputs, one forward call per token, one device-to-host copy of the outputs), max over ranks"}
-
-    cpu = None
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        Xc = W.make_tokens(cfg, 64, seed=args.seed + 99)
-        cpu = cpu_baseline(cfg, lay, Xc, args.cpu_seconds)
-
-    line = {
-        "metric": "sparse-FFN decode tokens/s per layer", "value": value, "unit": "tokens/s",
-        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": cfg.description + (f", {rows} rows (per-row fp32 scales)" if rows else ""),
-                   "batch": 1, "tokens_per_step": T,
-                   "replicas": R, "l2": f"inputs larger than L2: {R} weight replicas rotated per token, "
-                                        f"{bytes_step / T / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
-                   "parallelism": f"replicas x{dist.world} (no exchange)",
-                   "mean_active_neurons": float(counts.mean())},
-        "effective_gbs": eff_gbs,
-        "roofline": roofline,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": int(launches_per_step * args.steps),
-        "clocks": clocks,
-    }
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        e_max = time_eager(one_step, s, e2e_steps, dist)
+        _check_errors(handles)
+        out["e2e"] = {"value": dist.sum(e2e_steps * T) / (e_max / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": T * cfg.d * e, "d2h_bytes_per_step": T * cfg.d * 4, "steps": e2e_steps,
+                      "timing": "CUDA events around the eager loop (per step: one host-to-device copy of the step's "
+                                "inputs, one forward call per token, one device-to-host copy of the outputs), "
+                                "max over ranks"}
+    out["_lay"] = lay
     del g
-    for h in handles:
-        h.close()
-    return 0
+    _free(handles)
+    return out
 
-# ---------------------------------------------------------------- the batched path
-def run_batch(args, dist):
+
+def measure_batch(cfg, b, args, dist, dev):
     """b tokens per forward_batch call: predictor of the batch, union of its sets, the
     union's rows once for all b tokens.  A step is BATCHES_PER_STEP such calls over
     rotating weight replicas, captured in one CUDA graph."""
     import torch
 
     import activation_sparse_ffn_threshold_b200 as sf
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
-    BATCHES_PER_STEP = 16
-    dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
-    torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[args.workload]
-    b = args.batch
     lay = W.make_layer(cfg, seed=args.seed)
     Xh = W.make_tokens(cfg, BATCHES_PER_STEP * b, seed=args.seed + dist.rank, stream_key=b).reshape(
         BATCHES_PER_STEP, b, cfg.d)
     e = cfg.esize
-    props = torch.cuda.get_device_properties(dev)
-    l2 = props.L2_cache_size
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_batch = W.touched_bytes(cfg, W.expected_union_density(lay.p, b) * cfg.n, b)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
     handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b) for _ in range(R)]
     info = handles[0].info()
-    path = "tcgen05" if cfg.dtype == "f16" and cfg.d % 128 == 0 else "cuda-core"
     torch.cuda.synchronize()
-
     X = torch.from_numpy(Xh).to(dev)
     Y = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32, device=dev)
-    unions = []
+    unions = np.empty(BATCHES_PER_STEP, np.int64)
     for i in range(BATCHES_PER_STEP):  # union sizes, for the algorithmic byte count
         _, idx, cnt = handles[0].forward_batch(X[i], return_sets=True)
         m = torch.zeros(cfg.n, dtype=torch.bool, device=dev)
         for t in range(b):
             m[idx[t, :int(cnt[t])].long()] = True
-        unions.append(int(m.sum()))
-    unions = np.array(unions, dtype=np.int64)
+        unions[i] = int(m.sum())
     bytes_batch = info["predictor_bytes"] + unions * info["row_bytes_per_neuron"] + b * cfg.d * (e + 4)
-    bytes_step = float(bytes_batch.sum())
-
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
+
+    def step():
         for i in range(BATCHES_PER_STEP):
-            handles[i % R].forward_batch(X[i], Y[i])
-    torch.cuda.synchronize()
-    launches0 = sum(h.info()["launches"] for h in handles)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        for i in range(BATCHES_PER_STEP):
-            handles[i % R].forward_batch(X[i], Y[i])
-    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize()
-    gpu_uuid = str(props.uuid)
-    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_id) as clk:
-        dist.barrier()
-        torch.cuda.synchronize()
-        with torch.cuda.stream(s):
-            start.record(s)
-            for _ in range(args.steps):
-                g.replay()
-            stop.record(s)
-        torch.cuda.synchronize()
-        dist.barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    clocks = clk.summary()
-    err = max(h.get_error() for h in handles)
-    if err:
-        raise SystemExit(f"device-side error latched: {err}")
-    t_max = dist.max(elapsed_ms)
-    tokens_total = dist.sum(args.steps * BATCHES_PER_STEP * b)
-    value = tokens_total / (t_max / 1e3)
-    batch_us = elapsed_ms * 1e3 / (args.steps * BATCHES_PER_STEP)
-    achieved = float(bytes_batch.mean()) / (batch_us / 1e6) / 1e9
-    peak, peak_kind = measured_peak()
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None,
-                "kernel": f"one batch of {b} tokens ({launches_per_step // BATCHES_PER_STEP} kernels, {path} path); "
-                          "duration = CUDA-event time of the timed region / batches",
-                "algorithmic_bytes_per_launch": float(bytes_batch.mean()), "avg_launch_us": batch_us,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s", "traffic_source": None}
-
-    e2e = None
-    if not args.no_e2e:
-        xin = torch.from_numpy(Xh).pin_memory()
-        yout = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32).pin_memory()
-        xd = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=X.dtype, device=dev)
-        yd = torch.empty((BATCHES_PER_STEP, b, cfg.d), dtype=torch.float32, device=dev)
-        e2e_steps = max(1, min(args.steps, 20))
-
-        def one_step():  # the step's inputs in one copy, one call per batch, the outputs in one copy
-            xd.copy_(xin, non_blocking=True)
-            for i in range(BATCHES_PER_STEP):
-                handles[i % R].forward_batch(xd[i], yd[i], stream=s)
-            yout.copy_(yd, non_blocking=True)
-        with torch.cuda.stream(s):
-            one_step()
-        torch.cuda.synchronize()
-        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        dist.barrier()
-        with torch.cuda.stream(s):
-            a.record(s)
-            for _ in range(e2e_steps):
-                one_step()
-            c.record(s)
-        torch.cuda.synchronize()
-        e_max = dist.max(a.elapsed_time(c))
-        e2e = {"value": dist.sum(e2e_steps * BATCHES_PER_STEP * b) / (e_max / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * e,
-               "d2h_bytes_per_step": BATCHES_PER_STEP * b * cfg.d * 4,
-               "steps": e2e_steps, "timing": "CUDA events around the eager loop (per step: one host-to-device copy "
-                                            "of the step's inputs, the API calls, one device-to-host copy of the "
-                                            "outputs), max over ranks"}
-
-    line = {
-        "metric": "sparse-FFN batched decode tokens/s per layer", "value": value, "unit": "tokens/s",
-        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16" if e == 2 else "f32", "data": "synthetic",
-        "config": {"workload": cfg.description, "batch": b, "batches_per_step": BATCHES_PER_STEP,
-                   "path": path, "replicas": R,
-                   "l2": f"inputs larger than L2: {R} weight replicas rotated per batch, "
-                         f"{bytes_step / BATCHES_PER_STEP / 1e6:.1f} MB touched per batch, L2 {l2 / 1e6:.0f} MB",
-                   "parallelism": f"replicas x{dist.world} (no exchange)",
-                   "mean_union_rows": float(unions.mean())},
-        "effective_gbs": bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9,
-        "roofline": roofline,
-        "cpu_baseline": None,
-        "e2e": e2e,
-        "gpu_launches": int(launches_per_step * args.steps),
-        "clocks": clocks,
-    }
-    if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+            handles[i % R].forward_batch(X[i], Y[i], stream=s)
+    g, launches = capture(s, step, handles)
+    ms, t_max, clocks = time_graph(g, s, args.steps, args.warmup, dist, _gpu_id(dev))
+    _check_errors(handles)
+    unit_us = ms * 1e3 / (args.steps * BATCHES_PER_STEP)
+    path = batch_path_name(handles[0], b)
+    out = {"value": dist.sum(args.steps * BATCHES_PER_STEP * b) / (t_max / 1e3), "unit": "tokens/s",
+           "ms_per_step": t_max / args.steps, "avg_us": unit_us, "avg_of": f"one batch of {b} tokens",
+           "replicas": R, "path": path, "kernels_per_batch": launches // BATCHES_PER_STEP,
+           "mean_union_rows": float(unions.mean()), "gpu_launches": int(launches * args.steps), "clocks": clocks,
+           "bytes_per_step": float(bytes_batch.sum())}
+    out["roofline"] = roofline(float(bytes_batch.mean()), unit_us,
+                               f"one batch of {b} tokens ({launches // BATCHES_PER_STEP} kernels, {path}); "
+                               "duration = CUDA-event time of the timed region / batches")
+    out["effective_gbs"] = float(bytes_batch.sum()) * args.steps / (ms / 1e3) / 1e9
     del g
-    for h in handles:
-        h.close()
-    return 0
+    _free(handles)
+    return out
 
 
-# ---------------------------------------------------------------- the residual stack
-def run_stack(args, dist):
+def batch_path_name(h, b) -> str:
+    inf = h.info()
+    return {0: "auto", 1: "cuda-core", 2: "tcgen05"}.get(inf["batch_path"], "?") + \
+        (f" (auto: {'tcgen05' if inf['wdtype'] == 1 and inf['d'] % 128 == 0 and b >= 2 else 'cuda-core'})"
+         if inf["batch_path"] == 0 else "")
+
+
+def measure_stack(cfg, args, dist, dev, lookahead=False, rows=None):
     """x_{l+1} = x_l + FFN_l(x_l) through the workload's layers, one token per
     forward_stack call; a step is the workload's tokens, captured in one CUDA graph."""
     import torch
 
     import activation_sparse_ffn_threshold_b200 as sf
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
-    dev = torch.device("cuda", dist.local_rank if dist.world > 1 else 0)
-    torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[args.workload]
     T, NL = cfg.tokens, cfg.layers
     layers = W.make_stack(cfg, seed=args.seed)
     Xh = W.make_tokens(cfg, T, seed=args.seed + dist.rank).astype(np.float32)
-    rows = None if args.rows == "native" else args.rows
     handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for lay in layers]
-    la = bool(args.lookahead)
     info = handles[0].info()
     e = cfg.esize
-    props = torch.cuda.get_device_properties(dev)
-    l2 = props.L2_cache_size
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     X = torch.from_numpy(Xh).to(dev)
     Y = torch.empty_like(X)
     active = np.zeros(NL)
-    # per-layer set sizes (the same decisions as the fused path), for the byte count; quantized
-    # rows run the fused path only, so their sets come from fp16 handles of the same layers
-    count_handles = handles if rows is None else [sf.SparseFFN.from_layer(lay, device=dev) for lay in layers]
-    for t in range(T):
-        _, _, cnt = sf.forward_stack(count_handles, X[t], return_sets=True, lookahead=la)
+    for t in range(T):  # the sets the stack's own launches use, for the byte count
+        _, _, cnt = sf.forward_stack(handles, X[t], return_sets=True, lookahead=lookahead)
         active += cnt.cpu().numpy().reshape(NL)
-    if rows is not None:
-        for h in count_handles:
-            h.close()
     active /= T
     bytes_layer_tok = info["predictor_bytes"] + active * info["row_bytes_per_neuron"] + cfg.d * (e + 4)
-    bytes_step = float(bytes_layer_tok.sum()) * T
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
+
+    def step():
         for t in range(T):
-            sf.forward_stack(handles, X[t], Y[t], stream=s, lookahead=la)
-    torch.cuda.synchronize()
-    launches0 = sum(h.info()["launches"] for h in handles)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        for t in range(T):
-            sf.forward_stack(handles, X[t], Y[t], stream=s, lookahead=la)
-    launches_per_step = sum(h.info()["launches"] for h in handles) - launches0
-    for _ in range(args.warmup):
-        g.replay()
-    torch.cuda.synchronize()
-    gpu_uuid = str(props.uuid)
-    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_id) as clk:
-        dist.barrier()
-        torch.cuda.synchronize()
-        with torch.cuda.stream(s):
-            start.record(s)
-            for _ in range(args.steps):
-                g.replay()
-            stop.record(s)
-        torch.cuda.synchronize()
-        dist.barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    clocks = clk.summary()
-    err = max(h.get_error() for h in handles)
-    if err:
-        raise SystemExit(f"device-side error latched: {err}")
-    t_max = dist.max(elapsed_ms)
-    value = dist.sum(args.steps * T * NL) / (t_max / 1e3)
-    layer_us = elapsed_ms * 1e3 / (args.steps * T * NL)
-    achieved = float(bytes_layer_tok.mean()) / (layer_us / 1e6) / 1e9
-    peak, peak_kind = measured_peak()
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None,
-                "kernel": (f"k_decode_ahead (look-ahead stack), {launches_per_step // T} launches per token: the "
-                           "input rounding, layer 0's predictor, one per layer" if la else
-                           f"k_decode1, one launch per layer and token ({launches_per_step // T} launches per token "
-                           "with the input rounding)") + "; duration = CUDA-event time of the region / layer-tokens",
-                "algorithmic_bytes_per_launch": float(bytes_layer_tok.mean()), "avg_launch_us": layer_us,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s", "traffic_source": None}
-    e2e = None
+            sf.forward_stack(handles, X[t], Y[t], stream=s, lookahead=lookahead)
+    g, launches = capture(s, step, handles)
+    ms, t_max, clocks = time_graph(g, s, args.steps, args.warmup, dist, _gpu_id(dev))
+    _check_errors(handles)
+    layer_us = ms * 1e3 / (args.steps * T * NL)
+    out = {"value": dist.sum(args.steps * T * NL) / (t_max / 1e3), "unit": "layer-tokens/s",
+           "ms_per_step": t_max / args.steps, "avg_us": layer_us, "avg_of": "one layer of one token",
+           "layers": NL, "launches_per_token": launches // T, "gpu_launches": int(launches * args.steps),
+           "mean_active_neurons_per_layer": [float(v) for v in active], "clocks": clocks,
+           "bytes_per_step": float(bytes_layer_tok.sum()) * T,
+           "l2": f"inputs larger than L2: {NL} distinct layers per token, "
+                 f"{float(bytes_layer_tok.sum()) / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB"}
+    kern = (f"k_decode_ahead (look-ahead stack), {launches // T} launches per token: the input rounding, layer 0's "
+            "predictor, one per layer" if lookahead else
+            f"k_decode1, one launch per layer and token ({launches // T} launches per token with the input rounding)")
+    out["roofline"] = roofline(float(bytes_layer_tok.mean()), layer_us,
+                               kern + "; duration = CUDA-event time of the region / layer-tokens")
+    out["effective_gbs"] = float(bytes_layer_tok.sum()) * T * args.steps / (ms / 1e3) / 1e9
     if not args.no_e2e:
         xin = torch.from_numpy(Xh).pin_memory()
         yout = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
@@ -695,49 +594,154 @@ def run_stack(args, dist):
         def one_step():  # the step's inputs in one copy, one stack call per token, the outputs in one copy
             xd.copy_(xin, non_blocking=True)
             for t in range(T):
-                sf.forward_stack(handles, xd[t], yd[t], stream=s, lookahead=la)
+                sf.forward_stack(handles, xd[t], yd[t], stream=s, lookahead=lookahead)
             yout.copy_(yd, non_blocking=True)
-        with torch.cuda.stream(s):
-            one_step()
-        torch.cuda.synchronize()
-        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        dist.barrier()
-        with torch.cuda.stream(s):
-            a.record(s)
-            for _ in range(e2e_steps):
-                one_step()
-            c.record(s)
-        torch.cuda.synchronize()
-        e_max = dist.max(a.elapsed_time(c))
-        e2e = {"value": dist.sum(e2e_steps * T * NL) / (e_max / 1e3), "unit": "layer-tokens/s",
-               "h2d_bytes_per_step": T * cfg.d * 4, "d2h_bytes_per_step": T * cfg.d * 4,
-               "steps": e2e_steps, "timing": "CUDA events around the eager loop (per step: one host-to-device copy "
-                                            "of the step's inputs, the API calls, one device-to-host copy of the "
-                                            "outputs), max over ranks"}
+        e_max = time_eager(one_step, s, e2e_steps, dist)
+        out["e2e"] = {"value": dist.sum(e2e_steps * T * NL) / (e_max / 1e3), "unit": "layer-tokens/s",
+                      "h2d_bytes_per_step": T * cfg.d * 4, "d2h_bytes_per_step": T * cfg.d * 4,
+                      "steps": e2e_steps}
+    del g
+    _free(handles)
+    return out
+
+
+BATCHES_PER_STEP = 16
+
+# The other workloads, each measured the same way as the headline inside the default run:
+# (workload, what, batch)
+PER_CONFIG = [
+    ("tiny_relu_f32", "single", 1),
+    ("opt6.7b_relu", "single", 1),
+    ("llama7b_reglu_stack", "stack", 1),
+    ("llama7b_reglu_stack", "stack_lookahead", 1),
+    ("opt30b_relu", "single", 1),
+    ("opt30b_relu", "batch", 2),
+    ("opt30b_relu", "batch", 4),
+    ("opt30b_relu", "batch", 8),
+    ("70b_reglu", "batch", 2),
+    ("70b_reglu", "batch", 4),
+    ("70b_reglu", "batch", 8),
+    ("70b_reglu", "batch", 16),
+    ("70b_reglu", "batch", 32),
+]
+
+
+def _summary(cfg, what, b, m):
+    """One per_config record: the numbers a reader compares across workloads."""
+    r = m["roofline"]
+    return {"workload": cfg.description, "what": what, "batch": b, "value": m["value"], "unit": m["unit"],
+            "avg_us": m["avg_us"], "avg_of": m["avg_of"], "achieved_gbs": r["achieved"], "frac": r["frac"],
+            "algorithmic_bytes": r["algorithmic_bytes_per_launch"], "traffic": r["traffic"],
+            **({"path": m["path"], "mean_union_rows": m["mean_union_rows"], "kernels_per_batch":
+                m["kernels_per_batch"]} if "path" in m else {}),
+            **({"mean_active_neurons": m["mean_active_neurons"]} if "mean_active_neurons" in m else {}),
+            **({"mean_active_neurons_per_layer": m["mean_active_neurons_per_layer"],
+                "launches_per_token": m["launches_per_token"]} if "layers" in m else {}),
+            **({"e2e": m["e2e"]["value"]} if m.get("e2e") else {}),
+            "clocks": {"sm_mhz": m["clocks"].get("sm_mhz"), "reasons": m["clocks"].get("reasons")}}
+
+
+def run_sfnn(args, dist):
+    """The headline: batch-1 decode of the workload (default: the 70B-shaped ReGLU
+    layer, the largest single-GPU configuration), then every other configuration."""
+    dev = _device(dist)
+    cfg = W.CONFIGS[args.workload]
+    rows = None if args.rows == "native" else args.rows
+    m = measure_single(cfg, args, dist, dev, rows=rows, headline=True)
+    lay = m.pop("_lay")
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        Xc = W.make_tokens(cfg, 64, seed=args.seed + 99)
+        cpu = cpu_baseline(cfg, lay, Xc, args.cpu_seconds)
+    del lay
+    per = None
+    if not args.no_per_config:
+        per = {}
+        steps = args.steps
+        for name, what, b in PER_CONFIG:
+            if name == args.workload and what == "single":
+                continue
+            c = W.CONFIGS[name]
+            key = f"{name}:{what}:b{b}"
+            if what == "single":
+                r = measure_single(c, args, dist, dev)
+                r.pop("_lay", None)
+            elif what == "batch":
+                r = measure_batch(c, b, args, dist, dev)
+            else:
+                r = measure_stack(c, args, dist, dev, lookahead=(what == "stack_lookahead"))
+            per[key] = _summary(c, what, b, r)
+            log(f"{key}: {r['value']:.1f} {r['unit']}, {r['avg_us']:.2f} us, frac {r['roofline']['frac']:.3f}")
+        args.steps = steps
+    T = cfg.tokens
     line = {
-        "metric": f"sparse-FFN decode layer-tokens/s ({NL}-layer residual stack"
-                  f"{', sets predicted one layer ahead' if la else ''})", "value": value,
-        "unit": "layer-tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": cfg.description, "batch": 1, "layers": NL, "tokens_per_step": T,
-                   "predictor": "one layer ahead" if la else "own layer", "rows": args.rows,
-                   "l2": f"inputs larger than L2: {NL} distinct layers per token, "
-                         f"{float(bytes_layer_tok.sum()) / 1e6:.1f} MB touched per token, L2 {l2 / 1e6:.0f} MB",
+        "metric": "sparse-FFN decode tokens/s per layer", "value": m["value"], "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16" if cfg.esize == 2 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.description + (f", {rows} rows (per-row fp32 scales)" if rows else ""),
+                   "batch": 1, "tokens_per_step": T, "replicas": m["replicas"],
+                   "l2": f"inputs larger than L2: {m['replicas']} weight replicas rotated per token, "
+                         f"{m['bytes_per_step'] / T / 1e6:.1f} MB touched per token",
                    "parallelism": f"replicas x{dist.world} (no exchange)",
-                   "mean_active_neurons_per_layer": [float(v) for v in active]},
-        "effective_gbs": bytes_step * args.steps / (elapsed_ms / 1e3) / 1e9,
-        "roofline": roofline,
-        "cpu_baseline": None,
-        "e2e": e2e,
-        "gpu_launches": int(launches_per_step * args.steps),
-        "clocks": clocks,
+                   "mean_active_neurons": m["mean_active_neurons"]},
+        "effective_gbs": m["effective_gbs"],
+        "roofline": m["roofline"],
+        "cpu_baseline": cpu,
+        "e2e": m.get("e2e"),
+        "gpu_launches": m["gpu_launches"],
+        "clocks": m["clocks"],
+        "per_config": per,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
-    del g
-    for h in handles:
-        h.close()
+    return 0
+
+
+def run_batch(args, dist):
+    dev = _device(dist)
+    cfg = W.CONFIGS[args.workload]
+    b = args.batch
+    m = measure_batch(cfg, b, args, dist, dev)
+    line = {
+        "metric": "sparse-FFN batched decode tokens/s per layer", "value": m["value"], "unit": "tokens/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16" if cfg.esize == 2 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": b, "batches_per_step": BATCHES_PER_STEP,
+                   "path": m["path"], "replicas": m["replicas"],
+                   "l2": f"inputs larger than L2: {m['replicas']} weight replicas rotated per batch, "
+                         f"{m['bytes_per_step'] / BATCHES_PER_STEP / 1e6:.1f} MB touched per batch",
+                   "parallelism": f"replicas x{dist.world} (no exchange)", "mean_union_rows": m["mean_union_rows"]},
+        "effective_gbs": m["effective_gbs"], "roofline": m["roofline"], "cpu_baseline": None, "e2e": None,
+        "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_stack(args, dist):
+    dev = _device(dist)
+    cfg = W.CONFIGS[args.workload]
+    la = bool(args.lookahead)
+    rows = None if args.rows == "native" else args.rows
+    m = measure_stack(cfg, args, dist, dev, lookahead=la, rows=rows)
+    line = {
+        "metric": f"sparse-FFN decode layer-tokens/s ({cfg.layers}-layer residual stack"
+                  f"{', sets predicted one layer ahead' if la else ''})", "value": m["value"],
+        "unit": "layer-tokens/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": cfg.description, "batch": 1, "layers": cfg.layers, "tokens_per_step": cfg.tokens,
+                   "predictor": "one layer ahead" if la else "own layer", "rows": args.rows, "l2": m["l2"],
+                   "parallelism": f"replicas x{dist.world} (no exchange)",
+                   "mean_active_neurons_per_layer": m["mean_active_neurons_per_layer"]},
+        "effective_gbs": m["effective_gbs"], "roofline": m["roofline"], "cpu_baseline": None, "e2e": m.get("e2e"),
+        "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
     return 0
 
 

@@ -87,14 +87,21 @@ typedef enum { SFNN_F32 = 0, SFNN_F16 = 1, SFNN_I8 = 2, SFNN_I4 = 3 } sfnn_dtype
  * up/gate and down projections (gathered GEMMs) on tcgen05 tensor cores, with fp32
  * accumulation and the activations rounded to fp16 between the two projections; it
  * needs fp16 weights, d a multiple of 128 and max_batch >= 2 (the predictor part also
- * r a multiple of 64, else the CUDA-core predictor runs).  AUTO takes it for every
- * batch of 2 or more tokens where it is available (measured faster at every batch
- * size), and the CUDA-core path otherwise.
+ * r a multiple of 64, else the CUDA-core predictor runs).  The fused path runs a batch
+ * of 2 to 4 tokens in one launch of the multi-token kernel on CUDA cores (the
+ * single-token kernel's plan with every weight read once for all tokens: predictor
+ * rows, and the union of the tokens' active rows, each row applied only to the tokens
+ * whose sets hold it); it needs fp16 weights, d <= 16384 and r <= 1024.  AUTO takes the
+ * fused path for 2 to 4 tokens and the tensor cores for more: a union of a few tokens'
+ * sets is too thin to be a real contraction, while from 8 tokens on it is dense enough
+ * that the tensor cores' gathered GEMMs beat CUDA cores; where a path does not fit a
+ * layer, the next one serves (fused -> tensor cores -> CUDA cores).
  */
 typedef enum {
     SFNN_BATCH_AUTO = 0,
     SFNN_BATCH_CUDA_CORE = 1,   /* multi-token gather on CUDA cores */
-    SFNN_BATCH_TENSOR_CORE = 2  /* dense and gathered GEMMs on tcgen05 tensor cores */
+    SFNN_BATCH_TENSOR_CORE = 2, /* dense and gathered GEMMs on tcgen05 tensor cores */
+    SFNN_BATCH_FUSED = 3        /* 2..4 tokens: one fused launch on CUDA cores; more: as AUTO */
 } sfnn_batch_path;
 
 /*
@@ -131,8 +138,8 @@ typedef struct {
      * codes are packed two per byte, element 2k in the low nibble of byte k.  Needs
      * wdtype = SFNN_F16 and d a multiple of 16 (int8) or 32 (int4); such a layer runs
      * the fused single-token path only (sfnn_forward without explicit sets,
-     * sfnn_forward_stack[_lookahead] with b = 1) and sfnn_predict; other calls return
-     * SFNN_ERR_UNSUPPORTED.  Any other value (0 included) stores the rows in wdtype.
+     * sfnn_forward_batch and sfnn_forward_stack[_lookahead] with b = 1) and sfnn_predict;
+     * other calls return SFNN_ERR_UNSUPPORTED.  Any other value (0 included) stores the rows in wdtype.
      * The pages deploy weight-quantized models (PowerInfer in INT4 on the smaller PC,
      * 53ai.com "sparsity for LLM inference" page, evaluation) without fixing a scheme.
      */
@@ -195,7 +202,10 @@ SFNN_API sfnn_status sfnn_forward(sfnn_handle h, const void *x, const int32_t *i
  * applied to the tokens active on each row: as a batch's sets accumulate, the
  * benefit of sparsity shrinks (53ai.com page, section 工程效果), so the rows are
  * shared by every token that needs them.  The kernels follow sfnn_set_batch_path.
- * A layer with int8 rows returns SFNN_ERR_UNSUPPORTED.
+ * With b = 1 the fused single-token kernel runs (as in sfnn_forward, unless it is
+ * disabled), and idx/counts return the set that kernel itself decided and read:
+ * each tile's active positions as its rows were gathered, listed by one small
+ * kernel after it.  A layer with quantized rows returns SFNN_ERR_UNSUPPORTED for b > 1.
  *   X      [b x d] wdtype;  Y [b x d] fp32 out
  *   idx    [b x n] int32 out or NULL: token t's set in row t (first counts[t] entries)
  *   counts [b] int32 out or NULL: |S_t|
@@ -207,8 +217,9 @@ SFNN_API sfnn_status sfnn_forward_batch(sfnn_handle h, const void *X, int32_t b,
  * A stack of layers with a residual stream:  X_{l+1} = X_l + FFN_l(round(X_l)),
  * where round() converts the fp32 residual to the layers' wdtype (nearest even).
  * The pages name no normalisation between the layers; none is applied.  With
- * b = 1 every layer runs the fused single-token kernel (unless disabled); with
- * idx/counts requested or b > 1, the batched path.
+ * b = 1 every layer runs the fused single-token kernel (unless disabled), and
+ * idx/counts, when requested, return the sets those launches used; with b > 1, the
+ * batched path.
  * All layers share d, wdtype and max_batch >= b (and n when idx != NULL).
  *   layers [num_layers] HOST array of handles
  *   X0     [b x d] fp32 in;  XL [b x d] fp32 out (may alias X0)
@@ -224,11 +235,14 @@ SFNN_API sfnn_status sfnn_forward_stack(const sfnn_handle *layers, int32_t num_l
  * predictor, which forecasts the next layer's sparsity one step early (53ai.com
  * "sparsity for LLM inference" page, section "如何推理加速").  Layer 0 predicts from
  * round(X_0).  The sets, and so XL, may differ from sfnn_forward_stack's.
- * With b = 1 and no idx/counts, and every layer on the fused kernel with the same
- * number of tiles (SMs), the stack runs as num_layers + 1 launches of one look-ahead
- * kernel: launch l does layer l's rows on the set launch l-1 predicted and layer l+1's
- * predictor, with one bounded grid barrier.  Otherwise the batched path, with each
- * layer's prediction issued before the previous layer's reduce.
+ * With b = 1, and every layer on the fused kernel with the same number of tiles
+ * (SMs), the stack runs as num_layers + 1 launches of one look-ahead kernel: launch l
+ * does layer l's rows on the set launch l-1 predicted and layer l+1's predictor, with
+ * one bounded grid barrier; idx/counts, when requested, return the lists each launch
+ * consumed (listed after it by one small kernel; with sets requested, one handle
+ * serving two consecutive layers takes the batched path instead, whose lists it
+ * would otherwise overwrite).  Otherwise the batched path, with each layer's
+ * prediction issued before the previous layer's reduce.
  * Arguments, sharing rules and idx/counts layout as sfnn_forward_stack.
  */
 SFNN_API sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int32_t num_layers, const float *X0,
@@ -243,6 +257,22 @@ SFNN_API sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int
  * it on a layer it does not fit (shared memory or SM count).
  */
 SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
+
+/*
+ * The fused few-token path (SFNN_BATCH_FUSED, and AUTO for 2 to 4 tokens) reads the
+ * hot prefix of the layer densely (enabled by default): the neurons that the offline
+ * hotness profile puts in a b-token batch's union with probability >= 0.99
+ * (1 - (1 - p)^b >= 0.99, at most 64 per SM tile) have their gate/up rows read and
+ * multiplied for every token while the predictor's grid barrier completes, before the
+ * sets are known; the cold tail is gathered by the union as usual.  The rows of a
+ * prefix neuron that no token's set holds are read and dropped (the set semantics are
+ * unchanged: a row applies only to the tokens whose sets hold it, and y is bitwise the
+ * same either way).  This is the power-law split of the pages -- a few hot neurons
+ * carry most activations (hexiedandong.com PowerInfer news page, the paragraph on
+ * figure (a)) and every token of a batch needs them (53ai.com page, section 工程效果).
+ * Without a hotness profile there is no prefix.  Disabling it keeps every read sparse.
+ */
+SFNN_API sfnn_status sfnn_set_hot_prefix(sfnn_handle h, int32_t enable);
 
 /*
  * Fault injection for tests (synchronises `stream`): the next fused decode launch
@@ -280,7 +310,9 @@ SFNN_API sfnn_status sfnn_set_profile_events(sfnn_handle h, sfnn_event_t before,
  * the call needs 4*r rounded up to 256, plus 4*ceil(n/32) bytes of it, and returns
  * SFNN_ERR_UNSUPPORTED, launching nothing, when r and n need more.  It calls no
  * allocation routine.  The first call on a device looks up that device's address of
- * the array (cudaGetSymbolAddress); make it before any stream capture.  Every call
+ * the array (cudaGetSymbolAddress); make it before any stream capture.  The address
+ * is kept for the life of the process: a cudaDeviceReset of that device frees the
+ * array with its context, and the entry point must not be called on it again.  Every call
  * shares the array: calls that overlap on the GPU (other streams, other host threads)
  * race and must be serialised by the caller.  Asynchronous on `stream`.
  */

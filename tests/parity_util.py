@@ -32,6 +32,35 @@ def mask_from_idx(idx_row, count, n):
     return m
 
 
+GUARD = 64  # canary words on each side of an output buffer
+_PAT = 0x7FC0DEAD  # a NaN bit pattern that no kernel writes
+
+
+def guarded(shape, dtype=torch.float32):
+    """(raw, inner): an output buffer `inner` with canary words on both sides in `raw`
+    (the kernels must write inside it only).  inner starts 256 bytes into raw."""
+    n = int(np.prod(shape))
+    raw = torch.full((n + 2 * GUARD,), _PAT, dtype=torch.int32, device="cuda")
+    return raw, raw[GUARD:GUARD + n].view(dtype).view(shape)
+
+
+def assert_guards(*raws):
+    for raw in raws:
+        r = raw.cpu().numpy()
+        assert (r[:GUARD] == _PAT).all() and (r[-GUARD:] == _PAT).all(), "a kernel wrote outside its output buffer"
+
+
+def fused_step(h, xd):
+    """One token through the fused single-token kernel with the set that kernel itself
+    decided and read (forward_batch at b = 1), outputs inside canary words: (y, mask)."""
+    gy, Y = guarded((1, h.d))
+    gi, idx = guarded((1, h.n), torch.int32)
+    gc, cnt = guarded((1,), torch.int32)
+    h.forward_batch(xd.reshape(1, -1), Y, idx=idx, counts=cnt, return_sets=True)
+    assert_guards(gy, gi, gc)
+    return Y[0].cpu().numpy(), mask_from_idx(idx[0].cpu().numpy(), cnt[0].item(), h.n)
+
+
 def check_token(layer, x, y_gpu, mask_gpu, what=""):
     """Oracle step for token x; arbitrate the sets; tolerance on y.  Returns the error ratio."""
     ref = oracle.forward(layer, x, NTHREADS)

@@ -1,7 +1,8 @@
 """GPU parity at the full sizes of the five workloads (sampled tokens), through the C ABI.
 
-Each token's predicted set must match the oracle's (arbitration band 1e-3 on
-the logit) and y must be within 2e-3 * max|y_ref|.  Batches are checked token
+Each token's set -- the one the fused single-token kernel itself decided and read,
+and for batches the one the batch path used -- must match the oracle's
+(arbitration band 1e-3 on the logit) and y must be within 2e-3 * max|y_ref|.  Batches are checked token
 by token; the 4-layer ReGLU stack both teacher-forced layer by layer and end
 to end with per-layer arbitration.  The single-token workload is also run the
 way the benchmark times it: captured in a CUDA graph over rotating replicas.
@@ -15,7 +16,7 @@ import torch
 import activation_sparse_ffn_threshold_b200 as sf
 import oracle
 import workload as W
-from parity_util import NTHREADS, check_token, dev, mask_from_idx
+from parity_util import NTHREADS, assert_guards, check_token, dev, fused_step, guarded, mask_from_idx
 
 pytestmark = pytest.mark.gpu
 
@@ -27,10 +28,18 @@ def _free():
 
 def _single_token_checks(cfg, lay, h, X):
     for t in range(X.shape[0]):
-        idx, cnt = h.predict(dev(X[t]))
-        m = mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n)
-        y = h.forward(dev(X[t])).cpu().numpy()
+        y, m = fused_step(h, dev(X[t]))
         check_token(lay, X[t], y, m, f"{cfg.name} token {t}")
+        # the call without the set output is the same kernel: bitwise the same y
+        gy, y2 = guarded((cfg.d,))
+        h.forward(dev(X[t]), y2)
+        assert_guards(gy)
+        assert np.array_equal(y2.cpu().numpy(), y)
+        # and the multi-kernel predictor decides as the fused kernel does (outside the band)
+        idx, cnt = h.predict(dev(X[t]))
+        z_ref = oracle.predictor(X[t], lay.A, lay.B, lay.c, NTHREADS)[1]
+        _, mism = oracle.arbitrate(z_ref, m, mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n))
+        assert mism.size == 0
 
 
 def test_tiny_relu_f32_all_tokens():
@@ -75,10 +84,9 @@ def test_opt67b_graph_replicas_match_eager():
     Yg = Y.cpu().numpy()
     Xh = X.cpu().numpy()
     for k in range(K):
-        ye = hs[0].forward(X[k]).cpu().numpy()
+        ye, m = fused_step(hs[0], X[k])
         assert np.array_equal(Yg[k], ye)
-        idx, cnt = hs[0].predict(X[k])
-        check_token(lay, Xh[k], Yg[k], mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n), f"graph step {k}")
+        check_token(lay, Xh[k], Yg[k], m, f"graph step {k}")
     del hs, g
     _free()
 
@@ -94,10 +102,10 @@ def test_llama7b_reglu_stack_full_size():
         _, recs = oracle.forward_stack(layers, x0, nthreads=NTHREADS)
         for li, (lay, h) in enumerate(zip(layers, hs)):
             xin = recs[li]["x_in"]
-            idx, cnt = h.predict(dev(xin))
-            y = h.forward(dev(xin)).cpu().numpy()
-            check_token(lay, xin, y, mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n), f"t={t} layer {li}")
-        # end to end, with each layer's set arbitrated against the GPU's
+            y, m = fused_step(h, dev(xin))
+            check_token(lay, xin, y, m, f"t={t} layer {li}")
+        # end to end (the fused kernel per layer, with the sets it used), each layer's set
+        # arbitrated against the GPU's
         X0 = torch.from_numpy(X[t].astype(np.float32)).cuda()
         XL, sidx, scnt = sf.forward_stack(hs, X0, return_sets=True)
         masks = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), cfg.n) for l in range(cfg.layers)]
@@ -118,7 +126,10 @@ def test_batched_full_size(name, batches):
     h = sf.SparseFFN.from_layer(lay, max_batch=max(batches))
     for b in batches:
         X = W.make_tokens(cfg, b, seed=2, stream_key=b)
-        Y, idx, cnt = h.forward_batch(dev(X), return_sets=True)
+        (gy, Y), (gi, idx), (gc, cnt) = guarded((b, cfg.d)), guarded((b, cfg.n), torch.int32), \
+            guarded((b,), torch.int32)
+        h.forward_batch(dev(X), Y, idx=idx, counts=cnt, return_sets=True)
+        assert_guards(gy, gi, gc)
         Y, idx, cnt = Y.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()
         for t in range(b):
             check_token(lay, X[t], Y[t], mask_from_idx(idx[t], cnt[t], cfg.n), f"{name} b={b} t={t}")

@@ -1,20 +1,25 @@
-"""Degenerate cases of the method on every path (fused single token, tensor-core and
-CUDA-core batches, residual stack):
+"""Degenerate cases of the method on every path (fused single token, fused few-token,
+tensor-core and CUDA-core batches, residual stack):
 
 * a predictor that switches every neuron off: empty sets, y exactly zero, and the
   stack's output exactly its input;
 * a predictor that switches every neuron on: the dense FFN;
 * fewer neurons than SMs (n = 37 and n = 1: tiles of one neuron, empty tiles of work);
 * the smallest d the fp16 layout allows (d = 16, r = 8) and a tensor-core layer with
-  a single 128-column tile (d = 128).
+  a single 128-column tile (d = 128);
+* a layer larger than the device's memory: sfnn_create returns SFNN_ERR_OOM (its
+  first allocation fails before any input is read) and the context stays usable.
 """
+import ctypes
+
 import numpy as np
 import pytest
+import torch
 
 import activation_sparse_ffn_threshold_b200 as sf
 import oracle
 import workload as W
-from parity_util import NTHREADS, check_token, dev, mask_from_idx
+from parity_util import NTHREADS, check_token, dev, fused_step, mask_from_idx
 
 pytestmark = pytest.mark.gpu
 
@@ -32,12 +37,13 @@ def all_paths(cfg, lay, X, max_batch=4):
     batch paths (each batch path reports its own predictor's sets)."""
     h = sf.SparseFFN.from_layer(lay, max_batch=max_batch)
     ys, sets = [], []
-    for x in X:
-        ys.append(h.forward(dev(x)).cpu().numpy())
-        idx, cnt = h.predict(dev(x))
-        sets.append(mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n))
+    for x in X:  # the fused kernel, with the set it used
+        y, m = fused_step(h, dev(x))
+        ys.append(y)
+        sets.append(m)
     out = {"fused": (np.stack(ys), sets)}
-    for name, path in (("cuda-core", sf.BATCH_CUDA_CORE), ("tensor-core", sf.BATCH_TENSOR_CORE)):
+    for name, path in (("cuda-core", sf.BATCH_CUDA_CORE), ("tensor-core", sf.BATCH_TENSOR_CORE),
+                       ("fused-multi", sf.BATCH_FUSED)):
         try:
             h.set_batch_path(path)
         except sf.SfnnError:
@@ -90,3 +96,20 @@ def test_small_shapes(base, d, n, r):
     for name, (Y, sets) in out.items():
         for t in range(4):
             check_token(lay, X[t], Y[t], sets[t], f"{name} d={d} n={n} t={t}")
+
+
+def test_layer_beyond_device_memory_is_oom():
+    # fp16 ReLU rows of d = 65536, n = 2^20 need 2 * 2^20 * 65536 * 2 bytes = 256 GiB;
+    # the library allocates before it reads any input, so small stand-ins suffice
+    lib = sf.load_library()
+    tiny = torch.zeros(64, dtype=torch.float16, device="cuda")
+    p = tiny.data_ptr()
+    desc = sf.LayerDesc(65536, 1 << 20, 8, 1, sf.RELU, sf.F16, p, None, p, p, p, p, p, None, 0)
+    hdl = ctypes.c_void_p()
+    st = lib.sfnn_create(ctypes.byref(desc), None, ctypes.byref(hdl))
+    assert st == sf.STATUS_CODES["SFNN_ERR_OOM"] and not hdl.value
+    cfg, lay = layer("opt6.7b_relu", 256, 700, 64, seed=90)  # the device still serves a layer
+    h = sf.SparseFFN.from_layer(lay)
+    x = W.make_tokens(cfg, 1, seed=91)[0]
+    y, m = fused_step(h, dev(x))
+    check_token(lay, x, y, m, "after a failed create")

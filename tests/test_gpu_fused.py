@@ -1,6 +1,8 @@
 """The fused single-token decode kernel (one launch per token).
 
-* it agrees with the multi-kernel path and with the oracle, on layers whose
+* it agrees with the multi-kernel path and with the oracle -- its own set (the
+  positions each tile decided and read, reported by the kernel) against the oracle's
+  set, then y -- on layers whose
   tiles hold one or several B^T chunks and whose rows need one or several
   columns per thread (fp32 and fp16, ReLU and ReGLU, ragged n);
 * consecutive launches on the same handle (programmatic dependent launch lets
@@ -16,7 +18,7 @@ import torch
 import activation_sparse_ffn_threshold_b200 as sf
 import oracle
 import workload as W
-from parity_util import check_token, dev, mask_from_idx
+from parity_util import check_token, dev, fused_step, mask_from_idx
 
 pytestmark = pytest.mark.gpu
 
@@ -38,13 +40,15 @@ def test_fused_matches_multikernel_and_oracle(base, d, n, r):
     for t in range(4):
         xd = dev(X[t])
         h.set_fused_decode(True)
-        yf = h.forward(xd).cpu().numpy()
+        yf, mf = fused_step(h, xd)
+        assert np.array_equal(h.forward(xd).cpu().numpy(), yf)
         h.set_fused_decode(False)
         ym = h.forward(xd).cpu().numpy()
+        _, idx, cnt = h.forward_batch(xd.reshape(1, -1), return_sets=True)
         h.set_fused_decode(True)
         assert oracle.within_tolerance(yf, ym.astype(np.float64))[0]
-        idx, cnt = h.predict(xd)
-        check_token(lay, X[t], yf, mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n), f"{base} t={t}")
+        check_token(lay, X[t], yf, mf, f"{base} t={t} fused")
+        check_token(lay, X[t], ym, mask_from_idx(idx[0].cpu().numpy(), cnt[0].item(), cfg.n), f"{base} t={t} multi")
     assert h.get_error() == 0
 
 
@@ -62,8 +66,9 @@ def test_back_to_back_launches_same_handle():
     assert torch.equal(Y1, Y2)
     Xh = X.cpu().numpy()
     for t in (0, 7, 15):
-        idx, cnt = h.predict(X[t])
-        check_token(lay, Xh[t], Y1[t].cpu().numpy(), mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n))
+        y, m = fused_step(h, X[t])
+        assert np.array_equal(y, Y1[t].cpu().numpy())
+        check_token(lay, Xh[t], y, m)
     assert h.get_error() == 0
 
 

@@ -8,8 +8,10 @@ unchanged).
   ReLU and ReGLU, d up to 8192, ragged n, and the full OPT-6.7B- and 70B-shaped layers;
 * results are bitwise reproducible; the rows cost a half (int8) or a quarter (int4) of
   the bytes of fp16 rows;
-* only the fused single-token path serves such a layer: batches, explicit sets and
-  the multi-kernel path are refused with SFNN_ERR_UNSUPPORTED, the predictor works.
+* only the fused single-token path serves such a layer (also at b = 1 through
+  forward_batch, which returns the set the kernel used: that set is the one checked);
+  batches, explicit sets and the multi-kernel path are refused with
+  SFNN_ERR_UNSUPPORTED, the predictor works.
 """
 import numpy as np
 import pytest
@@ -17,7 +19,7 @@ import pytest
 import activation_sparse_ffn_threshold_b200 as sf
 import oracle
 import workload as W
-from parity_util import NTHREADS, REL_TOL, dev, mask_from_idx
+from parity_util import NTHREADS, REL_TOL, dev, fused_step
 
 pytestmark = pytest.mark.gpu
 
@@ -39,9 +41,7 @@ def run_tokens(cfg, lay, h, count, seed, rows):
     X = W.make_tokens(cfg, count, seed=seed)
     for t in range(count):
         xd = dev(X[t])
-        y = h.forward(xd).cpu().numpy()
-        idx, cnt = h.predict(xd)
-        m = mask_from_idx(idx.cpu().numpy(), cnt.item(), cfg.n)
+        y, m = fused_step(h, xd)
         check_token_q(lay, qr, X[t], y, m, f"{cfg.name} t={t}")
         assert np.array_equal(h.forward(xd).cpu().numpy(), y)
 

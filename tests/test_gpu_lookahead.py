@@ -1,9 +1,10 @@
 """The look-ahead residual stack: layer l+1's set predicted from layer l's input.
 
 * the fused look-ahead kernel (one launch per layer plus one) and the multi-kernel
-  look-ahead path both match the oracle's look-ahead stack, with every layer's set
-  arbitrated against the oracle's, for ReLU and ReGLU, at a reduced size and at the
-  full LLaMA-7B-shaped 4-layer ReGLU stack;
+  look-ahead path both match the oracle's look-ahead stack, with every layer's set --
+  each path's own: the lists the fused launches consumed, the masks the multi-kernel
+  path compacted -- arbitrated against the oracle's, for ReLU and ReGLU, at a reduced
+  size and at the full LLaMA-7B-shaped 4-layer ReGLU stack;
 * the sets really are predicted one layer early: they differ from the plain stack's;
 * one layer (nothing to look ahead of) gives the plain stack's result;
 * batches of tokens through the multi-kernel path, on tensor and CUDA cores;
@@ -27,29 +28,47 @@ def _x0(cfg, seed):
     return W.make_tokens(cfg, 1, seed=seed)[0].astype(np.float32)
 
 
-def _run(hs, x0):
-    """(XL of the fused path, XL of the multi-kernel path, that path's per-layer masks)."""
-    X0 = torch.from_numpy(x0).cuda()
-    XL_fused = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
-    XL_sets, sidx, scnt = sf.forward_stack(hs, X0, return_sets=True, lookahead=True)
+def _stack_sets(hs, X0):
+    XL, sidx, scnt = sf.forward_stack(hs, X0, return_sets=True, lookahead=True)
     n = hs[0].n
-    masks = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), n) for l in range(len(hs))]
-    return XL_fused, XL_sets.cpu().numpy(), masks
+    return XL.cpu().numpy(), [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), n) for l in range(len(hs))]
+
+
+def _run(hs, x0):
+    """[(what, XL, per-layer masks)] of the fused path and of the multi-kernel path, each
+    with the sets it used itself (the fused kernel's set output is checked against its
+    plain call, which must give bitwise the same XL)."""
+    X0 = torch.from_numpy(x0).cuda()
+    XL_plain = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
+    XL_fused, m_fused = _stack_sets(hs, X0)
+    distinct = all(a is not b for a, b in zip(hs, hs[1:]))
+    if distinct:  # the fused path serves a set request (else the multi-kernel path does)
+        assert np.array_equal(XL_plain, XL_fused)
+    for h in hs:
+        h.set_fused_decode(False)
+    try:
+        XL_multi, m_multi = _stack_sets(hs, X0)
+    finally:
+        for h in hs:
+            h.set_fused_decode(True)
+    out = [("multi-kernel", XL_multi, m_multi)]
+    out.append(("fused", XL_fused, m_fused) if distinct else ("fused (its sets unreported)", XL_plain, m_multi))
+    return out
 
 
 def _check(layers, hs, x0, qrows=None):
-    XL_fused, XL_sets, masks = _run(hs, x0)
-    xref, recs = oracle.forward_stack_lookahead(layers, x0.astype(np.float64), masks_other=masks,
-                                                nthreads=NTHREADS, qrows=qrows)
-    for l, rec in enumerate(recs):
-        assert rec["mismatches"].size == 0, f"layer {l}: sets differ outside the arbitration band"
+    runs = _run(hs, x0)
     base = x0.astype(np.float64)
-    for what, XL in (("fused", XL_fused), ("multi-kernel", XL_sets)):
+    for what, XL, masks in runs:
+        xref, recs = oracle.forward_stack_lookahead(layers, x0.astype(np.float64), masks_other=masks,
+                                                    nthreads=NTHREADS, qrows=qrows)
+        for l, rec in enumerate(recs):
+            assert rec["mismatches"].size == 0, f"{what}, layer {l}: sets differ outside the arbitration band"
         ok, ratio = oracle.within_tolerance(XL.astype(np.float64) - base, xref - base)
         assert ok, f"{what}: max|dx|/max|dx_ref| = {ratio:.3e}"
     for h in hs:
         assert h.get_error() == 0
-    return XL_fused, masks, recs
+    return runs[-1][1], runs[-1][2], None
 
 
 @pytest.mark.parametrize("base", ["llama7b_reglu_stack", "opt6.7b_relu"])
@@ -106,7 +125,7 @@ def test_lookahead_one_layer_is_the_plain_stack():
     b = sf.forward_stack([h], X0).cpu().numpy()
     # the same set (the predictors' orders are the same); the rows are shared out to the
     # CTAs differently, so y agrees within the tolerance, and with the oracle's
-    _, _, masks = _run([h], x0)
+    _, masks = _stack_sets([h], X0)
     xref, recs = oracle.forward_stack([lay], x0.astype(np.float64), masks_other=masks)
     assert recs[0]["mismatches"].size == 0
     base = x0.astype(np.float64)
@@ -123,19 +142,18 @@ def test_lookahead_one_handle_for_every_layer():
     _check([lay] * 3, [h] * 3, _x0(cfg, 57))
 
 
-def test_lookahead_int8_rows():
-    # Two layers: with look-ahead both sets are predicted from u_0, so they do not depend
-    # on the rows' storage, and the sets of fp16 handles of the same layers (int8 rows run
-    # the fused kernel only, which returns no sets) serve for the arbitration.
+@pytest.mark.parametrize("rows", ["int8", "int4"])
+def test_lookahead_quantized_rows(rows):
+    # int8 / int4 rows run the fused kernel only; its set output gives the sets it used
     cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
-    layers = [W.make_layer(cfg, seed=58, layer=l) for l in range(2)]
-    hs = [sf.SparseFFN.from_layer(l, rows="int8") for l in layers]
+    layers = [W.make_layer(cfg, seed=58, layer=l) for l in range(3)]
+    hs = [sf.SparseFFN.from_layer(l, rows=rows) for l in layers]
     x0 = _x0(cfg, 59)
     X0 = torch.from_numpy(x0).cuda()
     XL = sf.forward_stack(hs, X0, lookahead=True).cpu().numpy()
-    hf = [sf.SparseFFN.from_layer(l) for l in layers]
-    _, _, masks = _run(hf, x0)
-    qrows = [oracle.quantize_layer(l) for l in layers]
+    XL_sets, masks = _stack_sets(hs, X0)
+    assert np.array_equal(XL, XL_sets)
+    qrows = [oracle.quantize_layer(l, bits=8 if rows == "int8" else 4) for l in layers]
     xref, recs = oracle.forward_stack_lookahead(layers, x0.astype(np.float64), masks_other=masks,
                                                 nthreads=NTHREADS, qrows=qrows)
     assert all(r["mismatches"].size == 0 for r in recs)
@@ -151,9 +169,9 @@ def test_lookahead_empty_sets_leave_the_input():
         l.c = np.full_like(l.c, -1e4)  # every logit far below the threshold
     hs = [sf.SparseFFN.from_layer(l) for l in layers]
     x0 = _x0(cfg, 61)
-    XL_fused, XL_sets, masks = _run(hs, x0)
-    assert all(m.sum() == 0 for m in masks)
-    assert np.array_equal(XL_fused, x0) and np.array_equal(XL_sets, x0)
+    for _, XL, masks in _run(hs, x0):
+        assert all(m.sum() == 0 for m in masks)
+        assert np.array_equal(XL, x0)
 
 
 def test_lookahead_barrier_timeout_is_reported_and_recovers():

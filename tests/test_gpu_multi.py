@@ -1,0 +1,120 @@
+"""The multi-token fused kernel: a batch of 2 to 4 tokens in one launch on CUDA cores.
+
+* every token agrees with the oracle, with the set that kernel itself decided and read
+  (its per-token set output) arbitrated against the oracle's, for ReLU and ReGLU,
+  ragged n, d up to 8192 and 2, 3 or 4 tokens;
+* it agrees with the tensor-core path within the tolerance, is bitwise reproducible,
+  and its set output changes nothing (the plain call gives bitwise the same Y);
+* a token's row of Y does not depend on which other tokens share the batch (a row
+  applies only to the tokens whose sets hold it);
+* AUTO takes it for 2 to 4 tokens on the full OPT-30B- and 70B-shaped layers, and the
+  residual stack runs through it;
+* outputs stay inside their buffers (canary words on both sides).
+"""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_ffn_threshold_b200 as sf
+import oracle
+import workload as W
+from parity_util import NTHREADS, assert_guards, check_token, dev, guarded, mask_from_idx
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    ("opt6.7b_relu", 1024, 3001, 128),
+    ("70b_reglu", 2048, 5003, 256),
+    ("opt30b_relu", 7168, 4099, 1024),
+    ("70b_reglu", 8192, 1500, 1024),
+]
+
+
+def run_multi(h, X, sets=True):
+    """(Y, per-token masks) of one forward_batch call, outputs inside canary words."""
+    b = X.shape[0]
+    gy, Y = guarded((b, h.d))
+    if not sets:
+        h.forward_batch(dev(X), Y)
+        assert_guards(gy)
+        return Y.cpu().numpy(), None
+    gi, idx = guarded((b, h.n), torch.int32)
+    gc, cnt = guarded((b,), torch.int32)
+    h.forward_batch(dev(X), Y, idx=idx, counts=cnt, return_sets=True)
+    assert_guards(gy, gi, gc)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    return Y.cpu().numpy(), [mask_from_idx(idx[t], cnt[t], h.n) for t in range(b)]
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+@pytest.mark.parametrize("base,d,n,r", SHAPES)
+def test_multi_matches_oracle(base, d, n, r, b):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=71)
+    h = sf.SparseFFN.from_layer(lay, max_batch=4)
+    h.set_batch_path(sf.BATCH_FUSED)
+    X = W.make_tokens(cfg, b, seed=72 + b)
+    Y, masks = run_multi(h, X)
+    for t in range(b):
+        check_token(lay, X[t], Y[t], masks[t], f"{base} d={d} b={b} t={t}")
+    Y2, _ = run_multi(h, X, sets=False)
+    assert np.array_equal(Y, Y2)  # the set output changes nothing; bitwise reproducible
+    Y3, masks3 = run_multi(h, X)
+    assert np.array_equal(Y, Y3) and all(np.array_equal(a, c) for a, c in zip(masks, masks3))
+    if d % 128 == 0:
+        h.set_batch_path(sf.BATCH_TENSOR_CORE)
+        Yt, masks_t = run_multi(h, X)
+        for t in range(b):
+            if np.array_equal(masks[t], masks_t[t]):
+                assert oracle.within_tolerance(Y[t], Yt[t].astype(np.float64))[0]
+    assert h.get_error() == 0
+
+
+def test_rows_do_not_depend_on_the_other_tokens():
+    cfg = W.small_config(W.CONFIGS["70b_reglu"], d=2048, n=5003, r=256)
+    lay = W.make_layer(cfg, seed=73)
+    h = sf.SparseFFN.from_layer(lay, max_batch=4)
+    h.set_batch_path(sf.BATCH_FUSED)
+    X = W.make_tokens(cfg, 6, seed=74)
+    Ya, ma = run_multi(h, X[[0, 1, 2, 3]])
+    Yb, mb = run_multi(h, X[[4, 0, 5]])
+    assert np.array_equal(ma[0], mb[1])
+    # the same rows, the same order of every sum: token 0's output is bitwise the same
+    assert np.array_equal(Ya[0], Yb[1])
+    y1, m1 = run_multi(h, X[[0, 5]])
+    assert np.array_equal(Ya[0], y1[0])
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("name,batches", [("opt30b_relu", (2, 4)), ("70b_reglu", (2, 3, 4))])
+def test_multi_full_size_auto(name, batches):
+    cfg = W.CONFIGS[name]
+    lay = W.make_layer(cfg, seed=0)
+    h = sf.SparseFFN.from_layer(lay, max_batch=max(batches))
+    assert h.info()["batch_path"] == sf.BATCH_AUTO
+    for b in batches:
+        X = W.make_tokens(cfg, b, seed=75, stream_key=b)
+        Y, masks = run_multi(h, X)
+        for t in range(b):
+            check_token(lay, X[t], Y[t], masks[t], f"{name} b={b} t={t}")
+    assert h.get_error() == 0
+    del h
+    torch.cuda.empty_cache()
+
+
+def test_stack_of_two_tokens_through_the_multi_kernel():
+    cfg = W.small_config(W.CONFIGS["llama7b_reglu_stack"], d=1024, n=2500, r=128)
+    layers = [W.make_layer(cfg, seed=76, layer=l) for l in range(3)]
+    hs = [sf.SparseFFN.from_layer(l, max_batch=2) for l in layers]
+    X0 = W.make_tokens(cfg, 2, seed=77).astype(np.float32)
+    XL, sidx, scnt = sf.forward_stack(hs, torch.from_numpy(X0).cuda(), return_sets=True)
+    XL_plain = sf.forward_stack(hs, torch.from_numpy(X0).cuda())
+    assert torch.equal(XL, XL_plain)
+    XL = XL.cpu().numpy()
+    for t in range(2):
+        masks = [mask_from_idx(sidx[l, t].cpu().numpy(), scnt[l, t].item(), cfg.n) for l in range(3)]
+        xref, recs = oracle.forward_stack(layers, X0[t].astype(np.float64), masks_other=masks, nthreads=NTHREADS)
+        assert all(r["mismatches"].size == 0 for r in recs)
+        base = X0[t].astype(np.float64)
+        assert oracle.within_tolerance(XL[t].astype(np.float64) - base, xref - base)[0]
+    assert all(h.get_error() == 0 for h in hs)
