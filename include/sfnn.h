@@ -40,6 +40,14 @@
  *    latched in the handle and returned by sfnn_get_error.
  *  - A handle must not be used from two streams at the same time: its scratch
  *    memory is shared by its calls.
+ *  - The fused kernels (single token, few tokens, look-ahead stack) run one CTA per
+ *    SM that fills the SM's registers, and synchronise all their CTAs with grid
+ *    barriers: every SM must be able to take one of them.  A kernel that occupies an
+ *    SM on another stream delays the CTA bound for it, and the barriers wait for that
+ *    CTA (correct, but slower); if it does not arrive within about one second the
+ *    launch gives up and latches SFNN_ERR_TIMEOUT.  Two fused launches of different
+ *    handles on concurrent streams can each hold part of the SMs and so time out:
+ *    serialise them.
  *  - Index lists have set semantics: they hold each selected neuron once, in
  *    the caller's original numbering, in the handle's internal (hotness) order,
  *    which is deterministic.

@@ -103,3 +103,26 @@ def test_grid_barrier_timeout_is_reported_and_recovers():
     y_again = h.forward(xd).cpu().numpy()
     assert np.array_equal(y_again, y_ok)
     assert h.get_error() == 0
+
+
+def test_fused_kernels_beside_a_kernel_on_another_stream():
+    """The fused kernels' grid barriers need all their CTAs resident; a kernel that holds
+    an SM on another stream (a bounded spin of ~20 ms here) delays the CTAs that would
+    run there, and the barriers wait for them (well inside their one-second bound):
+    results stay exact and no error is latched."""
+    cfg = W.small_config(W.CONFIGS["70b_reglu"], d=2048, n=5003, r=256)
+    lay = W.make_layer(cfg, seed=19)
+    h = sf.SparseFFN.from_layer(lay, max_batch=4)
+    X = dev(W.make_tokens(cfg, 4, seed=20))
+    y_ref = h.forward(X[0]).clone()
+    Y_ref = h.forward_batch(X).clone()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    for _ in range(2):
+        with torch.cuda.stream(side):
+            torch.cuda._sleep(40_000_000)  # ~20 ms at the B200's clocks
+        y = h.forward(X[0])
+        Y = h.forward_batch(X)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_ref) and torch.equal(Y, Y_ref)
+    assert h.get_error() == 0

@@ -118,3 +118,30 @@ def test_stack_of_two_tokens_through_the_multi_kernel():
         base = X0[t].astype(np.float64)
         assert oracle.within_tolerance(XL[t].astype(np.float64) - base, xref - base)[0]
     assert all(h.get_error() == 0 for h in hs)
+
+
+@pytest.mark.parametrize("base", ["opt6.7b_relu", "70b_reglu"])
+def test_hot_prefix_changes_nothing(base):
+    """The hot prefix only moves the hottest rows' gate/up dots ahead of the predictor's
+    barrier: the same dots, the same sums, bitwise the same Y and sets."""
+    cfg = W.small_config(W.CONFIGS[base], d=2048, n=5003, r=256)
+    lay = W.make_layer(cfg, seed=78)
+    h = sf.SparseFFN.from_layer(lay, max_batch=4)
+    h.set_batch_path(sf.BATCH_FUSED)
+    for b in (2, 3, 4):
+        X = W.make_tokens(cfg, b, seed=79 + b)
+        Y_on, m_on = run_multi(h, X)
+        h.set_hot_prefix(False)
+        Y_off, m_off = run_multi(h, X)
+        h.set_hot_prefix(True)
+        assert np.array_equal(Y_on, Y_off)
+        assert all(np.array_equal(a, c) for a, c in zip(m_on, m_off))
+        for t in range(b):
+            check_token(lay, X[t], Y_on[t], m_on[t], f"{base} b={b} t={t}")
+    # without a hotness profile there is no prefix, and the layer still decodes correctly
+    h0 = sf.SparseFFN.from_layer(lay, max_batch=4, use_hotness=False)
+    X = W.make_tokens(cfg, 3, seed=90)
+    Y, masks = run_multi(h0, X)
+    for t in range(3):
+        check_token(lay, X[t], Y[t], masks[t], f"{base} identity order t={t}")
+    assert h.get_error() == 0 and h0.get_error() == 0
