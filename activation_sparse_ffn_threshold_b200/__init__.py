@@ -52,7 +52,7 @@ class LayerDesc(ctypes.Structure):
                 ("w_up", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("b", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p), ("pa", ctypes.c_void_p), ("pb", ctypes.c_void_p),
                 ("pc", ctypes.c_void_p), ("hotness", ctypes.POINTER(ctypes.c_float)),
-                ("rows_dtype", ctypes.c_int32)]
+                ("rows_dtype", ctypes.c_int32), ("order", ctypes.c_int32)]
 
 
 class Info(ctypes.Structure):
@@ -160,12 +160,15 @@ class SparseFFN:
     """
 
     def __init__(self, w_up, w_down, b, A, B, c, act: str = "relu", w_gate=None, hotness=None,
-                 max_batch: int = 1, device=None, stream=None, rows: str | None = None):
+                 max_batch: int = 1, device=None, stream=None, rows: str | None = None, order: str = "dealt"):
         """``rows="int8"`` / ``"int4"`` stores the FFN rows as int8 / int4 codes with
         per-row fp32 scales (fp16 layers; single-token fused path only, see
-        sfnn_layer_desc.rows_dtype)."""
+        sfnn_layer_desc.rows_dtype).  ``order`` ("dealt" or "packed") is the storage
+        order of the neurons by hotness (sfnn_layer_desc.order)."""
         if rows not in (None, "int8", "int4"):
             raise ValueError("rows must be None, 'int8' or 'int4'")
+        if order not in ("dealt", "packed"):
+            raise ValueError("order must be 'dealt' or 'packed'")
         lib = load_library()
         device = torch.device(device or "cuda")
         dtype = w_up.dtype if isinstance(w_up, torch.Tensor) else torch.from_numpy(np.asarray(w_up[:1])).dtype
@@ -189,7 +192,7 @@ class SparseFFN:
                          w_up_t.data_ptr(), w_gate_t.data_ptr() if w_gate_t is not None else None,
                          b_t.data_ptr(), w_down_t.data_ptr(), A_t.data_ptr(), B_t.data_ptr(), c_t.data_ptr(),
                          self._hot.ctypes.data_as(ctypes.POINTER(ctypes.c_float)) if self._hot is not None
-                         else None, {"int8": I8, "int4": I4}.get(rows, 0))
+                         else None, {"int8": I8, "int4": I4}.get(rows, 0), 0 if order == "dealt" else 1)
         self.rows = rows
         self._h = ctypes.c_void_p()
         with torch.cuda.device(device):
@@ -198,11 +201,11 @@ class SparseFFN:
 
     @classmethod
     def from_layer(cls, layer, max_batch: int = 1, use_hotness: bool = True, device=None, stream=None,
-                   rows: str | None = None):
+                   rows: str | None = None, order: str = "dealt"):
         """Build from a record with w_up, w_gate, b, w_down, A, B, c, p and cfg.act (numpy arrays)."""
         return cls(layer.w_up, layer.w_down, layer.b, layer.A, layer.B, layer.c, act=layer.cfg.act,
                    w_gate=layer.w_gate, hotness=layer.p if use_hotness else None, max_batch=max_batch,
-                   device=device, stream=stream, rows=rows)
+                   device=device, stream=stream, rows=rows, order=order)
 
     # ------------------------------------------------------------------ helpers
     def _check_x(self, x, rows=None):

@@ -67,6 +67,7 @@ sfnn_status check_desc(const sfnn_layer_desc *d) {
   if (d->max_batch > kMaxBatch) return SFNN_ERR_UNSUPPORTED;
   if ((int64_t)d->r * d->max_batch > 32768) return SFNN_ERR_UNSUPPORTED;
   if (d->n > kMaxNeurons || d->d > (1 << 16)) return SFNN_ERR_UNSUPPORTED;
+  if (d->order != SFNN_ORDER_DEALT && d->order != SFNN_ORDER_PACKED) return SFNN_ERR_INVALID_ARG;
   return SFNN_OK;
 }
 
@@ -331,7 +332,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   } else {
     std::iota(by_rank.begin(), by_rank.end(), 0);
   }
-  for (int k = 0; k < L.n; ++k) perm[decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
+  const bool packed = desc->hotness && desc->order == SFNN_ORDER_PACKED;
+  for (int k = 0; k < L.n; ++k) perm[packed ? k : decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
   for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
   for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
   // The multi-token kernel's hot prefix for b tokens: the hottest ranks whose neuron is in
@@ -339,7 +341,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   h->hot_on = true;
   for (int b = 0; b <= kMultiMaxTokens; ++b) {
     h->hot_rows[b] = 0;
-    if (!desc->hotness || b < 2) continue;
+    if (!desc->hotness || packed || b < 2) continue;
     int k = 0;
     while (k < L.n && k < 64 * G) {
       const float q = desc->hotness[by_rank[k]];

@@ -66,6 +66,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
+    ap.add_argument("--order", choices=["dealt", "packed", "identity"], default="dealt",
+                    help="storage order of the neurons: hotness ranks dealt round-robin to the SM tiles (default), "
+                         "hot-packed-first, or the original order (no hotness profile)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--rows", choices=["native", "int8", "int4"], default="native",
                     help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 / int4 "
@@ -402,6 +405,11 @@ def _free(*objs):
     torch.cuda.empty_cache()
 
 
+def _order_kw(args):
+    order = getattr(args, "order", "dealt")
+    return {"use_hotness": order != "identity", "order": "packed" if order == "packed" else "dealt"}
+
+
 def measure_single(cfg, args, dist, dev, rows=None, headline=False):
     """Batch-1 decode: the workload's tokens, one forward call each, over rotating weight
     replicas, captured in one CUDA graph; one step = one replay."""
@@ -420,7 +428,7 @@ def measure_single(cfg, args, dist, dev, rows=None, headline=False):
     # replicas: bytes touched between two visits of a replica >= 2 x L2 (at most one per
     # token: a layer too small for that, the tiny fp32 one, stays L2-resident anyway)
     R = args.replicas or min(T, max(2, 1 + math.ceil(2 * l2 / per_token)))
-    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows) for _ in range(R)]
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows, **_order_kw(args)) for _ in range(R)]
     info = handles[0].info()
     torch.cuda.synchronize()
     X = torch.from_numpy(Xh).to(dev)
@@ -495,7 +503,7 @@ def measure_batch(cfg, b, args, dist, dev):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_batch = W.touched_bytes(cfg, W.expected_union_density(lay.p, b) * cfg.n, b)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
-    handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b) for _ in range(R)]
+    handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b, **_order_kw(args)) for _ in range(R)]
     info = handles[0].info()
     torch.cuda.synchronize()
     X = torch.from_numpy(Xh).to(dev)
@@ -680,7 +688,7 @@ def run_sfnn(args, dist):
         "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16" if cfg.esize == 2 else "f32", "data": "synthetic",
         "config": {"workload": cfg.description + (f", {rows} rows (per-row fp32 scales)" if rows else ""),
-                   "batch": 1, "tokens_per_step": T, "replicas": m["replicas"],
+                   "batch": 1, "tokens_per_step": T, "replicas": m["replicas"], "order": args.order,
                    "l2": f"inputs larger than L2: {m['replicas']} weight replicas rotated per token, "
                          f"{m['bytes_per_step'] / T / 1e6:.1f} MB touched per token",
                    "parallelism": f"replicas x{dist.world} (no exchange)",
@@ -709,7 +717,7 @@ def run_batch(args, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16" if cfg.esize == 2 else "f32", "data": "synthetic",
         "config": {"workload": cfg.description, "batch": b, "batches_per_step": BATCHES_PER_STEP,
-                   "path": m["path"], "replicas": m["replicas"],
+                   "path": m["path"], "replicas": m["replicas"], "order": args.order,
                    "l2": f"inputs larger than L2: {m['replicas']} weight replicas rotated per batch, "
                          f"{m['bytes_per_step'] / BATCHES_PER_STEP / 1e6:.1f} MB touched per batch",
                    "parallelism": f"replicas x{dist.world} (no exchange)", "mean_union_rows": m["mean_union_rows"]},

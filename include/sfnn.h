@@ -152,7 +152,19 @@ typedef struct {
      * 53ai.com "sparsity for LLM inference" page, evaluation) without fixing a scheme.
      */
     int32_t rows_dtype;
+    /*
+     * Storage order of the neurons when a hotness profile is given (sfnn_order):
+     * SFNN_ORDER_DEALT (0, the default) deals the hotness ranks round-robin to the SM
+     * tiles of the fused kernels, hottest first inside each tile, so every tile gets the
+     * same mix of hot and cold neurons; SFNN_ORDER_PACKED (1) stores the neurons in
+     * plain descending hotness, the hot ones contiguous at the front (one tile then holds
+     * the hottest neurons; the few-token path reads no hot prefix).  Both follow
+     * PowerInfer's offline hot/cold profiling (53ai.com page, section 概述).
+     */
+    int32_t order;
 } sfnn_layer_desc;
+
+typedef enum { SFNN_ORDER_DEALT = 0, SFNN_ORDER_PACKED = 1 } sfnn_order;
 
 /* Read-only facts about a handle (sizes in bytes). */
 typedef struct {

@@ -20,7 +20,7 @@ import torch
 import activation_sparse_ffn_threshold_b200 as sf
 import oracle
 import workload as W
-from parity_util import L, NTHREADS, check_token, dev, mask_from_idx
+from parity_util import L, NTHREADS, check_token, dev, fused_step, mask_from_idx
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "powerinfer_example.json")
@@ -161,21 +161,39 @@ def test_reduced_shapes_parity(small_layer):
 
 
 def test_determinism_and_hotness_invariance(small_layer):
+    """The storage order (hotness dealt to the tiles, hot-packed-first, or the original
+    order without a profile) changes no set and y only within rounding, on the fused
+    single-token kernel, the few-token kernel and the tensor-core batch path."""
     cfg, lay = small_layer
-    h_hot = sf.SparseFFN.from_layer(lay, use_hotness=True)
-    h_id = sf.SparseFFN.from_layer(lay, use_hotness=False)
+    hs = {"dealt": sf.SparseFFN.from_layer(lay, use_hotness=True, max_batch=4),
+          "packed": sf.SparseFFN.from_layer(lay, use_hotness=True, max_batch=4, order="packed"),
+          "identity": sf.SparseFFN.from_layer(lay, use_hotness=False, max_batch=4)}
     X = W.make_tokens(cfg, 4, seed=7)
     for t in range(4):
         xd = dev(X[t])
-        a = h_hot.forward(xd).cpu().numpy()
-        b = h_hot.forward(xd).cpu().numpy()
-        assert np.array_equal(a, b)
-        c = h_id.forward(xd).cpu().numpy()
-        assert oracle.within_tolerance(c, a.astype(np.float64))[0]
-        i1, c1 = h_hot.predict(xd)
-        i2, c2 = h_id.predict(xd)
-        assert c1.item() == c2.item()
-        assert set(i1[: c1.item()].cpu().tolist()) == set(i2[: c2.item()].cpu().tolist())
+        a = hs["dealt"].forward(xd).cpu().numpy()
+        assert np.array_equal(a, hs["dealt"].forward(xd).cpu().numpy())
+        sets = {}
+        for name, h in hs.items():
+            y, m = fused_step(h, xd)
+            assert oracle.within_tolerance(y, a.astype(np.float64))[0], name
+            check_token(lay, X[t], y, m, f"{name} t={t}")
+            sets[name] = m
+        assert np.array_equal(sets["dealt"], sets["packed"]) and np.array_equal(sets["dealt"], sets["identity"])
+    for path in (sf.BATCH_FUSED, sf.BATCH_TENSOR_CORE):
+        Ys = {}
+        for name, h in hs.items():
+            try:
+                h.set_batch_path(path)
+            except sf.SfnnError:  # a layer this path cannot serve
+                continue
+            Y, idx, cnt = h.forward_batch(dev(X), return_sets=True)
+            Ys[name] = Y.cpu().numpy()
+            for t in range(4):
+                check_token(lay, X[t], Ys[name][t], mask_from_idx(idx[t].cpu().numpy(), cnt[t].item(), cfg.n),
+                            f"{name} path {path} t={t}")
+        for name in Ys:
+            assert oracle.within_tolerance(Ys[name], Ys["dealt"].astype(np.float64))[0]
 
 
 @pytest.mark.parametrize("act", ["relu", "reglu"])
