@@ -34,7 +34,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt, h->scnt};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt, h->scnt, h->blist, h->bcnt};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -202,6 +202,11 @@ void plan_decode1(sfnn_ctx *h, int G) {
   P.rq = L.rows_q;
   P.rscale = h->rscale;
   P.nseg = (L.d / (L.rows_q ? 128 / L.rows_q : L.vec) + 255) / 256;  // 4 KB C1 segments of a row
+  P.blist = h->blist;
+  P.bcnt = h->bcnt;
+  // the rebalancing's scratch (counts, their prefix, the share) lives in the CTA's
+  // 512-word reduce buffer
+  P.quota = 2 * G + 3 <= kDecode1Threads ? std::min(h->quota, P.tile_max) : 0;
   if (L.r / L.vec > 32 * 4) return;
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
@@ -336,6 +341,19 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   for (int k = 0; k < L.n; ++k) perm[packed ? k : decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
   for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
   for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
+  // The single-token kernel's quota of own rows per CTA: 0.8 of a tile's expected active
+  // count under the profile (at least 2; no profile, no rebalancing).
+  h->quota = 0;
+  if (desc->hotness) {
+    double mean = 0.0;
+    for (int i = 0; i < L.n; ++i) {
+      const float q = desc->hotness[i];
+      mean += std::isnan(q) ? 0.0 : std::min(1.0, std::max(0.0, (double)q));
+    }
+    mean /= G;
+    const int qv = (int)std::floor(0.8 * mean);
+    h->quota = qv >= 2 ? qv : 0;
+  }
   // The multi-token kernel's hot prefix for b tokens: the hottest ranks whose neuron is in
   // a b-token union with probability 1 - (1 - p)^b >= 0.99 (at most 64 rows per tile).
   h->hot_on = true;
@@ -376,7 +394,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {&h->bias, n * e, true},
       {(void **)&h->perm, n * 4, true},
       {(void **)&h->iperm, n * 4, true},
-      {(void **)&h->h, mb * r * 4, false},
+      {(void **)&h->h, std::max<size_t>(mb, 2) * r * 4, false},
       {(void **)&h->mask, mb * L.nwords * 4, false},
       {(void **)&h->ulist, n * 4, false},
       {(void **)&h->utok, n * 4, false},
@@ -391,6 +409,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->alist, n * sizeof(int2), false},
       {(void **)&h->acnt, (size_t)G * 4, false},
       {(void **)&h->scnt, (size_t)G * 4 * mb, false},
+      {(void **)&h->blist, n * sizeof(int2), false},
+      {(void **)&h->bcnt, (size_t)G * 4, false},
       {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
       {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
   };

@@ -55,6 +55,9 @@ struct sfnn_ctx {
   uint64_t *bar;     // grid barrier arrival counter of the fused kernel
   int2 *alist;       // [n] look-ahead stack: this layer's predicted active lists per tile
   int32_t *acnt;     // [G]   (storage position, bias) pairs and counts, from the launch before
+  int2 *blist;       // [n] rebalancing: each tile's active (storage position, bias) pairs
+  int32_t *bcnt;     // [G]   and their counts (single-token fused kernel)
+  int quota;         // its per-CTA quota of own rows (0: no rebalancing)
   int32_t *scnt;     // [max_batch][G] per-tile counts of the sets a fused launch used (lists: ulist
                      //   for one token, acoef's words for several)
   int multi_max;     // largest batch the multi-token fused kernel serves (0: none)

@@ -10,16 +10,17 @@
 //   so every tile holds the same mix of hot and cold neurons (equal expected work),
 //   hottest first inside the tile.
 //
-//   A   h_j = relu(A^T[j] . x): one warp per predictor row, every chunk of the row
-//       requested at once (the first row before waiting for the previous kernel).
-//       h goes to global memory; grid barrier.
-//   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron; each warp's B^T rows
-//       stream through 4 shared-memory stages of its own (16-byte cp.async copies,
-//       the first ones requested during phase A); neuron i is active iff
-//       z_i > 0 (sigmoid(z) > 0.5).  The tile's active positions are compacted in order.
-//   C1  up (and gate) dot products of the tile's active rows, split in 4 KB segments
-//       spread over all warps (2-deep register pipeline); segment sums added in a
-//       fixed order, then ReLU / ReGLU.  Rows of inactive neurons are never requested.
+//   A   h_j = relu(A^T[j] . x): each predictor row split in two halves over a pair of
+//       warps, every chunk of the first half row requested before waiting for the
+//       previous kernel; the halves' sums go to global memory; grid barrier.
+//   B   z_i = B^T[i] . h + c_i for the tile, one warp per neuron (h = relu of the two
+//       halves' sum, formed once per CTA); each warp's B^T rows stream through 4
+//       shared-memory stages of its own (16-byte cp.async copies, the first ones requested
+//       during phase A); neuron i is active iff z_i > 0 (sigmoid(z) > 0.5).  The tile's
+//       active positions are compacted in order.
+//   C1  up (and gate) dot products of the active rows, split in 4 KB segments spread
+//       over all warps (2-deep register pipeline); segment sums added in a fixed order,
+//       then ReLU / ReGLU.  Rows of inactive neurons are never requested.
 //   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
 //       column accumulators; each thread's chunks stream through up to 8 private
 //       shared-memory stages, the first ones requested at C1's start.
@@ -27,16 +28,19 @@
 //       slice of all G partials in a fixed order (two-phase, deterministic) -> y
 //       (+ residual, + rounded next-layer input).
 //
-// Every CTA works on the active rows of its own tile: the rows are never exchanged, so
-// the kernel has two grid barriers, and the hotness deal keeps the tiles' expected
-// counts equal (the busiest tile of a token typically holds 1.5-1.7x the mean).
+// Which CTA reads which active rows: the hotness deal keeps the tiles' expected counts
+// equal, but the busiest tile of a token still holds ~1.5x the mean, and with its own
+// tile's rows alone that CTA finishes long after the others.  With a quota (set from the
+// hotness profile: 0.8 of a tile's expected count) each CTA keeps its first `quota` rows,
+// publishes its tile's list and arrives on a split grid barrier; after its own rows' C1
+// it waits there, and the rows past the quota in all tiles are shared out evenly over
+// the CTAs in tile order -- a function of the counts alone, so every sum keeps a fixed
+// order and results stay bitwise reproducible.  Without a quota every CTA takes its own
+// tile's rows (two grid barriers).
 //
-// The predictor's dot products keep the order of the multi-kernel predictor (lane l
-// takes 16-byte chunks l, l+32, ... into one accumulator, then a butterfly sum), so
-// both paths decide every neuron identically.  PDL: the kernel lets the next one
-// launch at once and reads x, and writes anything, only after griddepcontrol.wait.
-// Both grid barriers are bounded: on a timeout the kernel latches SFNN_ERR_TIMEOUT and
-// returns without a result.
+// PDL: the kernel lets the next one launch at once and reads x, and writes anything,
+// only after griddepcontrol.wait.  Every grid barrier is bounded: on a timeout the
+// kernel latches SFNN_ERR_TIMEOUT and returns without a result.
 #include "async.cuh"
 #include "common.cuh"
 #include "decode1.cuh"
@@ -68,6 +72,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   float *h_s = reinterpret_cast<float *>(smem + L.h);
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
+  unsigned long long *target_s = reinterpret_cast<unsigned long long *>(cnt_s + 2);  // split barrier
   unsigned char *bstage = smem + L.bstage;
   unsigned char *dstage = smem + L.dstage;
 
@@ -83,16 +88,20 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const size_t rowB = (size_t)P.d * RB / 8;  // bytes of one stored row
 
   pdl_launch_dependents();
-  const int j0 = c + G * warp;  // this warp's first row of A^T
+  // A^T rows are split in halves over warp pairs: warp w takes half (w & 1) of the rows
+  // j = c + G (w >> 1) + 8 G k, so that a lane's part of its first half row (at most 16
+  // chunks for d <= 8192 fp16) is requested before anything else.
+  const int apair = warp >> 1, ahalf = warp & 1;
+  const int hca = (nch_d + 1) / 2;  // chunks of a row's first half
+  const int abeg = ahalf * hca, aend = ahalf ? nch_d : hca;
+  const int j0 = c + G * apair;  // this warp's first row of A^T
 
   // ---------------------------------------------------------------- A: hidden layer
-  // The first batch of the warp's first row is requested before anything else: phase A
-  // is the critical path into the first grid barrier.
   uint4 w0[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
-    const int ch = lane + 32 * u;
-    if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
+    const int ch = abeg + lane + 32 * u;
+    if (j0 < r && ch < aend) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
   }
   const T *cp = static_cast<const T *>(P.cvec);
   const T *bp = static_cast<const T *>(P.bias);
@@ -106,8 +115,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   // B^T rows of this warp's neurons stream through DB shared-memory stages private to the
   // warp; each lane copies (cp.async) exactly the chunks it will read, so only its own
   // wait is needed.  The first DB rows are requested during phase A, after x and the
-  // warp's row of A^T (the critical path into the first grid barrier), and land while
-  // phase A and the barrier run.
+  // warp's half rows of A^T (the critical path into the first grid barrier), and land
+  // while phase A and the barrier run.
   unsigned char *bst = bstage + (size_t)warp * DB * nch_r * 16;
   auto stage_b = [&](int s, int p) {  // row p of the tile into stage s; always one group
     if (p < tn) {
@@ -128,25 +137,27 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 #pragma unroll
     for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
   }
-  for (int j = j0; j < r; j += G * kW) {
+  // each half row's dot product (chunks ascending in one chain, then a butterfly sum) goes
+  // to hbuf[half][j]; h_j = relu(first half + second half) is formed after the barrier
+  for (int j = j0; j < r; j += G * (kW / 2)) {
     const T *row = At + (size_t)j * d;
-    float acc = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
-    for (int cb = 0; cb < nch_d; cb += 32 * 16) {
-      if (j != j0 || cb != 0) {  // the first batch of the first row is already in w0
+    float acc = 0.f;
+    for (int cb = abeg; cb < aend; cb += 32 * 16) {
+      if (j != j0 || cb != abeg) {  // the first batch of the first row is already in w0
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int ch = cb + lane + 32 * u;
-          if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
+          if (ch < aend) w0[u] = ld_stream(row + (size_t)ch * V);
         }
       }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int ch = cb + lane + 32 * u;
-        if (ch < nch_d) acc = dot_chunk_smem<T>(w0[u], xs, ch, acc);
+        if (ch < aend) acc = dot_chunk_smem<T>(w0[u], xs, ch, acc);
       }
     }
     const float hs = warp_sum(acc);
-    if (lane == 0) P.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
+    if (lane == 0) P.hbuf[(size_t)ahalf * r + j] = hs;
   }
   if (j0 < r) {
 #pragma unroll
@@ -168,9 +179,15 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 
   // ---------------------------------------------------------------- B: logits + threshold
   {
-    // h once per CTA from L2 (every warp needs all of it), then into registers
-    for (int i = tid; i < r / 4; i += kT)
-      reinterpret_cast<float4 *>(h_s)[i] = __ldcg(reinterpret_cast<const float4 *>(P.hbuf) + i);
+    // h = relu(first half + second half) once per CTA from L2 (every warp needs all of
+    // it), then into registers
+    for (int i = tid; i < r / 4; i += kT) {
+      const float4 a = __ldcg(reinterpret_cast<const float4 *>(P.hbuf) + i);
+      const float4 b = __ldcg(reinterpret_cast<const float4 *>(P.hbuf + r) + i);
+      const float4 h4 = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+      reinterpret_cast<float4 *>(h_s)[i] = make_float4(h4.x > 0.f ? h4.x : 0.f, h4.y > 0.f ? h4.y : 0.f,
+                                                       h4.z > 0.f ? h4.z : 0.f, h4.w > 0.f ? h4.w : 0.f);  // NaN -> 0
+    }
     __syncthreads();
     float hreg[MAXH][V];
 #pragma unroll
@@ -243,12 +260,26 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     for (int k = tid; k < cnt; k += kT) P.set_pos[t0 + k] = act_s[k];
     if (tid == 0) P.set_cnt[c] = cnt;
   }
+  // Rebalancing (quota > 0): the busiest tile of a token holds ~1.5x the mean count, and
+  // the CTAs that finish their rows early would leave the HBM stream to it.  So each CTA
+  // keeps the first `quota` of its tile's active rows, publishes its list, and arrives on
+  // a grid barrier whose wait comes after the own rows' up/gate dots; then the rows past
+  // the quota in every tile are shared out evenly over all CTAs, in tile order (a
+  // function of the counts alone: deterministic).
+  const int quota = P.quota;
+  if (quota > 0) {
+    for (int k = tid; k < cnt; k += kT) P.blist[t0 + k] = make_int2(act_s[k], __float_as_int(bias_s[k]));
+    if (tid == 0) P.bcnt[c] = cnt;
+    cta_grid_arrive(P, target_s);  // its CTA barrier orders the list before the release
+  }
+  const int own = quota > 0 ? min(cnt, quota) : cnt;
+  int nrows = own;  // rows of this CTA whose place in act_s is known
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread;
   // the first DD rows are requested right after C1's first loads and land while C1 runs
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
-    if (k < cnt) {
+    if (k < nrows) {
       const unsigned char *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * rowB;
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
@@ -268,20 +299,22 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   };
 
   // ---------------------------------------------------------------- C1: up / gate dots
-  {
-    constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
+  constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
+  constexpr int SU = kSegChunks / 32;             // chunks per lane and segment
+  const int nseg = P.nseg;
+  const int per_row = NPG * nseg;
+  const int nch_r8 = d / VR;  // 16-byte chunks of a row
+  // rows [kb, ke): their segments spread over all warps, 2-deep register pipeline;
+  // `pre` stages of C2 are requested behind the first loads
+  auto c1 = [&](int kb, int ke, int pre) {
     constexpr int D = 2;
-    constexpr int SU = kSegChunks / 32;  // chunks per lane and segment
-    const int nseg = P.nseg;
-    const int per_row = NPG * nseg;
-    const int items = cnt * per_row;
-    const int nch_r8 = d / VR;  // 16-byte chunks of a row
+    const int items = (ke - kb) * per_row;
     uint4 wc[D][SU];
 #pragma unroll
     for (int s = 0; s < D; ++s) {
       const int it = warp + kW * s;
       if (it < items) {
-        const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+        const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
         const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
@@ -290,14 +323,13 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         }
       }
     }
-#pragma unroll
-    for (int s = 0; s < DD; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
+    for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
       for (int s = 0; s < D; ++s) {
         const int it = ib + kW * s;
         if (it < items) {
-          const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+          const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
           float a = 0.f;
 #pragma unroll
           for (int u = 0; u < SU; ++u) {
@@ -313,7 +345,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
           }
           const int itn = it + D * kW;
           if (itn < items) {
-            const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
+            const int kn = kb + itn / per_row, pjn = (itn % per_row) / nseg, sgn = itn % per_row - pjn * nseg;
             const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
@@ -326,26 +358,88 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         }
       }
     }
-    __syncthreads();
-    for (int k = tid; k < cnt; k += kT) {
-      float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
-      for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
-      if (ACT == SFNN_REGLU)
-        for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
-      float sd = 1.f;
-      if (QR) {  // the codes' sums times their rows' scales; the down row's folded into a
-        const float *sc = P.rscale + (size_t)act_s[k] * nproj;
-        g *= sc[0];
-        if (ACT == SFNN_REGLU) u *= sc[1];
-        sd = sc[nproj - 1];
-      }
-      const float pre = g + bias_s[k];
-      const float relu = pre > 0.f ? pre : 0.f;
-      a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
-      if (QR) a_s[k] *= sd;
+  };
+  const int pre = quota > 0 ? min(DD, own) : DD;
+  c1(0, own, pre);
+  int total = own;
+  if (quota > 0) {
+    if (!cta_grid_wait(P, target_s, flag_s)) {
+      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+      return;
+    }
+    // every tile's count; e_t = the rows past the quota; CTA c takes the global excess
+    // rows [floor(cE/G), floor((c+1)E/G)), row g being slot quota + g - epre[t] of the tile
+    // t with epre[t] <= g < epre[t + 1]
+    int *cnt_all = reinterpret_cast<int *>(red2);  // [G], then the prefix [G + 1] and the share
+    int *epre = cnt_all + G;
+    int *ext = epre + G + 1;
+    for (int t = tid; t < G; t += kT) {
+      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
+      cnt_all[t] = min(max(__ldcg(P.bcnt + t), 0), sz);
     }
     __syncthreads();
+    if (warp == 0) {
+      int base = 0;
+      for (int wi = 0; wi < G; wi += 32) {
+        const int t = wi + lane;
+        const int e = t < G ? max(0, cnt_all[t] - quota) : 0;
+        int incl = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (t < G) epre[t] = base + incl - e;
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) {
+        epre[G] = base;
+        const int F = (int)(((int64_t)c * base) / G);
+        ext[0] = (int)(((int64_t)(c + 1) * base) / G) - F;
+        ext[1] = F;
+      }
+    }
+    __syncthreads();
+    const int f = ext[0], F = ext[1];
+    for (int j = tid; j < f; j += kT) {
+      const int g = F + j;
+      int lo = 0, hi = G;  // the largest t with epre[t] <= g
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (epre[mid] <= g)
+          lo = mid;
+        else
+          hi = mid;
+      }
+      const int2 e = __ldcg(P.blist + decode1_tile_start(lo, P.n, G) + quota + (g - epre[lo]));
+      act_s[own + j] = e.x;
+      bias_s[own + j] = __int_as_float(e.y);
+    }
+    __syncthreads();
+    total = own + f;
+    nrows = total;
+    c1(own, total, 0);
   }
+  __syncthreads();
+  for (int k = tid; k < total; k += kT) {
+    float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
+    for (int sg = 0; sg < nseg; ++sg) g += dots[(k * 2 + 0) * nseg + sg];
+    if (ACT == SFNN_REGLU)
+      for (int sg = 0; sg < nseg; ++sg) u += dots[(k * 2 + 1) * nseg + sg];
+    float sd = 1.f;
+    if (QR) {  // the codes' sums times their rows' scales; the down row's folded into a
+      const float *sc = P.rscale + (size_t)act_s[k] * nproj;
+      g *= sc[0];
+      if (ACT == SFNN_REGLU) u *= sc[1];
+      sd = sc[nproj - 1];
+    }
+    const float pre_act = g + bias_s[k];
+    const float relu = pre_act > 0.f ? pre_act : 0.f;
+    a_s[k] = ACT == SFNN_RELU ? relu : relu * u;
+    if (QR) a_s[k] *= sd;
+  }
+  __syncthreads();
+  for (int s = pre; s < DD; ++s) stage_d(s, s);  // C2's first stages not requested yet
 
   // ---------------------------------------------------------------- C2: down projection
   float acc[MAXM][V];
@@ -353,11 +447,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   for (int m = 0; m < MAXM; ++m)
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
-  for (int kb = 0; kb < cnt; kb += DD) {
+  for (int kb = 0; kb < total; kb += DD) {
 #pragma unroll
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
-      if (k < cnt) {
+      if (k < total) {
         cp_async_wait<DD - 1>();  // this thread's chunks of row k have landed
         const float a = a_s[k];
 #pragma unroll
@@ -446,11 +540,9 @@ cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, b
   cfg.blockDim = dim3(kT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = fused_launch_attrs(attr, pdl);
   return cudaLaunchKernelEx(&cfg, k_decode1<T, ACT, MAXM, R>, P);
 }
 

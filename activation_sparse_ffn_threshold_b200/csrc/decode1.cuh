@@ -1,6 +1,7 @@
 // decode1.cuh -- parameters and shared-memory plan of the fused single-token decode kernel.
 #pragma once
 
+#include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -25,7 +26,7 @@ struct Decode1Params {
   float *y;                                  // [d] output
   const float *resid;                        // [d] or null: y = resid + FFN(x)
   void *xnext;                               // [d] or null: round(y) in wdtype
-  float *hbuf;                               // [r] predictor hidden layer (scratch)
+  float *hbuf;                               // [2][r] predictor hidden layer (halves; scratch)
   float *part;                               // [G][d] per-CTA partial sums (scratch)
   uint64_t *bar;                             // grid barrier arrival counter (scratch, zeroed at create)
   int32_t *err;                              // latched device error
@@ -35,6 +36,10 @@ struct Decode1Params {
   int nseg;      // 4 KB segments of one projection row (C1 work items per row and projection)
   int rq;        // rows are 8- or 4-bit codes (0: dt); rscale [n][nproj] their fp32 scales
   const float *rscale;
+  int quota;         // rebalancing of the active rows: own rows kept per CTA, the rest shared out
+                     //   evenly after a split grid barrier (0: every CTA takes its own tile's rows)
+  int2 *blist;       // [n] each tile's active (storage position, bias) pairs, at start(c)
+  int32_t *bcnt;     // [G] their counts
   int hot;           // multi-token kernel: ranks of the hot prefix whose gate/up rows are read before
                      //   the sets are known (0: none); rank k is position k / G of tile k % G
   int32_t *set_pos;  // null, or [n]: tile c's active storage positions at [start(c), start(c) + cnt)
@@ -81,7 +86,7 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) 
   o = decode1_align(o + ((tm + 31) / 32) * 4 + 16, 16);
   L.wpref = o;  // exclusive prefix of the bit words' population counts
   o = decode1_align(o + ((tm + 31) / 32 + 1) * 4, 16);
-  L.bars = o;  // the active count and a flag
+  L.bars = o;  // the active count, a flag, the split barrier's target
   o = decode1_align(o + 16, 16);
   // The two staging areas share one region: B^T rows are staged only in phase B, the
   // W_down chunks only after it (the CTA synchronises in between).
@@ -177,6 +182,17 @@ __host__ __device__ inline MultiLayout decode_multi_layout(const Decode1Params &
   o = decode1_align(o + (bsz > dsz ? bsz : dsz), 16);
   L.total = o;
   return L;
+}
+
+// Launch attributes of the persistent fused kernels: cooperative (the runtime then
+// guarantees that all of a launch's CTAs are resident at once, which its grid barriers
+// rely on) and, when asked, programmatic dependent launch.  Returns the count.
+inline unsigned fused_launch_attrs(cudaLaunchAttribute (&attr)[2], bool pdl) {
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  return pdl ? 2u : 1u;
 }
 
 cudaError_t configure_decode_multi();

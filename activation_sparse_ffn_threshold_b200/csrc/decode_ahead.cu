@@ -25,8 +25,9 @@
 // share (its own tile's rows up to the share, then rows the fuller tiles leave over),
 // which removes the busiest tile's surplus from the critical path at the cost of one
 // dependent load.  The stack's first launch runs the predictor half only (layer 0 on
-// u_0); its last launch has no next predictor.  The predictor's dot products keep the
-// single-layer kernel's orders, so both decide every neuron identically.
+// u_0); its last launch has no next predictor.  Its predictor sums each row of A'^T in
+// one warp (the single-token kernel splits rows over two warps), so the two kernels' sums
+// may differ in rounding.
 #include "async.cuh"
 #include "common.cuh"
 #include "decode1.cuh"
@@ -516,11 +517,9 @@ cudaError_t launch_t(const Decode1Params &P, const AheadParams &Q, size_t smem, 
   cfg.blockDim = dim3(kT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = fused_launch_attrs(attr, pdl);
   return cudaLaunchKernelEx(&cfg, k_decode_ahead<T, ACT, MAXM, R>, P, Q);
 }
 

@@ -526,11 +526,9 @@ cudaError_t launch_t(const Decode1Params &P, size_t smem, cudaStream_t stream, b
   cfg.blockDim = dim3(kT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = fused_launch_attrs(attr, pdl);
   return cudaLaunchKernelEx(&cfg, k_decode_multi<NB, ACT, MAXM>, P);
 }
 

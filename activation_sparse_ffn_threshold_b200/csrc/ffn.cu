@@ -28,8 +28,6 @@ __global__ void __launch_bounds__(kThreads)
     k_up(const T *__restrict__ rows, const T *__restrict__ bias, const T *__restrict__ X,
          const int32_t *__restrict__ ulist, const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
          float *__restrict__ acoef, int d, int b, int nproj) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   constexpr int V = Elem<T>::kVec;
   const int lane = threadIdx.x & 31;
   const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -88,8 +86,6 @@ template <typename T, int TB>
 __global__ void __launch_bounds__(kThreads)
     k_down(const T *__restrict__ rows, const float *__restrict__ acoef, const int32_t *__restrict__ ulist,
            const int32_t *__restrict__ ucount, float *__restrict__ part, int d, int b, int nproj, int splits) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   constexpr int V = Elem<T>::kVec;
   constexpr int SW = 32 * V;  // columns per CTA slice
   extern __shared__ float red[];  // [kWarps][TB][SW]
@@ -141,8 +137,6 @@ __global__ void __launch_bounds__(kThreads)
 template <typename OUT>
 __global__ void k_reduce(const float *__restrict__ part, int splits, int64_t bd, const float *resid, float *Y,
                          OUT *__restrict__ xnext) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= bd) return;
   float s = 0.f;
@@ -165,9 +159,13 @@ cudaError_t up_act(const sfnn_ctx *h, const void *X, int b, cudaStream_t s) {
   const T *rows = static_cast<const T *>(h->rows);
   const T *bias = static_cast<const T *>(h->bias);
   const T *Xp = static_cast<const T *>(X);
-  return launch_pdl(b == 1 ? k_up<T, ACT, 1> : k_up<T, ACT, 8>, dim3(grid), dim3(kThreads), 0, s, rows, bias, Xp,
-                    static_cast<const int32_t *>(h->ulist), static_cast<const uint32_t *>(h->utok),
-                    static_cast<const int32_t *>(h->ucount), h->acoef, L.d, b, L.nproj);
+  if (b == 1)
+    k_up<T, ACT, 1><<<grid, kThreads, 0, s>>>(rows, bias, Xp, h->ulist, h->utok, h->ucount, h->acoef, L.d, b,
+                                               L.nproj);
+  else
+    k_up<T, ACT, 8><<<grid, kThreads, 0, s>>>(rows, bias, Xp, h->ulist, h->utok, h->ucount, h->acoef, L.d, b,
+                                               L.nproj);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -184,10 +182,10 @@ cudaError_t down_tb(const sfnn_ctx *h, int b, int *splits_out, cudaStream_t s) {
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
   const size_t smem = (size_t)kWarps * TB * SW * sizeof(float);
   auto kern = k_down<T, TB>;
+  kern<<<dim3(ds, splits), kThreads, smem, s>>>(static_cast<const T *>(h->rows), h->acoef, h->ulist, h->ucount,
+                                                h->part, L.d, b, L.nproj, splits);
   *splits_out = splits;
-  return launch_pdl(kern, dim3(ds, splits), dim3(kThreads), smem, s, static_cast<const T *>(h->rows),
-                    static_cast<const float *>(h->acoef), static_cast<const int32_t *>(h->ulist),
-                    static_cast<const int32_t *>(h->ucount), h->part, L.d, b, L.nproj, splits);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -225,10 +223,10 @@ cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *res
   const int64_t bd = (int64_t)b * h->L.d;
   const int grid = (int)((bd + 255) / 256);
   if (h->L.dt == SFNN_F16)
-    return launch_pdl(k_reduce<__half>, dim3(grid), dim3(256), 0, s, static_cast<const float *>(h->part), splits, bd,
-                      resid, Y, static_cast<__half *>(xnext));
-  return launch_pdl(k_reduce<float>, dim3(grid), dim3(256), 0, s, static_cast<const float *>(h->part), splits, bd, resid,
-                    Y, static_cast<float *>(xnext));
+    k_reduce<__half><<<grid, 256, 0, s>>>(h->part, splits, bd, resid, Y, static_cast<__half *>(xnext));
+  else
+    k_reduce<float><<<grid, 256, 0, s>>>(h->part, splits, bd, resid, Y, static_cast<float *>(xnext));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s) {

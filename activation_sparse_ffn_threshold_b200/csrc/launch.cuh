@@ -2,29 +2,9 @@
 // size limits the host checks when a layer is created.
 #pragma once
 
-#include "async.cuh"
 #include "common.cuh"
 
 namespace sfnn {
-
-// Launch with programmatic dependent launch: the kernel may start while the previous one
-// in the stream finishes, so every kernel launched this way calls pdl_wait() before it
-// touches memory that earlier kernels write or read (and pdl_launch_dependents() first,
-// to let the next one start early in turn).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
 
 constexpr int kMaxNeurons = 1 << 20;                  // n: the union's per-word offsets live in shared memory
 constexpr int kUnionSmemMax = (kMaxNeurons / 32) * 4;  // bytes of those offsets at the largest n

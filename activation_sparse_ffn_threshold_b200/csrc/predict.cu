@@ -27,8 +27,6 @@ constexpr int kWarps = kThreads / 32;
 template <typename T, int TB>
 __global__ void __launch_bounds__(kThreads) k_hidden(const T *__restrict__ At, const T *__restrict__ X,
                                                      float *__restrict__ H, int r, int d, int b) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   constexpr int V = Elem<T>::kVec;
   constexpr int U = 4;
   const int lane = threadIdx.x & 31;
@@ -80,8 +78,6 @@ template <typename T, int TB>
 __global__ void __launch_bounds__(kThreads) k_logits(const T *__restrict__ Bt, const T *__restrict__ cvec,
                                                      const float *__restrict__ H, uint32_t *__restrict__ mask,
                                                      int n, int r, int b, int nwords) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   constexpr int V = Elem<T>::kVec;
   extern __shared__ float hs[];  // [b][r]
   __shared__ uint32_t bits_s[TB];
@@ -145,8 +141,6 @@ __global__ void __launch_bounds__(1024) k_mask_from_idx(const int32_t *__restric
                                                         const int32_t *__restrict__ iperm,
                                                         uint32_t *__restrict__ mask, int n, int nwords,
                                                         int32_t *err) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   for (int w = threadIdx.x; w < nwords; w += blockDim.x) mask[w] = 0u;
   __syncthreads();
   int k = *count;
@@ -226,8 +220,6 @@ constexpr int kUnionStage = 32 * 33;  // words of one warp's staged masks (rows 
 __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
                                                          int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
                                                          int32_t *__restrict__ ucount) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   uint32_t *stage = reinterpret_cast<uint32_t *>(woff + ((nwords + 3) & ~3)) + warp * kUnionStage;
@@ -288,8 +280,6 @@ __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restr
 __global__ void __launch_bounds__(1024) k_compact(const uint32_t *__restrict__ mask, int nwords, int n,
                                                   const int32_t *__restrict__ perm, int32_t *__restrict__ idx_out,
                                                   int32_t *__restrict__ cnt_out) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   const int t = blockIdx.x;
   const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
   const int w0 = threadIdx.x * wpt;
@@ -349,8 +339,11 @@ cudaError_t hidden_impl(const sfnn_ctx *h, const void *X, int b, cudaStream_t s)
   const int grid = (L.r + kWarps - 1) / kWarps;
   const T *At = static_cast<const T *>(h->At);
   const T *Xp = static_cast<const T *>(X);
-  return launch_pdl(b == 1 ? k_hidden<T, 1> : k_hidden<T, 8>, dim3(grid), dim3(kThreads), 0, s, At, Xp, h->h, L.r,
-                    L.d, b);
+  if (b == 1)
+    k_hidden<T, 1><<<grid, kThreads, 0, s>>>(At, Xp, h->h, L.r, L.d, b);
+  else
+    k_hidden<T, 8><<<grid, kThreads, 0, s>>>(At, Xp, h->h, L.r, L.d, b);
+  return cudaGetLastError();
 }
 
 constexpr int kLogitsSmemMax = 32768 * sizeof(float);  // r * max_batch <= 32768 (checked at create)
@@ -360,9 +353,9 @@ cudaError_t logits_tb(const sfnn_ctx *h, int b, cudaStream_t s) {
   const Layout &L = h->L;
   const size_t smem = (size_t)b * L.r * sizeof(float);
   auto kern = k_logits<T, TB>;
-  return launch_pdl(kern, dim3(L.nwords), dim3(kThreads), smem, s, static_cast<const T *>(h->Bt),
-                    static_cast<const T *>(h->cvec), static_cast<const float *>(h->h), h->mask, L.n, L.r, b,
-                    L.nwords);
+  kern<<<L.nwords, kThreads, smem, s>>>(static_cast<const T *>(h->Bt), static_cast<const T *>(h->cvec), h->h,
+                                        h->mask, L.n, L.r, b, L.nwords);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -397,8 +390,8 @@ cudaError_t launch_logits(const sfnn_ctx *h, int b, cudaStream_t s) {
 }
 
 cudaError_t launch_mask_from_idx(const sfnn_ctx *h, const int32_t *idx, const int32_t *count, cudaStream_t s) {
-  return launch_pdl(k_mask_from_idx, dim3(1), dim3(1024), 0, s, idx, count, static_cast<const int32_t *>(h->iperm),
-                    h->mask, h->L.n, h->L.nwords, h->err);
+  k_mask_from_idx<<<1, 1024, 0, s>>>(idx, count, h->iperm, h->mask, h->L.n, h->L.nwords, h->err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *idx_out, int32_t *cnt_out,
@@ -407,12 +400,12 @@ cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *i
   cudaError_t e = cudaSuccess;
   if (want_union) {
     const size_t smem = ((size_t)(L.nwords + 3) / 4 * 4 + (size_t)(kUnionThreads / 32) * kUnionStage) * 4;
-    e = launch_pdl(k_union, dim3(1), dim3(kUnionThreads), smem, s, static_cast<const uint32_t *>(h->mask), L.nwords,
-                   L.n, b, h->ulist, h->utok, h->ucount);
+    k_union<<<1, kUnionThreads, smem, s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
+    e = cudaGetLastError();
   }
   if (e == cudaSuccess && (idx_out || cnt_out)) {
-    e = launch_pdl(k_compact, dim3(b), dim3(1024), 0, s, static_cast<const uint32_t *>(h->mask), L.nwords, L.n,
-                   static_cast<const int32_t *>(h->perm), idx_out, cnt_out);
+    k_compact<<<b, 1024, 0, s>>>(h->mask, L.nwords, L.n, h->perm, idx_out, cnt_out);
+    e = cudaGetLastError();
   }
   return e;
 }

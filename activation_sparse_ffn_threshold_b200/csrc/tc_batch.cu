@@ -195,8 +195,6 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
                                                const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
                                                __half *__restrict__ H, int hstride, int d, int b, int N, int nproj,
                                                int stages, int32_t *err) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
@@ -282,8 +280,6 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
                                                  int hstride, const int32_t *__restrict__ ulist,
                                                  const int32_t *__restrict__ ucount, float *__restrict__ part, int d,
                                                  int b, int N, int nproj, int splits, int stages, int32_t *err) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -354,8 +350,6 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
 __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At, const __half *__restrict__ X,
                                                    float *__restrict__ hp, int d, int r, int b, int N, int splits,
                                                    int stages, int32_t *err) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -413,8 +407,6 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
 
 __global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N, int r, __half *__restrict__ hhi,
                           __half *__restrict__ hlo) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;  // t * r + j over N tokens
   if (i >= N * r) return;
   const int t = i / r;
@@ -434,8 +426,6 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
                                                    const __half *__restrict__ hhi, const __half *__restrict__ hlo,
                                                    uint32_t *__restrict__ mask, int n, int r, int nwords, int b, int N,
                                                    int stages, int32_t *err) {
-  pdl_launch_dependents();  // launched with programmatic dependent launch
-  pdl_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -533,16 +523,20 @@ cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStrea
   splits = std::min(splits, L.d / kTK);
   splits = std::min<int>(splits, (int)(cap / ((size_t)b * L.r)));
   splits = splits < 1 ? 1 : splits;
-  cudaError_t e = launch_pdl(k_tc_hidden, dim3(rtiles, splits), dim3(kTT), hidden_smem(N), s,
-                             static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r, b,
-                             N, splits, kPredStages, h->err);
+  k_tc_hidden<<<dim3(rtiles, splits), kTT, hidden_smem(N), s>>>(
+      static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r, b, N, splits,
+      kPredStages, h->err);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   __half *hhi = h->hpair, *hlo = h->hpair + (size_t)32 * L.r;
-  e = launch_pdl(k_tc_hsum, dim3((N * L.r + 255) / 256), dim3(256), 0, s, h->part, splits, b, N, L.r, hhi, hlo);
+  k_tc_hsum<<<(N * L.r + 255) / 256, 256, 0, s>>>(h->part, splits, b, N, L.r, hhi, hlo);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_tc_logits, dim3((L.n + kTM - 1) / kTM), dim3(kTT), logits_smem(N), s,
-                    static_cast<const __half *>(h->Bt), static_cast<const __half *>(h->cvec), hhi, hlo, h->mask, L.n,
-                    L.r, L.nwords, b, N, kPredStages, h->err);
+  k_tc_logits<<<(L.n + kTM - 1) / kTM, kTT, logits_smem(N), s>>>(static_cast<const __half *>(h->Bt),
+                                                                  static_cast<const __half *>(h->cvec), hhi, hlo,
+                                                                  h->mask, L.n, L.r, L.nwords, b, N, kPredStages,
+                                                                  h->err);
+  return cudaGetLastError();
 }
 
 // Up / gate of the union rows for all b tokens -> h->hact; then the down projection into
@@ -553,20 +547,25 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int hs = tc_hstride(L.n);
   const __half *rows = static_cast<const __half *>(h->rows);
   const int up_grid = (L.n + kTM - 1) / kTM;
-  cudaError_t e = launch_pdl(L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU> : k_tc_up<SFNN_RELU>, dim3(up_grid), dim3(kTT),
-                             up_smem(L.act, N), s, rows, static_cast<const __half *>(h->bias),
-                             static_cast<const __half *>(X), h->ulist, h->utok, h->ucount, h->hact, hs, L.d, b, N,
-                             L.nproj, kUpStages, h->err);
+  if (L.act == SFNN_REGLU)
+    k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+  else
+    k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int mtiles = L.d / kTM;
   // one wave: three CTAs fit on an SM (3 stages of 20 KB); the output tiles times the
   // splits of the union fill them without a tail
   int splits = (3 * h->num_sms) / mtiles;
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
+  k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part, L.d, b, N,
+                                                            L.nproj, splits, kDownStages, h->err);
   *splits_out = splits;
-  return launch_pdl(k_tc_down, dim3(mtiles, splits), dim3(kTT), down_smem(N), s, rows,
-                    static_cast<const __half *>(h->hact), hs, h->ulist, h->ucount, h->part, L.d, b, N, L.nproj,
-                    splits, kDownStages, h->err);
+  return cudaGetLastError();
 }
 
 }  // namespace sfnn

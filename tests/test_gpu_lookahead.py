@@ -81,7 +81,10 @@ def test_lookahead_stack_matches_oracle(base):
     # predicted one layer early: some layer's set differs from the plain stack's
     _, sidx, scnt = sf.forward_stack(hs, torch.from_numpy(x0).cuda(), return_sets=True)
     plain = [mask_from_idx(sidx[l, 0].cpu().numpy(), scnt[l, 0].item(), cfg.n) for l in range(4)]
-    assert np.array_equal(masks[0], plain[0])  # layer 0 predicts from its own input either way
+    # layer 0 predicts from its own input either way (the two kernels sum the predictor in
+    # different orders: they may part only within the arbitration band)
+    _, z0, _ = oracle.predictor(x0.astype(cfg.np_dtype), layers[0].A, layers[0].B, layers[0].c, NTHREADS)
+    assert oracle.arbitrate(z0, masks[0], plain[0])[1].size == 0
     assert any(not np.array_equal(masks[l], plain[l]) for l in range(1, 4))
 
 
