@@ -137,6 +137,7 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
     P.set_pos = sets ? reinterpret_cast<int32_t *>(h->acoef) : nullptr;
     P.set_cnt = sets ? h->scnt : nullptr;
     P.hot = h->hot_on ? h->hot_rows[b] : 0;
+    P.quota = h->quota_multi[b];
     SFNN_TRY(launch_decode_multi(P, b, s, true));
     record_if(after, s);
     if (sets)
@@ -207,6 +208,8 @@ void plan_decode1(sfnn_ctx *h, int G) {
   // the rebalancing's scratch (counts, their prefix, the share) lives in the CTA's
   // 512-word reduce buffer
   P.quota = 2 * G + 3 <= kDecode1Threads ? std::min(h->quota, P.tile_max) : 0;
+  for (int b = 0; b <= kMultiMaxTokens; ++b)  // the prefix must stay with its tile: else no rebalancing
+    if (2 * G + 3 > kDecode1Threads || h->quota_multi[b] > P.tile_max) h->quota_multi[b] = 0;
   if (L.r / L.vec > 32 * 4) return;
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
@@ -369,6 +372,20 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
     }
     h->hot_rows[b] = k;
   }
+  // The multi-token kernel's quota for b tokens: 0.8 of a tile's expected union count,
+  // and at least the tile's hot prefix (whose dots only the tile's own CTA holds).
+  for (int b = 0; b <= kMultiMaxTokens; ++b) {
+    h->quota_multi[b] = 0;
+    if (!desc->hotness || b < 2) continue;
+    double u = 0.0;
+    for (int i = 0; i < L.n; ++i) {
+      const float q = desc->hotness[i];
+      const double p = std::isnan(q) ? 0.0 : std::min(1.0, std::max(0.0, (double)q));
+      u += 1.0 - std::pow(1.0 - p, b);
+    }
+    const int qv = std::max((int)std::floor(0.8 * u / G), (h->hot_rows[b] + G - 1) / G);
+    h->quota_multi[b] = qv >= 2 ? qv : 0;
+  }
   if (desc->hotness) {
     for (int b = 1; b <= kMaxBatch; ++b) {
       double u = 0.0;
@@ -394,7 +411,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {&h->bias, n * e, true},
       {(void **)&h->perm, n * 4, true},
       {(void **)&h->iperm, n * 4, true},
-      {(void **)&h->h, std::max<size_t>(mb, 2) * r * 4, false},
+      {(void **)&h->h, 2 * mb * r * 4, false},  // [2][r] halves (fused kernels) or [mb][r]
       {(void **)&h->mask, mb * L.nwords * 4, false},
       {(void **)&h->ulist, n * 4, false},
       {(void **)&h->utok, n * 4, false},

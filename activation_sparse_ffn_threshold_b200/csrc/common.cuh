@@ -40,7 +40,7 @@ struct sfnn_ctx {
   int32_t *perm;   // [n] internal -> original
   int32_t *iperm;  // [n] original -> internal
   // scratch
-  float *h;          // [max_batch][r]
+  float *h;          // [2 * max_batch][r]: the hidden layer (fused kernels: per token two half sums)
   uint32_t *mask;    // [max_batch][nwords]
   int32_t *ulist;    // [n] union list (internal positions, ascending)
   uint32_t *utok;    // [n] tokens active on each union row (bit t)
@@ -58,6 +58,7 @@ struct sfnn_ctx {
   int2 *blist;       // [n] rebalancing: each tile's active (storage position, bias) pairs
   int32_t *bcnt;     // [G]   and their counts (single-token fused kernel)
   int quota;         // its per-CTA quota of own rows (0: no rebalancing)
+  int quota_multi[sfnn::kMultiMaxTokens + 1];  // the same for the multi-token kernel, by batch size
   int32_t *scnt;     // [max_batch][G] per-tile counts of the sets a fused launch used (lists: ulist
                      //   for one token, acoef's words for several)
   int multi_max;     // largest batch the multi-token fused kernel serves (0: none)

@@ -367,55 +367,10 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       cp_async_wait<0>();  // no copy into shared memory outlives the CTA
       return;
     }
-    // every tile's count; e_t = the rows past the quota; CTA c takes the global excess
-    // rows [floor(cE/G), floor((c+1)E/G)), row g being slot quota + g - epre[t] of the tile
-    // t with epre[t] <= g < epre[t + 1]
-    int *cnt_all = reinterpret_cast<int *>(red2);  // [G], then the prefix [G + 1] and the share
-    int *epre = cnt_all + G;
-    int *ext = epre + G + 1;
-    for (int t = tid; t < G; t += kT) {
-      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
-      cnt_all[t] = min(max(__ldcg(P.bcnt + t), 0), sz);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int base = 0;
-      for (int wi = 0; wi < G; wi += 32) {
-        const int t = wi + lane;
-        const int e = t < G ? max(0, cnt_all[t] - quota) : 0;
-        int incl = e;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        if (t < G) epre[t] = base + incl - e;
-        base += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (lane == 0) {
-        epre[G] = base;
-        const int F = (int)(((int64_t)c * base) / G);
-        ext[0] = (int)(((int64_t)(c + 1) * base) / G) - F;
-        ext[1] = F;
-      }
-    }
-    __syncthreads();
-    const int f = ext[0], F = ext[1];
-    for (int j = tid; j < f; j += kT) {
-      const int g = F + j;
-      int lo = 0, hi = G;  // the largest t with epre[t] <= g
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (epre[mid] <= g)
-          lo = mid;
-        else
-          hi = mid;
-      }
-      const int2 e = __ldcg(P.blist + decode1_tile_start(lo, P.n, G) + quota + (g - epre[lo]));
+    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
       act_s[own + j] = e.x;
       bias_s[own + j] = __int_as_float(e.y);
-    }
-    __syncthreads();
+    });
     total = own + f;
     nrows = total;
     c1(own, total, 0);

@@ -126,5 +126,61 @@ __device__ __forceinline__ bool cta_grid_wait(const Decode1Params &P, const unsi
   return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
+// Rebalancing of a fused kernel's active rows, after the split barrier's wait: every
+// tile's count (P.bcnt, clamped to the tile), e_t = the rows past `quota`, and CTA c's
+// even share of them, the global excess rows [floor(cE/G), floor((c+1)E/G)) in tile
+// order -- row g is slot quota + g - epre[t] of the tile t with epre[t] <= g < epre[t+1].
+// `scratch` holds 2G + 3 ints of shared memory.  take(j, entry) receives the CTA's j-th
+// extra row's list entry (P.blist); returns the CTA's count of extra rows.  A function of
+// the counts alone: every CTA computes the same assignment.
+template <class Take>
+__device__ __forceinline__ int share_excess(const Decode1Params &P, int quota, int *scratch, Take take) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = P.G, c = blockIdx.x;
+  int *cnt_all = scratch, *epre = scratch + G, *ext = epre + G + 1;
+  for (int t = tid; t < G; t += blockDim.x) {
+    const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
+    cnt_all[t] = min(max(__ldcg(P.bcnt + t), 0), sz);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int wi = 0; wi < G; wi += 32) {
+      const int t = wi + lane;
+      const int e = t < G ? max(0, cnt_all[t] - quota) : 0;
+      int incl = e;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (t < G) epre[t] = base + incl - e;
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      epre[G] = base;
+      const int F = (int)(((int64_t)c * base) / G);
+      ext[0] = (int)(((int64_t)(c + 1) * base) / G) - F;
+      ext[1] = F;
+    }
+  }
+  __syncthreads();
+  const int f = ext[0], F = ext[1];
+  for (int j = tid; j < f; j += blockDim.x) {
+    const int g = F + j;
+    int lo = 0, hi = G;  // the largest t with epre[t] <= g
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (epre[mid] <= g)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    take(j, __ldcg(P.blist + decode1_tile_start(lo, P.n, G) + quota + (g - epre[lo])));
+  }
+  __syncthreads();
+  return f;
+}
+
 }  // namespace
 }  // namespace sfnn

@@ -7,8 +7,9 @@
 // tile of neurons (hotness ranks dealt round-robin to the tiles, hottest first inside
 // each), two bounded grid barriers -- with every weight read once for all NB tokens:
 //
-//   A   h_t = relu(A^T x_t) for the NB tokens: one warp per predictor row, the row read
-//       once and multiplied by the NB inputs held in shared memory.  Grid barrier.
+//   A   h_t = relu(A^T x_t) for the NB tokens: each predictor row split in halves over a
+//       warp pair, read once and multiplied by the NB inputs held in shared memory.  Grid
+//       barrier (split: the hot prefix below runs between its arrival and its wait).
 //   B   z_t = B^T h_t + c for the tile: each neuron's B^T row is split in two halves
 //       over a pair of warps (so that each lane holds the NB hidden layers' values for
 //       2 chunks in registers), half rows streaming through 6 shared-memory stages per
@@ -99,14 +100,19 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   const int words = (tn + 31) / 32;
 
   pdl_launch_dependents();
-  const int j0 = c + G * warp;  // this warp's first row of A^T
+  // A^T rows split in halves over warp pairs (as in the single-token kernel): a lane's
+  // whole share of its first half row is requested before the wait for the previous kernel
+  const int apair = warp >> 1, ahalf = warp & 1;
+  const int hca = (nch_d + 1) / 2;
+  const int abeg = ahalf * hca, aend = ahalf ? nch_d : hca;
+  const int j0 = c + G * apair;  // this warp's first row of A^T
 
   // ---------------------------------------------------------------- A: hidden layers
   uint4 w0[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
-    const int ch = lane + 32 * u;
-    if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
+    const int ch = abeg + lane + 32 * u;
+    if (j0 < r && ch < aend) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
   }
   const __half *cp = static_cast<const __half *>(P.cvec);
   const __half *bp = static_cast<const __half *>(P.bias);
@@ -142,29 +148,30 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
 #pragma unroll
     for (int s = 0; s < kMB; ++s) stage_b(s, pair + kPairs * s);
   }
-  for (int j = j0; j < r; j += G * kW) {
+  // each token's half-row sums go to hbuf[t][half][j]; h is formed after the barrier
+  for (int j = j0; j < r; j += G * (kW / 2)) {
     const __half *row = At + (size_t)j * d;
     float2 acc[NB];
 #pragma unroll
     for (int t = 0; t < NB; ++t) acc[t] = make_float2(0.f, 0.f);
-    for (int cb = 0; cb < nch_d; cb += 32 * 16) {
-      if (j != j0 || cb != 0) {
+    for (int cb = abeg; cb < aend; cb += 32 * 16) {
+      if (j != j0 || cb != abeg) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int ch = cb + lane + 32 * u;
-          if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
+          if (ch < aend) w0[u] = ld_stream(row + (size_t)ch * V);
         }
       }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int ch = cb + lane + 32 * u;
-        if (ch < nch_d) dot_tokens<NB>(w0[u], xs, xstride, ch, ALL, acc);
+        if (ch < aend) dot_tokens<NB>(w0[u], xs, xstride, ch, ALL, acc);
       }
     }
 #pragma unroll
     for (int t = 0; t < NB; ++t) {
       const float hs = warp_sum(acc[t].x + acc[t].y);
-      if (lane == 0) P.hbuf[(size_t)t * r + j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
+      if (lane == 0) P.hbuf[((size_t)t * 2 + ahalf) * r + j] = hs;
     }
   }
   if (j0 < r) {
@@ -219,8 +226,14 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
 
   // ---------------------------------------------------------------- B: logits + threshold
   {
-    for (int i = tid; i < NB * r / 4; i += kT)
-      reinterpret_cast<float4 *>(h_s)[i] = __ldcg(reinterpret_cast<const float4 *>(P.hbuf) + i);
+    for (int i = tid; i < NB * r / 4; i += kT) {  // h_t = relu(first half + second half); NaN -> 0
+      const int t = i / (r / 4), q = i - t * (r / 4);
+      const float4 a = __ldcg(reinterpret_cast<const float4 *>(P.hbuf + (size_t)t * 2 * r) + q);
+      const float4 b = __ldcg(reinterpret_cast<const float4 *>(P.hbuf + ((size_t)t * 2 + 1) * r) + q);
+      const float4 h4 = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+      reinterpret_cast<float4 *>(h_s)[i] = make_float4(h4.x > 0.f ? h4.x : 0.f, h4.y > 0.f ? h4.y : 0.f,
+                                                       h4.z > 0.f ? h4.z : 0.f, h4.w > 0.f ? h4.w : 0.f);
+    }
     __syncthreads();
     float2 hreg[NB][MH][4];
 #pragma unroll
@@ -338,10 +351,23 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   }
   const int kp = __syncthreads_count(tid < hp && ((ubits[tid >> 5] >> (tid & 31)) & 1u));  // union rows in the prefix
   const int cnt = *cnt_s;
+  // Rebalancing, as in the single-token kernel: each CTA keeps its first `quota` union rows
+  // (at least its hot prefix, whose dots only it holds), publishes its list (position |
+  // token mask << 24, b) and arrives on a split grid barrier; after its own rows' dots it
+  // takes an even share of all tiles' rows past the quota.
+  const int quota = P.quota;
+  if (quota > 0) {
+    for (int k = tid; k < cnt; k += kT)
+      P.blist[t0 + k] = make_int2(act_s[k] | (int)(tok_s[k] << 24), __float_as_int(bias_s[k]));
+    if (tid == 0) P.bcnt[c] = cnt;
+    cta_grid_arrive(P, target_s);
+  }
+  const int own = quota > 0 ? min(cnt, quota) : cnt;
+  int nrows = own;  // union rows of this CTA whose place in act_s is known
 
   auto dslot = [&](int s, int m) { return stage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // union row k's down row into stage s; always one group
-    if (k < cnt) {
+    if (k < nrows) {
       const unsigned char *row = rows + ((size_t)act_s[k] * nproj + (nproj - 1)) * rowB;
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
@@ -353,15 +379,18 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   };
 
   // ---------------------------------------------------------------- C1: gate / up dots
-  {
+  // rows [kb, ke) (after the prefix), their segments over all warps, 2-deep register
+  // pipeline, dots only for the tokens active on each row; `pre` stages of C2 requested
+  // behind the first loads
+  auto c1 = [&](int kb, int ke, int pre) {
     constexpr int D = 2;
-    const int items = (cnt - kp) * per_row;  // the union rows after the prefix
+    const int items = (ke - kb) * per_row;
     uint4 wc[D][SU];
 #pragma unroll
     for (int s = 0; s < D; ++s) {
       const int it = warp + kW * s;
       if (it < items) {
-        const int k = kp + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+        const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
         const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
@@ -370,14 +399,13 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
         }
       }
     }
-#pragma unroll
-    for (int s = 0; s < DD; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
+    for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
       for (int s = 0; s < D; ++s) {
         const int it = ib + kW * s;
         if (it < items) {
-          const int k = kp + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+          const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
           const uint32_t tm = tok_s[k];
           float2 acc[NB];
 #pragma unroll
@@ -389,7 +417,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
           }
           const int itn = it + D * kW;
           if (itn < items) {
-            const int kn = kp + itn / per_row, pjn = (itn % per_row) / nseg, sgn = itn % per_row - pjn * nseg;
+            const int kn = kb + itn / per_row, pjn = (itn % per_row) / nseg, sgn = itn % per_row - pjn * nseg;
             const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
@@ -407,25 +435,43 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
         }
       }
     }
-    __syncthreads();
-    for (int e = tid; e < cnt * NB; e += kT) {
-      const int k = e / NB, t = e - k * NB;
-      float a = 0.f;
-      if ((tok_s[k] >> t) & 1u) {
-        // the prefix's dots by tile position, the others' by union row
-        const float *dk = k < kp ? pdots + (size_t)(act_s[k] - t0) * 2 * nseg * NB : dots + (size_t)k * 2 * nseg * NB;
-        float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
-        for (int sg = 0; sg < nseg; ++sg) g += dk[(size_t)sg * NB + t];
-        if (ACT == SFNN_REGLU)
-          for (int sg = 0; sg < nseg; ++sg) u += dk[((size_t)nseg + sg) * NB + t];
-        const float pre = g + bias_s[k];
-        const float relu = pre > 0.f ? pre : 0.f;
-        a = ACT == SFNN_RELU ? relu : relu * u;
-      }
-      a_s[e] = a;
+  };
+  const int pre = quota > 0 ? min(DD, own) : DD;
+  c1(kp, own, pre);
+  int total = own;
+  if (quota > 0) {
+    if (!cta_grid_wait(P, target_s, flag_s)) {
+      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+      return;
     }
-    __syncthreads();
+    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
+      act_s[own + j] = e.x & 0xFFFFFF;
+      tok_s[own + j] = (uint32_t)e.x >> 24;
+      bias_s[own + j] = __int_as_float(e.y);
+    });
+    total = own + f;
+    nrows = total;
+    c1(own, total, 0);
   }
+  __syncthreads();
+  for (int e = tid; e < total * NB; e += kT) {
+    const int k = e / NB, t = e - k * NB;
+    float a = 0.f;
+    if ((tok_s[k] >> t) & 1u) {
+      // the prefix's dots by tile position, the others' by union row
+      const float *dk = k < kp ? pdots + (size_t)(act_s[k] - t0) * 2 * nseg * NB : dots + (size_t)k * 2 * nseg * NB;
+      float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
+      for (int sg = 0; sg < nseg; ++sg) g += dk[(size_t)sg * NB + t];
+      if (ACT == SFNN_REGLU)
+        for (int sg = 0; sg < nseg; ++sg) u += dk[((size_t)nseg + sg) * NB + t];
+      const float pre_act = g + bias_s[k];
+      const float relu = pre_act > 0.f ? pre_act : 0.f;
+      a = ACT == SFNN_RELU ? relu : relu * u;
+    }
+    a_s[e] = a;
+  }
+  __syncthreads();
+  for (int s = pre; s < DD; ++s) stage_d(s, s);  // C2's first stages not requested yet
 
   // ---------------------------------------------------------------- C2: down projection
   float2 acc[MAXM][4][NB];
@@ -435,11 +481,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int t = 0; t < NB; ++t) acc[m][i][t] = make_float2(0.f, 0.f);
-  for (int kb = 0; kb < cnt; kb += DD) {
+  for (int kb = 0; kb < total; kb += DD) {
 #pragma unroll
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
-      if (k < cnt) {
+      if (k < total) {
         cp_async_wait<DD - 1>();  // this thread's chunks of row k have landed
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
