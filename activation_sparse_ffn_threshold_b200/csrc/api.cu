@@ -176,6 +176,11 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
   return SFNN_OK;
 }
 
+// The few-token kernel's rebalancing of union rows over the CTAs: measured slower than
+// each CTA taking its own tile's union rows (70B-shaped layer, 2 tokens: 98.5 against
+// 92.6 us per batch), so it is off.
+constexpr bool kMultiRebalance = false;
+
 // The fused single-token kernel's plan: one CTA per SM, each owning a contiguous tile of
 // neurons; h is held in registers (at most 4 chunks per lane), all CTAs must be resident.
 void plan_decode1(sfnn_ctx *h, int G) {
@@ -384,7 +389,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       u += 1.0 - std::pow(1.0 - p, b);
     }
     const int qv = std::max((int)std::floor(0.8 * u / G), (h->hot_rows[b] + G - 1) / G);
-    h->quota_multi[b] = qv >= 2 ? qv : 0;
+    h->quota_multi[b] = kMultiRebalance && qv >= 2 ? qv : 0;
   }
   if (desc->hotness) {
     for (int b = 1; b <= kMaxBatch; ++b) {

@@ -445,45 +445,17 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     }
   }
   if (!cta_grid_sync(P, flag_s)) return;
-  const int CW = (d + G - 1) / G;
-  const int col0 = c * CW;
-  const int ncol = max(0, min(CW, d - col0));
-  for (int cb = 0; cb < ncol; cb += kT) {
-    const int width = min(kT, ncol - cb);
-    const int gi = tid / width, j = tid % width;
-    const int ngu = kT / width;  // groups of partials summed in parallel
-    if (gi < ngu) {
-      const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
-      const float *src = P.part + col0 + cb + j;
-      float sum = 0.f;  // in ascending k; the first 24 loads issued at once, then 8 at a time
-      float v0[24];
+  // the stage region is free again: C2's copies have all landed
+  column_sums<1, 1>(P.part, d, G, reinterpret_cast<float4 *>(dstage), [&](int, int col, float4 v) {
+    const float t4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int u = 0; u < 24; ++u) v0[u] = k0 + u < k1 ? __ldcg(src + (size_t)(k0 + u) * d) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 24; ++u)
-        if (k0 + u < k1) sum += v0[u];
-      int k = k0 + 24;
-      for (; k + 8 <= k1; k += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(k + u) * d);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) sum += v[u];
-      }
-      for (; k < k1; ++k) sum += __ldcg(src + (size_t)k * d);
-      red2[gi * width + j] = sum;
+    for (int i = 0; i < 4; ++i) {
+      float tot = t4[i];
+      if (P.resid) tot = P.resid[col + i] + tot;
+      P.y[col + i] = tot;
+      if (P.xnext) static_cast<T *>(P.xnext)[col + i] = from_f<T>(tot);
     }
-    __syncthreads();
-    if (tid < width) {
-      float tot = 0.f;
-      for (int g = 0; g < ngu; ++g) tot += red2[g * width + tid];
-      const int col = col0 + cb + tid;
-      if (P.resid) tot = P.resid[col] + tot;
-      P.y[col] = tot;
-      if (P.xnext) static_cast<T *>(P.xnext)[col] = from_f<T>(tot);
-    }
-    __syncthreads();
-  }
+  });
 }
 
 __global__ void k_barrier_bump(uint64_t *count) { atomicAdd(reinterpret_cast<unsigned long long *>(count), 1ull); }

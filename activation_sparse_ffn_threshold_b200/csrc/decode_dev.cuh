@@ -126,6 +126,66 @@ __device__ __forceinline__ bool cta_grid_wait(const Decode1Params &P, const unsi
   return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
+// The fused kernels' final sums.  CTA c owns the columns [c CW, c CW + ncol) of each of
+// the NT outputs, CW = ceil(d / G) rounded up to a multiple of 4 so that the partials move
+// as float4s; the G partials part[(k NT + t) d + col] of a column are summed in ngu groups
+// of consecutive k in parallel (ascending k within a group, at most 16 loads per thread
+// in flight at once), then the groups in ascending order: a fixed order, deterministic.
+// `red` holds blockDim.x float4s of shared memory; out(t, col, v) receives the sums of
+// columns col..col+3 of output t.  The grouping depends on NTMAX (not NT), so that a
+// kernel instantiated for several output counts sums each output in the same order.
+template <int NT, int NTMAX, class Out>
+__device__ __forceinline__ void column_sums(const float *part, int d, int G, float4 *red, Out out) {
+  const int c = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
+  const int CW = (((d + G - 1) / G) + 3) & ~3;
+  const int col0 = c * CW;
+  const int nq = max(0, min(CW, d - col0)) / 4;  // float4 columns (d is a multiple of 4)
+  const int width_all = nq * NT;
+  if (width_all == 0) return;
+  const int ngu = max(1, min(G, nthr / min(nq * NTMAX, nthr)));
+  const int pass = nthr / ngu;  // (token, float4 column) pairs per pass
+  const size_t kstride = (size_t)NT * d / 4;
+  for (int cb = 0; cb < width_all; cb += pass) {
+    const int width = min(pass, width_all - cb);
+    const int gi = tid / pass, j = tid - gi * pass;
+    if (gi < ngu && j < width) {
+      const int e = cb + j, t = e / nq, q = e - t * nq;
+      const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * d + col0) + q;
+      const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int kb = k0; kb < k1; kb += 16) {
+        float4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          v[u] = kb + u < k1 ? __ldcg(src + (size_t)(kb + u) * kstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (kb + u < k1) {
+            s.x += v[u].x;
+            s.y += v[u].y;
+            s.z += v[u].z;
+            s.w += v[u].w;
+          }
+      }
+      red[gi * pass + j] = s;
+    }
+    __syncthreads();
+    if (tid < width) {
+      float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int g = 0; g < ngu; ++g) {
+        const float4 v = red[g * pass + tid];
+        tot.x += v.x;
+        tot.y += v.y;
+        tot.z += v.z;
+        tot.w += v.w;
+      }
+      const int e = cb + tid, t = e / nq, q = e - t * nq;
+      out(t, col0 + 4 * q, tot);
+    }
+    __syncthreads();
+  }
+}
+
 // Rebalancing of a fused kernel's active rows, after the split barrier's wait: every
 // tile's count (P.bcnt, clamped to the tile), e_t = the rows past `quota`, and CTA c's
 // even share of them, the global excess rows [floor(cE/G), floor((c+1)E/G)) in tile

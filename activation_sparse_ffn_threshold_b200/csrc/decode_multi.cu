@@ -523,46 +523,18 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
     }
   }
   if (!cta_grid_sync(P, flag_s)) return;
-  const int CW = (d + G - 1) / G;
-  const int col0 = c * CW;
-  const int ncol = max(0, min(CW, d - col0));
-  const int width_all = ncol * NB;  // (token, column) pairs of this CTA's slice
-  // groups of partials summed in parallel: a function of the slice width alone, so that a
-  // token's sums have the same order whatever the batch's size
-  const int ngu = max(1, kT / max(1, ncol * kMultiMaxTokens));
-  const int pass = kT / ngu;  // pairs per pass
-  for (int cb = 0; cb < width_all; cb += pass) {
-    const int width = min(pass, width_all - cb);
-    const int gi = tid / pass, j = tid % pass;
-    if (gi < ngu && j < width) {
-      const int e = cb + j, t = e / ncol, col = col0 + e - t * ncol;
-      const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
-      const float *src = P.part + (size_t)t * d + col;
-      const size_t kstride = (size_t)NB * d;
-      float sum = 0.f;  // in ascending k; loads issued 8 at a time
-      int k = k0;
-      for (; k + 8 <= k1; k += 8) {
-        float v[8];
+  // the stage region is free again: C2's copies have all landed
+  column_sums<NB, kMultiMaxTokens>(P.part, d, G, reinterpret_cast<float4 *>(stage), [&](int t, int col, float4 v) {
+    const float t4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (size_t)(k + u) * kstride);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) sum += v[u];
-      }
-      for (; k < k1; ++k) sum += __ldcg(src + (size_t)k * kstride);
-      red2[gi * width + j] = sum;
-    }
-    __syncthreads();
-    if (tid < width) {
-      float tot = 0.f;
-      for (int g = 0; g < ngu; ++g) tot += red2[g * width + tid];
-      const int e = cb + tid, t = e / ncol, col = col0 + e - t * ncol;
-      const size_t o = (size_t)t * d + col;
+    for (int i = 0; i < 4; ++i) {
+      const size_t o = (size_t)t * d + col + i;
+      float tot = t4[i];
       if (P.resid) tot = P.resid[o] + tot;
       P.y[o] = tot;
       if (P.xnext) static_cast<__half *>(P.xnext)[o] = __float2half_rn(tot);
     }
-    __syncthreads();
-  }
+  });
 }
 
 template <int NB, int ACT, int MAXM>
