@@ -114,8 +114,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 
   // B^T rows of this warp's neurons stream through DB shared-memory stages private to the
   // warp; each lane copies (cp.async) exactly the chunks it will read, so only its own
-  // wait is needed.  The first DB rows are requested during phase A, after x and the
-  // warp's half rows of A^T (the critical path into the first grid barrier), and land
+  // wait is needed.  The first DB rows are requested as soon as x has landed, and land
   // while phase A and the barrier run.
   unsigned char *bst = bstage + (size_t)warp * DB * nch_r * 16;
   auto stage_b = [&](int s, int p) {  // row p of the tile into stage s; always one group
@@ -133,10 +132,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
         __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
   __syncthreads();
-  if (j0 >= r) {
+  // every warp requests its first B^T stages now (x has landed), ahead of its A half rows
 #pragma unroll
-    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
-  }
+  for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
   // each half row's dot product (chunks ascending in one chain, then a butterfly sum) goes
   // to hbuf[half][j]; h_j = relu(first half + second half) is formed after the barrier
   for (int j = j0; j < r; j += G * (kW / 2)) {
@@ -158,10 +156,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     }
     const float hs = warp_sum(acc);
     if (lane == 0) P.hbuf[(size_t)ahalf * r + j] = hs;
-  }
-  if (j0 < r) {
-#pragma unroll
-    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
   }
   // c and b of the tile into shared memory
   if (tid < tn) {
@@ -204,7 +198,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       }
     }
     for (int pb = warp; pb < tn; pb += DB * kW) {
-#pragma unroll
+#pragma unroll 1
       for (int s = 0; s < DB; ++s) {
         const int p = pb + kW * s;
         if (p < tn) {
@@ -304,9 +298,27 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int nseg = P.nseg;
   const int per_row = NPG * nseg;
   const int nch_r8 = d / VR;  // 16-byte chunks of a row
-  // rows [kb, ke): their segments spread over all warps, 2-deep register pipeline;
-  // `pre` stages of C2 are requested behind the first loads
-  auto c1 = [&](int kb, int ke, int pre) {
+  // C1 runs over rows [kb, ke) in one or two passes: the own rows, then (rebalancing) the
+  // rows shared out after the split barrier's wait.  A pass spreads its rows' segments
+  // over all warps with a 2-deep register pipeline; the first requests `pre` stages of C2
+  // behind its first loads.
+  const int pre = quota > 0 ? min(DD, own) : DD;
+  int total = own;
+  for (int pass = 0, kb = 0, ke = own; pass < (quota > 0 ? 2 : 1); ++pass) {
+    if (pass == 1) {
+      if (!cta_grid_wait(P, target_s, flag_s)) {
+        cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+        return;
+      }
+      const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
+        act_s[own + j] = e.x;
+        bias_s[own + j] = __int_as_float(e.y);
+      });
+      total = own + f;
+      nrows = total;
+      kb = own;
+      ke = total;
+    }
     constexpr int D = 2;
     const int items = (ke - kb) * per_row;
     uint4 wc[D][SU];
@@ -323,7 +335,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         }
       }
     }
-    for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
+    if (pass == 0)
+      for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
       for (int s = 0; s < D; ++s) {
@@ -358,22 +371,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
         }
       }
     }
-  };
-  const int pre = quota > 0 ? min(DD, own) : DD;
-  c1(0, own, pre);
-  int total = own;
-  if (quota > 0) {
-    if (!cta_grid_wait(P, target_s, flag_s)) {
-      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-      return;
-    }
-    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
-      act_s[own + j] = e.x;
-      bias_s[own + j] = __int_as_float(e.y);
-    });
-    total = own + f;
-    nrows = total;
-    c1(own, total, 0);
   }
   __syncthreads();
   for (int k = tid; k < total; k += kT) {
@@ -403,7 +400,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
   for (int kb = 0; kb < total; kb += DD) {
-#pragma unroll
+#pragma unroll 1
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
       if (k < total) {

@@ -128,12 +128,12 @@ __device__ __forceinline__ bool cta_grid_wait(const Decode1Params &P, const unsi
 
 // The fused kernels' final sums.  CTA c owns the columns [c CW, c CW + ncol) of each of
 // the NT outputs, CW = ceil(d / G) rounded up to a multiple of 4 so that the partials move
-// as float4s; the G partials part[(k NT + t) d + col] of a column are summed in ngu groups
-// of consecutive k in parallel (ascending k within a group, at most 16 loads per thread
-// in flight at once), then the groups in ascending order: a fixed order, deterministic.
-// `red` holds blockDim.x float4s of shared memory; out(t, col, v) receives the sums of
-// columns col..col+3 of output t.  The grouping depends on NTMAX (not NT), so that a
-// kernel instantiated for several output counts sums each output in the same order.
+// as float4s.  The G partials part[(k NT + t) d + col] of a column are summed in ngu
+// groups of consecutive k in parallel (ascending k within a group, 8 loads in flight),
+// ngu a power of two, then the groups pairwise in a fixed tree: deterministic.  `red`
+// holds blockDim.x float4s of shared memory; out(t, col, v) receives the sums of columns
+// col..col+3 of output t.  The grouping depends on NTMAX (not NT), so that a kernel
+// instantiated for several output counts sums each output in the same order.
 template <int NT, int NTMAX, class Out>
 __device__ __forceinline__ void column_sums(const float *part, int d, int G, float4 *red, Out out) {
   const int c = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
@@ -142,46 +142,42 @@ __device__ __forceinline__ void column_sums(const float *part, int d, int G, flo
   const int nq = max(0, min(CW, d - col0)) / 4;  // float4 columns (d is a multiple of 4)
   const int width_all = nq * NT;
   if (width_all == 0) return;
-  const int ngu = max(1, min(G, nthr / min(nq * NTMAX, nthr)));
+  int ngu = 1;
+  while (ngu * 2 <= G && ngu * 2 * min(nq * NTMAX, nthr) <= nthr) ngu *= 2;
   const int pass = nthr / ngu;  // (token, float4 column) pairs per pass
   const size_t kstride = (size_t)NT * d / 4;
+  const int gi = tid / pass, j = tid - gi * pass;
   for (int cb = 0; cb < width_all; cb += pass) {
     const int width = min(pass, width_all - cb);
-    const int gi = tid / pass, j = tid - gi * pass;
+    const int e = cb + j, t = e / nq, q = e - t * nq;
     if (gi < ngu && j < width) {
-      const int e = cb + j, t = e / nq, q = e - t * nq;
       const float4 *src = reinterpret_cast<const float4 *>(part + (size_t)t * d + col0) + q;
       const int k0 = (int)(((int64_t)gi * G) / ngu), k1 = (int)(((int64_t)(gi + 1) * G) / ngu);
       float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int kb = k0; kb < k1; kb += 16) {
-        float4 v[16];
+      for (int kb = k0; kb < k1; kb += 8) {
+        float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
+        for (int u = 0; u < 8; ++u)
           v[u] = kb + u < k1 ? __ldcg(src + (size_t)(kb + u) * kstride) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (kb + u < k1) {
-            s.x += v[u].x;
-            s.y += v[u].y;
-            s.z += v[u].z;
-            s.w += v[u].w;
-          }
+        for (int u = 0; u < 8; ++u) {
+          s.x += v[u].x;
+          s.y += v[u].y;
+          s.z += v[u].z;
+          s.w += v[u].w;
+        }
       }
       red[gi * pass + j] = s;
     }
     __syncthreads();
-    if (tid < width) {
-      float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int g = 0; g < ngu; ++g) {
-        const float4 v = red[g * pass + tid];
-        tot.x += v.x;
-        tot.y += v.y;
-        tot.z += v.z;
-        tot.w += v.w;
+    for (int stride = ngu / 2; stride >= 1; stride /= 2) {  // group gi += group gi + stride
+      if (gi < stride && j < width) {
+        const float4 a = red[gi * pass + j], b = red[(gi + stride) * pass + j];
+        red[gi * pass + j] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
       }
-      const int e = cb + tid, t = e / nq, q = e - t * nq;
-      out(t, col0 + 4 * q, tot);
+      __syncthreads();
     }
+    if (gi == 0 && j < width) out(t, col0 + 4 * q, red[j]);
     __syncthreads();
   }
 }

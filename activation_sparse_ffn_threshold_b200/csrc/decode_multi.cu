@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
         }
       }
     for (int pb = pair; pb < tn; pb += kMB * kPairs) {
-#pragma unroll
+#pragma unroll 1
       for (int s = 0; s < kMB; ++s) {
         const int p = pb + kPairs * s;
         if (p < tn) {
@@ -379,10 +379,28 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   };
 
   // ---------------------------------------------------------------- C1: gate / up dots
-  // rows [kb, ke) (after the prefix), their segments over all warps, 2-deep register
-  // pipeline, dots only for the tokens active on each row; `pre` stages of C2 requested
-  // behind the first loads
-  auto c1 = [&](int kb, int ke, int pre) {
+  // rows [kb, ke) after the prefix in one or two passes (the own rows, then the rows
+  // shared out by the rebalancing), their segments over all warps, 2-deep register
+  // pipeline, dots only for the tokens active on each row; the first pass requests `pre`
+  // stages of C2 behind its first loads
+  const int pre = quota > 0 ? min(DD, own) : DD;
+  int total = own;
+  for (int pass = 0, kb = kp, ke = own; pass < (quota > 0 ? 2 : 1); ++pass) {
+    if (pass == 1) {
+      if (!cta_grid_wait(P, target_s, flag_s)) {
+        cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+        return;
+      }
+      const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
+        act_s[own + j] = e.x & 0xFFFFFF;
+        tok_s[own + j] = (uint32_t)e.x >> 24;
+        bias_s[own + j] = __int_as_float(e.y);
+      });
+      total = own + f;
+      nrows = total;
+      kb = own;
+      ke = total;
+    }
     constexpr int D = 2;
     const int items = (ke - kb) * per_row;
     uint4 wc[D][SU];
@@ -399,7 +417,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
         }
       }
     }
-    for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
+    if (pass == 0)
+      for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
       for (int s = 0; s < D; ++s) {
@@ -435,23 +454,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
         }
       }
     }
-  };
-  const int pre = quota > 0 ? min(DD, own) : DD;
-  c1(kp, own, pre);
-  int total = own;
-  if (quota > 0) {
-    if (!cta_grid_wait(P, target_s, flag_s)) {
-      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-      return;
-    }
-    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
-      act_s[own + j] = e.x & 0xFFFFFF;
-      tok_s[own + j] = (uint32_t)e.x >> 24;
-      bias_s[own + j] = __int_as_float(e.y);
-    });
-    total = own + f;
-    nrows = total;
-    c1(own, total, 0);
   }
   __syncthreads();
   for (int e = tid; e < total * NB; e += kT) {
@@ -482,7 +484,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
 #pragma unroll
       for (int t = 0; t < NB; ++t) acc[m][i][t] = make_float2(0.f, 0.f);
   for (int kb = 0; kb < total; kb += DD) {
-#pragma unroll
+#pragma unroll 1
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
       if (k < total) {

@@ -208,31 +208,40 @@ def measured_peak():
 
 
 # the sources k_decode1 is built from: a profile of it stays valid while they are unchanged
-DECODE1_SOURCES = ("async.cuh", "common.cuh", "decode1.cu", "decode1.cuh", "decode_dev.cuh")
+# The sources each measured path is built from: a committed ncu summary of a path stays
+# valid (its DRAM traffic is reported) while they are unchanged.
+PATH_SOURCES = {
+    "k_decode1": ("async.cuh", "common.cuh", "decode1.cu", "decode1.cuh", "decode_dev.cuh"),
+    "multi": ("async.cuh", "common.cuh", "decode_multi.cu", "decode1.cuh", "decode_dev.cuh"),
+    "tcgen05": ("async.cuh", "common.cuh", "tc_batch.cu", "predict.cu", "ffn.cu", "launch.cuh"),
+    "lookahead": ("async.cuh", "common.cuh", "decode_ahead.cu", "decode1.cuh", "decode_dev.cuh"),
+}
 
 
-def source_digest() -> str:
+def source_digest(path: str = "k_decode1") -> str:
     h = hashlib.sha256()
-    for name in DECODE1_SOURCES:
+    for name in PATH_SOURCES[path]:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per k_decode1 launch from the committed ncu summary of this workload,
-    if it was taken on the current sources."""
+def profiled_traffic(workload: str, summary: str | None = None, path: str = "k_decode1",
+                     key: str = "dram_bytes_per_token"):
+    """DRAM bytes per unit (token, batch or layer-token) from the committed ncu summary
+    profiles/<summary>.md, if it was taken on the current sources of `path`."""
+    summary = summary or f"k_decode1_{workload}"
     try:
-        text = open(os.path.join(ROOT, "profiles", f"k_decode1_{workload}.md")).read()
+        text = open(os.path.join(ROOT, "profiles", f"{summary}.md")).read()
     except OSError:
         return None, None
     sha = traffic = None
     for line in text.splitlines():
         if line.startswith("source_sha256_16:"):
             sha = line.split(":", 1)[1].strip()
-        if line.startswith("dram_bytes_per_token:"):
+        if line.startswith(f"{key}:"):
             traffic = float(line.split(":", 1)[1].strip())
-    if sha != source_digest():
+    if sha != source_digest(path):
         return None, "stale"
     return traffic, "ncu"
 
@@ -532,9 +541,11 @@ def measure_batch(cfg, b, args, dist, dev):
            "replicas": R, "path": path, "kernels_per_batch": launches // BATCHES_PER_STEP,
            "mean_union_rows": float(unions.mean()), "gpu_launches": int(launches * args.steps), "clocks": clocks,
            "bytes_per_step": float(bytes_batch.sum())}
+    tpath = "multi" if b <= 4 and handles[0].info()["wdtype"] == 1 else "tcgen05"
+    traffic, tsrc = profiled_traffic(cfg.name, f"batch_{cfg.name}_b{b}", tpath, "dram_bytes_per_batch")
     out["roofline"] = roofline(float(bytes_batch.mean()), unit_us,
                                f"one batch of {b} tokens ({launches // BATCHES_PER_STEP} kernels, {path}); "
-                               "duration = CUDA-event time of the timed region / batches")
+                               "duration = CUDA-event time of the timed region / batches", traffic, tsrc)
     out["effective_gbs"] = float(bytes_batch.sum()) * args.steps / (ms / 1e3) / 1e9
     del g
     _free(handles)
@@ -542,10 +553,12 @@ def measure_batch(cfg, b, args, dist, dev):
 
 
 def batch_path_name(h, b) -> str:
+    """The kernels AUTO (or the chosen path) runs for b tokens on this layer."""
     inf = h.info()
-    return {0: "auto", 1: "cuda-core", 2: "tcgen05"}.get(inf["batch_path"], "?") + \
-        (f" (auto: {'tcgen05' if inf['wdtype'] == 1 and inf['d'] % 128 == 0 and b >= 2 else 'cuda-core'})"
-         if inf["batch_path"] == 0 else "")
+    fused = inf["wdtype"] == 1 and 2 <= b <= 4  # fp16 layers: the few-token fused kernel
+    tc = inf["wdtype"] == 1 and inf["d"] % 128 == 0
+    auto = "fused few-token kernel (CUDA cores)" if fused else ("tcgen05" if tc else "cuda-core")
+    return {0: f"auto: {auto}", 1: "cuda-core", 2: "tcgen05", 3: f"fused: {auto}"}.get(inf["batch_path"], "?")
 
 
 def measure_stack(cfg, args, dist, dev, lookahead=False, rows=None):
@@ -589,8 +602,10 @@ def measure_stack(cfg, args, dist, dev, lookahead=False, rows=None):
     kern = (f"k_decode_ahead (look-ahead stack), {launches // T} launches per token: the input rounding, layer 0's "
             "predictor, one per layer" if lookahead else
             f"k_decode1, one launch per layer and token ({launches // T} launches per token with the input rounding)")
+    traffic, tsrc = profiled_traffic(cfg.name, f"stack_{cfg.name}{'_lookahead' if lookahead else ''}",
+                                     "lookahead" if lookahead else "k_decode1", "dram_bytes_per_layer_token")
     out["roofline"] = roofline(float(bytes_layer_tok.mean()), layer_us,
-                               kern + "; duration = CUDA-event time of the region / layer-tokens")
+                               kern + "; duration = CUDA-event time of the region / layer-tokens", traffic, tsrc)
     out["effective_gbs"] = float(bytes_layer_tok.sum()) * T * args.steps / (ms / 1e3) / 1e9
     if not args.no_e2e:
         xin = torch.from_numpy(Xh).pin_memory()
