@@ -18,12 +18,13 @@
 //       shared-memory stages of its own (16-byte cp.async copies, the first ones requested
 //       during phase A); neuron i is active iff z_i > 0 (sigmoid(z) > 0.5).  The tile's
 //       active positions are compacted in order.
-//   C1  up (and gate) dot products of the active rows, split in 4 KB segments spread
-//       over all warps (2-deep register pipeline); segment sums added in a fixed order,
-//       then ReLU / ReGLU.  Rows of inactive neurons are never requested.
+//   C1  up (and gate) dot products of the active rows, split in 4 KB segments dealt to
+//       the warps; each warp streams its segments through 3 shared-memory slots of its
+//       own (192 KB of the CTA's shared memory in flight); segment sums added in a fixed
+//       order, then ReLU / ReGLU.  Rows of inactive neurons are never requested.
 //   C2  the active rows of W_down (neuron-major, contiguous) are added into per-thread
-//       column accumulators; each thread's chunks stream through up to 8 private
-//       shared-memory stages, the first ones requested at C1's start.
+//       column accumulators; each thread's chunks stream through private shared-memory
+//       stages (128 KB of rows in flight per CTA).
 //   D   the CTA's partial y goes to global memory; grid barrier; CTA c sums a column
 //       slice of all G partials in a fixed order (two-phase, deterministic) -> y
 //       (+ residual, + rounded next-layer input).
@@ -57,9 +58,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr int VR = 128 / RB;           // row elements per 16-byte chunk
   constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
   constexpr int DB = kDecode1BStages;
-  constexpr int DD = decode1_dstages(MAXM);
+  constexpr int DD = decode1_c2stages(MAXM);
   extern __shared__ __align__(16) unsigned char smem[];
-  const Decode1Layout L = decode1_layout(P);
+  const Decode1Layout L = decode1_layout(P, true);
   unsigned char *xs = smem + L.x;
   float *bias_s = reinterpret_cast<float *>(smem + L.bias);  // b of the active rows, in order
   float *c_s = reinterpret_cast<float *>(smem + L.c);
@@ -269,8 +270,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int own = quota > 0 ? min(cnt, quota) : cnt;
   int nrows = own;  // rows of this CTA whose place in act_s is known
 
-  // C2's rows of W_down stream through DD shared-memory stages private to each thread;
-  // the first DD rows are requested right after C1's first loads and land while C1 runs
+  // C2's rows of W_down stream through DD shared-memory stages private to each thread,
+  // requested once C1 has left the staging region
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
     if (k < nrows) {
@@ -299,17 +300,15 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int per_row = NPG * nseg;
   const int nch_r8 = d / VR;  // 16-byte chunks of a row
   // C1 runs over rows [kb, ke) in one or two passes: the own rows, then (rebalancing) the
-  // rows shared out after the split barrier's wait.  A pass spreads its rows' segments
-  // over all warps with a 2-deep register pipeline; the first requests `pre` stages of C2
-  // behind its first loads.
-  const int pre = quota > 0 ? min(DD, own) : DD;
+  // rows shared out after the split barrier's wait.  A pass deals its rows' 4 KB segments
+  // round-robin to the warps; each warp streams its segments through kC1Ring shared-memory
+  // slots of its own, each lane copying (cp.async) exactly the 16-byte chunks it reads, so
+  // only its own wait is needed (as the B^T stages).
   int total = own;
+  unsigned char *cring = dstage + (size_t)warp * kC1Ring * kC1SegBytes;
   for (int pass = 0, kb = 0, ke = own; pass < (quota > 0 ? 2 : 1); ++pass) {
     if (pass == 1) {
-      if (!cta_grid_wait(P, target_s, flag_s)) {
-        cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-        return;
-      }
+      if (!cta_grid_wait(P, target_s, flag_s)) return;  // no copy in flight
       const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
         act_s[own + j] = e.x;
         bias_s[own + j] = __int_as_float(e.y);
@@ -319,58 +318,49 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       kb = own;
       ke = total;
     }
-    constexpr int D = 2;
     const int items = (ke - kb) * per_row;
-    uint4 wc[D][SU];
-#pragma unroll
-    for (int s = 0; s < D; ++s) {
-      const int it = warp + kW * s;
+    auto stage_c = [&](int slot, int i) {  // this warp's i-th segment into a slot; always one group
+      const int it = warp + kW * i;
       if (it < items) {
         const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
         const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
         for (int u = 0; u < SU; ++u) {
           const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
+          if (ch < nch_r8) cp_async16(cring + (size_t)slot * kC1SegBytes + (lane + 32 * u) * 16, row + (size_t)ch * 16);
         }
       }
-    }
-    if (pass == 0)
-      for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
-    for (int ib = warp; ib < items; ib += D * kW) {
+      cp_async_commit();
+    };
 #pragma unroll
-      for (int s = 0; s < D; ++s) {
-        const int it = ib + kW * s;
-        if (it < items) {
-          const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-          float a = 0.f;
+    for (int i = 0; i < kC1Ring; ++i) stage_c(i, i);
+    const int mine = items > warp ? (items - warp + kW - 1) / kW : 0;
+#pragma unroll 1
+    for (int i = 0; i < mine; ++i) {
+      const int slot = i % kC1Ring;
+      cp_async_wait<kC1Ring - 1>();  // this lane's chunks of segment i have landed
+      const int it = warp + kW * i;
+      const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+      const unsigned char *sl = cring + (size_t)slot * kC1SegBytes;
+      float a = 0.f;
 #pragma unroll
-          for (int u = 0; u < SU; ++u) {
-            const int ch = sg * kSegChunks + lane + 32 * u;
-            if (ch < nch_r8) {
-              if (RB == 4)
-                a = dot_chunk_i4(wc[s][u], xs, ch, a);
-              else if (RB == 8)
-                a = dot_chunk_i8(wc[s][u], xs, ch, a);
-              else
-                a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
-            }
-          }
-          const int itn = it + D * kW;
-          if (itn < items) {
-            const int kn = kb + itn / per_row, pjn = (itn % per_row) / nseg, sgn = itn % per_row - pjn * nseg;
-            const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
-#pragma unroll
-            for (int u = 0; u < SU; ++u) {
-              const int ch = sgn * kSegChunks + lane + 32 * u;
-              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
-            }
-          }
-          a = warp_sum(a);
-          if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+      for (int u = 0; u < SU; ++u) {
+        const int ch = sg * kSegChunks + lane + 32 * u;
+        if (ch < nch_r8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(sl + (lane + 32 * u) * 16);
+          if (RB == 4)
+            a = dot_chunk_i4(w, xs, ch, a);
+          else if (RB == 8)
+            a = dot_chunk_i8(w, xs, ch, a);
+          else
+            a = dot_chunk_smem<T>(w, xs, ch, a);
         }
       }
+      stage_c(slot, i + kC1Ring);
+      a = warp_sum(a);
+      if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
     }
+    cp_async_wait<0>();
   }
   __syncthreads();
   for (int k = tid; k < total; k += kT) {
@@ -391,7 +381,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     if (QR) a_s[k] *= sd;
   }
   __syncthreads();
-  for (int s = pre; s < DD; ++s) stage_d(s, s);  // C2's first stages not requested yet
+#pragma unroll 1
+  for (int s = 0; s < DD; ++s) stage_d(s, s);  // C2's first stages (the ring is free again)
 
   // ---------------------------------------------------------------- C2: down projection
   float acc[MAXM][V];
@@ -523,7 +514,7 @@ cudaError_t configure_decode1() {
 }
 
 int decode1_blocks_per_sm(const Decode1Params &P) {
-  const size_t smem = decode1_layout(P).total;
+  const size_t smem = decode1_layout(P, true).total;
   if (smem > (size_t)kSmemCap) return 0;
   const int nch = P.d / (P.dt == SFNN_F16 ? 8 : 4);
   if (nch > 4 * kT) return 0;  // beyond the kernel's register plan
@@ -539,7 +530,7 @@ cudaError_t launch_barrier_bump(uint64_t *count, cudaStream_t stream) {
 }
 
 cudaError_t launch_decode1(const Decode1Params &P, cudaStream_t stream, bool pdl) {
-  const size_t smem = decode1_layout(P).total;
+  const size_t smem = decode1_layout(P, true).total;
   if (P.dt != SFNN_F16)
     return P.act == SFNN_REGLU ? launch_act<float, SFNN_REGLU, float>(P, smem, stream, pdl)
                                : launch_act<float, SFNN_RELU, float>(P, smem, stream, pdl);

@@ -15,6 +15,11 @@ constexpr int kDecodeSmemCap = 227 * 1024;  // opt-in dynamic shared memory of o
 
 // W_down rows in flight per thread in the down phase, by 16-byte chunks per thread and row
 __host__ __device__ constexpr int decode1_dstages(int maxm) { return maxm == 1 ? 8 : (maxm == 2 ? 4 : 2); }
+// The single-token kernel's down phase has the whole staging region (128 KB of rows).
+__host__ __device__ constexpr int decode1_c2stages(int maxm) { return maxm == 1 ? 16 : (maxm == 2 ? 8 : 4); }
+// Its up/gate phase streams 4 KB row segments through this many shared-memory slots per warp.
+constexpr int kC1Ring = 3;
+constexpr int kC1SegBytes = 4096;
 // 16-byte chunks of a d-vector per thread (1, 2 or 4)
 __host__ __device__ inline int decode1_maxm(int nch_d) {
   return nch_d <= kDecode1Threads ? 1 : (nch_d <= 2 * kDecode1Threads ? 2 : 4);
@@ -52,16 +57,22 @@ struct Decode1Layout {
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Bytes of the staging region: B^T rows (phase B) and W_down chunks (C2) share it.
-__host__ __device__ inline size_t decode1_stage_bytes(const Decode1Params &P) {
+// Bytes of the staging region: B^T rows (phase B) and W_down chunks (C2) share it, and in
+// the single-token kernel (`ring`) the up/gate segments (C1) as well.
+__host__ __device__ inline size_t decode1_stage_bytes(const Decode1Params &P, bool ring = false) {
   const int vec = P.dt == SFNN_F16 ? 8 : 4;
   const int maxm = decode1_maxm(P.d / vec);
   const size_t bsz = (size_t)(kDecode1Threads / 32) * kDecode1BStages * (P.r / vec) * 16;
-  const size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
+  size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
+  if (ring) {
+    const size_t csz = (size_t)(kDecode1Threads / 32) * kC1Ring * kC1SegBytes;
+    const size_t c2 = (size_t)decode1_c2stages(maxm) * maxm * kDecode1Threads * 16;
+    dsz = csz > c2 ? csz : c2;
+  }
   return bsz > dsz ? bsz : dsz;
 }
 
-__host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) {
+__host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P, bool ring = false) {
   const size_t esz = P.dt == SFNN_F16 ? 2 : 4;
   const size_t tm = (size_t)P.tile_max;
   Decode1Layout L;
@@ -92,7 +103,7 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P) 
   // W_down chunks only after it (the CTA synchronises in between).
   L.bstage = o;  // [warp][stage][chunk of the row]: B^T rows staged per warp
   L.dstage = o;  // [stage][chunk m][thread]: W_down chunks staged per thread
-  o = decode1_align(o + decode1_stage_bytes(P), 16);
+  o = decode1_align(o + decode1_stage_bytes(P, ring), 16);
   L.total = o;
   return L;
 }
