@@ -85,6 +85,7 @@ def load_library():
         "sfnn_set_batch_path": ([P, I], S),
         "sfnn_set_fused_decode": ([P, I], S),
         "sfnn_set_hot_prefix": ([P, I], S),
+        "sfnn_set_fused_quota": ([P, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
         "sfnn_query": ([P, ctypes.POINTER(Info)], S),
@@ -257,6 +258,10 @@ class SparseFFN:
 
     def set_fused_decode(self, enable: bool):
         _check(self._lib.sfnn_set_fused_decode(self._h, int(bool(enable))), "sfnn_set_fused_decode")
+
+    def set_fused_quota(self, quota: int):
+        """The single-token kernel's rebalancing quota (0: off; -1: the profile's default)."""
+        _check(self._lib.sfnn_set_fused_quota(self._h, int(quota)), "sfnn_set_fused_quota")
 
     def set_hot_prefix(self, enable: bool):
         """Read the hot prefix densely on the fused few-token path (default on)."""

@@ -598,6 +598,14 @@ sfnn_status sfnn_set_batch_path(sfnn_handle h, int32_t path) {
   return SFNN_OK;
 }
 
+sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota) {
+  if (!h || quota < -1) return SFNN_ERR_INVALID_ARG;
+  if (!h->fused_ok) return SFNN_ERR_UNSUPPORTED;
+  const int q = quota == -1 ? h->quota : quota;
+  h->d1.quota = 2 * h->d1.G + 3 <= kDecode1Threads ? std::min(q, h->d1.tile_max) : 0;
+  return SFNN_OK;
+}
+
 sfnn_status sfnn_set_hot_prefix(sfnn_handle h, int32_t enable) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   h->hot_on = enable != 0;

@@ -89,9 +89,19 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const size_t rowB = (size_t)P.d * RB / 8;  // bytes of one stored row
 
   pdl_launch_dependents();
+  // The launch is cooperative: its CTAs start together once the previous kernel's CTAs
+  // have left the SMs, so the wait for that kernel costs little here, and x is requested
+  // first, ahead of the weights' streams.
+  pdl_wait();  // x (and every buffer this kernel writes) belongs to earlier kernels until here
+  uint4 xv[MAXM];
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    const int ch = tid + kT * m;
+    if (ch < nch_d) xv[m] = __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)ch * 16));
+  }
   // A^T rows are split in halves over warp pairs: warp w takes half (w & 1) of the rows
   // j = c + G (w >> 1) + 8 G k, so that a lane's part of its first half row (at most 16
-  // chunks for d <= 8192 fp16) is requested before anything else.
+  // chunks for d <= 8192 fp16) is requested at once.
   const int apair = warp >> 1, ahalf = warp & 1;
   const int hca = (nch_d + 1) / 2;  // chunks of a row's first half
   const int abeg = ahalf * hca, aend = ahalf ? nch_d : hca;
@@ -128,10 +138,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     }
     cp_async_commit();
   };
-  pdl_wait();  // x (and every buffer this kernel writes) belongs to earlier kernels until here
-  for (int i = tid; i < nch_d; i += kT)
-    *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
-        __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    const int ch = tid + kT * m;
+    if (ch < nch_d) *reinterpret_cast<uint4 *>(xs + (size_t)ch * 16) = xv[m];
+  }
   __syncthreads();
   // every warp requests its first B^T stages now (x has landed), ahead of its A half rows
 #pragma unroll
@@ -299,69 +310,77 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int nseg = P.nseg;
   const int per_row = NPG * nseg;
   const int nch_r8 = d / VR;  // 16-byte chunks of a row
-  // C1 runs over rows [kb, ke) in one or two passes: the own rows, then (rebalancing) the
-  // rows shared out after the split barrier's wait.  A pass deals its rows' 4 KB segments
-  // round-robin to the warps; each warp streams its segments through kC1Ring shared-memory
-  // slots of its own, each lane copying (cp.async) exactly the 16-byte chunks it reads, so
-  // only its own wait is needed (as the B^T stages).
+  // One stream of the rows' 4 KB segments, dealt round-robin to the warps; each warp keeps
+  // kC1Ring of its segments in flight in shared-memory slots of its own, each lane copying
+  // (cp.async) exactly the 16-byte chunks it reads, so only its own wait is needed (as the
+  // B^T stages).  With rebalancing, the split barrier's wait and the fetch of the rows
+  // shared out to this CTA happen at iteration M of every warp -- early enough that every
+  // warp still has own segments in flight behind it, so the stream does not drain -- and
+  // the rows are appended to the stream; with too few own segments, before the stream.
   int total = own;
+  int items = own * per_row;
   unsigned char *cring = dstage + (size_t)warp * kC1Ring * kC1SegBytes;
-  for (int pass = 0, kb = 0, ke = own; pass < (quota > 0 ? 2 : 1); ++pass) {
-    if (pass == 1) {
-      if (!cta_grid_wait(P, target_s, flag_s)) return;  // no copy in flight
-      const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
-        act_s[own + j] = e.x;
-        bias_s[own + j] = __int_as_float(e.y);
-      });
-      total = own + f;
-      nrows = total;
-      kb = own;
-      ke = total;
-    }
-    const int items = (ke - kb) * per_row;
-    auto stage_c = [&](int slot, int i) {  // this warp's i-th segment into a slot; always one group
-      const int it = warp + kW * i;
-      if (it < items) {
-        const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-        const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
-#pragma unroll
-        for (int u = 0; u < SU; ++u) {
-          const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_r8) cp_async16(cring + (size_t)slot * kC1SegBytes + (lane + 32 * u) * 16, row + (size_t)ch * 16);
-        }
-      }
-      cp_async_commit();
-    };
-#pragma unroll
-    for (int i = 0; i < kC1Ring; ++i) stage_c(i, i);
-    const int mine = items > warp ? (items - warp + kW - 1) / kW : 0;
-#pragma unroll 1
-    for (int i = 0; i < mine; ++i) {
-      const int slot = i % kC1Ring;
-      cp_async_wait<kC1Ring - 1>();  // this lane's chunks of segment i have landed
-      const int it = warp + kW * i;
-      const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-      const unsigned char *sl = cring + (size_t)slot * kC1SegBytes;
-      float a = 0.f;
+  auto share = [&]() {  // every thread: wait for the split barrier, append the shared-out rows
+    if (!cta_grid_wait(P, target_s, flag_s)) return false;
+    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
+      act_s[own + j] = e.x;
+      bias_s[own + j] = __int_as_float(e.y);
+    });
+    total = own + f;
+    nrows = total;
+    items = total * per_row;
+    return true;
+  };
+  const int mmin = items / kW;  // segments every warp has at least
+  const bool early = quota > 0 && mmin < kC1Ring + 2;
+  if (early && !share()) return;  // no copy in flight
+  const int M = quota > 0 && !early ? mmin - kC1Ring - 1 : -1;  // >= 1; segments M .. M + kC1Ring - 1 are own
+  auto stage_c = [&](int slot, int i) {  // this warp's i-th segment into a slot; always one group
+    const int it = warp + kW * i;
+    if (it < items) {
+      const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+      const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
       for (int u = 0; u < SU; ++u) {
         const int ch = sg * kSegChunks + lane + 32 * u;
-        if (ch < nch_r8) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(sl + (lane + 32 * u) * 16);
-          if (RB == 4)
-            a = dot_chunk_i4(w, xs, ch, a);
-          else if (RB == 8)
-            a = dot_chunk_i8(w, xs, ch, a);
-          else
-            a = dot_chunk_smem<T>(w, xs, ch, a);
-        }
+        if (ch < nch_r8) cp_async16(cring + (size_t)slot * kC1SegBytes + (lane + 32 * u) * 16, row + (size_t)ch * 16);
       }
-      stage_c(slot, i + kC1Ring);
-      a = warp_sum(a);
-      if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
     }
-    cp_async_wait<0>();
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int i = 0; i < kC1Ring; ++i) stage_c(i, i);
+#pragma unroll 1
+  for (int i = 0;; ++i) {
+    if (i == M && !share()) {  // every warp reaches iteration M with own segments left
+      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
+      return;
+    }
+    const int it = warp + kW * i;
+    if (it >= items) break;
+    const int slot = i % kC1Ring;
+    cp_async_wait<kC1Ring - 1>();  // this lane's chunks of segment i have landed
+    const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+    const unsigned char *sl = cring + (size_t)slot * kC1SegBytes;
+    float a = 0.f;
+#pragma unroll
+    for (int u = 0; u < SU; ++u) {
+      const int ch = sg * kSegChunks + lane + 32 * u;
+      if (ch < nch_r8) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(sl + (lane + 32 * u) * 16);
+        if (RB == 4)
+          a = dot_chunk_i4(w, xs, ch, a);
+        else if (RB == 8)
+          a = dot_chunk_i8(w, xs, ch, a);
+        else
+          a = dot_chunk_smem<T>(w, xs, ch, a);
+      }
+    }
+    stage_c(slot, i + kC1Ring);
+    a = warp_sum(a);
+    if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
   }
+  cp_async_wait<0>();
   __syncthreads();
   for (int k = tid; k < total; k += kT) {
     float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)

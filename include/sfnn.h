@@ -279,6 +279,17 @@ SFNN_API sfnn_status sfnn_forward_stack_lookahead(const sfnn_handle *layers, int
 SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
 
 /*
+ * The single-token fused kernel's rebalancing of active rows over its CTAs: each CTA keeps
+ * the first `quota` active rows of its own tile, and the rows past the quota in all tiles
+ * are shared out evenly over the CTAs after a grid barrier (results within rounding of
+ * quota 0, and deterministic for a given quota).  By default the quota is 0.8 of a tile's
+ * expected active count under the hotness profile when that count is 20 or more, else 0
+ * (no rebalancing).  quota >= 0 sets it (clamped to a tile's size); -1 restores the
+ * default.  Takes effect at the next launch.
+ */
+SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
+
+/*
  * The fused few-token path (SFNN_BATCH_FUSED, and AUTO for 2 to 4 tokens) reads the
  * hot prefix of the layer densely (enabled by default): the neurons that the offline
  * hotness profile puts in a b-token batch's union with probability >= 0.99

@@ -8,6 +8,9 @@
 * consecutive launches on the same handle (programmatic dependent launch lets
   the next one start early) stay correct and bitwise reproducible;
 * the residual stack runs through it;
+* its rebalancing of active rows over the CTAs (forced quotas, on a hot-packed layer
+  whose tiles hold very different counts; the wait for the shared-out rows before the
+  own rows' stream and inside it) gives the same sets and y within rounding, reproducibly;
 * a grid barrier that cannot complete runs out after its bound, latches
   SFNN_ERR_TIMEOUT, leaves the context usable, and the handle recovers.
 """
@@ -125,4 +128,28 @@ def test_fused_kernels_beside_a_kernel_on_another_stream():
         Y = h.forward_batch(X)
         torch.cuda.synchronize()
         assert torch.equal(y, y_ref) and torch.equal(Y, Y_ref)
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("base,d,n,r,quota", [
+    ("70b_reglu", 1024, 5003, 128, 2),     # few own segments: the wait comes before the stream
+    ("70b_reglu", 8192, 3001, 1024, 12),   # the wait inside the stream of own segments
+    ("opt6.7b_relu", 4096, 9000, 512, 6),
+])
+def test_rebalanced_rows_match(base, d, n, r, quota):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=21)
+    h = sf.SparseFFN.from_layer(lay, order="packed")  # the hottest neurons fill the first tiles
+    X = W.make_tokens(cfg, 3, seed=22)
+    for t in range(3):
+        xd = dev(X[t])
+        h.set_fused_quota(0)
+        y0, m0 = fused_step(h, xd)
+        h.set_fused_quota(quota)
+        y1, m1 = fused_step(h, xd)
+        assert np.array_equal(m0, m1)
+        assert oracle.within_tolerance(y1, y0.astype(np.float64))[0]
+        assert np.array_equal(h.forward(xd).cpu().numpy(), y1)  # deterministic for a quota
+        check_token(lay, X[t], y1, m1, f"{base} quota {quota} t={t}")
+    h.set_fused_quota(-1)
     assert h.get_error() == 0
