@@ -216,6 +216,12 @@ void plan_decode1(sfnn_ctx *h, int G) {
   for (int b = 0; b <= kMultiMaxTokens; ++b)  // the prefix must stay with its tile: else no rebalancing
     if (2 * G + 3 > kDecode1Threads || h->quota_multi[b] > P.tile_max) h->quota_multi[b] = 0;
   if (L.r / L.vec > 32 * 4) return;
+  // request depths (measured best on the 70B-, OPT-30B- and OPT-6.7B-shaped layers: 2-3%
+  // over 4 B^T stages, 8 early W_down rows, 2 segments in flight and 8 W_down stages)
+  P.bstages = 2;
+  P.c2pre = 4;
+  P.c1depth = 1;
+  P.c2stages = 4;
   if (decode1_blocks_per_sm(P) < 1) return;
   h->fused_ok = true;
   h->fused_on = true;
@@ -349,11 +355,13 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   for (int k = 0; k < L.n; ++k) perm[packed ? k : decode1_tile_start(k % G, L.n, G) + k / G] = by_rank[k];
   for (int p = 0; p < L.n; ++p) iperm[perm[p]] = p;
   for (int b = 0; b <= kMaxBatch; ++b) h->expected_union[b] = -1.0;
-  // The single-token kernel's quota of own rows per CTA: 0.8 of a tile's expected active
-  // count under the profile, when that count is 20 or more (measured: the rebalancing
-  // saves 3.4 us per token on the 70B-shaped layer, 23 rows per tile, is neutral on the
-  // OPT-30B-shaped one, 19.5, and costs 1.1 us on the OPT-6.7B-shaped one, 11); no
-  // profile, no rebalancing.
+  // The single-token kernel's quota of own rows per CTA: 0.9 of a tile's expected active
+  // count under the profile, when the own rows' up/gate bytes (quota x the rows read before
+  // the down phase) reach 96 KB -- the rebalancing's counts and lists take a few round trips
+  // under load, which the own rows' stream must cover.  Measured (us per token, no quota ->
+  // quota): 70B-shaped 63.4 -> 55.5 (23 rows per tile, 32 KB), OPT-30B-shaped 44.1 -> 40.1
+  // (19.5, 14 KB), LLaMA-7B-shaped 28.8 -> 27.2 (11.2, 16 KB); the OPT-6.7B-shaped layer
+  // (11, 8 KB: 81 KB) loses 2.4 with one.  No profile, no rebalancing.
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;
@@ -362,7 +370,10 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       mean += std::isnan(q) ? 0.0 : std::min(1.0, std::max(0.0, (double)q));
     }
     mean /= G;
-    h->quota = mean >= 20.0 ? (int)std::floor(0.8 * mean) : 0;
+    const double elem = L.rows_q ? L.rows_q / 8.0 : (double)(L.dt == SFNN_F16 ? 2 : 4);
+    const double c1_row = (L.nproj - 1) * (double)L.d * elem;  // up (and gate) bytes of a row
+    const int q = (int)std::floor(0.9 * mean);
+    h->quota = q * c1_row >= 96.0 * 1024 ? q : 0;
   }
   // The multi-token kernel's hot prefix for b tokens: the hottest ranks whose neuron is in
   // a b-token union with probability 1 - (1 - p)^b >= 0.99 (at most 64 rows per tile).
@@ -603,6 +614,23 @@ sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota) {
   if (!h->fused_ok) return SFNN_ERR_UNSUPPORTED;
   const int q = quota == -1 ? h->quota : quota;
   h->d1.quota = 2 * h->d1.G + 3 <= kDecode1Threads ? std::min(q, h->d1.tile_max) : 0;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_fused_depths(sfnn_handle h, int32_t bstages, int32_t c2pre, int32_t c1depth,
+                                  int32_t c2stages) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (bstages != -1 && (bstages < 1 || bstages > 8 || bstages == 5 || bstages == 7)) return SFNN_ERR_INVALID_ARG;
+  if (c2pre < -1 || c2pre > 16 || c1depth < -1 || c1depth == 0 || c1depth > 2) return SFNN_ERR_INVALID_ARG;
+  if (c2stages != -1 && (c2stages < 1 || c2stages > 16 || (c2stages & (c2stages - 1)))) return SFNN_ERR_INVALID_ARG;
+  if (!h->fused_ok) return SFNN_ERR_UNSUPPORTED;
+  Decode1Params P = h->d1;
+  if (bstages != -1) P.bstages = bstages;
+  if (c2pre != -1) P.c2pre = c2pre;
+  if (c1depth != -1) P.c1depth = c1depth;
+  if (c2stages != -1) P.c2stages = c2stages;
+  if (decode1_blocks_per_sm(P) < 1) return SFNN_ERR_UNSUPPORTED;
+  h->d1 = P;
   return SFNN_OK;
 }
 

@@ -57,8 +57,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   constexpr bool QR = RB <= 8;           // rows are codes with per-row scales
   constexpr int VR = 128 / RB;           // row elements per 16-byte chunk
   constexpr int MAXH = 4;  // chunks of h per lane (r <= 128 * V)
-  constexpr int DB = kDecode1BStages;
-  constexpr int DD = decode1_c2stages(MAXM);
+  const int DB = P.bstages;  // 1, 2, 3, 4, 6 or 8
+  const int DD = min(P.c2stages, decode1_c2stages(MAXM));  // 1, 2, 4, 8 or 16
   extern __shared__ __align__(16) unsigned char smem[];
   const Decode1Layout L = decode1_layout(P, true);
   unsigned char *xs = smem + L.x;
@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
   unsigned long long *target_s = reinterpret_cast<unsigned long long *>(cnt_s + 2);  // split barrier
+  int *next_s = cnt_s + 4;  // C1's next work item
+  int *ext_s = cnt_s + 5;   // C1's final row count once known (-1: not yet, -2: abandoned)
   unsigned char *bstage = smem + L.bstage;
   unsigned char *dstage = smem + L.dstage;
 
@@ -144,8 +146,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     if (ch < nch_d) *reinterpret_cast<uint4 *>(xs + (size_t)ch * 16) = xv[m];
   }
   __syncthreads();
-  // every warp requests its first B^T stages now (x has landed), ahead of its A half rows
-#pragma unroll
+  // every warp requests its first DB B^T rows now (x has landed), behind its first A^T half row
+#pragma unroll 1
   for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
   // each half row's dot product (chunks ascending in one chain, then a butterfly sum) goes
   // to hbuf[half][j]; h_j = relu(first half + second half) is formed after the barrier
@@ -214,7 +216,14 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       for (int s = 0; s < DB; ++s) {
         const int p = pb + kW * s;
         if (p < tn) {
-          cp_async_wait<DB - 1>();  // this lane's copies of row p have landed
+          switch (DB) {  // this lane's copies of row p have landed
+            case 1: cp_async_wait<0>(); break;
+            case 2: cp_async_wait<1>(); break;
+            case 3: cp_async_wait<2>(); break;
+            case 4: cp_async_wait<3>(); break;
+            case 6: cp_async_wait<5>(); break;
+            default: cp_async_wait<7>(); break;
+          }
           float a = 0.f;
 #pragma unroll
           for (int m = 0; m < MAXH; ++m) {
@@ -249,7 +258,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
       if (wi + lane < nwords) wpref[wi + lane] = base + incl - k;
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) *cnt_s = base;
+    if (lane == 0) {
+      *cnt_s = base;
+      *next_s = 0;
+      *ext_s = -1;
+    }
   }
   __syncthreads();
   for (int p = tid; p < tn; p += kT) {
@@ -269,9 +282,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   // Rebalancing (quota > 0): the busiest tile of a token holds ~1.5x the mean count, and
   // the CTAs that finish their rows early would leave the HBM stream to it.  So each CTA
   // keeps the first `quota` of its tile's active rows, publishes its list, and arrives on
-  // a grid barrier whose wait comes after the own rows' up/gate dots; then the rows past
-  // the quota in every tile are shared out evenly over all CTAs, in tile order (a
-  // function of the counts alone: deterministic).
+  // a grid barrier; one warp waits on it while the others stream the own rows, and the
+  // rows past the quota in every tile are shared out evenly over all CTAs, in tile order
+  // (a function of the counts alone: deterministic).
   const int quota = P.quota;
   if (quota > 0) {
     for (int k = tid; k < cnt; k += kT) P.blist[t0 + k] = make_int2(act_s[k], __float_as_int(bias_s[k]));
@@ -281,8 +294,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int own = quota > 0 ? min(cnt, quota) : cnt;
   int nrows = own;  // rows of this CTA whose place in act_s is known
 
-  // C2's rows of W_down stream through DD shared-memory stages private to each thread,
-  // requested once C1 has left the staging region
+  // C2's rows of W_down stream through DD shared-memory stages private to each thread
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
   auto stage_d = [&](int s, int k) {  // active row k into stage s; always one group
     if (k < nrows) {
@@ -310,77 +322,126 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   const int nseg = P.nseg;
   const int per_row = NPG * nseg;
   const int nch_r8 = d / VR;  // 16-byte chunks of a row
-  // One stream of the rows' 4 KB segments, dealt round-robin to the warps; each warp keeps
-  // kC1Ring of its segments in flight in shared-memory slots of its own, each lane copying
-  // (cp.async) exactly the 16-byte chunks it reads, so only its own wait is needed (as the
-  // B^T stages).  With rebalancing, the split barrier's wait and the fetch of the rows
-  // shared out to this CTA happen at iteration M of every warp -- early enough that every
-  // warp still has own segments in flight behind it, so the stream does not drain -- and
-  // the rows are appended to the stream; with too few own segments, before the stream.
+  // The rows' 4 KB segments are work items, handed out in order by a shared counter; each
+  // lane loads its SU chunks of a segment into registers (no L1 allocation), and a warp
+  // keeps two segments in flight: the next one's loads are issued before the current one
+  // is summed.  A segment's dot product does not depend on the warp that computes it.
   int total = own;
-  int items = own * per_row;
-  unsigned char *cring = dstage + (size_t)warp * kC1Ring * kC1SegBytes;
-  auto share = [&]() {  // every thread: wait for the split barrier, append the shared-out rows
-    if (!cta_grid_wait(P, target_s, flag_s)) return false;
-    const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
-      act_s[own + j] = e.x;
-      bias_s[own + j] = __int_as_float(e.y);
-    });
-    total = own + f;
-    nrows = total;
-    items = total * per_row;
-    return true;
+  int lim = own * per_row;  // items known to exist
+  bool known = quota == 0;  // the final count is known
+  uint4 wa[SU], wb[SU];
+  auto grab = [&]() {
+    int v = 0;
+    if (lane == 0) v = atomicAdd(next_s, 1);
+    return __shfl_sync(0xffffffffu, v, 0);
   };
-  const int mmin = items / kW;  // segments every warp has at least
-  const bool early = quota > 0 && mmin < kC1Ring + 2;
-  if (early && !share()) return;  // no copy in flight
-  const int M = quota > 0 && !early ? mmin - kC1Ring - 1 : -1;  // >= 1; segments M .. M + kC1Ring - 1 are own
-  auto stage_c = [&](int slot, int i) {  // this warp's i-th segment into a slot; always one group
-    const int it = warp + kW * i;
-    if (it < items) {
-      const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-      const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
-#pragma unroll
-      for (int u = 0; u < SU; ++u) {
-        const int ch = sg * kSegChunks + lane + 32 * u;
-        if (ch < nch_r8) cp_async16(cring + (size_t)slot * kC1SegBytes + (lane + 32 * u) * 16, row + (size_t)ch * 16);
-      }
+  auto avail = [&](int it) {  // 1: item `it` exists, 0: past the end, -1: abandoned
+    if (it < lim) return 1;
+    if (known) return 0;
+    int e = -1;  // the rebalancing's count: wait for warp 0 to publish it (bounded)
+    if (lane == 0) {
+      const uint64_t t0 = clock64();
+      while ((e = *reinterpret_cast<volatile int *>(ext_s)) == -1)
+        if ((uint64_t)(clock64() - t0) > 2 * kWaitCycles) {
+          latch_error(P.err, kErrTimeout);
+          e = -2;
+          break;
+        }
+      __threadfence_block();
     }
-    cp_async_commit();
+    e = __shfl_sync(0xffffffffu, e, 0);
+    __syncwarp();
+    if (e < 0) return -1;
+    known = true;
+    total = e;
+    nrows = e;
+    lim = e * per_row;
+    return it < lim ? 1 : 0;
   };
-#pragma unroll
-  for (int i = 0; i < kC1Ring; ++i) stage_c(i, i);
-#pragma unroll 1
-  for (int i = 0;; ++i) {
-    if (i == M && !share()) {  // every warp reaches iteration M with own segments left
-      cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-      return;
-    }
-    const int it = warp + kW * i;
-    if (it >= items) break;
-    const int slot = i % kC1Ring;
-    cp_async_wait<kC1Ring - 1>();  // this lane's chunks of segment i have landed
+  auto load_c = [&](uint4 *w, int it) {  // item `it` (which exists) into registers
     const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-    const unsigned char *sl = cring + (size_t)slot * kC1SegBytes;
+    const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
+#pragma unroll
+    for (int u = 0; u < SU; ++u) {
+      const int ch = sg * kSegChunks + lane + 32 * u;
+      if (ch < nch_r8) w[u] = ld_stream(row + (size_t)ch * 16);
+    }
+  };
+  auto sum_c = [&](const uint4 *w, int it) {  // its dot product into dots
+    const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
     float a = 0.f;
 #pragma unroll
     for (int u = 0; u < SU; ++u) {
       const int ch = sg * kSegChunks + lane + 32 * u;
       if (ch < nch_r8) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(sl + (lane + 32 * u) * 16);
         if (RB == 4)
-          a = dot_chunk_i4(w, xs, ch, a);
+          a = dot_chunk_i4(w[u], xs, ch, a);
         else if (RB == 8)
-          a = dot_chunk_i8(w, xs, ch, a);
+          a = dot_chunk_i8(w[u], xs, ch, a);
         else
-          a = dot_chunk_smem<T>(w, xs, ch, a);
+          a = dot_chunk_smem<T>(w[u], xs, ch, a);
       }
     }
-    stage_c(slot, i + kC1Ring);
     a = warp_sum(a);
     if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+  };
+  // Each warp's first two segments are requested before anything else (few rows: all of
+  // them), then C2's first rows: C1 reads into registers, so the staging region is free,
+  // and they land while C1 streams (rows shared out by the rebalancing come after the own
+  // rows; their stages follow C1).
+  const bool two = P.c1depth > 1;
+  int ia = grab(), ib = two ? grab() : 0;
+  int sa = ia < lim ? 1 : 2, sb = two ? (ib < lim ? 1 : 2) : 0;  // 2: not known yet
+  if (sa == 1) load_c(wa, ia);
+  if (sb == 1) load_c(wb, ib);
+  const int pre = min(min(DD, P.c2pre), own);
+#pragma unroll 1
+  for (int s = 0; s < pre; ++s) stage_d(s, s);
+  if (!known && warp == 0) {  // the split barrier's wait and the shared-out rows
+    int e = -2;
+    if (warp_grid_wait(P, target_s)) {
+      const int f = share_excess_warp(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 en) {
+        act_s[own + j] = en.x;
+        bias_s[own + j] = __int_as_float(en.y);
+      });
+      e = own + f;
+    }
+    if (lane == 0) {
+      __threadfence_block();  // the rows' entries before the count
+      *reinterpret_cast<volatile int *>(ext_s) = e;
+    }
+    __syncwarp();
   }
-  cp_async_wait<0>();
+  if (sa == 2) {
+    sa = avail(ia);
+    if (sa == 1) load_c(wa, ia);
+  }
+  if (sb == 2 && sa >= 0) {
+    sb = avail(ib);
+    if (sb == 1) load_c(wb, ib);
+  }
+  // two segments in flight (c1depth 2): while one is summed, the other's loads are
+  // outstanding; with one (sb stays 0), the next segment is requested after the sum
+#pragma unroll 1
+  while (sa > 0 || sb > 0) {
+    if (sa < 0 || sb < 0) break;
+    if (sa > 0) {
+      sum_c(wa, ia);
+      ia = grab();
+      sa = avail(ia);
+      if (sa > 0) load_c(wa, ia);
+    }
+    if (sb > 0 && sa >= 0) {
+      sum_c(wb, ib);
+      ib = grab();
+      sb = avail(ib);
+      if (sb > 0) load_c(wb, ib);
+    }
+  }
+  if (sa < 0 || sb < 0) {  // abandoned: the split barrier timed out (every warp sees it)
+    cp_async_wait<0>();
+    return;
+  }
   __syncthreads();
   for (int k = tid; k < total; k += kT) {
     float g = 0.f, u = 0.f;  // g: the ReLU'd projection (up for ReLU, gate for ReGLU)
@@ -401,7 +462,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
   }
   __syncthreads();
 #pragma unroll 1
-  for (int s = 0; s < DD; ++s) stage_d(s, s);  // C2's first stages (the ring is free again)
+  for (int s = pre; s < DD; ++s) stage_d(s, s);  // the rest of C2's first stages
 
   // ---------------------------------------------------------------- C2: down projection
   float acc[MAXM][V];
@@ -414,7 +475,13 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
       if (k < total) {
-        cp_async_wait<DD - 1>();  // this thread's chunks of row k have landed
+        switch (DD) {  // this thread's chunks of row k have landed
+          case 1: cp_async_wait<0>(); break;
+          case 2: cp_async_wait<1>(); break;
+          case 4: cp_async_wait<3>(); break;
+          case 8: cp_async_wait<7>(); break;
+          default: cp_async_wait<15>(); break;
+        }
         const float a = a_s[k];
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {

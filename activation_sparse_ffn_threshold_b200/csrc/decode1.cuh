@@ -15,11 +15,9 @@ constexpr int kDecodeSmemCap = 227 * 1024;  // opt-in dynamic shared memory of o
 
 // W_down rows in flight per thread in the down phase, by 16-byte chunks per thread and row
 __host__ __device__ constexpr int decode1_dstages(int maxm) { return maxm == 1 ? 8 : (maxm == 2 ? 4 : 2); }
-// The single-token kernel's down phase has the whole staging region (128 KB of rows).
+// The single-token kernel's down phase has the whole staging region (128 KB of rows): its
+// up/gate phase reads into registers.
 __host__ __device__ constexpr int decode1_c2stages(int maxm) { return maxm == 1 ? 16 : (maxm == 2 ? 8 : 4); }
-// Its up/gate phase streams 4 KB row segments through this many shared-memory slots per warp.
-constexpr int kC1Ring = 3;
-constexpr int kC1SegBytes = 4096;
 // 16-byte chunks of a d-vector per thread (1, 2 or 4)
 __host__ __device__ inline int decode1_maxm(int nch_d) {
   return nch_d <= kDecode1Threads ? 1 : (nch_d <= 2 * kDecode1Threads ? 2 : 4);
@@ -49,6 +47,12 @@ struct Decode1Params {
                      //   the sets are known (0: none); rank k is position k / G of tile k % G
   int32_t *set_pos;  // null, or [n]: tile c's active storage positions at [start(c), start(c) + cnt)
   int32_t *set_cnt;  //   and [G] their counts -- the set this launch used, for callers that ask
+  // The single-token kernel's request depths: more bytes in flight than keep HBM busy only
+  // queue, and delay the reads on the critical path (barrier polls, the hidden layer).
+  int bstages;   // B^T rows staged per warp (1, 2, 3, 4, 6 or 8)
+  int c2pre;     // W_down rows requested during C1 (0 .. the C2 stage count)
+  int c1depth;   // up/gate segments in flight per warp (1 or 2)
+  int c2stages;  // W_down rows in flight in C2 (1, 2, 4, 8 or 16; at most decode1_c2stages)
 };
 
 struct Decode1Layout {
@@ -57,22 +61,17 @@ struct Decode1Layout {
 
 __host__ __device__ inline size_t decode1_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Bytes of the staging region: B^T rows (phase B) and W_down chunks (C2) share it, and in
-// the single-token kernel (`ring`) the up/gate segments (C1) as well.
-__host__ __device__ inline size_t decode1_stage_bytes(const Decode1Params &P, bool ring = false) {
+// Bytes of the staging region: B^T rows (phase B) and W_down chunks (C2) share it; the
+// single-token kernel (`single`) stages more W_down rows than the others.
+__host__ __device__ inline size_t decode1_stage_bytes(const Decode1Params &P, bool single = false) {
   const int vec = P.dt == SFNN_F16 ? 8 : 4;
   const int maxm = decode1_maxm(P.d / vec);
-  const size_t bsz = (size_t)(kDecode1Threads / 32) * kDecode1BStages * (P.r / vec) * 16;
-  size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
-  if (ring) {
-    const size_t csz = (size_t)(kDecode1Threads / 32) * kC1Ring * kC1SegBytes;
-    const size_t c2 = (size_t)decode1_c2stages(maxm) * maxm * kDecode1Threads * 16;
-    dsz = csz > c2 ? csz : c2;
-  }
+  const size_t bsz = (size_t)(kDecode1Threads / 32) * (single ? P.bstages : kDecode1BStages) * (P.r / vec) * 16;
+  const size_t dsz = (size_t)(single ? decode1_c2stages(maxm) : decode1_dstages(maxm)) * maxm * kDecode1Threads * 16;
   return bsz > dsz ? bsz : dsz;
 }
 
-__host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P, bool ring = false) {
+__host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P, bool single = false) {
   const size_t esz = P.dt == SFNN_F16 ? 2 : 4;
   const size_t tm = (size_t)P.tile_max;
   Decode1Layout L;
@@ -97,13 +96,13 @@ __host__ __device__ inline Decode1Layout decode1_layout(const Decode1Params &P, 
   o = decode1_align(o + ((tm + 31) / 32) * 4 + 16, 16);
   L.wpref = o;  // exclusive prefix of the bit words' population counts
   o = decode1_align(o + ((tm + 31) / 32 + 1) * 4, 16);
-  L.bars = o;  // the active count, a flag, the split barrier's target
-  o = decode1_align(o + 16, 16);
+  L.bars = o;  // the active count, a flag, the split barrier's target, C1's item counter and row count
+  o = decode1_align(o + 32, 16);
   // The two staging areas share one region: B^T rows are staged only in phase B, the
   // W_down chunks only after it (the CTA synchronises in between).
   L.bstage = o;  // [warp][stage][chunk of the row]: B^T rows staged per warp
   L.dstage = o;  // [stage][chunk m][thread]: W_down chunks staged per thread
-  o = decode1_align(o + decode1_stage_bytes(P, ring), 16);
+  o = decode1_align(o + decode1_stage_bytes(P, single), 16);
   L.total = o;
   return L;
 }

@@ -81,6 +81,29 @@ __device__ __forceinline__ float dot_chunk_smem(const uint4 &w, const unsigned c
   return a;
 }
 
+// Two fp16 pairs (the halves of w and x, low half first) accumulated into a by sm_100's
+// mixed-precision FMA: it widens the fp16 operands exactly, their product is exact in fp32
+// and the sum is rounded once -- the result of widening first and fmaf, in one instruction.
+__device__ __forceinline__ float fma_h2(uint32_t w, uint32_t x, float a) {
+  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %1;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
+      : "+f"(a)
+      : "r"(w), "r"(x));
+  return a;
+}
+
+template <>
+__device__ __forceinline__ float dot_chunk_smem<__half>(const uint4 &w, const unsigned char *xs, int ch, float a) {
+  const uint4 x = *reinterpret_cast<const uint4 *>(xs + (size_t)ch * 16);
+  a = fma_h2(w.x, x.x, a);
+  a = fma_h2(w.y, x.y, a);
+  a = fma_h2(w.z, x.z, a);
+  return fma_h2(w.w, x.w, a);
+}
+
 // Grid barrier by thread 0, bracketed by CTA barriers; false (and the error latched)
 // if it timed out.  No separate fences: the CTA's writes happen before thread 0's
 // release add through the CTA barrier, and another CTA's reads after its thread 0's
@@ -182,47 +205,59 @@ __device__ __forceinline__ void column_sums(const float *part, int d, int G, flo
   }
 }
 
-// Rebalancing of a fused kernel's active rows, after the split barrier's wait: every
-// tile's count (P.bcnt, clamped to the tile), e_t = the rows past `quota`, and CTA c's
-// even share of them, the global excess rows [floor(cE/G), floor((c+1)E/G)) in tile
-// order -- row g is slot quota + g - epre[t] of the tile t with epre[t] <= g < epre[t+1].
-// `scratch` holds 2G + 3 ints of shared memory.  take(j, entry) receives the CTA's j-th
-// extra row's list entry (P.blist); returns the CTA's count of extra rows.  A function of
-// the counts alone: every CTA computes the same assignment.
-template <class Take>
-__device__ __forceinline__ int share_excess(const Decode1Params &P, int quota, int *scratch, Take take) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = P.G, c = blockIdx.x;
-  int *cnt_all = scratch, *epre = scratch + G, *ext = epre + G + 1;
-  for (int t = tid; t < G; t += blockDim.x) {
-    const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
-    cnt_all[t] = min(max(__ldcg(P.bcnt + t), 0), sz);
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int base = 0;
-    for (int wi = 0; wi < G; wi += 32) {
-      const int t = wi + lane;
-      const int e = t < G ? max(0, cnt_all[t] - quota) : 0;
-      int incl = e;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+// The split barrier's wait by one warp, so that the CTA's other warps keep working: lane 0
+// polls (bounded), and the warp's lanes read other CTAs' writes after the __syncwarp that
+// follows its acquire load.  false (and the error latched) if it timed out.
+__device__ __forceinline__ bool warp_grid_wait(const Decode1Params &P, const unsigned long long *slot) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    const uint64_t target = *slot;
+    const uint64_t t0 = clock64();
+    while (ld_acquire_gpu_u64(P.bar) < target)
+      if ((uint64_t)(clock64() - t0) > kWaitCycles) {
+        ok = false;
+        break;
       }
-      if (t < G) epre[t] = base + incl - e;
-      base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) {
-      epre[G] = base;
-      const int F = (int)(((int64_t)c * base) / G);
-      ext[0] = (int)(((int64_t)(c + 1) * base) / G) - F;
-      ext[1] = F;
-    }
+    if (!ok) latch_error(P.err, kErrTimeout);
   }
-  __syncthreads();
-  const int f = ext[0], F = ext[1];
-  for (int j = tid; j < f; j += blockDim.x) {
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// Rebalancing of a fused kernel's active rows, after the split barrier's wait, by one
+// warp: every tile's count (P.bcnt, clamped to the tile), e_t = the rows past `quota`,
+// and CTA c's even share of them, the global excess rows [floor(cE/G), floor((c+1)E/G))
+// in tile order -- row g is slot quota + g - epre[t] of the tile t with
+// epre[t] <= g < epre[t+1].  `scratch` holds G ints of shared memory.  take(j, entry)
+// receives the CTA's j-th extra row's list entry (P.blist); returns the CTA's count of
+// extra rows.  A function of the counts alone: every CTA computes the same assignment.
+template <class Take>
+__device__ __forceinline__ int share_excess_warp(const Decode1Params &P, int quota, int *scratch, Take take) {
+  const int lane = threadIdx.x & 31;
+  const int G = P.G, c = blockIdx.x;
+  int *epre = scratch;
+  int base = 0;
+  for (int wi = 0; wi < G; wi += 32) {
+    const int t = wi + lane;
+    int e = 0;
+    if (t < G) {
+      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
+      e = max(0, min(max(__ldcg(P.bcnt + t), 0), sz) - quota);
+    }
+    int incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (t < G) epre[t] = base + incl - e;
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  const int F = (int)(((int64_t)c * base) / G);
+  const int f = (int)(((int64_t)(c + 1) * base) / G) - F;
+  for (int j = lane; j < f; j += 32) {
     const int g = F + j;
     int lo = 0, hi = G;  // the largest t with epre[t] <= g
     while (hi - lo > 1) {
@@ -234,7 +269,21 @@ __device__ __forceinline__ int share_excess(const Decode1Params &P, int quota, i
     }
     take(j, __ldcg(P.blist + decode1_tile_start(lo, P.n, G) + quota + (g - epre[lo])));
   }
+  __syncwarp();
+  return f;
+}
+
+// The same by the whole CTA (warp 0 computes it; every thread returns the count, and the
+// entries taken are visible to all after it).  `scratch` holds G + 1 ints.
+template <class Take>
+__device__ __forceinline__ int share_excess(const Decode1Params &P, int quota, int *scratch, Take take) {
+  if (threadIdx.x < 32) {
+    const int f = share_excess_warp(P, quota, scratch + 1, take);
+    if (threadIdx.x == 0) scratch[0] = f;
+  }
   __syncthreads();
+  const int f = *reinterpret_cast<volatile int *>(scratch);
+  __syncthreads();  // every thread has read the count before the scratch is reused
   return f;
 }
 

@@ -69,6 +69,10 @@ def parse_args(argv=None):
     ap.add_argument("--order", choices=["dealt", "packed", "identity"], default="dealt",
                     help="storage order of the neurons: hotness ranks dealt round-robin to the SM tiles (default), "
                          "hot-packed-first, or the original order (no hotness profile)")
+    ap.add_argument("--fused-quota", type=int, default=-1,
+                    help="the single-token kernel's rebalancing quota (-1: the hotness profile's default)")
+    ap.add_argument("--fused-depths", default="",
+                    help="the single-token kernel's request depths 'bstages,c2pre,c1depth' (-1 keeps one)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--rows", choices=["native", "int8", "int4"], default="native",
                     help="storage of the FFN rows for the single-token line: the layer's dtype, or int8 / int4 "
@@ -438,6 +442,12 @@ def measure_single(cfg, args, dist, dev, rows=None, headline=False):
     # token: a layer too small for that, the tiny fp32 one, stays L2-resident anyway)
     R = args.replicas or min(T, max(2, 1 + math.ceil(2 * l2 / per_token)))
     handles = [sf.SparseFFN.from_layer(lay, device=dev, rows=rows, **_order_kw(args)) for _ in range(R)]
+    if args.fused_quota != -1:
+        for h in handles:
+            h.set_fused_quota(args.fused_quota)
+    if args.fused_depths:
+        for h in handles:
+            h.set_fused_depths(*[int(v) for v in args.fused_depths.split(",")])
     info = handles[0].info()
     torch.cuda.synchronize()
     X = torch.from_numpy(Xh).to(dev)
@@ -465,6 +475,10 @@ def measure_single(cfg, args, dist, dev, rows=None, headline=False):
            "avg_us": unit_us, "avg_of": "one token (one k_decode1 launch)", "replicas": R,
            "mean_active_neurons": float(counts.mean()), "gpu_launches": int(launches * args.steps),
            "clocks": clocks, "bytes_per_step": float(bytes_tok.sum())}
+    if args.fused_quota != -1:
+        out["fused_quota"] = args.fused_quota
+    if args.fused_depths:
+        out["fused_depths"] = args.fused_depths
     traffic, tsrc = (profiled_traffic(cfg.name) if rows is None else (None, None))
     out["roofline"] = roofline(float(bytes_tok.mean()), unit_us,
                                "k_decode1 (fused single-token decode), the only kernel the timed region launches; "

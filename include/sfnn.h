@@ -290,6 +290,19 @@ SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
 SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
 
 /*
+ * The single-token fused kernel's request depths (a tuning knob; the results do not depend
+ * on them): bstages = B^T rows staged per warp in phase B (1, 2, 3, 4, 6 or 8), c2pre =
+ * W_down rows requested while the up/gate rows stream (0 to 16), c1depth = up/gate segments
+ * in flight per warp (1 or 2), c2stages = W_down rows in flight in the down phase (1, 2, 4,
+ * 8 or 16, capped by the kernel's staging region: 16 when a W_down row is at most 8 KB,
+ * 8 up to 16 KB, else 4).  -1 keeps a value.  SFNN_ERR_INVALID_ARG for a value outside those sets;
+ * SFNN_ERR_UNSUPPORTED (nothing changed) when the kernel's shared memory would not fit or
+ * the layer has no fused kernel.  Takes effect at the next launch.
+ */
+SFNN_API sfnn_status sfnn_set_fused_depths(sfnn_handle h, int32_t bstages, int32_t c2pre, int32_t c1depth,
+                                           int32_t c2stages);
+
+/*
  * The fused few-token path (SFNN_BATCH_FUSED, and AUTO for 2 to 4 tokens) reads the
  * hot prefix of the layer densely (enabled by default): the neurons that the offline
  * hotness profile puts in a b-token batch's union with probability >= 0.99

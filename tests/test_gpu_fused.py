@@ -8,6 +8,8 @@
 * consecutive launches on the same handle (programmatic dependent launch lets
   the next one start early) stay correct and bitwise reproducible;
 * the residual stack runs through it;
+* its request depths (B^T stages, W_down rows requested early, up/gate segments in
+  flight) change nothing in the result: bitwise the same sets and y;
 * its rebalancing of active rows over the CTAs (forced quotas, on a hot-packed layer
   whose tiles hold very different counts; the wait for the shared-out rows before the
   own rows' stream and inside it) gives the same sets and y within rounding, reproducibly;
@@ -152,4 +154,28 @@ def test_rebalanced_rows_match(base, d, n, r, quota):
         assert np.array_equal(h.forward(xd).cpu().numpy(), y1)  # deterministic for a quota
         check_token(lay, X[t], y1, m1, f"{base} quota {quota} t={t}")
     h.set_fused_quota(-1)
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("base,d,n,r", [("70b_reglu", 8192, 5003, 1024), ("opt6.7b_relu", 4096, 9000, 1024),
+                                        ("tiny_relu_f32", 512, 2048, 64)])
+def test_request_depths_do_not_change_the_result(base, d, n, r):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=31)
+    h = sf.SparseFFN.from_layer(lay)
+    h.set_fused_quota(3)  # the rebalancing's wait runs beside the up/gate stream
+    X = W.make_tokens(cfg, 2, seed=32)
+    ref = [fused_step(h, dev(X[t])) for t in range(2)]
+    for depths in [(1, 0, 1, 1), (3, 16, 2, 16), (6, 2, 1, 2), (8, 5, 2, 4), (4, 8, 2, 8), (2, 4, 1, 8)]:
+        try:
+            h.set_fused_depths(*depths)
+        except RuntimeError as e:  # 8 stages of a 2 KB row do not fit beside a large x
+            assert "UNSUPPORTED" in str(e) and depths[0] == 8, e
+            continue
+        for t in range(2):
+            y, m = fused_step(h, dev(X[t]))
+            assert np.array_equal(m, ref[t][1]) and np.array_equal(y, ref[t][0]), depths
+    for bad in [(5, -1, -1, -1), (-1, 17, -1, -1), (-1, -1, 3, -1), (-1, -1, -1, 3)]:
+        with pytest.raises(RuntimeError):
+            h.set_fused_depths(*bad)
     assert h.get_error() == 0
