@@ -146,9 +146,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     if (ch < nch_d) *reinterpret_cast<uint4 *>(xs + (size_t)ch * 16) = xv[m];
   }
   __syncthreads();
-  // every warp requests its first DB B^T rows now (x has landed), behind its first A^T half row
+  // every warp requests its first two B^T rows now (x has landed), behind its first A^T half
+  // row, and the rest of its DB stages once its A^T rows have landed (more requests at once
+  // would only queue ahead of phase A's)
+  const int db0 = min(DB, 2);
 #pragma unroll 1
-  for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
+  for (int s = 0; s < db0; ++s) stage_b(s, warp + kW * s);
   // each half row's dot product (chunks ascending in one chain, then a butterfly sum) goes
   // to hbuf[half][j]; h_j = relu(first half + second half) is formed after the barrier
   for (int j = j0; j < r; j += G * (kW / 2)) {
@@ -171,6 +174,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     const float hs = warp_sum(acc);
     if (lane == 0) P.hbuf[(size_t)ahalf * r + j] = hs;
   }
+#pragma unroll 1
+  for (int s = db0; s < DB; ++s) stage_b(s, warp + kW * s);  // they land during the grid barrier
   // c and b of the tile into shared memory
   if (tid < tn) {
     c_s[tid] = to_f<T>(c_first);
