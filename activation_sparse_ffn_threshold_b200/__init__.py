@@ -86,6 +86,8 @@ def load_library():
         "sfnn_set_fused_decode": ([P, I], S),
         "sfnn_set_hot_prefix": ([P, I], S),
         "sfnn_set_fused_quota": ([P, I], S),
+        "sfnn_set_batch_quota": ([P, I], S),
+        "sfnn_set_batch_depths": ([P, I, I, I, I], S),
         "sfnn_set_fused_depths": ([P, I, I, I, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
@@ -263,6 +265,17 @@ class SparseFFN:
     def set_fused_quota(self, quota: int):
         """The single-token kernel's rebalancing quota (0: off; -1: the profile's default)."""
         _check(self._lib.sfnn_set_fused_quota(self._h, int(quota)), "sfnn_set_fused_quota")
+
+    def set_batch_depths(self, bstages: int = -1, c2pre: int = -1, c1depth: int = -1, c2stages: int = -1):
+        """The few-token kernel's request depths (B^T half rows per warp, W_down rows requested
+        during the up/gate stream, up/gate segments in flight per warp, W_down rows in flight
+        in the down phase); -1 keeps a value."""
+        _check(self._lib.sfnn_set_batch_depths(self._h, int(bstages), int(c2pre), int(c1depth), int(c2stages)),
+               "sfnn_set_batch_depths")
+
+    def set_batch_quota(self, enable: bool):
+        """The few-token kernel's rebalancing (off: each token's y independent of the batch)."""
+        _check(self._lib.sfnn_set_batch_quota(self._h, 1 if enable else 0), "sfnn_set_batch_quota")
 
     def set_fused_depths(self, bstages: int = -1, c2pre: int = -1, c1depth: int = -1, c2stages: int = -1):
         """The single-token kernel's request depths (B^T stages per warp, W_down rows requested

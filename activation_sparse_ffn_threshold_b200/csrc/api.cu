@@ -137,7 +137,11 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
     P.set_pos = sets ? reinterpret_cast<int32_t *>(h->acoef) : nullptr;
     P.set_cnt = sets ? h->scnt : nullptr;
     P.hot = h->hot_on ? h->hot_rows[b] : 0;
-    P.quota = h->quota_multi[b];
+    P.quota = h->batch_quota_off ? 0 : h->quota_multi[b];
+    P.bstages = h->mdepth[0];
+    P.c2pre = h->mdepth[1];
+    P.c1depth = h->mdepth[2];
+    P.c2stages = h->mdepth[3];
     SFNN_TRY(launch_decode_multi(P, b, s, true));
     record_if(after, s);
     if (sets)
@@ -175,11 +179,6 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
   h->launches += 4 + (predict ? 2 : (src == kSetGiven ? 1 : 0)) + ((idx_out || cnt_out) ? 1 : 0);
   return SFNN_OK;
 }
-
-// The few-token kernel's rebalancing of union rows over the CTAs: measured slower than
-// each CTA taking its own tile's union rows (70B-shaped layer, 2 tokens: 98.5 against
-// 92.6 us per batch), so it is off.
-constexpr bool kMultiRebalance = false;
 
 // The fused single-token kernel's plan: one CTA per SM, each owning a contiguous tile of
 // neurons; h is held in registers (at most 4 chunks per lane), all CTAs must be resident.
@@ -226,9 +225,17 @@ void plan_decode1(sfnn_ctx *h, int G) {
   h->fused_ok = true;
   h->fused_on = true;
   // the multi-token kernel: the largest batch (up to 4) whose plan fits, with its prefix
+  // the few-token kernel's request depths (measured best on the 70B-shaped layer at 2 and
+  // 4 tokens and the OPT-30B-shaped one at 2: within 1% of each other, and 9% over 6
+  // half rows with 2 segments in flight at 4 tokens)
+  h->mdepth[0] = 4;  // B^T half rows per warp
+  h->mdepth[1] = 2;
+  h->mdepth[2] = 1;
+  h->mdepth[3] = 4;
   for (int nb = std::min(h->max_batch, kMultiMaxTokens); nb >= 2; --nb) {
     Decode1Params Q = P;
     Q.hot = h->hot_rows[nb];
+    Q.bstages = h->mdepth[0];
     if (decode_multi_blocks_per_sm(Q, nb) >= 1) {
       h->multi_max = nb;
       break;
@@ -401,8 +408,11 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       const double p = std::isnan(q) ? 0.0 : std::min(1.0, std::max(0.0, (double)q));
       u += 1.0 - std::pow(1.0 - p, b);
     }
-    const int qv = std::max((int)std::floor(0.8 * u / G), (h->hot_rows[b] + G - 1) / G);
-    h->quota_multi[b] = kMultiRebalance && qv >= 2 ? qv : 0;
+    // as the single-token kernel's: 0.9 of a tile's expected union count when the own
+    // rows' up/gate bytes reach 96 KB, and never below the tile's hot prefix
+    const double elem = L.dt == SFNN_F16 ? 2.0 : 4.0;
+    const int qv = std::max((int)std::floor(0.9 * u / G), (h->hot_rows[b] + G - 1) / G);
+    h->quota_multi[b] = qv * (L.nproj - 1) * (double)L.d * elem >= 96.0 * 1024 ? qv : 0;
   }
   if (desc->hotness) {
     for (int b = 1; b <= kMaxBatch; ++b) {
@@ -631,6 +641,29 @@ sfnn_status sfnn_set_fused_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
   if (c2stages != -1) P.c2stages = c2stages;
   if (decode1_blocks_per_sm(P) < 1) return SFNN_ERR_UNSUPPORTED;
   h->d1 = P;
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre, int32_t c1depth,
+                                  int32_t c2stages) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (bstages != -1 && bstages != 2 && bstages != 4 && bstages != 6 && bstages != 8) return SFNN_ERR_INVALID_ARG;
+  if (c2pre < -1 || c2pre > 8 || c1depth < -1 || c1depth == 0 || c1depth > 2) return SFNN_ERR_INVALID_ARG;
+  if (c2stages != -1 && c2stages != 1 && c2stages != 2 && c2stages != 4 && c2stages != 8) return SFNN_ERR_INVALID_ARG;
+  if (h->multi_max < 2) return SFNN_ERR_UNSUPPORTED;
+  Decode1Params Q = h->d1;
+  Q.hot = h->hot_rows[h->multi_max];
+  Q.bstages = bstages != -1 ? bstages : h->mdepth[0];
+  if (decode_multi_blocks_per_sm(Q, h->multi_max) < 1) return SFNN_ERR_UNSUPPORTED;
+  const int v[4] = {bstages, c2pre, c1depth, c2stages};
+  for (int i = 0; i < 4; ++i)
+    if (v[i] != -1) h->mdepth[i] = v[i];
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  h->batch_quota_off = enable == 0;
   return SFNN_OK;
 }
 

@@ -59,6 +59,8 @@ struct sfnn_ctx {
   int32_t *bcnt;     // [G]   and their counts (single-token fused kernel)
   int quota;         // its per-CTA quota of own rows (0: no rebalancing)
   int quota_multi[sfnn::kMultiMaxTokens + 1];  // the same for the multi-token kernel, by batch size
+  bool batch_quota_off;  // the multi-token kernel's rebalancing switched off (batch-invariant rows)
+  int mdepth[4];         // the multi-token kernel's request depths (bstages, c2pre, c1depth, c2stages)
   int32_t *scnt;     // [max_batch][G] per-tile counts of the sets a fused launch used (lists: ulist
                      //   for one token, acoef's words for several)
   int multi_max;     // largest batch the multi-token fused kernel serves (0: none)

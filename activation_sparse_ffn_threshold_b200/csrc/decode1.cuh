@@ -183,11 +183,11 @@ __host__ __device__ inline MultiLayout decode_multi_layout(const Decode1Params &
   o = decode1_align(o + words * 4 + 16, 16);
   L.wpref = o;
   o = decode1_align(o + (words + 1) * 4, 16);
-  L.bars = o;  // the union count, a flag, the split barrier's target
-  o = decode1_align(o + 16, 16);
+  L.bars = o;  // the union count, a flag, the split barrier's target, C1's item counter and row count
+  o = decode1_align(o + 32, 16);
   L.stage = o;
   const int maxm = decode1_maxm(P.d / vec);
-  const size_t bsz = (size_t)(kDecode1Threads / 32) * kMultiBStages * 64 * 16;  // 2 chunks per lane and stage
+  const size_t bsz = (size_t)(kDecode1Threads / 32) * P.bstages * 64 * 16;  // 2 chunks per lane and stage
   const size_t dsz = (size_t)decode1_dstages(maxm) * maxm * kDecode1Threads * 16;
   o = decode1_align(o + (bsz > dsz ? bsz : dsz), 16);
   L.total = o;

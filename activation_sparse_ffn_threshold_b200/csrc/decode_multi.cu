@@ -33,7 +33,6 @@
 namespace sfnn {
 namespace {
 
-constexpr int kMB = kMultiBStages;
 
 __device__ __forceinline__ void unpack2(const uint4 &v, float2 (&f)[4]) {
   const __half2 *h = reinterpret_cast<const __half2 *>(&v);
@@ -41,19 +40,33 @@ __device__ __forceinline__ void unpack2(const uint4 &v, float2 (&f)[4]) {
   for (int i = 0; i < 4; ++i) f[i] = __half22float2(h[i]);
 }
 
-// acc[t] += w . x_t over one 16-byte chunk (8 elements), for the tokens in `tok`
+// a.x += w.lo x.lo and a.y += w.hi x.hi for one fp16 pair each, by sm_100's mixed-precision
+// FMA (the fp16 operands widen exactly and the product is exact in fp32: the result of
+// widening first and a packed fp32 FMA, without the conversions)
+__device__ __forceinline__ float2 fma_pair_h(uint32_t w, uint32_t x, float2 a) {
+  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.f16 %1, wh, xh, %1;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "r"(w), "r"(x));
+  return a;
+}
+
+// acc[t] += w . x_t over one 16-byte chunk (8 elements), for the tokens in `tok`: even
+// elements into acc[t].x, odd ones into acc[t].y, in element order
 template <int NB>
 __device__ __forceinline__ void dot_tokens(const uint4 &w, const unsigned char *xs, size_t tstride, int ch,
                                            uint32_t tok, float2 (&acc)[NB]) {
-  float2 wf[4];
-  unpack2(w, wf);
 #pragma unroll
   for (int t = 0; t < NB; ++t) {
     if ((tok >> t) & 1u) {
-      float2 xf[4];
-      unpack2(*reinterpret_cast<const uint4 *>(xs + t * tstride + (size_t)ch * 16), xf);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[t] = __ffma2_rn(wf[i], xf[i], acc[t]);
+      const uint4 x = *reinterpret_cast<const uint4 *>(xs + t * tstride + (size_t)ch * 16);
+      acc[t] = fma_pair_h(w.x, x.x, acc[t]);
+      acc[t] = fma_pair_h(w.y, x.y, acc[t]);
+      acc[t] = fma_pair_h(w.z, x.z, acc[t]);
+      acc[t] = fma_pair_h(w.w, x.w, acc[t]);
     }
   }
 }
@@ -62,7 +75,8 @@ template <int NB, int ACT, int MAXM>
 __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   constexpr int V = 8;   // fp16 elements per 16-byte chunk
   constexpr int MH = 2;  // chunks of a half row of B^T per lane (r <= 1024)
-  constexpr int DD = decode1_dstages(MAXM);
+  const int DD = min(P.c2stages, decode1_dstages(MAXM));  // W_down rows in flight: 1, 2, 4 or 8
+  const int kMB = P.bstages;                               // B^T half rows per warp: 2, 4, 6 or 8
   constexpr uint32_t ALL = (1u << NB) - 1u;
   extern __shared__ __align__(16) unsigned char smem[];
   const MultiLayout L = decode_multi_layout(P, NB);
@@ -83,6 +97,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
   unsigned long long *target_s = reinterpret_cast<unsigned long long *>(cnt_s + 2);
+  int *next_s = cnt_s + 4;  // C1's next work item
+  int *ext_s = cnt_s + 5;   // C1's final row count once known (-1: not yet, -2: abandoned)
   unsigned char *stage = smem + L.stage;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -140,12 +156,22 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
     cp_async_commit();
   };
   pdl_wait();  // X (and every buffer this kernel writes) belongs to earlier kernels until here
-  for (int i = tid; i < NB * nch_d; i += kT)
-    *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
-        __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+  {
+    uint4 xv[NB * MAXM];  // every load of X in flight at once, then into shared memory
+#pragma unroll
+    for (int m = 0; m < NB * MAXM; ++m) {
+      const int i = tid + kT * m;
+      if (i < NB * nch_d) xv[m] = __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+    }
+#pragma unroll
+    for (int m = 0; m < NB * MAXM; ++m) {
+      const int i = tid + kT * m;
+      if (i < NB * nch_d) *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) = xv[m];
+    }
+  }
   __syncthreads();
   if (j0 >= r) {
-#pragma unroll
+#pragma unroll 1
     for (int s = 0; s < kMB; ++s) stage_b(s, pair + kPairs * s);
   }
   // each token's half-row sums go to hbuf[t][half][j]; h is formed after the barrier
@@ -175,7 +201,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
     }
   }
   if (j0 < r) {
-#pragma unroll
+#pragma unroll 1
     for (int s = 0; s < kMB; ++s) stage_b(s, pair + kPairs * s);
   }
   if (tid < tn) {
@@ -253,7 +279,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
       for (int s = 0; s < kMB; ++s) {
         const int p = pb + kPairs * s;
         if (p < tn) {
-          cp_async_wait<kMB - 1>();  // this lane's copies of neuron p's half row have landed
+          switch (kMB) {  // this lane's copies of neuron p's half row have landed
+            case 2: cp_async_wait<1>(); break;
+            case 4: cp_async_wait<3>(); break;
+            case 6: cp_async_wait<5>(); break;
+            default: cp_async_wait<7>(); break;
+          }
           float2 a[NB];
 #pragma unroll
           for (int t = 0; t < NB; ++t) a[t] = make_float2(0.f, 0.f);
@@ -312,7 +343,11 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
       if (wi + lane < words) wpref[wi + lane] = base + incl - k;
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) *cnt_s = base;
+    if (lane == 0) {
+      *cnt_s = base;
+      *next_s = 0;
+      *ext_s = -1;
+    }
   } else if (P.set_pos && warp <= NB) {  // token (warp - 1)'s own set, for callers that ask
     const int t = warp - 1;
     int base = 0;
@@ -353,8 +388,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   const int cnt = *cnt_s;
   // Rebalancing, as in the single-token kernel: each CTA keeps its first `quota` union rows
   // (at least its hot prefix, whose dots only it holds), publishes its list (position |
-  // token mask << 24, b) and arrives on a split grid barrier; after its own rows' dots it
-  // takes an even share of all tiles' rows past the quota.
+  // token mask << 24, b) and arrives on a split grid barrier; one warp waits on it beside
+  // the own rows' stream, and the CTA takes an even share of all tiles' rows past the quota.
   const int quota = P.quota;
   if (quota > 0) {
     for (int k = tid; k < cnt; k += kT)
@@ -379,81 +414,122 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   };
 
   // ---------------------------------------------------------------- C1: gate / up dots
-  // rows [kb, ke) after the prefix in one or two passes (the own rows, then the rows
-  // shared out by the rebalancing), their segments over all warps, 2-deep register
-  // pipeline, dots only for the tokens active on each row; the first pass requests `pre`
-  // stages of C2 behind its first loads
-  const int pre = quota > 0 ? min(DD, own) : DD;
+  // The union rows after the hot prefix, [kp, total): their 4 KB segments are work items
+  // handed out in order by a shared counter, loaded into registers (no L1 allocation), dots
+  // only for the tokens active on each row; a warp keeps c1depth segments in flight.  A
+  // segment's dots do not depend on the warp that computes them.  C2's first rows are
+  // requested behind each warp's first segments; with rebalancing, warp 0 waits on the
+  // split barrier beside the stream and appends the rows shared out to this CTA.
   int total = own;
-  for (int pass = 0, kb = kp, ke = own; pass < (quota > 0 ? 2 : 1); ++pass) {
-    if (pass == 1) {
-      if (!cta_grid_wait(P, target_s, flag_s)) {
-        cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-        return;
+  int lim = (own - kp) * per_row;  // items known to exist
+  bool known = quota == 0;         // the final count is known
+  uint4 wa[SU], wb[SU];
+  auto grab = [&]() {
+    int v = 0;
+    if (lane == 0) v = atomicAdd(next_s, 1);
+    return __shfl_sync(0xffffffffu, v, 0);
+  };
+  auto avail = [&](int it) {  // 1: item `it` exists, 0: past the end, -1: abandoned
+    if (it < lim) return 1;
+    if (known) return 0;
+    int e = -1;  // the rebalancing's count: wait for warp 0 to publish it (bounded)
+    if (lane == 0) {
+      const uint64_t t0c = clock64();
+      while ((e = *reinterpret_cast<volatile int *>(ext_s)) == -1)
+        if ((uint64_t)(clock64() - t0c) > 2 * kWaitCycles) {
+          latch_error(P.err, kErrTimeout);
+          e = -2;
+          break;
+        }
+      __threadfence_block();
+    }
+    e = __shfl_sync(0xffffffffu, e, 0);
+    __syncwarp();
+    if (e < 0) return -1;
+    known = true;
+    total = e;
+    nrows = e;
+    lim = (e - kp) * per_row;
+    return it < lim ? 1 : 0;
+  };
+  auto load_c = [&](uint4 *w, int it) {  // item `it` (which exists) into registers
+    const int k = kp + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+    const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
+#pragma unroll
+    for (int u = 0; u < SU; ++u) {
+      const int ch = sg * kSegChunks + lane + 32 * u;
+      if (ch < nch_d) w[u] = ld_stream(row + (size_t)ch * 16);
+    }
+  };
+  auto sum_c = [&](const uint4 *w, int it) {  // its dots into dots, for the row's tokens
+    const int k = kp + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+    const uint32_t tm = tok_s[k];
+    float2 acc[NB];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) acc[t] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < SU; ++u) {
+      const int ch = sg * kSegChunks + lane + 32 * u;
+      if (ch < nch_d) dot_tokens<NB>(w[u], xs, xstride, ch, tm, acc);
+    }
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+      if ((tm >> t) & 1u) {  // warp-uniform: the item's row is the warp's
+        const float v = warp_sum(acc[t].x + acc[t].y);
+        if (lane == 0) dots[(((size_t)k * 2 + pj) * nseg + sg) * NB + t] = v;
       }
-      const int f = share_excess(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 e) {
-        act_s[own + j] = e.x & 0xFFFFFF;
-        tok_s[own + j] = (uint32_t)e.x >> 24;
-        bias_s[own + j] = __int_as_float(e.y);
+    }
+  };
+  const bool two = P.c1depth > 1;
+  int ia = grab(), ib = two ? grab() : 0;
+  int sa = ia < lim ? 1 : 2, sb = two ? (ib < lim ? 1 : 2) : 0;  // 2: not known yet
+  if (sa == 1) load_c(wa, ia);
+  if (sb == 1) load_c(wb, ib);
+  const int pre = min(min(DD, P.c2pre), own);
+  for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's first loads, which gate C2
+  if (!known && warp == 0) {  // the split barrier's wait and the shared-out rows
+    int e = -2;
+    if (warp_grid_wait(P, target_s)) {
+      const int f = share_excess_warp(P, quota, reinterpret_cast<int *>(red2), [&](int j, int2 en) {
+        act_s[own + j] = en.x & 0xFFFFFF;
+        tok_s[own + j] = (uint32_t)en.x >> 24;
+        bias_s[own + j] = __int_as_float(en.y);
       });
-      total = own + f;
-      nrows = total;
-      kb = own;
-      ke = total;
+      e = own + f;
     }
-    constexpr int D = 2;
-    const int items = (ke - kb) * per_row;
-    uint4 wc[D][SU];
-#pragma unroll
-    for (int s = 0; s < D; ++s) {
-      const int it = warp + kW * s;
-      if (it < items) {
-        const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-        const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
-#pragma unroll
-        for (int u = 0; u < SU; ++u) {
-          const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * 16);
-        }
-      }
+    if (lane == 0) {
+      __threadfence_block();  // the rows' entries before the count
+      *reinterpret_cast<volatile int *>(ext_s) = e;
     }
-    if (pass == 0)
-      for (int s = 0; s < pre; ++s) stage_d(s, s);  // behind C1's loads, which gate C2
-    for (int ib = warp; ib < items; ib += D * kW) {
-#pragma unroll
-      for (int s = 0; s < D; ++s) {
-        const int it = ib + kW * s;
-        if (it < items) {
-          const int k = kb + it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
-          const uint32_t tm = tok_s[k];
-          float2 acc[NB];
-#pragma unroll
-          for (int t = 0; t < NB; ++t) acc[t] = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int u = 0; u < SU; ++u) {
-            const int ch = sg * kSegChunks + lane + 32 * u;
-            if (ch < nch_d) dot_tokens<NB>(wc[s][u], xs, xstride, ch, tm, acc);
-          }
-          const int itn = it + D * kW;
-          if (itn < items) {
-            const int kn = kb + itn / per_row, pjn = (itn % per_row) / nseg, sgn = itn % per_row - pjn * nseg;
-            const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
-#pragma unroll
-            for (int u = 0; u < SU; ++u) {
-              const int ch = sgn * kSegChunks + lane + 32 * u;
-              if (ch < nch_d) wc[s][u] = ld_stream(row + (size_t)ch * 16);
-            }
-          }
-#pragma unroll
-          for (int t = 0; t < NB; ++t) {
-            if ((tm >> t) & 1u) {  // warp-uniform: the item's row is the warp's
-              const float v = warp_sum(acc[t].x + acc[t].y);
-              if (lane == 0) dots[(((size_t)k * 2 + pj) * nseg + sg) * NB + t] = v;
-            }
-          }
-        }
-      }
+    __syncwarp();
+  }
+  if (sa == 2) {
+    sa = avail(ia);
+    if (sa == 1) load_c(wa, ia);
+  }
+  if (sb == 2 && sa >= 0) {
+    sb = avail(ib);
+    if (sb == 1) load_c(wb, ib);
+  }
+#pragma unroll 1
+  while (sa > 0 || sb > 0) {
+    if (sa < 0 || sb < 0) break;
+    if (sa > 0) {
+      sum_c(wa, ia);
+      ia = grab();
+      sa = avail(ia);
+      if (sa > 0) load_c(wa, ia);
     }
+    if (sb > 0 && sa >= 0) {
+      sum_c(wb, ib);
+      ib = grab();
+      sb = avail(ib);
+      if (sb > 0) load_c(wb, ib);
+    }
+  }
+  if (sa < 0 || sb < 0) {  // abandoned: the split barrier timed out (every warp sees it)
+    cp_async_wait<0>();
+    return;
   }
   __syncthreads();
   for (int e = tid; e < total * NB; e += kT) {
@@ -488,7 +564,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
     for (int s = 0; s < DD; ++s) {
       const int k = kb + s;
       if (k < total) {
-        cp_async_wait<DD - 1>();  // this thread's chunks of row k have landed
+        switch (DD) {  // this thread's chunks of row k have landed
+          case 1: cp_async_wait<0>(); break;
+          case 2: cp_async_wait<1>(); break;
+          case 4: cp_async_wait<3>(); break;
+          default: cp_async_wait<7>(); break;
+        }
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
           if (tid + kT * m < nch_d) {

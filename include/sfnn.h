@@ -290,6 +290,28 @@ SFNN_API sfnn_status sfnn_set_fused_decode(sfnn_handle h, int32_t enable);
 SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
 
 /*
+ * The few-token fused kernel's rebalancing of union rows over its CTAs (on by default when
+ * the hotness profile makes it pay, as the single-token kernel's).  With it, the CTA that
+ * sums a row into its partial depends on the other tokens' sets, so a token's y can differ
+ * in rounding with the batch it is in (still deterministic for a given batch); enable = 0
+ * switches it off, and each token's y then does not depend on the other tokens at all.
+ * Takes effect at the next launch.
+ */
+SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
+
+/*
+ * The few-token fused kernel's request depths, as sfnn_set_fused_depths (the results do not
+ * depend on them): bstages = B^T half rows staged per warp (2, 4, 6 or 8), c2pre = W_down
+ * rows requested while the up/gate rows stream (0 to 8), c1depth = up/gate segments in
+ * flight per warp (1 or 2), c2stages = W_down rows in flight (1, 2, 4 or 8, capped by the
+ * staging region: 8 when a W_down row is at most 8 KB, else 4).  -1 keeps a value.
+ * SFNN_ERR_INVALID_ARG outside those sets; SFNN_ERR_UNSUPPORTED (nothing changed) when the
+ * kernel's shared memory would not fit or the handle has no few-token kernel.
+ */
+SFNN_API sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre, int32_t c1depth,
+                                           int32_t c2stages);
+
+/*
  * The single-token fused kernel's request depths (a tuning knob; the results do not depend
  * on them): bstages = B^T rows staged per warp in phase B (1, 2, 3, 4, 6 or 8), c2pre =
  * W_down rows requested while the up/gate rows stream (0 to 16), c1depth = up/gate segments

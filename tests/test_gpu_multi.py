@@ -5,10 +5,13 @@
   ragged n, d up to 8192 and 2, 3 or 4 tokens;
 * it agrees with the tensor-core path within the tolerance, is bitwise reproducible,
   and its set output changes nothing (the plain call gives bitwise the same Y);
-* a token's row of Y does not depend on which other tokens share the batch (a row
-  applies only to the tokens whose sets hold it);
+* with the rebalancing of union rows over the CTAs switched off, a token's row of Y does
+  not depend on which other tokens share the batch (a row applies only to the tokens
+  whose sets hold it); with it on (the full-size 70B-shaped layer), the sets are the
+  same, Y agrees within rounding and is bitwise reproducible for a given batch;
 * AUTO takes it for 2 to 4 tokens on the full OPT-30B- and 70B-shaped layers, and the
   residual stack runs through it;
+* its request depths change nothing in the result (bitwise the same Y and sets);
 * outputs stay inside their buffers (canary words on both sides).
 """
 import numpy as np
@@ -75,6 +78,7 @@ def test_rows_do_not_depend_on_the_other_tokens():
     lay = W.make_layer(cfg, seed=73)
     h = sf.SparseFFN.from_layer(lay, max_batch=4)
     h.set_batch_path(sf.BATCH_FUSED)
+    h.set_batch_quota(False)
     X = W.make_tokens(cfg, 6, seed=74)
     Ya, ma = run_multi(h, X[[0, 1, 2, 3]])
     Yb, mb = run_multi(h, X[[4, 0, 5]])
@@ -97,6 +101,26 @@ def test_multi_full_size_auto(name, batches):
         Y, masks = run_multi(h, X)
         for t in range(b):
             check_token(lay, X[t], Y[t], masks[t], f"{name} b={b} t={t}")
+    assert h.get_error() == 0
+    del h
+    torch.cuda.empty_cache()
+
+
+def test_rebalanced_union_rows():
+    cfg = W.CONFIGS["70b_reglu"]
+    lay = W.make_layer(cfg, seed=0)
+    h = sf.SparseFFN.from_layer(lay, max_batch=2)
+    h.set_batch_path(sf.BATCH_FUSED)
+    X = W.make_tokens(cfg, 2, seed=80)
+    Y_on, m_on = run_multi(h, X)
+    assert np.array_equal(run_multi(h, X)[0], Y_on)  # deterministic for a given batch
+    h.set_batch_quota(False)
+    Y_off, m_off = run_multi(h, X)
+    h.set_batch_quota(True)
+    assert all(np.array_equal(a, c) for a, c in zip(m_on, m_off))
+    for t in range(2):
+        assert oracle.within_tolerance(Y_on[t].astype(np.float64), Y_off[t].astype(np.float64))[0]
+        check_token(lay, X[t], Y_on[t], m_on[t], f"70b b=2 rebalanced t={t}")
     assert h.get_error() == 0
     del h
     torch.cuda.empty_cache()
@@ -145,3 +169,26 @@ def test_hot_prefix_changes_nothing(base):
     for t in range(3):
         check_token(lay, X[t], Y[t], masks[t], f"{base} identity order t={t}")
     assert h.get_error() == 0 and h0.get_error() == 0
+
+
+@pytest.mark.parametrize("base,d,n,r", [("70b_reglu", 8192, 5003, 1024), ("opt6.7b_relu", 4096, 9000, 1024)])
+def test_batch_request_depths_do_not_change_the_result(base, d, n, r):
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=33)
+    h = sf.SparseFFN.from_layer(lay, max_batch=3)
+    h.set_batch_path(sf.BATCH_FUSED)
+    X = W.make_tokens(cfg, 3, seed=34)
+    ref = run_multi(h, X)
+    for depths in [(2, 0, 1, 1), (4, 8, 2, 2), (8, 1, 1, 8), (6, 4, 2, 4)]:
+        try:
+            h.set_batch_depths(*depths)
+        except RuntimeError as e:  # 8 W_down stages of 16 KB rows, or 8 B^T stages, may not fit
+            assert "UNSUPPORTED" in str(e) or "INVALID" in str(e), e
+            continue
+        Y, m = run_multi(h, X)
+        assert np.array_equal(Y, ref[0]), depths
+        assert all(np.array_equal(a, c) for a, c in zip(m, ref[1])), depths
+    for bad in [(3, -1, -1, -1), (-1, 9, -1, -1), (-1, -1, 0, -1), (-1, -1, -1, 16)]:
+        with pytest.raises(RuntimeError):
+            h.set_batch_depths(*bad)
+    assert h.get_error() == 0
