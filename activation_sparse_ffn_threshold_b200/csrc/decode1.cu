@@ -174,8 +174,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     const float hs = warp_sum(acc);
     if (lane == 0) P.hbuf[(size_t)ahalf * r + j] = hs;
   }
-#pragma unroll 1
-  for (int s = db0; s < DB; ++s) stage_b(s, warp + kW * s);  // they land during the grid barrier
   // c and b of the tile into shared memory
   if (tid < tn) {
     c_s[tid] = to_f<T>(c_first);
@@ -185,7 +183,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode1(const Decode1Params P) {
     c_s[i] = to_f<T>(cp[t0 + i]);
     a_s[i] = to_f<T>(bp[t0 + i]);
   }
-  if (!cta_grid_sync(P, flag_s)) {
+  cta_grid_arrive(P, target_s);
+  // the rest of the first DB B^T rows go out after the arrival (its release would otherwise
+  // wait for them to land), and land during the barrier
+#pragma unroll 1
+  for (int s = db0; s < DB; ++s) stage_b(s, warp + kW * s);
+  if (!cta_grid_wait(P, target_s, flag_s)) {
     cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     return;
   }

@@ -8,11 +8,12 @@
 // halves (one CTA of 16 warps per SM, as the single-layer kernel):
 //
 //   P1  u_l, and the active lists of layer l (written by the previous launch), into
-//       shared memory; h' = relu(A'^T u_l) for the CTA's rows of layer l+1's A' (one warp
-//       per row, its first batch requested before the previous kernel ends); C1 / C2 on
-//       the CTA's share of layer l's active rows, as in the single-layer kernel; the
-//       CTA's partial y to global memory; the first B'^T rows of layer l+1's tile
-//       requested into the staging region C2 has left.
+//       shared memory; C1 / C2 on the CTA's share of layer l's active rows, as in the
+//       single-layer kernel; h' = relu(A'^T u_l) for the CTA's rows of layer l+1's A'
+//       (one warp per row, its first batch requested during C2: h' is needed only after
+//       the barrier, while C1 needs only the lists); the CTA's partial y to global
+//       memory; the first B'^T rows of layer l+1's tile requested into the staging
+//       region C2 has left, after the barrier's arrival.
 //   grid barrier (the launch's only one)
 //   P2  the fixed-order column reduce of the partials -> y_l (+ residual), u_{l+1};
 //       z' = B'^T h' + c' on layer l+1's tile -> its active list, kept in global memory
@@ -60,6 +61,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   int *cnt_s = reinterpret_cast<int *>(smem + L.bars);
   int *flag_s = cnt_s + 1;
   int *ncnt_s = cnt_s + 2;
+  unsigned long long *target_s = reinterpret_cast<unsigned long long *>(cnt_s + 4);  // the barrier's target
   unsigned char *bstage = smem + L.bstage;
   unsigned char *dstage = smem + L.dstage;
 
@@ -80,14 +82,9 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   pdl_launch_dependents();
   const int j0 = c + G * warp;  // this warp's first row of A'^T
 
-  // Weights only until griddepcontrol.wait: the first batch of the warp's row of A'^T,
-  // and c', b' at tile position tid.
-  uint4 w0[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int ch = lane + 32 * u;
-    if (next && j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
-  }
+  // Before griddepcontrol.wait only c', b' at tile position tid (weights); after it, u_l
+  // and this layer's lists are requested first (they gate everything), then the first
+  // batch of the warp's row of A'^T.
   const T *cp = static_cast<const T *>(Q.cvec);
   const T *bp = static_cast<const T *>(Q.bias);
   T c_first = from_f<T>(0.f), b_first = from_f<T>(0.f);
@@ -98,9 +95,21 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   for (int i = tid; i < (Q.tile_max + 31) / 32; i += kT) bits[i] = 0u;
 
   pdl_wait();  // u_l, this layer's lists and every buffer written here belong to earlier kernels until here
-  for (int i = tid; i < nch_d; i += kT)
-    *reinterpret_cast<uint4 *>(xs + (size_t)i * 16) =
-        __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)i * 16));
+  uint4 xv[MAXM];
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    const int ch = tid + kT * m;
+    if (ch < nch_d) xv[m] = __ldcg(reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(P.x) + (size_t)ch * 16));
+  }
+  int2 l_first = make_int2(0, 0);
+  int c_tile = 0;
+  if (cur && tid < tn) l_first = __ldcg(Q.list_in + t0 + tid);
+  if (cur && tid < G) c_tile = __ldcg(Q.cnt_in + tid);
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    const int ch = tid + kT * m;
+    if (ch < nch_d) *reinterpret_cast<uint4 *>(xs + (size_t)ch * 16) = xv[m];
+  }
   // The active rows are shared out evenly: CTA c takes T_c = floor((c+1)K/G) - floor(cK/G)
   // of the layer's K rows, first o_c = min(cnt_c, T_c) of its own tile's, then f_c = T_c - o_c
   // of the rows the tiles with more than their share leave over (e_t = cnt_t - o_t each,
@@ -110,50 +119,61 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   int *own = epre + G + 1;
   if (cur) {
     for (int i = tid; i < tn; i += kT) {  // the own tile's slots arrive with the counts
-      const int2 e = __ldcg(Q.list_in + t0 + i);
+      const int2 e = i == tid ? l_first : __ldcg(Q.list_in + t0 + i);
       act_s[i] = e.x;
       bias_s[i] = __int_as_float(e.y);
     }
     for (int t = tid; t < G; t += kT) {
       const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
-      cnt_all[t] = min(max(__ldcg(Q.cnt_in + t), 0), sz);
+      cnt_all[t] = min(max(t == tid ? c_tile : __ldcg(Q.cnt_in + t), 0), sz);
     }
   }
   __syncthreads();
   if (cur && warp == 0) {
-    int K = 0;
-    for (int t = lane; t < G; t += 32) K += cnt_all[t];
-    K = __reduce_add_sync(0xffffffffu, K);
-    int baseE = 0, baseF = 0;
-    for (int wi = 0; wi < G; wi += 32) {
-      const int t = wi + lane;
-      int e = 0, f = 0, o = 0;
-      if (t < G) {
-        const int share = (int)(((int64_t)(t + 1) * K) / G - ((int64_t)t * K) / G);
-        o = min(cnt_all[t], share);
-        e = cnt_all[t] - o;
-        f = share - o;
-      }
-      int ie = e, jf = f;  // inclusive scans of e and f over the tiles
+    // Lane l walks the tiles [l tpl, (l + 1) tpl) in order, twice: once for its sums of
+    // e_t and f_t, then (after a scan over the lanes) for epre[t] and this CTA's o, f, F.
+    // Shares in 32-bit arithmetic: floor(tK/G) = t q + floor(t rm / G), K = q G + rm.
+    const int tpl = (G + 31) / 32;
+    const int tb = min(G, lane * tpl), te = min(G, tb + tpl);
+    int ks = 0;
+    for (int t = tb; t < te; ++t) ks += cnt_all[t];
+    const int K = __reduce_add_sync(0xffffffffu, ks);
+    const int q = K / G, rm = K - q * G;
+    int es = 0, fs = 0;
+    for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
+      const int fh = ((t + 1) * rm) / G;
+      const int share = q + fh - fl;
+      fl = fh;
+      const int o = min(cnt_all[t], share);
+      es += cnt_all[t] - o;
+      fs += share - o;
+    }
+    int ie = es, jf = fs;  // inclusive scans of the lanes' sums
 #pragma unroll
-      for (int s = 1; s < 32; s <<= 1) {
-        const int ye = __shfl_up_sync(0xffffffffu, ie, s), yf = __shfl_up_sync(0xffffffffu, jf, s);
-        if (lane >= s) {
-          ie += ye;
-          jf += yf;
-        }
+    for (int sh = 1; sh < 32; sh <<= 1) {
+      const int ye = __shfl_up_sync(0xffffffffu, ie, sh), yf = __shfl_up_sync(0xffffffffu, jf, sh);
+      if (lane >= sh) {
+        ie += ye;
+        jf += yf;
       }
-      if (t < G) epre[t] = baseE + ie - e;
+    }
+    int be = ie - es, bf = jf - fs;
+    for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
+      const int fh = ((t + 1) * rm) / G;
+      const int share = q + fh - fl;
+      fl = fh;
+      const int o = min(cnt_all[t], share);
+      epre[t] = be;
       if (t == c) {
         own[0] = o;
-        own[1] = f;
-        own[2] = baseF + jf - f;
+        own[1] = share - o;
+        own[2] = bf;
       }
-      baseE += __shfl_sync(0xffffffffu, ie, 31);
-      baseF += __shfl_sync(0xffffffffu, jf, 31);
+      be += cnt_all[t] - o;
+      bf += share - o;
     }
-    if (lane == 0) {
-      epre[G] = baseE;
+    if (lane == 31) {
+      epre[G] = be;
       own[3] = K;
     }
   }
@@ -171,47 +191,13 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       else
         hi = mid;
     }
-    const int share = (int)(((int64_t)(lo + 1) * K) / G - ((int64_t)lo * K) / G);
+    const int q = K / G, rm = K - q * G;
+    const int share = q + ((lo + 1) * rm) / G - (lo * rm) / G;
     const int k = min(cnt_all[lo], share) + g - epre[lo];
     return __ldcg(Q.list_in + decode1_tile_start(lo, P.n, G) + k);
   };
   int2 ex0 = make_int2(0, 0);
-  if (tid < f_c) ex0 = excess_entry(tid);  // lands while A' runs
-
-  // ---------------------------------------------------------------- A': next hidden layer
-  if (next) {
-    for (int j = j0; j < r; j += G * kW) {
-      const T *row = At + (size_t)j * d;
-      float acc = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
-      for (int cb = 0; cb < nch_d; cb += 32 * 16) {
-        if (j != j0 || cb != 0) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int ch = cb + lane + 32 * u;
-            if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int ch = cb + lane + 32 * u;
-          if (ch < nch_d) acc = dot_chunk_smem<T>(w0[u], xs, ch, acc);
-        }
-      }
-      const float hs = warp_sum(acc);
-      if (lane == 0) Q.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
-    }
-  }
-
-  if (tid < f_c) {
-    act_s[o_c + tid] = ex0.x;
-    bias_s[o_c + tid] = __int_as_float(ex0.y);
-  }
-  for (int j = tid + kT; j < f_c; j += kT) {
-    const int2 e = excess_entry(j);
-    act_s[o_c + j] = e.x;
-    bias_s[o_c + j] = __int_as_float(e.y);
-  }
-  __syncthreads();
+  if (tid < f_c) ex0 = excess_entry(tid);  // lands while the own rows' first segments are requested
   const int cnt = o_c + f_c;
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread
@@ -241,6 +227,17 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   for (int m = 0; m < MAXM; ++m)
 #pragma unroll
     for (int v = 0; v < V; ++v) acc[m][v] = 0.f;
+  // The layer's own work comes first: C1 and C2 need only the lists, while the next
+  // layer's A'^T rows are requested during C2 and summed after it (h' is needed only
+  // after the grid barrier).
+  uint4 w0[16];
+  auto load_a = [&]() {  // the first batch of the warp's row of A'^T
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int ch = lane + 32 * u;
+      if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
+    }
+  };
   if (cur) {
     // -------------------------------------------------------------- C1: up / gate dots
     constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;
@@ -251,20 +248,38 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
     const int items = cnt * per_row;
     const int nch_r8 = d / VR;
     uint4 wc[D][SU];
+    auto load_item = [&](int s, int it) {
+      const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+      const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
+#pragma unroll
+      for (int u = 0; u < SU; ++u) {
+        const int ch = sg * kSegChunks + lane + 32 * u;
+        if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
+      }
+    };
+    // the warp's first D segments: the own rows' at once, the shared-out rows' once their
+    // entries are in shared memory
 #pragma unroll
     for (int s = 0; s < D; ++s) {
       const int it = warp + kW * s;
-      if (it < items) {
-        const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
-        const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
-#pragma unroll
-        for (int u = 0; u < SU; ++u) {
-          const int ch = sg * kSegChunks + lane + 32 * u;
-          if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
-        }
-      }
+      if (it < items && it / per_row < o_c) load_item(s, it);
     }
+    if (tid < f_c) {
+      act_s[o_c + tid] = ex0.x;
+      bias_s[o_c + tid] = __int_as_float(ex0.y);
+    }
+    for (int j = tid + kT; j < f_c; j += kT) {
+      const int2 e = excess_entry(j);
+      act_s[o_c + j] = e.x;
+      bias_s[o_c + j] = __int_as_float(e.y);
+    }
+    __syncthreads();
 #pragma unroll
+    for (int s = 0; s < D; ++s) {
+      const int it = warp + kW * s;
+      if (it < items && it / per_row >= o_c) load_item(s, it);
+    }
+#pragma unroll 1
     for (int s = 0; s < DD; ++s) stage_d(s, s);
     for (int ib = warp; ib < items; ib += D * kW) {
 #pragma unroll
@@ -319,6 +334,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       if (QR) a_s[k] *= sd;
     }
     __syncthreads();
+    if (next) load_a();  // lands during C2
 
     // -------------------------------------------------------------- C2: down projection
     for (int kb = 0; kb < cnt; kb += DD) {
@@ -352,6 +368,32 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       }
     }
     cp_async_wait<0>();
+  } else if (next) {
+    load_a();
+  }
+
+  // ---------------------------------------------------------------- A': next hidden layer
+  if (next) {
+    for (int j = j0; j < r; j += G * kW) {
+      const T *row = At + (size_t)j * d;
+      float acc1 = 0.f;  // one chain in ascending chunk order (the multi-kernel predictor's order)
+      for (int cb = 0; cb < nch_d; cb += 32 * 16) {
+        if (j != j0 || cb != 0) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int ch = cb + lane + 32 * u;
+            if (ch < nch_d) w0[u] = ld_stream(row + (size_t)ch * V);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int ch = cb + lane + 32 * u;
+          if (ch < nch_d) acc1 = dot_chunk_smem<T>(w0[u], xs, ch, acc1);
+        }
+      }
+      const float hs = warp_sum(acc1);
+      if (lane == 0) Q.hbuf[j] = hs > 0.f ? hs : 0.f;  // NaN -> 0
+    }
   }
   __syncthreads();  // C2's stages and activations are consumed: the region takes B'^T rows
 
@@ -369,8 +411,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
     cp_async_commit();
   };
   if (next) {
-#pragma unroll
-    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
     if (tid < un) {
       c_s[tid] = to_f<T>(c_first);
       a_s[tid] = to_f<T>(b_first);
@@ -391,7 +431,14 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       }
     }
   }
-  if (!cta_grid_sync(P, flag_s)) {
+  cta_grid_arrive(P, target_s);
+  // the first DB B'^T rows go out after the arrival (its release would otherwise wait for
+  // them to land), and land during the barrier
+  if (next) {
+#pragma unroll 1
+    for (int s = 0; s < DB; ++s) stage_b(s, warp + kW * s);
+  }
+  if (!cta_grid_wait(P, target_s, flag_s)) {
     cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     return;
   }

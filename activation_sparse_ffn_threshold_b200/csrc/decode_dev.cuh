@@ -237,26 +237,46 @@ __device__ __forceinline__ int share_excess_warp(const Decode1Params &P, int quo
   const int lane = threadIdx.x & 31;
   const int G = P.G, c = blockIdx.x;
   int *epre = scratch;
-  int base = 0;
-  for (int wi = 0; wi < G; wi += 32) {
-    const int t = wi + lane;
-    int e = 0;
-    if (t < G) {
-      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
-      e = max(0, min(max(__ldcg(P.bcnt + t), 0), sz) - quota);
-    }
-    int incl = e;
+  // lane l takes the tiles [l tpl, (l + 1) tpl) (tpl <= 8: G <= 254), all its counts
+  // requested at once; e_t goes to epre[t], then in place to the exclusive prefix
+  const int tpl = (G + 31) / 32;
+  const int tb = min(G, lane * tpl), te = min(G, tb + tpl);
+  int cv[8];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+  for (int i = 0; i < 8; ++i) cv[i] = tb + i < te ? __ldcg(P.bcnt + tb + i) : 0;
+  int es = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = tb + i;
+    if (t < te) {
+      const int sz = decode1_tile_start(t + 1, P.n, G) - decode1_tile_start(t, P.n, G);
+      const int e = max(0, min(max(cv[i], 0), sz) - quota);
+      epre[t] = e;
+      es += e;
     }
-    if (t < G) epre[t] = base + incl - e;
-    base += __shfl_sync(0xffffffffu, incl, 31);
   }
+  int incl = es;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int be = incl - es;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = tb + i;
+    if (t < te) {
+      const int e = epre[t];
+      epre[t] = be;
+      be += e;
+    }
+  }
+  const int E = __shfl_sync(0xffffffffu, incl, 31);
   __syncwarp();
-  const int F = (int)(((int64_t)c * base) / G);
-  const int f = (int)(((int64_t)(c + 1) * base) / G) - F;
+  // CTA c's share: [floor(cE/G), floor((c+1)E/G)), with floor(cE/G) = c q + floor(c rm / G)
+  const int q = E / G, rm = E - q * G;
+  const int F = c * q + (c * rm) / G;
+  const int f = q + ((c + 1) * rm) / G - (c * rm) / G;
   for (int j = lane; j < f; j += 32) {
     const int g = F + j;
     int lo = 0, hi = G;  // the largest t with epre[t] <= g

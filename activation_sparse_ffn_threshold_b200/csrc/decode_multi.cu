@@ -200,10 +200,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
       if (lane == 0) P.hbuf[((size_t)t * 2 + ahalf) * r + j] = hs;
     }
   }
-  if (j0 < r) {
-#pragma unroll 1
-    for (int s = 0; s < kMB; ++s) stage_b(s, pair + kPairs * s);
-  }
   if (tid < tn) {
     c_s[tid] = __half2float(c_first);
     a_s[tid] = __half2float(b_first);
@@ -217,6 +213,12 @@ __global__ void __launch_bounds__(kT, 1) k_decode_multi(const Decode1Params P) {
   const int nseg = P.nseg;
   const int per_row = NPG * nseg;
   cta_grid_arrive(P, target_s);
+  // the B^T stages of the warps with an A^T row go out after the arrival: its release
+  // would otherwise wait for them to land
+  if (j0 < r) {
+#pragma unroll 1
+    for (int s = 0; s < kMB; ++s) stage_b(s, pair + kPairs * s);
+  }
   // The hot prefix (the tile's first hp positions: neurons in a batch's union with
   // probability >= 0.99) is read densely: its gate/up dots for every token are computed
   // while the barrier completes, before the sets are known; a prefix row that no token's
