@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   constexpr bool QR = RB <= 8;           // rows are codes with per-row scales
   constexpr int VR = 128 / RB;           // row elements per 16-byte chunk
   constexpr int MAXH = 4;              // chunks of h' per lane (r <= 128 * V)
-  constexpr int DB = kDecode1BStages;
+  const int DB = min(P.bstages, kDecode1BStages);  // B'^T rows staged per warp: 1, 2, 3 or 4
   constexpr int DD = decode1_dstages(MAXM);
   extern __shared__ __align__(16) unsigned char smem[];
   const Decode1Layout L = decode_ahead_layout(P, Q);
@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
   int *flag_s = cnt_s + 1;
   int *ncnt_s = cnt_s + 2;
   unsigned long long *target_s = reinterpret_cast<unsigned long long *>(cnt_s + 4);  // the barrier's target
+  int *next_s = cnt_s + 6;  // C1's next work item
+  int *ext_s = cnt_s + 7;   // C1's final row count once known (-1: not yet)
   unsigned char *bstage = smem + L.bstage;
   unsigned char *dstage = smem + L.dstage;
 
@@ -93,6 +95,10 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
     b_first = bp[u0 + tid];
   }
   for (int i = tid; i < (Q.tile_max + 31) / 32; i += kT) bits[i] = 0u;
+  if (tid == 0) {
+    *next_s = 0;
+    *ext_s = -1;
+  }
 
   pdl_wait();  // u_l, this layer's lists and every buffer written here belong to earlier kernels until here
   uint4 xv[MAXM];
@@ -129,76 +135,17 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
     }
   }
   __syncthreads();
-  if (cur && warp == 0) {
-    // Lane l walks the tiles [l tpl, (l + 1) tpl) in order, twice: once for its sums of
-    // e_t and f_t, then (after a scan over the lanes) for epre[t] and this CTA's o, f, F.
-    // Shares in 32-bit arithmetic: floor(tK/G) = t q + floor(t rm / G), K = q G + rm.
-    const int tpl = (G + 31) / 32;
-    const int tb = min(G, lane * tpl), te = min(G, tb + tpl);
+  // every warp: the layer's row count K and this CTA's own rows o_c = min(cnt_c, T_c), with
+  // floor(tK/G) = t q + floor(t rm / G), K = q G + rm (32-bit arithmetic)
+  int K = 0, o_c = 0;
+  if (cur) {
     int ks = 0;
-    for (int t = tb; t < te; ++t) ks += cnt_all[t];
-    const int K = __reduce_add_sync(0xffffffffu, ks);
+    for (int t = lane; t < G; t += 32) ks += cnt_all[t];
+    K = __reduce_add_sync(0xffffffffu, ks);
     const int q = K / G, rm = K - q * G;
-    int es = 0, fs = 0;
-    for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
-      const int fh = ((t + 1) * rm) / G;
-      const int share = q + fh - fl;
-      fl = fh;
-      const int o = min(cnt_all[t], share);
-      es += cnt_all[t] - o;
-      fs += share - o;
-    }
-    int ie = es, jf = fs;  // inclusive scans of the lanes' sums
-#pragma unroll
-    for (int sh = 1; sh < 32; sh <<= 1) {
-      const int ye = __shfl_up_sync(0xffffffffu, ie, sh), yf = __shfl_up_sync(0xffffffffu, jf, sh);
-      if (lane >= sh) {
-        ie += ye;
-        jf += yf;
-      }
-    }
-    int be = ie - es, bf = jf - fs;
-    for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
-      const int fh = ((t + 1) * rm) / G;
-      const int share = q + fh - fl;
-      fl = fh;
-      const int o = min(cnt_all[t], share);
-      epre[t] = be;
-      if (t == c) {
-        own[0] = o;
-        own[1] = share - o;
-        own[2] = bf;
-      }
-      be += cnt_all[t] - o;
-      bf += share - o;
-    }
-    if (lane == 31) {
-      epre[G] = be;
-      own[3] = K;
-    }
+    o_c = min(cnt_all[c], q + ((c + 1) * rm) / G - (c * rm) / G);
   }
-  __syncthreads();
-  const int o_c = cur ? own[0] : 0, f_c = cur ? own[1] : 0, F_c = cur ? own[2] : 0, K = cur ? own[3] : 0;
-  // this CTA's excess row j is the layer's excess row g = F_c + j: tile t with
-  // epre[t] <= g < epre[t + 1], slot o_t + g - epre[t] of that tile
-  auto excess_entry = [&](int j) {
-    const int g = F_c + j;
-    int lo = 0, hi = G;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (epre[mid] <= g)
-        lo = mid;
-      else
-        hi = mid;
-    }
-    const int q = K / G, rm = K - q * G;
-    const int share = q + ((lo + 1) * rm) / G - (lo * rm) / G;
-    const int k = min(cnt_all[lo], share) + g - epre[lo];
-    return __ldcg(Q.list_in + decode1_tile_start(lo, P.n, G) + k);
-  };
-  int2 ex0 = make_int2(0, 0);
-  if (tid < f_c) ex0 = excess_entry(tid);  // lands while the own rows' first segments are requested
-  const int cnt = o_c + f_c;
+  int cnt = o_c;  // this CTA's rows; the shared-out ones are appended during C1
 
   // C2's rows of W_down stream through DD shared-memory stages private to each thread
   auto dslot = [&](int s, int m) { return dstage + (((size_t)s * MAXM + m) * kT + tid) * 16; };
@@ -221,7 +168,6 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
     }
     cp_async_commit();
   };
-
   float acc[MAXM][V];
 #pragma unroll
   for (int m = 0; m < MAXM; ++m)
@@ -238,82 +184,174 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       if (j0 < r && ch < nch_d) w0[u] = ld_stream(At + (size_t)j0 * d + (size_t)ch * V);
     }
   };
+  int cpre = 0;  // C2 stages requested during C1
   if (cur) {
     // -------------------------------------------------------------- C1: up / gate dots
+    // The rows' 4 KB segments are work items handed out in order by a shared counter
+    // (own rows first), loaded into registers; warp 0 meanwhile computes the share's
+    // prefix, fetches the shared-out rows' entries and publishes the final count.
     constexpr int NPG = ACT == SFNN_REGLU ? 2 : 1;
-    constexpr int D = 2;
     constexpr int SU = kSegChunks / 32;
     const int nseg = P.nseg;
     const int per_row = NPG * nseg;
-    const int items = cnt * per_row;
     const int nch_r8 = d / VR;
-    uint4 wc[D][SU];
-    auto load_item = [&](int s, int it) {
-      const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
+    int lim = o_c * per_row;  // items known to exist
+    bool known = false;
+    uint4 wa[SU], wb[SU];
+    auto grab = [&]() {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(next_s, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    auto avail = [&](int it) {  // 1: item `it` exists, 0: past the end, -1: abandoned
+      if (it < lim) return 1;
+      if (known) return 0;
+      int e = -1;  // the final count: wait for warp 0 to publish it (bounded)
+      if (lane == 0) {
+        const uint64_t tw = clock64();
+        while ((e = *reinterpret_cast<volatile int *>(ext_s)) == -1)
+          if ((uint64_t)(clock64() - tw) > 2 * kWaitCycles) {
+            latch_error(P.err, kErrTimeout);
+            e = -2;
+            break;
+          }
+        __threadfence_block();
+      }
+      e = __shfl_sync(0xffffffffu, e, 0);
+      __syncwarp();
+      if (e < 0) return -1;
+      known = true;
+      cnt = e;
+      lim = e * per_row;
+      return it < lim ? 1 : 0;
+    };
+    auto load_c = [&](uint4 *w, int it) {
+      const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
       const unsigned char *row = rows + ((size_t)act_s[k] * nproj + pj) * rowB;
 #pragma unroll
       for (int u = 0; u < SU; ++u) {
         const int ch = sg * kSegChunks + lane + 32 * u;
-        if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
+        if (ch < nch_r8) w[u] = ld_stream(row + (size_t)ch * 16);
       }
     };
-    // the warp's first D segments: the own rows' at once, the shared-out rows' once their
-    // entries are in shared memory
+    auto sum_c = [&](const uint4 *w, int it) {
+      const int k = it / per_row, pj = (it % per_row) / nseg, sg = it % per_row - pj * nseg;
+      float a = 0.f;
 #pragma unroll
-    for (int s = 0; s < D; ++s) {
-      const int it = warp + kW * s;
-      if (it < items && it / per_row < o_c) load_item(s, it);
-    }
-    if (tid < f_c) {
-      act_s[o_c + tid] = ex0.x;
-      bias_s[o_c + tid] = __int_as_float(ex0.y);
-    }
-    for (int j = tid + kT; j < f_c; j += kT) {
-      const int2 e = excess_entry(j);
-      act_s[o_c + j] = e.x;
-      bias_s[o_c + j] = __int_as_float(e.y);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int s = 0; s < D; ++s) {
-      const int it = warp + kW * s;
-      if (it < items && it / per_row >= o_c) load_item(s, it);
-    }
-#pragma unroll 1
-    for (int s = 0; s < DD; ++s) stage_d(s, s);
-    for (int ib = warp; ib < items; ib += D * kW) {
-#pragma unroll
-      for (int s = 0; s < D; ++s) {
-        const int it = ib + kW * s;
-        if (it < items) {
-          const int k = it / per_row, pj = (it - k * per_row) / nseg, sg = it - k * per_row - pj * nseg;
-          float a = 0.f;
-#pragma unroll
-          for (int u = 0; u < SU; ++u) {
-            const int ch = sg * kSegChunks + lane + 32 * u;
-            if (ch < nch_r8) {
-              if (RB == 4)
-                a = dot_chunk_i4(wc[s][u], xs, ch, a);
-              else if (RB == 8)
-                a = dot_chunk_i8(wc[s][u], xs, ch, a);
-              else
-                a = dot_chunk_smem<T>(wc[s][u], xs, ch, a);
-            }
-          }
-          const int itn = it + D * kW;
-          if (itn < items) {
-            const int kn = itn / per_row, pjn = (itn - kn * per_row) / nseg, sgn = itn - kn * per_row - pjn * nseg;
-            const unsigned char *row = rows + ((size_t)act_s[kn] * nproj + pjn) * rowB;
-#pragma unroll
-            for (int u = 0; u < SU; ++u) {
-              const int ch = sgn * kSegChunks + lane + 32 * u;
-              if (ch < nch_r8) wc[s][u] = ld_stream(row + (size_t)ch * 16);
-            }
-          }
-          a = warp_sum(a);
-          if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+      for (int u = 0; u < SU; ++u) {
+        const int ch = sg * kSegChunks + lane + 32 * u;
+        if (ch < nch_r8) {
+          if (RB == 4)
+            a = dot_chunk_i4(w[u], xs, ch, a);
+          else if (RB == 8)
+            a = dot_chunk_i8(w[u], xs, ch, a);
+          else
+            a = dot_chunk_smem<T>(w[u], xs, ch, a);
         }
       }
+      a = warp_sum(a);
+      if (lane == 0) dots[(k * 2 + pj) * nseg + sg] = a;
+    };
+    const bool two = P.c1depth > 1;
+    int ia = grab(), ib = two ? grab() : 0;
+    int sa = ia < lim ? 1 : 2, sb = two ? (ib < lim ? 1 : 2) : 0;  // 2: not known yet
+    if (sa == 1) load_c(wa, ia);
+    if (sb == 1) load_c(wb, ib);
+    cpre = min(DD, o_c);
+#pragma unroll 1
+    for (int s = 0; s < cpre; ++s) stage_d(s, s);
+    if (warp == 0) {
+      // Lane l walks the tiles [l tpl, (l + 1) tpl) in order, twice: once for its sums of
+      // e_t and f_t, then (after a scan over the lanes) for epre[t] and this CTA's f, F.
+      const int q = K / G, rm = K - q * G;
+      const int tpl = (G + 31) / 32;
+      const int tb = min(G, lane * tpl), te = min(G, tb + tpl);
+      int es = 0, fs = 0;
+      for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
+        const int fh = ((t + 1) * rm) / G;
+        const int share = q + fh - fl;
+        fl = fh;
+        const int o = min(cnt_all[t], share);
+        es += cnt_all[t] - o;
+        fs += share - o;
+      }
+      int ie = es, jf = fs;  // inclusive scans of the lanes' sums
+#pragma unroll
+      for (int sh = 1; sh < 32; sh <<= 1) {
+        const int ye = __shfl_up_sync(0xffffffffu, ie, sh), yf = __shfl_up_sync(0xffffffffu, jf, sh);
+        if (lane >= sh) {
+          ie += ye;
+          jf += yf;
+        }
+      }
+      int be = ie - es, bf = jf - fs;
+      for (int t = tb, fl = (tb * rm) / G; t < te; ++t) {
+        const int fh = ((t + 1) * rm) / G;
+        const int share = q + fh - fl;
+        fl = fh;
+        const int o = min(cnt_all[t], share);
+        epre[t] = be;
+        if (t == c) {
+          own[1] = share - o;
+          own[2] = bf;
+        }
+        be += cnt_all[t] - o;
+        bf += share - o;
+      }
+      if (lane == 31) epre[G] = be;
+      __syncwarp();
+      // this CTA's excess row j is the layer's excess row g = F + j: tile t with
+      // epre[t] <= g < epre[t + 1], slot o_t + g - epre[t] of that tile
+      const int f_c = own[1], F_c = own[2];
+      for (int j = lane; j < f_c; j += 32) {
+        const int g = F_c + j;
+        int lo = 0, hi = G;
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (epre[mid] <= g)
+            lo = mid;
+          else
+            hi = mid;
+        }
+        const int share = q + ((lo + 1) * rm) / G - (lo * rm) / G;
+        const int2 e = __ldcg(Q.list_in + decode1_tile_start(lo, P.n, G) + min(cnt_all[lo], share) + g - epre[lo]);
+        act_s[o_c + j] = e.x;
+        bias_s[o_c + j] = __int_as_float(e.y);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();  // the rows' entries before the count
+        *reinterpret_cast<volatile int *>(ext_s) = o_c + f_c;
+      }
+      __syncwarp();
+    }
+    if (sa == 2) {
+      sa = avail(ia);
+      if (sa == 1) load_c(wa, ia);
+    }
+    if (sb == 2 && sa >= 0) {
+      sb = avail(ib);
+      if (sb == 1) load_c(wb, ib);
+    }
+#pragma unroll 1
+    while (sa > 0 || sb > 0) {
+      if (sa < 0 || sb < 0) break;
+      if (sa > 0) {
+        sum_c(wa, ia);
+        ia = grab();
+        sa = avail(ia);
+        if (sa > 0) load_c(wa, ia);
+      }
+      if (sb > 0 && sa >= 0) {
+        sum_c(wb, ib);
+        ib = grab();
+        sb = avail(ib);
+        if (sb > 0) load_c(wb, ib);
+      }
+    }
+    if (sa < 0 || sb < 0) {  // abandoned (warp 0 always publishes: defensive)
+      cp_async_wait<0>();
+      return;
     }
     __syncthreads();
     for (int k = tid; k < cnt; k += kT) {
@@ -334,6 +372,8 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       if (QR) a_s[k] *= sd;
     }
     __syncthreads();
+#pragma unroll 1
+    for (int s = cpre; s < DD; ++s) stage_d(s, s);  // the rest of C2's first stages
     if (next) load_a();  // lands during C2
 
     // -------------------------------------------------------------- C2: down projection
@@ -508,11 +548,16 @@ __global__ void __launch_bounds__(kT, 1) k_decode_ahead(const Decode1Params P, c
       }
     }
     for (int pb = warp; pb < un; pb += DB * kW) {
-#pragma unroll
+#pragma unroll 1
       for (int s = 0; s < DB; ++s) {
         const int p = pb + kW * s;
         if (p < un) {
-          cp_async_wait<DB - 1>();
+          switch (DB) {  // this lane's copies of row p have landed
+            case 1: cp_async_wait<0>(); break;
+            case 2: cp_async_wait<1>(); break;
+            case 3: cp_async_wait<2>(); break;
+            default: cp_async_wait<3>(); break;
+          }
           float a = 0.f;
 #pragma unroll
           for (int m = 0; m < MAXH; ++m) {
