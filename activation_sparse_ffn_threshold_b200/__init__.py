@@ -88,6 +88,7 @@ def load_library():
         "sfnn_set_fused_quota": ([P, I], S),
         "sfnn_set_batch_quota": ([P, I], S),
         "sfnn_set_batch_depths": ([P, I, I, I, I], S),
+        "sfnn_tune_batch_paths": ([P, P], S),
         "sfnn_set_fused_depths": ([P, I, I, I, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
@@ -272,6 +273,14 @@ class SparseFFN:
         in the down phase); -1 keeps a value."""
         _check(self._lib.sfnn_set_batch_depths(self._h, int(bstages), int(c2pre), int(c1depth), int(c2stages)),
                "sfnn_set_batch_depths")
+
+    def tune_batch_paths(self, stream=None):
+        """Measure which path serves AUTO batches just above the few-token kernel's size
+        faster (two few-token launches or tensor cores) and make AUTO take it (set-up call)."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.device(self.device):
+            _check(self._lib.sfnn_tune_batch_paths(self._h, ctypes.c_void_p(s.cuda_stream)), "sfnn_tune_batch_paths")
 
     def set_batch_quota(self, enable: bool):
         """The few-token kernel's rebalancing (off: each token's y independent of the batch)."""

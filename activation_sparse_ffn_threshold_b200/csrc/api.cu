@@ -9,6 +9,7 @@
 #include <cstring>
 #include <new>
 #include <numeric>
+#include <random>
 #include <vector>
 
 #include "common.cuh"
@@ -124,29 +125,46 @@ sfnn_status run_layer(sfnn_ctx *h, const void *X, int b, SetSource src, const in
     h->launches += sets ? 2 : 1;
     return SFNN_OK;
   }
-  // a few tokens: the multi-token fused kernel on CUDA cores (AUTO and FUSED), when it fits
-  const bool multi = b >= 2 && b <= h->multi_max && predict && !ahead && h->fused_on &&
-                     (h->batch_path == SFNN_BATCH_AUTO || h->batch_path == SFNN_BATCH_FUSED);
+  // a few tokens: the multi-token fused kernel on CUDA cores (AUTO and FUSED), when it fits:
+  // up to multi_max tokens in one launch; up to twice that in two launches of at most
+  // multi_max (FUSED, or AUTO where sfnn_tune_batch_paths measured them faster than the
+  // tensor-core path)
+  const bool fusedish = predict && !ahead && h->fused_on && h->multi_max >= 2 &&
+                        (h->batch_path == SFNN_BATCH_AUTO || h->batch_path == SFNN_BATCH_FUSED);
+  const bool multi = fusedish && b >= 2 &&
+                     (b <= h->multi_max ||
+                      (b <= 2 * h->multi_max && (h->batch_path == SFNN_BATCH_FUSED || h->auto_chunked[b])));
   if (multi) {
     const bool sets = idx_out || cnt_out;
-    Decode1Params P = h->d1;
-    P.x = X;
-    P.y = Y;
-    P.resid = resid;
-    P.xnext = xnext;
-    P.set_pos = sets ? reinterpret_cast<int32_t *>(h->acoef) : nullptr;
-    P.set_cnt = sets ? h->scnt : nullptr;
-    P.hot = h->hot_on ? h->hot_rows[b] : 0;
-    P.quota = h->batch_quota_off ? 0 : h->quota_multi[b];
-    P.bstages = h->mdepth[0];
-    P.c2pre = h->mdepth[1];
-    P.c1depth = h->mdepth[2];
-    P.c2stages = h->mdepth[3];
-    SFNN_TRY(launch_decode_multi(P, b, s, true));
+    const size_t xe = h->L.dt == SFNN_F16 ? 2 : 4;
+    auto chunk = [&](int o, int cb) -> sfnn_status {  // tokens [o, o + cb)
+      Decode1Params P = h->d1;
+      P.x = static_cast<const unsigned char *>(X) + (size_t)o * h->L.d * xe;
+      P.y = Y + (size_t)o * h->L.d;
+      P.resid = resid ? resid + (size_t)o * h->L.d : nullptr;
+      P.xnext = xnext ? static_cast<unsigned char *>(xnext) + (size_t)o * h->L.d * xe : nullptr;
+      P.set_pos = sets ? reinterpret_cast<int32_t *>(h->acoef) : nullptr;
+      P.set_cnt = sets ? h->scnt : nullptr;
+      P.hot = h->hot_on ? h->hot_rows[cb] : 0;
+      P.quota = h->batch_quota_off ? 0 : h->quota_multi[cb];
+      P.bstages = h->mdepth[0];
+      P.c2pre = h->mdepth[1];
+      P.c1depth = h->mdepth[2];
+      P.c2stages = h->mdepth[3];
+      SFNN_TRY(launch_decode_multi(P, cb, s, true));
+      if (sets)
+        SFNN_TRY(launch_tile_sets(P.set_pos, 1, h->scnt, h->perm, h->L.n, P.G, idx_out ? idx_out + (size_t)o * h->L.n : nullptr,
+                                  cnt_out ? cnt_out + o : nullptr, s, cb));
+      h->launches += sets ? 2 : 1;
+      return SFNN_OK;
+    };
+    const sfnn_status st = b <= h->multi_max ? chunk(0, b) : chunk(0, (b + 1) / 2);  // b = 5: 3 + 2
+    if (st != SFNN_OK) return st;
+    if (b > h->multi_max) {
+      const sfnn_status st2 = chunk((b + 1) / 2, b / 2);
+      if (st2 != SFNN_OK) return st2;
+    }
     record_if(after, s);
-    if (sets)
-      SFNN_TRY(launch_tile_sets(P.set_pos, 1, h->scnt, h->perm, h->L.n, P.G, idx_out, cnt_out, s, b));
-    h->launches += sets ? 2 : 1;
     return SFNN_OK;
   }
   const bool tc = tc_batch_supported(h) && (h->batch_path == SFNN_BATCH_TENSOR_CORE ||
@@ -659,6 +677,67 @@ sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
   for (int i = 0; i < 4; ++i)
     if (v[i] != -1) h->mdepth[i] = v[i];
   return SFNN_OK;
+}
+
+sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
+  for (int b = 0; b <= kMaxBatch; ++b) h->auto_chunked[b] = false;
+  const int bmax = std::min(h->max_batch, 2 * h->multi_max);
+  if (h->multi_max < 2 || bmax <= h->multi_max || !tc_batch_supported(h)) return SFNN_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xe = h->L.dt == SFNN_F16 ? 2 : 4, d = h->L.d;
+  // synthetic inputs: unit-variance Gaussian tokens (fixed seed), the scale the predictor's
+  // bias is calibrated for
+  std::vector<uint16_t> xh((size_t)bmax * d);
+  std::vector<float> xf((size_t)bmax * d);
+  std::mt19937 rng(12345);
+  std::normal_distribution<float> nd(0.f, 1.f);
+  for (size_t i = 0; i < xf.size(); ++i) xf[i] = nd(rng);
+  void *X = nullptr;
+  float *Y = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  sfnn_status st = SFNN_OK;
+  if (cudaMalloc(&X, (size_t)bmax * d * xe) != cudaSuccess || cudaMalloc(&Y, (size_t)bmax * d * 4) != cudaSuccess ||
+      cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    st = SFNN_ERR_OOM;
+  } else {
+    if (xe == 2) {
+      for (size_t i = 0; i < xf.size(); ++i) {
+        const __half hv = __float2half_rn(xf[i]);
+        std::memcpy(&xh[i], &hv, 2);
+      }
+      cudaMemcpy(X, xh.data(), xh.size() * 2, cudaMemcpyHostToDevice);
+    } else {
+      cudaMemcpy(X, xf.data(), xf.size() * 4, cudaMemcpyHostToDevice);
+    }
+    const int saved = h->batch_path;
+    auto time_path = [&](int path, int b, float *ms) -> sfnn_status {
+      h->batch_path = path;
+      for (int i = 0; i < 7; ++i) {
+        if (i == 2) cudaEventRecord(e0, s);  // 2 warm-up calls, 5 timed
+        const sfnn_status r = run_layer(h, X, b, kSetPredict, nullptr, nullptr, nullptr, nullptr, nullptr, Y, nullptr,
+                                        nullptr, s);
+        if (r != SFNN_OK) return r;
+      }
+      cudaEventRecord(e1, s);
+      if (cudaEventSynchronize(e1) != cudaSuccess) return SFNN_ERR_CUDA;
+      cudaEventElapsedTime(ms, e0, e1);
+      return SFNN_OK;
+    };
+    for (int b = h->multi_max + 1; b <= bmax && st == SFNN_OK; ++b) {
+      float t_multi = 0.f, t_tc = 0.f;
+      st = time_path(SFNN_BATCH_FUSED, b, &t_multi);
+      if (st == SFNN_OK) st = time_path(SFNN_BATCH_TENSOR_CORE, b, &t_tc);
+      if (st == SFNN_OK) h->auto_chunked[b] = t_multi < t_tc;
+    }
+    h->batch_path = saved;
+  }
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (X) cudaFree(X);
+  if (Y) cudaFree(Y);
+  return st;
 }
 
 sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable) {

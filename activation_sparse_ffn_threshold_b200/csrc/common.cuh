@@ -61,6 +61,7 @@ struct sfnn_ctx {
   int quota_multi[sfnn::kMultiMaxTokens + 1];  // the same for the multi-token kernel, by batch size
   bool batch_quota_off;  // the multi-token kernel's rebalancing switched off (batch-invariant rows)
   int mdepth[4];         // the multi-token kernel's request depths (bstages, c2pre, c1depth, c2stages)
+  bool auto_chunked[sfnn::kMaxBatch + 1];  // AUTO: b tokens as two few-token launches (measured faster)
   int32_t *scnt;     // [max_batch][G] per-tile counts of the sets a fused launch used (lists: ulist
                      //   for one token, acoef's words for several)
   int multi_max;     // largest batch the multi-token fused kernel serves (0: none)

@@ -527,6 +527,9 @@ def measure_batch(cfg, b, args, dist, dev):
     per_batch = W.touched_bytes(cfg, W.expected_union_density(lay.p, b) * cfg.n, b)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
     handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b, **_order_kw(args)) for _ in range(R)]
+    if 4 < b <= 8:  # AUTO's measured choice between two few-token launches and tensor cores
+        for h in handles:
+            h.tune_batch_paths()
     info = handles[0].info()
     torch.cuda.synchronize()
     X = torch.from_numpy(Xh).to(dev)
@@ -549,14 +552,16 @@ def measure_batch(cfg, b, args, dist, dev):
     ms, t_max, clocks = time_graph(g, s, args.steps, args.warmup, dist, _gpu_id(dev))
     _check_errors(handles)
     unit_us = ms * 1e3 / (args.steps * BATCHES_PER_STEP)
-    path = batch_path_name(handles[0], b)
+    path = batch_path_name(handles[0], b, launches // BATCHES_PER_STEP)
     out = {"value": dist.sum(args.steps * BATCHES_PER_STEP * b) / (t_max / 1e3), "unit": "tokens/s",
            "ms_per_step": t_max / args.steps, "avg_us": unit_us, "avg_of": f"one batch of {b} tokens",
            "replicas": R, "path": path, "kernels_per_batch": launches // BATCHES_PER_STEP,
            "mean_union_rows": float(unions.mean()), "gpu_launches": int(launches * args.steps), "clocks": clocks,
            "bytes_per_step": float(bytes_batch.sum())}
-    tpath = "multi" if b <= 4 and handles[0].info()["wdtype"] == 1 else "tcgen05"
-    traffic, tsrc = profiled_traffic(cfg.name, f"batch_{cfg.name}_b{b}", tpath, "dram_bytes_per_batch")
+    two = b > 4 and launches // BATCHES_PER_STEP == 2
+    tpath = "multi" if (b <= 4 and handles[0].info()["wdtype"] == 1) or two else "tcgen05"
+    summary = f"batch_{cfg.name}_b{b}" + ("_two_launches" if two else "")
+    traffic, tsrc = profiled_traffic(cfg.name, summary, tpath, "dram_bytes_per_batch")
     out["roofline"] = roofline(float(bytes_batch.mean()), unit_us,
                                f"one batch of {b} tokens ({launches // BATCHES_PER_STEP} kernels, {path}); "
                                "duration = CUDA-event time of the timed region / batches", traffic, tsrc)
@@ -566,12 +571,14 @@ def measure_batch(cfg, b, args, dist, dev):
     return out
 
 
-def batch_path_name(h, b) -> str:
+def batch_path_name(h, b, kernels_per_batch) -> str:
     """The kernels AUTO (or the chosen path) runs for b tokens on this layer."""
     inf = h.info()
     fused = inf["wdtype"] == 1 and 2 <= b <= 4  # fp16 layers: the few-token fused kernel
+    two = inf["wdtype"] == 1 and b > 4 and kernels_per_batch == 2  # two few-token launches
     tc = inf["wdtype"] == 1 and inf["d"] % 128 == 0
-    auto = "fused few-token kernel (CUDA cores)" if fused else ("tcgen05" if tc else "cuda-core")
+    auto = ("fused few-token kernel (CUDA cores)" if fused else
+            "two fused few-token launches (measured faster)" if two else ("tcgen05" if tc else "cuda-core"))
     return {0: f"auto: {auto}", 1: "cuda-core", 2: "tcgen05", 3: f"fused: {auto}"}.get(inf["batch_path"], "?")
 
 

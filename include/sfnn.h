@@ -300,6 +300,18 @@ SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
 SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
 
 /*
+ * Measures, on this handle, which path serves AUTO batches of multi_max + 1 .. 2 multi_max
+ * tokens faster (multi_max: the few-token kernel's largest batch, 4 when it fits; at most
+ * the handle's max_batch): two few-token launches of at most multi_max tokens each, or the
+ * tensor-core batch path, on synthetic unit-variance tokens (fixed seed), 2 warm-up and 5
+ * timed calls each, and makes AUTO take the faster one for each such b (SFNN_BATCH_FUSED
+ * always takes the two launches).  Without this call AUTO takes the tensor-core path there.
+ * Allocates and frees temporary device memory and synchronises `stream`: a set-up call, not
+ * for graph capture.  SFNN_OK with nothing measured when the handle has no such b.
+ */
+SFNN_API sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream);
+
+/*
  * The few-token fused kernel's request depths, as sfnn_set_fused_depths (the results do not
  * depend on them): bstages = B^T half rows staged per warp (2, 4, 6 or 8), c2pre = W_down
  * rows requested while the up/gate rows stream (0 to 8), c1depth = up/gate segments in

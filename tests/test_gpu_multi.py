@@ -11,6 +11,8 @@
   same, Y agrees within rounding and is bitwise reproducible for a given batch;
 * AUTO takes it for 2 to 4 tokens on the full OPT-30B- and 70B-shaped layers, and the
   residual stack runs through it;
+* 5 to 8 tokens as two few-token launches (FUSED, and AUTO after the measured choice)
+  agree with the oracle per token;
 * its request depths change nothing in the result (bitwise the same Y and sets);
 * outputs stay inside their buffers (canary words on both sides).
 """
@@ -191,4 +193,28 @@ def test_batch_request_depths_do_not_change_the_result(base, d, n, r):
     for bad in [(3, -1, -1, -1), (-1, 9, -1, -1), (-1, -1, 0, -1), (-1, -1, -1, 16)]:
         with pytest.raises(RuntimeError):
             h.set_batch_depths(*bad)
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("b", [5, 6, 8])
+def test_two_launch_batches(b):
+    cfg = W.small_config(W.CONFIGS["70b_reglu"], d=2048, n=5003, r=256)
+    lay = W.make_layer(cfg, seed=35)
+    h = sf.SparseFFN.from_layer(lay, max_batch=8)
+    X = W.make_tokens(cfg, b, seed=36 + b)
+    h.set_batch_path(sf.BATCH_FUSED)
+    Y, masks = run_multi(h, X)
+    for t in range(b):
+        check_token(lay, X[t], Y[t], masks[t], f"two launches b={b} t={t}")
+    # each half is exactly the few-token kernel's result on that half alone
+    h.set_batch_quota(False)
+    Yq, _ = run_multi(h, X)
+    Ya, _ = run_multi(h, X[: (b + 1) // 2])
+    assert np.array_equal(Yq[: (b + 1) // 2], Ya)
+    h.set_batch_quota(True)
+    h.set_batch_path(sf.BATCH_AUTO)
+    h.tune_batch_paths()
+    Y2, m2 = run_multi(h, X)
+    for t in range(b):
+        check_token(lay, X[t], Y2[t], m2[t], f"auto after tuning b={b} t={t}")
     assert h.get_error() == 0
