@@ -3,6 +3,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "context.cuh"
 
 namespace sfnn {
 

@@ -217,7 +217,7 @@ def measured_peak():
 PATH_SOURCES = {
     "k_decode1": ("async.cuh", "common.cuh", "decode1.cu", "decode1.cuh", "decode_dev.cuh"),
     "multi": ("async.cuh", "common.cuh", "decode_multi.cu", "decode1.cuh", "decode_dev.cuh"),
-    "tcgen05": ("async.cuh", "common.cuh", "tc_batch.cu", "predict.cu", "ffn.cu", "launch.cuh"),
+    "tcgen05": ("async.cuh", "common.cuh", "context.cuh", "tc_batch.cu", "predict.cu", "ffn.cu", "launch.cuh"),
     "lookahead": ("async.cuh", "common.cuh", "decode_ahead.cu", "decode1.cuh", "decode_dev.cuh"),
 }
 
