@@ -7,8 +7,7 @@
 
 namespace sfnn {
 
-constexpr int kMaxNeurons = 1 << 20;                  // n: the union's per-word offsets live in shared memory
-constexpr int kUnionSmemMax = (kMaxNeurons / 32) * 4;  // bytes of those offsets at the largest n
+constexpr int kMaxNeurons = 1 << 20;  // n at most
 
 cudaError_t configure_predict();  // one-time kernel attributes (shared-memory limits)
 cudaError_t configure_ffn();

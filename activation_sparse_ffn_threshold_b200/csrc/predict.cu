@@ -207,22 +207,23 @@ __device__ __forceinline__ void transpose32(uint32_t *a) {
 }
 
 // The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
-// token t's set holds the row).  One CTA of kUnionThreads.  A warp takes 32 consecutive
-// bit words at a time, lane l word w = w0 + l: its b tokens' words arrive by coalesced
-// loads (the warp reads 32 consecutive words of one token at a time), the union word is
-// their OR, and a 32 x 32 bit transpose turns them into the token masks of the word's 32
-// rows.  Pass 1 counts each word's union bits, a block scan turns the counts into first
-// positions; pass 2 stages the warp's masks in shared memory and writes the rows word by
-// word, lane i taking bit i, so that the stores of a word are contiguous.
-constexpr int kUnionThreads = 512;
-constexpr int kUnionStage = 32 * 33;  // words of one warp's staged masks (rows padded to 33)
+// token t's set holds the row).  CTA k takes the 32 bit words [32k, 32k + 32): its threads
+// first count the union bits of all earlier words (every CTA in parallel, each bit word's
+// b token words read with coalesced loads, then OR and popc), so that no CTA waits on
+// another; then its first warp, lane l on word 32k + l, ORs the word's token words, turns
+// them into the token masks of the word's 32 rows by a 32 x 32 bit transpose, and writes
+// the rows word by word through a shared-memory stage, lane i taking bit i, so that the
+// stores of a word are contiguous.  The last CTA writes the union's size.
+constexpr int kUnionThreads = 1024;
+constexpr int kUnionStage = 32 * 33;  // words of the warp's staged masks (rows padded to 33)
 
 __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
                                                          int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
                                                          int32_t *__restrict__ ucount) {
-  extern __shared__ int woff[];  // [nwords]: union bits of each word, then its first position
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  uint32_t *stage = reinterpret_cast<uint32_t *>(woff + ((nwords + 3) & ~3)) + warp * kUnionStage;
+  __shared__ uint32_t stage[kUnionStage];
+  __shared__ int red[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int w0 = blockIdx.x * 32;
   const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
   auto load = [&](int w, uint32_t *mw) {  // token words of bit word w (w < nwords) -> their union
 #pragma unroll
@@ -232,48 +233,46 @@ __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restr
     for (int t = 0; t < kMaxBatch; ++t) u |= mw[t];
     return w == nwords - 1 ? u & tail : u;
   };
-  for (int w = threadIdx.x; w < nwords; w += blockDim.x) {
-    uint32_t mw[kMaxBatch];
-    woff[w] = __popc(load(w, mw));
-  }
-  __syncthreads();
-  const int per = (nwords + blockDim.x - 1) / blockDim.x;  // words per thread in the scan
-  const int s0 = threadIdx.x * per;
-  int sum = 0;
-  for (int k = 0; k < per; ++k)
-    if (s0 + k < nwords) sum += woff[s0 + k];
-  int total;
-  int run = block_exclusive_scan(sum, &total);
-  for (int k = 0; k < per; ++k)
-    if (s0 + k < nwords) {
-      const int v = woff[s0 + k];
-      woff[s0 + k] = run;
-      run += v;
-    }
-  __syncthreads();
-  for (int w0 = warp * 32; w0 < nwords; w0 += nwarps * 32) {  // warp-uniform
-    const int w = w0 + lane;
-    uint32_t mw[kMaxBatch];
-    const uint32_t u = w < nwords ? load(w, mw) : 0u;
-    const int base = w < nwords ? woff[w] : 0;
-    if (u != 0u) {
-      transpose32(mw);  // mw[i]: the tokens whose sets hold row 32 w + i
+  int before = 0;  // union bits of the words before this CTA's
+  for (int w = threadIdx.x; w < w0; w += blockDim.x) {
+    uint32_t u = 0u;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = mw[i];
-    }
-    __syncwarp();
-    for (int l = 0; l < 32; ++l) {
-      const uint32_t ul = __shfl_sync(0xffffffffu, u, l);
-      const int bl = __shfl_sync(0xffffffffu, base, l);
-      if ((ul >> lane) & 1u) {
-        const int pos = bl + __popc(ul & ((1u << lane) - 1u));
-        ulist[pos] = (w0 + l) * 32 + lane;
-        utok[pos] = stage[l * 33 + lane];
-      }
-    }
-    __syncwarp();
+    for (int t = 0; t < kMaxBatch; ++t) u |= t < b ? __ldcg(mask + (size_t)t * nwords + w) : 0u;
+    before += __popc(u);  // w < w0 <= nwords - 1: never the tail word
   }
-  if (threadIdx.x == 0) *ucount = total;
+  before = __reduce_add_sync(0xffffffffu, before);
+  if (lane == 0) red[warp] = before;
+  __syncthreads();
+  if (warp != 0) return;
+  int base = lane < (int)(blockDim.x >> 5) ? red[lane] : 0;
+  base = __reduce_add_sync(0xffffffffu, base);
+  const int w = w0 + lane;
+  uint32_t mw[kMaxBatch];
+  const uint32_t u = w < nwords ? load(w, mw) : 0u;
+  const int k = __popc(u);
+  int incl = k;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int first = base + incl - k;  // the first union position of word w
+  if (u != 0u) {
+    transpose32(mw);  // mw[i]: the tokens whose sets hold row 32 w + i
+#pragma unroll
+    for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = mw[i];
+  }
+  __syncwarp();
+  for (int l = 0; l < 32; ++l) {
+    const uint32_t ul = __shfl_sync(0xffffffffu, u, l);
+    const int bl = __shfl_sync(0xffffffffu, first, l);
+    if ((ul >> lane) & 1u) {
+      const int pos = bl + __popc(ul & ((1u << lane) - 1u));
+      ulist[pos] = (w0 + l) * 32 + lane;
+      utok[pos] = stage[l * 33 + lane];
+    }
+  }
+  if (blockIdx.x == gridDim.x - 1 && lane == 31) *ucount = base + incl;
 }
 
 // Block t: token t's set as indices in the caller's numbering, ascending in storage order.
@@ -368,9 +367,6 @@ cudaError_t logits_impl(const sfnn_ctx *h, int b, cudaStream_t s) {
 }  // namespace
 
 cudaError_t configure_predict() {
-  cudaError_t e0 = cudaFuncSetAttribute(k_union, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kUnionSmemMax + (kUnionThreads / 32) * kUnionStage * 4);
-  if (e0 != cudaSuccess) return e0;
   const void *ks[] = {(const void *)k_logits<float, 1>, (const void *)k_logits<float, 8>,
                       (const void *)k_logits<float, 32>, (const void *)k_logits<__half, 1>,
                       (const void *)k_logits<__half, 8>, (const void *)k_logits<__half, 32>};
@@ -399,8 +395,7 @@ cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *i
   const Layout &L = h->L;
   cudaError_t e = cudaSuccess;
   if (want_union) {
-    const size_t smem = ((size_t)(L.nwords + 3) / 4 * 4 + (size_t)(kUnionThreads / 32) * kUnionStage) * 4;
-    k_union<<<1, kUnionThreads, smem, s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
+    k_union<<<(L.nwords + 31) / 32, kUnionThreads, 0, s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && (idx_out || cnt_out)) {
