@@ -88,7 +88,7 @@ def load_library():
         "sfnn_set_fused_quota": ([P, I], S),
         "sfnn_set_batch_quota": ([P, I], S),
         "sfnn_set_batch_depths": ([P, I, I, I, I], S),
-        "sfnn_tune_batch_paths": ([P, P], S),
+        "sfnn_tune_batch_paths": ([P, P, P], S),
         "sfnn_set_fused_depths": ([P, I, I, I, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
         "sfnn_set_profile_events": ([P, P, P], S),
@@ -276,11 +276,14 @@ class SparseFFN:
 
     def tune_batch_paths(self, stream=None):
         """Measure which path serves AUTO batches just above the few-token kernel's size
-        faster (two few-token launches or tensor cores) and make AUTO take it (set-up call)."""
+        faster (two few-token launches or tensor cores) and make AUTO take it (set-up call).
+        Returns {b: (ms of two launches, ms of tensor cores)} for the b it measured."""
         import torch
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        ms = (ctypes.c_float * 18)()
         with torch.cuda.device(self.device):
-            _check(self._lib.sfnn_tune_batch_paths(self._h, ctypes.c_void_p(s.cuda_stream)), "sfnn_tune_batch_paths")
+            _check(self._lib.sfnn_tune_batch_paths(self._h, ms, ctypes.c_void_p(s.cuda_stream)), "sfnn_tune_batch_paths")
+        return {b: (ms[2 * b], ms[2 * b + 1]) for b in range(9) if ms[2 * b + 1] > 0}
 
     def set_batch_quota(self, enable: bool):
         """The few-token kernel's rebalancing (off: each token's y independent of the batch)."""

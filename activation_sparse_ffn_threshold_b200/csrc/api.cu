@@ -679,7 +679,7 @@ sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
   return SFNN_OK;
 }
 
-sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream) {
+sfnn_status sfnn_tune_batch_paths(sfnn_handle h, float *ms_out, sfnn_stream_t stream) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   if (!same_device(h)) return SFNN_ERR_INVALID_ARG;
   for (int b = 0; b <= kMaxBatch; ++b) h->auto_chunked[b] = false;
@@ -714,8 +714,8 @@ sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream) {
     const int saved = h->batch_path;
     auto time_path = [&](int path, int b, float *ms) -> sfnn_status {
       h->batch_path = path;
-      for (int i = 0; i < 7; ++i) {
-        if (i == 2) cudaEventRecord(e0, s);  // 2 warm-up calls, 5 timed
+      for (int i = 0; i < 13; ++i) {
+        if (i == 3) cudaEventRecord(e0, s);  // 3 warm-up calls, 10 timed
         const sfnn_status r = run_layer(h, X, b, kSetPredict, nullptr, nullptr, nullptr, nullptr, nullptr, Y, nullptr,
                                         nullptr, s);
         if (r != SFNN_OK) return r;
@@ -726,10 +726,18 @@ sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream) {
       return SFNN_OK;
     };
     for (int b = h->multi_max + 1; b <= bmax && st == SFNN_OK; ++b) {
-      float t_multi = 0.f, t_tc = 0.f;
-      st = time_path(SFNN_BATCH_FUSED, b, &t_multi);
-      if (st == SFNN_OK) st = time_path(SFNN_BATCH_TENSOR_CORE, b, &t_tc);
-      if (st == SFNN_OK) h->auto_chunked[b] = t_multi < t_tc;
+      float t_multi = 0.f, t_tc = 0.f, t_tc2 = 0.f;
+      st = time_path(SFNN_BATCH_TENSOR_CORE, b, &t_tc);  // tensor cores, two launches, tensor cores
+      if (st == SFNN_OK) st = time_path(SFNN_BATCH_FUSED, b, &t_multi);
+      if (st == SFNN_OK) st = time_path(SFNN_BATCH_TENSOR_CORE, b, &t_tc2);
+      t_tc = std::min(t_tc, t_tc2);
+      // two launches only when clearly faster (5 %): the tensor-core path's time varies less
+      // with the batch's union
+      if (st == SFNN_OK) h->auto_chunked[b] = t_multi < 0.95f * t_tc;
+      if (ms_out && st == SFNN_OK) {
+        ms_out[2 * b] = t_multi / 10.f;
+        ms_out[2 * b + 1] = t_tc / 10.f;
+      }
     }
     h->batch_path = saved;
   }

@@ -527,9 +527,11 @@ def measure_batch(cfg, b, args, dist, dev):
     per_batch = W.touched_bytes(cfg, W.expected_union_density(lay.p, b) * cfg.n, b)
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
     handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b, **_order_kw(args)) for _ in range(R)]
+    tuned = None
     if 4 < b <= 8:  # AUTO's measured choice between two few-token launches and tensor cores
         for h in handles:
-            h.tune_batch_paths()
+            t = h.tune_batch_paths()
+            tuned = tuned or t
     info = handles[0].info()
     torch.cuda.synchronize()
     X = torch.from_numpy(Xh).to(dev)
@@ -558,6 +560,8 @@ def measure_batch(cfg, b, args, dist, dev):
            "replicas": R, "path": path, "kernels_per_batch": launches // BATCHES_PER_STEP,
            "mean_union_rows": float(unions.mean()), "gpu_launches": int(launches * args.steps), "clocks": clocks,
            "bytes_per_step": float(bytes_batch.sum())}
+    if tuned:  # ms per call of (two few-token launches, tensor cores), synthetic tokens
+        out["tuned_ms"] = {str(k): [round(v[0], 4), round(v[1], 4)] for k, v in tuned.items()}
     two = b > 4 and launches // BATCHES_PER_STEP == 2
     tpath = "multi" if (b <= 4 and handles[0].info()["wdtype"] == 1) or two else "tcgen05"
     summary = f"batch_{cfg.name}_b{b}" + ("_two_launches" if two else "")
@@ -678,6 +682,7 @@ def _summary(cfg, what, b, m):
             "algorithmic_bytes": r["algorithmic_bytes_per_launch"], "traffic": r["traffic"],
             **({"path": m["path"], "mean_union_rows": m["mean_union_rows"], "kernels_per_batch":
                 m["kernels_per_batch"]} if "path" in m else {}),
+            **({"tuned_ms": m["tuned_ms"]} if "tuned_ms" in m else {}),
             **({"mean_active_neurons": m["mean_active_neurons"]} if "mean_active_neurons" in m else {}),
             **({"mean_active_neurons_per_layer": m["mean_active_neurons_per_layer"],
                 "launches_per_token": m["launches_per_token"]} if "layers" in m else {}),
@@ -756,7 +761,8 @@ def run_batch(args, dist):
                    "path": m["path"], "replicas": m["replicas"], "order": args.order,
                    "l2": f"inputs larger than L2: {m['replicas']} weight replicas rotated per batch, "
                          f"{m['bytes_per_step'] / BATCHES_PER_STEP / 1e6:.1f} MB touched per batch",
-                   "parallelism": f"replicas x{dist.world} (no exchange)", "mean_union_rows": m["mean_union_rows"]},
+                   "parallelism": f"replicas x{dist.world} (no exchange)", "mean_union_rows": m["mean_union_rows"],
+                   **({"tuned_ms": m["tuned_ms"]} if "tuned_ms" in m else {})},
         "effective_gbs": m["effective_gbs"], "roofline": m["roofline"], "cpu_baseline": None, "e2e": None,
         "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
     }

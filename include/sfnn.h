@@ -303,13 +303,16 @@ SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
  * Measures, on this handle, which path serves AUTO batches of multi_max + 1 .. 2 multi_max
  * tokens faster (multi_max: the few-token kernel's largest batch, 4 when it fits; at most
  * the handle's max_batch): two few-token launches of at most multi_max tokens each, or the
- * tensor-core batch path, on synthetic unit-variance tokens (fixed seed), 2 warm-up and 5
- * timed calls each, and makes AUTO take the faster one for each such b (SFNN_BATCH_FUSED
- * always takes the two launches).  Without this call AUTO takes the tensor-core path there.
+ * tensor-core batch path, on synthetic unit-variance tokens (fixed seed), 3 warm-up and 10
+ * timed calls each (the tensor-core path twice, around the other), and makes AUTO take the
+ * two launches for each such b where they are at least 5 % faster (SFNN_BATCH_FUSED always
+ * takes them).  Without this call AUTO takes the tensor-core path there.  ms_out (null, or
+ * 2 (2 multi_max + 1) floats) receives per b the milliseconds of one call of each path, at
+ * [2b] (two launches) and [2b + 1] (tensor cores).
  * Allocates and frees temporary device memory and synchronises `stream`: a set-up call, not
  * for graph capture.  SFNN_OK with nothing measured when the handle has no such b.
  */
-SFNN_API sfnn_status sfnn_tune_batch_paths(sfnn_handle h, sfnn_stream_t stream);
+SFNN_API sfnn_status sfnn_tune_batch_paths(sfnn_handle h, float *ms_out, sfnn_stream_t stream);
 
 /*
  * The few-token fused kernel's request depths, as sfnn_set_fused_depths (the results do not
