@@ -86,6 +86,10 @@ def parse_args(argv=None):
     ap.add_argument("--batch", type=int, default=1,
                     help="tokens per forward call: 1 is the single-token decode (the headline); b > 1 "
                          "times the batched union path on b tokens at a time")
+    ap.add_argument("--batch-path", choices=["auto", "cuda_core", "tensor_core", "fused"], default="auto",
+                    help="with --batch > 1: the batched path; auto measures, for 4 < b <= 8, two few-token "
+                         "launches against tensor cores before timing (a profiler slows the launches and "
+                         "skews that measurement: name the path there)")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="CPU budget of the reference arm (warm-up and timed steps together)")
     return ap.parse_args(argv)
@@ -528,7 +532,11 @@ def measure_batch(cfg, b, args, dist, dev):
     R = args.replicas or max(2, 1 + math.ceil(2 * l2 / per_batch))
     handles = [sf.SparseFFN.from_layer(lay, device=dev, max_batch=b, **_order_kw(args)) for _ in range(R)]
     tuned = None
-    if 4 < b <= 8:  # AUTO's measured choice between two few-token launches and tensor cores
+    bpath = {"auto": sf.BATCH_AUTO, "cuda_core": sf.BATCH_CUDA_CORE, "tensor_core": sf.BATCH_TENSOR_CORE,
+             "fused": sf.BATCH_FUSED}[args.batch_path]
+    for h in handles:
+        h.set_batch_path(bpath)
+    if bpath == sf.BATCH_AUTO and 4 < b <= 8:  # AUTO's measured choice: two few-token launches or tensor cores
         for h in handles:
             t = h.tune_batch_paths()
             tuned = tuned or t
