@@ -35,7 +35,7 @@ struct DeviceGuard {
 void free_handle(sfnn_ctx *h) {
   if (!h) return;
   void *bufs[] = {h->rows, h->At,    h->Bt,    h->cvec,  h->bias, h->perm, h->iperm, h->h,
-                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->rscale, h->alist, h->acnt, h->scnt, h->blist, h->bcnt};
+                  h->mask, h->ulist, h->utok,  h->ucount, h->acoef, h->part, h->xin,   h->err, h->bar, h->hact, h->hpair, h->upart, h->tcnt, h->rscale, h->alist, h->acnt, h->scnt, h->blist, h->bcnt};
   for (void *p : bufs)
     if (p) cudaFree(p);
   delete h;
@@ -476,6 +476,9 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->bcnt, (size_t)G * 4, false},
       {(void **)&h->hact, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)32 * tc_hstride(L.n) * 2 : 0, false},
       {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
+      {(void **)&h->upart, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? tc_up_partial_bytes(h->num_sms, (int)mb) : 0,
+       false},
+      {(void **)&h->tcnt, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)tc_hstride(L.n) / 128 * 4 : 0, false},
   };
   for (auto &q : reqs) {
     if (q.bytes == 0) continue;  // not needed by this layer
@@ -493,6 +496,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, sizeof(uint64_t), s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->alist, 0, n * sizeof(int2), s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->acnt, 0, (size_t)G * 4, s);
+  if (ce == cudaSuccess && h->tcnt) ce = cudaMemsetAsync(h->tcnt, 0, (size_t)tc_hstride(L.n) / 128 * 4, s);
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();

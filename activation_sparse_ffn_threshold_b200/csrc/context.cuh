@@ -30,6 +30,8 @@ struct sfnn_ctx {
   __half *hact;      // [32][n rounded up to 128] fp16 activations (tensor-core batch path) or null
   __half *hpair;     // [2][32][r] the batch's hidden layer as fp16 hi and lo parts (same path)
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
+  float *upart;      // tensor-core up projection: fp32 partials of tiles split between CTAs
+  int32_t *tcnt;     // [n / 128 rounded up] its per-tile arrival counters (zero between launches)
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
   uint64_t *bar;     // grid barrier arrival counter of the fused kernel

@@ -144,20 +144,21 @@ __device__ __forceinline__ void tc_end(uint32_t tmem) {
 }
 // The K loop: `load(s, it)` copies iteration it's operands into stage s (cp.async, all
 // threads); `issue(stage_smem_addr, it)` issues its MMAs (thread 0), which are committed
-// to the stage's mbarrier; the stage is refilled once they are done.  Returns false if a
-// wait ran out (then `fail` is set).  On return every MMA has completed (or failed) and
-// the accumulators may be read after tc_fence_after.
+// to the stage's mbarrier; the stage is refilled once they are done.  `base` counts the
+// iterations this CTA ran in earlier calls (they fix the stage and mbarrier phase of
+// each iteration).  Returns false if a wait ran out (then `fail` is set).  On return every
+// MMA has completed (or failed) and the accumulators may be read after tc_fence_after.
 template <class Load, class Issue>
 __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_bytes, int stages, int nk,
-                                            uint64_t *mbar, int *fail, Load load, Issue issue) {
+                                            uint64_t *mbar, int *fail, Load load, Issue issue, int base = 0) {
   const int tid = threadIdx.x;
   for (int s = 0; s < stages - 1; ++s) {
-    if (s < nk) load(s, s);
+    if (s < nk) load((base + s) % stages, s);
     cp_async_commit();
   }
   bool ok = true;
   for (int it = 0; it < nk && ok; ++it) {
-    const int s = it % stages;
+    const int j = base + it, s = j % stages;
     // committed groups: stages - 1 + it; iteration it's is the (it + 1)-th oldest
     switch (stages) {
       case 2: cp_async_wait<0>(); break;
@@ -173,86 +174,68 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
     }
     const int nx = it + stages - 1;  // refill the stage iteration it - 1 read, once its MMAs are done
     if (nx < nk) {
-      if (it >= 1 && !mb_wait(&mbar[(it - 1) % stages], (uint32_t)(((it - 1) / stages) & 1))) *fail = 1;
-      load(nx % stages, nx);
+      if (it >= 1 && !mb_wait(&mbar[(j - 1) % stages], (uint32_t)(((j - 1) / stages) & 1))) *fail = 1;
+      load((base + nx) % stages, nx);
     }
     cp_async_commit();
     __syncthreads();
     ok = *fail == 0;
   }
   cp_async_wait<0>();
-  if (ok && nk > 0 && !mb_wait(&mbar[(nk - 1) % stages], (uint32_t)(((nk - 1) / stages) & 1))) *fail = 1;
+  if (ok && nk > 0 && !mb_wait(&mbar[(base + nk - 1) % stages], (uint32_t)(((base + nk - 1) / stages) & 1)))
+    *fail = 1;
   tc_fence_after();
   __syncthreads();
   return *fail == 0;
 }
 
 // ---------------------------------------------------------------- k_tc_up
+// Stream-K: the union's 128-row tiles times their d/64 K chunks are T iterations, and CTA
+// g of G runs iterations [g T / G, (g + 1) T / G) -- so every SM stays busy however few
+// tiles the union makes.  A CTA's range is cut at tile edges into segments.  A segment that
+// is a whole tile ends in the epilogue; a part of a tile leaves its fp32 accumulators in
+// upart (slot 2g for the CTA's first tile, 2g + 1 for its last) and counts itself in
+// tcnt[tile]; the tile's last segment to arrive adds the tile's partials in CTA order
+// (deterministic), runs the epilogue and zeroes the counter for the next launch.  No CTA
+// waits for another.
 // smem per stage: NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B).
 template <int ACT>
 __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
                                                const __half *__restrict__ X, const int32_t *__restrict__ ulist,
                                                const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
                                                __half *__restrict__ H, int hstride, int d, int b, int N, int nproj,
-                                               int stages, int32_t *err) {
+                                               int stages, float *__restrict__ upart, int32_t *__restrict__ tcnt,
+                                               int32_t *err) {
   constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
-  __shared__ int fail;
+  __shared__ int fail, last_s;
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int U = *ucount;
-  const int u0 = blockIdx.x * kTM;
-  if (u0 >= U) return;
+  const int nk = d / kTK;
+  const int64_t T = (int64_t)((U + kTM - 1) / kTM) * nk;
+  const int64_t G = T < (int64_t)gridDim.x ? T : (int64_t)gridDim.x;  // every range non-empty
+  const int64_t g = blockIdx.x;
+  if (g >= G) return;
+  int64_t i0 = g * T / G;
+  const int64_t i1 = (g + 1) * T / G;
+  // the CTA whose range holds iteration i: the largest g' with g' T / G <= i
+  auto cta_of = [&](int64_t i) { return ((i + 1) * G + T - 1) / T - 1; };
+  const int first_tile = (int)(i0 / nk);
   const uint32_t stage_bytes = NP * 16384u + (uint32_t)N * 128u;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
-
-  // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
-  const int c8 = tid & 7;
-  const __half *src[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int u = u0 + (tid >> 3) + 16 * i;
-    u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
-    src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
-  }
-  auto load = [&](int s, int kc) {
-    unsigned char *st = smem + (size_t)s * stage_bytes;
-#pragma unroll
-    for (int j = 0; j < NP; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
-    unsigned char *xt = st + NP * 16384;
-    for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
-      const int t = q >> 3, c = q & 7;
-      const int tt = t < b ? t : b - 1;
-      cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
-    }
-  };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
-  auto issue = [&](uint32_t st, int it) {
-    const uint32_t xt = st + NP * 16384;
-#pragma unroll
-    for (int k = 0; k < kTK / 16; ++k) {
-      const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
-        umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
-                 (it > 0 || k > 0) ? 1u : 0u);
-    }
-  };
-  if (!tc_mainloop(smem, stage_bytes, stages, d / kTK, mbar, &fail, load, issue)) {
-    if (tid == 0) latch_error(err, kErrTimeout);
-  } else {
-    const int row = warp * 32 + lane;
-    const int u = u0 + row;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    float g[32], up[32];
-    for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + c0, g + c0);
-    if (ACT == SFNN_REGLU)
-      for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + N + c0, up + c0);
+  const int c8 = tid & 7, row = warp * 32 + lane;
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  bool ok = true;
+  int base = 0;  // iterations run so far (stage and mbarrier phase of the next one)
+
+  // bias + ReLU / ReGLU of this thread's row of tile m; zero for the tokens whose set
+  // does not hold the row -> H[token][union] (fp16)
+  auto epilogue = [&](int m, const float *gs, const float *us) {
+    const int u = m * kTM + row;
     if (u < U) {
       const int p = ulist[u];
       const uint32_t tm = utok[u];
@@ -260,15 +243,102 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       for (int t = 0; t < N; ++t) {
         float a = 0.f;
         if (t < b && ((tm >> t) & 1u)) {
-          const float pre = g[t] + bv;
+          const float pre = gs[t] + bv;
           a = pre > 0.f ? pre : 0.f;
-          if (ACT == SFNN_REGLU) a *= up[t];
+          if (ACT == SFNN_REGLU) a *= us[t];
         }
         H[(size_t)t * hstride + u] = __float2half_rn(a);
       }
     } else if (u < hstride) {  // the union's padding up to the down GEMM's K chunks: zeros
       for (int t = 0; t < N; ++t) H[(size_t)t * hstride + u] = __float2half_rn(0.f);
     }
+  };
+
+  while (i0 < i1) {
+    const int m = (int)(i0 / nk);
+    const int k0 = (int)(i0 - (int64_t)m * nk);
+    const int k1 = (int)(i1 - (int64_t)m * nk < nk ? i1 - (int64_t)m * nk : nk);
+    const int u0 = m * kTM;
+    // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
+    const __half *src[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int u = u0 + (tid >> 3) + 16 * i;
+      u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
+      src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
+    }
+    auto load = [&](int s, int it) {
+      const int kc = k0 + it;
+      unsigned char *st = smem + (size_t)s * stage_bytes;
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
+      unsigned char *xt = st + NP * 16384;
+      for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
+        const int t = q >> 3, c = q & 7;
+        const int tt = t < b ? t : b - 1;
+        cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+      }
+    };
+    auto issue = [&](uint32_t st, int it) {
+      const uint32_t xt = st + NP * 16384;
+#pragma unroll
+      for (int k = 0; k < kTK / 16; ++k) {
+        const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
+                   (it > 0 || k > 0) ? 1u : 0u);
+      }
+    };
+    if (ok && !tc_mainloop(smem, stage_bytes, stages, k1 - k0, mbar, &fail, load, issue, base)) {
+      ok = false;
+      if (tid == 0) latch_error(err, kErrTimeout);
+    }
+    base += k1 - k0;
+    float gs[32], us[32];
+    if (ok) {
+      for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + c0, gs + c0);
+      if (ACT == SFNN_REGLU)
+        for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + N + c0, us + c0);
+    } else {  // after a timeout the tile is still counted (the error is latched)
+      for (int t = 0; t < 32; ++t) gs[t] = us[t] = 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();  // every TMEM read is done before the next segment's MMAs
+    if (k0 == 0 && k1 == nk) {
+      epilogue(m, gs, us);
+    } else {
+      const int slot = 2 * (int)g + (m == first_tile ? 0 : 1);
+      for (int t = 0; t < b; ++t) {
+        upart[((size_t)slot * NP * b + t) * kTM + row] = gs[t];
+        if (ACT == SFNN_REGLU) upart[((size_t)slot * NP * b + b + t) * kTM + row] = us[t];
+      }
+      __threadfence();
+      __syncthreads();
+      const int64_t ga = cta_of((int64_t)m * nk), gb = cta_of((int64_t)m * nk + nk - 1);
+      if (tid == 0) {
+        const int prev = atomicAdd(&tcnt[m], 1);
+        last_s = prev == (int)(gb - ga);
+        if (last_s) tcnt[m] = 0;  // every segment of the tile has arrived: ready for the next launch
+      }
+      __syncthreads();
+      if (last_s) {
+        __threadfence();
+        for (int t = 0; t < b; ++t) gs[t] = us[t] = 0.f;
+        for (int64_t q = ga; q <= gb; ++q) {  // CTA order
+          const int qs = 2 * (int)q + ((int)((q * T / G) / nk) == m ? 0 : 1);
+          for (int t = 0; t < b; ++t) {
+            gs[t] += __ldcg(&upart[((size_t)qs * NP * b + t) * kTM + row]);
+            if (ACT == SFNN_REGLU) us[t] += __ldcg(&upart[((size_t)qs * NP * b + b + t) * kTM + row]);
+          }
+        }
+        epilogue(m, gs, us);
+      }
+    }
+    i0 = (int64_t)(m + 1) * nk;
   }
   tc_end(tmem);
 }
@@ -496,6 +566,13 @@ bool tc_predict_supported(const sfnn_ctx *h) { return tc_batch_supported(h) && h
 
 int tc_hstride(int n) { return (n + kTM - 1) / kTM * kTM; }
 
+// k_tc_up's grid: two CTAs per SM (3 stages of at most 37 KB each fit twice).
+int tc_up_ctas(int num_sms) { return 2 * num_sms; }
+
+size_t tc_up_partial_bytes(int num_sms, int max_batch) {
+  return (size_t)2 * tc_up_ctas(num_sms) * 2 * (size_t)max_batch * kTM * sizeof(float);
+}
+
 cudaError_t configure_tc_batch() {
   cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)up_smem(SFNN_RELU, 32));
@@ -546,15 +623,15 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int N = b <= 16 ? 16 : 32;
   const int hs = tc_hstride(L.n);
   const __half *rows = static_cast<const __half *>(h->rows);
-  const int up_grid = (L.n + kTM - 1) / kTM;
+  const int up_grid = tc_up_ctas(h->num_sms);
   if (L.act == SFNN_REGLU)
     k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
         rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->upart, h->tcnt, h->err);
   else
     k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
         rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->err);
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->upart, h->tcnt, h->err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int mtiles = L.d / kTM;
