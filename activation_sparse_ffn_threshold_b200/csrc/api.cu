@@ -387,6 +387,8 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   // quota): 70B-shaped 63.4 -> 55.5 (23 rows per tile, 32 KB), OPT-30B-shaped 44.1 -> 40.1
   // (19.5, 14 KB), LLaMA-7B-shaped 28.8 -> 27.2 (11.2, 16 KB); the OPT-6.7B-shaped layer
   // (11, 8 KB: 81 KB) loses 2.4 with one.  No profile, no rebalancing.
+  h->tc_up_ctas_per_sm = 2;
+  h->tc_up_kps = 1;
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;
@@ -680,6 +682,16 @@ sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
   const int v[4] = {bstages, c2pre, c1depth, c2stages};
   for (int i = 0; i < 4; ++i)
     if (v[i] != -1) h->mdepth[i] = v[i];
+  return SFNN_OK;
+}
+
+sfnn_status sfnn_set_batch_tc_up(sfnn_handle h, int32_t ctas_per_sm, int32_t chunks_per_step) {
+  if (!h) return SFNN_ERR_INVALID_ARG;
+  if (ctas_per_sm < -1 || ctas_per_sm == 0 || ctas_per_sm > 2) return SFNN_ERR_INVALID_ARG;
+  if (chunks_per_step < -1 || chunks_per_step == 0 || chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
+  if (!tc_batch_supported(h)) return SFNN_ERR_UNSUPPORTED;
+  if (ctas_per_sm != -1) h->tc_up_ctas_per_sm = ctas_per_sm;
+  if (chunks_per_step != -1) h->tc_up_kps = chunks_per_step;
   return SFNN_OK;
 }
 

@@ -36,7 +36,6 @@ bool tc_batch_supported(const sfnn_ctx *h);
 bool tc_predict_supported(const sfnn_ctx *h);  // and r a multiple of 64
 cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStream_t s);
 int tc_hstride(int n);
-int tc_up_ctas(int num_sms);
 size_t tc_up_partial_bytes(int num_sms, int max_batch);
 cudaError_t configure_tc_batch();
 cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits_out, cudaStream_t s);

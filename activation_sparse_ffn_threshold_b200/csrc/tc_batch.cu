@@ -190,7 +190,8 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
 }
 
 // ---------------------------------------------------------------- k_tc_up
-// Stream-K: the union's 128-row tiles times their d/64 K chunks are T iterations, and CTA
+// Stream-K: the union's 128-row tiles times their d/(64 kps) K steps are T iterations (a
+// step stages kps 64-wide K chunks of every row: 128 kps contiguous bytes), and CTA
 // g of G runs iterations [g T / G, (g + 1) T / G) -- so every SM stays busy however few
 // tiles the union makes.  A CTA's range is cut at tile edges into segments.  A segment that
 // is a whole tile ends in the epilogue; a part of a tile leaves its fp32 accumulators in
@@ -198,14 +199,14 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
 // tcnt[tile]; the tile's last segment to arrive adds the tile's partials in CTA order
 // (deterministic), runs the epilogue and zeroes the counter for the next launch.  No CTA
 // waits for another.
-// smem per stage: NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B).
+// smem per stage: kps times (NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B)).
 template <int ACT>
 __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
                                                const __half *__restrict__ X, const int32_t *__restrict__ ulist,
                                                const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
                                                __half *__restrict__ H, int hstride, int d, int b, int N, int nproj,
-                                               int stages, float *__restrict__ upart, int32_t *__restrict__ tcnt,
-                                               int32_t *err) {
+                                               int stages, int kps, float *__restrict__ upart,
+                                               int32_t *__restrict__ tcnt, int32_t *err) {
   constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int U = *ucount;
-  const int nk = d / kTK;
+  const int nk = d / (kTK * kps);  // K steps of a tile
   const int64_t T = (int64_t)((U + kTM - 1) / kTM) * nk;
   const int64_t G = T < (int64_t)gridDim.x ? T : (int64_t)gridDim.x;  // every range non-empty
   const int64_t g = blockIdx.x;
@@ -224,7 +225,8 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   // the CTA whose range holds iteration i: the largest g' with g' T / G <= i
   auto cta_of = [&](int64_t i) { return ((i + 1) * G + T - 1) / T - 1; };
   const int first_tile = (int)(i0 / nk);
-  const uint32_t stage_bytes = NP * 16384u + (uint32_t)N * 128u;
+  const uint32_t chunk_bytes = NP * 16384u + (uint32_t)N * 128u;  // a multiple of 1024
+  const uint32_t stage_bytes = (uint32_t)kps * chunk_bytes;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
   const int c8 = tid & 7, row = warp * 32 + lane;
@@ -268,29 +270,33 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
     }
     auto load = [&](int s, int it) {
-      const int kc = k0 + it;
-      unsigned char *st = smem + (size_t)s * stage_bytes;
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
+      for (int a = 0; a < kps; ++a) {
+        const int kc = (k0 + it) * kps + a;
+        unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
-      unsigned char *xt = st + NP * 16384;
-      for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
-        const int t = q >> 3, c = q & 7;
-        const int tt = t < b ? t : b - 1;
-        cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+#pragma unroll
+          for (int j = 0; j < NP; ++j)
+            cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
+        unsigned char *xt = st + NP * 16384;
+        for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
+          const int t = q >> 3, c = q & 7;
+          const int tt = t < b ? t : b - 1;
+          cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+        }
       }
     };
     auto issue = [&](uint32_t st, int it) {
-      const uint32_t xt = st + NP * 16384;
+      for (int a = 0; a < kps; ++a) {
+        const uint32_t at = st + (uint32_t)a * chunk_bytes, xt = at + NP * 16384;
 #pragma unroll
-      for (int k = 0; k < kTK / 16; ++k) {
-        const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
+        for (int k = 0; k < kTK / 16; ++k) {
+          const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(st + j * 16384 + k * 32, 16, 1024), bd, idesc,
-                   (it > 0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < NP; ++j)
+            umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(at + j * 16384 + k * 32, 16, 1024), bd, idesc,
+                     (it > 0 || a > 0 || k > 0) ? 1u : 0u);
+        }
       }
     };
     if (ok && !tc_mainloop(smem, stage_bytes, stages, k1 - k0, mbar, &fail, load, issue, base)) {
@@ -551,7 +557,9 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
 
 constexpr int kUpStages = 3, kDownStages = 3, kPredStages = 4;
 
-size_t up_smem(int act, int N) { return (size_t)kUpStages * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024; }
+size_t up_smem(int act, int N, int kps) {
+  return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024;
+}
 size_t down_smem(int N) { return (size_t)kDownStages * (16384 + N * 128) + 1024; }
 size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
 size_t logits_smem(int N) { return (size_t)kPredStages * (16384 + 2 * N * 128) + 1024; }
@@ -566,19 +574,18 @@ bool tc_predict_supported(const sfnn_ctx *h) { return tc_batch_supported(h) && h
 
 int tc_hstride(int n) { return (n + kTM - 1) / kTM * kTM; }
 
-// k_tc_up's grid: two CTAs per SM (3 stages of at most 37 KB each fit twice).
-int tc_up_ctas(int num_sms) { return 2 * num_sms; }
-
+// k_tc_up's largest grid: two CTAs per SM (3 stages of one K chunk, at most 37 KB each,
+// fit twice); its partials: two slots per CTA.
 size_t tc_up_partial_bytes(int num_sms, int max_batch) {
-  return (size_t)2 * tc_up_ctas(num_sms) * 2 * (size_t)max_batch * kTM * sizeof(float);
+  return (size_t)2 * (2 * num_sms) * 2 * (size_t)max_batch * kTM * sizeof(float);
 }
 
 cudaError_t configure_tc_batch() {
   cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)up_smem(SFNN_RELU, 32));
+                                       (int)up_smem(SFNN_RELU, 32, 2));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)up_smem(SFNN_REGLU, 32));
+                             (int)up_smem(SFNN_REGLU, 32, 2));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32));
   if (e == cudaSuccess)
@@ -623,15 +630,16 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int N = b <= 16 ? 16 : 32;
   const int hs = tc_hstride(L.n);
   const __half *rows = static_cast<const __half *>(h->rows);
-  const int up_grid = tc_up_ctas(h->num_sms);
+  const int up_grid = h->tc_up_ctas_per_sm * h->num_sms;
+  const int kps = L.d % (2 * kTK) == 0 ? h->tc_up_kps : 1;
   if (L.act == SFNN_REGLU)
-    k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+    k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N, kps), s>>>(
         rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->upart, h->tcnt, h->err);
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
   else
-    k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N), s>>>(
+    k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N, kps), s>>>(
         rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, h->upart, h->tcnt, h->err);
+        h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int mtiles = L.d / kTM;

@@ -300,6 +300,17 @@ SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
 SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
 
 /*
+ * The tensor-core batch path's up projection shape (a tuning knob; the results do not depend
+ * on it beyond the order in which a split tile's partial sums are added): ctas_per_sm = its
+ * CTAs per SM (1 or 2; the union's (128-row tile, K step) pairs are shared out evenly
+ * among them), chunks_per_step = 64-wide K chunks of every row staged per step (1 or 2;
+ * 2 needs d a multiple of 128 and fits one CTA per SM).  -1 keeps a value.
+ * SFNN_ERR_INVALID_ARG outside those sets; SFNN_ERR_UNSUPPORTED when the layer has no
+ * tensor-core batch path.  Takes effect at the next launch.
+ */
+SFNN_API sfnn_status sfnn_set_batch_tc_up(sfnn_handle h, int32_t ctas_per_sm, int32_t chunks_per_step);
+
+/*
  * Measures, on this handle, which path serves AUTO batches of multi_max + 1 .. 2 multi_max
  * tokens faster (multi_max: the few-token kernel's largest batch, 4 when it fits; at most
  * the handle's max_batch): two few-token launches of at most multi_max tokens each, or the
