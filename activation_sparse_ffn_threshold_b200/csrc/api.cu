@@ -387,8 +387,13 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   // quota): 70B-shaped 63.4 -> 55.5 (23 rows per tile, 32 KB), OPT-30B-shaped 44.1 -> 40.1
   // (19.5, 14 KB), LLaMA-7B-shaped 28.8 -> 27.2 (11.2, 16 KB); the OPT-6.7B-shaped layer
   // (11, 8 KB: 81 KB) loses 2.4 with one.  No profile, no rebalancing.
+  // the tensor-core up projection: 2 K chunks per step (256 contiguous bytes of each row
+  // per request round) on as many CTAs per SM as fit, up to 2.  Measured (us per batch,
+  // CTAs per SM x chunks: 2x1 / 1x1 / 1x2 / 2x2): 70B-shaped b = 8 184 / 199 / 175 / 188,
+  // b = 32 297 / 326 / 283 / 303 (2x2 fits one CTA per SM there, so it runs two waves);
+  // OPT-30B-shaped b = 8 124 / 137 / 122 / 115 (2x2 fits twice)
   h->tc_up_ctas_per_sm = 2;
-  h->tc_up_kps = 1;
+  h->tc_up_kps = 2;
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;

@@ -574,10 +574,25 @@ bool tc_predict_supported(const sfnn_ctx *h) { return tc_batch_supported(h) && h
 
 int tc_hstride(int n) { return (n + kTM - 1) / kTM * kTM; }
 
-// k_tc_up's largest grid: two CTAs per SM (3 stages of one K chunk, at most 37 KB each,
-// fit twice); its partials: two slots per CTA.
+// k_tc_up's largest grid: two CTAs per SM; its partials: two slots per CTA.
 size_t tc_up_partial_bytes(int num_sms, int max_batch) {
   return (size_t)2 * (2 * num_sms) * 2 * (size_t)max_batch * kTM * sizeof(float);
+}
+
+// k_tc_up CTAs that fit on an SM at once for this shape (measured once per shape).
+static int up_fit(int act, int N, int kps) {
+  static int cache[2][2][2] = {};
+  int &c = cache[act == SFNN_REGLU][N == 32][kps - 1];
+  if (c == 0) {
+    int nb = 0;
+    const cudaError_t e =
+        act == SFNN_REGLU
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_up<SFNN_REGLU>, kTT, up_smem(act, N, kps))
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_up<SFNN_RELU>, kTT, up_smem(act, N, kps));
+    if (e != cudaSuccess) cudaGetLastError();
+    c = e == cudaSuccess && nb > 0 ? nb : 1;
+  }
+  return c;
 }
 
 cudaError_t configure_tc_batch() {
@@ -592,6 +607,10 @@ cudaError_t configure_tc_batch() {
     e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)logits_smem(32));
+  // the occupancy of every up-projection shape, outside any stream capture
+  for (int act : {SFNN_RELU, SFNN_REGLU})
+    for (int N : {16, 32})
+      for (int kps : {1, 2}) up_fit(act, N, kps);
   return e;
 }
 
@@ -630,8 +649,8 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int N = b <= 16 ? 16 : 32;
   const int hs = tc_hstride(L.n);
   const __half *rows = static_cast<const __half *>(h->rows);
-  const int up_grid = h->tc_up_ctas_per_sm * h->num_sms;
   const int kps = L.d % (2 * kTK) == 0 ? h->tc_up_kps : 1;
+  const int up_grid = std::min(h->tc_up_ctas_per_sm, up_fit(L.act, N, kps)) * h->num_sms;
   if (L.act == SFNN_REGLU)
     k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N, kps), s>>>(
         rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,

@@ -302,9 +302,11 @@ SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
 /*
  * The tensor-core batch path's up projection shape (a tuning knob; the results do not depend
  * on it beyond the order in which a split tile's partial sums are added): ctas_per_sm = its
- * CTAs per SM (1 or 2; the union's (128-row tile, K step) pairs are shared out evenly
- * among them), chunks_per_step = 64-wide K chunks of every row staged per step (1 or 2;
- * 2 needs d a multiple of 128 and fits one CTA per SM).  -1 keeps a value.
+ * CTAs per SM (1 or 2, capped by how many fit in shared memory; the union's (128-row tile,
+ * K step) pairs are shared out evenly among them), chunks_per_step = 64-wide K chunks of
+ * every row staged per step (1 or 2; two make each row's reads 256 contiguous bytes).
+ * Default 2 and 2 (one CTA per SM fits for ReGLU layers and for ReLU layers past 16
+ * tokens).  -1 keeps a value.
  * SFNN_ERR_INVALID_ARG outside those sets; SFNN_ERR_UNSUPPORTED when the layer has no
  * tensor-core batch path.  Takes effect at the next launch.
  */
