@@ -394,6 +394,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   // OPT-30B-shaped b = 8 124 / 137 / 122 / 115 (2x2 fits twice)
   h->tc_up_ctas_per_sm = 2;
   h->tc_up_kps = 2;
+  h->tc_down_mps = 1;
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;
@@ -690,13 +691,16 @@ sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
   return SFNN_OK;
 }
 
-sfnn_status sfnn_set_batch_tc_up(sfnn_handle h, int32_t ctas_per_sm, int32_t chunks_per_step) {
+sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32_t up_chunks_per_step,
+                                    int32_t down_tiles_per_cta) {
   if (!h) return SFNN_ERR_INVALID_ARG;
-  if (ctas_per_sm < -1 || ctas_per_sm == 0 || ctas_per_sm > 2) return SFNN_ERR_INVALID_ARG;
-  if (chunks_per_step < -1 || chunks_per_step == 0 || chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
+  if (up_ctas_per_sm < -1 || up_ctas_per_sm == 0 || up_ctas_per_sm > 2) return SFNN_ERR_INVALID_ARG;
+  if (up_chunks_per_step < -1 || up_chunks_per_step == 0 || up_chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
+  if (down_tiles_per_cta < -1 || down_tiles_per_cta == 0 || down_tiles_per_cta > 2) return SFNN_ERR_INVALID_ARG;
   if (!tc_batch_supported(h)) return SFNN_ERR_UNSUPPORTED;
-  if (ctas_per_sm != -1) h->tc_up_ctas_per_sm = ctas_per_sm;
-  if (chunks_per_step != -1) h->tc_up_kps = chunks_per_step;
+  if (up_ctas_per_sm != -1) h->tc_up_ctas_per_sm = up_ctas_per_sm;
+  if (up_chunks_per_step != -1) h->tc_up_kps = up_chunks_per_step;
+  if (down_tiles_per_cta != -1) h->tc_down_mps = down_tiles_per_cta;
   return SFNN_OK;
 }
 

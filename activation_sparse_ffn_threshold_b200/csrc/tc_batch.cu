@@ -12,9 +12,9 @@
 //              (K-major), accumulators in TMEM.  Epilogue: + b, ReLU / ReGLU, zero for
 //              the tokens whose set does not hold the row -> H[token][union] (fp16).
 //   k_tc_down  Y^T[cols][token] = W_down[U]^T . H^T over a split of the union: A = the
-//              gathered down rows, 128 output columns each (MN-major: a row is contiguous
-//              along d), B = H (K-major) -> part[split][token][cols]; k_reduce adds the
-//              splits in a fixed order.
+//              gathered down rows, 128 (or 256) output columns each (MN-major: a row is
+//              contiguous along d), B = H (K-major) -> part[split][token][cols]; k_reduce
+//              adds the splits in a fixed order.
 //   k_tc_hidden, k_tc_hsum, k_tc_logits  the predictor of the batch (dense GEMMs over
 //              A^T and B^T), ending in the token-major decision masks k_compact reads.
 //
@@ -350,12 +350,15 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
 }
 
 // ---------------------------------------------------------------- k_tc_down
-// smem per stage: the A tile (64 union rows x 128 columns, MN-major, 16 KB) + the H tile
-// (N tokens x 64 union entries, K-major).
+// A CTA computes mps adjacent 128-column output tiles (each a TMEM accumulator of N
+// columns) over its split of the union.  smem per stage: mps A tiles (64 union rows x 128
+// columns, MN-major, 16 KB each) + the H tile (N tokens x 64 union entries, K-major).  A
+// warp's copy instruction covers 2 / mps union rows of 256 mps contiguous bytes.
 __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows, const __half *__restrict__ H,
                                                  int hstride, const int32_t *__restrict__ ulist,
                                                  const int32_t *__restrict__ ucount, float *__restrict__ part, int d,
-                                                 int b, int N, int nproj, int splits, int stages, int32_t *err) {
+                                                 int b, int N, int nproj, int splits, int stages, int mps,
+                                                 int32_t *err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -366,31 +369,35 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   const int U = *ucount;
   const int nkc = (U + kTK - 1) / kTK;
   const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
-  const int col0 = mt * kTM;
-  const uint32_t stage_bytes = 16384u + (uint32_t)N * 128u;
+  const int col0 = mt * kTM * mps;
+  const uint32_t a_bytes = (uint32_t)mps * 16384u;
+  const uint32_t stage_bytes = a_bytes + (uint32_t)N * 128u;
 
   if (c0 == c1) {  // an empty split still provides its (zero) partial
-    for (int q = tid; q < b * kTM; q += kTT) part[((size_t)ks * b + q / kTM) * d + col0 + q % kTM] = 0.f;
+    for (int q = tid; q < b * kTM * mps; q += kTT)
+      part[((size_t)ks * b + q / (kTM * mps)) * d + col0 + q % (kTM * mps)] = 0.f;
     return;
   }
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
 
-  // A: chunk q = tid + 128 i -> union row k = q / 16 of the stage, 16-byte column chunk
-  // c = q % 16; MN atom m' = c / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
+  // A: chunk q = tid + 128 i -> union row k = q / (16 mps) of the stage, 16-byte column
+  // chunk c = q % (16 mps) of its 256 mps bytes: tile mp = c / 16, and within it MN atom
+  // m' = (c % 16) / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
+  const int cpr = 16 * mps;  // 16-byte chunks of a row
   auto load = [&](int s, int it) {
     const int kc = c0 + it;
     unsigned char *st = smem + (size_t)s * stage_bytes;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 8 * mps; ++i) {
       const int q = tid + kTT * i;
-      const int k = q >> 4, c = q & 15;
+      const int k = q / cpr, c = q % cpr;
       int u = kc * kTK + k;
       u = u < U ? u : U - 1;  // past the union: a repeated row times H's zero padding
-      const int k0 = k & 7, k1 = k >> 3, mp = c >> 3, cc = c & 7;
-      const uint32_t off = (uint32_t)(mp * 1024 + k1 * 2048 + k0 * 128 + ((cc ^ k0) << 4));
+      const int mp = c >> 4, c16 = c & 15;
+      const int k0 = k & 7, k1 = k >> 3, ma = c16 >> 3, cc = c16 & 7;
+      const uint32_t off = (uint32_t)(mp * 16384 + ma * 1024 + k1 * 2048 + k0 * 128 + ((cc ^ k0) << 4));
       cp16(st, off, rows + ((size_t)ulist[u] * nproj + (nproj - 1)) * d + col0 + c * 8);
     }
-    unsigned char *ht = st + 16384;
+    unsigned char *ht = st + a_bytes;
     for (int q = tid; q < N * 8; q += kTT) {
       const int t = q >> 3, c = q & 7;
       cp16(ht, kmajor_off(t, c), H + (size_t)t * hstride + (size_t)kc * kTK + c * 8);
@@ -398,11 +405,12 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   };
   const uint32_t idesc = idesc_f16(kTM, N, 1, 0);
   auto issue = [&](uint32_t st, int it) {
-    const uint32_t ht = st + 16384;
+    const uint32_t ht = st + a_bytes;
 #pragma unroll
     for (int k = 0; k < kTK / 16; ++k)
-      umma_f16(tmem, sdesc_sw128(st + k * 4096, 1024, 2048), sdesc_sw128(ht + k * 32, 16, 1024), idesc,
-               (it > 0 || k > 0) ? 1u : 0u);
+      for (int mp = 0; mp < mps; ++mp)
+        umma_f16(tmem + (uint32_t)(mp * N), sdesc_sw128(st + mp * 16384 + k * 4096, 1024, 2048),
+                 sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
   };
   if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue)) {
     if (tid == 0) latch_error(err, kErrTimeout);
@@ -410,8 +418,10 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
     const int m = warp * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     float v[32];
-    for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
-    for (int t = 0; t < b; ++t) part[((size_t)ks * b + t) * d + col0 + m] = v[t];
+    for (int mp = 0; mp < mps; ++mp) {
+      for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + mp * N + cb, v + cb);
+      for (int t = 0; t < b; ++t) part[((size_t)ks * b + t) * d + col0 + mp * kTM + m] = v[t];
+    }
   }
   tc_end(tmem);
 }
@@ -560,7 +570,7 @@ constexpr int kUpStages = 3, kDownStages = 3, kPredStages = 4;
 size_t up_smem(int act, int N, int kps) {
   return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024;
 }
-size_t down_smem(int N) { return (size_t)kDownStages * (16384 + N * 128) + 1024; }
+size_t down_smem(int N, int mps) { return (size_t)kDownStages * (mps * 16384 + N * 128) + 1024; }
 size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
 size_t logits_smem(int N) { return (size_t)kPredStages * (16384 + 2 * N * 128) + 1024; }
 
@@ -595,6 +605,19 @@ static int up_fit(int act, int N, int kps) {
   return c;
 }
 
+// k_tc_down CTAs that fit on an SM at once (measured once per shape).
+static int down_fit(int N, int mps) {
+  static int cache[2][2] = {};
+  int &c = cache[N == 32][mps - 1];
+  if (c == 0) {
+    int nb = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_down, kTT, down_smem(N, mps));
+    if (e != cudaSuccess) cudaGetLastError();
+    c = e == cudaSuccess && nb > 0 ? nb : 1;
+  }
+  return c;
+}
+
 cudaError_t configure_tc_batch() {
   cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)up_smem(SFNN_RELU, 32, 2));
@@ -602,7 +625,7 @@ cudaError_t configure_tc_batch() {
     e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)up_smem(SFNN_REGLU, 32, 2));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32));
+    e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 2));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
   if (e == cudaSuccess)
@@ -611,6 +634,8 @@ cudaError_t configure_tc_batch() {
   for (int act : {SFNN_RELU, SFNN_REGLU})
     for (int N : {16, 32})
       for (int kps : {1, 2}) up_fit(act, N, kps);
+  for (int N : {16, 32})
+    for (int mps : {1, 2}) down_fit(N, mps);
   return e;
 }
 
@@ -661,13 +686,13 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
         h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int mtiles = L.d / kTM;
-  // one wave: three CTAs fit on an SM (3 stages of 20 KB); the output tiles times the
-  // splits of the union fill them without a tail
-  int splits = (3 * h->num_sms) / mtiles;
+  const int mps = L.d % (2 * kTM) == 0 ? h->tc_down_mps : 1;
+  const int mtiles = L.d / (kTM * mps);
+  // one wave: the output tiles times the splits of the union fill the CTAs that fit at once
+  int splits = (down_fit(N, mps) * h->num_sms) / mtiles;
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
-  k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part, L.d, b, N,
-                                                            L.nproj, splits, kDownStages, h->err);
+  k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N, mps), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
+                                                                 L.d, b, N, L.nproj, splits, kDownStages, mps, h->err);
   *splits_out = splits;
   return cudaGetLastError();
 }

@@ -90,8 +90,9 @@ def parse_args(argv=None):
                     help="with --batch > 1: the batched path; auto measures, for 4 < b <= 8, two few-token "
                          "launches against tensor cores before timing (a profiler slows the launches and "
                          "skews that measurement: name the path there)")
-    ap.add_argument("--tc-up", default="",
-                    help="with --batch > 1: the tensor-core up projection's shape, 'ctas_per_sm,chunks_per_step'")
+    ap.add_argument("--tc-shape", default="",
+                    help="with --batch > 1: the tensor-core kernels' shape, "
+                         "'up_ctas_per_sm,up_chunks_per_step,down_tiles_per_cta'")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="CPU budget of the reference arm (warm-up and timed steps together)")
     return ap.parse_args(argv)
@@ -538,8 +539,8 @@ def measure_batch(cfg, b, args, dist, dev):
              "fused": sf.BATCH_FUSED}[args.batch_path]
     for h in handles:
         h.set_batch_path(bpath)
-        if args.tc_up:
-            h.set_batch_tc_up(*[int(v) for v in args.tc_up.split(",")])
+        if args.tc_shape:
+            h.set_batch_tc_shape(*[int(v) for v in args.tc_shape.split(",")])
     if bpath == sf.BATCH_AUTO and 4 < b <= 8:  # AUTO's measured choice: two few-token launches or tensor cores
         for h in handles:
             t = h.tune_batch_paths()

@@ -300,17 +300,19 @@ SFNN_API sfnn_status sfnn_set_fused_quota(sfnn_handle h, int32_t quota);
 SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
 
 /*
- * The tensor-core batch path's up projection shape (a tuning knob; the results do not depend
- * on it beyond the order in which a split tile's partial sums are added): ctas_per_sm = its
- * CTAs per SM (1 or 2, capped by how many fit in shared memory; the union's (128-row tile,
- * K step) pairs are shared out evenly among them), chunks_per_step = 64-wide K chunks of
- * every row staged per step (1 or 2; two make each row's reads 256 contiguous bytes).
- * Default 2 and 2 (one CTA per SM fits for ReGLU layers and for ReLU layers past 16
- * tokens).  -1 keeps a value.
- * SFNN_ERR_INVALID_ARG outside those sets; SFNN_ERR_UNSUPPORTED when the layer has no
- * tensor-core batch path.  Takes effect at the next launch.
+ * The tensor-core batch path's kernel shapes (a tuning knob; the results do not depend on
+ * it beyond the order in which partial sums are added).  Up projection: up_ctas_per_sm =
+ * its CTAs per SM (1 or 2, capped by how many fit in shared memory; the union's (128-row
+ * tile, K step) pairs are shared out evenly among them), up_chunks_per_step = 64-wide K
+ * chunks of every row staged per step (1 or 2; two make each row's reads 256 contiguous
+ * bytes).  Down projection: down_tiles_per_cta = 128-column output tiles per CTA (1 or 2;
+ * two make each W_down row's reads 512 contiguous bytes; needs d a multiple of 256, else
+ * 1 is used).  Defaults 2, 2, 1.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those
+ * sets; SFNN_ERR_UNSUPPORTED when the layer has no tensor-core batch path.  Takes effect at
+ * the next launch.
  */
-SFNN_API sfnn_status sfnn_set_batch_tc_up(sfnn_handle h, int32_t ctas_per_sm, int32_t chunks_per_step);
+SFNN_API sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32_t up_chunks_per_step,
+                                             int32_t down_tiles_per_cta);
 
 /*
  * Measures, on this handle, which path serves AUTO batches of multi_max + 1 .. 2 multi_max
