@@ -589,32 +589,44 @@ size_t tc_up_partial_bytes(int num_sms, int max_batch) {
   return (size_t)2 * (2 * num_sms) * 2 * (size_t)max_batch * kTM * sizeof(float);
 }
 
-// k_tc_up CTAs that fit on an SM at once for this shape (measured once per shape).
+// CTAs of `func` with `dyn` bytes of dynamic shared memory that fit on an SM at once: by
+// shared memory (what the SM holds over each CTA's dynamic + static + reserved bytes), by
+// registers and by tensor memory (kTmemCols of 512 columns each).  Worked out from the
+// device's and the kernel's attributes: the occupancy calculator assumes a shared-memory
+// carveout smaller than the one launches get.
+static int fit_per_sm(const void *func, size_t dyn) {
+  int dev = 0, smem_sm = 0, reserved = 0, regs_sm = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, func) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  int n = (int)((size_t)smem_sm / (dyn + fa.sharedSizeBytes + (size_t)reserved));
+  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * (kTT / 32);  // per-warp granules of 256
+  n = std::min(n, regs_cta > 0 ? regs_sm / regs_cta : n);
+  n = std::min(n, 512 / kTmemCols);
+  return n > 0 ? n : 1;
+}
+
+// k_tc_up CTAs that fit on an SM at once for this shape (worked out once per shape).
 static int up_fit(int act, int N, int kps) {
   static int cache[2][2][2] = {};
   int &c = cache[act == SFNN_REGLU][N == 32][kps - 1];
-  if (c == 0) {
-    int nb = 0;
-    const cudaError_t e =
-        act == SFNN_REGLU
-            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_up<SFNN_REGLU>, kTT, up_smem(act, N, kps))
-            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_up<SFNN_RELU>, kTT, up_smem(act, N, kps));
-    if (e != cudaSuccess) cudaGetLastError();
-    c = e == cudaSuccess && nb > 0 ? nb : 1;
-  }
+  if (c == 0)
+    c = act == SFNN_REGLU ? fit_per_sm((const void *)k_tc_up<SFNN_REGLU>, up_smem(act, N, kps))
+                          : fit_per_sm((const void *)k_tc_up<SFNN_RELU>, up_smem(act, N, kps));
   return c;
 }
 
-// k_tc_down CTAs that fit on an SM at once (measured once per shape).
+// k_tc_down CTAs that fit on an SM at once (worked out once per shape).
 static int down_fit(int N, int mps) {
   static int cache[2][2] = {};
   int &c = cache[N == 32][mps - 1];
-  if (c == 0) {
-    int nb = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_tc_down, kTT, down_smem(N, mps));
-    if (e != cudaSuccess) cudaGetLastError();
-    c = e == cudaSuccess && nb > 0 ? nb : 1;
-  }
+  if (c == 0) c = fit_per_sm((const void *)k_tc_down, down_smem(N, mps));
   return c;
 }
 
@@ -630,7 +642,7 @@ cudaError_t configure_tc_batch() {
     e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)logits_smem(32));
-  // the occupancy of every up-projection shape, outside any stream capture
+  // the CTAs per SM of every up and down shape, outside any stream capture
   for (int act : {SFNN_RELU, SFNN_REGLU})
     for (int N : {16, 32})
       for (int kps : {1, 2}) up_fit(act, N, kps);
