@@ -354,11 +354,12 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
 // columns) over its split of the union.  smem per stage: mps A tiles (64 union rows x 128
 // columns, MN-major, 16 KB each) + the H tile (N tokens x 64 union entries, K-major).  A
 // warp's copy instruction covers 2 / mps union rows of 256 mps contiguous bytes.
+template <int MPS>
 __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows, const __half *__restrict__ H,
                                                  int hstride, const int32_t *__restrict__ ulist,
                                                  const int32_t *__restrict__ ucount, float *__restrict__ part, int d,
-                                                 int b, int N, int nproj, int splits, int stages, int mps,
-                                                 int32_t *err) {
+                                                 int b, int N, int nproj, int splits, int stages, int32_t *err) {
+  constexpr int mps = MPS;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -383,11 +384,12 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   // A: chunk q = tid + 128 i -> union row k = q / (16 mps) of the stage, 16-byte column
   // chunk c = q % (16 mps) of its 256 mps bytes: tile mp = c / 16, and within it MN atom
   // m' = (c % 16) / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
-  const int cpr = 16 * mps;  // 16-byte chunks of a row
+  constexpr int cpr = 16 * mps;  // 16-byte chunks of a row
   auto load = [&](int s, int it) {
     const int kc = c0 + it;
     unsigned char *st = smem + (size_t)s * stage_bytes;
-    for (int i = 0; i < 8 * mps; ++i) {
+#pragma unroll
+    for (int i = 0; i < 8 * mps; ++i) {  // unrolled: the union indices are loaded together
       const int q = tid + kTT * i;
       const int k = q / cpr, c = q % cpr;
       int u = kc * kTK + k;
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
     const uint32_t ht = st + a_bytes;
 #pragma unroll
     for (int k = 0; k < kTK / 16; ++k)
+#pragma unroll
       for (int mp = 0; mp < mps; ++mp)
         umma_f16(tmem + (uint32_t)(mp * N), sdesc_sw128(st + mp * 16384 + k * 4096, 1024, 2048),
                  sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
@@ -418,6 +421,7 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
     const int m = warp * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     float v[32];
+#pragma unroll
     for (int mp = 0; mp < mps; ++mp) {
       for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + mp * N + cb, v + cb);
       for (int t = 0; t < b; ++t) part[((size_t)ks * b + t) * d + col0 + mp * kTM + m] = v[t];
@@ -626,7 +630,8 @@ static int up_fit(int act, int N, int kps) {
 static int down_fit(int N, int mps) {
   static int cache[2][2] = {};
   int &c = cache[N == 32][mps - 1];
-  if (c == 0) c = fit_per_sm((const void *)k_tc_down, down_smem(N, mps));
+  if (c == 0)
+    c = fit_per_sm(mps == 2 ? (const void *)k_tc_down<2> : (const void *)k_tc_down<1>, down_smem(N, mps));
   return c;
 }
 
@@ -637,7 +642,9 @@ cudaError_t configure_tc_batch() {
     e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)up_smem(SFNN_REGLU, 32, 2));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 2));
+    e = cudaFuncSetAttribute(k_tc_down<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 1));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_down<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 2));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
   if (e == cudaSuccess)
@@ -703,8 +710,12 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   // one wave: the output tiles times the splits of the union fill the CTAs that fit at once
   int splits = (down_fit(N, mps) * h->num_sms) / mtiles;
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
-  k_tc_down<<<dim3(mtiles, splits), kTT, down_smem(N, mps), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
-                                                                 L.d, b, N, L.nproj, splits, kDownStages, mps, h->err);
+  if (mps == 2)
+    k_tc_down<2><<<dim3(mtiles, splits), kTT, down_smem(N, 2), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
+                                                                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
+  else
+    k_tc_down<1><<<dim3(mtiles, splits), kTT, down_smem(N, 1), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
+                                                                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
   *splits_out = splits;
   return cudaGetLastError();
 }
