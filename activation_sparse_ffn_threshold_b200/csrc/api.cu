@@ -390,11 +390,13 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   // the tensor-core up projection: 2 K chunks per step (256 contiguous bytes of each row
   // per request round) on as many CTAs per SM as fit, up to 2.  Measured (us per batch,
   // CTAs per SM x chunks: 2x1 / 1x1 / 1x2 / 2x2): 70B-shaped b = 8 184 / 199 / 175 / 188,
-  // b = 32 297 / 326 / 283 / 303 (2x2 fits one CTA per SM there, so it runs two waves);
-  // OPT-30B-shaped b = 8 124 / 137 / 122 / 115 (2x2 fits twice)
+  // b = 32 297 / 326 / 283 / 303 (2x2 launched two CTAs per SM there, one fitting);
+  // OPT-30B-shaped b = 8 124 / 137 / 122 / 115 (2x2 fits twice).  The down projection: two
+  // 128-column tiles per CTA (512 contiguous bytes of each W_down row): 70B-shaped b = 32
+  // 282 -> 272, b = 8 and OPT-30B-shaped b = 8 unchanged (170, 114)
   h->tc_up_ctas_per_sm = 2;
   h->tc_up_kps = 2;
-  h->tc_down_mps = 1;
+  h->tc_down_mps = 2;
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;

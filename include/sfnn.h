@@ -307,7 +307,7 @@ SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
  * chunks of every row staged per step (1 or 2; two make each row's reads 256 contiguous
  * bytes).  Down projection: down_tiles_per_cta = 128-column output tiles per CTA (1 or 2;
  * two make each W_down row's reads 512 contiguous bytes; needs d a multiple of 256, else
- * 1 is used).  Defaults 2, 2, 1.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those
+ * 1 is used).  Defaults 2, 2, 2.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those
  * sets; SFNN_ERR_UNSUPPORTED when the layer has no tensor-core batch path.  Takes effect at
  * the next launch.
  */
