@@ -144,13 +144,10 @@ __device__ __forceinline__ void tc_end(uint32_t tmem) {
 }
 // The K loop: `load(s, it)` copies iteration it's operands into stage s (cp.async, all
 // threads); `issue(stage_smem_addr, it)` issues its MMAs (thread 0), which are committed
-// to the stage's mbarrier.  Each iteration first refills the stage the previous
-// iteration's MMAs read (once they are done) and only then waits for its own stage, so
-// `stages` - 1 to `stages` stages of copies stay in flight.  `base` counts the iterations
-// this CTA ran in earlier calls (they fix the stage and mbarrier phase of each iteration).
-// Returns false if a wait ran out (then `fail` is set; every thread takes the same exit).
-// On return every MMA has completed (or failed) and the accumulators may be read after
-// tc_fence_after.
+// to the stage's mbarrier; the stage is refilled once they are done.  `base` counts the
+// iterations this CTA ran in earlier calls (they fix the stage and mbarrier phase of
+// each iteration).  Returns false if a wait ran out (then `fail` is set).  On return every
+// MMA has completed (or failed) and the accumulators may be read after tc_fence_after.
 template <class Load, class Issue>
 __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_bytes, int stages, int nk,
                                             uint64_t *mbar, int *fail, Load load, Issue issue, int base = 0) {
@@ -160,36 +157,33 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
     cp_async_commit();
   }
   bool ok = true;
-  for (int it = 0; it < nk; ++it) {
+  for (int it = 0; it < nk && ok; ++it) {
     const int j = base + it, s = j % stages;
-    bool bad = false;
-    const int nx = it + stages - 1;  // into the stage iteration it - 1 read, once its MMAs are done
-    if (nx < nk) {
-      if (it >= 1 && !mb_wait(&mbar[(j - 1) % stages], (uint32_t)(((j - 1) / stages) & 1))) bad = true;
-      if (!bad) load((base + nx) % stages, nx);
-    }
-    cp_async_commit();
-    // committed groups: stages + it; iteration it's is the (it + 1)-th oldest
+    // committed groups: stages - 1 + it; iteration it's is the (it + 1)-th oldest
     switch (stages) {
-      case 2: cp_async_wait<1>(); break;
-      case 3: cp_async_wait<2>(); break;
-      default: cp_async_wait<3>(); break;
+      case 2: cp_async_wait<0>(); break;
+      case 3: cp_async_wait<1>(); break;
+      default: cp_async_wait<2>(); break;
     }
     fence_async_smem();
-    if (__syncthreads_or(bad)) {  // the same decision in every thread
-      ok = false;
-      break;
-    }
+    __syncthreads();
     if (tid == 0) {
       tc_fence_after();
       issue(smem_u32(smem + (size_t)s * stage_bytes), it);
       umma_commit(&mbar[s]);
     }
+    const int nx = it + stages - 1;  // refill the stage iteration it - 1 read, once its MMAs are done
+    if (nx < nk) {
+      if (it >= 1 && !mb_wait(&mbar[(j - 1) % stages], (uint32_t)(((j - 1) / stages) & 1))) *fail = 1;
+      load((base + nx) % stages, nx);
+    }
+    cp_async_commit();
+    __syncthreads();
+    ok = *fail == 0;
   }
   cp_async_wait<0>();
   if (ok && nk > 0 && !mb_wait(&mbar[(base + nk - 1) % stages], (uint32_t)(((base + nk - 1) / stages) & 1)))
-    ok = false;
-  if (!ok) *fail = 1;
+    *fail = 1;
   tc_fence_after();
   __syncthreads();
   return *fail == 0;
