@@ -14,6 +14,7 @@
 //             fixed order through shared memory -> part[ks][t][cols].
 //   k_reduce  y = sum over ks of part[ks] in ascending ks (+ residual).
 // Every sum runs in a fixed order, so results are bitwise reproducible.
+#include "async.cuh"
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -137,6 +138,8 @@ __global__ void __launch_bounds__(kThreads)
 template <typename OUT>
 __global__ void k_reduce(const float *__restrict__ part, int splits, int64_t bd, const float *resid, float *Y,
                          OUT *__restrict__ xnext) {
+  pdl_wait();  // the partials (the kernel before) are complete
+  pdl_launch_dependents();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= bd) return;
   float s = 0.f;
@@ -223,10 +226,10 @@ cudaError_t launch_reduce(const sfnn_ctx *h, int b, int splits, const float *res
   const int64_t bd = (int64_t)b * h->L.d;
   const int grid = (int)((bd + 255) / 256);
   if (h->L.dt == SFNN_F16)
-    k_reduce<__half><<<grid, 256, 0, s>>>(h->part, splits, bd, resid, Y, static_cast<__half *>(xnext));
-  else
-    k_reduce<float><<<grid, 256, 0, s>>>(h->part, splits, bd, resid, Y, static_cast<float *>(xnext));
-  return cudaGetLastError();
+    return launch_pdl(k_reduce<__half>, dim3(grid), dim3(256), 0, s, (const float *)h->part, splits, bd, resid, Y,
+                      static_cast<__half *>(xnext));
+  return launch_pdl(k_reduce<float>, dim3(grid), dim3(256), 0, s, (const float *)h->part, splits, bd, resid, Y,
+                    static_cast<float *>(xnext));
 }
 
 cudaError_t launch_round(const float *X, void *out, int dt, int64_t count, cudaStream_t s) {

@@ -15,6 +15,7 @@
 //   k_compact  masks -> ascending index lists (per token, in caller numbering)
 //              and the union of the tokens' sets with, per union row, the bit
 //              set of tokens active on it (warp ballot + block prefix sum).
+#include "async.cuh"
 #include "common.cuh"
 #include "launch.cuh"
 
@@ -222,6 +223,8 @@ __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restr
                                                          int32_t *__restrict__ ucount) {
   __shared__ uint32_t stage[kUnionStage];
   __shared__ int red[32];
+  pdl_wait();  // the masks (the kernel before) are complete
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int w0 = blockIdx.x * 32;
   const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
@@ -395,8 +398,8 @@ cudaError_t launch_compact(const sfnn_ctx *h, int b, bool want_union, int32_t *i
   const Layout &L = h->L;
   cudaError_t e = cudaSuccess;
   if (want_union) {
-    k_union<<<(L.nwords + 31) / 32, kUnionThreads, 0, s>>>(h->mask, L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
-    e = cudaGetLastError();
+    e = launch_pdl(k_union, dim3((L.nwords + 31) / 32), dim3(kUnionThreads), 0, s, (const uint32_t *)h->mask,
+                   L.nwords, L.n, b, h->ulist, h->utok, h->ucount);
   }
   if (e == cudaSuccess && (idx_out || cnt_out)) {
     k_compact<<<b, 1024, 0, s>>>(h->mask, L.nwords, L.n, h->perm, idx_out, cnt_out);

@@ -142,18 +142,20 @@ __device__ __forceinline__ void tc_end(uint32_t tmem) {
   __syncthreads();
   if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, kTmemCols);
 }
-// The K loop: `load(s, it)` copies iteration it's operands into stage s (cp.async, all
-// threads); `issue(stage_smem_addr, it)` issues its MMAs (thread 0), which are committed
+// The K loop: `load(s, it, what)` copies iteration it's operands (`what`: kLoadA the
+// weights, kLoadB the activations, kLoadAll both) into stage s (cp.async, all threads); `issue(stage_smem_addr, it)` issues its MMAs (thread 0), which are committed
 // to the stage's mbarrier; the stage is refilled once they are done.  `base` counts the
 // iterations this CTA ran in earlier calls (they fix the stage and mbarrier phase of
 // each iteration).  Returns false if a wait ran out (then `fail` is set).  On return every
 // MMA has completed (or failed) and the accumulators may be read after tc_fence_after.
+constexpr int kLoadA = 1, kLoadB = 2, kLoadAll = 3;  // `load`'s operands: the weights, the activations
 template <class Load, class Issue>
 __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_bytes, int stages, int nk,
-                                            uint64_t *mbar, int *fail, Load load, Issue issue, int base = 0) {
+                                            uint64_t *mbar, int *fail, Load load, Issue issue, int base = 0,
+                                            int a_pre = 0) {
   const int tid = threadIdx.x;
-  for (int s = 0; s < stages - 1; ++s) {
-    if (s < nk) load((base + s) % stages, s);
+  for (int s = 0; s < stages - 1; ++s) {  // a_pre: iterations whose weights were copied already
+    if (s < nk) load((base + s) % stages, s, s < a_pre ? kLoadB : kLoadAll);
     cp_async_commit();
   }
   bool ok = true;
@@ -175,7 +177,7 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
     const int nx = it + stages - 1;  // refill the stage iteration it - 1 read, once its MMAs are done
     if (nx < nk) {
       if (it >= 1 && !mb_wait(&mbar[(j - 1) % stages], (uint32_t)(((j - 1) / stages) & 1))) *fail = 1;
-      load((base + nx) % stages, nx);
+      load((base + nx) % stages, nx, kLoadAll);
     }
     cp_async_commit();
     __syncthreads();
@@ -214,6 +216,8 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   __shared__ int fail, last_s;
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();  // the union (the kernel before) is complete
+  pdl_launch_dependents();
   const int U = *ucount;
   const int nk = d / (kTK * kps);  // K steps of a tile
   const int64_t T = (int64_t)((U + kTM - 1) / kTM) * nk;
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
       src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
     }
-    auto load = [&](int s, int it) {
+    auto load = [&](int s, int it, int) {
       for (int a = 0; a < kps; ++a) {
         const int kc = (k0 + it) * kps + a;
         unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
@@ -367,7 +371,9 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt = blockIdx.x, ks = blockIdx.y;
-  const int U = *ucount;
+  // The union (two kernels before) is complete when this grid starts: the up projection
+  // lets it start only after its own griddepcontrol.wait.  Its list is read through L2.
+  const int U = __ldcg(ucount);
   const int nkc = (U + kTK - 1) / kTK;
   const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
   const int col0 = mt * kTM * mps;
@@ -375,6 +381,8 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   const uint32_t stage_bytes = a_bytes + (uint32_t)N * 128u;
 
   if (c0 == c1) {  // an empty split still provides its (zero) partial
+    pdl_wait();
+    pdl_launch_dependents();
     for (int q = tid; q < b * kTM * mps; q += kTT)
       part[((size_t)ks * b + q / (kTM * mps)) * d + col0 + q % (kTM * mps)] = 0.f;
     return;
@@ -385,24 +393,28 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
   // chunk c = q % (16 mps) of its 256 mps bytes: tile mp = c / 16, and within it MN atom
   // m' = (c % 16) / 8, chunk cc = c % 8 of its 128-byte row; k = 8 k1 + k0.
   constexpr int cpr = 16 * mps;  // 16-byte chunks of a row
-  auto load = [&](int s, int it) {
+  auto load = [&](int s, int it, int what) {
     const int kc = c0 + it;
     unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
 #pragma unroll
-    for (int i = 0; i < 8 * mps; ++i) {  // unrolled: the union indices are loaded together
-      const int q = tid + kTT * i;
-      const int k = q / cpr, c = q % cpr;
-      int u = kc * kTK + k;
-      u = u < U ? u : U - 1;  // past the union: a repeated row times H's zero padding
-      const int mp = c >> 4, c16 = c & 15;
-      const int k0 = k & 7, k1 = k >> 3, ma = c16 >> 3, cc = c16 & 7;
-      const uint32_t off = (uint32_t)(mp * 16384 + ma * 1024 + k1 * 2048 + k0 * 128 + ((cc ^ k0) << 4));
-      cp16(st, off, rows + ((size_t)ulist[u] * nproj + (nproj - 1)) * d + col0 + c * 8);
+      for (int i = 0; i < 8 * mps; ++i) {  // unrolled: the union indices are loaded together
+        const int q = tid + kTT * i;
+        const int k = q / cpr, c = q % cpr;
+        int u = kc * kTK + k;
+        u = u < U ? u : U - 1;  // past the union: a repeated row times H's zero padding
+        const int mp = c >> 4, c16 = c & 15;
+        const int k0 = k & 7, k1 = k >> 3, ma = c16 >> 3, cc = c16 & 7;
+        const uint32_t off = (uint32_t)(mp * 16384 + ma * 1024 + k1 * 2048 + k0 * 128 + ((cc ^ k0) << 4));
+        cp16(st, off, rows + ((size_t)__ldcg(ulist + u) * nproj + (nproj - 1)) * d + col0 + c * 8);
+      }
     }
-    unsigned char *ht = st + a_bytes;
-    for (int q = tid; q < N * 8; q += kTT) {
-      const int t = q >> 3, c = q & 7;
-      cp16(ht, kmajor_off(t, c), H + (size_t)t * hstride + (size_t)kc * kTK + c * 8);
+    if (what & kLoadB) {
+      unsigned char *ht = st + a_bytes;
+      for (int q = tid; q < N * 8; q += kTT) {
+        const int t = q >> 3, c = q & 7;
+        cp16(ht, kmajor_off(t, c), H + (size_t)t * hstride + (size_t)kc * kTK + c * 8);
+      }
     }
   };
   const uint32_t idesc = idesc_f16(kTM, N, 1, 0);
@@ -415,7 +427,12 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
         umma_f16(tmem + (uint32_t)(mp * N), sdesc_sw128(st + mp * 16384 + k * 4096, 1024, 2048),
                  sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
   };
-  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue)) {
+  // the first stages' W_down rows while the up projection finishes; H after it has
+  const int a_pre = min(stages - 1, c1 - c0);
+  for (int i = 0; i < a_pre; ++i) load(i, i, kLoadA);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue, 0, a_pre)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int m = warp * 32 + lane;
@@ -451,6 +468,8 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
   const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
   const uint32_t stage_bytes = 16384u + (uint32_t)N * 128u;
   if (c0 == c1) {
+    pdl_wait();
+    pdl_launch_dependents();
     for (int q = tid; q < b * kTM; q += kTT) {
       const int t = q / kTM, j = j0 + q % kTM;
       if (j < r) hp[((size_t)ks * b + t) * r + j] = 0.f;
@@ -459,20 +478,24 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
   }
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const int c8 = tid & 7;
-  auto load = [&](int s, int it) {
+  auto load = [&](int s, int it, int what) {
     const int kc = c0 + it;
     unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int row = (tid >> 3) + 16 * i;
-      const int j = j0 + row < r ? j0 + row : r - 1;
-      cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        const int j = j0 + row < r ? j0 + row : r - 1;
+        cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
+      }
     }
-    unsigned char *xt = st + 16384;
-    for (int q = tid; q < N * 8; q += kTT) {
-      const int t = q >> 3, c = q & 7;
-      const int tt = t < b ? t : b - 1;
-      cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+    if (what & kLoadB) {
+      unsigned char *xt = st + 16384;
+      for (int q = tid; q < N * 8; q += kTT) {
+        const int t = q >> 3, c = q & 7;
+        const int tt = t < b ? t : b - 1;
+        cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
+      }
     }
   };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
@@ -482,7 +505,12 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
       umma_f16(tmem, sdesc_sw128(st + k * 32, 16, 1024), sdesc_sw128(st + 16384 + k * 32, 16, 1024), idesc,
                (it > 0 || k > 0) ? 1u : 0u);
   };
-  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue)) {
+  // the first stages' A^T rows (weights) before the kernel before completes; x after it
+  const int a_pre = min(stages - 1, c1 - c0);
+  for (int i = 0; i < a_pre; ++i) load(i, i, kLoadA);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!tc_mainloop(smem, stage_bytes, stages, c1 - c0, mbar, &fail, load, issue, 0, a_pre)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int j = j0 + warp * 32 + lane;
@@ -497,6 +525,8 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
 
 __global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N, int r, __half *__restrict__ hhi,
                           __half *__restrict__ hlo) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;  // t * r + j over N tokens
   if (i >= N * r) return;
   const int t = i / r;
@@ -526,19 +556,23 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
   const uint32_t stage_bytes = 16384u + 2u * (uint32_t)N * 128u;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const int c8 = tid & 7;
-  auto load = [&](int s, int kc) {
+  auto load = [&](int s, int kc, int what) {
     unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int row = (tid >> 3) + 16 * i;
-      const int nn = i0 + row < n ? i0 + row : n - 1;
-      cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        const int nn = i0 + row < n ? i0 + row : n - 1;
+        cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
+      }
     }
-    unsigned char *ht = st + 16384;
-    for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
-      const int half = q / (N * 8), qq = q - half * N * 8;
-      const int t = qq >> 3, c = qq & 7;
-      cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
+    if (what & kLoadB) {
+      unsigned char *ht = st + 16384;
+      for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
+        const int half = q / (N * 8), qq = q - half * N * 8;
+        const int t = qq >> 3, c = qq & 7;
+        cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
+      }
     }
   };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
@@ -551,7 +585,12 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
       umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
     }
   };
-  if (!tc_mainloop(smem, stage_bytes, stages, r / kTK, mbar, &fail, load, issue)) {
+  // the first stages' B^T rows (weights) while the hidden layer is summed; h after it
+  const int a_pre = min(stages - 1, r / kTK);
+  for (int i = 0; i < a_pre; ++i) load(i, i, kLoadA);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!tc_mainloop(smem, stage_bytes, stages, r / kTK, mbar, &fail, load, issue, 0, a_pre)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int i = i0 + warp * 32 + lane;
@@ -670,20 +709,19 @@ cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStrea
   splits = std::min(splits, L.d / kTK);
   splits = std::min<int>(splits, (int)(cap / ((size_t)b * L.r)));
   splits = splits < 1 ? 1 : splits;
-  k_tc_hidden<<<dim3(rtiles, splits), kTT, hidden_smem(N), s>>>(
-      static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r, b, N, splits,
-      kPredStages, h->err);
-  cudaError_t e = cudaGetLastError();
+  // every kernel of the chain starts early (programmatic serialization) and copies its
+  // first weight stages before it waits for the one before
+  cudaError_t e = launch_pdl(k_tc_hidden, dim3(rtiles, splits), dim3(kTT), hidden_smem(N), s,
+                             static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r,
+                             b, N, splits, kPredStages, h->err);
   if (e != cudaSuccess) return e;
   __half *hhi = h->hpair, *hlo = h->hpair + (size_t)32 * L.r;
-  k_tc_hsum<<<(N * L.r + 255) / 256, 256, 0, s>>>(h->part, splits, b, N, L.r, hhi, hlo);
-  e = cudaGetLastError();
+  e = launch_pdl(k_tc_hsum, dim3((N * L.r + 255) / 256), dim3(256), 0, s, (const float *)h->part, splits, b, N, L.r,
+                 hhi, hlo);
   if (e != cudaSuccess) return e;
-  k_tc_logits<<<(L.n + kTM - 1) / kTM, kTT, logits_smem(N), s>>>(static_cast<const __half *>(h->Bt),
-                                                                  static_cast<const __half *>(h->cvec), hhi, hlo,
-                                                                  h->mask, L.n, L.r, L.nwords, b, N, kPredStages,
-                                                                  h->err);
-  return cudaGetLastError();
+  return launch_pdl(k_tc_logits, dim3((L.n + kTM - 1) / kTM), dim3(kTT), logits_smem(N), s,
+                    static_cast<const __half *>(h->Bt), static_cast<const __half *>(h->cvec), (const __half *)hhi,
+                    (const __half *)hlo, h->mask, L.n, L.r, L.nwords, b, N, kPredStages, h->err);
 }
 
 // Up / gate of the union rows for all b tokens -> h->hact; then the down projection into
@@ -695,29 +733,21 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const __half *rows = static_cast<const __half *>(h->rows);
   const int kps = L.d % (2 * kTK) == 0 ? h->tc_up_kps : 1;
   const int up_grid = std::min(h->tc_up_ctas_per_sm, up_fit(L.act, N, kps)) * h->num_sms;
-  if (L.act == SFNN_REGLU)
-    k_tc_up<SFNN_REGLU><<<up_grid, kTT, up_smem(L.act, N, kps), s>>>(
-        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
-  else
-    k_tc_up<SFNN_RELU><<<up_grid, kTT, up_smem(L.act, N, kps), s>>>(
-        rows, static_cast<const __half *>(h->bias), static_cast<const __half *>(X), h->ulist, h->utok, h->ucount,
-        h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU> : k_tc_up<SFNN_RELU>, dim3(up_grid),
+                             dim3(kTT), up_smem(L.act, N, kps), s, rows, static_cast<const __half *>(h->bias),
+                             static_cast<const __half *>(X), (const int32_t *)h->ulist, (const uint32_t *)h->utok,
+                             (const int32_t *)h->ucount, h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart,
+                             h->tcnt, h->err);
   if (e != cudaSuccess) return e;
   const int mps = L.d % (2 * kTM) == 0 ? h->tc_down_mps : 1;
   const int mtiles = L.d / (kTM * mps);
   // one wave: the output tiles times the splits of the union fill the CTAs that fit at once
   int splits = (down_fit(N, mps) * h->num_sms) / mtiles;
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
-  if (mps == 2)
-    k_tc_down<2><<<dim3(mtiles, splits), kTT, down_smem(N, 2), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
-                                                                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
-  else
-    k_tc_down<1><<<dim3(mtiles, splits), kTT, down_smem(N, 1), s>>>(rows, h->hact, hs, h->ulist, h->ucount, h->part,
-                                                                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
   *splits_out = splits;
-  return cudaGetLastError();
+  return launch_pdl(mps == 2 ? k_tc_down<2> : k_tc_down<1>, dim3(mtiles, splits), dim3(kTT), down_smem(N, mps), s,
+                    rows, (const __half *)h->hact, hs, (const int32_t *)h->ulist, (const int32_t *)h->ucount, h->part,
+                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
 }
 
 }  // namespace sfnn
