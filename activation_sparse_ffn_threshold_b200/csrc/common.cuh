@@ -22,23 +22,6 @@ struct Layout {
   int rows_q;  // rows stored as 8- or 4-bit codes with per-row fp32 scales (0: in dt)
 };
 
-// Launch with programmatic stream serialization: the kernel may start while the one before
-// it in the stream finishes (it reads nothing that kernel writes before griddepcontrol.wait).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
-
 }  // namespace sfnn
 
 

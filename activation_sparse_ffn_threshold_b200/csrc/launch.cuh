@@ -9,6 +9,23 @@ namespace sfnn {
 
 constexpr int kMaxNeurons = 1 << 20;  // n at most
 
+// Launch with programmatic stream serialization: the kernel may start while the one before
+// it in the stream finishes (it reads nothing that kernel writes before griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t configure_predict();  // one-time kernel attributes (shared-memory limits)
 cudaError_t configure_ffn();
 cudaError_t launch_layout(sfnn_ctx *h, const sfnn_layer_desc *desc, cudaStream_t s);
