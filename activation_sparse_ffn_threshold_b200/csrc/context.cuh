@@ -30,8 +30,8 @@ struct sfnn_ctx {
   __half *hact;      // [32][n rounded up to 128] fp16 activations (tensor-core batch path) or null
   __half *hpair;     // [2][32][r] the batch's hidden layer as fp16 hi and lo parts (same path)
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
-  float *upart;      // tensor-core logits and up projection: fp32 partials of tiles split between CTAs
-  int32_t *tcnt;     // [n / 128 rounded up] their per-tile arrival counters (zero between launches)
+  float *upart;      // tensor-core up projection: fp32 partials of tiles split between CTAs
+  int32_t *tcnt;     // [n / 128 rounded up] its per-tile arrival counters (zero between launches)
   int tc_up_ctas_per_sm;  // its grid: CTAs per SM (1 or 2; at most as many as fit)
   int tc_up_kps;          // and the 64-wide K chunks of every row it stages per step (1 or 2)
   int tc_down_mps;        // the down projection's 128-column output tiles per CTA (1 or 2)

@@ -451,9 +451,9 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
 // k_tc_hidden: partial hidden layer hp[ks][t][j] = A^T[j] . x_t over the ks-th split of d
 // (A^T rows contiguous, 128 per CTA).  k_tc_hsum: h = relu(sum over ks in order), split
 // into fp16 hi + lo (h - hi), the B operand pair of the logits.  k_tc_logits: z[i][t] =
-// B^T[i] . (hi_t + lo_t) + c_i for tiles of 128 neurons shared out stream-K (two MMAs per
-// step into one fp32 accumulator, so h keeps about 22 bits), active iff z > 0 -> one mask
-// word per warp and token by ballot (token-major masks, as k_compact reads them).
+// B^T[i] . (hi_t + lo_t) + c_i for 128 neurons per CTA (two MMAs per step into one fp32
+// accumulator, so h keeps about 22 bits), active iff z > 0 -> one mask word per warp and
+// token by ballot (token-major masks, as k_compact reads them).
 __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At, const __half *__restrict__ X,
                                                    float *__restrict__ hp, int d, int r, int b, int N, int splits,
                                                    int stages, int32_t *err) {
@@ -545,130 +545,65 @@ __global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N
 __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt, const __half *__restrict__ cvec,
                                                    const __half *__restrict__ hhi, const __half *__restrict__ hlo,
                                                    uint32_t *__restrict__ mask, int n, int r, int nwords, int b, int N,
-                                                   int stages, float *__restrict__ lpart, int32_t *__restrict__ tcnt,
-                                                   int32_t *err) {
+                                                   int stages, int32_t *err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
-  __shared__ int fail, last_s;
+  __shared__ int fail;
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // stream-K over (128-neuron tile, K chunk) steps, as the up projection: CTA g runs steps
-  // [g T / G, (g + 1) T / G); a tile split between CTAs is finished by its last segment
-  const int nk = r / kTK;
-  const int64_t T = (int64_t)((n + kTM - 1) / kTM) * nk;
-  const int64_t G = T < (int64_t)gridDim.x ? T : (int64_t)gridDim.x;
-  const int64_t g = blockIdx.x;
-  if (g >= G) {
-    pdl_wait();
-    pdl_launch_dependents();
-    return;
-  }
-  int64_t i0 = g * T / G;
-  const int64_t i1 = (g + 1) * T / G;
-  auto cta_of = [&](int64_t i) { return ((i + 1) * G + T - 1) / T - 1; };
-  const int first_tile = (int)(i0 / nk);
+  const int i0 = blockIdx.x * kTM;
   const uint32_t stage_bytes = 16384u + 2u * (uint32_t)N * 128u;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
-  const int c8 = tid & 7, row = warp * 32 + lane;
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  const int c8 = tid & 7;
+  auto load = [&](int s, int kc, int what) {
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        const int nn = i0 + row < n ? i0 + row : n - 1;
+        cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
+      }
+    }
+    if (what & kLoadB) {
+      unsigned char *ht = st + 16384;
+      for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
+        const int half = q / (N * 8), qq = q - half * N * 8;
+        const int t = qq >> 3, c = qq & 7;
+        cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
+      }
+    }
+  };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
-  bool ok = true;
-  int base = 0;
-
-  // z = acc + c_i > 0 for this thread's neuron of tile m -> one mask word per warp and token
-  auto epilogue = [&](int m, const float *v) {
-    const int i = m * kTM + row;
+  auto issue = [&](uint32_t st, int it) {
+    const uint32_t ht = st + 16384;
+#pragma unroll
+    for (int k = 0; k < kTK / 16; ++k) {
+      const uint64_t ad = sdesc_sw128(st + k * 32, 16, 1024);
+      umma_f16(tmem, ad, sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
+      umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
+    }
+  };
+  // the first stages' B^T rows (weights) while the hidden layer is summed; h after it
+  const int a_pre = min(stages - 1, r / kTK);
+  for (int i = 0; i < a_pre; ++i) load(i, i, kLoadA);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!tc_mainloop(smem, stage_bytes, stages, r / kTK, mbar, &fail, load, issue, 0, a_pre)) {
+    if (tid == 0) latch_error(err, kErrTimeout);
+  } else {
+    const int i = i0 + warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float v[32];
+    for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
     const float cv = i < n ? __half2float(cvec[i]) : 0.f;
-    const int word = (m * kTM + warp * 32) >> 5;
+    const int word = (i0 + warp * 32) >> 5;
     for (int t = 0; t < b; ++t) {
       const bool on = i < n && v[t] + cv > 0.f;  // NaN -> inactive
       const uint32_t bits = __ballot_sync(0xffffffffu, on);
       if (lane == 0 && word < nwords) mask[(size_t)t * nwords + word] = bits;
     }
-  };
-
-  bool waited = false;
-  while (i0 < i1) {
-    const int m = (int)(i0 / nk);
-    const int k0 = (int)(i0 - (int64_t)m * nk);
-    const int k1 = (int)(i1 - (int64_t)m * nk < nk ? i1 - (int64_t)m * nk : nk);
-    const int n0 = m * kTM;
-    auto load = [&](int s, int it, int what) {
-      const int kc = k0 + it;
-      unsigned char *st = smem + (size_t)s * stage_bytes;
-      if (what & kLoadA) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = (tid >> 3) + 16 * i;
-          const int nn = n0 + rr < n ? n0 + rr : n - 1;
-          cp16(st, kmajor_off(rr, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
-        }
-      }
-      if (what & kLoadB) {
-        unsigned char *ht = st + 16384;
-        for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
-          const int half = q / (N * 8), qq = q - half * N * 8;
-          const int t = qq >> 3, c = qq & 7;
-          cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
-        }
-      }
-    };
-    auto issue = [&](uint32_t st, int it) {
-      const uint32_t ht = st + 16384;
-#pragma unroll
-      for (int k = 0; k < kTK / 16; ++k) {
-        const uint64_t ad = sdesc_sw128(st + k * 32, 16, 1024);
-        umma_f16(tmem, ad, sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
-        umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
-      }
-    };
-    int a_pre = 0;
-    if (!waited) {  // the first segment's first B^T stages (weights) while h is summed; h after it
-      a_pre = min(stages - 1, k1 - k0);
-      for (int q = 0; q < a_pre; ++q) load(q, q, kLoadA);
-      pdl_wait();
-      pdl_launch_dependents();
-      waited = true;
-    }
-    if (ok && !tc_mainloop(smem, stage_bytes, stages, k1 - k0, mbar, &fail, load, issue, base, a_pre)) {
-      ok = false;
-      if (tid == 0) latch_error(err, kErrTimeout);
-    }
-    base += k1 - k0;
-    float v[32];
-    if (ok) {
-      for (int cb = 0; cb < N; cb += 16) tmem_ld16(lane_addr + cb, v + cb);
-    } else {  // after a timeout the tile is still counted (the error is latched)
-      for (int t = 0; t < 32; ++t) v[t] = 0.f;
-    }
-    tc_fence_before();
-    __syncthreads();  // every TMEM read is done before the next segment's MMAs
-    if (k0 == 0 && k1 == nk) {
-      epilogue(m, v);
-    } else {
-      const int slot = 2 * (int)g + (m == first_tile ? 0 : 1);
-      for (int t = 0; t < b; ++t) lpart[((size_t)slot * b + t) * kTM + row] = v[t];
-      __threadfence();
-      __syncthreads();
-      const int64_t ga = cta_of((int64_t)m * nk), gb = cta_of((int64_t)m * nk + nk - 1);
-      if (tid == 0) {
-        const int prev = atomicAdd(&tcnt[m], 1);
-        last_s = prev == (int)(gb - ga);
-        if (last_s) tcnt[m] = 0;  // every segment of the tile has arrived: ready for the next launch
-      }
-      __syncthreads();
-      if (last_s) {
-        __threadfence();
-        for (int t = 0; t < b; ++t) v[t] = 0.f;
-        for (int64_t q = ga; q <= gb; ++q) {  // CTA order
-          const int qs = 2 * (int)q + ((int)((q * T / G) / nk) == m ? 0 : 1);
-          for (int t = 0; t < b; ++t) v[t] += __ldcg(&lpart[((size_t)qs * b + t) * kTM + row]);
-        }
-        epilogue(m, v);
-      }
-    }
-    i0 = (int64_t)(m + 1) * nk;
   }
   tc_end(tmem);
 }
@@ -739,15 +674,6 @@ static int down_fit(int N, int mps) {
   return c;
 }
 
-// k_tc_logits CTAs that fit on an SM at once (at most 2: its partials use the up
-// projection's two slots per CTA of a two-CTA-per-SM grid).
-static int logits_fit(int N) {
-  static int cache[2] = {};
-  int &c = cache[N == 32];
-  if (c == 0) c = std::min(2, fit_per_sm((const void *)k_tc_logits, logits_smem(N)));
-  return c;
-}
-
 cudaError_t configure_tc_batch() {
   cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)up_smem(SFNN_RELU, 32, 2));
@@ -766,10 +692,8 @@ cudaError_t configure_tc_batch() {
   for (int act : {SFNN_RELU, SFNN_REGLU})
     for (int N : {16, 32})
       for (int kps : {1, 2}) up_fit(act, N, kps);
-  for (int N : {16, 32}) {
+  for (int N : {16, 32})
     for (int mps : {1, 2}) down_fit(N, mps);
-    logits_fit(N);
-  }
   return e;
 }
 
@@ -795,11 +719,9 @@ cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStrea
   e = launch_pdl(k_tc_hsum, dim3((N * L.r + 255) / 256), dim3(256), 0, s, (const float *)h->part, splits, b, N, L.r,
                  hhi, hlo);
   if (e != cudaSuccess) return e;
-  // the logits' stream-K partials and tile counters are the up projection's (the two never
-  // run at the same time: the up projection waits for the union, which waits for them)
-  return launch_pdl(k_tc_logits, dim3(logits_fit(N) * h->num_sms), dim3(kTT), logits_smem(N), s,
+  return launch_pdl(k_tc_logits, dim3((L.n + kTM - 1) / kTM), dim3(kTT), logits_smem(N), s,
                     static_cast<const __half *>(h->Bt), static_cast<const __half *>(h->cvec), (const __half *)hhi,
-                    (const __half *)hlo, h->mask, L.n, L.r, L.nwords, b, N, kPredStages, h->upart, h->tcnt, h->err);
+                    (const __half *)hlo, h->mask, L.n, L.r, L.nwords, b, N, kPredStages, h->err);
 }
 
 // Up / gate of the union rows for all b tokens -> h->hact; then the down projection into
