@@ -88,7 +88,7 @@ def load_library():
         "sfnn_set_fused_quota": ([P, I], S),
         "sfnn_set_batch_quota": ([P, I], S),
         "sfnn_set_batch_depths": ([P, I, I, I, I], S),
-        "sfnn_set_batch_tc_shape": ([P, I, I, I, I], S),
+        "sfnn_set_batch_tc_shape": ([P, I, I, I], S),
         "sfnn_tune_batch_paths": ([P, P, P], S),
         "sfnn_set_fused_depths": ([P, I, I, I, I], S),
         "sfnn_debug_stall_next_barrier": ([P, P], S),
@@ -276,14 +276,12 @@ class SparseFFN:
                "sfnn_set_batch_depths")
 
     def set_batch_tc_shape(self, up_ctas_per_sm: int = -1, up_chunks_per_step: int = -1,
-                           down_tiles_per_cta: int = -1, pred_chunks_per_step: int = -1):
+                           down_tiles_per_cta: int = -1):
         """The tensor-core path's kernel shapes: the up projection's CTAs per SM (1 or 2) and
         64-wide K chunks of every row staged per step (1 or 2), the down projection's
-        128-column output tiles per CTA (1 or 2), the predictor GEMMs' K chunks per step
-        (1 or 2); -1 keeps a value."""
+        128-column output tiles per CTA (1 or 2); -1 keeps a value."""
         _check(self._lib.sfnn_set_batch_tc_shape(self._h, int(up_ctas_per_sm), int(up_chunks_per_step),
-                                                 int(down_tiles_per_cta), int(pred_chunks_per_step)),
-               "sfnn_set_batch_tc_shape")
+                                                 int(down_tiles_per_cta)), "sfnn_set_batch_tc_shape")
 
     def tune_batch_paths(self, stream=None):
         """Measure which path serves AUTO batches just above the few-token kernel's size

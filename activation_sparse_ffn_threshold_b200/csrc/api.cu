@@ -397,7 +397,6 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   h->tc_up_ctas_per_sm = 2;
   h->tc_up_kps = 2;
   h->tc_down_mps = 2;
-  h->tc_pred_kps = 1;
   h->quota = 0;
   if (desc->hotness) {
     double mean = 0.0;
@@ -695,9 +694,8 @@ sfnn_status sfnn_set_batch_depths(sfnn_handle h, int32_t bstages, int32_t c2pre,
 }
 
 sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32_t up_chunks_per_step,
-                                    int32_t down_tiles_per_cta, int32_t pred_chunks_per_step) {
+                                    int32_t down_tiles_per_cta) {
   if (!h) return SFNN_ERR_INVALID_ARG;
-  if (pred_chunks_per_step < -1 || pred_chunks_per_step == 0 || pred_chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
   if (up_ctas_per_sm < -1 || up_ctas_per_sm == 0 || up_ctas_per_sm > 2) return SFNN_ERR_INVALID_ARG;
   if (up_chunks_per_step < -1 || up_chunks_per_step == 0 || up_chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
   if (down_tiles_per_cta < -1 || down_tiles_per_cta == 0 || down_tiles_per_cta > 2) return SFNN_ERR_INVALID_ARG;
@@ -705,7 +703,6 @@ sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32
   if (up_ctas_per_sm != -1) h->tc_up_ctas_per_sm = up_ctas_per_sm;
   if (up_chunks_per_step != -1) h->tc_up_kps = up_chunks_per_step;
   if (down_tiles_per_cta != -1) h->tc_down_mps = down_tiles_per_cta;
-  if (pred_chunks_per_step != -1) h->tc_pred_kps = pred_chunks_per_step;
   return SFNN_OK;
 }
 

@@ -35,7 +35,6 @@ struct sfnn_ctx {
   int tc_up_ctas_per_sm;  // its grid: CTAs per SM (1 or 2; at most as many as fit)
   int tc_up_kps;          // and the 64-wide K chunks of every row it stages per step (1 or 2)
   int tc_down_mps;        // the down projection's 128-column output tiles per CTA (1 or 2)
-  int tc_pred_kps;        // the predictor GEMMs' 64-wide K chunks of every row per step (1 or 2)
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error
   uint64_t *bar;     // grid barrier arrival counter of the fused kernel

@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kTT) k_tc_down(const __half *__restrict__ rows
 // token by ballot (token-major masks, as k_compact reads them).
 __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At, const __half *__restrict__ X,
                                                    float *__restrict__ hp, int d, int r, int b, int N, int splits,
-                                                   int stages, int kps, int32_t *err) {
+                                                   int stages, int32_t *err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -464,10 +464,9 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j0 = blockIdx.x * kTM, ks = blockIdx.y;
-  const int nkc = d / (kTK * kps);  // K steps of kps 64-wide chunks
+  const int nkc = d / kTK;
   const int c0 = (int)(((int64_t)ks * nkc) / splits), c1 = (int)(((int64_t)(ks + 1) * nkc) / splits);
-  const uint32_t chunk_bytes = 16384u + (uint32_t)N * 128u;  // a multiple of 1024
-  const uint32_t stage_bytes = (uint32_t)kps * chunk_bytes;
+  const uint32_t stage_bytes = 16384u + (uint32_t)N * 128u;
   if (c0 == c1) {
     pdl_wait();
     pdl_launch_dependents();
@@ -480,36 +479,31 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const int c8 = tid & 7;
   auto load = [&](int s, int it, int what) {
-    for (int a = 0; a < kps; ++a) {
-      const int kc = (c0 + it) * kps + a;
-      unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
-      if (what & kLoadA) {
+    const int kc = c0 + it;
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = (tid >> 3) + 16 * i;
-          const int j = j0 + row < r ? j0 + row : r - 1;
-          cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        const int j = j0 + row < r ? j0 + row : r - 1;
+        cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
       }
-      if (what & kLoadB) {
-        unsigned char *xt = st + 16384;
-        for (int q = tid; q < N * 8; q += kTT) {
-          const int t = q >> 3, c = q & 7;
-          const int tt = t < b ? t : b - 1;
-          cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
-        }
+    }
+    if (what & kLoadB) {
+      unsigned char *xt = st + 16384;
+      for (int q = tid; q < N * 8; q += kTT) {
+        const int t = q >> 3, c = q & 7;
+        const int tt = t < b ? t : b - 1;
+        cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
       }
     }
   };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
   auto issue = [&](uint32_t st, int it) {
-    for (int a = 0; a < kps; ++a) {
-      const uint32_t at = st + (uint32_t)a * chunk_bytes;
 #pragma unroll
-      for (int k = 0; k < kTK / 16; ++k)
-        umma_f16(tmem, sdesc_sw128(at + k * 32, 16, 1024), sdesc_sw128(at + 16384 + k * 32, 16, 1024), idesc,
-                 (it > 0 || a > 0 || k > 0) ? 1u : 0u);
-    }
+    for (int k = 0; k < kTK / 16; ++k)
+      umma_f16(tmem, sdesc_sw128(st + k * 32, 16, 1024), sdesc_sw128(st + 16384 + k * 32, 16, 1024), idesc,
+               (it > 0 || k > 0) ? 1u : 0u);
   };
   // the first stages' A^T rows (weights) before the kernel before completes; x after it
   const int a_pre = min(stages - 1, c1 - c0);
@@ -551,7 +545,7 @@ __global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N
 __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt, const __half *__restrict__ cvec,
                                                    const __half *__restrict__ hhi, const __half *__restrict__ hlo,
                                                    uint32_t *__restrict__ mask, int n, int r, int nwords, int b, int N,
-                                                   int stages, int kps, int32_t *err) {
+                                                   int stages, int32_t *err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -559,52 +553,44 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
   unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i0 = blockIdx.x * kTM;
-  const uint32_t chunk_bytes = 16384u + 2u * (uint32_t)N * 128u;  // a multiple of 1024
-  const uint32_t stage_bytes = (uint32_t)kps * chunk_bytes;
+  const uint32_t stage_bytes = 16384u + 2u * (uint32_t)N * 128u;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const int c8 = tid & 7;
-  const int nk = r / (kTK * kps);  // K steps of kps 64-wide chunks
-  auto load = [&](int s, int it, int what) {
-    for (int a = 0; a < kps; ++a) {
-      const int kc = it * kps + a;
-      unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
-      if (what & kLoadA) {
+  auto load = [&](int s, int kc, int what) {
+    unsigned char *st = smem + (size_t)s * stage_bytes;
+    if (what & kLoadA) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = (tid >> 3) + 16 * i;
-          const int nn = i0 + row < n ? i0 + row : n - 1;
-          cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int row = (tid >> 3) + 16 * i;
+        const int nn = i0 + row < n ? i0 + row : n - 1;
+        cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
       }
-      if (what & kLoadB) {
-        unsigned char *ht = st + 16384;
-        for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
-          const int half = q / (N * 8), qq = q - half * N * 8;
-          const int t = qq >> 3, c = qq & 7;
-          cp16(ht + half * N * 128, kmajor_off(t, c),
-               (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
-        }
+    }
+    if (what & kLoadB) {
+      unsigned char *ht = st + 16384;
+      for (int q = tid; q < 2 * N * 8; q += kTT) {  // hi rows, then lo rows
+        const int half = q / (N * 8), qq = q - half * N * 8;
+        const int t = qq >> 3, c = qq & 7;
+        cp16(ht + half * N * 128, kmajor_off(t, c), (half ? hlo : hhi) + (size_t)t * r + (size_t)kc * kTK + c * 8);
       }
     }
   };
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
   auto issue = [&](uint32_t st, int it) {
-    for (int a = 0; a < kps; ++a) {
-      const uint32_t at = st + (uint32_t)a * chunk_bytes, ht = at + 16384;
+    const uint32_t ht = st + 16384;
 #pragma unroll
-      for (int k = 0; k < kTK / 16; ++k) {
-        const uint64_t ad = sdesc_sw128(at + k * 32, 16, 1024);
-        umma_f16(tmem, ad, sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || a > 0 || k > 0) ? 1u : 0u);
-        umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
-      }
+    for (int k = 0; k < kTK / 16; ++k) {
+      const uint64_t ad = sdesc_sw128(st + k * 32, 16, 1024);
+      umma_f16(tmem, ad, sdesc_sw128(ht + k * 32, 16, 1024), idesc, (it > 0 || k > 0) ? 1u : 0u);
+      umma_f16(tmem, ad, sdesc_sw128(ht + N * 128 + k * 32, 16, 1024), idesc, 1u);
     }
   };
   // the first stages' B^T rows (weights) while the hidden layer is summed; h after it
-  const int a_pre = min(stages - 1, nk);
+  const int a_pre = min(stages - 1, r / kTK);
   for (int i = 0; i < a_pre; ++i) load(i, i, kLoadA);
   pdl_wait();
   pdl_launch_dependents();
-  if (!tc_mainloop(smem, stage_bytes, stages, nk, mbar, &fail, load, issue, 0, a_pre)) {
+  if (!tc_mainloop(smem, stage_bytes, stages, r / kTK, mbar, &fail, load, issue, 0, a_pre)) {
     if (tid == 0) latch_error(err, kErrTimeout);
   } else {
     const int i = i0 + warp * 32 + lane;
@@ -628,12 +614,8 @@ size_t up_smem(int act, int N, int kps) {
   return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024;
 }
 size_t down_smem(int N, int mps) { return (size_t)kDownStages * (mps * 16384 + N * 128) + 1024; }
-// the predictor's stages: 4 of one K chunk, or with two chunks per step 3 (hidden layer:
-// one CTA per SM) or 2 (logits: two CTAs per SM, the same shared memory as 4 x 1)
-int hidden_stages(int kps) { return kps == 2 ? 3 : kPredStages; }
-int logits_stages(int kps) { return kps == 2 ? 2 : kPredStages; }
-size_t hidden_smem(int N, int kps) { return (size_t)hidden_stages(kps) * kps * (16384 + N * 128) + 1024; }
-size_t logits_smem(int N, int kps) { return (size_t)logits_stages(kps) * kps * (16384 + 2 * N * 128) + 1024; }
+size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
+size_t logits_smem(int N) { return (size_t)kPredStages * (16384 + 2 * N * 128) + 1024; }
 
 }  // namespace
 
@@ -703,11 +685,9 @@ cudaError_t configure_tc_batch() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_down<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 2));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max(hidden_smem(32, 1), hidden_smem(32, 2)));
+    e = cudaFuncSetAttribute(k_tc_hidden, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hidden_smem(32));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_logits, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max(logits_smem(32, 1), logits_smem(32, 2)));
+    e = cudaFuncSetAttribute(k_tc_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)logits_smem(32));
   // the CTAs per SM of every up and down shape, outside any stream capture
   for (int act : {SFNN_RELU, SFNN_REGLU})
     for (int N : {16, 32})
@@ -725,25 +705,23 @@ cudaError_t launch_tc_predict(const sfnn_ctx *h, const void *X, int b, cudaStrea
   // split d so that the hidden layer runs on about one CTA per SM; the partials fit in
   // the down projection's partial-sum buffer
   const size_t cap = (size_t)std::max<size_t>((size_t)kMaxSplits * h->max_batch, (size_t)std::min(h->num_sms, L.n)) * L.d;
-  const int hkps = L.d % (2 * kTK) == 0 ? h->tc_pred_kps : 1;
-  const int lkps = L.r % (2 * kTK) == 0 ? h->tc_pred_kps : 1;
   int splits = (h->num_sms + rtiles - 1) / rtiles;
-  splits = std::min(splits, L.d / (kTK * hkps));
+  splits = std::min(splits, L.d / kTK);
   splits = std::min<int>(splits, (int)(cap / ((size_t)b * L.r)));
   splits = splits < 1 ? 1 : splits;
   // every kernel of the chain starts early (programmatic serialization) and copies its
   // first weight stages before it waits for the one before
-  cudaError_t e = launch_pdl(k_tc_hidden, dim3(rtiles, splits), dim3(kTT), hidden_smem(N, hkps), s,
+  cudaError_t e = launch_pdl(k_tc_hidden, dim3(rtiles, splits), dim3(kTT), hidden_smem(N), s,
                              static_cast<const __half *>(h->At), static_cast<const __half *>(X), h->part, L.d, L.r,
-                             b, N, splits, hidden_stages(hkps), hkps, h->err);
+                             b, N, splits, kPredStages, h->err);
   if (e != cudaSuccess) return e;
   __half *hhi = h->hpair, *hlo = h->hpair + (size_t)32 * L.r;
   e = launch_pdl(k_tc_hsum, dim3((N * L.r + 255) / 256), dim3(256), 0, s, (const float *)h->part, splits, b, N, L.r,
                  hhi, hlo);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_tc_logits, dim3((L.n + kTM - 1) / kTM), dim3(kTT), logits_smem(N, lkps), s,
+  return launch_pdl(k_tc_logits, dim3((L.n + kTM - 1) / kTM), dim3(kTT), logits_smem(N), s,
                     static_cast<const __half *>(h->Bt), static_cast<const __half *>(h->cvec), (const __half *)hhi,
-                    (const __half *)hlo, h->mask, L.n, L.r, L.nwords, b, N, logits_stages(lkps), lkps, h->err);
+                    (const __half *)hlo, h->mask, L.n, L.r, L.nwords, b, N, kPredStages, h->err);
 }
 
 // Up / gate of the union rows for all b tokens -> h->hact; then the down projection into

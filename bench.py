@@ -92,7 +92,7 @@ def parse_args(argv=None):
                          "skews that measurement: name the path there)")
     ap.add_argument("--tc-shape", default="",
                     help="with --batch > 1: the tensor-core kernels' shape, "
-                         "'up_ctas_per_sm,up_chunks_per_step,down_tiles_per_cta[,pred_chunks_per_step]'")
+                         "'up_ctas_per_sm,up_chunks_per_step,down_tiles_per_cta'")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="CPU budget of the reference arm (warm-up and timed steps together)")
     return ap.parse_args(argv)

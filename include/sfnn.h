@@ -307,14 +307,12 @@ SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
  * chunks of every row staged per step (1 or 2; two make each row's reads 256 contiguous
  * bytes).  Down projection: down_tiles_per_cta = 128-column output tiles per CTA (1 or 2;
  * two make each W_down row's reads 512 contiguous bytes; needs d a multiple of 256, else
- * 1 is used).  Predictor: pred_chunks_per_step = 64-wide K chunks of every A^T and B^T row
- * staged per step (1 or 2; 2 needs d, r multiples of 128, else 1 is used for that GEMM).
- * Defaults 2, 2, 2, 1.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those sets;
- * SFNN_ERR_UNSUPPORTED when the layer has no tensor-core batch path.  Takes effect at the
- * next launch.
+ * 1 is used).  Defaults 2, 2, 2.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those
+ * sets; SFNN_ERR_UNSUPPORTED when the layer has no tensor-core batch path.  Takes effect at
+ * the next launch.
  */
 SFNN_API sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32_t up_chunks_per_step,
-                                             int32_t down_tiles_per_cta, int32_t pred_chunks_per_step);
+                                             int32_t down_tiles_per_cta);
 
 /*
  * Measures, on this handle, which path serves AUTO batches of multi_max + 1 .. 2 multi_max

@@ -75,7 +75,7 @@ def test_null_and_invalid_arguments_return_status():
     assert lib.sfnn_set_batch_quota(None, 1) == 1
     assert lib.sfnn_tune_batch_paths(None, None, None) == 1
     assert lib.sfnn_set_batch_depths(None, 6, 4, 2, 4) == 1
-    assert lib.sfnn_set_batch_tc_shape(None, 2, 1, 1, 1) == 1
+    assert lib.sfnn_set_batch_tc_shape(None, 2, 1, 1) == 1
     assert lib.sfnn_set_fused_depths(None, 4, 8, 2, 8) == 1
     assert lib.sfnn_forward(None, 1, None, None, 1, None) == 1
     assert lib.sfnn_predict(None, 1, 1, 1, None) == 1
