@@ -185,97 +185,55 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *total) {
   return before + incl - v;
 }
 
-// 32 x 32 bit transpose in registers: afterwards bit t of a[i] is what bit i of a[t] was.
-// Recursive block swap: exchange the off-diagonal 16 x 16 blocks, then 8 x 8 inside each
-// half, down to single bits (5 rounds of 16 masked swaps), done on bit-reversed words so
-// that bit 0 is the first column.
-__device__ __forceinline__ void transpose32(uint32_t *a) {
-#pragma unroll
-  for (int k = 0; k < 32; ++k) a[k] = __brev(a[k]);
-  uint32_t m = 0x0000ffffu;
-#pragma unroll
-  for (int j = 16; j != 0; j >>= 1) {
-#pragma unroll
-    for (int k = 0; k < 32; k = (k + j + 1) & ~j) {
-      const uint32_t t = (a[k] ^ (a[k + j] >> j)) & m;
-      a[k] ^= t;
-      a[k + j] ^= t << j;
-    }
-    m ^= m << (j >> 1);
-  }
-#pragma unroll
-  for (int k = 0; k < 32; ++k) a[k] = __brev(a[k]);
-}
-
 // The union of the b tokens' sets, ascending, with each union row's token mask (bit t:
-// token t's set holds the row).  CTA k takes the 32 bit words [32k, 32k + 32): its threads
-// first count the union bits of all earlier words (every CTA in parallel, each bit word's
-// b token words read with coalesced loads, then OR and popc), so that no CTA waits on
-// another; then its first warp, lane l on word 32k + l, ORs the word's token words, turns
-// them into the token masks of the word's 32 rows by a 32 x 32 bit transpose, and writes
-// the rows word by word through a shared-memory stage, lane i taking bit i, so that the
-// stores of a word are contiguous.  The last CTA writes the union's size.
+// token t's set holds the row).  CTA k takes the 32 bit words [32k, 32k + 32), warp j word
+// 32k + j: lane t loads token t's word while the CTA's threads count the union bits of all
+// earlier words (each bit word's b token words OR-ed, then popc), so that no CTA waits on
+// another and both are one round of loads.  A warp ORs its word's token words, takes its
+// first union position from the counts (earlier words, then the CTA's earlier warps), and
+// lane i, on row 32 (32k + j) + i, gathers bit i of every token's word by shuffles and
+// writes the row if the union holds it.  The last CTA writes the union's size.
 constexpr int kUnionThreads = 1024;
-constexpr int kUnionStage = 32 * 33;  // words of the warp's staged masks (rows padded to 33)
 
 __global__ void __launch_bounds__(kUnionThreads) k_union(const uint32_t *__restrict__ mask, int nwords, int n, int b,
                                                          int32_t *__restrict__ ulist, uint32_t *__restrict__ utok,
                                                          int32_t *__restrict__ ucount) {
-  __shared__ uint32_t stage[kUnionStage];
-  __shared__ int red[32];
+  __shared__ int red[32], wcnt[32];
   pdl_wait();  // the masks (the kernel before) are complete
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int w0 = blockIdx.x * 32;
-  const uint32_t tail = (n & 31) ? (1u << (n & 31)) - 1u : 0xffffffffu;  // bits of the last word below n
-  auto load = [&](int w, uint32_t *mw) {  // token words of bit word w (w < nwords) -> their union
-#pragma unroll
-    for (int t = 0; t < kMaxBatch; ++t) mw[t] = t < b ? __ldcg(mask + (size_t)t * nwords + w) : 0u;
-    uint32_t u = 0u;
-#pragma unroll
-    for (int t = 0; t < kMaxBatch; ++t) u |= mw[t];
-    return w == nwords - 1 ? u & tail : u;
-  };
+  const int w0 = blockIdx.x * 32, w = w0 + warp;
+  const uint32_t full = 0xffffffffu;
+  const uint32_t mine = w < nwords && lane < b ? __ldcg(mask + (size_t)lane * nwords + w) : 0u;
   int before = 0;  // union bits of the words before this CTA's
-  for (int w = threadIdx.x; w < w0; w += blockDim.x) {
+  for (int v = threadIdx.x; v < w0; v += blockDim.x) {
     uint32_t u = 0u;
 #pragma unroll
-    for (int t = 0; t < kMaxBatch; ++t) u |= t < b ? __ldcg(mask + (size_t)t * nwords + w) : 0u;
-    before += __popc(u);  // w < w0 <= nwords - 1: never the tail word
+    for (int t = 0; t < kMaxBatch; ++t) u |= t < b ? __ldcg(mask + (size_t)t * nwords + v) : 0u;
+    before += __popc(u);  // v < w0 <= nwords - 1: never the tail word
   }
-  before = __reduce_add_sync(0xffffffffu, before);
-  if (lane == 0) red[warp] = before;
+  uint32_t u = __reduce_or_sync(full, mine);
+  if (w == nwords - 1 && (n & 31)) u &= (1u << (n & 31)) - 1u;  // bits of the last word below n
+  before = __reduce_add_sync(full, before);
+  if (lane == 0) {
+    red[warp] = before;
+    wcnt[warp] = __popc(u);
+  }
   __syncthreads();
-  if (warp != 0) return;
-  int base = lane < (int)(blockDim.x >> 5) ? red[lane] : 0;
-  base = __reduce_add_sync(0xffffffffu, base);
-  const int w = w0 + lane;
-  uint32_t mw[kMaxBatch];
-  const uint32_t u = w < nwords ? load(w, mw) : 0u;
-  const int k = __popc(u);
-  int incl = k;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  const int base = __reduce_add_sync(full, red[lane]);  // 32 warps
+  const int wc = wcnt[lane];
+  const int first = base + __reduce_add_sync(full, lane < warp ? wc : 0);
+  uint32_t tok = 0u;  // the tokens whose sets hold row 32 w + lane
+  for (int t = 0; t < b; ++t) tok |= ((__shfl_sync(full, mine, t) >> lane) & 1u) << t;
+  if ((u >> lane) & 1u) {
+    const int pos = first + __popc(u & ((1u << lane) - 1u));
+    ulist[pos] = w * 32 + lane;
+    utok[pos] = tok;
   }
-  const int first = base + incl - k;  // the first union position of word w
-  if (u != 0u) {
-    transpose32(mw);  // mw[i]: the tokens whose sets hold row 32 w + i
-#pragma unroll
-    for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = mw[i];
+  if (blockIdx.x == gridDim.x - 1 && warp == 0) {
+    const int total = base + __reduce_add_sync(full, wc);
+    if (lane == 0) *ucount = total;
   }
-  __syncwarp();
-  for (int l = 0; l < 32; ++l) {
-    const uint32_t ul = __shfl_sync(0xffffffffu, u, l);
-    const int bl = __shfl_sync(0xffffffffu, first, l);
-    if ((ul >> lane) & 1u) {
-      const int pos = bl + __popc(ul & ((1u << lane) - 1u));
-      ulist[pos] = (w0 + l) * 32 + lane;
-      utok[pos] = stage[l * 33 + lane];
-    }
-  }
-  if (blockIdx.x == gridDim.x - 1 && lane == 31) *ucount = base + incl;
 }
 
 // Block t: token t's set as indices in the caller's numbering, ascending in storage order.
