@@ -488,7 +488,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
       {(void **)&h->hpair, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)2 * 32 * r * 2 : 0, false},
       {(void **)&h->upart, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? tc_up_partial_bytes(h->num_sms, (int)mb) : 0,
        false},
-      {(void **)&h->tcnt, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)tc_hstride(L.n) / 64 * 4 : 0, false},
+      {(void **)&h->tcnt, L.dt == SFNN_F16 && !L.rows_q && mb >= 2 ? (size_t)tc_hstride(L.n) / 128 * 4 : 0, false},
   };
   for (auto &q : reqs) {
     if (q.bytes == 0) continue;  // not needed by this layer
@@ -506,7 +506,7 @@ sfnn_status sfnn_create(const sfnn_layer_desc *desc, sfnn_stream_t stream, sfnn_
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->bar, 0, sizeof(uint64_t), s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->alist, 0, n * sizeof(int2), s);
   if (ce == cudaSuccess) ce = cudaMemsetAsync(h->acnt, 0, (size_t)G * 4, s);
-  if (ce == cudaSuccess && h->tcnt) ce = cudaMemsetAsync(h->tcnt, 0, (size_t)tc_hstride(L.n) / 64 * 4, s);
+  if (ce == cudaSuccess && h->tcnt) ce = cudaMemsetAsync(h->tcnt, 0, (size_t)tc_hstride(L.n) / 128 * 4, s);
   if (ce == cudaSuccess) ce = configure_predict();
   if (ce == cudaSuccess) ce = configure_ffn();
   if (ce == cudaSuccess) ce = configure_decode1();
@@ -697,8 +697,7 @@ sfnn_status sfnn_set_batch_tc_shape(sfnn_handle h, int32_t up_ctas_per_sm, int32
                                     int32_t down_tiles_per_cta) {
   if (!h) return SFNN_ERR_INVALID_ARG;
   if (up_ctas_per_sm < -1 || up_ctas_per_sm == 0 || up_ctas_per_sm > 2) return SFNN_ERR_INVALID_ARG;
-  if (up_chunks_per_step != -1 && up_chunks_per_step != 1 && up_chunks_per_step != 2 && up_chunks_per_step != 4)
-    return SFNN_ERR_INVALID_ARG;
+  if (up_chunks_per_step < -1 || up_chunks_per_step == 0 || up_chunks_per_step > 2) return SFNN_ERR_INVALID_ARG;
   if (down_tiles_per_cta < -1 || down_tiles_per_cta == 0 || down_tiles_per_cta > 2) return SFNN_ERR_INVALID_ARG;
   if (!tc_batch_supported(h)) return SFNN_ERR_UNSUPPORTED;
   if (up_ctas_per_sm != -1) h->tc_up_ctas_per_sm = up_ctas_per_sm;

@@ -31,9 +31,9 @@ struct sfnn_ctx {
   __half *hpair;     // [2][32][r] the batch's hidden layer as fp16 hi and lo parts (same path)
   float *part;       // [kMaxSplits][max_batch][d] partial sums of the down projection
   float *upart;      // tensor-core up projection: fp32 partials of tiles split between CTAs
-  int32_t *tcnt;     // [n / 64 rounded up] its per-tile arrival counters (zero between launches)
+  int32_t *tcnt;     // [n / 128 rounded up] its per-tile arrival counters (zero between launches)
   int tc_up_ctas_per_sm;  // its grid: CTAs per SM (1 or 2; at most as many as fit)
-  int tc_up_kps;          // and the 64-wide K chunks of every row it stages per step (1, 2, or 4 on 64-row tiles)
+  int tc_up_kps;          // and the 64-wide K chunks of every row it stages per step (1 or 2)
   int tc_down_mps;        // the down projection's 128-column output tiles per CTA (1 or 2)
   void *xin;         // [max_batch][d] wdtype: layer input inside a stack
   int32_t *err;      // [1] latched device-side error

@@ -201,11 +201,8 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
 // tcnt[tile]; the tile's last segment to arrive adds the tile's partials in CTA order
 // (deterministic), runs the epilogue and zeroes the counter for the next launch.  No CTA
 // waits for another.
-// MT = 128 union rows per tile, or 64: then the MMA's M is 64 and its accumulator rows sit
-// in TMEM lanes 0-15 of each warp's 32 (row 16 w + l in lane 32 w + l), so a step can
-// stage twice the K (4 chunks: 512 contiguous bytes of each row) in the same shared memory.
-// smem per stage: kps times (NP tiles of MT rows (MT x 128 B each) + the x tile (N rows x 128 B)).
-template <int ACT, int MT>
+// smem per stage: kps times (NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B)).
+template <int ACT>
 __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
                                                const __half *__restrict__ X, const int32_t *__restrict__ ulist,
                                                const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
@@ -213,8 +210,6 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
                                                int stages, int kps, float *__restrict__ upart,
                                                int32_t *__restrict__ tcnt, int32_t *err) {
   constexpr int NP = ACT == SFNN_REGLU ? 2 : 1;  // projections with a dot: (gate,) up
-  constexpr int RPT = MT / 16;                    // rows each thread copies
-  constexpr uint32_t kA = MT * 128u;               // bytes of one projection's tile per chunk
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t mbar[8];
   __shared__ uint32_t tmem_slot;
@@ -225,7 +220,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   pdl_launch_dependents();
   const int U = *ucount;
   const int nk = d / (kTK * kps);  // K steps of a tile
-  const int64_t T = (int64_t)((U + MT - 1) / MT) * nk;
+  const int64_t T = (int64_t)((U + kTM - 1) / kTM) * nk;
   const int64_t G = T < (int64_t)gridDim.x ? T : (int64_t)gridDim.x;  // every range non-empty
   const int64_t g = blockIdx.x;
   if (g >= G) return;
@@ -234,14 +229,11 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   // the CTA whose range holds iteration i: the largest g' with g' T / G <= i
   auto cta_of = [&](int64_t i) { return ((i + 1) * G + T - 1) / T - 1; };
   const int first_tile = (int)(i0 / nk);
-  const uint32_t chunk_bytes = NP * kA + (uint32_t)N * 128u;  // a multiple of 1024
+  const uint32_t chunk_bytes = NP * 16384u + (uint32_t)N * 128u;  // a multiple of 1024
   const uint32_t stage_bytes = (uint32_t)kps * chunk_bytes;
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
-  const uint32_t idesc = idesc_f16(MT, N, 0, 0);
-  const int c8 = tid & 7;
-  // this thread's accumulator row (MT = 64: lanes 16-31 hold no row)
-  const int row = MT == 128 ? warp * 32 + lane : warp * 16 + lane;
-  const bool has_row = MT == 128 || lane < 16;
+  const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
+  const int c8 = tid & 7, row = warp * 32 + lane;
   const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
   bool ok = true;
   int base = 0;  // iterations run so far (stage and mbarrier phase of the next one)
@@ -249,8 +241,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
   // bias + ReLU / ReGLU of this thread's row of tile m; zero for the tokens whose set
   // does not hold the row -> H[token][union] (fp16)
   auto epilogue = [&](int m, const float *gs, const float *us) {
-    const int u = m * MT + row;
-    if (!has_row) return;
+    const int u = m * kTM + row;
     if (u < U) {
       const int p = ulist[u];
       const uint32_t tm = utok[u];
@@ -273,11 +264,11 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
     const int m = (int)(i0 / nk);
     const int k0 = (int)(i0 - (int64_t)m * nk);
     const int k1 = (int)(i1 - (int64_t)m * nk < nk ? i1 - (int64_t)m * nk : nk);
-    const int u0 = m * MT;
-    // this thread's RPT rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
-    const __half *src[RPT];
+    const int u0 = m * kTM;
+    // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
+    const __half *src[8];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
+    for (int i = 0; i < 8; ++i) {
       int u = u0 + (tid >> 3) + 16 * i;
       u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
       src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
@@ -287,11 +278,11 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
         const int kc = (k0 + it) * kps + a;
         unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
 #pragma unroll
-        for (int i = 0; i < RPT; ++i)
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
           for (int j = 0; j < NP; ++j)
-            cp16(st + j * kA, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
-        unsigned char *xt = st + NP * kA;
+            cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
+        unsigned char *xt = st + NP * 16384;
         for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
           const int t = q >> 3, c = q & 7;
           const int tt = t < b ? t : b - 1;
@@ -301,13 +292,13 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
     };
     auto issue = [&](uint32_t st, int it) {
       for (int a = 0; a < kps; ++a) {
-        const uint32_t at = st + (uint32_t)a * chunk_bytes, xt = at + NP * kA;
+        const uint32_t at = st + (uint32_t)a * chunk_bytes, xt = at + NP * 16384;
 #pragma unroll
         for (int k = 0; k < kTK / 16; ++k) {
           const uint64_t bd = sdesc_sw128(xt + k * 32, 16, 1024);
 #pragma unroll
           for (int j = 0; j < NP; ++j)
-            umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(at + j * kA + k * 32, 16, 1024), bd, idesc,
+            umma_f16(tmem + (uint32_t)(j * N), sdesc_sw128(at + j * 16384 + k * 32, 16, 1024), bd, idesc,
                      (it > 0 || a > 0 || k > 0) ? 1u : 0u);
         }
       }
@@ -331,11 +322,10 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
       epilogue(m, gs, us);
     } else {
       const int slot = 2 * (int)g + (m == first_tile ? 0 : 1);
-      if (has_row)
-        for (int t = 0; t < b; ++t) {
-          upart[((size_t)slot * NP * b + t) * kTM + row] = gs[t];
-          if (ACT == SFNN_REGLU) upart[((size_t)slot * NP * b + b + t) * kTM + row] = us[t];
-        }
+      for (int t = 0; t < b; ++t) {
+        upart[((size_t)slot * NP * b + t) * kTM + row] = gs[t];
+        if (ACT == SFNN_REGLU) upart[((size_t)slot * NP * b + b + t) * kTM + row] = us[t];
+      }
       __threadfence();
       __syncthreads();
       const int64_t ga = cta_of((int64_t)m * nk), gb = cta_of((int64_t)m * nk + nk - 1);
@@ -345,7 +335,7 @@ __global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, 
         if (last_s) tcnt[m] = 0;  // every segment of the tile has arrived: ready for the next launch
       }
       __syncthreads();
-      if (last_s && has_row) {
+      if (last_s) {
         __threadfence();
         for (int t = 0; t < b; ++t) gs[t] = us[t] = 0.f;
         for (int64_t q = ga; q <= gb; ++q) {  // CTA order
@@ -620,10 +610,8 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
 
 constexpr int kUpStages = 3, kDownStages = 3, kPredStages = 4;
 
-// kps = 4 runs on 64-row tiles (the same rows x K per stage as 2 chunks of 128 rows)
-int up_rows(int kps) { return kps == 4 ? 64 : 128; }
 size_t up_smem(int act, int N, int kps) {
-  return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * up_rows(kps) * 128 + N * 128) + 1024;
+  return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024;
 }
 size_t down_smem(int N, int mps) { return (size_t)kDownStages * (mps * 16384 + N * 128) + 1024; }
 size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
@@ -668,14 +656,12 @@ static int fit_per_sm(const void *func, size_t dyn) {
 }
 
 // k_tc_up CTAs that fit on an SM at once for this shape (worked out once per shape).
-static const void *up_kernel(int act, int kps) {
-  if (kps == 4) return act == SFNN_REGLU ? (const void *)k_tc_up<SFNN_REGLU, 64> : (const void *)k_tc_up<SFNN_RELU, 64>;
-  return act == SFNN_REGLU ? (const void *)k_tc_up<SFNN_REGLU, 128> : (const void *)k_tc_up<SFNN_RELU, 128>;
-}
 static int up_fit(int act, int N, int kps) {
-  static int cache[2][2][3] = {};
-  int &c = cache[act == SFNN_REGLU][N == 32][kps == 4 ? 2 : kps - 1];
-  if (c == 0) c = fit_per_sm(up_kernel(act, kps), up_smem(act, N, kps));
+  static int cache[2][2][2] = {};
+  int &c = cache[act == SFNN_REGLU][N == 32][kps - 1];
+  if (c == 0)
+    c = act == SFNN_REGLU ? fit_per_sm((const void *)k_tc_up<SFNN_REGLU>, up_smem(act, N, kps))
+                          : fit_per_sm((const void *)k_tc_up<SFNN_RELU>, up_smem(act, N, kps));
   return c;
 }
 
@@ -689,17 +675,11 @@ static int down_fit(int N, int mps) {
 }
 
 cudaError_t configure_tc_batch() {
-  cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)std::max(up_smem(SFNN_RELU, 32, 2), up_smem(SFNN_RELU, 16, 4)));
+  cudaError_t e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)up_smem(SFNN_RELU, 32, 2));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)up_smem(SFNN_REGLU, 32, 2));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_up<SFNN_RELU, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)up_smem(SFNN_RELU, 16, 4));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)up_smem(SFNN_REGLU, 16, 4));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_down<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 1));
   if (e == cudaSuccess)
@@ -711,8 +691,7 @@ cudaError_t configure_tc_batch() {
   // the CTAs per SM of every up and down shape, outside any stream capture
   for (int act : {SFNN_RELU, SFNN_REGLU})
     for (int N : {16, 32})
-      for (int kps : {1, 2, 4})
-        if (kps < 4 || N == 16) up_fit(act, N, kps);
+      for (int kps : {1, 2}) up_fit(act, N, kps);
   for (int N : {16, 32})
     for (int mps : {1, 2}) down_fit(N, mps);
   return e;
@@ -752,17 +731,13 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int N = b <= 16 ? 16 : 32;
   const int hs = tc_hstride(L.n);
   const __half *rows = static_cast<const __half *>(h->rows);
-  // 4 chunks per step (64-row tiles) where their three stages fit (N = 16) and d allows
-  int kps = h->tc_up_kps;
-  if (kps == 4 && (N != 16 || L.d % (4 * kTK) != 0)) kps = 2;
-  if (kps == 2 && L.d % (2 * kTK) != 0) kps = 1;
+  const int kps = L.d % (2 * kTK) == 0 ? h->tc_up_kps : 1;
   const int up_grid = std::min(h->tc_up_ctas_per_sm, up_fit(L.act, N, kps)) * h->num_sms;
-  auto kern = kps == 4 ? (L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU, 64> : k_tc_up<SFNN_RELU, 64>)
-                       : (L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU, 128> : k_tc_up<SFNN_RELU, 128>);
-  cudaError_t e = launch_pdl(kern, dim3(up_grid), dim3(kTT), up_smem(L.act, N, kps), s, rows,
-                             static_cast<const __half *>(h->bias), static_cast<const __half *>(X),
-                             (const int32_t *)h->ulist, (const uint32_t *)h->utok, (const int32_t *)h->ucount,
-                             h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart, h->tcnt, h->err);
+  cudaError_t e = launch_pdl(L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU> : k_tc_up<SFNN_RELU>, dim3(up_grid),
+                             dim3(kTT), up_smem(L.act, N, kps), s, rows, static_cast<const __half *>(h->bias),
+                             static_cast<const __half *>(X), (const int32_t *)h->ulist, (const uint32_t *)h->utok,
+                             (const int32_t *)h->ucount, h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart,
+                             h->tcnt, h->err);
   if (e != cudaSuccess) return e;
   const int mps = L.d % (2 * kTM) == 0 ? h->tc_down_mps : 1;
   const int mtiles = L.d / (kTM * mps);

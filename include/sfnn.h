@@ -304,9 +304,8 @@ SFNN_API sfnn_status sfnn_set_batch_quota(sfnn_handle h, int32_t enable);
  * it beyond the order in which partial sums are added).  Up projection: up_ctas_per_sm =
  * its CTAs per SM (1 or 2, capped by how many fit in shared memory; the union's (128-row
  * tile, K step) pairs are shared out evenly among them), up_chunks_per_step = 64-wide K
- * chunks of every row staged per step (1, 2 or 4; two make each row's reads 256 contiguous
- * bytes, four 512 on tiles of 64 rows, used up to 16 tokens and d a multiple of 256, else
- * two).  Down projection: down_tiles_per_cta = 128-column output tiles per CTA (1 or 2;
+ * chunks of every row staged per step (1 or 2; two make each row's reads 256 contiguous
+ * bytes).  Down projection: down_tiles_per_cta = 128-column output tiles per CTA (1 or 2;
  * two make each W_down row's reads 512 contiguous bytes; needs d a multiple of 256, else
  * 1 is used).  Defaults 2, 2, 2.  -1 keeps a value.  SFNN_ERR_INVALID_ARG outside those
  * sets; SFNN_ERR_UNSUPPORTED when the layer has no tensor-core batch path.  Takes effect at

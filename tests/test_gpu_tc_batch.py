@@ -13,8 +13,8 @@
   unions smaller than the grid (one K chunk per CTA, every tile split), and a union of
   50003 rows at d = 128 whose runs hold whole tiles between split ones, both reproducible
   launch after launch (the per-tile counters return to zero), for one and two CTAs per SM
-  and one, two and four K chunks per step (four: 64-row tiles, up to 16 tokens); the down
-  projection with one and two 128-column tiles per CTA;
+  and one and two K chunks per step; the down projection with one and two 128-column
+  tiles per CTA;
 * the full-size batch configurations (OPT-30B-shaped b = 8, 70B-shaped b = 32) match
   the oracle on every token;
 * layers it cannot serve (fp32 weights, d not a multiple of 128) refuse the path.
@@ -79,7 +79,7 @@ def test_tc_batch_full_size(name, b):
 
 @pytest.mark.parametrize("base", ["opt6.7b_relu", "70b_reglu"])
 @pytest.mark.parametrize("b", [4, 20])
-@pytest.mark.parametrize("shape", [(2, 1, 1), (1, 2, 2), (1, 4, 2)])
+@pytest.mark.parametrize("shape", [(2, 1, 1), (1, 2, 2)])
 def test_tc_batch_runs_of_whole_tiles(base, b, shape):
     # every neuron on: the union is all 50003 rows, 391 tiles of 2 K chunks, more steps
     # than the grid has CTAs
@@ -107,13 +107,13 @@ def test_tc_batch_kernel_shapes(base, d, n, r):
     h = sf.SparseFFN.from_layer(lay, max_batch=32)
     for b in (3, 32):
         X = W.make_tokens(cfg, b, seed=49, stream_key=b)
-        for shape in [(1, 1, 1), (2, 1, 2), (1, 2, 1), (2, 2, 2), (1, 4, 2), (2, 4, 1)]:
+        for shape in [(1, 1, 1), (2, 1, 2), (1, 2, 1), (2, 2, 2)]:
             h.set_batch_tc_shape(*shape)
             Y, idx, cnt = run_batch(h, X, sf.BATCH_TENSOR_CORE)
             for t in range(b):
                 check_token(lay, X[t], Y[t], mask_from_idx(idx[t], cnt[t], n), f"{base} {shape} b={b} t={t}")
             assert np.array_equal(run_batch(h, X, sf.BATCH_TENSOR_CORE)[0], Y)
-    for bad in [(3, 1, 1), (1, 3, 1), (1, 8, 1), (1, 1, 3), (0, 1, 1)]:
+    for bad in [(3, 1, 1), (1, 4, 1), (1, 1, 3), (0, 1, 1)]:
         with pytest.raises(sf.SfnnError):
             h.set_batch_tc_shape(*bad)
     assert h.get_error() == 0
