@@ -34,7 +34,6 @@ namespace sfnn {
 namespace {
 
 constexpr int kTT = 128;  // threads per CTA (4 warps: warp w reads TMEM lanes 32w..32w+31)
-constexpr int kUpT = 256;  // k_tc_up: 8 warps copy; warps 0-3 also read the accumulators
 constexpr int kTM = 128;  // MMA M
 constexpr int kTK = 64;   // K of a stage: 64 fp16 = one 128-byte swizzle row
 constexpr int kTmemCols = 64;
@@ -204,7 +203,7 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
 // waits for another.
 // smem per stage: kps times (NP tiles of 128 rows (16 KB each) + the x tile (N rows x 128 B)).
 template <int ACT>
-__global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
+__global__ void __launch_bounds__(kTT) k_tc_up(const __half *__restrict__ rows, const __half *__restrict__ bias,
                                                const __half *__restrict__ X, const int32_t *__restrict__ ulist,
                                                const uint32_t *__restrict__ utok, const int32_t *__restrict__ ucount,
                                                __half *__restrict__ H, int hstride, int d, int b, int N, int nproj,
@@ -235,8 +234,7 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
   const uint32_t tmem = tc_begin(mbar, stages, &tmem_slot, &fail);
   const uint32_t idesc = idesc_f16(kTM, N, 0, 0);
   const int c8 = tid & 7, row = warp * 32 + lane;
-  const bool has_row = warp < 4;  // warps 0-3 hold the accumulator rows (TMEM lanes 32 w ..)
-  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
   bool ok = true;
   int base = 0;  // iterations run so far (stage and mbarrier phase of the next one)
 
@@ -244,7 +242,6 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
   // does not hold the row -> H[token][union] (fp16)
   auto epilogue = [&](int m, const float *gs, const float *us) {
     const int u = m * kTM + row;
-    if (!has_row) return;
     if (u < U) {
       const int p = ulist[u];
       const uint32_t tm = utok[u];
@@ -268,11 +265,11 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
     const int k0 = (int)(i0 - (int64_t)m * nk);
     const int k1 = (int)(i1 - (int64_t)m * nk < nk ? i1 - (int64_t)m * nk : nk);
     const int u0 = m * kTM;
-    // this thread's 4 rows of the tile (row = tid/8 + 32 i) and its 16-byte chunk (tid % 8)
-    const __half *src[4];
+    // this thread's 8 rows of the tile (row = tid/8 + 16 i) and its 16-byte chunk (tid % 8)
+    const __half *src[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int u = u0 + (tid >> 3) + 32 * i;
+    for (int i = 0; i < 8; ++i) {
+      int u = u0 + (tid >> 3) + 16 * i;
       u = u < U ? u : U - 1;  // the tile's tail repeats a row; its results are not stored
       src[i] = rows + (size_t)ulist[u] * nproj * d + c8 * 8;
     }
@@ -281,12 +278,12 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
         const int kc = (k0 + it) * kps + a;
         unsigned char *st = smem + (size_t)s * stage_bytes + (size_t)a * chunk_bytes;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
           for (int j = 0; j < NP; ++j)
-            cp16(st + j * 16384, kmajor_off((tid >> 3) + 32 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
+            cp16(st + j * 16384, kmajor_off((tid >> 3) + 16 * i, c8), src[i] + (size_t)j * d + (size_t)kc * kTK);
         unsigned char *xt = st + NP * 16384;
-        for (int q = tid; q < N * 8; q += kUpT) {  // x rows: token q/8 (tokens past b repeat the last one)
+        for (int q = tid; q < N * 8; q += kTT) {  // x rows: token q/8 (tokens past b repeat the last one)
           const int t = q >> 3, c = q & 7;
           const int tt = t < b ? t : b - 1;
           cp16(xt, kmajor_off(t, c), X + (size_t)tt * d + (size_t)kc * kTK + c * 8);
@@ -312,7 +309,7 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
     }
     base += k1 - k0;
     float gs[32], us[32];
-    if (ok && has_row) {
+    if (ok) {
       for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + c0, gs + c0);
       if (ACT == SFNN_REGLU)
         for (int c0 = 0; c0 < N; c0 += 16) tmem_ld16(lane_addr + N + c0, us + c0);
@@ -325,11 +322,10 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
       epilogue(m, gs, us);
     } else {
       const int slot = 2 * (int)g + (m == first_tile ? 0 : 1);
-      if (has_row)
-        for (int t = 0; t < b; ++t) {
-          upart[((size_t)slot * NP * b + t) * kTM + row] = gs[t];
-          if (ACT == SFNN_REGLU) upart[((size_t)slot * NP * b + b + t) * kTM + row] = us[t];
-        }
+      for (int t = 0; t < b; ++t) {
+        upart[((size_t)slot * NP * b + t) * kTM + row] = gs[t];
+        if (ACT == SFNN_REGLU) upart[((size_t)slot * NP * b + b + t) * kTM + row] = us[t];
+      }
       __threadfence();
       __syncthreads();
       const int64_t ga = cta_of((int64_t)m * nk), gb = cta_of((int64_t)m * nk + nk - 1);
@@ -339,7 +335,7 @@ __global__ void __launch_bounds__(kUpT) k_tc_up(const __half *__restrict__ rows,
         if (last_s) tcnt[m] = 0;  // every segment of the tile has arrived: ready for the next launch
       }
       __syncthreads();
-      if (last_s && has_row) {
+      if (last_s) {
         __threadfence();
         for (int t = 0; t < b; ++t) gs[t] = us[t] = 0.f;
         for (int64_t q = ga; q <= gb; ++q) {  // CTA order
@@ -641,7 +637,7 @@ size_t tc_up_partial_bytes(int num_sms, int max_batch) {
 // registers and by tensor memory (kTmemCols of 512 columns each).  Worked out from the
 // device's and the kernel's attributes: the occupancy calculator assumes a shared-memory
 // carveout smaller than the one launches get.
-static int fit_per_sm(const void *func, size_t dyn, int threads = kTT) {
+static int fit_per_sm(const void *func, size_t dyn) {
   int dev = 0, smem_sm = 0, reserved = 0, regs_sm = 0;
   cudaFuncAttributes fa;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -653,7 +649,7 @@ static int fit_per_sm(const void *func, size_t dyn, int threads = kTT) {
     return 1;
   }
   int n = (int)((size_t)smem_sm / (dyn + fa.sharedSizeBytes + (size_t)reserved));
-  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * (threads / 32);  // per-warp granules of 256
+  const int regs_cta = ((fa.numRegs * 32 + 255) / 256 * 256) * (kTT / 32);  // per-warp granules of 256
   n = std::min(n, regs_cta > 0 ? regs_sm / regs_cta : n);
   n = std::min(n, 512 / kTmemCols);
   return n > 0 ? n : 1;
@@ -664,8 +660,8 @@ static int up_fit(int act, int N, int kps) {
   static int cache[2][2][2] = {};
   int &c = cache[act == SFNN_REGLU][N == 32][kps - 1];
   if (c == 0)
-    c = act == SFNN_REGLU ? fit_per_sm((const void *)k_tc_up<SFNN_REGLU>, up_smem(act, N, kps), kUpT)
-                          : fit_per_sm((const void *)k_tc_up<SFNN_RELU>, up_smem(act, N, kps), kUpT);
+    c = act == SFNN_REGLU ? fit_per_sm((const void *)k_tc_up<SFNN_REGLU>, up_smem(act, N, kps))
+                          : fit_per_sm((const void *)k_tc_up<SFNN_RELU>, up_smem(act, N, kps));
   return c;
 }
 
@@ -738,7 +734,7 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   const int kps = L.d % (2 * kTK) == 0 ? h->tc_up_kps : 1;
   const int up_grid = std::min(h->tc_up_ctas_per_sm, up_fit(L.act, N, kps)) * h->num_sms;
   cudaError_t e = launch_pdl(L.act == SFNN_REGLU ? k_tc_up<SFNN_REGLU> : k_tc_up<SFNN_RELU>, dim3(up_grid),
-                             dim3(kUpT), up_smem(L.act, N, kps), s, rows, static_cast<const __half *>(h->bias),
+                             dim3(kTT), up_smem(L.act, N, kps), s, rows, static_cast<const __half *>(h->bias),
                              static_cast<const __half *>(X), (const int32_t *)h->ulist, (const uint32_t *)h->utok,
                              (const int32_t *)h->ucount, h->hact, hs, L.d, b, N, L.nproj, kUpStages, kps, h->upart,
                              h->tcnt, h->err);
