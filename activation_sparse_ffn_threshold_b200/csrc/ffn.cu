@@ -143,15 +143,7 @@ __global__ void k_reduce(const float *__restrict__ part, int splits, int64_t bd,
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= bd) return;
   float s = 0.f;
-  int k = 0;
-  for (; k + 8 <= splits; k += 8) {  // eight loads in flight, added in split order
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = part[(size_t)(k + u) * bd + i];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) s += v[u];
-  }
-  for (; k < splits; ++k) s += part[(size_t)k * bd + i];
+  for (int k = 0; k < splits; ++k) s += part[(size_t)k * bd + i];
   if (resid) s = resid[i] + s;
   Y[i] = s;
   if (xnext) xnext[i] = from_f<OUT>(s);

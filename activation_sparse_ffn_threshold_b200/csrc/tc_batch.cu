@@ -533,18 +533,8 @@ __global__ void k_tc_hsum(const float *__restrict__ hp, int splits, int b, int N
   float h = 0.f;
   if (t < b) {
     const int j = i - t * r;
-    const float *q = hp + (size_t)t * r + j;
-    const size_t step = (size_t)b * r;
     float s = 0.f;
-    int k = 0;
-    for (; k + 8 <= splits; k += 8) {  // eight loads in flight, added in split order
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = q[(size_t)(k + u) * step];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) s += v[u];
-    }
-    for (; k < splits; ++k) s += q[(size_t)k * step];
+    for (int k = 0; k < splits; ++k) s += hp[((size_t)k * b + t) * r + j];
     h = s > 0.f ? s : 0.f;  // NaN -> 0
   }
   const __half hi = __float2half_rn(h);
