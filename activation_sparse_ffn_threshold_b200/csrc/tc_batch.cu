@@ -121,11 +121,6 @@ __device__ __forceinline__ uint32_t kmajor_off(int row, int c) {
 __device__ __forceinline__ void cp16(unsigned char *base, uint32_t off, const void *src) {
   cp_async16(base + off, src);
 }
-// The same copy with L2 filling 256-byte spans from DRAM: a row read 128 bytes per step
-// then reaches DRAM in 256-byte runs, and the next step's 128 bytes come from L2.
-__device__ __forceinline__ void cp16_l2_256(unsigned char *base, uint32_t off, const void *src) {
-  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(smem_u32(base + off)), "l"(src) : "memory");
-}
 
 // ---------------------------------------------------------------- shared pipeline
 // All threads: init the stage mbarriers, allocate tensor memory (warp 0), publish.
@@ -491,7 +486,7 @@ __global__ void __launch_bounds__(kTT) k_tc_hidden(const __half *__restrict__ At
       for (int i = 0; i < 8; ++i) {
         const int row = (tid >> 3) + 16 * i;
         const int j = j0 + row < r ? j0 + row : r - 1;
-        cp16_l2_256(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
+        cp16(st, kmajor_off(row, c8), At + (size_t)j * d + (size_t)kc * kTK + c8 * 8);
       }
     }
     if (what & kLoadB) {
@@ -568,7 +563,7 @@ __global__ void __launch_bounds__(kTT) k_tc_logits(const __half *__restrict__ Bt
       for (int i = 0; i < 8; ++i) {
         const int row = (tid >> 3) + 16 * i;
         const int nn = i0 + row < n ? i0 + row : n - 1;
-        cp16_l2_256(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
+        cp16(st, kmajor_off(row, c8), Bt + (size_t)nn * r + (size_t)kc * kTK + c8 * 8);
       }
     }
     if (what & kLoadB) {
