@@ -165,9 +165,7 @@ __device__ __forceinline__ bool tc_mainloop(unsigned char *smem, uint32_t stage_
     switch (stages) {
       case 2: cp_async_wait<0>(); break;
       case 3: cp_async_wait<1>(); break;
-      case 4: cp_async_wait<2>(); break;
-      case 5: cp_async_wait<3>(); break;
-      default: cp_async_wait<4>(); break;  // 6 stages (mbar[] holds 8)
+      default: cp_async_wait<2>(); break;
     }
     fence_async_smem();
     __syncthreads();
@@ -615,9 +613,7 @@ constexpr int kUpStages = 3, kDownStages = 3, kPredStages = 4;
 size_t up_smem(int act, int N, int kps) {
   return (size_t)kUpStages * kps * ((act == SFNN_REGLU ? 2 : 1) * 16384 + N * 128) + 1024;
 }
-// one 128-column tile per CTA: 6 stages (5 at N = 32) so that two CTAs per SM still fit
-int down_stages(int N, int mps) { return mps == 2 ? kDownStages : (N == 16 ? 6 : 5); }
-size_t down_smem(int N, int mps) { return (size_t)down_stages(N, mps) * (mps * 16384 + N * 128) + 1024; }
+size_t down_smem(int N, int mps) { return (size_t)kDownStages * (mps * 16384 + N * 128) + 1024; }
 size_t hidden_smem(int N) { return (size_t)kPredStages * (16384 + N * 128) + 1024; }
 size_t logits_smem(int N) { return (size_t)kPredStages * (16384 + 2 * N * 128) + 1024; }
 
@@ -685,8 +681,7 @@ cudaError_t configure_tc_batch() {
     e = cudaFuncSetAttribute(k_tc_up<SFNN_REGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)up_smem(SFNN_REGLU, 32, 2));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_down<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)std::max(down_smem(16, 1), down_smem(32, 1)));
+    e = cudaFuncSetAttribute(k_tc_down<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 1));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_tc_down<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)down_smem(32, 2));
   if (e == cudaSuccess)
@@ -752,7 +747,7 @@ cudaError_t launch_tc_batch(const sfnn_ctx *h, const void *X, int b, int *splits
   *splits_out = splits;
   return launch_pdl(mps == 2 ? k_tc_down<2> : k_tc_down<1>, dim3(mtiles, splits), dim3(kTT), down_smem(N, mps), s,
                     rows, (const __half *)h->hact, hs, (const int32_t *)h->ulist, (const int32_t *)h->ucount, h->part,
-                    L.d, b, N, L.nproj, splits, down_stages(N, mps), h->err);
+                    L.d, b, N, L.nproj, splits, kDownStages, h->err);
 }
 
 }  // namespace sfnn
