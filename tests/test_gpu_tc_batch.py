@@ -15,6 +15,9 @@
   launch after launch (the per-tile counters return to zero), for one and two CTAs per SM
   and one and two K chunks per step; the down projection with one and two 128-column
   tiles per CTA;
+* in stream order with other kernels writing its input just before and reading its
+  output just after (no host synchronisation), it gives the isolated calls' results
+  bitwise;
 * the full-size batch configurations (OPT-30B-shaped b = 8, 70B-shaped b = 32) match
   the oracle on every token;
 * layers it cannot serve (fp32 weights, d not a multiple of 128) refuse the path.
@@ -116,6 +119,39 @@ def test_tc_batch_kernel_shapes(base, d, n, r):
     for bad in [(3, 1, 1), (1, 4, 1), (1, 1, 3), (0, 1, 1)]:
         with pytest.raises(sf.SfnnError):
             h.set_batch_tc_shape(*bad)
+    assert h.get_error() == 0
+
+
+@pytest.mark.parametrize("base,d,n,r", [SHAPES[1], SHAPES[2]])
+def test_tc_batch_in_stream_order_with_other_kernels(base, d, n, r):
+    # the chain's kernels start early (dependent launch) and read only weights before their
+    # wait: an input written by another kernel just before the call, and an output read by
+    # one just after, on the same stream with no host synchronisation, are what isolated
+    # calls give, bitwise
+    import torch
+    cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
+    lay = W.make_layer(cfg, seed=50)
+    h = sf.SparseFFN.from_layer(lay, max_batch=32)
+    h.set_batch_path(sf.BATCH_TENSOR_CORE)
+    bs = [8, 3, 32, 17, 8]
+    Xs = [torch.from_numpy(W.make_tokens(cfg, b, seed=60 + i, stream_key=b)).cuda() for i, b in enumerate(bs)]
+    ref = []
+    for X in Xs:  # isolated
+        ref.append(h.forward_batch(X).clone())
+        torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    xin = torch.empty((32, d), dtype=Xs[0].dtype, device="cuda")
+    y = torch.empty((32, d), dtype=torch.float32, device="cuda")
+    outs = []
+    with torch.cuda.stream(s):
+        for X in Xs:
+            b = X.shape[0]
+            xin[:b].copy_(X * 1.0)  # a kernel writes the input right before the call
+            h.forward_batch(xin[:b], y[:b], stream=s)
+            outs.append(y[:b] * 1.0)  # and one reads the output right after
+    torch.cuda.synchronize()
+    for i, (a, e) in enumerate(zip(outs, ref)):
+        assert torch.equal(a, e), f"batch {i} (b = {bs[i]})"
     assert h.get_error() == 0
 
 
