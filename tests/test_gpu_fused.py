@@ -6,7 +6,9 @@
   tiles hold one or several B^T chunks and whose rows need one or several
   columns per thread (fp32 and fp16, ReLU and ReGLU, ragged n);
 * consecutive launches on the same handle (programmatic dependent launch lets
-  the next one start early) stay correct and bitwise reproducible;
+  the next one start early) stay correct and bitwise reproducible, also with other
+  kernels writing the input right before each call and reading the output right after
+  (single token, few-token batches, the look-ahead stack);
 * the residual stack runs through it;
 * its request depths (B^T stages, W_down rows requested early, up/gate segments in
   flight) change nothing in the result: bitwise the same sets and y;
@@ -75,6 +77,50 @@ def test_back_to_back_launches_same_handle():
         assert np.array_equal(y, Y1[t].cpu().numpy())
         check_token(lay, Xh[t], y, m)
     assert h.get_error() == 0
+
+
+def test_fused_paths_in_stream_order_with_other_kernels():
+    # the fused kernels start early (dependent launch) and read only weights before their
+    # wait: inputs written by another kernel right before each call and outputs read right
+    # after, on one stream with no host synchronisation, give the isolated calls' results
+    # bitwise -- single token, few-token batches, and the look-ahead stack
+    cfg = W.small_config(W.CONFIGS["70b_reglu"], d=2048, n=5003, r=256)
+    layers = [W.make_layer(cfg, seed=15 + l, layer=l) for l in range(2)]
+    hs = [sf.SparseFFN.from_layer(l, max_batch=4) for l in layers]
+    h = hs[0]
+    X = dev(W.make_tokens(cfg, 12, seed=16))
+    X32 = X.float()
+    plan = [("one", 1), ("batch", 2), ("one", 1), ("batch", 4), ("stack", 1), ("batch", 3), ("one", 1)]
+
+    def call(kind, x, y, stream=None):
+        if kind == "one":
+            return h.forward(x[0], y[0], stream=stream)
+        if kind == "batch":
+            return h.forward_batch(x, y, stream=stream)
+        return sf.forward_stack(hs, x[0], y[0], lookahead=True, stream=stream)
+
+    ref = []
+    for i, (kind, b) in enumerate(plan):  # isolated
+        x = (X32 if kind == "stack" else X)[i:i + b]
+        y = torch.empty((b, cfg.d), dtype=torch.float32, device="cuda")
+        call(kind, x.clone(), y)
+        torch.cuda.synchronize()
+        ref.append(y.clone())
+    s = torch.cuda.Stream()
+    xin = torch.empty((4, cfg.d), dtype=X.dtype, device="cuda")
+    xin32 = torch.empty((4, cfg.d), dtype=torch.float32, device="cuda")
+    yout = torch.empty((4, cfg.d), dtype=torch.float32, device="cuda")
+    outs = []
+    with torch.cuda.stream(s):
+        for i, (kind, b) in enumerate(plan):
+            buf = xin32 if kind == "stack" else xin
+            buf[:b].copy_((X32 if kind == "stack" else X)[i:i + b] * 1.0)  # written right before
+            call(kind, buf[:b], yout[:b], stream=s)
+            outs.append(yout[:b] * 1.0)  # read right after
+    torch.cuda.synchronize()
+    for i, (a, e) in enumerate(zip(outs, ref)):
+        assert torch.equal(a, e), f"call {i} ({plan[i][0]}, b = {plan[i][1]})"
+    assert all(x.get_error() == 0 for x in hs)
 
 
 def test_stack_through_fused_kernel():
