@@ -101,10 +101,10 @@ def test_tc_batch_runs_of_whole_tiles(base, b, shape):
     assert h.get_error() == 0
 
 
-@pytest.mark.parametrize("base,d,n,r", [SHAPES[1], SHAPES[3]])
+@pytest.mark.parametrize("base,d,n,r", [SHAPES[1], SHAPES[3], ("opt6.7b_relu", 1152, 2001, 128)])
 def test_tc_batch_kernel_shapes(base, d, n, r):
     # up CTAs per SM x K chunks per step x down tiles per CTA: the same sets, y within the
-    # tolerance of the oracle
+    # tolerance of the oracle (d = 1152: two down tiles per CTA fall back to one)
     cfg = W.small_config(W.CONFIGS[base], d=d, n=n, r=r)
     lay = W.make_layer(cfg, seed=48)
     h = sf.SparseFFN.from_layer(lay, max_batch=32)
